@@ -1,0 +1,383 @@
+"""Benchmark: MoE FFN layer forward + backward on B200, tokens/s.
+
+One step = the whole hot path over one batch: route (logits, softmax/top-k,
+counts, offsets, slot rows) -> permute -> grouped SwiGLU FFN forward ->
+combine -> combine backward -> grouped FFN backward (dgrad + wgrad) ->
+unpermute-grad + router grad.  Inputs are seeded synthetic tensors already
+resident in HBM; L2 is flushed (256 MiB write) between timed steps, outside
+the timed events.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--capacity-factor] [--impl {ours,reference}]
+
+Multi-GPU (torchrun, one process per GPU): data parallel with weak scaling,
+each rank runs its own token batch (seed = rank) through its own copy of the
+layer; there is no collective inside a step.  The timed region is bracketed
+by a barrier and a device synchronisation; the time is the max over ranks.
+
+``--impl reference`` times the float64 CPU oracle on the host cores on a
+bounded token sample of the same workload (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mixture_experts_layer_offsets_b200 import inputs  # noqa: E402
+
+METRIC = "MoE FFN fwd+bwd tokens/s on 1 B200; grouped-GEMM % of tensor-core peak"
+FLUSH_BYTES = 256 << 20
+# kernel launches of one step, per C-ABI call (bf16 path)
+LAUNCHES = {"route": 3, "permute": 1, "ffn_fwd": 2, "combine": 1, "combine_bwd": 1,
+            "ffn_bwd": 4, "route_bwd": 4, "padded_dispatch": 2}
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            pk = json.load(fh)
+        return pk, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def _workload_desc(cfg, capacity):
+    d = {"workload": f"{cfg.name}: T={cfg.T} d_model={cfg.d_model} E={cfg.E} top_k={cfg.top_k} "
+                     f"d_ff={cfg.d_ff} {cfg.dtype}",
+         "T": cfg.T, "d_model": cfg.d_model, "E": cfg.E, "top_k": cfg.top_k, "d_ff": cfg.d_ff,
+         "routing": "skewed (logit bias std 2)" if cfg.bias_std else "near-uniform random",
+         "l2": "flushed between timed steps (256 MiB write, outside the timed events)",
+         "weight_grad_dtype": "fp32"}
+    if capacity:
+        d["layout"] = f"padded capacity C={capacity} (overflow dropped)"
+    else:
+        d["layout"] = "dropless, device-scheduled grouped GEMM"
+    return d
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------- our arm
+def run_ours(args, rank, world):
+    from mixture_experts_layer_offsets_b200.layer import MoELayer, capacity_for
+
+    cfg = inputs.CONFIGS[args.workload]
+    if cfg.dtype not in ("f32", "bf16"):
+        raise SystemExit(f"workload {cfg.name}: dtype {cfg.dtype} is not implemented")
+    dev = torch.device("cuda", torch.cuda.current_device())
+    capacity = capacity_for(cfg.R, cfg.E, *cfg.padded_cf) if args.capacity_factor and cfg.padded_cf else None
+    inp = inputs.make_inputs(cfg, device=dev, seed=rank)
+    L = MoELayer(cfg.T, cfg.d_model, cfg.E, cfg.top_k, cfg.d_ff, cfg.dtype, dev,
+                 dw_dtype="f32", capacity=capacity)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    x, wr, b, w1, w2, dout = (inp[k] for k in ("x", "w_router", "bias", "w1", "w2", "dout"))
+    phases = ["route", "dispatch", "ffn_fwd", "combine", "combine_bwd", "ffn_bwd", "route_bwd"]
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
+        s, dt = L.shape, L.cdtype
+        from mixture_experts_layer_offsets_b200 import capi
+        mark(0)
+        capi.moe_route(s, dt, x, wr, b, L.logits, L.topk_idx, L.topk_gate, L.counts, L.offsets,
+                       L.slot_row, L.ws)
+        mark(1)
+        if capacity:
+            capi.moe_padded_dispatch(s, dt, capacity, x, L.topk_idx, L.slot_row, L.offsets,
+                                     L.x_perm, L.pad_row, L.offsets_pad)
+        else:
+            capi.moe_permute(s, dt, x, L.slot_row, L.x_perm, L.perm_src)
+        mark(2)
+        capi.moe_grouped_ffn_fwd(s, dt, L.rows, L.x_perm, L.ffn_offsets, w1, w2, L.act, L.y_perm,
+                                 L.ws)
+        mark(3)
+        capi.moe_combine(s, dt, L.y_perm, L.row_map, L.topk_gate, L.out)
+        mark(4)
+        capi.moe_combine_bwd(s, dt, dout, L.y_perm, L.row_map, L.topk_gate, L.dy_perm, L.dgate)
+        mark(5)
+        capi.moe_grouped_ffn_bwd(s, dt, L.rows, L.dy_perm, L.x_perm, L.act, L.ffn_offsets, w1, w2,
+                                 L.dx_perm, L.dw1, L.dw2, capi.MOE_F32, L.ws)
+        mark(6)
+        capi.moe_route_bwd(s, dt, x, wr, L.logits, L.topk_idx, L.dgate, L.dx_perm, L.row_map,
+                           L.dx, L.dw_router, L.ws)
+        mark(7)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if L.device_status() != 0:
+        raise SystemExit("device status reported a timeout during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(args.steps)]
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    for i in range(args.steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop() if sampler else None
+    per_step = [e[0].elapsed_time(e[7]) for e in evs]
+    ph = {p: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, p in enumerate(phases)}
+    total_ms = sum(per_step)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    status = L.device_status()
+
+    # e2e: through the public API with host buffers, copies inside the timed region
+    e2e = run_e2e(args, L, inp, dev, flush, capacity, world)
+
+    if rank != 0:
+        return None
+    tokens_per_s = cfg.T * world / (ms_per_step / 1e3)
+    pk, pk_kind = _peaks()
+    gemm_ms = ph["ffn_fwd"] + ph["ffn_bwd"]
+    rows = L.rows
+    gemm_flop = 18.0 * cfg.R * cfg.d_model * cfg.d_ff   # algorithmic (dropless) FLOPs per step
+    achieved = gemm_flop / (gemm_ms / 1e3) / 1e12
+    peak = pk["bf16_tflops"] if cfg.dtype == "bf16" else None
+    launches_per_step = (LAUNCHES["route"] + (LAUNCHES["padded_dispatch"] if capacity else LAUNCHES["permute"])
+                         + LAUNCHES["ffn_fwd"] + LAUNCHES["combine"] + LAUNCHES["combine_bwd"]
+                         + LAUNCHES["ffn_bwd"] + LAUNCHES["route_bwd"])
+    line = {
+        "metric": METRIC, "value": round(tokens_per_s, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
+        "data": "synthetic (seeded; random-init weights)",
+        "config": _workload_desc(cfg, capacity),
+        "roofline": {
+            "bound": "tensor", "kernel": "grouped GEMM (tcgen05), all 6 launches of a step",
+            "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4) if peak else None,
+            "peak_kind": f"bf16_tflops burst, {pk_kind}", "traffic": None,
+            "algorithmic_flop_per_step": gemm_flop, "gemm_ms_per_step": round(gemm_ms, 4),
+            "rows_computed": rows,
+        },
+        "phases_ms": {k: round(v, 4) for k, v in ph.items()},
+        "gpu_launches": launches_per_step * args.steps,
+        "device_status": status,
+        "e2e": e2e,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, budget_s=args.cpu_seconds)
+    return line
+
+
+def run_e2e(args, L, inp, dev, flush, capacity, world):
+    """Same metric through the public API with pinned host buffers: per step the
+    inputs x and dout go host->device and the outputs out and dx come back."""
+    from mixture_experts_layer_offsets_b200 import capi  # noqa: F401
+    hx = inp["x"].cpu().pin_memory()
+    hd = inp["dout"].cpu().pin_memory()
+    hout = torch.empty_like(hx).pin_memory()
+    hdx = torch.empty_like(hx).pin_memory()
+    dx_in = torch.empty_like(inp["x"])
+    ddout = torch.empty_like(inp["dout"])
+    wr, b, w1, w2 = inp["w_router"], inp["bias"], inp["w1"], inp["w2"]
+
+    def step():
+        dx_in.copy_(hx, non_blocking=True)
+        ddout.copy_(hd, non_blocking=True)
+        L.step(dx_in, wr, b, w1, w2, ddout)
+        hout.copy_(L.out, non_blocking=True)
+        hdx.copy_(L.dx, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    n = max(1, args.steps // 2)
+    st, en = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    times = []
+    if world > 1:
+        torch.distributed.barrier()
+    for _ in range(n):
+        flush.zero_()
+        st.record()
+        step()
+        en.record()
+        torch.cuda.synchronize()
+        times.append(st.elapsed_time(en))
+    ms = sum(times) / n
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    T = inp["x"].shape[0]
+    nbytes = hx.numel() * hx.element_size()
+    return {"value": round(T * world / (ms / 1e3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": 2 * nbytes, "d2h_bytes_per_step": 2 * nbytes,
+            "ms_per_step": round(ms, 4), "api": "MoELayer.step (C ABI) with pinned host buffers"}
+
+
+# ------------------------------------------------- CPU oracle (baseline)
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        if info:
+            return max(i.get("num_threads", 1) for i in info)
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def cpu_baseline(cfg, budget_s=12.0, chunk=64):
+    """Float64 oracle fwd+bwd on micro-batches of `chunk` tokens of the workload's
+    shapes until `budget_s` seconds of CPU work have run; tokens/s."""
+    from oracle import moe_ref as ref
+    g = torch.Generator().manual_seed(0)
+    T, d, E, k, f = cfg.T, cfg.d_model, cfg.E, cfg.top_k, cfg.d_ff
+    wr = (torch.randn(E, d, generator=g) * cfg.router_std).to(cfg.act_dtype).double().numpy()
+    w1 = (torch.randn(E, 2 * f, d, generator=g) * cfg.w_std).to(cfg.weight_dtype).double().numpy()
+    w2 = (torch.randn(E, d, f, generator=g) * cfg.w_std).to(cfg.weight_dtype).double().numpy()
+    bias = (torch.randn(E, generator=g) * cfg.bias_std).double().numpy() if cfg.bias_std else None
+    done = 0
+    t0 = time.perf_counter()
+    while True:
+        x = torch.randn(chunk, d, generator=g).to(cfg.act_dtype).double().numpy()
+        dout = torch.randn(chunk, d, generator=g).to(cfg.act_dtype).double().numpy()
+        ref.layer_fwd_bwd(x, wr, w1, w2, dout, k, bias)
+        done += chunk
+        el = time.perf_counter() - t0
+        if el >= budget_s or done >= T:
+            break
+    return {"value": round(done / el, 2), "unit": "tokens/s", "cores": _blas_threads(),
+            "kind": "oracle",
+            "sample": f"{done} of {T} tokens of {cfg.name} in micro-batches of {chunk} "
+                      f"(full expert weights; float64 NumPy), {el:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    cfg = inputs.CONFIGS[args.workload]
+    steps = []
+    budget = max(2.0, args.cpu_seconds / max(1, args.steps))
+    for _ in range(args.warmup):
+        cpu_baseline(cfg, budget_s=min(1.0, budget))
+    for _ in range(args.steps):
+        steps.append(cpu_baseline(cfg, budget_s=budget))
+    v = statistics.mean(s["value"] for s in steps)
+    cb = dict(steps[-1])
+    cb["value"] = round(v, 2)
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 2), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(cfg.T / v * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": _workload_desc(cfg, None), "cpu_baseline": cb,
+            "e2e": {"value": round(v, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="bf16_e8", choices=sorted(inputs.CONFIGS))
+    ap.add_argument("--capacity-factor", action="store_true",
+                    help="padded-capacity layout (workloads that define a capacity factor)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line:
+            print(json.dumps(line), flush=True)
+        return
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    try:
+        line = run_ours(args, rank, world)
+        if line:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,223 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) token-routed Mixture-of-Experts FFN layer.
+ *
+ * One layer, forward and backward, on one GPU: router logits with fused
+ * softmax/top-k, on-device expert counts and offsets, a rowwise permute into
+ * contiguous per-expert buffers, a device-scheduled grouped SwiGLU GEMM,
+ * a gate-weighted combine, and the backward of each step; plus MXFP8 block
+ * quantisation.
+ *
+ * Sources (news pages about the Olmo-core 3 release; they describe the method
+ * in prose only):
+ *   [kongchang]  "Ai2 Olmo-core 3：MoE训练吞吐量提升2.7倍的秘诀", sections
+ *                容量税 (capacity tax), 路由不只是模型问题，更是系统问题 (routing
+ *                is a systems problem), 吞吐量数字的边界条件 (boundary conditions).
+ *   [bytechap]   "Olmo-core 3 mở rộng quy mô đào tạo mixture-of-experts lên hàng
+ *                nghìn tỷ tham số", section "Cách thức hoạt động" (how it works).
+ *   [aikraft]    "Прорыв в масштабируемости и производительности", section
+ *                "Технические оптимизации: от MXFP8 до маршрутизации".
+ *
+ * Conventions for every entry point
+ *   - Notation: T tokens, d = d_model, E experts, k = top_k, f = d_ff,
+ *     R = T*k permuted rows.  All matrices are row-major and dense.
+ *   - Every pointer argument is a DEVICE pointer owned by the caller, unless
+ *     the argument is documented as host memory.  The library keeps no
+ *     pointer after a call returns and allocates no device memory: scratch
+ *     comes from the caller's workspace (see moe_workspace_size).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*,
+ *     NULL = the legacy default stream), makes no host synchronisation and
+ *     no device-to-host copy: routing metadata never returns to the host
+ *     ([kongchang] routing section: metadata stays on the GPU; [bytechap] how
+ *     it works: the CPU queues work without waiting).  Calls can be captured
+ *     in a CUDA graph.
+ *   - Device pointers must be 16-byte aligned.  Row counts and offsets are
+ *     int32.
+ *   - Errors: a call validates its arguments on the host before it launches
+ *     anything and returns MOE_ERR_INVALID_ARG (bad sizes, null or misaligned
+ *     pointers, too small workspace) or MOE_ERR_UNSUPPORTED (valid but not
+ *     implemented, e.g. a shape the tensor-core tiles do not cover); nothing
+ *     is launched in that case.  MOE_ERR_CUDA reports a failed launch.
+ *     A kernel that gives up a bounded wait records MOE_ERR_TIMEOUT in the
+ *     workspace status word; read it with moe_get_device_status.  No C++
+ *     exception crosses this interface.
+ *   - dtype: MOE_F32 (fp32 everywhere, CUDA-core GEMMs), MOE_BF16 (bf16
+ *     activations and weights, fp32 accumulation, tcgen05 tensor cores).
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,
+  MOE_ERR_UNSUPPORTED = 2,
+  MOE_ERR_CUDA = 3,
+  MOE_ERR_TIMEOUT = 4
+} moe_status;
+
+typedef enum moe_dtype { MOE_F32 = 0, MOE_BF16 = 1, MOE_MXFP8 = 2 } moe_dtype;
+
+/* The problem as the pages state it: T tokens of width d_model, E experts,
+ * each token routed to top_k of them, expert hidden width d_ff.
+ * Limits: 1 <= top_k <= min(E, 32), E <= 1024, d_model % 8 == 0,
+ * d_ff % 8 == 0, T >= 0, T * top_k < 2^31. */
+typedef struct moe_shape {
+  int32_t T;
+  int32_t d_model;
+  int32_t E;
+  int32_t top_k;
+  int32_t d_ff;
+} moe_shape;
+
+/* Library version string (static storage). */
+const char* moe_version(void);
+
+/* Bytes of device workspace that the calls taking `ws` need for this shape.
+ * `rows` is the largest row count passed to moe_grouped_ffn_bwd (T*top_k
+ * for the dropless layout, E*capacity for the padded one); 0 means T*top_k.
+ * The first 256 bytes hold the status word; it must be zeroed once by the
+ * caller (cudaMemset) before the first call. */
+size_t moe_workspace_size(moe_shape shape, int dtype, int64_t rows);
+
+/* Read and clear the workspace status word (MOE_OK or MOE_ERR_TIMEOUT).
+ * Diagnostic only: this call SYNCHRONISES `stream` and copies 4 bytes to
+ * the host, unlike every other call. */
+moe_status moe_get_device_status(void* ws, void* stream, int32_t* status_out);
+
+/* ---- a1 + a2: route ------------------------------------------------------
+ * [kongchang] capacity tax: each token is routed to a few of the experts;
+ * routing section: routing metadata (split sizes and expert GEMM group sizes)
+ * stays on the GPU.
+ *   logits[t,e]  = sum_c x[t,c] * w_router[e,c] + bias[e]      (fp32 [T,E])
+ *   p            = softmax over e of logits[t,:]
+ *   topk_idx[t,j]: experts ordered by (-logits, e), first k     (int32 [T,k])
+ *                  -- the lowest index wins ties
+ *   topk_gate[t,j] = p[t, topk_idx[t,j]], not renormalised      (fp32 [T,k])
+ *   counts[e]     = #{(t,j): topk_idx[t,j] == e}               (int32 [E])
+ *   offsets       = exclusive prefix sum of counts             (int32 [E+1])
+ *   slot_row[t,j] = offsets[e] + #{t' < t : e in topk_idx[t']}  (int32 [T,k])
+ * x: [T,d] (fp32 for MOE_F32, bf16 for MOE_BF16); w_router: [E,d] same type;
+ * bias: fp32 [E] or NULL.  ws/ws_bytes: workspace (moe_workspace_size).
+ * The discrete steps are exact given the fp32 logits: indices, counts,
+ * offsets and rows are deterministic. */
+moe_status moe_route(moe_shape shape, int dtype, const void* x, const void* w_router,
+                     const float* bias, float* logits, int32_t* topk_idx, float* topk_gate,
+                     int32_t* counts, int32_t* offsets, int32_t* slot_row, void* ws,
+                     size_t ws_bytes, void* stream);
+
+/* ---- a3: rowwise permute -------------------------------------------------
+ * [bytechap] how it works: rowwise dispatch places routed rows directly in
+ * the experts' input buffers.
+ *   x_perm[slot_row[t,j], :] = x[t, :];  perm_src[slot_row[t,j]] = t
+ * x: [T,d]; x_perm: [T*k, d] same type; perm_src: int32 [T*k]. */
+moe_status moe_permute(moe_shape shape, int dtype, const void* x, const int32_t* slot_row,
+                       void* x_perm, int32_t* perm_src, void* stream);
+
+/* ---- a4: grouped SwiGLU FFN, forward -------------------------------------
+ * [kongchang] routing section: a device-scheduled grouped GEMM handles the
+ * uneven per-expert shapes; the tile scheduler reads `offsets` from device
+ * memory (no host round trip for group sizes).
+ * For expert e and rows r in [offsets[e], offsets[e+1]):
+ *   a = X W1[e,0:f]^T, u = X W1[e,f:2f]^T, h = silu(a)*u, y = h W2[e]^T
+ * rows:     number of rows of x_perm / y_perm / act_saved (T*k dropless;
+ *           E*capacity padded).  offsets[E] <= rows.
+ * x_perm:   [rows, d];  w1: [E, 2f, d] (gate rows then up rows);
+ * w2:       [E, d, f];  act_saved: [rows, 3f] = a | u | h (saved for bwd);
+ * y_perm:   [rows, d].  Rows outside every expert segment are not written.
+ * MOE_BF16 needs d % 256 == 0 and f % 128 == 0 (tensor-core tiles).
+ * mx must be NULL (MXFP8 GEMMs are not part of this version). */
+moe_status moe_grouped_ffn_fwd(moe_shape shape, int dtype, int64_t rows, const void* x_perm,
+                               const int32_t* offsets, const void* w1, const void* w2,
+                               const void* mx, void* act_saved, void* y_perm, void* ws,
+                               size_t ws_bytes, void* stream);
+
+/* ---- a5: gate-weighted combine -------------------------------------------
+ *   out[t,:] = sum_{j ascending, slot_row[t,j] >= 0} topk_gate[t,j] * y_perm[slot_row[t,j],:]
+ * fp32 accumulation, rounded once to the output type.  A row index of -1
+ * (a pair dropped by the padded layout) contributes nothing.
+ * y_perm: [rows, d]; out: [T, d]. */
+moe_status moe_combine(moe_shape shape, int dtype, const void* y_perm, const int32_t* slot_row,
+                       const float* topk_gate, void* out, void* stream);
+
+/* ---- a6: combine backward ------------------------------------------------
+ *   dgate[t,j]            = <dout[t,:], y_perm[slot_row[t,j],:]>   (fp32 [T,k])
+ *   dy_perm[slot_row[t,j]] = topk_gate[t,j] * dout[t,:]           ([rows, d])
+ * Pairs with slot_row -1 get dgate 0 and write no row.  Rows of dy_perm not
+ * named by slot_row are not written (zero them once for the padded layout). */
+moe_status moe_combine_bwd(moe_shape shape, int dtype, const void* dout, const void* y_perm,
+                           const int32_t* slot_row, const float* topk_gate, void* dy_perm,
+                           float* dgate, void* stream);
+
+/* ---- a7 + a8: grouped SwiGLU FFN, backward -------------------------------
+ * Per expert e on its rows: dh = dy W2[e]; s = sigmoid(a);
+ *   da = dh*u*s*(1 + a*(1-s)); du = dh*silu(a);
+ *   dx_perm = da W1[e,0:f] + du W1[e,f:2f];
+ *   dW2[e] = dy^T h; dW1[e,0:f] = da^T x; dW1[e,f:2f] = du^T x.
+ * An expert with no rows gets dW1[e] = dW2[e] = 0 (dW is overwritten).
+ * dy_perm, x_perm: [rows, d]; act_saved: [rows, 3f] from the forward;
+ * dx_perm: [rows, d]; dw1: [E, 2f, d]; dw2: [E, d, f] of type dw_dtype
+ * (MOE_F32 or MOE_BF16; MOE_F32 only when dtype is MOE_F32).
+ * Uses 2*f*rows elements of scratch in `ws` for [da | du]. */
+moe_status moe_grouped_ffn_bwd(moe_shape shape, int dtype, int64_t rows, const void* dy_perm,
+                               const void* x_perm, const void* act_saved,
+                               const int32_t* offsets, const void* w1, const void* w2,
+                               const void* mx, void* dx_perm, void* dw1, void* dw2,
+                               int dw_dtype, void* ws, size_t ws_bytes, void* stream);
+
+/* ---- a9: unpermute-grad + router grad ------------------------------------
+ *   dx[t,:]  = sum_{j, slot_row[t,j] >= 0} dx_perm[slot_row[t,j],:] + sum_e dl[t,e] w_router[e,:]
+ *   dl[t,:]  = p * (dp - <p, dp>),  p = softmax(logits[t,:]),
+ *              dp[e] = dgate[t,j] where e = topk_idx[t,j], else 0
+ *   dw_router = dl^T x                                   (fp32 [E, d], overwritten)
+ * x, dx: [T, d]; w_router: [E, d]; logits fp32 [T,E]; dgate fp32 [T,k].
+ * Deterministic: fixed summation order, no floating-point atomics. */
+moe_status moe_route_bwd(moe_shape shape, int dtype, const void* x, const void* w_router,
+                         const float* logits, const int32_t* topk_idx, const float* dgate,
+                         const void* dx_perm, const int32_t* slot_row, void* dx,
+                         float* dw_router, void* ws, size_t ws_bytes, void* stream);
+
+/* ---- a10: MXFP8 quantisation ---------------------------------------------
+ * [kongchang] boundary-conditions section: MXFP8 shares one scale among every
+ * 32 elements; an FP32 master weight is kept.  Rule (OCP MX reading):
+ *   per block V of 32: amax = max|V_i|; e = floor(log2 amax) - 8, clamped to
+ *   [-127, 127] (amax == 0 -> -127); scale byte = e + 127 (E8M0);
+ *   q_i = E4M3 round-to-nearest-even of V_i / 2^e, saturated to +-448, the
+ *   sign bit taken from V_i.
+ * src: [rows, K] of src_dtype (MOE_F32 or MOE_BF16).
+ * axis 0: blocks of 32 along each row (K % 32 == 0); scale: u8 [rows, K/32].
+ * axis 1: blocks of 32 consecutive rows within each column, restarting at
+ *   every segment start seg_offsets[g] (device int32 [nseg+1], or NULL for one
+ *   segment [0, rows)); a segment's last partial block is zero-padded.
+ *   scale: u8 [S, K] with S = sum_g ceil(len_g / 32), segment by segment;
+ *   the buffer must hold rows/32 + nseg + 1 rows (K % 16 == 0).
+ * q: u8 [rows, K].  Bytes are exact (bit-for-bit with the rule above). */
+moe_status mxfp8_quantize(int64_t rows, int64_t K, int src_dtype, const void* src, int axis,
+                          const int32_t* seg_offsets, int nseg, uint8_t* q, uint8_t* scale,
+                          void* stream);
+
+/* ---- a11: padded-capacity comparison layout ------------------------------
+ * [kongchang] routing section: the report compares the device-scheduled
+ * grouped GEMM with padding every expert batch to one uniform capacity.
+ * With capacity C (e.g. ceil(1.25 * T*k / E)): a pair (t,j) with rank
+ * q = slot_row[t,j] - offsets[topk_idx[t,j]] is kept iff q < C and then
+ *   x_pad[e*C + q, :] = x[t, :],  pad_row[t,j] = e*C + q;  else pad_row = -1.
+ * Unused rows of x_pad are zeroed; offsets_pad[e] = e*C (int32 [E+1]).
+ * The grouped FFN, combine, combine-bwd and route-bwd calls then take
+ * rows = E*C, offsets_pad and pad_row in place of offsets and slot_row.
+ * x_pad: [E*C, d]; pad_row: int32 [T,k]. */
+moe_status moe_padded_dispatch(moe_shape shape, int dtype, int32_t capacity, const void* x,
+                               const int32_t* topk_idx, const int32_t* slot_row,
+                               const int32_t* offsets, void* x_pad, int32_t* pad_row,
+                               int32_t* offsets_pad, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,180 @@
+"""Thin ctypes binding of ``include/moe.h`` (argument marshalling only).
+
+Every function here has the name of its C entry point and forwards torch
+tensors as raw device pointers plus the current CUDA stream.  No step of the
+method runs in Python; if the CUDA library is missing the import of a
+function fails loudly (there is no fallback).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmoe_b200.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "moe.h")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = range(5)
+MOE_F32, MOE_BF16, MOE_MXFP8 = 0, 1, 2
+STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
+                3: "MOE_ERR_CUDA", 4: "MOE_ERR_TIMEOUT"}
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} returned {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+class moe_shape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("d_model", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("top_k", ctypes.c_int32), ("d_ff", ctypes.c_int32)]
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+_SIGS = {
+    "moe_version": (ctypes.c_char_p, []),
+    "moe_workspace_size": (_SZ, [moe_shape, _I, _I64]),
+    "moe_get_device_status": (_I, [_P, _P, _P]),
+    "moe_route": (_I, [moe_shape, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "moe_permute": (_I, [moe_shape, _I, _P, _P, _P, _P, _P]),
+    "moe_grouped_ffn_fwd": (_I, [moe_shape, _I, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "moe_combine": (_I, [moe_shape, _I, _P, _P, _P, _P, _P]),
+    "moe_combine_bwd": (_I, [moe_shape, _I, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_grouped_ffn_bwd": (_I, [moe_shape, _I, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                 _I, _P, _SZ, _P]),
+    "moe_route_bwd": (_I, [moe_shape, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "mxfp8_quantize": (_I, [_I64, _I64, _I, _P, _I, _P, _I, _P, _P, _P]),
+    "moe_padded_dispatch": (_I, [moe_shape, _I, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _P, _P]),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the in-tree CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m mixture_experts_layer_offsets_b200.build`")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(l, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = l
+    return _lib
+
+
+def header_symbols() -> list[str]:
+    """Entry points declared in include/moe.h."""
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:moe_status|size_t|const char\*)\s+(\w+)\s*\(", txt, re.M)))
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is not None:
+        return stream if isinstance(stream, int) else stream.cuda_stream
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _check(name: str, status: int) -> None:
+    if status != MOE_OK:
+        raise MoEError(name, status)
+
+
+def shape_of(T: int, d_model: int, E: int, top_k: int, d_ff: int) -> moe_shape:
+    return moe_shape(T, d_model, E, top_k, d_ff)
+
+
+def moe_version() -> str:
+    return lib().moe_version().decode()
+
+
+def moe_workspace_size(shape: moe_shape, dtype: int, rows: int = 0) -> int:
+    return lib().moe_workspace_size(shape, dtype, rows)
+
+
+def moe_get_device_status(ws, stream=None) -> int:
+    out = ctypes.c_int32(0)
+    _check("moe_get_device_status",
+           lib().moe_get_device_status(_ptr(ws), _stream(stream), ctypes.byref(out)))
+    return out.value
+
+
+def moe_route(shape, dtype, x, w_router, bias, logits, topk_idx, topk_gate, counts, offsets,
+              slot_row, ws, stream=None) -> None:
+    _check("moe_route", lib().moe_route(
+        shape, dtype, _ptr(x), _ptr(w_router), _ptr(bias), _ptr(logits), _ptr(topk_idx),
+        _ptr(topk_gate), _ptr(counts), _ptr(offsets), _ptr(slot_row), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_permute(shape, dtype, x, slot_row, x_perm, perm_src, stream=None) -> None:
+    _check("moe_permute", lib().moe_permute(shape, dtype, _ptr(x), _ptr(slot_row), _ptr(x_perm),
+                                            _ptr(perm_src), _stream(stream)))
+
+
+def moe_grouped_ffn_fwd(shape, dtype, rows, x_perm, offsets, w1, w2, act_saved, y_perm, ws,
+                        mx=None, stream=None) -> None:
+    _check("moe_grouped_ffn_fwd", lib().moe_grouped_ffn_fwd(
+        shape, dtype, rows, _ptr(x_perm), _ptr(offsets), _ptr(w1), _ptr(w2), _ptr(mx),
+        _ptr(act_saved), _ptr(y_perm), _ptr(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
+
+
+def moe_combine(shape, dtype, y_perm, slot_row, topk_gate, out, stream=None) -> None:
+    _check("moe_combine", lib().moe_combine(shape, dtype, _ptr(y_perm), _ptr(slot_row),
+                                            _ptr(topk_gate), _ptr(out), _stream(stream)))
+
+
+def moe_combine_bwd(shape, dtype, dout, y_perm, slot_row, topk_gate, dy_perm, dgate,
+                    stream=None) -> None:
+    _check("moe_combine_bwd", lib().moe_combine_bwd(
+        shape, dtype, _ptr(dout), _ptr(y_perm), _ptr(slot_row), _ptr(topk_gate), _ptr(dy_perm),
+        _ptr(dgate), _stream(stream)))
+
+
+def moe_grouped_ffn_bwd(shape, dtype, rows, dy_perm, x_perm, act_saved, offsets, w1, w2,
+                        dx_perm, dw1, dw2, dw_dtype, ws, mx=None, stream=None) -> None:
+    _check("moe_grouped_ffn_bwd", lib().moe_grouped_ffn_bwd(
+        shape, dtype, rows, _ptr(dy_perm), _ptr(x_perm), _ptr(act_saved), _ptr(offsets),
+        _ptr(w1), _ptr(w2), _ptr(mx), _ptr(dx_perm), _ptr(dw1), _ptr(dw2), dw_dtype, _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_route_bwd(shape, dtype, x, w_router, logits, topk_idx, dgate, dx_perm, slot_row, dx,
+                  dw_router, ws, stream=None) -> None:
+    _check("moe_route_bwd", lib().moe_route_bwd(
+        shape, dtype, _ptr(x), _ptr(w_router), _ptr(logits), _ptr(topk_idx), _ptr(dgate),
+        _ptr(dx_perm), _ptr(slot_row), _ptr(dx), _ptr(dw_router), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def mxfp8_quantize(rows, K, src_dtype, src, axis, seg_offsets, nseg, q, scale,
+                   stream=None) -> None:
+    _check("mxfp8_quantize", lib().mxfp8_quantize(
+        rows, K, src_dtype, _ptr(src), axis, _ptr(seg_offsets), nseg, _ptr(q), _ptr(scale),
+        _stream(stream)))
+
+
+def moe_padded_dispatch(shape, dtype, capacity, x, topk_idx, slot_row, offsets, x_pad, pad_row,
+                        offsets_pad, stream=None) -> None:
+    _check("moe_padded_dispatch", lib().moe_padded_dispatch(
+        shape, dtype, capacity, _ptr(x), _ptr(topk_idx), _ptr(slot_row), _ptr(offsets),
+        _ptr(x_pad), _ptr(pad_row), _ptr(offsets_pad), _stream(stream)))

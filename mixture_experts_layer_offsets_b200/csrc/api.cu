@@ -1,0 +1,240 @@
+// api.cu -- the extern "C" entry points declared in include/moe.h: argument
+// validation on the host, workspace carving, and dispatch to the kernels.
+// Nothing here computes on the host and nothing synchronises a stream (except
+// the documented diagnostic moe_get_device_status).
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// All pointers non-null and 16-byte aligned.
+template <typename... P>
+inline bool ptrs_ok(P... ps) {
+  const void* arr[] = {static_cast<const void*>(ps)...};
+  for (const void* p : arr)
+    if (!p || !aligned16(p)) return false;
+  return true;
+}
+
+inline bool dtype_act_ok(int dtype) { return dtype == MOE_F32 || dtype == MOE_BF16; }
+
+moe_status shape_ok(const moe_shape& s) {
+  if (s.T < 0 || s.d_model <= 0 || s.E <= 0 || s.top_k <= 0 || s.d_ff <= 0) return MOE_ERR_INVALID_ARG;
+  if (s.E > 1024 || s.top_k > s.E || s.top_k > 32) return MOE_ERR_INVALID_ARG;
+  if (s.d_model % 8 || s.d_ff % 8) return MOE_ERR_INVALID_ARG;
+  if ((int64_t)s.T * s.top_k >= (int64_t)1 << 31) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+inline moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+inline int* status_word(void* ws) { return static_cast<int*>(ws); }
+inline void* scratch(void* ws) { return static_cast<uint8_t*>(ws) + kStatusBytes; }
+
+size_t ws_need(const moe_shape& s, int dtype, int64_t rows) {
+  if (rows <= 0) rows = (int64_t)s.T * s.top_k;
+  FfnShape fs{s.d_model, s.E, s.d_ff, rows};
+  size_t need = route_ws_bytes(s.T, s.E, s.top_k);
+  need = std::max(need, route_bwd_ws_bytes(s.T, s.d_model, s.E));
+  need = std::max(need, ffn_bwd_ws_bytes(fs, dtype != MOE_F32));
+  return kStatusBytes + align256(need);
+}
+
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_version(void) { return "moe-b200 0.1 (sm_100a)"; }
+
+size_t moe_workspace_size(moe_shape shape, int dtype, int64_t rows) {
+  if (shape_ok(shape) != MOE_OK) return 0;
+  return ws_need(shape, dtype, rows);
+}
+
+moe_status moe_get_device_status(void* ws, void* stream, int32_t* status_out) {
+  if (!ws || !status_out) return MOE_ERR_INVALID_ARG;
+  int32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, as_stream(stream));
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, sizeof(v), as_stream(stream));
+  if (e == cudaSuccess) e = cudaStreamSynchronize(as_stream(stream));
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  *status_out = v;
+  return MOE_OK;
+}
+
+moe_status moe_route(moe_shape s, int dtype, const void* x, const void* w_router, const float* bias,
+                     float* logits, int32_t* topk_idx, float* topk_gate, int32_t* counts,
+                     int32_t* offsets, int32_t* slot_row, void* ws, size_t ws_bytes,
+                     void* stream) {
+  moe_status st = shape_ok(s);
+  if (st != MOE_OK) return st;
+  if (!dtype_act_ok(dtype)) return dtype == MOE_MXFP8 ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
+  if (!ptrs_ok(w_router, counts, offsets, ws)) return MOE_ERR_INVALID_ARG;
+  if (s.T > 0 && !ptrs_ok(x, logits, topk_idx, topk_gate, slot_row)) return MOE_ERR_INVALID_ARG;
+  if (bias && !aligned16(bias)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < ws_need(s, dtype, 0)) return MOE_ERR_INVALID_ARG;
+  RouteArgs a{x, w_router, bias, s.T, s.d_model, s.E, s.top_k, logits, topk_idx, topk_gate,
+              counts, offsets, slot_row, scratch(ws)};
+  return cuda_status(route_launch(a, dtype == MOE_BF16, as_stream(stream)));
+}
+
+moe_status moe_permute(moe_shape s, int dtype, const void* x, const int32_t* slot_row,
+                       void* x_perm, int32_t* perm_src, void* stream) {
+  moe_status st = shape_ok(s);
+  if (st != MOE_OK) return st;
+  if (!dtype_act_ok(dtype)) return dtype == MOE_MXFP8 ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
+  if (s.T == 0) return MOE_OK;
+  if (!ptrs_ok(x, slot_row, x_perm, perm_src)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(permute_launch(dtype == MOE_BF16, x, slot_row, x_perm, perm_src, s.T,
+                                    s.d_model, s.top_k, as_stream(stream)));
+}
+
+moe_status moe_grouped_ffn_fwd(moe_shape s, int dtype, int64_t rows, const void* x_perm,
+                               const int32_t* offsets, const void* w1, const void* w2,
+                               const void* mx, void* act_saved, void* y_perm, void* ws,
+                               size_t ws_bytes, void* stream) {
+  moe_status st = shape_ok(s);
+  if (st != MOE_OK) return st;
+  if (dtype == MOE_MXFP8 || mx) return MOE_ERR_UNSUPPORTED;
+  if (!dtype_act_ok(dtype) || rows < 0 || rows >= ((int64_t)1 << 31)) return MOE_ERR_INVALID_ARG;
+  if (!ptrs_ok(offsets, w1, w2, ws)) return MOE_ERR_INVALID_ARG;
+  if (rows > 0 && !ptrs_ok(x_perm, act_saved, y_perm)) return MOE_ERR_INVALID_ARG;
+  (void)ws_bytes;
+  FfnShape fs{s.d_model, s.E, s.d_ff, rows};
+  cudaStream_t cs = as_stream(stream);
+  if (dtype == MOE_F32)
+    return cuda_status(ffn_fwd_f32(fs, static_cast<const float*>(x_perm), offsets,
+                                   static_cast<const float*>(w1), static_cast<const float*>(w2),
+                                   static_cast<float*>(act_saved), static_cast<float*>(y_perm), cs));
+  if (s.d_model % 256 || s.d_ff % 256) return MOE_ERR_UNSUPPORTED;
+  return cuda_status(
+      ffn_fwd_bf16(fs, x_perm, offsets, w1, w2, act_saved, y_perm, status_word(ws), cs));
+}
+
+moe_status moe_combine(moe_shape s, int dtype, const void* y_perm, const int32_t* slot_row,
+                       const float* topk_gate, void* out, void* stream) {
+  moe_status st = shape_ok(s);
+  if (st != MOE_OK) return st;
+  if (!dtype_act_ok(dtype)) return dtype == MOE_MXFP8 ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
+  if (s.T == 0) return MOE_OK;
+  if (!ptrs_ok(y_perm, slot_row, topk_gate, out)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(combine_launch(dtype == MOE_BF16, y_perm, slot_row, topk_gate, out, s.T,
+                                    s.d_model, s.top_k, as_stream(stream)));
+}
+
+moe_status moe_combine_bwd(moe_shape s, int dtype, const void* dout, const void* y_perm,
+                           const int32_t* slot_row, const float* topk_gate, void* dy_perm,
+                           float* dgate, void* stream) {
+  moe_status st = shape_ok(s);
+  if (st != MOE_OK) return st;
+  if (!dtype_act_ok(dtype)) return dtype == MOE_MXFP8 ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
+  if (s.T == 0) return MOE_OK;
+  if (!ptrs_ok(dout, y_perm, slot_row, topk_gate, dy_perm, dgate)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(combine_bwd_launch(dtype == MOE_BF16, dout, y_perm, slot_row, topk_gate,
+                                        dy_perm, dgate, s.T, s.d_model, s.top_k,
+                                        as_stream(stream)));
+}
+
+moe_status moe_grouped_ffn_bwd(moe_shape s, int dtype, int64_t rows, const void* dy_perm,
+                               const void* x_perm, const void* act_saved,
+                               const int32_t* offsets, const void* w1, const void* w2,
+                               const void* mx, void* dx_perm, void* dw1, void* dw2,
+                               int dw_dtype, void* ws, size_t ws_bytes, void* stream) {
+  moe_status st = shape_ok(s);
+  if (st != MOE_OK) return st;
+  if (dtype == MOE_MXFP8 || mx) return MOE_ERR_UNSUPPORTED;
+  if (!dtype_act_ok(dtype) || rows < 0 || rows >= ((int64_t)1 << 31)) return MOE_ERR_INVALID_ARG;
+  if (dw_dtype != MOE_F32 && dw_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (dtype == MOE_F32 && dw_dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
+  if (!ptrs_ok(offsets, w1, w2, dw1, dw2, ws)) return MOE_ERR_INVALID_ARG;
+  if (rows > 0 && !ptrs_ok(dy_perm, x_perm, act_saved, dx_perm)) return MOE_ERR_INVALID_ARG;
+  FfnShape fs{s.d_model, s.E, s.d_ff, rows};
+  if (ws_bytes < kStatusBytes + ffn_bwd_ws_bytes(fs, dtype == MOE_BF16)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t cs = as_stream(stream);
+  if (dtype == MOE_F32)
+    return cuda_status(ffn_bwd_f32(fs, static_cast<const float*>(dy_perm),
+                                   static_cast<const float*>(x_perm),
+                                   static_cast<const float*>(act_saved), offsets,
+                                   static_cast<const float*>(w1), static_cast<const float*>(w2),
+                                   static_cast<float*>(dx_perm), static_cast<float*>(dw1),
+                                   static_cast<float*>(dw2), scratch(ws), cs));
+  if (s.d_model % 256 || s.d_ff % 256) return MOE_ERR_UNSUPPORTED;
+  return cuda_status(ffn_bwd_bf16(fs, dy_perm, x_perm, act_saved, offsets, w1, w2, dx_perm, dw1,
+                                  dw2, dw_dtype == MOE_F32, scratch(ws), status_word(ws), cs));
+}
+
+moe_status moe_route_bwd(moe_shape s, int dtype, const void* x, const void* w_router,
+                         const float* logits, const int32_t* topk_idx, const float* dgate,
+                         const void* dx_perm, const int32_t* slot_row, void* dx,
+                         float* dw_router, void* ws, size_t ws_bytes, void* stream) {
+  moe_status st = shape_ok(s);
+  if (st != MOE_OK) return st;
+  if (!dtype_act_ok(dtype)) return dtype == MOE_MXFP8 ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
+  if (!ptrs_ok(w_router, dw_router, ws)) return MOE_ERR_INVALID_ARG;
+  if (s.T > 0 && !ptrs_ok(x, logits, topk_idx, dgate, dx_perm, slot_row, dx))
+    return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < kStatusBytes + route_bwd_ws_bytes(s.T, s.d_model, s.E)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(route_bwd_launch(dtype == MOE_BF16, x, w_router, logits, topk_idx, dgate,
+                                      dx_perm, slot_row, dx, dw_router, s.T, s.d_model, s.E,
+                                      s.top_k, scratch(ws), as_stream(stream)));
+}
+
+moe_status mxfp8_quantize(int64_t rows, int64_t K, int src_dtype, const void* src, int axis,
+                          const int32_t* seg_offsets, int nseg, uint8_t* q, uint8_t* scale,
+                          void* stream) {
+  if (rows < 0 || K < 0 || (src_dtype != MOE_F32 && src_dtype != MOE_BF16)) return MOE_ERR_INVALID_ARG;
+  if (axis == 0) {
+    if (K % 32) return MOE_ERR_INVALID_ARG;
+  } else if (axis == 1) {
+    if (K % 16) return MOE_ERR_INVALID_ARG;
+    if (seg_offsets && (nseg < 1 || nseg > 1024 || !aligned16(seg_offsets))) return MOE_ERR_INVALID_ARG;
+  } else {
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (rows == 0 || K == 0) return MOE_OK;
+  if (!ptrs_ok(src, q, scale)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(mxfp8_launch(rows, K, src_dtype == MOE_BF16, src, axis, seg_offsets, nseg, q,
+                                  scale, as_stream(stream)));
+}
+
+moe_status moe_padded_dispatch(moe_shape s, int dtype, int32_t capacity, const void* x,
+                               const int32_t* topk_idx, const int32_t* slot_row,
+                               const int32_t* offsets, void* x_pad, int32_t* pad_row,
+                               int32_t* offsets_pad, void* stream) {
+  moe_status st = shape_ok(s);
+  if (st != MOE_OK) return st;
+  if (!dtype_act_ok(dtype)) return dtype == MOE_MXFP8 ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
+  if (capacity <= 0 || (int64_t)capacity * s.E >= ((int64_t)1 << 31)) return MOE_ERR_INVALID_ARG;
+  if (!ptrs_ok(offsets, x_pad, offsets_pad)) return MOE_ERR_INVALID_ARG;
+  if (s.T > 0 && !ptrs_ok(x, topk_idx, slot_row, pad_row)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(padded_dispatch_launch(dtype == MOE_BF16, capacity, x, topk_idx, slot_row,
+                                            offsets, x_pad, pad_row, offsets_pad, s.T, s.d_model,
+                                            s.E, s.top_k, as_stream(stream)));
+}
+
+}  // extern "C"

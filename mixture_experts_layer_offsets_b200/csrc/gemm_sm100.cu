@@ -1,0 +1,646 @@
+// gemm_sm100.cu -- device-scheduled grouped GEMM on the 5th-generation tensor
+// cores (tcgen05 + TMEM + TMA), bf16 operands, fp32 accumulation, with the
+// SwiGLU forward and backward fused into the epilogues; and the bf16 expert
+// FFN forward/backward built from it.
+//
+// Page: "Ai2 Olmo-core 3：MoE训练吞吐量提升2.7倍的秘诀" (kongchang.com), section
+// 路由不只是模型问题，更是系统问题: a device-scheduled grouped GEMM handles the
+// uneven per-expert shapes produced by routing, packing the small GEMMs of all
+// experts into one kernel without padding; group sizes never go back to the host.
+//
+// Kernel structure (one CTA per SM, persistent; 6 warps):
+//   warp 0      TMA producer (one thread): A/B tiles -> S-stage smem ring
+//   warp 1      MMA issuer (one thread issues tcgen05.mma M=128 N=BN K=16;
+//               the warp zeroes ragged K tails of weight-gradient tiles)
+//   warps 2..5  epilogue: tcgen05.ld TMEM -> registers -> fused math -> global
+// TMEM holds two BN-column fp32 accumulators so the epilogue of one tile
+// overlaps the main loop of the next.
+//
+// Tile scheduler: each CTA reads offsets[0..E] from device memory into shared
+// memory and builds the per-expert tile prefix itself; tile t of the launch is
+// then found by a binary search.  The host never learns the group sizes: it
+// launches one CTA per SM and idle CTAs exit.
+//   GROUP_M (forward, dgrad): expert g owns rows [off[g], off[g+1]) of A and
+//     of the output; M tiles of 128 rows; rows of a tile beyond the segment
+//     are computed but not stored.
+//   GROUP_K (wgrad): expert g owns the K range [off[g], off[g+1]) of both
+//     operands (the token axis); the rows of the last K block that belong to
+//     the next expert are zeroed in shared memory before the MMA reads them;
+//     an expert without rows writes a zero tile.
+//
+// Shared-memory operand layouts (128-byte swizzle, matching the TMA swizzle):
+//   K-major  (rows of K contiguous): 128-B rows, 8-row groups 1024 B apart
+//            (SBO = 1024); the K=16 slices of a 64-wide stage start 32 B apart.
+//   MN-major (rows of M/N contiguous, K along rows): boxes of 64 M/N elements
+//            x 64 K rows; 8-K-row groups 1024 B apart (SBO), 64-element M/N
+//            blocks 8192 B apart (LBO); K=16 slices start 2048 B apart.
+//
+// Every mbarrier wait is bounded (common.cuh); on a timeout the kernel records
+// MOE_ERR_TIMEOUT, raises a CTA-wide abort flag, waits (bounded) for its own
+// TMA loads and MMAs in flight, frees TMEM and returns.
+#include "common.cuh"
+#include "internal.h"
+
+#include <cudaTypedefs.h>
+
+namespace moe {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int kThreads = 192;
+constexpr uint32_t kABytes = BM * BK * 2;  // 16 KB
+
+enum : int { EPI_SWIGLU_FWD = 0, EPI_STORE = 1, EPI_SWIGLU_BWD = 2, EPI_WGRAD = 3 };
+
+struct GemmParams {
+  CUtensorMap tmA;
+  CUtensorMap tmB;
+  const int32_t* offsets;
+  int E;
+  int M;        // GROUP_K: output rows per expert
+  int N;        // GROUP_M: output columns (SwiGLU forward: f); GROUP_K: output columns
+  int K;        // GROUP_M: reduction length
+  int b_rows;   // GROUP_M: rows of B per expert in the flattened weight tensor
+  int f;        // d_ff
+  __nv_bfloat16* out;
+  int64_t ld_out;
+  float* out_f32;          // EPI_WGRAD with fp32 output (else out)
+  const __nv_bfloat16* act;
+  int64_t ld_act;
+  int64_t out_group;       // EPI_WGRAD: elements per expert
+  int* status;
+};
+
+template <int BN> struct Cfg {
+  static constexpr uint32_t kBBytes = BN * BK * 2;
+  static constexpr uint32_t kStage = kABytes + kBBytes;
+  static constexpr int kStages = (BN == 256) ? 4 : 6;
+  static constexpr uint32_t kTmemCols = 2 * BN;
+  static constexpr size_t kSmem = 1024 + (size_t)kStages * kStage + 256 + 2 * 1025 * 4;
+};
+
+// ------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                          uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accum));
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(slot)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+#define MOE_R8(i) "=r"(r[i + 0]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), \
+                  "=r"(r[i + 4]), "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
+#define MOE_T8(i) "+r"(r[i + 0]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), \
+                  "+r"(r[i + 4]), "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7])
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : MOE_R8(0), MOE_R8(8), MOE_R8(16), MOE_R8(24)
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+// Orders every later use of r after the preceding wait::ld.
+__device__ __forceinline__ void tmem_tie(uint32_t (&r)[32]) {
+  asm volatile("" : MOE_T8(0), MOE_T8(8), MOE_T8(16), MOE_T8(24));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+__device__ __forceinline__ void store_64B(void* dst, const uint32_t (&v)[16]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+__device__ __forceinline__ float sigmoidf_(float a) { return 1.f / (1.f + __expf(-a)); }
+
+// ------------------------------------------------------------ tile decode
+struct TileInfo {
+  int g, m0, n0, rows, nkb, kbase, klast;
+};
+
+template <int BN, int EPI, bool GROUP_K>
+__device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, const int* s_off,
+                                                const int* s_pre, int nN) {
+  TileInfo ti;
+  if constexpr (GROUP_K) {
+    const int per = (p.M / BM) * nN;
+    ti.g = t / per;
+    const int local = t - ti.g * per;
+    ti.m0 = (local / nN) * BM;
+    ti.n0 = (local % nN) * BN;
+    ti.rows = BM;
+    const int k0 = s_off[ti.g], kg = s_off[ti.g + 1] - k0;
+    ti.kbase = k0;
+    ti.nkb = (kg + BK - 1) / BK;
+    ti.klast = kg - (ti.nkb - 1) * BK;
+  } else {
+    int lo = 0, hi = p.E - 1;
+    while (lo < hi) {  // last expert whose tile prefix is <= t (skips empty experts)
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_pre[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    ti.g = lo;
+    const int local = t - s_pre[lo];
+    const int mt = local / nN, nt = local - mt * nN;
+    ti.m0 = s_off[lo] + mt * BM;
+    ti.rows = min(BM, s_off[lo + 1] - s_off[lo] - mt * BM);
+    ti.n0 = nt * (EPI == EPI_SWIGLU_FWD ? 128 : BN);
+    ti.kbase = lo * p.b_rows;
+    ti.nkb = p.K / BK;
+    ti.klast = BK;
+  }
+  return ti;
+}
+
+// ------------------------------------------------------------------ kernel
+template <int BN, bool A_MN, bool B_MN, int EPI, bool GROUP_K>
+__global__ void __launch_bounds__(kThreads, 1)
+grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
+  using C = Cfg<BN>;
+  constexpr int S = C::kStages;
+  static_assert(EPI != EPI_SWIGLU_FWD || BN == 256, "SwiGLU forward pairs 128 gate + 128 up columns");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::kStage);
+  uint64_t* empty = full + S;
+  uint64_t* tfull = empty + S;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+  int* s_off = reinterpret_cast<int*>(smem + S * C::kStage + 256);
+  int* s_pre = s_off + 1025;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = p.E;
+  const int nN = GROUP_K ? p.N / BN : (EPI == EPI_SWIGLU_FWD ? p.N / 128 : p.N / BN);
+
+  for (int g = threadIdx.x; g <= E; g += kThreads) s_off[g] = p.offsets[g];
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+      for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 128); }
+      mbar_init(drain, 1);
+      *s_abort = 0;
+      fence_mbar_init();
+    }
+    __syncwarp();
+    tmem_alloc(s_tmem, C::kTmemCols);
+    tc_fence_before();
+  }
+  __syncthreads();
+  if constexpr (!GROUP_K) {
+    if (warp == 1) {  // per-expert tile prefix (E <= 1024: 32 experts per lane)
+      const int lo = lane * 32, hi = min(lo + 32, E);
+      int s = 0;
+      for (int g = lo; g < hi; ++g) s += ((s_off[g + 1] - s_off[g] + BM - 1) / BM) * nN;
+      int incl = s;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+      }
+      int run = incl - s;
+      for (int g = lo; g < hi; ++g) {
+        s_pre[g] = run;
+        run += ((s_off[g + 1] - s_off[g] + BM - 1) / BM) * nN;
+      }
+      if (lane == 31) s_pre[E] = incl;
+    }
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+  const int total = GROUP_K ? E * (p.M / BM) * nN : s_pre[E];
+
+  auto fail = [&]() {
+    record_status(p.status, MOE_ERR_TIMEOUT);
+    *s_abort = 1;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tmA);
+      tma_prefetch_desc(&p.tmB);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const TileInfo ti = decode_tile<BN, EPI, GROUP_K>(t, p, s_off, s_pre, nN);
+        for (int kb = 0; kb < ti.nkb; ++kb, ++it) {
+          if (*s_abort) { ok = false; break; }
+          const int s = it % S;
+          if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1)) { fail(); ok = false; break; }
+          uint8_t* sa = smem + s * C::kStage;
+          uint8_t* sb = sa + kABytes;
+          mbar_arrive_expect_tx(&full[s], C::kStage);
+          const int kc = kb * BK;
+          if constexpr (!A_MN) {
+            tma_load_2d(sa, &p.tmA, kc, ti.m0, &full[s]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 2; ++i) tma_load_2d(sa + i * 8192, &p.tmA, ti.m0 + 64 * i, ti.kbase + kc, &full[s]);
+          }
+          if constexpr (!B_MN) {
+#pragma unroll
+            for (int i = 0; i < BN / 128; ++i) {
+              const int row = ti.kbase + (EPI == EPI_SWIGLU_FWD ? (i == 0 ? ti.n0 : p.f + ti.n0)
+                                                               : ti.n0 + 128 * i);
+              tma_load_2d(sb + i * 16384, &p.tmB, kc, row, &full[s]);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < BN / 64; ++i)
+              tma_load_2d(sb + i * 8192, &p.tmB, ti.n0 + 64 * i, ti.kbase + kc, &full[s]);
+          }
+        }
+      }
+      if (!ok) {  // let this CTA's loads in flight land before shared memory is released
+        for (uint32_t j = it > (uint32_t)S ? it - S : 0; j < it; ++j)
+          (void)mbar_wait(&full[j % S], (j / S) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA
+    constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)A_MN << 15) |
+                               ((uint32_t)B_MN << 16) | ((uint32_t)(BN >> 3) << 17) |
+                               ((uint32_t)(BM >> 4) << 24);
+    uint32_t it = 0, acc_it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      const TileInfo ti = decode_tile<BN, EPI, GROUP_K>(t, p, s_off, s_pre, nN);
+      const int acc = acc_it & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&tempty[acc], ((acc_it >> 1) & 1) ^ 1))) {
+        if (lane == 0) fail();
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * BN;
+      for (int kb = 0; kb < ti.nkb; ++kb, ++it) {
+        if (__any_sync(0xffffffffu, *s_abort)) { ok = false; break; }
+        const int s = it % S;
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (it / S) & 1))) {
+          if (lane == 0) fail();
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint8_t* sa = smem + s * C::kStage;
+        uint8_t* sb = sa + kABytes;
+        if constexpr (GROUP_K) {
+          if (kb == ti.nkb - 1 && ti.klast < BK) {
+            // Rows [klast, 64) of every 64-row box hold the next expert's tokens: zero them.
+            const int nz = (BK - ti.klast) * 8;  // 16-byte pieces per box
+            constexpr int kBoxes = 2 + BN / 64;
+            for (int i = lane; i < nz * kBoxes; i += 32) {
+              const int box = i / nz, rem = i - box * nz;
+              uint8_t* base = box < 2 ? sa + box * 8192 : sb + (box - 2) * 8192;
+              *reinterpret_cast<uint4*>(base + (ti.klast + rem / 8) * 128 + (rem & 7) * 16) =
+                  make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+          }
+        }
+        __syncwarp();
+        if (lane == 0) {
+          const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sb);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = A_MN ? sdesc(a0 + k * 2048, 8192, 1024) : sdesc(a0 + k * 32, 16, 1024);
+            const uint64_t bd = B_MN ? sdesc(b0 + k * 2048, 8192, 1024) : sdesc(b0 + k * 32, 16, 1024);
+            umma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0);
+          }
+          umma_commit(&empty[s]);
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+      if (lane == 0) umma_commit(&tfull[acc]);
+      __syncwarp();
+      ++acc_it;
+    }
+    if (!ok && lane == 0) {  // wait for this thread's MMAs before TMEM is freed
+      umma_commit(drain);
+      (void)mbar_wait(drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    uint32_t acc_it = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      if (__any_sync(0xffffffffu, *s_abort)) break;
+      const TileInfo ti = decode_tile<BN, EPI, GROUP_K>(t, p, s_off, s_pre, nN);
+      const int acc = acc_it & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], (acc_it >> 1) & 1))) {
+        fail();
+        break;
+      }
+      tc_fence_after();
+      const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+      const bool valid = row < ti.rows;
+      auto release = [&]() {
+        tc_fence_before();
+        mbar_arrive(&tempty[acc]);
+      };
+      if constexpr (EPI == EPI_SWIGLU_FWD) {
+        __nv_bfloat16* arow = p.out + (int64_t)(ti.m0 + row) * p.ld_out;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t g[32], u[32];
+          tmem_ld32(ta + c * 32, g);
+          tmem_ld32(ta + 128 + c * 32, u);
+          tmem_wait_ld();
+          tmem_tie(g);
+          tmem_tie(u);
+          if (c == 3) release();
+          if (valid) {
+            uint32_t pa[16], pu[16], ph[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float a0 = __uint_as_float(g[2 * i]), a1 = __uint_as_float(g[2 * i + 1]);
+              const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+              pa[i] = pack_bf16(a0, a1);
+              pu[i] = pack_bf16(u0, u1);
+              ph[i] = pack_bf16(a0 * sigmoidf_(a0) * u0, a1 * sigmoidf_(a1) * u1);
+            }
+            const int col = ti.n0 + c * 32;
+            store_64B(arow + col, pa);
+            store_64B(arow + p.f + col, pu);
+            store_64B(arow + 2 * p.f + col, ph);
+          }
+        }
+      } else if constexpr (EPI == EPI_STORE) {
+        __nv_bfloat16* orow = p.out + (int64_t)(ti.m0 + row) * p.ld_out + ti.n0;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(ta + c * 32, v);
+          tmem_wait_ld();
+          tmem_tie(v);
+          if (c == BN / 32 - 1) release();
+          if (valid) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            store_64B(orow + c * 32, pk);
+          }
+        }
+      } else if constexpr (EPI == EPI_SWIGLU_BWD) {
+        const int64_t grow = ti.m0 + row;
+        const __nv_bfloat16* arow = p.act + grow * p.ld_act;
+        __nv_bfloat16* drow = p.out + grow * p.ld_out;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          const int col = ti.n0 + c * 32;
+          uint32_t av[16], uv[16];
+          if (valid) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint4 x = *reinterpret_cast<const uint4*>(arow + col + 8 * i);
+              const uint4 y = *reinterpret_cast<const uint4*>(arow + p.f + col + 8 * i);
+              av[4 * i] = x.x; av[4 * i + 1] = x.y; av[4 * i + 2] = x.z; av[4 * i + 3] = x.w;
+              uv[4 * i] = y.x; uv[4 * i + 1] = y.y; uv[4 * i + 2] = y.z; uv[4 * i + 3] = y.w;
+            }
+          }
+          uint32_t v[32];
+          tmem_ld32(ta + c * 32, v);
+          tmem_wait_ld();
+          tmem_tie(v);
+          if (c == BN / 32 - 1) release();
+          if (valid) {
+            uint32_t pda[16], pdu[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float da[2], du[2];
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const float dh = __uint_as_float(v[2 * i + h]);
+                const float a = h ? bf_hi(av[i]) : bf_lo(av[i]);
+                const float u = h ? bf_hi(uv[i]) : bf_lo(uv[i]);
+                const float s = sigmoidf_(a);
+                da[h] = dh * u * s * (1.f + a * (1.f - s));
+                du[h] = dh * a * s;
+              }
+              pda[i] = pack_bf16(da[0], da[1]);
+              pdu[i] = pack_bf16(du[0], du[1]);
+            }
+            store_64B(drow + col, pda);
+            store_64B(drow + p.f + col, pdu);
+          }
+        }
+      } else {  // EPI_WGRAD
+        const int64_t ooff = (int64_t)ti.g * p.out_group + (int64_t)(ti.m0 + row) * p.ld_out + ti.n0;
+        if (ti.nkb == 0) {
+          release();
+          if (p.out_f32) {
+            float4* o = reinterpret_cast<float4*>(p.out_f32 + ooff);
+            for (int i = 0; i < BN / 4; ++i) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+          } else {
+            uint4* o = reinterpret_cast<uint4*>(p.out + ooff);
+            for (int i = 0; i < BN / 8; ++i) o[i] = make_uint4(0, 0, 0, 0);
+          }
+        } else {
+#pragma unroll 1
+          for (int c = 0; c < BN / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(ta + c * 32, v);
+            tmem_wait_ld();
+            tmem_tie(v);
+            if (c == BN / 32 - 1) release();
+            if (p.out_f32) {
+              uint4* o = reinterpret_cast<uint4*>(p.out_f32 + ooff + c * 32);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) o[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            } else {
+              uint32_t pk[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+              store_64B(p.out + ooff + c * 32, pk);
+            }
+          }
+        }
+      }
+      ++acc_it;
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+cudaError_t get_encode() {
+  if (g_encode) return cudaSuccess;
+  cudaDriverEntryPointQueryResult q;
+  void* fn = nullptr;
+  cudaError_t err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+  if (err != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return cudaSuccess;
+}
+
+// 2-D bf16 tensor map over [outer, inner] with row stride `ld` elements.
+bool tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
+          uint32_t box_inner, uint32_t box_outer) {
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {ld * 2};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t es[2] = {1, 1};
+  return g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, bool A_MN, bool B_MN, int EPI, bool GROUP_K>
+cudaError_t launch(const GemmParams& p, int64_t tile_bound, cudaStream_t st) {
+  auto kern = grouped_gemm_sm100<BN, A_MN, B_MN, EPI, GROUP_K>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Cfg<BN>::kSmem);
+  if (err != cudaSuccess) return err;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tile_bound, num_sms()));
+  kern<<<grid, kThreads, Cfg<BN>::kSmem, st>>>(p);
+  return cudaGetLastError();
+}
+
+GemmParams base_params(const FfnShape& s, const int32_t* offsets, int* status) {
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.offsets = offsets;
+  p.E = s.E;
+  p.f = s.f;
+  p.status = status;
+  return p;
+}
+
+int64_t m_tile_bound(const FfnShape& s) { return s.rows / BM + s.E; }
+
+}  // namespace
+
+cudaError_t ffn_fwd_bf16(const FfnShape& s, const void* x_perm, const int32_t* offsets,
+                         const void* w1, const void* w2, void* act, void* y_perm, int* status,
+                         cudaStream_t st) {
+  if (s.rows == 0) return cudaSuccess;
+  cudaError_t err = get_encode();
+  if (err != cudaSuccess) return err;
+  const int d = s.d, f = s.f, E = s.E;
+  const __nv_bfloat16* actb = static_cast<const __nv_bfloat16*>(act);
+  // gate/up GEMM + SwiGLU: act = [a | u | h]
+  GemmParams p1 = base_params(s, offsets, status);
+  if (!tmap(&p1.tmA, x_perm, d, s.rows, d, 64, 128) ||
+      !tmap(&p1.tmB, w1, d, (uint64_t)E * 2 * f, d, 64, 128))
+    return cudaErrorInvalidValue;
+  p1.N = f; p1.K = d; p1.b_rows = 2 * f;
+  p1.out = static_cast<__nv_bfloat16*>(act); p1.ld_out = 3 * f;
+  if ((err = launch<256, false, false, EPI_SWIGLU_FWD, false>(p1, m_tile_bound(s) * (f / 128), st)) != cudaSuccess)
+    return err;
+  // down GEMM: y = h W2^T
+  GemmParams p2 = base_params(s, offsets, status);
+  if (!tmap(&p2.tmA, actb + 2 * f, f, s.rows, 3 * f, 64, 128) ||
+      !tmap(&p2.tmB, w2, f, (uint64_t)E * d, f, 64, 128))
+    return cudaErrorInvalidValue;
+  p2.N = d; p2.K = f; p2.b_rows = d;
+  p2.out = static_cast<__nv_bfloat16*>(y_perm); p2.ld_out = d;
+  return launch<256, false, false, EPI_STORE, false>(p2, m_tile_bound(s) * (d / 256), st);
+}
+
+cudaError_t ffn_bwd_bf16(const FfnShape& s, const void* dy_perm, const void* x_perm,
+                         const void* act, const int32_t* offsets, const void* w1, const void* w2,
+                         void* dx_perm, void* dw1, void* dw2, bool dw_f32, void* scratch,
+                         int* status, cudaStream_t st) {
+  cudaError_t err = get_encode();
+  if (err != cudaSuccess) return err;
+  const int d = s.d, f = s.f, E = s.E;
+  const __nv_bfloat16* actb = static_cast<const __nv_bfloat16*>(act);
+  __nv_bfloat16* dadu = static_cast<__nv_bfloat16*>(scratch);
+  const uint64_t rows_tm = std::max<int64_t>(s.rows, 1);  // tensor maps need a non-zero extent
+  if (s.rows > 0) {
+    // dgrad 1: dh = dy W2[e], fused SwiGLU backward -> dadu = [da | du]
+    GemmParams p3 = base_params(s, offsets, status);
+    if (!tmap(&p3.tmA, dy_perm, d, s.rows, d, 64, 128) ||
+        !tmap(&p3.tmB, w2, f, (uint64_t)E * d, f, 64, 64))
+      return cudaErrorInvalidValue;
+    p3.N = f; p3.K = d; p3.b_rows = d;
+    p3.out = dadu; p3.ld_out = 2 * f;
+    p3.act = actb; p3.ld_act = 3 * f;
+    if ((err = launch<256, false, true, EPI_SWIGLU_BWD, false>(p3, m_tile_bound(s) * (f / 256), st)) != cudaSuccess)
+      return err;
+    // dgrad 2: dx = [da | du] W1[e]
+    GemmParams p4 = base_params(s, offsets, status);
+    if (!tmap(&p4.tmA, dadu, 2 * f, s.rows, 2 * f, 64, 128) ||
+        !tmap(&p4.tmB, w1, d, (uint64_t)E * 2 * f, d, 64, 64))
+      return cudaErrorInvalidValue;
+    p4.N = d; p4.K = 2 * f; p4.b_rows = 2 * f;
+    p4.out = static_cast<__nv_bfloat16*>(dx_perm); p4.ld_out = d;
+    if ((err = launch<256, false, true, EPI_STORE, false>(p4, m_tile_bound(s) * (d / 256), st)) != cudaSuccess)
+      return err;
+  }
+  // wgrad 2: dW2[e] = dy^T h   (M = d, N = f, K = the expert's rows)
+  GemmParams p5 = base_params(s, offsets, status);
+  if (!tmap(&p5.tmA, dy_perm, d, rows_tm, d, 64, 64) ||
+      !tmap(&p5.tmB, actb + 2 * f, f, rows_tm, 3 * f, 64, 64))
+    return cudaErrorInvalidValue;
+  p5.M = d; p5.N = f;
+  p5.out = static_cast<__nv_bfloat16*>(dw2); p5.out_f32 = dw_f32 ? static_cast<float*>(dw2) : nullptr;
+  p5.ld_out = f; p5.out_group = (int64_t)d * f;
+  if ((err = launch<256, true, true, EPI_WGRAD, true>(p5, (int64_t)E * (d / 128) * (f / 256), st)) != cudaSuccess)
+    return err;
+  // wgrad 1: dW1[e] = [da | du]^T x   (M = 2f, N = d)
+  GemmParams p6 = base_params(s, offsets, status);
+  if (!tmap(&p6.tmA, dadu, 2 * f, rows_tm, 2 * f, 64, 64) ||
+      !tmap(&p6.tmB, x_perm, d, rows_tm, d, 64, 64))
+    return cudaErrorInvalidValue;
+  p6.M = 2 * f; p6.N = d;
+  p6.out = static_cast<__nv_bfloat16*>(dw1); p6.out_f32 = dw_f32 ? static_cast<float*>(dw1) : nullptr;
+  p6.ld_out = d; p6.out_group = (int64_t)2 * f * d;
+  return launch<256, true, true, EPI_WGRAD, true>(p6, (int64_t)E * (2 * f / 128) * (d / 256), st);
+}
+
+}  // namespace moe

@@ -1,0 +1,84 @@
+// internal.h -- host-side declarations shared by the library's .cu files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+namespace moe {
+
+inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
+
+// ---------------------------------------------------------------- routing
+struct RouteArgs {
+  const void* x;
+  const void* w_router;
+  const float* bias;
+  int T, d, E, k;
+  float* logits;
+  int32_t* topk_idx;
+  float* topk_gate;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* slot_row;
+  void* scratch;            // route_ws_bytes(T, E, k) bytes
+  // filled in by route_launch
+  int32_t* blockcounts = nullptr;
+  int32_t* localrank = nullptr;
+};
+size_t route_ws_bytes(int T, int E, int k);
+cudaError_t route_launch(const RouteArgs& a, bool bf16, cudaStream_t st);
+
+// ---------------------------------------------------------- row movement
+cudaError_t permute_launch(bool bf16, const void* x, const int32_t* slot_row, void* x_perm,
+                           int32_t* perm_src, int T, int d, int k, cudaStream_t st);
+cudaError_t combine_launch(bool bf16, const void* y_perm, const int32_t* slot_row,
+                           const float* gate, void* out, int T, int d, int k, cudaStream_t st);
+cudaError_t combine_bwd_launch(bool bf16, const void* dout, const void* y_perm,
+                               const int32_t* slot_row, const float* gate, void* dy_perm,
+                               float* dgate, int T, int d, int k, cudaStream_t st);
+cudaError_t padded_dispatch_launch(bool bf16, int capacity, const void* x, const int32_t* topk_idx,
+                                   const int32_t* slot_row, const int32_t* offsets, void* x_pad,
+                                   int32_t* pad_row, int32_t* offsets_pad, int T, int d, int E,
+                                   int k, cudaStream_t st);
+
+// ------------------------------------------------------------ router bwd
+size_t route_bwd_ws_bytes(int T, int d, int E);
+cudaError_t route_bwd_launch(bool bf16, const void* x, const void* w_router, const float* logits,
+                             const int32_t* topk_idx, const float* dgate, const void* dx_perm,
+                             const int32_t* slot_row, void* dx, float* dw_router, int T, int d,
+                             int E, int k, void* scratch, cudaStream_t st);
+
+// ----------------------------------------------------------------- MXFP8
+cudaError_t mxfp8_launch(int64_t rows, int64_t K, bool src_bf16, const void* src, int axis,
+                         const int32_t* seg_offsets, int nseg, uint8_t* q, uint8_t* scale,
+                         cudaStream_t st);
+
+// ---------------------------------------------------------- grouped FFN
+struct FfnShape {
+  int d, E, f;
+  int64_t rows;
+};
+size_t ffn_bwd_ws_bytes(const FfnShape& s, bool bf16);
+// fp32 path: CUDA-core grouped GEMMs
+cudaError_t ffn_fwd_f32(const FfnShape& s, const float* x_perm, const int32_t* offsets,
+                        const float* w1, const float* w2, float* act, float* y_perm,
+                        cudaStream_t st);
+cudaError_t ffn_bwd_f32(const FfnShape& s, const float* dy_perm, const float* x_perm,
+                        const float* act, const int32_t* offsets, const float* w1,
+                        const float* w2, float* dx_perm, float* dw1, float* dw2, void* scratch,
+                        cudaStream_t st);
+// bf16 path: tcgen05 tensor-core grouped GEMMs
+cudaError_t ffn_fwd_bf16(const FfnShape& s, const void* x_perm, const int32_t* offsets,
+                         const void* w1, const void* w2, void* act, void* y_perm, int* status,
+                         cudaStream_t st);
+cudaError_t ffn_bwd_bf16(const FfnShape& s, const void* dy_perm, const void* x_perm,
+                         const void* act, const int32_t* offsets, const void* w1, const void* w2,
+                         void* dx_perm, void* dw1, void* dw2, bool dw_f32, void* scratch,
+                         int* status, cudaStream_t st);
+
+int num_sms();
+
+}  // namespace moe

@@ -1,0 +1,284 @@
+// route.cu -- router logits, fused softmax/top-k, on-device histogram and
+// prefix scan of expert counts, and the slot row of every (token, slot) pair.
+//
+// Page: "Ai2 Olmo-core 3：MoE训练吞吐量提升2.7倍的秘诀" (kongchang.com), section
+// 路由不只是模型问题，更是系统问题 (routing is a systems problem): routing metadata
+// (split sizes, expert GEMM group sizes) stays on the GPU; section 容量税: each
+// token activates a few of the experts through a route function.
+//
+// Three launches, no host round trip:
+//   1. route_topk_kernel   -- per block of TB tokens: fp32 logits (CUDA-core dot
+//      products), softmax, top-k (warp argmax, lowest index wins ties), the
+//      block's per-expert counts and each pair's rank among the block's pairs
+//      of the same expert;
+//   2. block_scan_kernel    -- per expert: exclusive scan of the block counts in
+//      block order (gives each block's base inside the expert) and the total;
+//   3. slot_rows_kernel     -- offsets = exclusive scan of the totals;
+//      slot_row = offsets[e] + block base + rank within the block.
+// Rows inside an expert segment therefore follow token order, and every
+// integer is deterministic.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kRouteThreads = 256;
+constexpr int kDC = 32;  // d-chunk staged in shared memory
+
+// Tokens per block: keep the [TB, E] logit tile within 32 KB.
+__host__ __device__ inline int route_tb(int E) { return E <= 256 ? 32 : (E <= 512 ? 16 : 8); }
+
+// EC experts per pass of the dot-product phase.
+template <typename T, int TB, int EC>
+__global__ void __launch_bounds__(kRouteThreads)
+route_topk_kernel(const T* __restrict__ x, const T* __restrict__ w, const float* __restrict__ bias,
+                  int ntok, int d, int E, int k, float* __restrict__ logits,
+                  int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate,
+                  int32_t* __restrict__ blockcounts, int32_t* __restrict__ localrank, int nb) {
+  constexpr int kPer = TB * EC / kRouteThreads;  // outputs per thread
+  static_assert(kPer >= 1 && (TB * EC) % kRouteThreads == 0, "tile");
+  __shared__ float xs[TB][kDC + 1];
+  __shared__ float ws[EC][kDC + 1];
+  __shared__ int32_t sel[TB][32];
+  extern __shared__ float lg[];  // [TB][E]
+
+  const int tid = threadIdx.x;
+  const int t0 = blockIdx.x * TB;
+  const int col = tid % EC;
+  const int row0 = tid / EC;
+  constexpr int kRowStep = kRouteThreads / EC;
+
+  for (int e0 = 0; e0 < E; e0 += EC) {
+    float acc[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) acc[i] = 0.f;
+    for (int c0 = 0; c0 < d; c0 += kDC) {
+      for (int i = tid; i < TB * kDC; i += kRouteThreads) {
+        const int r = i / kDC, c = i % kDC;
+        const int t = t0 + r;
+        xs[r][c] = (t < ntok && c0 + c < d) ? to_f32(x[(int64_t)t * d + c0 + c]) : 0.f;
+      }
+      for (int i = tid; i < EC * kDC; i += kRouteThreads) {
+        const int r = i / kDC, c = i % kDC;
+        const int e = e0 + r;
+        ws[r][c] = (e < E && c0 + c < d) ? to_f32(w[(int64_t)e * d + c0 + c]) : 0.f;
+      }
+      __syncthreads();
+#pragma unroll 8
+      for (int c = 0; c < kDC; ++c) {
+        const float wv = ws[col][c];
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) acc[i] = fmaf(xs[row0 + i * kRowStep][c], wv, acc[i]);
+      }
+      __syncthreads();
+    }
+    const int e = e0 + col;
+    if (e < E) {
+      const float b = bias ? bias[e] : 0.f;
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) lg[(row0 + i * kRowStep) * E + e] = acc[i] + b;
+    }
+  }
+  __syncthreads();
+
+  // ---- softmax + top-k: one warp per token
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int r = warp; r < TB; r += kRouteThreads / 32) {
+    const int t = t0 + r;
+    if (t >= ntok) {
+      if (lane < k) sel[r][lane] = -1;
+      continue;
+    }
+    const float* row = lg + r * E;
+    float m = -INFINITY;
+    for (int e = lane; e < E; e += 32) m = fmaxf(m, row[e]);
+    m = warp_max(m);
+    float s = 0.f;
+    for (int e = lane; e < E; e += 32) {
+      s += expf(row[e] - m);
+      logits[(int64_t)t * E + e] = row[e];
+    }
+    s = warp_sum(s);
+    uint32_t taken = 0;  // bit i <-> expert lane + 32 i
+    for (int j = 0; j < k; ++j) {
+      float bv = 0.f;
+      int be = -1;
+      for (int i = 0, e = lane; e < E; ++i, e += 32) {
+        if (taken & (1u << i)) continue;
+        const float v = row[e];
+        if (be < 0 || v > bv) { bv = v; be = e; }  // ascending e: ties keep the lower index
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        if (oe >= 0 && (be < 0 || ov > bv || (ov == bv && oe < be))) { bv = ov; be = oe; }
+      }
+      if ((be & 31) == lane) taken |= 1u << (be >> 5);
+      if (lane == 0) {
+        topk_idx[(int64_t)t * k + j] = be;
+        topk_gate[(int64_t)t * k + j] = expf(bv - m) / s;
+        sel[r][j] = be;
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- per-block counts and ranks (token order inside the block)
+  for (int i = tid; i < TB * k; i += kRouteThreads) {
+    const int r = i / k, j = i % k;
+    const int t = t0 + r;
+    if (t >= ntok) continue;
+    const int e = sel[r][j];
+    int rank = 0;
+    for (int rr = 0; rr < r; ++rr)
+      for (int jj = 0; jj < k; ++jj) rank += (sel[rr][jj] == e);
+    localrank[(int64_t)t * k + j] = rank;
+  }
+  const int nvalid = min(TB, ntok - t0);
+  for (int e = tid; e < E; e += kRouteThreads) {
+    int c = 0;
+    for (int r = 0; r < nvalid; ++r)
+      for (int j = 0; j < k; ++j) c += (sel[r][j] == e);
+    blockcounts[(int64_t)e * nb + blockIdx.x] = c;
+  }
+}
+
+// Exclusive scan of blockcounts[e][0..nb) for expert e = blockIdx.x.
+__global__ void __launch_bounds__(256)
+block_scan_kernel(const int32_t* __restrict__ blockcounts, int32_t* __restrict__ blockoffs, int nb,
+                  int32_t* __restrict__ counts) {
+  __shared__ int32_t warp_tot[8];
+  __shared__ int32_t carry;
+  const int e = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int32_t* src = blockcounts + (int64_t)e * nb;
+  int32_t* dst = blockoffs + (int64_t)e * nb;
+  if (tid == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < nb; base += 256) {
+    const int i = base + tid;
+    const int v = i < nb ? src[i] : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int wbase = 0, total = 0;
+    for (int w2 = 0; w2 < 8; ++w2) {
+      if (w2 < warp) wbase += warp_tot[w2];
+      total += warp_tot[w2];
+    }
+    const int c = carry;
+    if (i < nb) dst[i] = c + wbase + incl - v;
+    __syncthreads();
+    if (tid == 0) carry = c + total;
+    __syncthreads();
+  }
+  if (tid == 0) counts[e] = carry;
+}
+
+// Exclusive scan of counts[0..E) into s_off[0..E] by one block (E <= 1024).
+__device__ void block_offsets(const int32_t* __restrict__ counts, int E, int32_t* s_off) {
+  __shared__ int32_t lane_tot[32];
+  const int tid = threadIdx.x;
+  if (tid < 32) {
+    const int lo = tid * 32, hi = min(lo + 32, E);
+    int s = 0;
+    for (int e = lo; e < hi; ++e) s += counts[e];
+    int incl = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (tid >= o) incl += n;
+    }
+    int run = incl - s;
+    for (int e = lo; e < hi; ++e) {
+      s_off[e] = run;
+      run += counts[e];
+    }
+    if (tid == 31) s_off[E] = incl;
+    lane_tot[tid] = incl;
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(256)
+slot_rows_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ localrank,
+                 const int32_t* __restrict__ blockoffs, const int32_t* __restrict__ counts,
+                 int ntok, int E, int k, int tb, int nb, int32_t* __restrict__ offsets,
+                 int32_t* __restrict__ slot_row) {
+  __shared__ int32_t s_off[1025];
+  block_offsets(counts, E, s_off);
+  if (blockIdx.x == 0)
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) offsets[e] = s_off[e];
+  const int64_t n = (int64_t)ntok * k;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int t = (int)(i / k);
+    const int e = topk_idx[i];
+    slot_row[i] = s_off[e] + blockoffs[(int64_t)e * nb + t / tb] + localrank[i];
+  }
+}
+
+template <typename T, int TB, int EC>
+cudaError_t launch_topk(const RouteArgs& a, int nb, cudaStream_t st) {
+  const size_t lg_bytes = sizeof(float) * TB * a.E;
+  auto kern = route_topk_kernel<T, TB, EC>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)lg_bytes);
+  if (err != cudaSuccess) return err;
+  kern<<<nb, kRouteThreads, lg_bytes, st>>>(
+      static_cast<const T*>(a.x), static_cast<const T*>(a.w_router), a.bias, a.T, a.d, a.E, a.k,
+      a.logits, a.topk_idx, a.topk_gate, a.blockcounts, a.localrank, nb);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t dispatch_topk(const RouteArgs& a, int nb, cudaStream_t st) {
+  const int tb = route_tb(a.E);
+  if (tb == 32) {
+    if (a.E <= 8) return launch_topk<T, 32, 8>(a, nb, st);
+    if (a.E <= 32) return launch_topk<T, 32, 32>(a, nb, st);
+    return launch_topk<T, 32, 64>(a, nb, st);
+  }
+  if (tb == 16) return launch_topk<T, 16, 64>(a, nb, st);
+  return launch_topk<T, 8, 64>(a, nb, st);
+}
+
+}  // namespace
+
+size_t route_ws_bytes(int T, int E, int k) {
+  const int tb = route_tb(E);
+  const size_t nb = (size_t)((T + tb - 1) / tb);
+  return align256(nb * E * 4) * 2 + align256((size_t)T * k * 4);
+}
+
+cudaError_t route_launch(const RouteArgs& a0, bool bf16, cudaStream_t st) {
+  RouteArgs a = a0;
+  const int tb = route_tb(a.E);
+  const int nb = (a.T + tb - 1) / tb;
+  uint8_t* ws = static_cast<uint8_t*>(a.scratch);
+  a.blockcounts = reinterpret_cast<int32_t*>(ws);
+  int32_t* blockoffs = reinterpret_cast<int32_t*>(ws + align256((size_t)nb * a.E * 4));
+  a.localrank = reinterpret_cast<int32_t*>(ws + 2 * align256((size_t)nb * a.E * 4));
+  cudaError_t err;
+  if (nb > 0) {
+    err = bf16 ? dispatch_topk<__nv_bfloat16>(a, nb, st) : dispatch_topk<float>(a, nb, st);
+    if (err != cudaSuccess) return err;
+  }
+  // With T == 0 the scan still writes zero counts and offsets.
+  block_scan_kernel<<<a.E, 256, 0, st>>>(a.blockcounts, blockoffs, nb, a.counts);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  const int64_t n = (int64_t)a.T * a.k;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 1184));
+  slot_rows_kernel<<<grid, 256, 0, st>>>(a.topk_idx, a.localrank, blockoffs, a.counts, a.T, a.E,
+                                          a.k, tb, nb, a.offsets, a.slot_row);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,112 @@
+"""Device buffers for one MoE FFN layer and the call sequence of its forward
+and backward pass through the C ABI.
+
+PyTorch only allocates device memory here; every step runs in the CUDA
+library (``capi``).  Forward: moe_route -> moe_permute -> moe_grouped_ffn_fwd
+-> moe_combine.  Backward: moe_combine_bwd -> moe_grouped_ffn_bwd ->
+moe_route_bwd.  With ``capacity`` set, the padded-capacity comparison layout
+is used instead (moe_padded_dispatch after the route, uniform E x capacity
+rows in the grouped FFN, dropped pairs marked -1).
+"""
+
+from __future__ import annotations
+
+import torch
+
+from . import capi
+
+_DT = {"f32": capi.MOE_F32, "bf16": capi.MOE_BF16}
+
+
+def capacity_for(rows: int, E: int, cf_num: int = 5, cf_den: int = 4) -> int:
+    """Uniform per-expert capacity ceil(cf * rows / E) for cf = cf_num / cf_den."""
+    return -((-cf_num * rows) // (cf_den * E))
+
+
+class MoELayer:
+    def __init__(self, T: int, d_model: int, E: int, top_k: int, d_ff: int, dtype: str = "bf16",
+                 device="cuda", dw_dtype: str | None = None, capacity: int | None = None):
+        if dtype not in _DT:
+            raise ValueError(f"dtype {dtype!r} is not supported by the layer path")
+        self.T, self.d, self.E, self.k, self.f = T, d_model, E, top_k, d_ff
+        self.dtype = dtype
+        self.cdtype = _DT[dtype]
+        self.dw_dtype = dw_dtype or "f32"
+        self.capacity = capacity
+        self.shape = capi.shape_of(T, d_model, E, top_k, d_ff)
+        self.R = T * top_k
+        self.rows = E * capacity if capacity else self.R
+        tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+        wdt = torch.float32 if self.dw_dtype == "f32" else torch.bfloat16
+        dev = torch.device(device)
+        i32 = dict(dtype=torch.int32, device=dev)
+        f32 = dict(dtype=torch.float32, device=dev)
+        act = dict(dtype=tdt, device=dev)
+        rows = max(self.rows, 1)
+        self.logits = torch.empty(T, E, **f32)
+        self.topk_idx = torch.empty(T, top_k, **i32)
+        self.topk_gate = torch.empty(T, top_k, **f32)
+        self.counts = torch.empty(E, **i32)
+        self.offsets = torch.empty(E + 1, **i32)
+        self.slot_row = torch.empty(T, top_k, **i32)
+        self.perm_src = torch.empty(max(self.R, 1), **i32)
+        self.x_perm = torch.empty(rows, d_model, **act)
+        self.act = torch.empty(rows, 3 * d_ff, **act)
+        self.y_perm = torch.empty(rows, d_model, **act)
+        self.out = torch.empty(T, d_model, **act)
+        self.dgate = torch.empty(T, top_k, **f32)
+        self.dy_perm = torch.zeros(rows, d_model, **act)
+        self.dx_perm = torch.empty(rows, d_model, **act)
+        self.dw1 = torch.empty(E, 2 * d_ff, d_model, dtype=wdt, device=dev)
+        self.dw2 = torch.empty(E, d_model, d_ff, dtype=wdt, device=dev)
+        self.dx = torch.empty(T, d_model, **act)
+        self.dw_router = torch.empty(E, d_model, **f32)
+        if capacity:
+            self.pad_row = torch.empty(T, top_k, **i32)
+            self.offsets_pad = torch.empty(E + 1, **i32)
+        nbytes = capi.moe_workspace_size(self.shape, self.cdtype, self.rows)
+        if nbytes == 0:
+            raise ValueError("invalid MoE shape")
+        self.ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+
+    # the row map and offsets that the grouped FFN and combine steps use
+    @property
+    def row_map(self):
+        return self.pad_row if self.capacity else self.slot_row
+
+    @property
+    def ffn_offsets(self):
+        return self.offsets_pad if self.capacity else self.offsets
+
+    def forward(self, x, w_router, bias, w1, w2, stream=None):
+        s, dt = self.shape, self.cdtype
+        capi.moe_route(s, dt, x, w_router, bias, self.logits, self.topk_idx, self.topk_gate,
+                       self.counts, self.offsets, self.slot_row, self.ws, stream)
+        if self.capacity:
+            capi.moe_padded_dispatch(s, dt, self.capacity, x, self.topk_idx, self.slot_row,
+                                     self.offsets, self.x_perm, self.pad_row, self.offsets_pad,
+                                     stream)
+        else:
+            capi.moe_permute(s, dt, x, self.slot_row, self.x_perm, self.perm_src, stream)
+        capi.moe_grouped_ffn_fwd(s, dt, self.rows, self.x_perm, self.ffn_offsets, w1, w2,
+                                 self.act, self.y_perm, self.ws, stream=stream)
+        capi.moe_combine(s, dt, self.y_perm, self.row_map, self.topk_gate, self.out, stream)
+        return self.out
+
+    def backward(self, dout, x, w_router, w1, w2, stream=None):
+        s, dt = self.shape, self.cdtype
+        capi.moe_combine_bwd(s, dt, dout, self.y_perm, self.row_map, self.topk_gate,
+                             self.dy_perm, self.dgate, stream)
+        capi.moe_grouped_ffn_bwd(s, dt, self.rows, self.dy_perm, self.x_perm, self.act,
+                                 self.ffn_offsets, w1, w2, self.dx_perm, self.dw1, self.dw2,
+                                 _DT[self.dw_dtype], self.ws, stream=stream)
+        capi.moe_route_bwd(s, dt, x, w_router, self.logits, self.topk_idx, self.dgate,
+                           self.dx_perm, self.row_map, self.dx, self.dw_router, self.ws, stream)
+        return self.dx
+
+    def step(self, x, w_router, bias, w1, w2, dout, stream=None):
+        self.forward(x, w_router, bias, w1, w2, stream)
+        return self.backward(dout, x, w_router, w1, w2, stream)
+
+    def device_status(self, stream=None) -> int:
+        return capi.moe_get_device_status(self.ws, stream)

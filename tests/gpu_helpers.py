@@ -1,0 +1,52 @@
+"""Helpers shared by the GPU parity tests (run the CUDA path; compare to the oracle)."""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from mixture_experts_layer_offsets_b200 import inputs
+from mixture_experts_layer_offsets_b200.layer import MoELayer
+from oracle import moe_ref as ref
+
+# Tolerances on relative Frobenius error, by compute dtype.
+TOL = {"f32": 1e-5, "bf16": 1e-2}
+
+
+def f64(t) -> np.ndarray:
+    if t is None:
+        return None
+    return t.detach().to(torch.float64).cpu().numpy()
+
+
+def i64(t) -> np.ndarray:
+    return t.detach().to(torch.int64).cpu().numpy()
+
+
+def rel(a, b) -> float:
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    nb = np.linalg.norm(b)
+    return float(np.linalg.norm(a - b) / (nb if nb > 0 else 1.0))
+
+
+def run_layer(cfg, seed=0, capacity=None, dw_dtype="f32"):
+    """Seeded inputs drawn on the CPU, copied to the GPU, one fwd+bwd step."""
+    cpu = inputs.make_inputs(cfg, device="cpu", seed=seed)
+    dev = {k: (v.cuda() if v is not None else None) for k, v in cpu.items()}
+    L = MoELayer(cfg.T, cfg.d_model, cfg.E, cfg.top_k, cfg.d_ff, cfg.dtype, "cuda",
+                 dw_dtype=dw_dtype, capacity=capacity)
+    L.step(dev["x"], dev["w_router"], dev["bias"], dev["w1"], dev["w2"], dev["dout"])
+    torch.cuda.synchronize()
+    assert L.device_status() == 0
+    return cpu, L
+
+
+def oracle_for(cpu, L, capacity=None):
+    """Oracle pass on the same inputs; discrete routing taken on the device's logits."""
+    args = (f64(cpu["x"]), f64(cpu["w_router"]), f64(cpu["w1"]), f64(cpu["w2"]), f64(cpu["dout"]),
+            L.k)
+    bias = f64(cpu["bias"]) if cpu["bias"] is not None else None
+    if capacity:
+        return ref.padded_layer_fwd_bwd(*args, capacity, bias, select_logits=f64(L.logits))
+    return ref.layer_fwd_bwd(*args, bias, select_logits=f64(L.logits))

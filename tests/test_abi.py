@@ -1,0 +1,134 @@
+"""The C-ABI library loads, exports every entry point that include/moe.h
+declares, and rejects bad arguments on the host before touching the GPU.
+
+No compute call runs here (there may be no GPU): every call below is
+rejected by host-side validation, which the library performs before any CUDA
+call.
+"""
+
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+from mixture_experts_layer_offsets_b200 import capi
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(capi.LIB_PATH):
+        from mixture_experts_layer_offsets_b200 import build
+        build.build()
+    return capi.lib()
+
+
+def test_exports_every_header_symbol(lib):
+    declared = capi.header_symbols()
+    assert {"moe_route", "moe_permute", "moe_grouped_ffn_fwd", "moe_grouped_ffn_bwd",
+            "moe_combine", "mxfp8_quantize"} <= set(declared)
+    out = subprocess.run(["nm", "-D", "--defined-only", capi.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    missing = [s for s in declared if s not in exported]
+    assert not missing, missing
+    for s in declared:
+        assert hasattr(lib, s)
+
+
+def test_version_string(lib):
+    assert "sm_100a" in capi.moe_version()
+
+
+def test_library_is_built_for_sm100a(lib):
+    out = subprocess.run(["strings", capi.LIB_PATH], capture_output=True, text=True).stdout
+    assert "sm_100a" in out
+
+
+SHAPE = dict(T=64, d_model=256, E=8, top_k=2, d_ff=256)
+
+
+def _shape(**kw):
+    s = dict(SHAPE)
+    s.update(kw)
+    return capi.moe_shape(**s)
+
+
+@pytest.mark.parametrize("bad", [dict(top_k=9), dict(top_k=0), dict(E=0), dict(E=2048, top_k=2),
+                                 dict(d_model=260), dict(d_ff=12), dict(T=-1), dict(top_k=33, E=64),
+                                 dict(T=1 << 30, top_k=4)])
+def test_workspace_size_rejects_bad_shapes(lib, bad):
+    assert capi.moe_workspace_size(_shape(**bad), capi.MOE_BF16, 0) == 0
+
+
+def test_workspace_size_grows_with_rows(lib):
+    s = _shape()
+    a = capi.moe_workspace_size(s, capi.MOE_BF16, 0)
+    b = capi.moe_workspace_size(s, capi.MOE_BF16, 64 * 2 * 4)
+    assert 256 < a < b
+
+
+FAKE = 1 << 20  # an aligned non-null address that is never dereferenced
+
+
+def _route(lib, shape, dtype=capi.MOE_BF16, x=FAKE, w=FAKE, bias=None, ptr=FAKE, ws=FAKE,
+           ws_bytes=1 << 30):
+    return lib.moe_route(shape, dtype, x, w, bias, ptr, ptr, ptr, ptr, ptr, ptr, ws, ws_bytes, None)
+
+
+def test_route_validation(lib):
+    ok = _shape()
+    assert _route(lib, _shape(top_k=9)) == capi.MOE_ERR_INVALID_ARG
+    assert _route(lib, ok, x=None) == capi.MOE_ERR_INVALID_ARG
+    assert _route(lib, ok, x=FAKE + 4) == capi.MOE_ERR_INVALID_ARG   # misaligned
+    assert _route(lib, ok, ws_bytes=16) == capi.MOE_ERR_INVALID_ARG
+    assert _route(lib, ok, dtype=7) == capi.MOE_ERR_INVALID_ARG
+    assert _route(lib, ok, dtype=capi.MOE_MXFP8) == capi.MOE_ERR_UNSUPPORTED
+    assert _route(lib, ok, bias=FAKE + 8) == capi.MOE_ERR_INVALID_ARG
+
+
+def test_ffn_validation(lib):
+    s = _shape()
+    f = lib.moe_grouped_ffn_fwd
+    assert f(s, capi.MOE_BF16, 128, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) \
+        == capi.MOE_ERR_UNSUPPORTED  # MXFP8 operands are not part of this version
+    assert f(s, capi.MOE_MXFP8, 128, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, 1 << 30, None) \
+        == capi.MOE_ERR_UNSUPPORTED
+    assert f(s, capi.MOE_BF16, -1, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, 1 << 30, None) \
+        == capi.MOE_ERR_INVALID_ARG
+    assert f(_shape(d_model=136), capi.MOE_BF16, 128, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE,
+             FAKE, 1 << 30, None) == capi.MOE_ERR_UNSUPPORTED  # tensor-core tiles need d % 256
+    b = lib.moe_grouped_ffn_bwd
+    args = [FAKE] * 6
+    assert b(s, capi.MOE_BF16, 128, *args, None, FAKE, FAKE, FAKE, 9, FAKE, 1 << 30, None) \
+        == capi.MOE_ERR_INVALID_ARG  # bad dw dtype
+    assert b(s, capi.MOE_F32, 128, *args, None, FAKE, FAKE, FAKE, capi.MOE_BF16, FAKE, 1 << 30,
+             None) == capi.MOE_ERR_INVALID_ARG
+    assert b(s, capi.MOE_BF16, 128, *args, None, FAKE, FAKE, FAKE, capi.MOE_F32, FAKE, 300, None) \
+        == capi.MOE_ERR_INVALID_ARG  # workspace too small
+
+
+def test_row_ops_validation(lib):
+    s = _shape()
+    assert lib.moe_permute(s, capi.MOE_BF16, FAKE, None, FAKE, FAKE, None) == capi.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine(s, capi.MOE_BF16, FAKE, FAKE, FAKE + 2, FAKE, None) == capi.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine_bwd(_shape(top_k=40, E=64), capi.MOE_BF16, *([FAKE] * 6), None) \
+        == capi.MOE_ERR_INVALID_ARG
+    assert lib.moe_padded_dispatch(s, capi.MOE_BF16, 0, *([FAKE] * 7), None) == capi.MOE_ERR_INVALID_ARG
+    assert lib.moe_route_bwd(s, capi.MOE_BF16, *([FAKE] * 9), FAKE, 16, None) == capi.MOE_ERR_INVALID_ARG
+    # T == 0 is a valid no-op for the row movers
+    assert lib.moe_permute(_shape(T=0), capi.MOE_BF16, None, None, None, None, None) == capi.MOE_OK
+
+
+def test_mxfp8_validation(lib):
+    q = lib.mxfp8_quantize
+    assert q(4, 48, capi.MOE_BF16, FAKE, 0, None, 0, FAKE, FAKE, None) == capi.MOE_ERR_INVALID_ARG
+    assert q(4, 64, capi.MOE_BF16, FAKE, 2, None, 0, FAKE, FAKE, None) == capi.MOE_ERR_INVALID_ARG
+    assert q(4, 64, 5, FAKE, 0, None, 0, FAKE, FAKE, None) == capi.MOE_ERR_INVALID_ARG
+    assert q(4, 24, capi.MOE_F32, FAKE, 1, None, 0, FAKE, FAKE, None) == capi.MOE_ERR_INVALID_ARG
+    assert q(4, 64, capi.MOE_F32, FAKE, 1, FAKE, 0, FAKE, FAKE, None) == capi.MOE_ERR_INVALID_ARG
+    assert q(0, 64, capi.MOE_F32, None, 0, None, 0, None, None, None) == capi.MOE_OK
+
+
+def test_status_query_validation(lib):
+    assert lib.moe_get_device_status(None, None, ctypes.byref(ctypes.c_int32())) == capi.MOE_ERR_INVALID_ARG

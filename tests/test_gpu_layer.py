@@ -1,0 +1,115 @@
+"""GPU parity of the whole layer (route -> permute -> grouped SwiGLU FFN ->
+combine, and the backward of each) against the float64 oracle.
+
+Sizes are small enough for the oracle to finish in seconds but span several
+128-row tiles per expert with ragged tails, empty experts, top_k = E, a
+single token, and the padded-capacity layout.  Integer outputs (indices,
+counts, offsets, rows, permutation, permuted rows) must be bit-exact; values
+must meet the relative Frobenius tolerance of their dtype.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import TOL, f64, i64, oracle_for, rel, run_layer
+from mixture_experts_layer_offsets_b200.inputs import CONFIGS, shrink
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    # the fp32 workload exactly as specified
+    "tiny_f32": CONFIGS["tiny_f32"],
+    # bf16, random routing; ~350 rows per expert -> 3 M tiles, ragged tail
+    "bf16_e8_small": shrink(CONFIGS["bf16_e8"], name="bf16_e8_small", T=700, d_model=512, d_ff=256),
+    # bf16, skewed routing with a logit bias: heavy-tailed counts, empty experts
+    "bf16_skew_small": shrink(CONFIGS["bf16_skew_e128"], name="bf16_skew_small", T=600,
+                              d_model=256, E=32, top_k=2, d_ff=256, router_std=1 / 16.0),
+    # top_k = E: every expert sees every token (dense mixture)
+    "bf16_dense": shrink(CONFIGS["bf16_e8"], name="bf16_dense", T=300, d_model=256, E=4, top_k=4,
+                         d_ff=256, router_std=0.05),
+    # a single token; fp32
+    "f32_one_token": shrink(CONFIGS["tiny_f32"], name="f32_one_token", T=1, d_model=16, E=4,
+                            top_k=3, d_ff=8),
+    # fp32 with E = 128 (mostly empty experts)
+    "f32_e128": shrink(CONFIGS["tiny_f32"], name="f32_e128", T=40, d_model=64, E=128, top_k=4,
+                       d_ff=32, router_std=0.125),
+}
+
+
+def _check_routing(L, o):
+    assert np.array_equal(i64(L.topk_idx), o["idx"])
+    assert np.array_equal(i64(L.counts), o["counts"])
+    assert np.array_equal(i64(L.offsets), o["offsets"])
+    assert np.array_equal(i64(L.slot_row), o["slot_row"])
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_layer_matches_oracle(name):
+    cfg = CASES[name]
+    tol = TOL[cfg.dtype]
+    cpu, L = run_layer(cfg)
+    o = oracle_for(cpu, L)
+    _check_routing(L, o)
+    R = cfg.R
+    assert np.array_equal(i64(L.perm_src[:R]), o["perm_src"])
+    # the permuted rows are exact copies
+    assert torch.equal(L.x_perm[:R].cpu(), cpu["x"][L.perm_src[:R].long().cpu()])
+    assert rel(f64(L.logits), o["logits"]) <= tol
+    assert rel(f64(L.topk_gate), o["gate"]) <= tol
+    f = cfg.d_ff
+    act = f64(L.act[:R])
+    checks = {
+        "a": (act[:, :f], o["a"]), "u": (act[:, f:2 * f], o["u"]), "h": (act[:, 2 * f:], o["h"]),
+        "y_perm": (f64(L.y_perm[:R]), o["y_perm"]), "out": (f64(L.out), o["out"]),
+        "dgate": (f64(L.dgate), o["dgate"]), "dy_perm": (f64(L.dy_perm[:R]), o["dy_perm"]),
+        "dx_perm": (f64(L.dx_perm[:R]), o["dx_perm"]), "dw1": (f64(L.dw1), o["dw1"]),
+        "dw2": (f64(L.dw2), o["dw2"]), "dx": (f64(L.dx), o["dx"]),
+        "dw_router": (f64(L.dw_router), o["dw_router"]),
+    }
+    errs = {k: rel(a, b) for k, (a, b) in checks.items()}
+    bad = {k: v for k, v in errs.items() if not v <= tol}
+    assert not bad, (name, errs)
+    # empty experts get exactly zero weight gradients
+    for e in np.nonzero(o["counts"] == 0)[0]:
+        assert not L.dw1[e].any() and not L.dw2[e].any()
+
+
+def test_bf16_weight_grads_in_bf16():
+    cfg = CASES["bf16_e8_small"]
+    cpu, L = run_layer(cfg, dw_dtype="bf16")
+    o = oracle_for(cpu, L)
+    assert L.dw1.dtype == torch.bfloat16
+    assert rel(f64(L.dw1), o["dw1"]) <= TOL["bf16"]
+    assert rel(f64(L.dw2), o["dw2"]) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("name,cap", [("bf16_skew_small", 40), ("tiny_f32", 80), ("bf16_e8_small", 400)])
+def test_padded_capacity_matches_oracle(name, cap):
+    cfg = CASES[name]
+    tol = TOL[cfg.dtype]
+    cpu, L = run_layer(cfg, capacity=cap)
+    o = oracle_for(cpu, L, capacity=cap)
+    _check_routing(L, o)
+    assert np.array_equal(i64(L.pad_row), o["pad_row"])
+    assert np.array_equal(i64(L.offsets_pad), np.arange(cfg.E + 1) * cap)
+    # kept rows are exact copies, unused rows are zero
+    xp = L.x_perm.cpu()
+    pr = o["pad_row"]
+    for j in range(cfg.top_k):
+        keep = pr[:, j] >= 0
+        assert torch.equal(xp[torch.from_numpy(pr[keep, j])], cpu["x"][torch.from_numpy(np.nonzero(keep)[0])])
+    used = np.zeros(cfg.E * cap, dtype=bool)
+    used[pr[pr >= 0]] = True
+    assert not xp[torch.from_numpy(~used)].any()
+    for key, dev in (("out", L.out), ("dgate", L.dgate), ("dx", L.dx), ("dw1", L.dw1),
+                     ("dw2", L.dw2), ("dw_router", L.dw_router)):
+        assert rel(f64(dev), o[key]) <= tol, key
+
+
+def test_routing_is_deterministic_across_runs():
+    cfg = CASES["bf16_skew_small"]
+    _, a = run_layer(cfg)
+    _, b = run_layer(cfg)
+    for name in ("logits", "topk_idx", "topk_gate", "slot_row", "out", "dx", "dw1", "dw_router"):
+        assert torch.equal(getattr(a, name), getattr(b, name)), name
