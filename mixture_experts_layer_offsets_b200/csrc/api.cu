@@ -97,7 +97,7 @@ moe_status moe_route(moe_shape s, int dtype, const void* x, const void* w_router
   if (!ptrs_ok(w_router, counts, offsets, ws)) return MOE_ERR_INVALID_ARG;
   if (s.T > 0 && !ptrs_ok(x, logits, topk_idx, topk_gate, slot_row)) return MOE_ERR_INVALID_ARG;
   if (bias && !aligned16(bias)) return MOE_ERR_INVALID_ARG;
-  if (ws_bytes < ws_need(s, dtype, 0)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < kStatusBytes + route_ws_bytes(s.T, s.E, s.top_k)) return MOE_ERR_INVALID_ARG;
   RouteArgs a{x, w_router, bias, s.T, s.d_model, s.E, s.top_k, logits, topk_idx, topk_gate,
               counts, offsets, slot_row, scratch(ws)};
   return cuda_status(route_launch(a, dtype == MOE_BF16, as_stream(stream)));
