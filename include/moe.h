@@ -111,6 +111,37 @@ moe_status moe_route(moe_shape shape, int dtype, const void* x, const void* w_ro
                      int32_t* counts, int32_t* offsets, int32_t* slot_row, void* ws,
                      size_t ws_bytes, void* stream);
 
+/* ---- moe_route without a caller workspace --------------------------------
+ * The pages have no counterpart for this call.  It exists for callers that
+ * cannot allocate device memory: for example a plugin hosted by a framework
+ * that owns all device memory and offers no allocation hook, code on a
+ * latency-critical path where cudaMalloc/cudaFree could synchronise the
+ * device and stall queued work, or a deployment whose device-memory footprint
+ * is fixed at start-up.  It computes exactly what moe_route computes, from the
+ * same arguments minus the workspace.
+ *   Scratch: the per-block expert counts, their scan and the in-block ranks
+ *   live in one fixed array inside this library, MOE_ROUTE_NOALLOC_MAX_SCRATCH
+ *   bytes of device memory that every GPU loading the library holds until the
+ *   process exits.  The call allocates nothing (no cudaMalloc, no cudaFree, no
+ *   allocating library routine).
+ *   Limit: the shape needs 2*r(4*E*nb) + r(4*T*top_k) bytes of scratch, where
+ *   r() rounds up to a multiple of 256, nb = ceil(T / tb) and tb = 32 for
+ *   E <= 256, 16 for E <= 512, else 8; above MOE_ROUTE_NOALLOC_MAX_SCRATCH the
+ *   call returns MOE_ERR_UNSUPPORTED and runs nothing (use moe_route then).
+ *   First call on a device: it looks up the array's device address with that
+ *   device current (a one-time set-up per device); make that first call
+ *   before any stream capture.
+ *   Sharing: all calls on a device use the same array, which keeps whatever
+ *   the last call left in it; nothing in it has to start at zero because each
+ *   call writes every scratch byte before reading it.  Calls whose kernels can
+ *   overlap on the GPU (different streams without ordering between them) race
+ *   on the array and produce wrong results: order them on one stream. */
+#define MOE_ROUTE_NOALLOC_MAX_SCRATCH (4u << 20)
+moe_status moe_route_noalloc(moe_shape shape, int dtype, const void* x, const void* w_router,
+                             const float* bias, float* logits, int32_t* topk_idx,
+                             float* topk_gate, int32_t* counts, int32_t* offsets,
+                             int32_t* slot_row, void* stream);
+
 /* ---- a3: rowwise permute -------------------------------------------------
  * [bytechap] how it works: rowwise dispatch places routed rows directly in
  * the experts' input buffers.

@@ -42,6 +42,7 @@ _SIGS = {
     "moe_workspace_size": (_SZ, [moe_shape, _I, _I64]),
     "moe_get_device_status": (_I, [_P, _P, _P]),
     "moe_route": (_I, [moe_shape, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "moe_route_noalloc": (_I, [moe_shape, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_permute": (_I, [moe_shape, _I, _P, _P, _P, _P, _P]),
     "moe_grouped_ffn_fwd": (_I, [moe_shape, _I, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "moe_combine": (_I, [moe_shape, _I, _P, _P, _P, _P, _P]),
@@ -123,6 +124,15 @@ def moe_route(shape, dtype, x, w_router, bias, logits, topk_idx, topk_gate, coun
         shape, dtype, _ptr(x), _ptr(w_router), _ptr(bias), _ptr(logits), _ptr(topk_idx),
         _ptr(topk_gate), _ptr(counts), _ptr(offsets), _ptr(slot_row), _ptr(ws),
         ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_route_noalloc(shape, dtype, x, w_router, bias, logits, topk_idx, topk_gate, counts,
+                      offsets, slot_row, stream=None) -> None:
+    """moe_route without a workspace: for callers that cannot allocate device
+    memory; its scratch is a fixed array inside the library (see include/moe.h)."""
+    _check("moe_route_noalloc", lib().moe_route_noalloc(
+        shape, dtype, _ptr(x), _ptr(w_router), _ptr(bias), _ptr(logits), _ptr(topk_idx),
+        _ptr(topk_gate), _ptr(counts), _ptr(offsets), _ptr(slot_row), _stream(stream)))
 
 
 def moe_permute(shape, dtype, x, slot_row, x_perm, perm_src, stream=None) -> None:

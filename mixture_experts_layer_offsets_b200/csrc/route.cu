@@ -282,3 +282,78 @@ cudaError_t route_launch(const RouteArgs& a0, bool bf16, cudaStream_t st) {
 }
 
 }  // namespace moe
+
+// ---------------------------------------------------------------------------
+// moe_route_noalloc: the same routing step for callers that cannot allocate
+// device memory (a plugin inside a framework that owns all device memory, a
+// latency-critical path where cudaMalloc could synchronise the device, a
+// deployment with a footprint fixed at start-up).  Its scratch is one fixed
+// array of this library instead of a caller workspace.
+#include <mutex>
+
+namespace moe {
+
+// Device scratch of moe_route_noalloc, shared by every call on a device.
+static __device__ __align__(256) uint8_t g_route_scratch[MOE_ROUTE_NOALLOC_MAX_SCRATCH];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// In host code g_route_scratch names a host-side stand-in, not device memory:
+// the kernels get the array's device address, looked up once per device with
+// that device current.
+cudaError_t noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    err = cudaGetSymbolAddress(&p, g_route_scratch);
+    if (err != cudaSuccess) return err;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+}  // namespace
+}  // namespace moe
+
+extern "C" moe_status moe_route_noalloc(moe_shape s, int dtype, const void* x,
+                                        const void* w_router, const float* bias, float* logits,
+                                        int32_t* topk_idx, float* topk_gate, int32_t* counts,
+                                        int32_t* offsets, int32_t* slot_row, void* stream) {
+  using namespace moe;
+  // the argument rules of moe_route
+  if (s.T < 0 || s.d_model <= 0 || s.E <= 0 || s.top_k <= 0 || s.d_ff <= 0) return MOE_ERR_INVALID_ARG;
+  if (s.E > 1024 || s.top_k > s.E || s.top_k > 32) return MOE_ERR_INVALID_ARG;
+  if (s.d_model % 8 || s.d_ff % 8) return MOE_ERR_INVALID_ARG;
+  if ((int64_t)s.T * s.top_k >= (int64_t)1 << 31) return MOE_ERR_INVALID_ARG;
+  if (dtype == MOE_MXFP8) return MOE_ERR_UNSUPPORTED;
+  if (dtype != MOE_F32 && dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  const void* always[] = {w_router, counts, offsets};
+  for (const void* p : always)
+    if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (s.T > 0) {
+    const void* per_token[] = {x, logits, topk_idx, topk_gate, slot_row};
+    for (const void* p : per_token)
+      if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  }
+  if (bias && !aligned16(bias)) return MOE_ERR_INVALID_ARG;
+  // the fixed scratch bounds the shapes this variant can take
+  if (route_ws_bytes(s.T, s.E, s.top_k) > MOE_ROUTE_NOALLOC_MAX_SCRATCH) return MOE_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  if (noalloc_scratch(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
+  RouteArgs a{x, w_router, bias, s.T, s.d_model, s.E, s.top_k, logits, topk_idx, topk_gate,
+              counts, offsets, slot_row, scratch};
+  return route_launch(a, dtype == MOE_BF16, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
