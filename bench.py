@@ -5,7 +5,8 @@ counts, offsets, slot rows) -> permute -> grouped SwiGLU FFN forward ->
 combine -> combine backward -> grouped FFN backward (dgrad + wgrad) ->
 unpermute-grad + router grad.  Inputs are seeded synthetic tensors already
 resident in HBM; L2 is flushed (256 MiB write) between timed steps, outside
-the timed events.
+the timed events.  The timed step is a CUDA-graph replay of the C-ABI calls;
+the per-phase breakdown comes from eager steps with events between calls.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--capacity-factor] [--impl {ours,reference}]
@@ -124,6 +125,8 @@ def run_ours(args, rank, world):
     from mixture_experts_layer_offsets_b200.layer import MoELayer, capacity_for
 
     cfg = inputs.CONFIGS[args.workload]
+    if args.tokens:
+        cfg = inputs.shrink(cfg, name=f"{cfg.name}@T{args.tokens}", T=args.tokens)
     if cfg.dtype not in ("f32", "bf16"):
         raise SystemExit(f"workload {cfg.name}: dtype {cfg.dtype} is not implemented")
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -172,7 +175,20 @@ def run_ours(args, rank, world):
     if L.device_status() != 0:
         raise SystemExit("device status reported a timeout during warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(args.steps)]
+    # The timed step is one CUDA-graph replay of the whole path (the library makes
+    # no host synchronisation and no allocation, so the step captures as is).
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    with torch.cuda.graph(graph):
+        step()
+    torch.cuda.synchronize()
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
     sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     if world > 1:
         torch.distributed.barrier()
@@ -182,23 +198,37 @@ def run_ours(args, rank, world):
         time.sleep(0.3)
     for i in range(args.steps):
         flush.zero_()
-        step(evs[i])
+        evs[i][0].record(stream)
+        graph.replay()
+        evs[i][1].record(stream)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     clocks = sampler.stop() if sampler else None
-    per_step = [e[0].elapsed_time(e[7]) for e in evs]
-    ph = {p: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, p in enumerate(phases)}
+    per_step = [a.elapsed_time(b) for a, b in evs]
     total_ms = sum(per_step)
     if world > 1:
         t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         total_ms = float(t.item())
     ms_per_step = total_ms / args.steps
+
+    # Phase breakdown: eager steps with CUDA events between the calls; a GPU-side
+    # delay before each step lets the host enqueue the whole step first, so the
+    # events see device time only.
+    nph = min(args.steps, 10)
+    pevs = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(nph)]
+    for i in range(nph):
+        flush.zero_()
+        torch.cuda._sleep(3_000_000)
+        step(pevs[i])
+    torch.cuda.synchronize()
+    ph = {p: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in pevs) for i, p in enumerate(phases)}
     status = L.device_status()
+    del graph
 
     # e2e: through the public API with host buffers, copies inside the timed region
-    e2e = run_e2e(args, L, inp, dev, flush, capacity, world)
+    e2e = None if args.no_e2e else run_e2e(args, L, inp, dev, flush, capacity, world)
 
     if rank != 0:
         return None
@@ -227,6 +257,8 @@ def run_ours(args, rank, world):
             "rows_computed": rows,
         },
         "phases_ms": {k: round(v, 4) for k, v in ph.items()},
+        "timing": "value: CUDA-graph replay of the step, CUDA events per step; phases_ms and "
+                  "roofline: eager steps with events between calls (host kept ahead of the GPU)",
         "gpu_launches": launches_per_step * args.steps,
         "device_status": status,
         "e2e": e2e,
@@ -354,6 +386,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override T (smaller cases for profiling); not a bench line")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -99,7 +99,7 @@ moe_status moe_route(moe_shape s, int dtype, const void* x, const void* w_router
   if (bias && !aligned16(bias)) return MOE_ERR_INVALID_ARG;
   if (ws_bytes < kStatusBytes + route_ws_bytes(s.T, s.E, s.top_k)) return MOE_ERR_INVALID_ARG;
   RouteArgs a{x, w_router, bias, s.T, s.d_model, s.E, s.top_k, logits, topk_idx, topk_gate,
-              counts, offsets, slot_row, scratch(ws)};
+              counts, offsets, slot_row, scratch(ws), status_word(ws)};
   return cuda_status(route_launch(a, dtype == MOE_BF16, as_stream(stream)));
 }
 
@@ -201,7 +201,7 @@ moe_status moe_route_bwd(moe_shape s, int dtype, const void* x, const void* w_ro
   if (ws_bytes < kStatusBytes + route_bwd_ws_bytes(s.T, s.d_model, s.E)) return MOE_ERR_INVALID_ARG;
   return cuda_status(route_bwd_launch(dtype == MOE_BF16, x, w_router, logits, topk_idx, dgate,
                                       dx_perm, slot_row, dx, dw_router, s.T, s.d_model, s.E,
-                                      s.top_k, scratch(ws), as_stream(stream)));
+                                      s.top_k, scratch(ws), status_word(ws), as_stream(stream)));
 }
 
 moe_status mxfp8_quantize(int64_t rows, int64_t K, int src_dtype, const void* src, int axis,

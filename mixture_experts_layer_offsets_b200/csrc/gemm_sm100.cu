@@ -8,11 +8,12 @@
 // uneven per-expert shapes produced by routing, packing the small GEMMs of all
 // experts into one kernel without padding; group sizes never go back to the host.
 //
-// Kernel structure (one CTA per SM, persistent; 6 warps):
+// Kernel structure (one CTA per SM, persistent; 10 warps):
 //   warp 0      TMA producer (one thread): A/B tiles -> S-stage smem ring
 //   warp 1      MMA issuer (one thread issues tcgen05.mma M=128 N=BN K=16;
 //               the warp zeroes ragged K tails of weight-gradient tiles)
-//   warps 2..5  epilogue: tcgen05.ld TMEM -> registers -> fused math -> global
+//   warps 2..9  epilogue, two warps per TMEM lane quarter, each on half of the
+//               columns: tcgen05.ld TMEM -> registers -> fused math -> global
 // TMEM holds two BN-column fp32 accumulators so the epilogue of one tile
 // overlaps the main loop of the next.
 //
@@ -49,14 +50,24 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
 constexpr uint32_t kABytes = BM * BK * 2;  // 16 KB
 
-enum : int { EPI_SWIGLU_FWD = 0, EPI_STORE = 1, EPI_SWIGLU_BWD = 2, EPI_WGRAD = 3 };
+enum : int {
+  EPI_SWIGLU_FWD = 0,  // gate|up accumulators -> a, u, h = silu(a) u
+  EPI_STORE = 1,       // bf16 store
+  EPI_SWIGLU_BWD = 2,  // dh -> da, du (loads a, u)
+  EPI_WGRAD = 3,       // per-group weight gradient, fp32 (TMA store) or bf16
+  EPI_ROUTER = 4,      // logits -> softmax, top-k, block counts and ranks
+  EPI_ROUTER_DX = 5    // dx = acc + sum_j dx_perm[slot_row[t, j]]
+};
+
+constexpr int kRouterKMax = 8;  // top-k kept in registers by the router epilogue
 
 struct GemmParams {
   CUtensorMap tmA;
   CUtensorMap tmB;
+  CUtensorMap tmOut;       // EPI_WGRAD fp32 output: boxes of 32 columns x 16 rows
   const int32_t* offsets;
   int E;
   int M;        // GROUP_K: output rows per expert
@@ -71,6 +82,20 @@ struct GemmParams {
   int64_t ld_act;
   int64_t out_group;       // EPI_WGRAD: elements per expert
   int* status;
+  // EPI_ROUTER (one group of rows_total tokens; N = number of experts)
+  int rows_total;
+  int topk;
+  int nb;                  // 128-token blocks
+  const float* bias;
+  float* logits;
+  int32_t* topk_idx;
+  float* topk_gate;
+  int32_t* blockcounts;    // [N][nb]
+  int32_t* localrank;      // [rows_total][topk]
+  // GROUP_K without offsets: groups are consecutive splits of `split` rows
+  int split;
+  // EPI_ROUTER_DX
+  const int32_t* slot_row; // [rows_total][topk]
 };
 
 template <int BN> struct Cfg {
@@ -78,7 +103,17 @@ template <int BN> struct Cfg {
   static constexpr uint32_t kStage = kABytes + kBBytes;
   static constexpr int kStages = (BN == 256) ? 4 : 6;
   static constexpr uint32_t kTmemCols = 2 * BN;
-  static constexpr size_t kSmem = 1024 + (size_t)kStages * kStage + 256 + 2 * 1025 * 4;
+  static constexpr int kBoxRows = BN < 128 ? BN : 128;  // rows of one K-major B box
+  // shared memory after the stage ring: barriers (256 B), offsets and tile prefix
+  // (2 x 1025 ints), router selections (128 x kRouterKMax ints), then a 1024-aligned
+  // staging area for TMA stores (8 epilogue warps x 16 rows x 128 B)
+  static constexpr size_t kOffMisc = (size_t)kStages * kStage;
+  static constexpr size_t kOffSoff = kOffMisc + 256;
+  static constexpr size_t kOffSel = kOffSoff + 2 * 1025 * 4;
+  static constexpr size_t kOffStore = (kOffSel + 128 * kRouterKMax * 4 + 1023) & ~size_t(1023);
+  static constexpr size_t kStoreBytes = 8 * 16 * 128;
+  static constexpr size_t kSmem = 1024 + kOffStore + kStoreBytes;
+  static_assert(kSmem <= 232448, "shared memory per CTA");
 };
 
 // ------------------------------------------------------------ PTX wrappers
@@ -132,6 +167,29 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : MOE_R8(0), MOE_R8(8), MOE_R8(16), MOE_R8(24)
       : "r"(taddr));
 }
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : MOE_R8(0), MOE_R8(8)
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_tie16(uint32_t (&r)[16]) {
+  asm volatile("" : MOE_T8(0), MOE_T8(8));
+}
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* tm, int x, int y, const void* smem_src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(tm)),
+               "r"(x), "r"(y), "r"(smem_u32(smem_src))
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void tma_store_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void tma_store_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -152,6 +210,17 @@ __device__ __forceinline__ void store_64B(void* dst, const uint32_t (&v)[16]) {
   for (int i = 0; i < 4; ++i) d[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
 }
 __device__ __forceinline__ float sigmoidf_(float a) { return 1.f / (1.f + __expf(-a)); }
+// 32 bf16 of a (at col) and of u (at f + col) from one row of the saved activations.
+__device__ __forceinline__ void load_au(const __nv_bfloat16* arow, int col, int f,
+                                        uint32_t (&av)[16], uint32_t (&uv)[16]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 x = *reinterpret_cast<const uint4*>(arow + col + 8 * i);
+    const uint4 y = *reinterpret_cast<const uint4*>(arow + f + col + 8 * i);
+    av[4 * i] = x.x; av[4 * i + 1] = x.y; av[4 * i + 2] = x.z; av[4 * i + 3] = x.w;
+    uv[4 * i] = y.x; uv[4 * i + 1] = y.y; uv[4 * i + 2] = y.z; uv[4 * i + 3] = y.w;
+  }
+}
 
 // ------------------------------------------------------------ tile decode
 struct TileInfo {
@@ -209,18 +278,26 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
   uint64_t* drain = tempty + 2;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
-  int* s_off = reinterpret_cast<int*>(smem + S * C::kStage + 256);
+  int* s_off = reinterpret_cast<int*>(smem + C::kOffSoff);
   int* s_pre = s_off + 1025;
+  int* s_sel = reinterpret_cast<int*>(smem + C::kOffSel);  // EPI_ROUTER: [128][kRouterKMax]
+  uint8_t* s_store = smem + C::kOffStore;                   // TMA-store staging
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = p.E;
-  const int nN = GROUP_K ? p.N / BN : (EPI == EPI_SWIGLU_FWD ? p.N / 128 : p.N / BN);
+  const int nN = GROUP_K ? p.N / BN
+                         : (EPI == EPI_SWIGLU_FWD ? p.N / 128 : (EPI == EPI_ROUTER ? 1 : p.N / BN));
 
-  for (int g = threadIdx.x; g <= E; g += kThreads) s_off[g] = p.offsets[g];
+  for (int g = threadIdx.x; g <= E; g += kThreads)
+    s_off[g] = p.offsets ? p.offsets[g]
+                         : (GROUP_K ? min(g * p.split, p.rows_total) : (g == 0 ? 0 : p.rows_total));
   if (warp == 0) {
     if (lane == 0) {
       for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-      for (int a = 0; a < 2; ++a) { mbar_init(&tfull[a], 1); mbar_init(&tempty[a], 128); }
+      for (int a = 0; a < 2; ++a) {
+        mbar_init(&tfull[a], 1);
+        mbar_init(&tempty[a], EPI == EPI_ROUTER ? 128 : kThreads - 64);
+      }
       mbar_init(drain, 1);
       *s_abort = 0;
       fence_mbar_init();
@@ -283,11 +360,12 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
             for (int i = 0; i < 2; ++i) tma_load_2d(sa + i * 8192, &p.tmA, ti.m0 + 64 * i, ti.kbase + kc, &full[s]);
           }
           if constexpr (!B_MN) {
+            constexpr int kBox = C::kBoxRows;
 #pragma unroll
-            for (int i = 0; i < BN / 128; ++i) {
+            for (int i = 0; i < BN / kBox; ++i) {
               const int row = ti.kbase + (EPI == EPI_SWIGLU_FWD ? (i == 0 ? ti.n0 : p.f + ti.n0)
-                                                               : ti.n0 + 128 * i);
-              tma_load_2d(sb + i * 16384, &p.tmB, kc, row, &full[s]);
+                                                               : ti.n0 + kBox * i);
+              tma_load_2d(sb + i * kBox * 128, &p.tmB, kc, row, &full[s]);
             }
           } else {
 #pragma unroll
@@ -367,35 +445,52 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // Eight warps: two per TMEM lane quarter (warp % 4), each taking half of
+    // the tile's 32-column chunks.
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row = q * 32 + lane;
+    constexpr int kChunks = (EPI == EPI_SWIGLU_FWD ? 128 : BN) / 32;
+    constexpr int kMine = kChunks / 2;
+    const int c0 = half * kMine;
     uint32_t acc_it = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+    // The router epilogue keeps a whole logit row per thread: warps 2..5 only.
+    const bool idle = EPI == EPI_ROUTER && half == 1;
+    for (int t = blockIdx.x; t < total && !idle; t += gridDim.x) {
       if (__any_sync(0xffffffffu, *s_abort)) break;
       const TileInfo ti = decode_tile<BN, EPI, GROUP_K>(t, p, s_off, s_pre, nN);
       const int acc = acc_it & 1;
+      const bool valid = row < ti.rows;
+      // SwiGLU backward: a and u of the first chunk do not depend on the
+      // accumulator, so their loads are in flight while the main loop runs.
+      uint32_t av[16], uv[16];
+      const __nv_bfloat16* arow = nullptr;
+      if constexpr (EPI == EPI_SWIGLU_BWD) {
+        arow = p.act + (int64_t)(ti.m0 + row) * p.ld_act;
+        if (valid) load_au(arow, ti.n0 + c0 * 32, p.f, av, uv);
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], (acc_it >> 1) & 1))) {
         fail();
         break;
       }
       tc_fence_after();
       const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
-      const bool valid = row < ti.rows;
       auto release = [&]() {
         tc_fence_before();
         mbar_arrive(&tempty[acc]);
       };
       if constexpr (EPI == EPI_SWIGLU_FWD) {
-        __nv_bfloat16* arow = p.out + (int64_t)(ti.m0 + row) * p.ld_out;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        __nv_bfloat16* arow_out = p.out + (int64_t)(ti.m0 + row) * p.ld_out;
+#pragma unroll
+        for (int ci = 0; ci < kMine; ++ci) {
+          const int c = c0 + ci;
           uint32_t g[32], u[32];
           tmem_ld32(ta + c * 32, g);
           tmem_ld32(ta + 128 + c * 32, u);
           tmem_wait_ld();
           tmem_tie(g);
           tmem_tie(u);
-          if (c == 3) release();
+          if (ci == kMine - 1) release();
           if (valid) {
             uint32_t pa[16], pu[16], ph[16];
 #pragma unroll
@@ -407,20 +502,21 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
               ph[i] = pack_bf16(a0 * sigmoidf_(a0) * u0, a1 * sigmoidf_(a1) * u1);
             }
             const int col = ti.n0 + c * 32;
-            store_64B(arow + col, pa);
-            store_64B(arow + p.f + col, pu);
-            store_64B(arow + 2 * p.f + col, ph);
+            store_64B(arow_out + col, pa);
+            store_64B(arow_out + p.f + col, pu);
+            store_64B(arow_out + 2 * p.f + col, ph);
           }
         }
       } else if constexpr (EPI == EPI_STORE) {
         __nv_bfloat16* orow = p.out + (int64_t)(ti.m0 + row) * p.ld_out + ti.n0;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+#pragma unroll
+        for (int ci = 0; ci < kMine; ++ci) {
+          const int c = c0 + ci;
           uint32_t v[32];
           tmem_ld32(ta + c * 32, v);
           tmem_wait_ld();
           tmem_tie(v);
-          if (c == BN / 32 - 1) release();
+          if (ci == kMine - 1) release();
           if (valid) {
             uint32_t pk[16];
 #pragma unroll
@@ -429,27 +525,17 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
           }
         }
       } else if constexpr (EPI == EPI_SWIGLU_BWD) {
-        const int64_t grow = ti.m0 + row;
-        const __nv_bfloat16* arow = p.act + grow * p.ld_act;
-        __nv_bfloat16* drow = p.out + grow * p.ld_out;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          const int col = ti.n0 + c * 32;
-          uint32_t av[16], uv[16];
-          if (valid) {
+        __nv_bfloat16* drow = p.out + (int64_t)(ti.m0 + row) * p.ld_out;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const uint4 x = *reinterpret_cast<const uint4*>(arow + col + 8 * i);
-              const uint4 y = *reinterpret_cast<const uint4*>(arow + p.f + col + 8 * i);
-              av[4 * i] = x.x; av[4 * i + 1] = x.y; av[4 * i + 2] = x.z; av[4 * i + 3] = x.w;
-              uv[4 * i] = y.x; uv[4 * i + 1] = y.y; uv[4 * i + 2] = y.z; uv[4 * i + 3] = y.w;
-            }
-          }
+        for (int ci = 0; ci < kMine; ++ci) {
+          const int col = ti.n0 + (c0 + ci) * 32;
+          uint32_t an[16], un[16];
+          if (ci + 1 < kMine && valid) load_au(arow, col + 32, p.f, an, un);  // one chunk ahead
           uint32_t v[32];
-          tmem_ld32(ta + c * 32, v);
+          tmem_ld32(ta + (c0 + ci) * 32, v);
           tmem_wait_ld();
           tmem_tie(v);
-          if (c == BN / 32 - 1) release();
+          if (ci == kMine - 1) release();
           if (valid) {
             uint32_t pda[16], pdu[16];
 #pragma unroll
@@ -470,41 +556,205 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
             store_64B(drow + col, pda);
             store_64B(drow + p.f + col, pdu);
           }
+          if (ci + 1 < kMine) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) { av[i] = an[i]; uv[i] = un[i]; }
+          }
+        }
+      } else if constexpr (EPI == EPI_ROUTER) {
+        // logits (+ bias), softmax over the p.N experts, top-k (lowest index wins
+        // ties), then this 128-token block's per-expert counts and in-block ranks.
+        const int Er = p.N, k = p.topk;
+        const int64_t tok = ti.m0 + row;
+        float topv[kRouterKMax];
+        int topi[kRouterKMax];
+#pragma unroll
+        for (int j = 0; j < kRouterKMax; ++j) { topv[j] = -INFINITY; topi[j] = -1; }
+        float mx = -INFINITY;
+        float* lrow = p.logits + tok * Er;
+#pragma unroll 1
+        for (int c = 0; c < BN / 16; ++c) {
+          uint32_t v[16];
+          tmem_ld16(ta + c * 16, v);
+          tmem_wait_ld();
+          tmem_tie16(v);
+          float l[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int e = c * 16 + i;
+            l[i] = e < Er ? __uint_as_float(v[i]) + (p.bias ? p.bias[e] : 0.f) : -INFINITY;
+            if (e < Er) {
+              mx = fmaxf(mx, l[i]);
+              float cv = l[i];
+              int ci = e;
+#pragma unroll
+              for (int j = 0; j < kRouterKMax; ++j) {  // ascending e: equal values keep the lower index
+                if (j < k && (topi[j] < 0 || cv > topv[j])) {
+                  const float tv = topv[j]; topv[j] = cv; cv = tv;
+                  const int tix = topi[j]; topi[j] = ci; ci = tix;
+                }
+              }
+            }
+          }
+          if (valid) {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const int e0 = c * 16 + 4 * q4;
+              if ((Er & 3) == 0 && e0 + 4 <= Er)
+                *reinterpret_cast<float4*>(lrow + e0) = make_float4(l[4 * q4], l[4 * q4 + 1], l[4 * q4 + 2], l[4 * q4 + 3]);
+              else
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                  if (e0 + i < Er) lrow[e0 + i] = l[4 * q4 + i];
+            }
+          }
+        }
+        float sum = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < BN / 16; ++c) {
+          uint32_t v[16];
+          tmem_ld16(ta + c * 16, v);
+          tmem_wait_ld();
+          tmem_tie16(v);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int e = c * 16 + i;
+            if (e < Er) sum += expf(__uint_as_float(v[i]) + (p.bias ? p.bias[e] : 0.f) - mx);
+          }
+        }
+        release();
+        int* sel = s_sel + row * kRouterKMax;
+#pragma unroll
+        for (int j = 0; j < kRouterKMax; ++j) {
+          if (j < k) {
+            sel[j] = valid ? topi[j] : -1;
+            if (valid) {
+              p.topk_idx[tok * k + j] = topi[j];
+              p.topk_gate[tok * k + j] = expf(topv[j] - mx) / sum;
+            }
+          }
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (valid) {
+          for (int j = 0; j < k; ++j) {
+            const int e = sel[j];
+            int rank = 0;
+            for (int r2 = 0; r2 < row; ++r2)
+              for (int j2 = 0; j2 < k; ++j2) rank += (s_sel[r2 * kRouterKMax + j2] == e);
+            p.localrank[tok * k + j] = rank;
+          }
+        }
+        const int blk = ti.m0 / BM;
+        for (int e = row; e < Er; e += 128) {
+          int cnt = 0;
+          for (int r2 = 0; r2 < ti.rows; ++r2)
+            for (int j2 = 0; j2 < k; ++j2) cnt += (s_sel[r2 * kRouterKMax + j2] == e);
+          p.blockcounts[(int64_t)e * p.nb + blk] = cnt;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");  // s_sel is reused by the next tile
+      } else if constexpr (EPI == EPI_ROUTER_DX) {
+        // router backward: dx = dl w_router (the accumulator) + the token's k expert rows
+        const int k = p.topk;
+        const int64_t tok = ti.m0 + row;
+        int rj[kRouterKMax];
+#pragma unroll
+        for (int j = 0; j < kRouterKMax; ++j)
+          rj[j] = (valid && j < k) ? __ldg(p.slot_row + tok * k + j) : -1;
+        __nv_bfloat16* orow = p.out + tok * p.ld_out;
+#pragma unroll
+        for (int ci = 0; ci < kMine; ++ci) {
+          const int col = ti.n0 + (c0 + ci) * 32;
+          uint32_t v[32];
+          tmem_ld32(ta + (c0 + ci) * 32, v);
+          tmem_wait_ld();
+          tmem_tie(v);
+          if (ci == kMine - 1) release();
+          if (valid) {
+            float accf[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) accf[i] = __uint_as_float(v[i]);
+#pragma unroll
+            for (int j = 0; j < kRouterKMax; ++j) {
+              if (rj[j] < 0) continue;
+              const uint4* src = reinterpret_cast<const uint4*>(p.act + (int64_t)rj[j] * p.ld_act + col);
+#pragma unroll
+              for (int i4 = 0; i4 < 4; ++i4) {
+                const uint4 w = __ldg(src + i4);
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                  accf[8 * i4 + 2 * h] += bf_lo(ww[h]);
+                  accf[8 * i4 + 2 * h + 1] += bf_hi(ww[h]);
+                }
+              }
+            }
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(accf[2 * i], accf[2 * i + 1]);
+            store_64B(orow + col, pk);
+          }
         }
       } else {  // EPI_WGRAD
-        const int64_t ooff = (int64_t)ti.g * p.out_group + (int64_t)(ti.m0 + row) * p.ld_out + ti.n0;
-        if (ti.nkb == 0) {
-          release();
-          if (p.out_f32) {
-            float4* o = reinterpret_cast<float4*>(p.out_f32 + ooff);
-            for (int i = 0; i < BN / 4; ++i) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-          } else {
-            uint4* o = reinterpret_cast<uint4*>(p.out + ooff);
-            for (int i = 0; i < BN / 8; ++i) o[i] = make_uint4(0, 0, 0, 0);
+        const int64_t orow0 = (int64_t)ti.g * p.M + ti.m0 + q * 32;  // first output row of this warp
+        if (p.out_f32) {
+          // fp32: stage 16 rows x 32 columns in shared memory (128-byte swizzle) and
+          // write them with one TMA store per box: whole 128-byte lines to HBM.
+          uint8_t* sbuf = s_store + (warp - 2) * 2048;
+#pragma unroll 1
+          for (int ci = 0; ci < kMine; ++ci) {
+            uint32_t v[32];
+            if (ti.nkb > 0) {
+              tmem_ld32(ta + (c0 + ci) * 32, v);
+              tmem_wait_ld();
+              tmem_tie(v);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] = 0;
+            }
+            if (ci == kMine - 1) release();
+#pragma unroll 1
+            for (int hh = 0; hh < 2; ++hh) {
+              if (lane == 0) tma_store_wait_read();  // the previous box has left the buffer
+              __syncwarp();
+              if ((lane >> 4) == hh) {
+                const int r = lane & 15;
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                  *reinterpret_cast<uint4*>(sbuf + r * 128 + ((j ^ (r & 7)) * 16)) =
+                      make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+              }
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0)
+                tma_store_2d(&p.tmOut, ti.n0 + (c0 + ci) * 32, (int)(orow0 + 16 * hh), sbuf);
+            }
           }
         } else {
+          __nv_bfloat16* o = p.out + (orow0 + lane) * p.ld_out + ti.n0 + c0 * 32;
 #pragma unroll 1
-          for (int c = 0; c < BN / 32; ++c) {
-            uint32_t v[32];
-            tmem_ld32(ta + c * 32, v);
-            tmem_wait_ld();
-            tmem_tie(v);
-            if (c == BN / 32 - 1) release();
-            if (p.out_f32) {
-              uint4* o = reinterpret_cast<uint4*>(p.out_f32 + ooff + c * 32);
-#pragma unroll
-              for (int i = 0; i < 8; ++i) o[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-            } else {
-              uint32_t pk[16];
+          for (int ci = 0; ci < kMine; ++ci) {
+            uint32_t pk[16];
+            if (ti.nkb > 0) {
+              uint32_t v[32];
+              tmem_ld32(ta + (c0 + ci) * 32, v);
+              tmem_wait_ld();
+              tmem_tie(v);
 #pragma unroll
               for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-              store_64B(p.out + ooff + c * 32, pk);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) pk[i] = 0;
             }
+            if (ci == kMine - 1) release();
+            store_64B(o + ci * 32, pk);
           }
         }
       }
       ++acc_it;
     }
+  }
+  if constexpr (EPI == EPI_WGRAD) {
+    if (warp >= 2 && lane == 0) tma_store_wait_all();
   }
   __syncthreads();
   if (warp == 0) {
@@ -526,16 +776,16 @@ cudaError_t get_encode() {
   return cudaSuccess;
 }
 
-// 2-D bf16 tensor map over [outer, inner] with row stride `ld` elements.
+// 2-D tensor map over [outer, inner] with row stride `ld` elements, 128-byte swizzle.
 bool tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
-          uint32_t box_inner, uint32_t box_outer) {
+          uint32_t box_inner, uint32_t box_outer, bool f32 = false) {
   const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {ld * 2};
+  const cuuint64_t strides[1] = {ld * (f32 ? 4 : 2)};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t es[2] = {1, 1};
-  return g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  return g_encode(tm, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -562,7 +812,77 @@ GemmParams base_params(const FfnShape& s, const int32_t* offsets, int* status) {
 
 int64_t m_tile_bound(const FfnShape& s) { return s.rows / BM + s.E; }
 
+template <int BN>
+cudaError_t route_tc_bn(const RouteArgs& a, int nb, cudaStream_t st) {
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  if (!tmap(&p.tmA, a.x, a.d, a.T, a.d, 64, 128) ||
+      !tmap(&p.tmB, a.w_router, a.d, a.E, a.d, 64, Cfg<BN>::kBoxRows))
+    return cudaErrorInvalidValue;
+  p.offsets = nullptr;
+  p.E = 1;
+  p.rows_total = a.T;
+  p.N = a.E;
+  p.K = a.d;
+  p.topk = a.k;
+  p.nb = nb;
+  p.bias = a.bias;
+  p.logits = a.logits;
+  p.topk_idx = a.topk_idx;
+  p.topk_gate = a.topk_gate;
+  p.blockcounts = a.blockcounts;
+  p.localrank = a.localrank;
+  p.status = a.status;
+  return launch<BN, false, false, EPI_ROUTER, false>(p, nb, st);
+}
+
 }  // namespace
+
+bool route_tc_supported(int E, int k, int d) { return E <= 256 && k <= kRouterKMax && d % BK == 0; }
+
+cudaError_t route_tc_launch(const RouteArgs& a, int nb, cudaStream_t st) {
+  cudaError_t err = get_encode();
+  if (err != cudaSuccess) return err;
+  if (a.E <= 16) return route_tc_bn<16>(a, nb, st);
+  if (a.E <= 64) return route_tc_bn<64>(a, nb, st);
+  if (a.E <= 128) return route_tc_bn<128>(a, nb, st);
+  return route_tc_bn<256>(a, nb, st);
+}
+
+bool route_bwd_tc_supported(int E, int k, int d) {
+  return E % BM == 0 && k <= kRouterKMax && d % 256 == 0;
+}
+
+cudaError_t route_bwd_tc_launch(const void* x, const void* w_router, const void* dl_bf16,
+                                const void* dx_perm, const int32_t* slot_row, void* dx,
+                                float* partial, int splits, int T, int d, int E, int k,
+                                int* status, cudaStream_t st) {
+  cudaError_t err = get_encode();
+  if (err != cudaSuccess) return err;
+  // dx = dl W_r + sum_j dx_perm[slot_row[t, j]]   (M = T, N = d, K = E)
+  GemmParams p1;
+  memset(&p1, 0, sizeof(p1));
+  if (!tmap(&p1.tmA, dl_bf16, E, T, E, 64, 128) || !tmap(&p1.tmB, w_router, d, E, d, 64, 64))
+    return cudaErrorInvalidValue;
+  p1.E = 1; p1.rows_total = T; p1.N = d; p1.K = E; p1.topk = k;
+  p1.slot_row = slot_row;
+  p1.act = static_cast<const __nv_bfloat16*>(dx_perm); p1.ld_act = d;
+  p1.out = static_cast<__nv_bfloat16*>(dx); p1.ld_out = d;
+  p1.status = status;
+  if ((err = launch<256, false, true, EPI_ROUTER_DX, false>(p1, (int64_t)((T + BM - 1) / BM) * (d / 256), st)) != cudaSuccess)
+    return err;
+  // partial[s] = dl_s^T x_s over `splits` consecutive token ranges  (M = E, N = d)
+  GemmParams p2;
+  memset(&p2, 0, sizeof(p2));
+  if (!tmap(&p2.tmA, dl_bf16, E, T, E, 64, 64) || !tmap(&p2.tmB, x, d, T, d, 64, 64) ||
+      !tmap(&p2.tmOut, partial, d, (uint64_t)splits * E, d, 32, 16, true))
+    return cudaErrorInvalidValue;
+  p2.E = splits; p2.rows_total = T; p2.split = (T + splits - 1) / splits;
+  p2.M = E; p2.N = d;
+  p2.out_f32 = partial; p2.ld_out = d; p2.out_group = (int64_t)E * d;
+  p2.status = status;
+  return launch<256, true, true, EPI_WGRAD, true>(p2, (int64_t)splits * (E / BM) * (d / 256), st);
+}
 
 cudaError_t ffn_fwd_bf16(const FfnShape& s, const void* x_perm, const int32_t* offsets,
                          const void* w1, const void* w2, void* act, void* y_perm, int* status,
@@ -630,6 +950,7 @@ cudaError_t ffn_bwd_bf16(const FfnShape& s, const void* dy_perm, const void* x_p
   p5.M = d; p5.N = f;
   p5.out = static_cast<__nv_bfloat16*>(dw2); p5.out_f32 = dw_f32 ? static_cast<float*>(dw2) : nullptr;
   p5.ld_out = f; p5.out_group = (int64_t)d * f;
+  if (dw_f32 && !tmap(&p5.tmOut, dw2, f, (uint64_t)E * d, f, 32, 16, true)) return cudaErrorInvalidValue;
   if ((err = launch<256, true, true, EPI_WGRAD, true>(p5, (int64_t)E * (d / 128) * (f / 256), st)) != cudaSuccess)
     return err;
   // wgrad 1: dW1[e] = [da | du]^T x   (M = 2f, N = d)
@@ -640,6 +961,7 @@ cudaError_t ffn_bwd_bf16(const FfnShape& s, const void* dy_perm, const void* x_p
   p6.M = 2 * f; p6.N = d;
   p6.out = static_cast<__nv_bfloat16*>(dw1); p6.out_f32 = dw_f32 ? static_cast<float*>(dw1) : nullptr;
   p6.ld_out = d; p6.out_group = (int64_t)2 * f * d;
+  if (dw_f32 && !tmap(&p6.tmOut, dw1, d, (uint64_t)E * 2 * f, d, 32, 16, true)) return cudaErrorInvalidValue;
   return launch<256, true, true, EPI_WGRAD, true>(p6, (int64_t)E * (2 * f / 128) * (d / 256), st);
 }
 

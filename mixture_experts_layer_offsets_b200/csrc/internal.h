@@ -24,12 +24,17 @@ struct RouteArgs {
   int32_t* offsets;
   int32_t* slot_row;
   void* scratch;            // route_ws_bytes(T, E, k) bytes
+  int* status = nullptr;    // workspace status word (bounded waits), may be null
   // filled in by route_launch
   int32_t* blockcounts = nullptr;
   int32_t* localrank = nullptr;
 };
 size_t route_ws_bytes(int T, int E, int k);
 cudaError_t route_launch(const RouteArgs& a, bool bf16, cudaStream_t st);
+// tensor-core router (bf16): logits GEMM with softmax/top-k/counts/ranks fused in
+// the epilogue, one 128-token block per tile
+bool route_tc_supported(int E, int k, int d);
+cudaError_t route_tc_launch(const RouteArgs& a, int nb, cudaStream_t st);
 
 // ---------------------------------------------------------- row movement
 cudaError_t permute_launch(bool bf16, const void* x, const int32_t* slot_row, void* x_perm,
@@ -46,10 +51,16 @@ cudaError_t padded_dispatch_launch(bool bf16, int capacity, const void* x, const
 
 // ------------------------------------------------------------ router bwd
 size_t route_bwd_ws_bytes(int T, int d, int E);
+// tensor-core router backward (bf16, E a multiple of 128): dx and per-split dW_r partials
+bool route_bwd_tc_supported(int E, int k, int d);
+cudaError_t route_bwd_tc_launch(const void* x, const void* w_router, const void* dl_bf16,
+                                const void* dx_perm, const int32_t* slot_row, void* dx,
+                                float* partial, int splits, int T, int d, int E, int k,
+                                int* status, cudaStream_t st);
 cudaError_t route_bwd_launch(bool bf16, const void* x, const void* w_router, const float* logits,
                              const int32_t* topk_idx, const float* dgate, const void* dx_perm,
                              const int32_t* slot_row, void* dx, float* dw_router, int T, int d,
-                             int E, int k, void* scratch, cudaStream_t st);
+                             int E, int k, void* scratch, int* status, cudaStream_t st);
 
 // ----------------------------------------------------------------- MXFP8
 cudaError_t mxfp8_launch(int64_t rows, int64_t K, bool src_bf16, const void* src, int axis,

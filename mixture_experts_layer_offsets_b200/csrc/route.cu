@@ -8,7 +8,9 @@
 //
 // Three launches, no host round trip:
 //   1. route_topk_kernel   -- per block of TB tokens: fp32 logits (CUDA-core dot
-//      products), softmax, top-k (warp argmax, lowest index wins ties), the
+//      products; for E <= 32 each warp streams 4 token rows with 16-byte loads,
+//      for larger E shared-memory tiles), softmax, top-k (warp argmax, lowest
+//      index wins ties), the
 //      block's per-expert counts and each pair's rank among the block's pairs
 //      of the same expert;
 //   2. block_scan_kernel    -- per expert: exclusive scan of the block counts in
@@ -30,8 +32,56 @@ constexpr int kDC = 32;  // d-chunk staged in shared memory
 // Tokens per block: keep the [TB, E] logit tile within 32 KB.
 __host__ __device__ inline int route_tb(int E) { return E <= 256 ? 32 : (E <= 512 ? 16 : 8); }
 
-// EC experts per pass of the dot-product phase.
-template <typename T, int TB, int EC>
+// Logits of TB = 32 tokens for E <= EMAX experts: each warp takes 4 tokens,
+// each lane 16-byte chunks of their rows (coalesced reads of x) and keeps
+// 4 x EMAX partial dot products; the router rows come through L1.
+template <typename T, int EMAX>
+__device__ __forceinline__ void logits_narrow(const T* __restrict__ x, const T* __restrict__ w,
+                                              const float* __restrict__ bias, int ntok, int d,
+                                              int E, int t0, float* lg) {
+  constexpr int V = Vec16<T>::N;
+  constexpr int TPW = 4;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r0 = warp * TPW;
+  float acc[TPW][EMAX];
+#pragma unroll
+  for (int tt = 0; tt < TPW; ++tt)
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) acc[tt][e] = 0.f;
+  const int chunks = d / V;
+  for (int c = lane; c < chunks; c += 32) {
+    Vec16<T> xv[TPW];
+#pragma unroll
+    for (int tt = 0; tt < TPW; ++tt) {
+      const int t = t0 + r0 + tt;
+      xv[tt].raw = t < ntok ? ldg16(x + (int64_t)t * d + (int64_t)c * V) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) {
+      if (e < E) {
+        Vec16<T> wv;
+        wv.raw = ldg16(w + (int64_t)e * d + (int64_t)c * V);
+#pragma unroll
+        for (int tt = 0; tt < TPW; ++tt)
+#pragma unroll
+          for (int i = 0; i < V; ++i) acc[tt][e] = fmaf(xv[tt].get(i), wv.get(i), acc[tt][e]);
+      }
+    }
+  }
+#pragma unroll
+  for (int tt = 0; tt < TPW; ++tt)
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) {
+      if (e < E) {
+        const float v = warp_sum(acc[tt][e]);
+        if (lane == 0) lg[(r0 + tt) * E + e] = v + (bias ? bias[e] : 0.f);
+      }
+    }
+}
+
+// EC experts per pass of the dot-product phase; EMAX > 0 selects the narrow
+// (E <= EMAX, TB = 32) logit phase instead of the shared-memory tiles.
+template <typename T, int TB, int EC, int EMAX>
 __global__ void __launch_bounds__(kRouteThreads)
 route_topk_kernel(const T* __restrict__ x, const T* __restrict__ w, const float* __restrict__ bias,
                   int ntok, int d, int E, int k, float* __restrict__ logits,
@@ -39,8 +89,9 @@ route_topk_kernel(const T* __restrict__ x, const T* __restrict__ w, const float*
                   int32_t* __restrict__ blockcounts, int32_t* __restrict__ localrank, int nb) {
   constexpr int kPer = TB * EC / kRouteThreads;  // outputs per thread
   static_assert(kPer >= 1 && (TB * EC) % kRouteThreads == 0, "tile");
-  __shared__ float xs[TB][kDC + 1];
-  __shared__ float ws[EC][kDC + 1];
+  static_assert(EMAX == 0 || TB == 32, "the narrow phase covers 8 warps x 4 tokens");
+  __shared__ float xs[EMAX ? 1 : TB][kDC + 1];
+  __shared__ float ws[EMAX ? 1 : EC][kDC + 1];
   __shared__ int32_t sel[TB][32];
   extern __shared__ float lg[];  // [TB][E]
 
@@ -50,7 +101,8 @@ route_topk_kernel(const T* __restrict__ x, const T* __restrict__ w, const float*
   const int row0 = tid / EC;
   constexpr int kRowStep = kRouteThreads / EC;
 
-  for (int e0 = 0; e0 < E; e0 += EC) {
+  if constexpr (EMAX > 0) logits_narrow<T, EMAX>(x, w, bias, ntok, d, E, t0, lg);
+  else for (int e0 = 0; e0 < E; e0 += EC) {
     float acc[kPer];
 #pragma unroll
     for (int i = 0; i < kPer; ++i) acc[i] = 0.f;
@@ -225,10 +277,10 @@ slot_rows_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict
   }
 }
 
-template <typename T, int TB, int EC>
+template <typename T, int TB, int EC, int EMAX = 0>
 cudaError_t launch_topk(const RouteArgs& a, int nb, cudaStream_t st) {
   const size_t lg_bytes = sizeof(float) * TB * a.E;
-  auto kern = route_topk_kernel<T, TB, EC>;
+  auto kern = route_topk_kernel<T, TB, EC, EMAX>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)lg_bytes);
   if (err != cudaSuccess) return err;
@@ -242,8 +294,9 @@ template <typename T>
 cudaError_t dispatch_topk(const RouteArgs& a, int nb, cudaStream_t st) {
   const int tb = route_tb(a.E);
   if (tb == 32) {
-    if (a.E <= 8) return launch_topk<T, 32, 8>(a, nb, st);
-    if (a.E <= 32) return launch_topk<T, 32, 32>(a, nb, st);
+    if (a.E <= 8) return launch_topk<T, 32, 8, 8>(a, nb, st);
+    if (a.E <= 16) return launch_topk<T, 32, 8, 16>(a, nb, st);
+    if (a.E <= 32) return launch_topk<T, 32, 8, 32>(a, nb, st);
     return launch_topk<T, 32, 64>(a, nb, st);
   }
   if (tb == 16) return launch_topk<T, 16, 64>(a, nb, st);
@@ -260,7 +313,8 @@ size_t route_ws_bytes(int T, int E, int k) {
 
 cudaError_t route_launch(const RouteArgs& a0, bool bf16, cudaStream_t st) {
   RouteArgs a = a0;
-  const int tb = route_tb(a.E);
+  const bool tc = bf16 && a.T > 0 && route_tc_supported(a.E, a.k, a.d);
+  const int tb = tc ? 128 : route_tb(a.E);  // tokens per block of the count/rank pass
   const int nb = (a.T + tb - 1) / tb;
   uint8_t* ws = static_cast<uint8_t*>(a.scratch);
   a.blockcounts = reinterpret_cast<int32_t*>(ws);
@@ -268,7 +322,10 @@ cudaError_t route_launch(const RouteArgs& a0, bool bf16, cudaStream_t st) {
   a.localrank = reinterpret_cast<int32_t*>(ws + 2 * align256((size_t)nb * a.E * 4));
   cudaError_t err;
   if (nb > 0) {
-    err = bf16 ? dispatch_topk<__nv_bfloat16>(a, nb, st) : dispatch_topk<float>(a, nb, st);
+    if (tc)
+      err = route_tc_launch(a, nb, st);
+    else
+      err = bf16 ? dispatch_topk<__nv_bfloat16>(a, nb, st) : dispatch_topk<float>(a, nb, st);
     if (err != cudaSuccess) return err;
   }
   // With T == 0 the scan still writes zero counts and offsets.

@@ -16,15 +16,15 @@ namespace moe {
 namespace {
 
 constexpr int kTT = 32;   // tokens per tile
-constexpr int kEC = 32;   // experts per tile
-constexpr int kCols = 256;
 
-inline int route_bwd_splits(int T) { return std::max(1, std::min(32, T / 512)); }
+inline int route_bwd_splits(int T) { return std::max(1, std::min(128, T / 128)); }
 
-// dl, one warp per token (fp32, written to the workspace).
+// dl, one warp per token, written to the workspace in fp32 (CUDA-core path) or
+// bf16 (tensor-core path, where dl is a GEMM operand).
 __global__ void __launch_bounds__(256)
 dlogit_kernel(const float* __restrict__ logits, const int32_t* __restrict__ topk_idx,
-              const float* __restrict__ dgate, float* __restrict__ dl, int ntok, int E, int k) {
+              const float* __restrict__ dgate, float* __restrict__ dl,
+              __nv_bfloat16* __restrict__ dl_bf, int ntok, int E, int k) {
   const int lane = threadIdx.x & 31;
   for (int t = blockIdx.x * 8 + (threadIdx.x >> 5); t < ntok; t += gridDim.x * 8) {
     const float* l = logits + (int64_t)t * E;
@@ -43,87 +43,119 @@ dlogit_kernel(const float* __restrict__ logits, const int32_t* __restrict__ topk
       float dp = 0.f;
       for (int j = 0; j < k; ++j)
         if (__ldg(idx + j) == e) dp = __ldg(dg + j);
-      dl[(int64_t)t * E + e] = (expf(l[e] - m) / s) * (dp - pdp);
+      const float v = (expf(l[e] - m) / s) * (dp - pdp);
+      if (dl) dl[(int64_t)t * E + e] = v;
+      if (dl_bf) dl_bf[(int64_t)t * E + e] = __float2bfloat16_rn(v);
     }
   }
 }
 
-// dx = dl w_router + sum_j dx_perm[slot_row[t,j]]; tile of kTT tokens x kCols columns.
+// dx = dl w_router + sum_j dx_perm[slot_row[t,j]].  A warp takes 4 tokens and
+// walks their rows in 16-byte chunks (one chunk per lane): the router term
+// reuses each w_router chunk for the 4 tokens, dl comes from shared memory,
+// and the k expert rows of each token are gathered with 16-byte loads.
 template <typename T>
-__global__ void __launch_bounds__(kCols)
+__global__ void __launch_bounds__(256)
 dx_kernel(const float* __restrict__ dl, const T* __restrict__ w, const T* __restrict__ dx_perm,
           const int32_t* __restrict__ slot_row, T* __restrict__ dx, int ntok, int d, int E, int k) {
-  __shared__ float dls[kTT][kEC + 1];
-  __shared__ float ws[kEC][kCols];
-  const int tid = threadIdx.x;
-  const int t0 = blockIdx.x * kTT;
-  const int c = blockIdx.y * kCols + tid;
-  float acc[kTT];
-#pragma unroll
-  for (int i = 0; i < kTT; ++i) acc[i] = 0.f;
-  for (int e0 = 0; e0 < E; e0 += kEC) {
-    for (int i = tid; i < kTT * kEC; i += kCols) {
-      const int r = i / kEC, e = i % kEC;
-      dls[r][e] = (t0 + r < ntok && e0 + e < E) ? dl[(int64_t)(t0 + r) * E + e0 + e] : 0.f;
-    }
-    for (int e = 0; e < kEC; ++e)
-      ws[e][tid] = (e0 + e < E && c < d) ? to_f32(w[(int64_t)(e0 + e) * d + c]) : 0.f;
-    __syncthreads();
-#pragma unroll 4
-    for (int e = 0; e < kEC; ++e) {
-      const float wv = ws[e][tid];
-#pragma unroll
-      for (int i = 0; i < kTT; ++i) acc[i] = fmaf(dls[i][e], wv, acc[i]);
-    }
-    __syncthreads();
+  constexpr int V = Vec16<T>::N;
+  constexpr int TPW = 4;
+  extern __shared__ float s_dl[];  // [8 warps][TPW][E]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = (blockIdx.x * 8 + warp) * TPW;
+  float* my = s_dl + warp * TPW * E;
+  for (int i = lane; i < TPW * E; i += 32) {
+    const int t = t0 + i / E;
+    my[i] = t < ntok ? dl[(int64_t)t * E + i % E] : 0.f;
   }
-  if (c >= d) return;
-#pragma unroll 1
-  for (int i = 0; i < kTT; ++i) {
-    const int t = t0 + i;
-    if (t >= ntok) break;
-    float v = acc[i];
-    for (int j = 0; j < k; ++j) {
-      const int r = slot_row[(int64_t)t * k + j];
-      if (r >= 0) v += to_f32(dx_perm[(int64_t)r * d + c]);
+  __syncwarp();
+  const int chunks = d / V;
+  for (int c = lane; c < chunks; c += 32) {
+    float acc[TPW][V];
+#pragma unroll
+    for (int tt = 0; tt < TPW; ++tt)
+#pragma unroll
+      for (int i = 0; i < V; ++i) acc[tt][i] = 0.f;
+    for (int e = 0; e < E; ++e) {
+      Vec16<T> wv;
+      wv.raw = ldg16(w + (int64_t)e * d + (int64_t)c * V);
+#pragma unroll
+      for (int tt = 0; tt < TPW; ++tt) {
+        const float g = my[tt * E + e];
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[tt][i] = fmaf(g, wv.get(i), acc[tt][i]);
+      }
     }
-    dx[(int64_t)t * d + c] = from_f32<T>(v);
+#pragma unroll
+    for (int tt = 0; tt < TPW; ++tt) {
+      const int t = t0 + tt;
+      if (t >= ntok) break;
+#pragma unroll 8
+      for (int j = 0; j < k; ++j) {
+        const int r = __ldg(slot_row + (int64_t)t * k + j);
+        if (r < 0) continue;
+        Vec16<T> v;
+        v.raw = ldg16(dx_perm + (int64_t)r * d + (int64_t)c * V);
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[tt][i] += v.get(i);
+      }
+      Vec16<T> o;
+#pragma unroll
+      for (int i = 0; i < V; ++i) o.set(i, acc[tt][i]);
+      stg16(dx + (int64_t)t * d + (int64_t)c * V, o.raw);
+    }
   }
 }
 
-// partial[s][e][c] = sum over tokens of split s of dl[t,e] * x[t,c]
-template <typename T>
-__global__ void __launch_bounds__(kCols)
+// partial[s][e][c..c+V) = sum over the tokens of split s of dl[t,e] * x[t, c..c+V):
+// each thread owns one 16-byte column chunk and EB experts.
+template <typename T, int EB>
+__global__ void __launch_bounds__(256)
 dwr_partial_kernel(const float* __restrict__ dl, const T* __restrict__ x,
                    float* __restrict__ partial, int ntok, int d, int E, int tok_per_split) {
-  __shared__ float dls[kTT][kEC + 1];
-  const int tid = threadIdx.x;
-  const int c = blockIdx.x * kCols + tid;
-  const int e0 = blockIdx.y * kEC;
+  constexpr int V = Vec16<T>::N;
+  __shared__ float s_dl[kTT][EB];
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  const int e0 = blockIdx.y * EB;
   const int s = blockIdx.z;
   const int ta = s * tok_per_split, tb = min(ntok, ta + tok_per_split);
-  float acc[kEC];
+  const bool live = c < d / V;
+  float acc[EB][V];
 #pragma unroll
-  for (int i = 0; i < kEC; ++i) acc[i] = 0.f;
+  for (int e = 0; e < EB; ++e)
+#pragma unroll
+    for (int i = 0; i < V; ++i) acc[e][i] = 0.f;
   for (int t0 = ta; t0 < tb; t0 += kTT) {
-    for (int i = tid; i < kTT * kEC; i += kCols) {
-      const int r = i / kEC, e = i % kEC;
-      dls[r][e] = (t0 + r < tb && e0 + e < E) ? dl[(int64_t)(t0 + r) * E + e0 + e] : 0.f;
+    for (int i = threadIdx.x; i < kTT * EB; i += blockDim.x) {
+      const int r = i / EB, e = i % EB;
+      s_dl[r][e] = (t0 + r < tb && e0 + e < E) ? dl[(int64_t)(t0 + r) * E + e0 + e] : 0.f;
     }
     __syncthreads();
-    if (c < d) {
+    if (live) {
       const int n = min(kTT, tb - t0);
+#pragma unroll 4
       for (int r = 0; r < n; ++r) {
-        const float xv = to_f32(x[(int64_t)(t0 + r) * d + c]);
+        Vec16<T> xv;
+        xv.raw = ldg16(x + (int64_t)(t0 + r) * d + (int64_t)c * V);
 #pragma unroll
-        for (int e = 0; e < kEC; ++e) acc[e] = fmaf(dls[r][e], xv, acc[e]);
+        for (int e = 0; e < EB; ++e) {
+          const float g = s_dl[r][e];
+#pragma unroll
+          for (int i = 0; i < V; ++i) acc[e][i] = fmaf(g, xv.get(i), acc[e][i]);
+        }
       }
     }
     __syncthreads();
   }
-  if (c >= d) return;
-  for (int e = 0; e < kEC && e0 + e < E; ++e)
-    partial[((int64_t)s * E + e0 + e) * d + c] = acc[e];
+  if (!live) return;
+#pragma unroll
+  for (int e = 0; e < EB; ++e) {
+    if (e0 + e >= E) break;
+    float* dst = partial + ((int64_t)s * E + e0 + e) * d + (int64_t)c * V;
+#pragma unroll
+    for (int i = 0; i < V; i += 4)
+      *reinterpret_cast<float4*>(dst + i) = make_float4(acc[e][i], acc[e][i + 1], acc[e][i + 2], acc[e][i + 3]);
+  }
 }
 
 __global__ void dwr_reduce_kernel(const float* __restrict__ partial, float* __restrict__ dw,
@@ -140,23 +172,41 @@ template <typename T>
 cudaError_t route_bwd_t(const void* x, const void* w_router, const float* logits,
                         const int32_t* topk_idx, const float* dgate, const void* dx_perm,
                         const int32_t* slot_row, void* dx, float* dw_router, int T_, int d, int E,
-                        int k, void* scratch, cudaStream_t st) {
+                        int k, void* scratch, int* status, cudaStream_t st) {
+  constexpr int V = Vec16<T>::N;
+  constexpr int EB = 8;
   const int splits = route_bwd_splits(T_);
   float* dl = static_cast<float*>(scratch);
   float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) +
                                             align256((size_t)T_ * E * 4));
   const int64_t n = (int64_t)E * d;
+  const int lgrid = std::min((T_ + 7) / 8, num_sms() * 8);
+  if (T_ > 0 && sizeof(T) == 2 && route_bwd_tc_supported(E, k, d)) {
+    // tensor cores: dl (bf16) is the A operand of both the dx and the dW_r GEMM
+    __nv_bfloat16* dl_bf = static_cast<__nv_bfloat16*>(scratch);
+    const int tsplits = std::max(1, std::min(32, T_ / 1024));
+    dlogit_kernel<<<lgrid, 256, 0, st>>>(logits, topk_idx, dgate, nullptr, dl_bf, T_, E, k);
+    cudaError_t err = route_bwd_tc_launch(x, w_router, dl_bf, dx_perm, slot_row, dx, partial,
+                                          tsplits, T_, d, E, k, status, st);
+    if (err != cudaSuccess) return err;
+    dwr_reduce_kernel<<<(int)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, st>>>(
+        partial, dw_router, n, tsplits);
+    return cudaGetLastError();
+  }
   if (T_ > 0) {
-    dlogit_kernel<<<std::min((T_ + 7) / 8, num_sms() * 8), 256, 0, st>>>(logits, topk_idx, dgate,
-                                                                         dl, T_, E, k);
-    dim3 g1((T_ + kTT - 1) / kTT, (d + kCols - 1) / kCols);
-    dx_kernel<T><<<g1, kCols, 0, st>>>(dl, static_cast<const T*>(w_router),
-                                       static_cast<const T*>(dx_perm), slot_row,
-                                       static_cast<T*>(dx), T_, d, E, k);
+    dlogit_kernel<<<lgrid, 256, 0, st>>>(logits, topk_idx, dgate, dl, nullptr, T_, E, k);
+    const size_t dl_smem = (size_t)8 * 4 * E * sizeof(float);
+    auto dxk = dx_kernel<T>;
+    cudaError_t err = cudaFuncSetAttribute(dxk, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)dl_smem);
+    if (err != cudaSuccess) return err;
+    dxk<<<(T_ + 31) / 32, 256, dl_smem, st>>>(dl, static_cast<const T*>(w_router),
+                                              static_cast<const T*>(dx_perm), slot_row,
+                                              static_cast<T*>(dx), T_, d, E, k);
     const int tps = (T_ + splits - 1) / splits;
-    dim3 g2((d + kCols - 1) / kCols, (E + kEC - 1) / kEC, splits);
-    dwr_partial_kernel<T><<<g2, kCols, 0, st>>>(dl, static_cast<const T*>(x), partial, T_, d, E,
-                                                tps);
+    dim3 g2((d / V + 255) / 256, (E + EB - 1) / EB, splits);
+    dwr_partial_kernel<T, EB><<<g2, 256, 0, st>>>(dl, static_cast<const T*>(x), partial, T_, d,
+                                                  E, tps);
     dwr_reduce_kernel<<<(int)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, st>>>(
         partial, dw_router, n, splits);
   } else {
@@ -174,12 +224,12 @@ size_t route_bwd_ws_bytes(int T, int d, int E) {
 cudaError_t route_bwd_launch(bool bf16, const void* x, const void* w_router, const float* logits,
                              const int32_t* topk_idx, const float* dgate, const void* dx_perm,
                              const int32_t* slot_row, void* dx, float* dw_router, int T, int d,
-                             int E, int k, void* scratch, cudaStream_t st) {
+                             int E, int k, void* scratch, int* status, cudaStream_t st) {
   if (bf16)
     return route_bwd_t<__nv_bfloat16>(x, w_router, logits, topk_idx, dgate, dx_perm, slot_row, dx,
-                                      dw_router, T, d, E, k, scratch, st);
+                                      dw_router, T, d, E, k, scratch, status, st);
   return route_bwd_t<float>(x, w_router, logits, topk_idx, dgate, dx_perm, slot_row, dx,
-                            dw_router, T, d, E, k, scratch, st);
+                            dw_router, T, d, E, k, scratch, status, st);
 }
 
 }  // namespace moe

@@ -28,6 +28,10 @@ CASES = {
     # top_k = E: every expert sees every token (dense mixture)
     "bf16_dense": shrink(CONFIGS["bf16_e8"], name="bf16_dense", T=300, d_model=256, E=4, top_k=4,
                          d_ff=256, router_std=0.05),
+    # bf16, E = 128 (tensor-core router forward and backward), two dW_r token splits
+    # with ragged tails, ~80 rows per expert
+    "bf16_e128_small": shrink(CONFIGS["bf16_e128"], name="bf16_e128_small", T=2600, d_model=256,
+                              d_ff=256, router_std=1 / 16.0),
     # a single token; fp32
     "f32_one_token": shrink(CONFIGS["tiny_f32"], name="f32_one_token", T=1, d_model=16, E=4,
                             top_k=3, d_ff=8),
