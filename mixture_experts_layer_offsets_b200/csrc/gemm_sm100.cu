@@ -43,6 +43,7 @@
 #include "internal.h"
 
 #include <cudaTypedefs.h>
+#include <stdlib.h>
 
 namespace moe {
 
@@ -98,12 +99,15 @@ struct GemmParams {
   const int32_t* slot_row; // [rows_total][topk]
 };
 
-template <int BN> struct Cfg {
-  static constexpr uint32_t kBBytes = BN * BK * 2;
+template <int BN, bool PAIR = false> struct Cfg {
+  // PAIR: a CTA pair computes a 256-row tile; each CTA holds its 128 A rows and half
+  // of the BN B rows (cta_group::2).
+  static constexpr uint32_t kBBytes = (PAIR ? BN / 2 : BN) * BK * 2;
   static constexpr uint32_t kStage = kABytes + kBBytes;
-  static constexpr int kStages = (BN == 256) ? 4 : 6;
+  static constexpr int kStages = PAIR ? 6 : ((BN == 256) ? 4 : 6);
   static constexpr uint32_t kTmemCols = 2 * BN;
   static constexpr int kBoxRows = BN < 128 ? BN : 128;  // rows of one K-major B box
+  static constexpr int kTileM = PAIR ? 2 * BM : BM;     // rows of one scheduled tile
   // shared memory after the stage ring: barriers (256 B), offsets and tile prefix
   // (2 x 1025 ints), router selections (128 x kRouterKMax ints), then a 1024-aligned
   // staging area for TMA stores (8 epilogue warps x 16 rows x 128 B)
@@ -113,6 +117,7 @@ template <int BN> struct Cfg {
   static constexpr size_t kOffStore = (kOffSel + 128 * kRouterKMax * 4 + 1023) & ~size_t(1023);
   static constexpr size_t kStoreBytes = 8 * 16 * 128;
   static constexpr size_t kSmem = 1024 + kOffStore + kStoreBytes;
+  static_assert(128 * kRouterKMax * 4 >= 4 * 256 * 4, "router histogram fits the selection area");
   static_assert(kSmem <= 232448, "shared memory per CTA");
 };
 
@@ -135,6 +140,60 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
           smem_u32(bar))
       : "memory");
 }
+// ---- CTA-pair (cta_group::2) forms
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// shared::cluster address of the same shared variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+// TMA load into this CTA's shared memory, completing on the leader CTA's barrier.
+__device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* tm, int x, int y,
+                                                 uint32_t leader_bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(leader_bar)
+      : "memory");
+}
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                               uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accum));
+}
+// Arrive on the barrier at this offset in both CTAs of the pair once the MMAs are done.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)), "h"((uint16_t)3)
+      : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(slot)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -227,7 +286,7 @@ struct TileInfo {
   int g, m0, n0, rows, nkb, kbase, klast;
 };
 
-template <int BN, int EPI, bool GROUP_K>
+template <int BN, int EPI, bool GROUP_K, int TM = BM>
 __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, const int* s_off,
                                                 const int* s_pre, int nN) {
   TileInfo ti;
@@ -251,8 +310,8 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, cons
     ti.g = lo;
     const int local = t - s_pre[lo];
     const int mt = local / nN, nt = local - mt * nN;
-    ti.m0 = s_off[lo] + mt * BM;
-    ti.rows = min(BM, s_off[lo + 1] - s_off[lo] - mt * BM);
+    ti.m0 = s_off[lo] + mt * TM;
+    ti.rows = min(TM, s_off[lo + 1] - s_off[lo] - mt * TM);
     ti.n0 = nt * (EPI == EPI_SWIGLU_FWD ? 128 : BN);
     ti.kbase = lo * p.b_rows;
     ti.nkb = p.K / BK;
@@ -262,12 +321,14 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, cons
 }
 
 // ------------------------------------------------------------------ kernel
-template <int BN, bool A_MN, bool B_MN, int EPI, bool GROUP_K>
+template <int BN, bool A_MN, bool B_MN, int EPI, bool GROUP_K, bool PAIR = false>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, PAIR>;
   constexpr int S = C::kStages;
   static_assert(EPI != EPI_SWIGLU_FWD || BN == 256, "SwiGLU forward pairs 128 gate + 128 up columns");
+  static_assert(!PAIR || (BN == 256 && !A_MN && !GROUP_K && EPI != EPI_ROUTER),
+                "CTA pairs serve the row-grouped GEMMs with N = 256");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -280,11 +341,17 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   int* s_off = reinterpret_cast<int*>(smem + C::kOffSoff);
   int* s_pre = s_off + 1025;
-  int* s_sel = reinterpret_cast<int*>(smem + C::kOffSel);  // EPI_ROUTER: [128][kRouterKMax]
+  int* s_sel = reinterpret_cast<int*>(smem + C::kOffSel);  // EPI_ROUTER: [4][256] histogram
   uint8_t* s_store = smem + C::kOffStore;                   // TMA-store staging
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = p.E;
+  // PAIR: the two CTAs of a cluster (ranks 0 and 1) share every tile; rank 0 (the
+  // leader) issues the MMAs for both.
+  const uint32_t rank = PAIR ? cluster_rank() : 0;
+  const bool leader = rank == 0;
+  const int tile0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int tstride = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   const int nN = GROUP_K ? p.N / BN
                          : (EPI == EPI_SWIGLU_FWD ? p.N / 128 : (EPI == EPI_ROUTER ? 1 : p.N / BN));
 
@@ -296,22 +363,24 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
       for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
       for (int a = 0; a < 2; ++a) {
         mbar_init(&tfull[a], 1);
-        mbar_init(&tempty[a], EPI == EPI_ROUTER ? 128 : kThreads - 64);
+        mbar_init(&tempty[a], PAIR ? 2 * (kThreads - 64) : (EPI == EPI_ROUTER ? 128 : kThreads - 64));
       }
       mbar_init(drain, 1);
       *s_abort = 0;
       fence_mbar_init();
     }
     __syncwarp();
-    tmem_alloc(s_tmem, C::kTmemCols);
+    if constexpr (PAIR) tmem_alloc_pair(s_tmem, C::kTmemCols);
+    else tmem_alloc(s_tmem, C::kTmemCols);
     tc_fence_before();
   }
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();  // the peer's barriers exist before anyone signals them
   if constexpr (!GROUP_K) {
     if (warp == 1) {  // per-expert tile prefix (E <= 1024: 32 experts per lane)
       const int lo = lane * 32, hi = min(lo + 32, E);
       int s = 0;
-      for (int g = lo; g < hi; ++g) s += ((s_off[g + 1] - s_off[g] + BM - 1) / BM) * nN;
+      for (int g = lo; g < hi; ++g) s += ((s_off[g + 1] - s_off[g] + C::kTileM - 1) / C::kTileM) * nN;
       int incl = s;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -321,7 +390,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
       int run = incl - s;
       for (int g = lo; g < hi; ++g) {
         s_pre[g] = run;
-        run += ((s_off[g + 1] - s_off[g] + BM - 1) / BM) * nN;
+        run += ((s_off[g + 1] - s_off[g] + C::kTileM - 1) / C::kTileM) * nN;
       }
       if (lane == 31) s_pre[E] = incl;
     }
@@ -335,6 +404,15 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
     record_status(p.status, MOE_ERR_TIMEOUT);
     *s_abort = 1;
   };
+  // this CTA's share of tile t (a pair splits the 256 rows 128 / 128)
+  auto decode = [&](int t) {
+    TileInfo ti = decode_tile<BN, EPI, GROUP_K, C::kTileM>(t, p, s_off, s_pre, nN);
+    if constexpr (PAIR) {
+      ti.m0 += BM * (int)rank;
+      ti.rows = max(0, min(BM, ti.rows - BM * (int)rank));
+    }
+    return ti;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -343,16 +421,33 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
       tma_prefetch_desc(&p.tmB);
       uint32_t it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const TileInfo ti = decode_tile<BN, EPI, GROUP_K>(t, p, s_off, s_pre, nN);
+      const uint32_t leader_full = PAIR ? map_to_rank(&full[0], 0) : 0;
+      for (int t = tile0; t < total && ok; t += tstride) {
+        const TileInfo ti = decode(t);
         for (int kb = 0; kb < ti.nkb; ++kb, ++it) {
           if (*s_abort) { ok = false; break; }
           const int s = it % S;
           if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1)) { fail(); ok = false; break; }
           uint8_t* sa = smem + s * C::kStage;
           uint8_t* sb = sa + kABytes;
-          mbar_arrive_expect_tx(&full[s], C::kStage);
           const int kc = kb * BK;
+          if constexpr (PAIR) {
+            // both CTAs' bytes complete on the leader's barrier; only the leader arrives
+            if (leader) mbar_arrive_expect_tx(&full[s], 2 * C::kStage);
+            const uint32_t bar = leader_full + 8 * s;
+            tma_load_2d_pair(sa, &p.tmA, kc, ti.m0, bar);
+            if constexpr (!B_MN) {
+              const int row = ti.kbase + (EPI == EPI_SWIGLU_FWD ? (rank == 0 ? ti.n0 : p.f + ti.n0)
+                                                               : ti.n0 + 128 * (int)rank);
+              tma_load_2d_pair(sb, &p.tmB, kc, row, bar);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 2; ++i)
+                tma_load_2d_pair(sb + i * 8192, &p.tmB, ti.n0 + 128 * (int)rank + 64 * i, ti.kbase + kc, bar);
+            }
+            continue;
+          }
+          mbar_arrive_expect_tx(&full[s], C::kStage);
           if constexpr (!A_MN) {
             tma_load_2d(sa, &p.tmA, kc, ti.m0, &full[s]);
           } else {
@@ -374,7 +469,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
           }
         }
       }
-      if (!ok) {  // let this CTA's loads in flight land before shared memory is released
+      if (!ok && leader) {  // let the loads in flight land before shared memory is released
         for (uint32_t j = it > (uint32_t)S ? it - S : 0; j < it; ++j)
           (void)mbar_wait(&full[j % S], (j / S) & 1);
       }
@@ -383,11 +478,11 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
     // ----------------------------------------------------------------- MMA
     constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)A_MN << 15) |
                                ((uint32_t)B_MN << 16) | ((uint32_t)(BN >> 3) << 17) |
-                               ((uint32_t)(BM >> 4) << 24);
+                               ((uint32_t)(C::kTileM >> 4) << 24);
     uint32_t it = 0, acc_it = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-      const TileInfo ti = decode_tile<BN, EPI, GROUP_K>(t, p, s_off, s_pre, nN);
+    for (int t = tile0; t < total && ok && leader; t += tstride) {
+      const TileInfo ti = decode(t);
       const int acc = acc_it & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&tempty[acc], ((acc_it >> 1) & 1) ^ 1))) {
         if (lane == 0) fail();
@@ -428,19 +523,25 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t ad = A_MN ? sdesc(a0 + k * 2048, 8192, 1024) : sdesc(a0 + k * 32, 16, 1024);
             const uint64_t bd = B_MN ? sdesc(b0 + k * 2048, 8192, 1024) : sdesc(b0 + k * 32, 16, 1024);
-            umma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0);
+            if constexpr (PAIR) umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0);
+            else umma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0);
           }
-          umma_commit(&empty[s]);
+          if constexpr (PAIR) umma_commit_pair(&empty[s]);
+          else umma_commit(&empty[s]);
         }
         __syncwarp();
       }
       if (!ok) break;
-      if (lane == 0) umma_commit(&tfull[acc]);
+      if (lane == 0) {
+        if constexpr (PAIR) umma_commit_pair(&tfull[acc]);
+        else umma_commit(&tfull[acc]);
+      }
       __syncwarp();
       ++acc_it;
     }
     if (!ok && lane == 0) {  // wait for this thread's MMAs before TMEM is freed
-      umma_commit(drain);
+      if constexpr (PAIR) umma_commit_pair(drain);
+      else umma_commit(drain);
       (void)mbar_wait(drain, 0);
     }
   } else {
@@ -456,9 +557,10 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
     uint32_t acc_it = 0;
     // The router epilogue keeps a whole logit row per thread: warps 2..5 only.
     const bool idle = EPI == EPI_ROUTER && half == 1;
-    for (int t = blockIdx.x; t < total && !idle; t += gridDim.x) {
+    const uint32_t leader_tempty = PAIR ? map_to_rank(&tempty[0], 0) : 0;
+    for (int t = tile0; t < total && !idle; t += tstride) {
       if (__any_sync(0xffffffffu, *s_abort)) break;
-      const TileInfo ti = decode_tile<BN, EPI, GROUP_K>(t, p, s_off, s_pre, nN);
+      const TileInfo ti = decode(t);
       const int acc = acc_it & 1;
       const bool valid = row < ti.rows;
       // SwiGLU backward: a and u of the first chunk do not depend on the
@@ -477,7 +579,8 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
       const uint32_t ta = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
       auto release = [&]() {
         tc_fence_before();
-        mbar_arrive(&tempty[acc]);
+        if constexpr (PAIR) mbar_arrive_remote(leader_tempty + 8 * acc);
+        else mbar_arrive(&tempty[acc]);
       };
       if constexpr (EPI == EPI_SWIGLU_FWD) {
         __nv_bfloat16* arow_out = p.out + (int64_t)(ti.m0 + row) * p.ld_out;
@@ -623,35 +726,53 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
           }
         }
         release();
-        int* sel = s_sel + row * kRouterKMax;
+        // block counts and in-block ranks: a per-warp histogram in shared memory
+        // (integer atomics: the counts do not depend on their order) and, for the
+        // rank, a count of the earlier lanes of this warp that picked the same expert
+        int* cnt = s_sel;  // [4 row quarters][256 experts]
+        const int wq = q;  // this warp's rows are 32 wq .. 32 wq + 31 of the tile
+        for (int i = row; i < 4 * 256; i += 128) cnt[i] = 0;
 #pragma unroll
         for (int j = 0; j < kRouterKMax; ++j) {
-          if (j < k) {
-            sel[j] = valid ? topi[j] : -1;
-            if (valid) {
-              p.topk_idx[tok * k + j] = topi[j];
-              p.topk_gate[tok * k + j] = expf(topv[j] - mx) / sum;
+          if (j < k && valid) {
+            p.topk_idx[tok * k + j] = topi[j];
+            p.topk_gate[tok * k + j] = expf(topv[j] - mx) / sum;
+          }
+          if (!valid) topi[j] = -1;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+#pragma unroll
+        for (int j = 0; j < kRouterKMax; ++j)
+          if (j < k && valid) atomicAdd(&cnt[wq * 256 + topi[j]], 1);
+        int rank[kRouterKMax];
+#pragma unroll
+        for (int j = 0; j < kRouterKMax; ++j) rank[j] = 0;
+        for (int l = 0; l < 31; ++l) {
+#pragma unroll
+          for (int j2 = 0; j2 < kRouterKMax; ++j2) {
+            if (j2 >= k) break;
+            const int v = __shfl_sync(0xffffffffu, topi[j2], l);
+            if (l < lane) {
+#pragma unroll
+              for (int j = 0; j < kRouterKMax; ++j) rank[j] += (v == topi[j]);
             }
           }
         }
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (valid) {
-          for (int j = 0; j < k; ++j) {
-            const int e = sel[j];
-            int rank = 0;
-            for (int r2 = 0; r2 < row; ++r2)
-              for (int j2 = 0; j2 < k; ++j2) rank += (s_sel[r2 * kRouterKMax + j2] == e);
-            p.localrank[tok * k + j] = rank;
+#pragma unroll
+          for (int j = 0; j < kRouterKMax; ++j) {
+            if (j < k) {
+              int r = rank[j];
+              for (int w2 = 0; w2 < wq; ++w2) r += cnt[w2 * 256 + topi[j]];
+              p.localrank[tok * k + j] = r;
+            }
           }
         }
         const int blk = ti.m0 / BM;
-        for (int e = row; e < Er; e += 128) {
-          int cnt = 0;
-          for (int r2 = 0; r2 < ti.rows; ++r2)
-            for (int j2 = 0; j2 < k; ++j2) cnt += (s_sel[r2 * kRouterKMax + j2] == e);
-          p.blockcounts[(int64_t)e * p.nb + blk] = cnt;
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");  // s_sel is reused by the next tile
+        for (int e = row; e < Er; e += 128)
+          p.blockcounts[(int64_t)e * p.nb + blk] = cnt[e] + cnt[256 + e] + cnt[512 + e] + cnt[768 + e];
+        asm volatile("bar.sync 1, 128;" ::: "memory");  // the histogram is reused by the next tile
       } else if constexpr (EPI == EPI_ROUTER_DX) {
         // router backward: dx = dl w_router (the accumulator) + the token's k expert rows
         const int k = p.topk;
@@ -757,9 +878,11 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
     if (warp >= 2 && lane == 0) tma_store_wait_all();
   }
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();  // the leader's MMAs read the peer's shared memory and TMEM
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::kTmemCols);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, C::kTmemCols);
+    else tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 
@@ -800,6 +923,38 @@ cudaError_t launch(const GemmParams& p, int64_t tile_bound, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// CTA-pair variant: clusters of 2 CTAs, as many as can be resident at once.
+template <int BN, bool B_MN, int EPI>
+cudaError_t launch_pair(const GemmParams& p, int64_t pair_tile_bound, cudaStream_t st) {
+  auto kern = grouped_gemm_sm100<BN, false, B_MN, EPI, false, true>;
+  constexpr size_t smem = Cfg<BN, true>::kSmem;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static int max_clusters[64] = {0};
+  int dev = 0;
+  if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+  if (dev < 64 && max_clusters[dev] == 0) {
+    cfg.gridDim = dim3(2 * (num_sms() / 2));
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) n = num_sms() / 2;
+    max_clusters[dev] = n;
+  }
+  const int clusters = (int)std::max<int64_t>(1, std::min<int64_t>(pair_tile_bound, dev < 64 ? max_clusters[dev] : num_sms() / 2));
+  cfg.gridDim = dim3(2 * clusters);
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
 GemmParams base_params(const FfnShape& s, const int32_t* offsets, int* status) {
   GemmParams p;
   memset(&p, 0, sizeof(p));
@@ -811,6 +966,16 @@ GemmParams base_params(const FfnShape& s, const int32_t* offsets, int* status) {
 }
 
 int64_t m_tile_bound(const FfnShape& s) { return s.rows / BM + s.E; }
+int64_t pair_tile_bound(const FfnShape& s) { return s.rows / (2 * BM) + s.E; }
+
+// CTA pairs (256-row tiles) pay off when experts hold many rows; with few rows
+// per expert the ragged last tile wastes more.  MOE_B200_PAIR=0/1 forces a mode.
+bool use_pairs(const FfnShape& s) {
+  const char* env = getenv("MOE_B200_PAIR");
+  if (env && env[0] == '0') return false;
+  if (env && env[0] == '1') return true;
+  return s.E > 0 && s.rows / s.E >= 1024;
+}
 
 template <int BN>
 cudaError_t route_tc_bn(const RouteArgs& a, int nb, cudaStream_t st) {
@@ -899,8 +1064,10 @@ cudaError_t ffn_fwd_bf16(const FfnShape& s, const void* x_perm, const int32_t* o
     return cudaErrorInvalidValue;
   p1.N = f; p1.K = d; p1.b_rows = 2 * f;
   p1.out = static_cast<__nv_bfloat16*>(act); p1.ld_out = 3 * f;
-  if ((err = launch<256, false, false, EPI_SWIGLU_FWD, false>(p1, m_tile_bound(s) * (f / 128), st)) != cudaSuccess)
-    return err;
+  const bool pairs = use_pairs(s);
+  err = pairs ? launch_pair<256, false, EPI_SWIGLU_FWD>(p1, pair_tile_bound(s) * (f / 128), st)
+              : launch<256, false, false, EPI_SWIGLU_FWD, false>(p1, m_tile_bound(s) * (f / 128), st);
+  if (err != cudaSuccess) return err;
   // down GEMM: y = h W2^T
   GemmParams p2 = base_params(s, offsets, status);
   if (!tmap(&p2.tmA, actb + 2 * f, f, s.rows, 3 * f, 64, 128) ||
@@ -908,7 +1075,8 @@ cudaError_t ffn_fwd_bf16(const FfnShape& s, const void* x_perm, const int32_t* o
     return cudaErrorInvalidValue;
   p2.N = d; p2.K = f; p2.b_rows = d;
   p2.out = static_cast<__nv_bfloat16*>(y_perm); p2.ld_out = d;
-  return launch<256, false, false, EPI_STORE, false>(p2, m_tile_bound(s) * (d / 256), st);
+  return pairs ? launch_pair<256, false, EPI_STORE>(p2, pair_tile_bound(s) * (d / 256), st)
+               : launch<256, false, false, EPI_STORE, false>(p2, m_tile_bound(s) * (d / 256), st);
 }
 
 cudaError_t ffn_bwd_bf16(const FfnShape& s, const void* dy_perm, const void* x_perm,
@@ -930,8 +1098,10 @@ cudaError_t ffn_bwd_bf16(const FfnShape& s, const void* dy_perm, const void* x_p
     p3.N = f; p3.K = d; p3.b_rows = d;
     p3.out = dadu; p3.ld_out = 2 * f;
     p3.act = actb; p3.ld_act = 3 * f;
-    if ((err = launch<256, false, true, EPI_SWIGLU_BWD, false>(p3, m_tile_bound(s) * (f / 256), st)) != cudaSuccess)
-      return err;
+    const bool pairs = use_pairs(s);
+    err = pairs ? launch_pair<256, true, EPI_SWIGLU_BWD>(p3, pair_tile_bound(s) * (f / 256), st)
+                : launch<256, false, true, EPI_SWIGLU_BWD, false>(p3, m_tile_bound(s) * (f / 256), st);
+    if (err != cudaSuccess) return err;
     // dgrad 2: dx = [da | du] W1[e]
     GemmParams p4 = base_params(s, offsets, status);
     if (!tmap(&p4.tmA, dadu, 2 * f, s.rows, 2 * f, 64, 128) ||
@@ -939,8 +1109,9 @@ cudaError_t ffn_bwd_bf16(const FfnShape& s, const void* dy_perm, const void* x_p
       return cudaErrorInvalidValue;
     p4.N = d; p4.K = 2 * f; p4.b_rows = 2 * f;
     p4.out = static_cast<__nv_bfloat16*>(dx_perm); p4.ld_out = d;
-    if ((err = launch<256, false, true, EPI_STORE, false>(p4, m_tile_bound(s) * (d / 256), st)) != cudaSuccess)
-      return err;
+    err = pairs ? launch_pair<256, true, EPI_STORE>(p4, pair_tile_bound(s) * (d / 256), st)
+                : launch<256, false, true, EPI_STORE, false>(p4, m_tile_bound(s) * (d / 256), st);
+    if (err != cudaSuccess) return err;
   }
   // wgrad 2: dW2[e] = dy^T h   (M = d, N = f, K = the expert's rows)
   GemmParams p5 = base_params(s, offsets, status);

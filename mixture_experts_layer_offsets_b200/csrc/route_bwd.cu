@@ -52,14 +52,15 @@ dlogit_kernel(const float* __restrict__ logits, const int32_t* __restrict__ topk
 
 // dx = dl w_router + sum_j dx_perm[slot_row[t,j]].  A warp takes 4 tokens and
 // walks their rows in 16-byte chunks (one chunk per lane): the router term
-// reuses each w_router chunk for the 4 tokens, dl comes from shared memory,
-// and the k expert rows of each token are gathered with 16-byte loads.
-template <typename T>
+// reuses each w_router chunk for the 4 tokens, dl comes from shared memory.
+// The rows' indices sit in lanes (lane tt*k + j holds token tt's slot j) and
+// all KMAX row chunks of a token are loaded before any is added.
+template <typename T, int TPW, int KMAX>
 __global__ void __launch_bounds__(256)
 dx_kernel(const float* __restrict__ dl, const T* __restrict__ w, const T* __restrict__ dx_perm,
           const int32_t* __restrict__ slot_row, T* __restrict__ dx, int ntok, int d, int E, int k) {
   constexpr int V = Vec16<T>::N;
-  constexpr int TPW = 4;
+  // TPW * k <= 32: the row indices of a warp's tokens fit its lanes
   extern __shared__ float s_dl[];  // [8 warps][TPW][E]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = (blockIdx.x * 8 + warp) * TPW;
@@ -67,6 +68,11 @@ dx_kernel(const float* __restrict__ dl, const T* __restrict__ w, const T* __rest
   for (int i = lane; i < TPW * E; i += 32) {
     const int t = t0 + i / E;
     my[i] = t < ntok ? dl[(int64_t)t * E + i % E] : 0.f;
+  }
+  int myrow = -1;
+  if (lane < TPW * k) {
+    const int t = t0 + lane / k;
+    if (t < ntok) myrow = slot_row[(int64_t)t * k + lane % k];
   }
   __syncwarp();
   const int chunks = d / V;
@@ -88,21 +94,26 @@ dx_kernel(const float* __restrict__ dl, const T* __restrict__ w, const T* __rest
     }
 #pragma unroll
     for (int tt = 0; tt < TPW; ++tt) {
-      const int t = t0 + tt;
-      if (t >= ntok) break;
-#pragma unroll 8
-      for (int j = 0; j < k; ++j) {
-        const int r = __ldg(slot_row + (int64_t)t * k + j);
-        if (r < 0) continue;
-        Vec16<T> v;
-        v.raw = ldg16(dx_perm + (int64_t)r * d + (int64_t)c * V);
+      for (int jb = 0; jb < k; jb += KMAX) {
+        Vec16<T> v[KMAX];
 #pragma unroll
-        for (int i = 0; i < V; ++i) acc[tt][i] += v.get(i);
+        for (int j = 0; j < KMAX; ++j) {
+          const int r = __shfl_sync(0xffffffffu, myrow, (tt * k + jb + j) & 31);
+          v[j].raw = (jb + j < k && r >= 0) ? ldg16(dx_perm + (int64_t)r * d + (int64_t)c * V)
+                                            : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j)
+#pragma unroll
+          for (int i = 0; i < V; ++i) acc[tt][i] += v[j].get(i);
       }
-      Vec16<T> o;
+      const int t = t0 + tt;
+      if (t < ntok) {
+        Vec16<T> o;
 #pragma unroll
-      for (int i = 0; i < V; ++i) o.set(i, acc[tt][i]);
-      stg16(dx + (int64_t)t * d + (int64_t)c * V, o.raw);
+        for (int i = 0; i < V; ++i) o.set(i, acc[tt][i]);
+        stg16(dx + (int64_t)t * d + (int64_t)c * V, o.raw);
+      }
     }
   }
 }
@@ -195,12 +206,13 @@ cudaError_t route_bwd_t(const void* x, const void* w_router, const float* logits
   }
   if (T_ > 0) {
     dlogit_kernel<<<lgrid, 256, 0, st>>>(logits, topk_idx, dgate, dl, nullptr, T_, E, k);
-    const size_t dl_smem = (size_t)8 * 4 * E * sizeof(float);
-    auto dxk = dx_kernel<T>;
+    const int tpw = k <= 8 ? 4 : 1;
+    const size_t dl_smem = (size_t)8 * tpw * E * sizeof(float);
+    auto dxk = k <= 4 ? dx_kernel<T, 4, 4> : (k <= 8 ? dx_kernel<T, 4, 8> : dx_kernel<T, 1, 8>);
     cudaError_t err = cudaFuncSetAttribute(dxk, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)dl_smem);
     if (err != cudaSuccess) return err;
-    dxk<<<(T_ + 31) / 32, 256, dl_smem, st>>>(dl, static_cast<const T*>(w_router),
+    dxk<<<(T_ + 8 * tpw - 1) / (8 * tpw), 256, dl_smem, st>>>(dl, static_cast<const T*>(w_router),
                                               static_cast<const T*>(dx_perm), slot_row,
                                               static_cast<T*>(dx), T_, d, E, k);
     const int tps = (T_ + splits - 1) / splits;
