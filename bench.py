@@ -38,6 +38,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from mixture_experts_layer_offsets_b200 import dist as mdist  # noqa: E402
 from mixture_experts_layer_offsets_b200 import inputs  # noqa: E402
 
 METRIC = "MoE FFN fwd+bwd tokens/s on 1 B200; grouped-GEMM % of tensor-core peak"
@@ -131,7 +132,7 @@ def run_ours(args, rank, world):
         raise SystemExit(f"workload {cfg.name}: dtype {cfg.dtype} is not implemented")
     dev = torch.device("cuda", torch.cuda.current_device())
     capacity = capacity_for(cfg.R, cfg.E, *cfg.padded_cf) if args.capacity_factor and cfg.padded_cf else None
-    inp = inputs.make_inputs(cfg, device=dev, seed=rank)
+    inp = inputs.make_inputs(cfg, device=dev, seed=mdist.rank_seed(0, rank))
     L = MoELayer(cfg.T, cfg.d_model, cfg.E, cfg.top_k, cfg.d_ff, cfg.dtype, dev,
                  dw_dtype="f32", capacity=capacity)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -206,11 +207,7 @@ def run_ours(args, rank, world):
         torch.distributed.barrier()
     clocks = sampler.stop() if sampler else None
     per_step = [a.elapsed_time(b) for a, b in evs]
-    total_ms = sum(per_step)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = mdist.max_over_ranks(sum(per_step), device=dev)
     ms_per_step = total_ms / args.steps
 
     # Phase breakdown: eager steps with CUDA events between the calls; a GPU-side
@@ -303,11 +300,7 @@ def run_e2e(args, L, inp, dev, flush, capacity, world):
         en.record()
         torch.cuda.synchronize()
         times.append(st.elapsed_time(en))
-    ms = sum(times) / n
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = mdist.max_over_ranks(sum(times) / n, device=dev)
     T = inp["x"].shape[0]
     nbytes = hx.numel() * hx.element_size()
     return {"value": round(T * world / (ms / 1e3), 1), "unit": "tokens/s",
