@@ -68,7 +68,7 @@ constexpr int kRouterKMax = 8;  // top-k kept in registers by the router epilogu
 struct GemmParams {
   CUtensorMap tmA;
   CUtensorMap tmB;
-  CUtensorMap tmOut;       // EPI_WGRAD fp32 output: boxes of 32 columns x 16 rows
+  CUtensorMap tmOut;       // output: bf16 boxes of 64 columns x 16 rows, or fp32 (wgrad) 32 x 16
   const int32_t* offsets;
   int E;
   int M;        // GROUP_K: output rows per expert
@@ -99,26 +99,30 @@ struct GemmParams {
   const int32_t* slot_row; // [rows_total][topk]
 };
 
-template <int BN, bool PAIR = false> struct Cfg {
+template <int BN, bool PAIR = false, int EPI = 1> struct Cfg {
   // PAIR: a CTA pair computes a 256-row tile; each CTA holds its 128 A rows and half
   // of the BN B rows (cta_group::2).
   static constexpr uint32_t kBBytes = (PAIR ? BN / 2 : BN) * BK * 2;
   static constexpr uint32_t kStage = kABytes + kBBytes;
-  static constexpr int kStages = PAIR ? 6 : ((BN == 256) ? 4 : 6);
   static constexpr uint32_t kTmemCols = 2 * BN;
   static constexpr int kBoxRows = BN < 128 ? BN : 128;  // rows of one K-major B box
   static constexpr int kTileM = PAIR ? 2 * BM : BM;     // rows of one scheduled tile
+  // TMA-store staging per epilogue warp: bf16 outputs use two 2 KB slots, the fp32
+  // weight gradient one; the router epilogues store directly.
+  static constexpr size_t kStoreBytes =
+      EPI == EPI_WGRAD ? 8 * 2048 : ((EPI == EPI_ROUTER || EPI == EPI_ROUTER_DX) ? 0 : 8 * 4096);
   // shared memory after the stage ring: barriers (256 B), offsets and tile prefix
-  // (2 x 1025 ints), router selections (128 x kRouterKMax ints), then a 1024-aligned
-  // staging area for TMA stores (8 epilogue warps x 16 rows x 128 B)
+  // (2 x 1025 ints), router histogram (128 x kRouterKMax ints), then the 1024-aligned
+  // staging area; as many stages as fit (up to 6)
+  static constexpr size_t kFixed = 1024 + 256 + 2 * 1025 * 4 + 128 * kRouterKMax * 4 + 1024 + kStoreBytes;
+  static constexpr int kStages = (232448 - kFixed) / kStage > 6 ? 6 : (int)((232448 - kFixed) / kStage);
   static constexpr size_t kOffMisc = (size_t)kStages * kStage;
   static constexpr size_t kOffSoff = kOffMisc + 256;
   static constexpr size_t kOffSel = kOffSoff + 2 * 1025 * 4;
   static constexpr size_t kOffStore = (kOffSel + 128 * kRouterKMax * 4 + 1023) & ~size_t(1023);
-  static constexpr size_t kStoreBytes = 8 * 16 * 128;
   static constexpr size_t kSmem = 1024 + kOffStore + kStoreBytes;
-  static_assert(128 * kRouterKMax * 4 >= 4 * 256 * 4, "router histogram fits the selection area");
   static_assert(kSmem <= 232448, "shared memory per CTA");
+  static_assert(128 * kRouterKMax * 4 >= 4 * 256 * 4, "router histogram fits the selection area");
 };
 
 // ------------------------------------------------------------ PTX wrappers
@@ -246,6 +250,9 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* tm, int x, int y
 __device__ __forceinline__ void tma_store_wait_read() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
+__device__ __forceinline__ void tma_store_wait_read_le1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
 __device__ __forceinline__ void tma_store_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
@@ -279,6 +286,41 @@ __device__ __forceinline__ void load_au(const __nv_bfloat16* arow, int col, int 
     av[4 * i] = x.x; av[4 * i + 1] = x.y; av[4 * i + 2] = x.z; av[4 * i + 3] = x.w;
     uv[4 * i] = y.x; uv[4 * i + 1] = y.y; uv[4 * i + 2] = y.z; uv[4 * i + 3] = y.w;
   }
+}
+
+// Store a 16-row x 64-column bf16 box whose rows are held by lanes 16*hh .. 16*hh+15
+// (each lane: its row's 64 values as 32 packed bf16x2 words).  The box is staged in one
+// of the warp's two 2 KB slots with the 128-byte swizzle and written by one TMA store
+// (whole lines, asynchronous).  A box that reaches past the valid rows (the last tile
+// of an expert: the next rows belong to the next expert) is written row by row instead.
+__device__ __forceinline__ void put_box_bf16(uint8_t* wbuf, uint32_t& slot, const CUtensorMap* tm,
+                                             const uint32_t (&v)[32], int hh, int x, int y,
+                                             int valid_rows, __nv_bfloat16* row_dst) {
+  const int lane = threadIdx.x & 31;
+  if (valid_rows <= 0) return;
+  const bool mine = (lane >> 4) == hh;
+  const int r = lane & 15;
+  if (valid_rows < 16) {
+    if (mine && r < valid_rows) {
+      uint4* d = reinterpret_cast<uint4*>(row_dst);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) d[j] = make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    }
+    return;
+  }
+  uint8_t* buf = wbuf + (slot & 1) * 2048;
+  if (lane == 0) tma_store_wait_read_le1();  // the store that used this slot has read it
+  __syncwarp();
+  if (mine) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      *reinterpret_cast<uint4*>(buf + r * 128 + ((j ^ (r & 7)) * 16)) =
+          make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) tma_store_2d(tm, x, y, buf);
+  ++slot;
 }
 
 // ------------------------------------------------------------ tile decode
@@ -324,7 +366,7 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, cons
 template <int BN, bool A_MN, bool B_MN, int EPI, bool GROUP_K, bool PAIR = false>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
-  using C = Cfg<BN, PAIR>;
+  using C = Cfg<BN, PAIR, EPI>;
   constexpr int S = C::kStages;
   static_assert(EPI != EPI_SWIGLU_FWD || BN == 256, "SwiGLU forward pairs 128 gate + 128 up columns");
   static_assert(!PAIR || (BN == 256 && !A_MN && !GROUP_K && EPI != EPI_ROUTER),
@@ -555,6 +597,13 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
     constexpr int kMine = kChunks / 2;
     const int c0 = half * kMine;
     uint32_t acc_it = 0;
+    // this warp's TMA-store staging: two 2 KB slots (bf16 outputs) or one (fp32 wgrad)
+    constexpr size_t kWarpStore = C::kStoreBytes / 8;
+    static_assert(EPI == EPI_ROUTER || EPI == EPI_ROUTER_DX ||
+                      kWarpStore >= (EPI == EPI_WGRAD ? 2048 : 4096),
+                  "staging slots of an epilogue warp fit its share of the store area");
+    uint8_t* wbuf = s_store + (warp - 2) * kWarpStore;
+    uint32_t slot = 0;
     // The router epilogue keeps a whole logit row per thread: warps 2..5 only.
     const bool idle = EPI == EPI_ROUTER && half == 1;
     const uint32_t leader_tempty = PAIR ? map_to_rank(&tempty[0], 0) : 0;
@@ -582,10 +631,14 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
         if constexpr (PAIR) mbar_arrive_remote(leader_tempty + 8 * acc);
         else mbar_arrive(&tempty[acc]);
       };
+      // rows of this CTA's tile that a box starting at tile row b0 may write
+      auto box_valid = [&](int b0) { return max(0, min(16, ti.rows - b0)); };
+      const int grow0 = ti.m0 + q * 32;  // first global row of this warp
       if constexpr (EPI == EPI_SWIGLU_FWD) {
-        __nv_bfloat16* arow_out = p.out + (int64_t)(ti.m0 + row) * p.ld_out;
+        // 64 gate columns per warp (two chunks): a, u, h as three boxes per row half
+        uint32_t pa[32], pu[32], ph[32];
 #pragma unroll
-        for (int ci = 0; ci < kMine; ++ci) {
+        for (int ci = 0; ci < 2; ++ci) {
           const int c = c0 + ci;
           uint32_t g[32], u[32];
           tmem_ld32(ta + c * 32, g);
@@ -593,54 +646,63 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
           tmem_wait_ld();
           tmem_tie(g);
           tmem_tie(u);
-          if (ci == kMine - 1) release();
-          if (valid) {
-            uint32_t pa[16], pu[16], ph[16];
+          if (ci == 1) release();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float a0 = __uint_as_float(g[2 * i]), a1 = __uint_as_float(g[2 * i + 1]);
-              const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
-              pa[i] = pack_bf16(a0, a1);
-              pu[i] = pack_bf16(u0, u1);
-              ph[i] = pack_bf16(a0 * sigmoidf_(a0) * u0, a1 * sigmoidf_(a1) * u1);
-            }
-            const int col = ti.n0 + c * 32;
-            store_64B(arow_out + col, pa);
-            store_64B(arow_out + p.f + col, pu);
-            store_64B(arow_out + 2 * p.f + col, ph);
+          for (int i = 0; i < 16; ++i) {
+            const float a0 = __uint_as_float(g[2 * i]), a1 = __uint_as_float(g[2 * i + 1]);
+            const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+            pa[16 * ci + i] = pack_bf16(a0, a1);
+            pu[16 * ci + i] = pack_bf16(u0, u1);
+            ph[16 * ci + i] = pack_bf16(a0 * sigmoidf_(a0) * u0, a1 * sigmoidf_(a1) * u1);
           }
         }
+        const int col = ti.n0 + c0 * 32;
+        __nv_bfloat16* arow = p.out + (int64_t)(ti.m0 + row) * p.ld_out;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int vr = box_valid(q * 32 + 16 * hh);
+          put_box_bf16(wbuf, slot, &p.tmOut, pa, hh, col, grow0 + 16 * hh, vr, arow + col);
+          put_box_bf16(wbuf, slot, &p.tmOut, pu, hh, p.f + col, grow0 + 16 * hh, vr, arow + p.f + col);
+          put_box_bf16(wbuf, slot, &p.tmOut, ph, hh, 2 * p.f + col, grow0 + 16 * hh, vr, arow + 2 * p.f + col);
+        }
       } else if constexpr (EPI == EPI_STORE) {
-        __nv_bfloat16* orow = p.out + (int64_t)(ti.m0 + row) * p.ld_out + ti.n0;
+        __nv_bfloat16* orow = p.out + (int64_t)(ti.m0 + row) * p.ld_out;
 #pragma unroll
-        for (int ci = 0; ci < kMine; ++ci) {
-          const int c = c0 + ci;
-          uint32_t v[32];
-          tmem_ld32(ta + c * 32, v);
-          tmem_wait_ld();
-          tmem_tie(v);
-          if (ci == kMine - 1) release();
-          if (valid) {
-            uint32_t pk[16];
+        for (int pc = 0; pc < kMine / 2; ++pc) {
+          uint32_t pk[32];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-            store_64B(orow + c * 32, pk);
+          for (int ci = 0; ci < 2; ++ci) {
+            uint32_t v[32];
+            tmem_ld32(ta + (c0 + 2 * pc + ci) * 32, v);
+            tmem_wait_ld();
+            tmem_tie(v);
+            if (pc == kMine / 2 - 1 && ci == 1) release();
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[16 * ci + i] = pack_bf16(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
           }
+          const int col = ti.n0 + (c0 + 2 * pc) * 32;
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh)
+            put_box_bf16(wbuf, slot, &p.tmOut, pk, hh, col, grow0 + 16 * hh,
+                         box_valid(q * 32 + 16 * hh), orow + col);
         }
       } else if constexpr (EPI == EPI_SWIGLU_BWD) {
         __nv_bfloat16* drow = p.out + (int64_t)(ti.m0 + row) * p.ld_out;
 #pragma unroll
-        for (int ci = 0; ci < kMine; ++ci) {
-          const int col = ti.n0 + (c0 + ci) * 32;
-          uint32_t an[16], un[16];
-          if (ci + 1 < kMine && valid) load_au(arow, col + 32, p.f, an, un);  // one chunk ahead
-          uint32_t v[32];
-          tmem_ld32(ta + (c0 + ci) * 32, v);
-          tmem_wait_ld();
-          tmem_tie(v);
-          if (ci == kMine - 1) release();
-          if (valid) {
-            uint32_t pda[16], pdu[16];
+        for (int pc = 0; pc < kMine / 2; ++pc) {
+          uint32_t pda[32], pdu[32];
+#pragma unroll
+          for (int ci = 0; ci < 2; ++ci) {
+            const int cidx = 2 * pc + ci;  // chunk of this warp, 0 .. kMine-1
+            const int col = ti.n0 + (c0 + cidx) * 32;
+            uint32_t an[16], un[16];
+            if (cidx + 1 < kMine && valid) load_au(arow, col + 32, p.f, an, un);  // one chunk ahead
+            uint32_t v[32];
+            tmem_ld32(ta + (c0 + cidx) * 32, v);
+            tmem_wait_ld();
+            tmem_tie(v);
+            if (cidx == kMine - 1) release();
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               float da[2], du[2];
@@ -649,19 +711,24 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
                 const float dh = __uint_as_float(v[2 * i + h]);
                 const float a = h ? bf_hi(av[i]) : bf_lo(av[i]);
                 const float u = h ? bf_hi(uv[i]) : bf_lo(uv[i]);
-                const float s = sigmoidf_(a);
-                da[h] = dh * u * s * (1.f + a * (1.f - s));
-                du[h] = dh * a * s;
+                const float sg = sigmoidf_(a);
+                da[h] = dh * u * sg * (1.f + a * (1.f - sg));
+                du[h] = dh * a * sg;
               }
-              pda[i] = pack_bf16(da[0], da[1]);
-              pdu[i] = pack_bf16(du[0], du[1]);
+              pda[16 * ci + i] = pack_bf16(da[0], da[1]);
+              pdu[16 * ci + i] = pack_bf16(du[0], du[1]);
             }
-            store_64B(drow + col, pda);
-            store_64B(drow + p.f + col, pdu);
-          }
-          if (ci + 1 < kMine) {
+            if (cidx + 1 < kMine) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) { av[i] = an[i]; uv[i] = un[i]; }
+              for (int i = 0; i < 16; ++i) { av[i] = an[i]; uv[i] = un[i]; }
+            }
+          }
+          const int col = ti.n0 + (c0 + 2 * pc) * 32;
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int vr = box_valid(q * 32 + 16 * hh);
+            put_box_bf16(wbuf, slot, &p.tmOut, pda, hh, col, grow0 + 16 * hh, vr, drow + col);
+            put_box_bf16(wbuf, slot, &p.tmOut, pdu, hh, p.f + col, grow0 + 16 * hh, vr, drow + p.f + col);
           }
         }
       } else if constexpr (EPI == EPI_ROUTER) {
@@ -820,7 +887,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
         if (p.out_f32) {
           // fp32: stage 16 rows x 32 columns in shared memory (128-byte swizzle) and
           // write them with one TMA store per box: whole 128-byte lines to HBM.
-          uint8_t* sbuf = s_store + (warp - 2) * 2048;
+          uint8_t* sbuf = wbuf;
 #pragma unroll 1
           for (int ci = 0; ci < kMine; ++ci) {
             uint32_t v[32];
@@ -874,8 +941,8 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
       ++acc_it;
     }
   }
-  if constexpr (EPI == EPI_WGRAD) {
-    if (warp >= 2 && lane == 0) tma_store_wait_all();
+  if constexpr (EPI == EPI_WGRAD || EPI == EPI_STORE || EPI == EPI_SWIGLU_FWD || EPI == EPI_SWIGLU_BWD) {
+    if (warp >= 2 && lane == 0) tma_store_wait_all();  // this warp's stores have left shared memory
   }
   __syncthreads();
   if constexpr (PAIR) cluster_sync();  // the leader's MMAs read the peer's shared memory and TMEM
@@ -916,10 +983,10 @@ template <int BN, bool A_MN, bool B_MN, int EPI, bool GROUP_K>
 cudaError_t launch(const GemmParams& p, int64_t tile_bound, cudaStream_t st) {
   auto kern = grouped_gemm_sm100<BN, A_MN, B_MN, EPI, GROUP_K>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)Cfg<BN>::kSmem);
+                                         (int)Cfg<BN, false, EPI>::kSmem);
   if (err != cudaSuccess) return err;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tile_bound, num_sms()));
-  kern<<<grid, kThreads, Cfg<BN>::kSmem, st>>>(p);
+  kern<<<grid, kThreads, Cfg<BN, false, EPI>::kSmem, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -927,7 +994,7 @@ cudaError_t launch(const GemmParams& p, int64_t tile_bound, cudaStream_t st) {
 template <int BN, bool B_MN, int EPI>
 cudaError_t launch_pair(const GemmParams& p, int64_t pair_tile_bound, cudaStream_t st) {
   auto kern = grouped_gemm_sm100<BN, false, B_MN, EPI, false, true>;
-  constexpr size_t smem = Cfg<BN, true>::kSmem;
+  constexpr size_t smem = Cfg<BN, true, EPI>::kSmem;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
@@ -982,7 +1049,7 @@ cudaError_t route_tc_bn(const RouteArgs& a, int nb, cudaStream_t st) {
   GemmParams p;
   memset(&p, 0, sizeof(p));
   if (!tmap(&p.tmA, a.x, a.d, a.T, a.d, 64, 128) ||
-      !tmap(&p.tmB, a.w_router, a.d, a.E, a.d, 64, Cfg<BN>::kBoxRows))
+      !tmap(&p.tmB, a.w_router, a.d, a.E, a.d, 64, Cfg<BN, false, EPI_ROUTER>::kBoxRows))
     return cudaErrorInvalidValue;
   p.offsets = nullptr;
   p.E = 1;
@@ -1064,6 +1131,7 @@ cudaError_t ffn_fwd_bf16(const FfnShape& s, const void* x_perm, const int32_t* o
     return cudaErrorInvalidValue;
   p1.N = f; p1.K = d; p1.b_rows = 2 * f;
   p1.out = static_cast<__nv_bfloat16*>(act); p1.ld_out = 3 * f;
+  if (!tmap(&p1.tmOut, act, 3 * f, s.rows, 3 * f, 64, 16)) return cudaErrorInvalidValue;
   const bool pairs = use_pairs(s);
   err = pairs ? launch_pair<256, false, EPI_SWIGLU_FWD>(p1, pair_tile_bound(s) * (f / 128), st)
               : launch<256, false, false, EPI_SWIGLU_FWD, false>(p1, m_tile_bound(s) * (f / 128), st);
@@ -1075,6 +1143,7 @@ cudaError_t ffn_fwd_bf16(const FfnShape& s, const void* x_perm, const int32_t* o
     return cudaErrorInvalidValue;
   p2.N = d; p2.K = f; p2.b_rows = d;
   p2.out = static_cast<__nv_bfloat16*>(y_perm); p2.ld_out = d;
+  if (!tmap(&p2.tmOut, y_perm, d, s.rows, d, 64, 16)) return cudaErrorInvalidValue;
   return pairs ? launch_pair<256, false, EPI_STORE>(p2, pair_tile_bound(s) * (d / 256), st)
                : launch<256, false, false, EPI_STORE, false>(p2, m_tile_bound(s) * (d / 256), st);
 }
@@ -1097,6 +1166,7 @@ cudaError_t ffn_bwd_bf16(const FfnShape& s, const void* dy_perm, const void* x_p
       return cudaErrorInvalidValue;
     p3.N = f; p3.K = d; p3.b_rows = d;
     p3.out = dadu; p3.ld_out = 2 * f;
+    if (!tmap(&p3.tmOut, dadu, 2 * f, s.rows, 2 * f, 64, 16)) return cudaErrorInvalidValue;
     p3.act = actb; p3.ld_act = 3 * f;
     const bool pairs = use_pairs(s);
     err = pairs ? launch_pair<256, true, EPI_SWIGLU_BWD>(p3, pair_tile_bound(s) * (f / 256), st)
@@ -1109,6 +1179,7 @@ cudaError_t ffn_bwd_bf16(const FfnShape& s, const void* dy_perm, const void* x_p
       return cudaErrorInvalidValue;
     p4.N = d; p4.K = 2 * f; p4.b_rows = 2 * f;
     p4.out = static_cast<__nv_bfloat16*>(dx_perm); p4.ld_out = d;
+    if (!tmap(&p4.tmOut, dx_perm, d, s.rows, d, 64, 16)) return cudaErrorInvalidValue;
     err = pairs ? launch_pair<256, true, EPI_STORE>(p4, pair_tile_bound(s) * (d / 256), st)
                 : launch<256, false, true, EPI_STORE, false>(p4, m_tile_bound(s) * (d / 256), st);
     if (err != cudaSuccess) return err;
