@@ -43,9 +43,12 @@ from mixture_experts_layer_offsets_b200 import inputs  # noqa: E402
 
 METRIC = "MoE FFN fwd+bwd tokens/s on 1 B200; grouped-GEMM % of tensor-core peak"
 FLUSH_BYTES = 256 << 20
-# kernel launches of one step, per C-ABI call (bf16 path)
+# kernel launches of one step, per C-ABI call (bf16 path; MXFP8 adds the operand
+# quantisations: 4 for the weight copies, 2 in the forward FFN call, 6 in the backward)
 LAUNCHES = {"route": 3, "permute": 1, "ffn_fwd": 2, "combine": 1, "combine_bwd": 1,
             "ffn_bwd": 4, "route_bwd": 4, "padded_dispatch": 2}
+LAUNCHES_MX = {"quantize_w": 4, "ffn_fwd": 4, "ffn_bwd": 10}
+FP8_OVER_BF16 = 2.0   # nominal dense tensor-core ratio (4.5 / 2.25 PFLOP/s)
 
 
 def _peaks():
@@ -64,6 +67,10 @@ def _workload_desc(cfg, capacity):
          "routing": "skewed (logit bias std 2)" if cfg.bias_std else "near-uniform random",
          "l2": "flushed between timed steps (256 MiB write, outside the timed events)",
          "weight_grad_dtype": "fp32"}
+    if cfg.dtype == "mxfp8":
+        d["operands"] = ("MXFP8 (E4M3 + E8M0 per 32 along K) for all six expert GEMMs; bf16 "
+                         "activations; FP32 master weights quantised to four MXFP8 copies "
+                         "every step (inside the timed step)")
     if capacity:
         d["layout"] = f"padded capacity C={capacity} (overflow dropped)"
     else:
@@ -128,8 +135,9 @@ def run_ours(args, rank, world):
     cfg = inputs.CONFIGS[args.workload]
     if args.tokens:
         cfg = inputs.shrink(cfg, name=f"{cfg.name}@T{args.tokens}", T=args.tokens)
-    if cfg.dtype not in ("f32", "bf16"):
-        raise SystemExit(f"workload {cfg.name}: dtype {cfg.dtype} is not implemented")
+    if args.dtype and args.dtype != cfg.dtype:
+        cfg = inputs.shrink(cfg, name=f"{cfg.name}@{args.dtype}", dtype=args.dtype)
+    mxfp8 = cfg.dtype == "mxfp8"
     dev = torch.device("cuda", torch.cuda.current_device())
     capacity = capacity_for(cfg.R, cfg.E, *cfg.padded_cf) if args.capacity_factor and cfg.padded_cf else None
     inp = inputs.make_inputs(cfg, device=dev, seed=mdist.rank_seed(0, rank))
@@ -138,7 +146,9 @@ def run_ours(args, rank, world):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     x, wr, b, w1, w2, dout = (inp[k] for k in ("x", "w_router", "bias", "w1", "w2", "dout"))
-    phases = ["route", "dispatch", "ffn_fwd", "combine", "combine_bwd", "ffn_bwd", "route_bwd"]
+    phases = ["quantize_w", "route", "dispatch", "ffn_fwd", "combine", "combine_bwd", "ffn_bwd",
+              "route_bwd"]
+    fdt = L.ffn_dtype
 
     def step(ev=None):
         def mark(i):
@@ -147,28 +157,31 @@ def run_ours(args, rank, world):
         s, dt = L.shape, L.cdtype
         from mixture_experts_layer_offsets_b200 import capi
         mark(0)
+        if mxfp8:
+            L.quantize_weights(w1, w2)
+        mark(1)
         capi.moe_route(s, dt, x, wr, b, L.logits, L.topk_idx, L.topk_gate, L.counts, L.offsets,
                        L.slot_row, L.ws)
-        mark(1)
+        mark(2)
         if capacity:
             capi.moe_padded_dispatch(s, dt, capacity, x, L.topk_idx, L.slot_row, L.offsets,
                                      L.x_perm, L.pad_row, L.offsets_pad)
         else:
             capi.moe_permute(s, dt, x, L.slot_row, L.x_perm, L.perm_src)
-        mark(2)
-        capi.moe_grouped_ffn_fwd(s, dt, L.rows, L.x_perm, L.ffn_offsets, w1, w2, L.act, L.y_perm,
-                                 L.ws)
         mark(3)
-        capi.moe_combine(s, dt, L.y_perm, L.row_map, L.topk_gate, L.out)
+        capi.moe_grouped_ffn_fwd(s, fdt, L.rows, L.x_perm, L.ffn_offsets, w1, w2, L.act, L.y_perm,
+                                 L.ws, mx=L.mx)
         mark(4)
-        capi.moe_combine_bwd(s, dt, dout, L.y_perm, L.row_map, L.topk_gate, L.dy_perm, L.dgate)
+        capi.moe_combine(s, dt, L.y_perm, L.row_map, L.topk_gate, L.out)
         mark(5)
-        capi.moe_grouped_ffn_bwd(s, dt, L.rows, L.dy_perm, L.x_perm, L.act, L.ffn_offsets, w1, w2,
-                                 L.dx_perm, L.dw1, L.dw2, capi.MOE_F32, L.ws)
+        capi.moe_combine_bwd(s, dt, dout, L.y_perm, L.row_map, L.topk_gate, L.dy_perm, L.dgate)
         mark(6)
+        capi.moe_grouped_ffn_bwd(s, fdt, L.rows, L.dy_perm, L.x_perm, L.act, L.ffn_offsets, w1,
+                                 w2, L.dx_perm, L.dw1, L.dw2, capi.MOE_F32, L.ws, mx=L.mx)
+        mark(7)
         capi.moe_route_bwd(s, dt, x, wr, L.logits, L.topk_idx, L.dgate, L.dx_perm, L.row_map,
                            L.dx, L.dw_router, L.ws)
-        mark(7)
+        mark(8)
 
     for _ in range(args.warmup):
         step()
@@ -214,7 +227,7 @@ def run_ours(args, rank, world):
     # delay before each step lets the host enqueue the whole step first, so the
     # events see device time only.
     nph = min(args.steps, 10)
-    pevs = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(nph)]
+    pevs = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in range(nph)]
     for i in range(nph):
         flush.zero_()
         torch.cuda._sleep(3_000_000)
@@ -235,10 +248,19 @@ def run_ours(args, rank, world):
     rows = L.rows
     gemm_flop = 18.0 * cfg.R * cfg.d_model * cfg.d_ff   # algorithmic (dropless) FLOPs per step
     achieved = gemm_flop / (gemm_ms / 1e3) / 1e12
-    peak = pk["bf16_tflops"] if cfg.dtype == "bf16" else None
-    launches_per_step = (LAUNCHES["route"] + (LAUNCHES["padded_dispatch"] if capacity else LAUNCHES["permute"])
-                         + LAUNCHES["ffn_fwd"] + LAUNCHES["combine"] + LAUNCHES["combine_bwd"]
-                         + LAUNCHES["ffn_bwd"] + LAUNCHES["route_bwd"])
+    if cfg.dtype == "bf16":
+        peak, peak_kind = pk["bf16_tflops"], f"bf16_tflops burst, {pk_kind}"
+    elif mxfp8:
+        peak = pk["bf16_tflops"] * FP8_OVER_BF16
+        peak_kind = (f"bf16_tflops burst ({pk_kind}) x {FP8_OVER_BF16} nominal fp8/bf16 ratio; "
+                     "the ffn phases include the activation quantisations")
+    else:
+        peak, peak_kind = None, "fp32 CUDA-core path: no tensor-core peak"
+    lt = dict(LAUNCHES, **(LAUNCHES_MX if mxfp8 else {"quantize_w": 0}))
+    launches_per_step = (lt["quantize_w"] + lt["route"]
+                         + (lt["padded_dispatch"] if capacity else lt["permute"])
+                         + lt["ffn_fwd"] + lt["combine"] + lt["combine_bwd"]
+                         + lt["ffn_bwd"] + lt["route_bwd"])
     line = {
         "metric": METRIC, "value": round(tokens_per_s, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
@@ -249,7 +271,7 @@ def run_ours(args, rank, world):
             "bound": "tensor", "kernel": "grouped GEMM (tcgen05), all 6 launches of a step",
             "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4) if peak else None,
-            "peak_kind": f"bf16_tflops burst, {pk_kind}", "traffic": None,
+            "peak_kind": peak_kind, "traffic": None,
             "algorithmic_flop_per_step": gemm_flop, "gemm_ms_per_step": round(gemm_ms, 4),
             "rows_computed": rows,
         },
@@ -262,7 +284,11 @@ def run_ours(args, rank, world):
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(cfg, budget_s=args.cpu_seconds)
+        line["cpu_baseline"] = (cpu_baseline(cfg, budget_s=args.cpu_seconds) if not mxfp8 else
+                                {"value": None, "unit": "tokens/s", "kind": "oracle", "cores": None,
+                                 "sample": "not run: the MXFP8 oracle quantises the full FP32 "
+                                           "expert weights (2.4e9 values) on every call, which "
+                                           "alone exceeds the CPU time budget"})
     return line
 
 
@@ -380,6 +406,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--dtype", default=None, choices=["f32", "bf16", "mxfp8"],
+                    help="run the workload's shapes at another compute dtype")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override T (smaller cases for profiling); not a bench line")
     args = ap.parse_args()

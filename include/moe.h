@@ -41,7 +41,11 @@
  *     workspace status word; read it with moe_get_device_status.  No C++
  *     exception crosses this interface.
  *   - dtype: MOE_F32 (fp32 everywhere, CUDA-core GEMMs), MOE_BF16 (bf16
- *     activations and weights, fp32 accumulation, tcgen05 tensor cores).
+ *     activations and weights, fp32 accumulation, tcgen05 tensor cores),
+ *     MOE_MXFP8 (grouped FFN calls only: bf16 activations, MXFP8 GEMM operands
+ *     with block-scaled tcgen05 MMAs, fp32 accumulation and weight gradients;
+ *     the route, permute and combine calls of such a layer take MOE_BF16, and
+ *     its workspace is sized with MOE_MXFP8).
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -150,6 +154,25 @@ moe_status moe_route_noalloc(moe_shape shape, int dtype, const void* x, const vo
 moe_status moe_permute(moe_shape shape, int dtype, const void* x, const int32_t* slot_row,
                        void* x_perm, int32_t* perm_src, void* stream);
 
+/* MXFP8 copies of the expert weights for dtype MOE_MXFP8, made from their FP32
+ * masters with mxfp8_quantize (typically once per optimizer step).  One pair of
+ * (E4M3 codes, E8M0 scales) per GEMM orientation, with d % 128 == 0, f % 128 == 0:
+ *   w1_q,  w1_s   W1 [E*2f, d] in blocks along d (axis 0):     q [E*2f, d], s [E*2f, d/32]
+ *   w1t_q, w1t_s  W1 in 32-row blocks along 2f (axis 1):       q [E*2f, d], s [E*2f/32, d]
+ *   w2_q,  w2_s   W2 [E*d, f] in blocks along f (axis 0):      q [E*d, f],  s [E*d, f/32]
+ *   w2t_q, w2t_s  W2 in 32-row blocks along d (axis 1):        q [E*d, f],  s [E*d/32, f]
+ * The forward GEMMs use w1 and w2, the input-gradient GEMMs w2t and w1t. */
+typedef struct moe_mx_weights {
+  const uint8_t* w1_q;
+  const uint8_t* w1_s;
+  const uint8_t* w1t_q;
+  const uint8_t* w1t_s;
+  const uint8_t* w2_q;
+  const uint8_t* w2_s;
+  const uint8_t* w2t_q;
+  const uint8_t* w2t_s;
+} moe_mx_weights;
+
 /* ---- a4: grouped SwiGLU FFN, forward -------------------------------------
  * [kongchang] routing section: a device-scheduled grouped GEMM handles the
  * uneven per-expert shapes; the tile scheduler reads `offsets` from device
@@ -161,8 +184,13 @@ moe_status moe_permute(moe_shape shape, int dtype, const void* x, const int32_t*
  * x_perm:   [rows, d];  w1: [E, 2f, d] (gate rows then up rows);
  * w2:       [E, d, f];  act_saved: [rows, 3f] = a | u | h (saved for bwd);
  * y_perm:   [rows, d].  Rows outside every expert segment are not written.
- * MOE_BF16 needs d % 256 == 0 and f % 128 == 0 (tensor-core tiles).
- * mx must be NULL (MXFP8 GEMMs are not part of this version). */
+ * MOE_BF16 needs d % 256 == 0 and f % 256 == 0 (tensor-core tiles); mx is NULL.
+ * MOE_MXFP8 (kongchang, boundary-conditions section: MXFP8 cuts GEMM time and
+ * saved-activation bytes): x_perm, act_saved and y_perm stay bf16; mx is a HOST
+ * pointer to a moe_mx_weights whose members are device pointers (w1, w2 are not
+ * read and may be NULL); x and h are quantised
+ * along their rows in the workspace and the GEMMs run block-scaled E4M3 x E4M3
+ * with fp32 accumulation.  Needs d % 128 == 0 and f % 128 == 0. */
 moe_status moe_grouped_ffn_fwd(moe_shape shape, int dtype, int64_t rows, const void* x_perm,
                                const int32_t* offsets, const void* w1, const void* w2,
                                const void* mx, void* act_saved, void* y_perm, void* ws,
@@ -193,8 +221,11 @@ moe_status moe_combine_bwd(moe_shape shape, int dtype, const void* dout, const v
  * An expert with no rows gets dW1[e] = dW2[e] = 0 (dW is overwritten).
  * dy_perm, x_perm: [rows, d]; act_saved: [rows, 3f] from the forward;
  * dx_perm: [rows, d]; dw1: [E, 2f, d]; dw2: [E, d, f] of type dw_dtype
- * (MOE_F32 or MOE_BF16; MOE_F32 only when dtype is MOE_F32).
- * Uses 2*f*rows elements of scratch in `ws` for [da | du]. */
+ * (MOE_F32 or MOE_BF16; MOE_F32 only when dtype is MOE_F32 or MOE_MXFP8).
+ * Uses 2*f*rows elements of scratch in `ws` for [da | du].
+ * MOE_MXFP8: dy_perm, x_perm, act_saved, dx_perm bf16; mx as for the forward;
+ * dy and [da | du] are quantised along their rows for the dgrad GEMMs, and dy, h,
+ * [da | du], x in 32-row blocks restarting at every expert for the wgrad GEMMs. */
 moe_status moe_grouped_ffn_bwd(moe_shape shape, int dtype, int64_t rows, const void* dy_perm,
                                const void* x_perm, const void* act_saved,
                                const int32_t* offsets, const void* w1, const void* w2,
@@ -225,8 +256,8 @@ moe_status moe_route_bwd(moe_shape shape, int dtype, const void* x, const void* 
  * axis 1: blocks of 32 consecutive rows within each column, restarting at
  *   every segment start seg_offsets[g] (device int32 [nseg+1], or NULL for one
  *   segment [0, rows)); a segment's last partial block is zero-padded.
- *   scale: u8 [S, K] with S = sum_g ceil(len_g / 32), segment by segment;
- *   the buffer must hold rows/32 + nseg + 1 rows (K % 16 == 0).
+ *   scale: u8 [S, K] with S = sum_g ceil(len_g / 32), segment by segment
+ *   (S <= rows/32 + nseg, a bound that needs no device data); K % 16 == 0.
  * q: u8 [rows, K].  Bytes are exact (bit-for-bit with the rule above). */
 moe_status mxfp8_quantize(int64_t rows, int64_t K, int src_dtype, const void* src, int axis,
                           const int32_t* seg_offsets, int nseg, uint8_t* q, uint8_t* scale,

@@ -33,6 +33,12 @@ class moe_shape(ctypes.Structure):
                 ("top_k", ctypes.c_int32), ("d_ff", ctypes.c_int32)]
 
 
+class moe_mx_weights(ctypes.Structure):
+    """MXFP8 copies of the expert weights (device pointers), see include/moe.h."""
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("w1_q", "w1_s", "w1t_q", "w1t_s", "w2_q", "w2_s", "w2t_q", "w2t_s")]
+
+
 _P = ctypes.c_void_p
 _I = ctypes.c_int
 _I64 = ctypes.c_int64
@@ -84,6 +90,8 @@ def _ptr(t) -> int | None:
         return None
     if isinstance(t, int):
         return t
+    if isinstance(t, ctypes.Structure):     # host struct passed by address
+        return ctypes.addressof(t)
     return t.data_ptr()
 
 

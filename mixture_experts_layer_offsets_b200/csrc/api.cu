@@ -60,10 +60,23 @@ size_t ws_need(const moe_shape& s, int dtype, int64_t rows) {
   size_t need = route_ws_bytes(s.T, s.E, s.top_k);
   need = std::max(need, route_bwd_ws_bytes(s.T, s.d_model, s.E));
   need = std::max(need, ffn_bwd_ws_bytes(fs, dtype != MOE_F32));
+  if (dtype == MOE_MXFP8) need = std::max(need, ffn_mx_ws_bytes(fs));
   return kStatusBytes + align256(need);
 }
 
 inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+// host copy of a moe_mx_weights: every pointer present and 16-byte aligned
+moe_status mx_weights_ok(const void* mx, MxWeights& w) {
+  if (!mx) return MOE_ERR_INVALID_ARG;
+  moe_mx_weights m;
+  memcpy(&m, mx, sizeof(m));
+  w = MxWeights{m.w1_q, m.w1_s, m.w1t_q, m.w1t_s, m.w2_q, m.w2_s, m.w2t_q, m.w2t_s};
+  const void* all[] = {m.w1_q, m.w1_s, m.w1t_q, m.w1t_s, m.w2_q, m.w2_s, m.w2t_q, m.w2t_s};
+  for (const void* q : all)
+    if (!q || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
 
 }  // namespace
 
@@ -120,13 +133,25 @@ moe_status moe_grouped_ffn_fwd(moe_shape s, int dtype, int64_t rows, const void*
                                size_t ws_bytes, void* stream) {
   moe_status st = shape_ok(s);
   if (st != MOE_OK) return st;
-  if (dtype == MOE_MXFP8 || mx) return MOE_ERR_UNSUPPORTED;
-  if (!dtype_act_ok(dtype) || rows < 0 || rows >= ((int64_t)1 << 31)) return MOE_ERR_INVALID_ARG;
+  if (rows < 0 || rows >= ((int64_t)1 << 31)) return MOE_ERR_INVALID_ARG;
+  FfnShape fs{s.d_model, s.E, s.d_ff, rows};
+  cudaStream_t cs = as_stream(stream);
+  if (dtype == MOE_MXFP8) {
+    MxWeights w;
+    moe_status vs = mx_weights_ok(mx, w);
+    if (vs != MOE_OK) return vs;
+    if (s.d_model % 128 || s.d_ff % 128) return MOE_ERR_UNSUPPORTED;
+    if (!ptrs_ok(offsets, ws)) return MOE_ERR_INVALID_ARG;
+    if (rows > 0 && !ptrs_ok(x_perm, act_saved, y_perm)) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < kStatusBytes + ffn_mx_ws_bytes(fs)) return MOE_ERR_INVALID_ARG;
+    return cuda_status(ffn_fwd_mx(fs, x_perm, offsets, w, act_saved, y_perm, scratch(ws),
+                                  status_word(ws), cs));
+  }
+  if (mx) return MOE_ERR_INVALID_ARG;
+  if (!dtype_act_ok(dtype)) return MOE_ERR_INVALID_ARG;
   if (!ptrs_ok(offsets, w1, w2, ws)) return MOE_ERR_INVALID_ARG;
   if (rows > 0 && !ptrs_ok(x_perm, act_saved, y_perm)) return MOE_ERR_INVALID_ARG;
   (void)ws_bytes;
-  FfnShape fs{s.d_model, s.E, s.d_ff, rows};
-  cudaStream_t cs = as_stream(stream);
   if (dtype == MOE_F32)
     return cuda_status(ffn_fwd_f32(fs, static_cast<const float*>(x_perm), offsets,
                                    static_cast<const float*>(w1), static_cast<const float*>(w2),
@@ -167,8 +192,23 @@ moe_status moe_grouped_ffn_bwd(moe_shape s, int dtype, int64_t rows, const void*
                                int dw_dtype, void* ws, size_t ws_bytes, void* stream) {
   moe_status st = shape_ok(s);
   if (st != MOE_OK) return st;
-  if (dtype == MOE_MXFP8 || mx) return MOE_ERR_UNSUPPORTED;
-  if (!dtype_act_ok(dtype) || rows < 0 || rows >= ((int64_t)1 << 31)) return MOE_ERR_INVALID_ARG;
+  if (rows < 0 || rows >= ((int64_t)1 << 31)) return MOE_ERR_INVALID_ARG;
+  if (dtype == MOE_MXFP8) {
+    MxWeights w;
+    moe_status vs = mx_weights_ok(mx, w);
+    if (vs != MOE_OK) return vs;
+    if (s.d_model % 128 || s.d_ff % 128) return MOE_ERR_UNSUPPORTED;
+    if (dw_dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
+    if (!ptrs_ok(offsets, dw1, dw2, ws)) return MOE_ERR_INVALID_ARG;
+    if (rows > 0 && !ptrs_ok(dy_perm, x_perm, act_saved, dx_perm)) return MOE_ERR_INVALID_ARG;
+    FfnShape fsm{s.d_model, s.E, s.d_ff, rows};
+    if (ws_bytes < kStatusBytes + ffn_mx_ws_bytes(fsm)) return MOE_ERR_INVALID_ARG;
+    return cuda_status(ffn_bwd_mx(fsm, dy_perm, x_perm, act_saved, offsets, w, dx_perm,
+                                  static_cast<float*>(dw1), static_cast<float*>(dw2), scratch(ws),
+                                  status_word(ws), as_stream(stream)));
+  }
+  if (mx) return MOE_ERR_INVALID_ARG;
+  if (!dtype_act_ok(dtype)) return MOE_ERR_INVALID_ARG;
   if (dw_dtype != MOE_F32 && dw_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
   if (dtype == MOE_F32 && dw_dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
   if (!ptrs_ok(offsets, w1, w2, dw1, dw2, ws)) return MOE_ERR_INVALID_ARG;

@@ -97,14 +97,28 @@ struct GemmParams {
   int split;
   // EPI_ROUTER_DX
   const int32_t* slot_row; // [rows_total][topk]
+  // MXFP8 operands: E8M0 scales, one byte per 32 K elements.
+  //   K-major operand (blocks along its rows):      s[row][K / 32]        (ld = K / 32)
+  //   MN-major operand (blocks of 32 K rows):       s[block row][MN]      (ld = MN extent)
+  //   GROUP_K operands: block rows restart at every group (segment) start.
+  const uint8_t* sfa;
+  const uint8_t* sfb;
+  int64_t ld_sfa, ld_sfb;
 };
 
-template <int BN, bool PAIR = false, int EPI = 1> struct Cfg {
+template <int BN, bool PAIR = false, int EPI = 1, bool FP8 = false> struct Cfg {
   // PAIR: a CTA pair computes a 256-row tile; each CTA holds its 128 A rows and half
   // of the BN B rows (cta_group::2).
-  static constexpr uint32_t kBBytes = (PAIR ? BN / 2 : BN) * BK * 2;
-  static constexpr uint32_t kStage = kABytes + kBBytes;
-  static constexpr uint32_t kTmemCols = 2 * BN;
+  // FP8 (MXFP8): 128 E4M3 elements (128 bytes) of K per stage, plus the stage's scale
+  // atoms for A (512 B) and B (BN / 128 x 512 B); TMEM columns 2 BN .. 2 BN + 7 hold the
+  // scales of the stage being multiplied.
+  static constexpr int kBKe = FP8 ? 128 : BK;  // K elements per stage
+  static constexpr uint32_t kBBytes = (PAIR ? BN / 2 : BN) * 128;
+  static constexpr uint32_t kSfBytes = FP8 ? 512 + (BN / 128) * 512 : 0;
+  static constexpr uint32_t kStage = kABytes + kBBytes + kSfBytes;
+  static_assert(kStage % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
+  static constexpr uint32_t kSfCol = 2 * BN;  // FP8: scale columns in TMEM
+  static constexpr uint32_t kTmemCols = FP8 ? 512 : 2 * BN;
   static constexpr int kBoxRows = BN < 128 ? BN : 128;  // rows of one K-major B box
   static constexpr int kTileM = PAIR ? 2 * BM : BM;     // rows of one scheduled tile
   // TMA-store staging per epilogue warp: bf16 outputs use two 2 KB slots, the fp32
@@ -144,6 +158,26 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
           smem_u32(bar))
       : "memory");
 }
+// ---- MXFP8: block-scaled E4M3 MMA (K = 32 per instruction, one E8M0 scale per row per
+// 32 K) and the shared-memory -> TMEM copy of a 128-row x 4-block scale atom.
+__device__ __forceinline__ void umma_mxf8(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                          uint32_t accum, uint32_t tsfa, uint32_t tsfb) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accum), "r"(tsfa), "r"(tsfb));
+}
+// 32 rows x 16 bytes from shared memory, broadcast to the four 32-lane quarters.
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc_src) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc_src)
+               : "memory");
+}
+// descriptor of a 512-byte scale atom: 32 rows of 16 bytes, no swizzle (8-row groups 128 B apart)
+__device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)(128 >> 4) << 16) |
+         ((uint64_t)(128 >> 4) << 32) | (1ull << 46);
+}
+
 // ---- CTA-pair (cta_group::2) forms
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -328,7 +362,7 @@ struct TileInfo {
   int g, m0, n0, rows, nkb, kbase, klast;
 };
 
-template <int BN, int EPI, bool GROUP_K, int TM = BM>
+template <int BN, int EPI, bool GROUP_K, int TM = BM, int KE = BK>
 __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, const int* s_off,
                                                 const int* s_pre, int nN) {
   TileInfo ti;
@@ -341,8 +375,8 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, cons
     ti.rows = BM;
     const int k0 = s_off[ti.g], kg = s_off[ti.g + 1] - k0;
     ti.kbase = k0;
-    ti.nkb = (kg + BK - 1) / BK;
-    ti.klast = kg - (ti.nkb - 1) * BK;
+    ti.nkb = (kg + KE - 1) / KE;
+    ti.klast = kg - (ti.nkb - 1) * KE;
   } else {
     int lo = 0, hi = p.E - 1;
     while (lo < hi) {  // last expert whose tile prefix is <= t (skips empty experts)
@@ -354,21 +388,26 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, cons
     const int mt = local / nN, nt = local - mt * nN;
     ti.m0 = s_off[lo] + mt * TM;
     ti.rows = min(TM, s_off[lo + 1] - s_off[lo] - mt * TM);
-    ti.n0 = nt * (EPI == EPI_SWIGLU_FWD ? 128 : BN);
+    ti.n0 = nt * (EPI == EPI_SWIGLU_FWD ? BN / 2 : BN);
     ti.kbase = lo * p.b_rows;
-    ti.nkb = p.K / BK;
-    ti.klast = BK;
+    ti.nkb = p.K / KE;
+    ti.klast = KE;
   }
   return ti;
 }
 
 // ------------------------------------------------------------------ kernel
-template <int BN, bool A_MN, bool B_MN, int EPI, bool GROUP_K, bool PAIR = false>
+template <int BN, bool A_MN, bool B_MN, int EPI, bool GROUP_K, bool PAIR = false, bool FP8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
-  using C = Cfg<BN, PAIR, EPI>;
+  using C = Cfg<BN, PAIR, EPI, FP8>;
+  static_assert(!FP8 || (BN == 128 && !PAIR), "MXFP8 tiles: 128 x 128, single CTA");
+  // epilogue warps 6..9 idle when a thread must hold a whole row (router) or the
+  // SwiGLU gate/up halves are 64 columns wide (BN = 128)
+  constexpr bool kHalfIdle = EPI == EPI_ROUTER || (EPI == EPI_SWIGLU_FWD && BN == 128);
   constexpr int S = C::kStages;
-  static_assert(EPI != EPI_SWIGLU_FWD || BN == 256, "SwiGLU forward pairs 128 gate + 128 up columns");
+  static_assert(EPI != EPI_SWIGLU_FWD || BN == 256 || (FP8 && BN == 128),
+                "SwiGLU forward pairs BN/2 gate with BN/2 up columns (128 + 128, or 64 + 64 for MXFP8)");
   static_assert(!PAIR || (BN == 256 && !A_MN && !GROUP_K && EPI != EPI_ROUTER),
                 "CTA pairs serve the row-grouped GEMMs with N = 256");
   extern __shared__ uint8_t smem_raw[];
@@ -395,7 +434,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
   const int tile0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int tstride = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   const int nN = GROUP_K ? p.N / BN
-                         : (EPI == EPI_SWIGLU_FWD ? p.N / 128 : (EPI == EPI_ROUTER ? 1 : p.N / BN));
+                         : (EPI == EPI_SWIGLU_FWD ? p.N / (BN / 2) : (EPI == EPI_ROUTER ? 1 : p.N / BN));
 
   for (int g = threadIdx.x; g <= E; g += kThreads)
     s_off[g] = p.offsets ? p.offsets[g]
@@ -405,7 +444,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
       for (int s = 0; s < S; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
       for (int a = 0; a < 2; ++a) {
         mbar_init(&tfull[a], 1);
-        mbar_init(&tempty[a], PAIR ? 2 * (kThreads - 64) : (EPI == EPI_ROUTER ? 128 : kThreads - 64));
+        mbar_init(&tempty[a], PAIR ? 2 * (kThreads - 64) : (kHalfIdle ? 128 : kThreads - 64));
       }
       mbar_init(drain, 1);
       *s_abort = 0;
@@ -437,6 +476,24 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
       if (lane == 31) s_pre[E] = incl;
     }
   }
+  if constexpr (GROUP_K && FP8) {
+    if (warp == 1) {  // first 32-row scale block of each group (blocks restart at group starts)
+      const int lo = lane * 32, hi = min(lo + 32, E);
+      int s = 0;
+      for (int g = lo; g < hi; ++g) s += (s_off[g + 1] - s_off[g] + 31) / 32;
+      int incl = s;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+      }
+      int run = incl - s;
+      for (int g = lo; g < hi; ++g) {
+        s_pre[g] = run;
+        run += (s_off[g + 1] - s_off[g] + 31) / 32;
+      }
+    }
+  }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
@@ -448,7 +505,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
   };
   // this CTA's share of tile t (a pair splits the 256 rows 128 / 128)
   auto decode = [&](int t) {
-    TileInfo ti = decode_tile<BN, EPI, GROUP_K, C::kTileM>(t, p, s_off, s_pre, nN);
+    TileInfo ti = decode_tile<BN, EPI, GROUP_K, C::kTileM, C::kBKe>(t, p, s_off, s_pre, nN);
     if constexpr (PAIR) {
       ti.m0 += BM * (int)rank;
       ti.rows = max(0, min(BM, ti.rows - BM * (int)rank));
@@ -456,7 +513,107 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
     return ti;
   };
 
-  if (warp == 0) {
+  if (warp == 0 && FP8) {
+    // ---------------------------------------------------- producer (MXFP8)
+    // The warp writes the stage's scale atoms (scale of row mn, block kb at byte
+    // (mn % 32) * 16 + (mn / 32) * 4 + kb), then lane 0 issues the TMA loads.
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tmA);
+      tma_prefetch_desc(&p.tmB);
+    }
+    uint32_t it = 0;
+    bool ok = true;
+    for (int t = tile0; t < total && ok; t += tstride) {
+      const TileInfo ti = decode(t);
+      for (int kb = 0; kb < ti.nkb; ++kb, ++it) {
+        if (__any_sync(0xffffffffu, *s_abort)) { ok = false; break; }
+        const int s = it % S;
+        bool w = true;
+        if (lane == 0) w = mbar_wait(&empty[s], ((it / S) & 1) ^ 1);
+        if (!__shfl_sync(0xffffffffu, w, 0)) {
+          if (lane == 0) fail();
+          ok = false;
+          break;
+        }
+        uint8_t* sa = smem + s * C::kStage;
+        uint8_t* sb = sa + kABytes;
+        uint8_t* sf = sb + C::kBBytes;
+        const int kc = kb * C::kBKe;  // first K element of the stage
+        // blocks of this stage that lie inside the group's K range (GROUP_K tails)
+        const int nblk = GROUP_K ? min(4, (ti.klast + 31) / 32 + 4 * (ti.nkb - 1 - kb)) : 4;
+        const int nblk_ok = GROUP_K ? (kb == ti.nkb - 1 ? (ti.klast + 31) / 32 : 4) : nblk;
+        auto atom = [&](uint8_t* dst, const uint8_t* sfp, int64_t ld, bool mn_major, int mn0,
+                        int rows_limit, int64_t blk0) {
+          uint32_t wd[4];
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int mn = mn0 + lane + 32 * g;
+            uint32_t v = 0x7F7F7F7Fu;  // scale 1.0 where no data is multiplied
+            if (!mn_major) {
+              if (mn < rows_limit) v = __ldg(reinterpret_cast<const uint32_t*>(sfp + (int64_t)mn * ld + blk0));
+            } else {
+              v = 0;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const uint32_t b = j < nblk_ok ? __ldg(sfp + (blk0 + j) * ld + mn) : 0x7Fu;
+                v |= b << (8 * j);
+              }
+            }
+            wd[g] = v;
+          }
+          *reinterpret_cast<uint4*>(dst + lane * 16) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+        };
+        (void)nblk;
+        if constexpr (GROUP_K) {
+          const int64_t blk = s_pre[ti.g] + kc / 32;  // both operands: segmented block rows
+          atom(sf, p.sfa, p.ld_sfa, true, ti.m0, 0, blk);
+          atom(sf + 512, p.sfb, p.ld_sfb, true, ti.n0, 0, blk);
+        } else {
+          if constexpr (!A_MN) atom(sf, p.sfa, p.ld_sfa, false, ti.m0, p.rows_total, kc / 32);
+          else atom(sf, p.sfa, p.ld_sfa, true, ti.m0, 0, (ti.kbase + kc) / 32);
+          if constexpr (!B_MN) {
+            // B rows: the expert's weight rows (SwiGLU: 64 gate rows, then 64 up rows)
+            if constexpr (EPI == EPI_SWIGLU_FWD) {
+              // rows n0 .. n0+63 and f + n0 .. f + n0 + 63: lane + 32 g covers them in order
+              uint32_t wd[4];
+#pragma unroll
+              for (int g = 0; g < 4; ++g) {
+                const int nn = lane + 32 * g;
+                const int row = ti.kbase + (nn < 64 ? ti.n0 + nn : p.f + ti.n0 + nn - 64);
+                wd[g] = __ldg(reinterpret_cast<const uint32_t*>(p.sfb + (int64_t)row * p.ld_sfb + kc / 32));
+              }
+              *reinterpret_cast<uint4*>(sf + 512 + lane * 16) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+            } else {
+              atom(sf + 512, p.sfb, p.ld_sfb, false, ti.kbase + ti.n0, 0x7FFFFFFF, kc / 32);
+            }
+          } else {
+            atom(sf + 512, p.sfb, p.ld_sfb, true, ti.n0, 0, (ti.kbase + kc) / 32);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[s], kABytes + C::kBBytes);
+          if constexpr (!A_MN) tma_load_2d(sa, &p.tmA, kc, ti.m0, &full[s]);
+          else tma_load_2d(sa, &p.tmA, ti.m0, ti.kbase + kc, &full[s]);
+          if constexpr (!B_MN) {
+            if constexpr (EPI == EPI_SWIGLU_FWD) {
+              tma_load_2d(sb, &p.tmB, kc, ti.kbase + ti.n0, &full[s]);
+              tma_load_2d(sb + 64 * 128, &p.tmB, kc, ti.kbase + p.f + ti.n0, &full[s]);
+            } else {
+              tma_load_2d(sb, &p.tmB, kc, ti.kbase + ti.n0, &full[s]);
+            }
+          } else {
+            tma_load_2d(sb, &p.tmB, ti.n0, ti.kbase + kc, &full[s]);
+          }
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      for (uint32_t j = it > (uint32_t)S ? it - S : 0; j < it; ++j)
+        (void)mbar_wait(&full[j % S], (j / S) & 1);
+    }
+  } else if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&p.tmA);
@@ -545,13 +702,17 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
         uint8_t* sa = smem + s * C::kStage;
         uint8_t* sb = sa + kABytes;
         if constexpr (GROUP_K) {
-          if (kb == ti.nkb - 1 && ti.klast < BK) {
-            // Rows [klast, 64) of every 64-row box hold the next expert's tokens: zero them.
-            const int nz = (BK - ti.klast) * 8;  // 16-byte pieces per box
-            constexpr int kBoxes = 2 + BN / 64;
+          if (kb == ti.nkb - 1 && ti.klast < C::kBKe) {
+            // Rows [klast, K rows of a box) of every box hold the next expert's tokens:
+            // zero them.  bf16 boxes are 64 M/N x 64 K rows (8 KB), fp8 boxes 128 x 128 (16 KB).
+            constexpr int kBoxRowsK = C::kBKe;
+            constexpr int kBoxBytes = kBoxRowsK * 128;
+            constexpr int kABoxes = kABytes / kBoxBytes;
+            constexpr int kBoxes = kABoxes + C::kBBytes / kBoxBytes;
+            const int nz = (kBoxRowsK - ti.klast) * 8;  // 16-byte pieces per box
             for (int i = lane; i < nz * kBoxes; i += 32) {
               const int box = i / nz, rem = i - box * nz;
-              uint8_t* base = box < 2 ? sa + box * 8192 : sb + (box - 2) * 8192;
+              uint8_t* base = box < kABoxes ? sa + box * kBoxBytes : sb + (box - kABoxes) * kBoxBytes;
               *reinterpret_cast<uint4*>(base + (ti.klast + rem / 8) * 128 + (rem & 7) * 16) =
                   make_uint4(0, 0, 0, 0);
             }
@@ -559,7 +720,25 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
           }
         }
         __syncwarp();
-        if (lane == 0) {
+        if (FP8 && lane == 0) {
+          // scales of this stage -> TMEM, then four K = 32 block-scaled MMAs
+          const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sb), f0 = smem_u32(sb + C::kBBytes);
+          const uint32_t tsf = tmem_base + C::kSfCol;
+          tmem_cp_sf(tsf, sf_desc(f0));
+          tmem_cp_sf(tsf + 4, sf_desc(f0 + 512));
+          constexpr uint32_t idesc_mx = ((uint32_t)A_MN << 15) | ((uint32_t)B_MN << 16) |
+                                        ((uint32_t)(BN >> 3) << 17) | (1u << 23) |
+                                        ((uint32_t)(BM >> 4) << 24);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t ad = A_MN ? sdesc(a0 + k * 4096, 16384, 1024) : sdesc(a0 + k * 32, 16, 1024);
+            const uint64_t bd = B_MN ? sdesc(b0 + k * 4096, 16384, 1024) : sdesc(b0 + k * 32, 16, 1024);
+            const uint32_t id = idesc_mx | ((uint32_t)k << 4) | ((uint32_t)k << 29);
+            umma_mxf8(d_tmem, ad, bd, id, (kb | k) != 0, tsf | ((uint32_t)k << 30),
+                      (tsf + 4) | ((uint32_t)k << 30));
+          }
+          umma_commit(&empty[s]);
+        } else if (lane == 0) {
           const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sb);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
@@ -593,7 +772,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     const int row = q * 32 + lane;
-    constexpr int kChunks = (EPI == EPI_SWIGLU_FWD ? 128 : BN) / 32;
+    constexpr int kChunks = (EPI == EPI_SWIGLU_FWD ? BN / 2 : BN) / 32;
     constexpr int kMine = kChunks / 2;
     const int c0 = half * kMine;
     uint32_t acc_it = 0;
@@ -605,7 +784,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
     uint8_t* wbuf = s_store + (warp - 2) * kWarpStore;
     uint32_t slot = 0;
     // The router epilogue keeps a whole logit row per thread: warps 2..5 only.
-    const bool idle = EPI == EPI_ROUTER && half == 1;
+    const bool idle = kHalfIdle && half == 1;
     const uint32_t leader_tempty = PAIR ? map_to_rank(&tempty[0], 0) : 0;
     for (int t = tile0; t < total && !idle; t += tstride) {
       if (__any_sync(0xffffffffu, *s_abort)) break;
@@ -642,7 +821,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
           const int c = c0 + ci;
           uint32_t g[32], u[32];
           tmem_ld32(ta + c * 32, g);
-          tmem_ld32(ta + 128 + c * 32, u);
+          tmem_ld32(ta + BN / 2 + c * 32, u);
           tmem_wait_ld();
           tmem_tie(g);
           tmem_tie(u);
@@ -967,13 +1146,16 @@ cudaError_t get_encode() {
 }
 
 // 2-D tensor map over [outer, inner] with row stride `ld` elements, 128-byte swizzle.
+// Elements are bf16, fp32 (f32) or bytes (u8: E4M3 codes).
 bool tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
-          uint32_t box_inner, uint32_t box_outer, bool f32 = false) {
+          uint32_t box_inner, uint32_t box_outer, bool f32 = false, bool u8 = false) {
   const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {ld * (f32 ? 4 : 2)};
+  const cuuint64_t strides[1] = {ld * (u8 ? 1 : (f32 ? 4 : 2))};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t es[2] = {1, 1};
-  return g_encode(tm, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+  const CUtensorMapDataType dt = u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                    : (f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+  return g_encode(tm, dt, 2,
                   const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -987,6 +1169,18 @@ cudaError_t launch(const GemmParams& p, int64_t tile_bound, cudaStream_t st) {
   if (err != cudaSuccess) return err;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tile_bound, num_sms()));
   kern<<<grid, kThreads, Cfg<BN, false, EPI>::kSmem, st>>>(p);
+  return cudaGetLastError();
+}
+
+// MXFP8 variant: 128 x 128 tiles of E4M3 operands with E8M0 block scales.
+template <bool A_MN, bool B_MN, int EPI, bool GROUP_K>
+cudaError_t launch_mx(const GemmParams& p, int64_t tile_bound, cudaStream_t st) {
+  auto kern = grouped_gemm_sm100<128, A_MN, B_MN, EPI, GROUP_K, false, true>;
+  constexpr size_t smem = Cfg<128, false, EPI, true>::kSmem;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tile_bound, num_sms()));
+  kern<<<grid, kThreads, smem, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -1205,6 +1399,174 @@ cudaError_t ffn_bwd_bf16(const FfnShape& s, const void* dy_perm, const void* x_p
   p6.ld_out = d; p6.out_group = (int64_t)2 * f * d;
   if (dw_f32 && !tmap(&p6.tmOut, dw1, d, (uint64_t)E * 2 * f, d, 32, 16, true)) return cudaErrorInvalidValue;
   return launch<256, true, true, EPI_WGRAD, true>(p6, (int64_t)E * (2 * f / 128) * (d / 256), st);
+}
+
+
+// ---------------------------------------------------------------- MXFP8 FFN
+// Activations arrive and leave in bf16; each GEMM operand is quantised along that
+// GEMM's K right before it is used (forward: x and h along their rows; dgrad: dy and
+// [da|du] along their rows, the weights along their rows of K via the moe_mx_weights
+// copies; wgrad: dy, h, [da|du] and x in 32-row blocks that restart at every expert's
+// first row).  Accumulation is fp32; outputs are bf16 (dW fp32).
+namespace {
+
+struct MxLayout {
+  size_t qx0, sx0, qh0, sh0;                         // forward
+  size_t dadu, qdy0, sdy0, qda0, sda0;               // backward, dgrad operands
+  size_t qdy1, sdy1, qh1, sh1, qda1, sda1, qx1, sx1;  // backward, wgrad operands
+  size_t fwd_bytes, bwd_bytes;
+};
+
+MxLayout mx_layout(const FfnShape& s) {
+  const size_t R = (size_t)s.rows, d = s.d, f = s.f;
+  const size_t sb = R / 32 + s.E + 1;  // 32-row blocks of a segmented (per expert) axis
+  MxLayout L;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { const size_t at = o; o += align256(bytes); return at; };
+  L.qx0 = take(R * d); L.sx0 = take(R * d / 32); L.qh0 = take(R * f); L.sh0 = take(R * f / 32);
+  L.fwd_bytes = o;
+  o = 0;
+  L.dadu = take(R * 2 * f * 2);
+  L.qdy0 = take(R * d); L.sdy0 = take(R * d / 32);
+  L.qda0 = take(R * 2 * f); L.sda0 = take(R * 2 * f / 32);
+  L.qdy1 = take(R * d); L.sdy1 = take(sb * d);
+  L.qh1 = take(R * f); L.sh1 = take(sb * f);
+  L.qda1 = take(R * 2 * f); L.sda1 = take(sb * 2 * f);
+  L.qx1 = take(R * d); L.sx1 = take(sb * d);
+  L.bwd_bytes = o;
+  return L;
+}
+
+GemmParams mx_params(const FfnShape& s, const int32_t* offsets, int* status) {
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.offsets = offsets;
+  p.E = s.E;
+  p.f = s.f;
+  p.status = status;
+  p.rows_total = (int)s.rows;
+  return p;
+}
+
+}  // namespace
+
+size_t ffn_mx_ws_bytes(const FfnShape& s) {
+  const MxLayout L = mx_layout(s);
+  return std::max(L.fwd_bytes, L.bwd_bytes);
+}
+
+cudaError_t ffn_fwd_mx(const FfnShape& s, const void* x_perm, const int32_t* offsets,
+                       const MxWeights& w, void* act, void* y_perm, void* scratch, int* status,
+                       cudaStream_t st) {
+  if (s.rows == 0) return cudaSuccess;
+  cudaError_t err = get_encode();
+  if (err != cudaSuccess) return err;
+  const int d = s.d, f = s.f, E = s.E;
+  const int64_t R = s.rows;
+  uint8_t* ws = static_cast<uint8_t*>(scratch);
+  const MxLayout L = mx_layout(s);
+  const __nv_bfloat16* actb = static_cast<const __nv_bfloat16*>(act);
+  // x along d; gate/up GEMM with the SwiGLU epilogue
+  if ((err = mxfp8_launch_ld(R, d, d, true, x_perm, 0, nullptr, 0, ws + L.qx0, ws + L.sx0, st)) != cudaSuccess)
+    return err;
+  GemmParams p1 = mx_params(s, offsets, status);
+  if (!tmap(&p1.tmA, ws + L.qx0, d, R, d, 128, 128, false, true) ||
+      !tmap(&p1.tmB, w.w1_q, d, (uint64_t)E * 2 * f, d, 128, 64, false, true) ||
+      !tmap(&p1.tmOut, act, 3 * f, R, 3 * f, 64, 16))
+    return cudaErrorInvalidValue;
+  p1.sfa = ws + L.sx0; p1.ld_sfa = d / 32;
+  p1.sfb = w.w1_s; p1.ld_sfb = d / 32;
+  p1.N = f; p1.K = d; p1.b_rows = 2 * f;
+  p1.out = static_cast<__nv_bfloat16*>(act); p1.ld_out = 3 * f;
+  if ((err = launch_mx<false, false, EPI_SWIGLU_FWD, false>(p1, m_tile_bound(s) * (f / 64), st)) != cudaSuccess)
+    return err;
+  // h along f; down GEMM
+  if ((err = mxfp8_launch_ld(R, f, 3 * f, true, actb + 2 * f, 0, nullptr, 0, ws + L.qh0, ws + L.sh0, st)) != cudaSuccess)
+    return err;
+  GemmParams p2 = mx_params(s, offsets, status);
+  if (!tmap(&p2.tmA, ws + L.qh0, f, R, f, 128, 128, false, true) ||
+      !tmap(&p2.tmB, w.w2_q, f, (uint64_t)E * d, f, 128, 128, false, true) ||
+      !tmap(&p2.tmOut, y_perm, d, R, d, 64, 16))
+    return cudaErrorInvalidValue;
+  p2.sfa = ws + L.sh0; p2.ld_sfa = f / 32;
+  p2.sfb = w.w2_s; p2.ld_sfb = f / 32;
+  p2.N = d; p2.K = f; p2.b_rows = d;
+  p2.out = static_cast<__nv_bfloat16*>(y_perm); p2.ld_out = d;
+  return launch_mx<false, false, EPI_STORE, false>(p2, m_tile_bound(s) * (d / 128), st);
+}
+
+cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_perm, const void* act,
+                       const int32_t* offsets, const MxWeights& w, void* dx_perm, float* dw1,
+                       float* dw2, void* scratch, int* status, cudaStream_t st) {
+  cudaError_t err = get_encode();
+  if (err != cudaSuccess) return err;
+  const int d = s.d, f = s.f, E = s.E;
+  const int64_t R = s.rows;
+  const uint64_t Rtm = std::max<int64_t>(R, 1);
+  uint8_t* ws = static_cast<uint8_t*>(scratch);
+  const MxLayout L = mx_layout(s);
+  const __nv_bfloat16* actb = static_cast<const __nv_bfloat16*>(act);
+  __nv_bfloat16* dadu = reinterpret_cast<__nv_bfloat16*>(ws + L.dadu);
+  if (R > 0) {
+    // dgrad 1: dh = dy W2 (dy along d, W2 along its d rows), SwiGLU backward -> [da | du]
+    if ((err = mxfp8_launch_ld(R, d, d, true, dy_perm, 0, nullptr, 0, ws + L.qdy0, ws + L.sdy0, st)) != cudaSuccess)
+      return err;
+    GemmParams p3 = mx_params(s, offsets, status);
+    if (!tmap(&p3.tmA, ws + L.qdy0, d, R, d, 128, 128, false, true) ||
+        !tmap(&p3.tmB, w.w2t_q, f, (uint64_t)E * d, f, 128, 128, false, true) ||
+        !tmap(&p3.tmOut, dadu, 2 * f, R, 2 * f, 64, 16))
+      return cudaErrorInvalidValue;
+    p3.sfa = ws + L.sdy0; p3.ld_sfa = d / 32;
+    p3.sfb = w.w2t_s; p3.ld_sfb = f;
+    p3.N = f; p3.K = d; p3.b_rows = d;
+    p3.out = dadu; p3.ld_out = 2 * f;
+    p3.act = actb; p3.ld_act = 3 * f;
+    if ((err = launch_mx<false, true, EPI_SWIGLU_BWD, false>(p3, m_tile_bound(s) * (f / 128), st)) != cudaSuccess)
+      return err;
+    // dgrad 2: dx = [da | du] W1 ([da | du] along 2f, W1 along its 2f rows)
+    if ((err = mxfp8_launch_ld(R, 2 * f, 2 * f, true, dadu, 0, nullptr, 0, ws + L.qda0, ws + L.sda0, st)) != cudaSuccess)
+      return err;
+    GemmParams p4 = mx_params(s, offsets, status);
+    if (!tmap(&p4.tmA, ws + L.qda0, 2 * f, R, 2 * f, 128, 128, false, true) ||
+        !tmap(&p4.tmB, w.w1t_q, d, (uint64_t)E * 2 * f, d, 128, 128, false, true) ||
+        !tmap(&p4.tmOut, dx_perm, d, R, d, 64, 16))
+      return cudaErrorInvalidValue;
+    p4.sfa = ws + L.sda0; p4.ld_sfa = 2 * f / 32;
+    p4.sfb = w.w1t_s; p4.ld_sfb = d;
+    p4.N = d; p4.K = 2 * f; p4.b_rows = 2 * f;
+    p4.out = static_cast<__nv_bfloat16*>(dx_perm); p4.ld_out = d;
+    if ((err = launch_mx<false, true, EPI_STORE, false>(p4, m_tile_bound(s) * (d / 128), st)) != cudaSuccess)
+      return err;
+    // wgrad operands along the token axis, blocks restarting at each expert
+    if ((err = mxfp8_launch_ld(R, d, d, true, dy_perm, 1, offsets, E, ws + L.qdy1, ws + L.sdy1, st)) != cudaSuccess ||
+        (err = mxfp8_launch_ld(R, f, 3 * f, true, actb + 2 * f, 1, offsets, E, ws + L.qh1, ws + L.sh1, st)) != cudaSuccess ||
+        (err = mxfp8_launch_ld(R, 2 * f, 2 * f, true, dadu, 1, offsets, E, ws + L.qda1, ws + L.sda1, st)) != cudaSuccess ||
+        (err = mxfp8_launch_ld(R, d, d, true, x_perm, 1, offsets, E, ws + L.qx1, ws + L.sx1, st)) != cudaSuccess)
+      return err;
+  }
+  // wgrad 2: dW2[e] = dy^T h  (M = d, N = f)
+  GemmParams p5 = mx_params(s, offsets, status);
+  if (!tmap(&p5.tmA, ws + L.qdy1, d, Rtm, d, 128, 128, false, true) ||
+      !tmap(&p5.tmB, ws + L.qh1, f, Rtm, f, 128, 128, false, true) ||
+      !tmap(&p5.tmOut, dw2, f, (uint64_t)E * d, f, 32, 16, true))
+    return cudaErrorInvalidValue;
+  p5.sfa = ws + L.sdy1; p5.ld_sfa = d;
+  p5.sfb = ws + L.sh1; p5.ld_sfb = f;
+  p5.M = d; p5.N = f;
+  p5.out_f32 = dw2; p5.ld_out = f; p5.out_group = (int64_t)d * f;
+  if ((err = launch_mx<true, true, EPI_WGRAD, true>(p5, (int64_t)E * (d / 128) * (f / 128), st)) != cudaSuccess)
+    return err;
+  // wgrad 1: dW1[e] = [da | du]^T x  (M = 2f, N = d)
+  GemmParams p6 = mx_params(s, offsets, status);
+  if (!tmap(&p6.tmA, ws + L.qda1, 2 * f, Rtm, 2 * f, 128, 128, false, true) ||
+      !tmap(&p6.tmB, ws + L.qx1, d, Rtm, d, 128, 128, false, true) ||
+      !tmap(&p6.tmOut, dw1, d, (uint64_t)E * 2 * f, d, 32, 16, true))
+    return cudaErrorInvalidValue;
+  p6.sfa = ws + L.sda1; p6.ld_sfa = 2 * f;
+  p6.sfb = ws + L.sx1; p6.ld_sfb = d;
+  p6.M = 2 * f; p6.N = d;
+  p6.out_f32 = dw1; p6.ld_out = d; p6.out_group = (int64_t)2 * f * d;
+  return launch_mx<true, true, EPI_WGRAD, true>(p6, (int64_t)E * (2 * f / 128) * (d / 128), st);
 }
 
 }  // namespace moe

@@ -66,6 +66,10 @@ cudaError_t route_bwd_launch(bool bf16, const void* x, const void* w_router, con
 cudaError_t mxfp8_launch(int64_t rows, int64_t K, bool src_bf16, const void* src, int axis,
                          const int32_t* seg_offsets, int nseg, uint8_t* q, uint8_t* scale,
                          cudaStream_t st);
+// the same with a source row stride of `ld` elements (q and scale stay dense)
+cudaError_t mxfp8_launch_ld(int64_t rows, int64_t K, int64_t ld, bool src_bf16, const void* src,
+                            int axis, const int32_t* seg_offsets, int nseg, uint8_t* q,
+                            uint8_t* scale, cudaStream_t st);
 
 // ---------------------------------------------------------- grouped FFN
 struct FfnShape {
@@ -89,6 +93,18 @@ cudaError_t ffn_bwd_bf16(const FfnShape& s, const void* dy_perm, const void* x_p
                          const void* act, const int32_t* offsets, const void* w1, const void* w2,
                          void* dx_perm, void* dw1, void* dw2, bool dw_f32, void* scratch,
                          int* status, cudaStream_t st);
+
+// MXFP8 path: E4M3 operands with E8M0 scales (see include/moe.h, moe_mx_weights)
+struct MxWeights {
+  const uint8_t *w1_q, *w1_s, *w1t_q, *w1t_s, *w2_q, *w2_s, *w2t_q, *w2t_s;
+};
+size_t ffn_mx_ws_bytes(const FfnShape& s);
+cudaError_t ffn_fwd_mx(const FfnShape& s, const void* x_perm, const int32_t* offsets,
+                       const MxWeights& w, void* act, void* y_perm, void* scratch, int* status,
+                       cudaStream_t st);
+cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_perm, const void* act,
+                       const int32_t* offsets, const MxWeights& w, void* dx_perm, float* dw1,
+                       float* dw2, void* scratch, int* status, cudaStream_t st);
 
 int num_sms();
 

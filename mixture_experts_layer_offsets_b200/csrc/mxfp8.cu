@@ -49,15 +49,15 @@ __device__ __forceinline__ uint32_t e4m3_pair(float hi, float lo) {
 // axis 0: a quad of lanes covers one 32-element block, 8 elements per lane.
 template <typename T>
 __global__ void __launch_bounds__(256)
-mx_rows_kernel(const T* __restrict__ src, int64_t nblocks, uint8_t* __restrict__ q,
-               uint8_t* __restrict__ scale) {
+mx_rows_kernel(const T* __restrict__ src, int64_t nblocks, int64_t kblocks, int64_t ld,
+               uint8_t* __restrict__ q, uint8_t* __restrict__ scale) {
   const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t blk = g >> 2;
   const int part = (int)(g & 3);
   const bool live = blk < nblocks;
   float v[8];
   if (live) {
-    const T* p = src + blk * 32 + part * 8;
+    const T* p = src + (blk / kblocks) * ld + (blk % kblocks) * 32 + part * 8;
     if constexpr (sizeof(T) == 2) {
       Vec16<T> a;
       a.raw = ldg16(p);
@@ -92,7 +92,7 @@ mx_rows_kernel(const T* __restrict__ src, int64_t nblocks, uint8_t* __restrict__
 // axis 1: one thread = one 32-row block x 8 columns; blocks restart at segments.
 template <typename T>
 __global__ void __launch_bounds__(128)
-mx_cols_kernel(const T* __restrict__ src, int64_t rows, int64_t K,
+mx_cols_kernel(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
                const int32_t* __restrict__ seg, int nseg, uint8_t* __restrict__ q,
                uint8_t* __restrict__ scale) {
   __shared__ int32_t s_pre[1026];   // block prefix per segment
@@ -125,7 +125,7 @@ mx_cols_kernel(const T* __restrict__ src, int64_t rows, int64_t K,
 #pragma unroll
     for (int i = 0; i < 8; ++i) amax[i] = 0.f;
     for (int64_t r = r0; r < r1; ++r) {
-      const T* p = src + r * K + col;
+      const T* p = src + r * ld + col;
 #pragma unroll
       for (int i = 0; i < 8; ++i) amax[i] = fmaxf(amax[i], fabsf(to_f32(p[i])));
     }
@@ -140,7 +140,7 @@ mx_cols_kernel(const T* __restrict__ src, int64_t rows, int64_t K,
     }
     *reinterpret_cast<uint2*>(scale + (int64_t)rb * K + col) = make_uint2(sb[0], sb[1]);
     for (int64_t r = r0; r < r1; ++r) {
-      const T* p = src + r * K + col;
+      const T* p = src + r * ld + col;
       float v[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) v[i] = to_f32(p[i]) * mul[i];
@@ -154,9 +154,9 @@ mx_cols_kernel(const T* __restrict__ src, int64_t rows, int64_t K,
 
 }  // namespace
 
-cudaError_t mxfp8_launch(int64_t rows, int64_t K, bool src_bf16, const void* src, int axis,
-                         const int32_t* seg_offsets, int nseg, uint8_t* q, uint8_t* scale,
-                         cudaStream_t st) {
+cudaError_t mxfp8_launch_ld(int64_t rows, int64_t K, int64_t ld, bool src_bf16, const void* src,
+                            int axis, const int32_t* seg_offsets, int nseg, uint8_t* q,
+                            uint8_t* scale, cudaStream_t st) {
   if (rows == 0 || K == 0) return cudaSuccess;
   if (axis == 0) {
     const int64_t nblocks = rows * K / 32;
@@ -164,10 +164,10 @@ cudaError_t mxfp8_launch(int64_t rows, int64_t K, bool src_bf16, const void* src
     const int grid = (int)((threads + 255) / 256);
     if (src_bf16)
       mx_rows_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(src),
-                                                          nblocks, q, scale);
+                                                          nblocks, K / 32, ld, q, scale);
     else
-      mx_rows_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(src), nblocks, q,
-                                                  scale);
+      mx_rows_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(src), nblocks, K / 32,
+                                                  ld, q, scale);
     return cudaGetLastError();
   }
   const int nsegs = seg_offsets ? nseg : 1;
@@ -175,11 +175,17 @@ cudaError_t mxfp8_launch(int64_t rows, int64_t K, bool src_bf16, const void* src
             (unsigned)std::min<int64_t>(rows / 32 + nsegs + 1, 65535));
   if (src_bf16)
     mx_cols_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(src),
-                                                        rows, K, seg_offsets, nsegs, q, scale);
+                                                        rows, K, ld, seg_offsets, nsegs, q, scale);
   else
-    mx_cols_kernel<float><<<grid, 128, 0, st>>>(static_cast<const float*>(src), rows, K,
+    mx_cols_kernel<float><<<grid, 128, 0, st>>>(static_cast<const float*>(src), rows, K, ld,
                                                 seg_offsets, nsegs, q, scale);
   return cudaGetLastError();
+}
+
+cudaError_t mxfp8_launch(int64_t rows, int64_t K, bool src_bf16, const void* src, int axis,
+                         const int32_t* seg_offsets, int nseg, uint8_t* q, uint8_t* scale,
+                         cudaStream_t st) {
+  return mxfp8_launch_ld(rows, K, K, src_bf16, src, axis, seg_offsets, nseg, q, scale, st);
 }
 
 }  // namespace moe

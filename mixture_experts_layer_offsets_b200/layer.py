@@ -7,6 +7,12 @@ library (``capi``).  Forward: moe_route -> moe_permute -> moe_grouped_ffn_fwd
 moe_route_bwd.  With ``capacity`` set, the padded-capacity comparison layout
 is used instead (moe_padded_dispatch after the route, uniform E x capacity
 rows in the grouped FFN, dropped pairs marked -1).
+
+dtype "mxfp8": bf16 activations and router, FP32 master expert weights whose
+MXFP8 copies (four orientations, see ``moe_mx_weights``) are made by
+mxfp8_quantize at the start of every forward, i.e. once per optimizer step
+when every step is one; the grouped FFN calls run with MOE_MXFP8 and write
+FP32 weight gradients.
 """
 
 from __future__ import annotations
@@ -15,7 +21,7 @@ import torch
 
 from . import capi
 
-_DT = {"f32": capi.MOE_F32, "bf16": capi.MOE_BF16}
+_DT = {"f32": capi.MOE_F32, "bf16": capi.MOE_BF16, "mxfp8": capi.MOE_MXFP8}
 
 
 def capacity_for(rows: int, E: int, cf_num: int = 5, cf_den: int = 4) -> int:
@@ -30,8 +36,14 @@ class MoELayer:
             raise ValueError(f"dtype {dtype!r} is not supported by the layer path")
         self.T, self.d, self.E, self.k, self.f = T, d_model, E, top_k, d_ff
         self.dtype = dtype
-        self.cdtype = _DT[dtype]
+        self.ffn_dtype = _DT[dtype]
+        # routing, permute and combine of the MXFP8 layer run on bf16 activations
+        self.cdtype = capi.MOE_BF16 if dtype == "mxfp8" else _DT[dtype]
         self.dw_dtype = dw_dtype or "f32"
+        if dtype == "mxfp8" and self.dw_dtype != "f32":
+            raise ValueError("the MXFP8 layer writes FP32 weight gradients")
+        if dtype == "mxfp8" and capacity:
+            raise ValueError("the padded layout is not offered with MXFP8")
         self.capacity = capacity
         self.shape = capi.shape_of(T, d_model, E, top_k, d_ff)
         self.R = T * top_k
@@ -64,7 +76,22 @@ class MoELayer:
         if capacity:
             self.pad_row = torch.empty(T, top_k, **i32)
             self.offsets_pad = torch.empty(E + 1, **i32)
-        nbytes = capi.moe_workspace_size(self.shape, self.cdtype, self.rows)
+        if dtype == "mxfp8":
+            u8 = dict(dtype=torch.uint8, device=dev)
+            self.mxq = dict(
+                w1_q=torch.empty(E * 2 * d_ff, d_model, **u8),
+                w1_s=torch.empty(E * 2 * d_ff, d_model // 32, **u8),
+                w1t_q=torch.empty(E * 2 * d_ff, d_model, **u8),
+                w1t_s=torch.empty(E * 2 * d_ff // 32, d_model, **u8),
+                w2_q=torch.empty(E * d_model, d_ff, **u8),
+                w2_s=torch.empty(E * d_model, d_ff // 32, **u8),
+                w2t_q=torch.empty(E * d_model, d_ff, **u8),
+                w2t_s=torch.empty(E * d_model // 32, d_ff, **u8),
+            )
+            self.mx = capi.moe_mx_weights(**{k: v.data_ptr() for k, v in self.mxq.items()})
+        else:
+            self.mx = None
+        nbytes = capi.moe_workspace_size(self.shape, self.ffn_dtype, self.rows)
         if nbytes == 0:
             raise ValueError("invalid MoE shape")
         self.ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
@@ -78,8 +105,19 @@ class MoELayer:
     def ffn_offsets(self):
         return self.offsets_pad if self.capacity else self.offsets
 
+    def quantize_weights(self, w1, w2, stream=None):
+        """MXFP8 copies of the FP32 master weights w1 [E, 2f, d], w2 [E, d, f]:
+        blocks along each GEMM's contraction axis (d and 2f for W1, f and d for W2)."""
+        E, d, f, q = self.E, self.d, self.f, self.mxq
+        for src, rows, K, name, axis in ((w1, E * 2 * f, d, "w1", 0), (w1, E * 2 * f, d, "w1t", 1),
+                                         (w2, E * d, f, "w2", 0), (w2, E * d, f, "w2t", 1)):
+            capi.mxfp8_quantize(rows, K, capi.MOE_F32, src, axis, None, 0, q[name + "_q"],
+                                q[name + "_s"], stream)
+
     def forward(self, x, w_router, bias, w1, w2, stream=None):
         s, dt = self.shape, self.cdtype
+        if self.mx is not None:
+            self.quantize_weights(w1, w2, stream)
         capi.moe_route(s, dt, x, w_router, bias, self.logits, self.topk_idx, self.topk_gate,
                        self.counts, self.offsets, self.slot_row, self.ws, stream)
         if self.capacity:
@@ -88,8 +126,8 @@ class MoELayer:
                                      stream)
         else:
             capi.moe_permute(s, dt, x, self.slot_row, self.x_perm, self.perm_src, stream)
-        capi.moe_grouped_ffn_fwd(s, dt, self.rows, self.x_perm, self.ffn_offsets, w1, w2,
-                                 self.act, self.y_perm, self.ws, stream=stream)
+        capi.moe_grouped_ffn_fwd(s, self.ffn_dtype, self.rows, self.x_perm, self.ffn_offsets, w1,
+                                 w2, self.act, self.y_perm, self.ws, mx=self.mx, stream=stream)
         capi.moe_combine(s, dt, self.y_perm, self.row_map, self.topk_gate, self.out, stream)
         return self.out
 
@@ -97,9 +135,9 @@ class MoELayer:
         s, dt = self.shape, self.cdtype
         capi.moe_combine_bwd(s, dt, dout, self.y_perm, self.row_map, self.topk_gate,
                              self.dy_perm, self.dgate, stream)
-        capi.moe_grouped_ffn_bwd(s, dt, self.rows, self.dy_perm, self.x_perm, self.act,
-                                 self.ffn_offsets, w1, w2, self.dx_perm, self.dw1, self.dw2,
-                                 _DT[self.dw_dtype], self.ws, stream=stream)
+        capi.moe_grouped_ffn_bwd(s, self.ffn_dtype, self.rows, self.dy_perm, self.x_perm,
+                                 self.act, self.ffn_offsets, w1, w2, self.dx_perm, self.dw1,
+                                 self.dw2, _DT[self.dw_dtype], self.ws, mx=self.mx, stream=stream)
         capi.moe_route_bwd(s, dt, x, w_router, self.logits, self.topk_idx, self.dgate,
                            self.dx_perm, self.row_map, self.dx, self.dw_router, self.ws, stream)
         return self.dx

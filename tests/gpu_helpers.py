@@ -10,7 +10,7 @@ from mixture_experts_layer_offsets_b200.layer import MoELayer
 from oracle import moe_ref as ref
 
 # Tolerances on relative Frobenius error, by compute dtype.
-TOL = {"f32": 1e-5, "bf16": 1e-2}
+TOL = {"f32": 1e-5, "bf16": 1e-2, "mxfp8": 5e-2}
 
 
 def f64(t) -> np.ndarray:

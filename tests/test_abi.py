@@ -91,9 +91,9 @@ def test_ffn_validation(lib):
     s = _shape()
     f = lib.moe_grouped_ffn_fwd
     assert f(s, capi.MOE_BF16, 128, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) \
-        == capi.MOE_ERR_UNSUPPORTED  # MXFP8 operands are not part of this version
+        == capi.MOE_ERR_INVALID_ARG  # MXFP8 weights given to a bf16 call
     assert f(s, capi.MOE_MXFP8, 128, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, 1 << 30, None) \
-        == capi.MOE_ERR_UNSUPPORTED
+        == capi.MOE_ERR_INVALID_ARG  # MXFP8 call without its weights
     assert f(s, capi.MOE_BF16, -1, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, 1 << 30, None) \
         == capi.MOE_ERR_INVALID_ARG
     assert f(_shape(d_model=136), capi.MOE_BF16, 128, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE,
@@ -132,3 +132,33 @@ def test_mxfp8_validation(lib):
 
 def test_status_query_validation(lib):
     assert lib.moe_get_device_status(None, None, ctypes.byref(ctypes.c_int32())) == capi.MOE_ERR_INVALID_ARG
+
+
+def _mxw(**kw):
+    fields = {n: FAKE for n, _ in capi.moe_mx_weights._fields_}
+    fields.update(kw)
+    return capi.moe_mx_weights(**fields)
+
+
+def test_mxfp8_ffn_validation(lib):
+    f, b = lib.moe_grouped_ffn_fwd, lib.moe_grouped_ffn_bwd
+    s = _shape()
+    mx = _mxw()
+    big = capi.moe_workspace_size(s, capi.MOE_MXFP8, 128)
+    assert big > capi.moe_workspace_size(s, capi.MOE_BF16, 128)   # room for the MXFP8 operands
+
+    def fwd(shape=s, mxw=mx, ws_bytes=big):
+        return f(shape, capi.MOE_MXFP8, 128, FAKE, FAKE, None, None, ctypes.addressof(mxw), FAKE,
+                 FAKE, FAKE, ws_bytes, None)
+
+    def bwd(dw_dtype=capi.MOE_F32, mxw=mx, ws_bytes=big):
+        return b(s, capi.MOE_MXFP8, 128, FAKE, FAKE, FAKE, FAKE, None, None, ctypes.addressof(mxw),
+                 FAKE, FAKE, FAKE, dw_dtype, FAKE, ws_bytes, None)
+
+    assert fwd(shape=_shape(d_model=192)) == capi.MOE_ERR_UNSUPPORTED     # d % 128
+    assert fwd(shape=_shape(d_ff=200)) == capi.MOE_ERR_UNSUPPORTED        # f % 128
+    assert fwd(mxw=_mxw(w2t_s=None)) == capi.MOE_ERR_INVALID_ARG
+    assert fwd(mxw=_mxw(w1_q=FAKE + 8)) == capi.MOE_ERR_INVALID_ARG      # misaligned
+    assert fwd(ws_bytes=big // 2) == capi.MOE_ERR_INVALID_ARG
+    assert bwd(dw_dtype=capi.MOE_BF16) == capi.MOE_ERR_INVALID_ARG       # dW is fp32
+    assert bwd(ws_bytes=1024) == capi.MOE_ERR_INVALID_ARG

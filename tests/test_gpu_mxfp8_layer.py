@@ -1,0 +1,96 @@
+"""GPU parity of the layer with MXFP8 expert GEMMs against the float64 oracle
+that quantises every GEMM operand along its contraction axis.
+
+Routing is bit-exact (bf16 router); the quantised weight copies are byte-exact
+with the oracle's MXFP8 rule; every value meets the MXFP8 relative Frobenius
+tolerance.  The layer keeps its activations in bf16, so the oracle takes its
+MXFP8 codes on the bf16-rounded activations, as the device does (an integer
+decision taken in the kernel's precision).  Sizes span several 128-row tiles per expert with ragged tails,
+empty experts (skewed routing), d and f that are odd multiples of 128, and a
+single token.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import TOL, f64, i64, rel, run_layer
+from mixture_experts_layer_offsets_b200.inputs import CONFIGS, shrink
+from oracle import moe_mx_ref as mxr
+from oracle import mxfp8_ref as mx
+
+pytestmark = pytest.mark.gpu
+
+BASE = CONFIGS["mxfp8_e128"]
+CASES = {
+    # ~150 rows per expert: two M tiles, ragged tail
+    "mx_e8": shrink(BASE, name="mx_e8", T=600, d_model=256, E=8, top_k=2, d_ff=256),
+    # d and f odd multiples of 128; top_k 4 of 16
+    "mx_e16_odd": shrink(BASE, name="mx_e16_odd", T=500, d_model=384, E=16, top_k=4, d_ff=384),
+    # skewed routing with a logit bias: heavy-tailed counts and empty experts
+    "mx_skew": shrink(BASE, name="mx_skew", T=700, d_model=128, E=32, top_k=2, d_ff=128,
+                      router_std=1 / 16.0, bias_std=2.0),
+    # one token
+    "mx_one_token": shrink(BASE, name="mx_one_token", T=1, d_model=128, E=4, top_k=2, d_ff=128),
+}
+
+
+def _oracle(cpu, L):
+    bias = f64(cpu["bias"]) if cpu["bias"] is not None else None
+    return mxr.layer_fwd_bwd_mx(f64(cpu["x"]), f64(cpu["w_router"]), f64(cpu["w1"]),
+                                f64(cpu["w2"]), f64(cpu["dout"]), L.k, bias,
+                                select_logits=f64(L.logits), act_round=mxr.round_bf16)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_mxfp8_layer_matches_oracle(name):
+    cfg = CASES[name]
+    tol = TOL["mxfp8"]
+    cpu, L = run_layer(cfg)
+    o = _oracle(cpu, L)
+    for key, dev in (("idx", L.topk_idx), ("counts", L.counts), ("offsets", L.offsets),
+                     ("slot_row", L.slot_row)):
+        assert np.array_equal(i64(dev), o[key]), key
+    R, f = cfg.R, cfg.d_ff
+    act = f64(L.act[:R])
+    checks = {
+        "logits": (f64(L.logits), o["logits"]), "gate": (f64(L.topk_gate), o["gate"]),
+        "a": (act[:, :f], o["a"]), "u": (act[:, f:2 * f], o["u"]), "h": (act[:, 2 * f:], o["h"]),
+        "y_perm": (f64(L.y_perm[:R]), o["y_perm"]), "out": (f64(L.out), o["out"]),
+        "dgate": (f64(L.dgate), o["dgate"]), "dy_perm": (f64(L.dy_perm[:R]), o["dy_perm"]),
+        "dx_perm": (f64(L.dx_perm[:R]), o["dx_perm"]), "dw1": (f64(L.dw1), o["dw1"]),
+        "dw2": (f64(L.dw2), o["dw2"]), "dx": (f64(L.dx), o["dx"]),
+        "dw_router": (f64(L.dw_router), o["dw_router"]),
+    }
+    errs = {k: rel(a, b) for k, (a, b) in checks.items()}
+    bad = {k: v for k, v in errs.items() if not v <= tol}
+    assert not bad, (name, errs)
+    for e in np.nonzero(o["counts"] == 0)[0]:
+        assert not L.dw1[e].any() and not L.dw2[e].any()
+
+
+def test_mxfp8_weight_copies_are_byte_exact():
+    cfg = CASES["mx_e16_odd"]
+    cpu, L = run_layer(cfg)
+    E, d, f = cfg.E, cfg.d_model, cfg.d_ff
+    w1 = f64(cpu["w1"]).reshape(E * 2 * f, d)
+    w2 = f64(cpu["w2"]).reshape(E * d, f)
+    for name, src, axis in (("w1", w1, 0), ("w1t", w1, 1), ("w2", w2, 0), ("w2t", w2, 1)):
+        q, s = mx.mxfp8_quantize(src, axis=axis)
+        assert np.array_equal(L.mxq[name + "_q"].cpu().numpy(), q), name
+        assert np.array_equal(L.mxq[name + "_s"].cpu().numpy(), s), name
+
+
+def test_mxfp8_is_closer_to_its_oracle_than_to_the_unquantised_layer():
+    """The device really computes with MXFP8 operands: its error against the
+    quantising oracle is well below its distance from the unquantised layer."""
+    from oracle import moe_ref as ref
+    cfg = CASES["mx_e8"]
+    cpu, L = run_layer(cfg)
+    o = _oracle(cpu, L)
+    bias = f64(cpu["bias"]) if cpu["bias"] is not None else None
+    u = ref.layer_fwd_bwd(f64(cpu["x"]), f64(cpu["w_router"]), f64(cpu["w1"]), f64(cpu["w2"]),
+                          f64(cpu["dout"]), L.k, bias, select_logits=f64(L.logits))
+    for key, dev in (("out", L.out), ("dw1", L.dw1), ("dx", L.dx)):
+        assert rel(f64(dev), o[key]) < 0.5 * rel(f64(dev), u[key]), key
+
