@@ -135,6 +135,8 @@ def run_ours(args, rank, world):
     cfg = inputs.CONFIGS[args.workload]
     if args.tokens:
         cfg = inputs.shrink(cfg, name=f"{cfg.name}@T{args.tokens}", T=args.tokens)
+    if args.experts:
+        cfg = inputs.shrink(cfg, name=f"{cfg.name}@E{args.experts}", E=args.experts)
     if args.dtype and args.dtype != cfg.dtype:
         cfg = inputs.shrink(cfg, name=f"{cfg.name}@{args.dtype}", dtype=args.dtype)
     mxfp8 = cfg.dtype == "mxfp8"
@@ -408,6 +410,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--dtype", default=None, choices=["f32", "bf16", "mxfp8"],
                     help="run the workload's shapes at another compute dtype")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="override E (smaller cases for profiling); not a bench line")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override T (smaller cases for profiling); not a bench line")
     args = ap.parse_args()

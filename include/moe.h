@@ -155,12 +155,23 @@ moe_status moe_permute(moe_shape shape, int dtype, const void* x, const int32_t*
                        void* x_perm, int32_t* perm_src, void* stream);
 
 /* MXFP8 copies of the expert weights for dtype MOE_MXFP8, made from their FP32
- * masters with mxfp8_quantize (typically once per optimizer step).  One pair of
- * (E4M3 codes, E8M0 scales) per GEMM orientation, with d % 128 == 0, f % 128 == 0:
- *   w1_q,  w1_s   W1 [E*2f, d] in blocks along d (axis 0):     q [E*2f, d], s [E*2f, d/32]
- *   w1t_q, w1t_s  W1 in 32-row blocks along 2f (axis 1):       q [E*2f, d], s [E*2f/32, d]
- *   w2_q,  w2_s   W2 [E*d, f] in blocks along f (axis 0):      q [E*d, f],  s [E*d, f/32]
- *   w2t_q, w2t_s  W2 in 32-row blocks along d (axis 1):        q [E*d, f],  s [E*d/32, f]
+ * masters by moe_mx_quantize_weights (once per optimizer step).  Every member is a
+ * device pointer to a buffer of the size given; d % 128 == 0 and f % 128 == 0.
+ * Element codes (E4M3, row-major, one byte per weight):
+ *   w1_q, w1t_q [E*2f, d]    W1 quantised in blocks of 32 along d / along 2f
+ *   w2_q, w2t_q [E*d, f]     W2 quantised in blocks of 32 along f / along d
+ * Scales (E8M0, E*2f*d/32 bytes for W1, E*d*f/32 for W2) are stored as the
+ * block-scaled MMA consumes them: 512-byte atoms covering 128 rows r (of the GEMM's
+ * M or N) x 4 consecutive 32-blocks kb along its K, the scale of (r, kb) at byte
+ *   (r % 32) * 16 + (r / 32) * 4 + kb.
+ * Atom order, with j a 128-wide K stage:
+ *   w1_s   atom (e * f/64 + t) * d/128 + j; atom rows 0..63 are the gate rows 64t..,
+ *          rows 64..127 the up rows f + 64t.. of W1[e] (the forward's gate/up tile)
+ *   w1t_s  atom (e * 2f/128 + j) * d/128 + n / 128, rows n = columns of W1[e],
+ *          K = its 2f rows
+ *   w2_s   atom (e * d/128 + r / 128) * f/128 + j, rows r = rows of W2[e]
+ *   w2t_s  atom (e * d/128 + j) * f/128 + n / 128, rows n = columns of W2[e], K = its
+ *          d rows
  * The forward GEMMs use w1 and w2, the input-gradient GEMMs w2t and w1t. */
 typedef struct moe_mx_weights {
   const uint8_t* w1_q;
@@ -172,6 +183,15 @@ typedef struct moe_mx_weights {
   const uint8_t* w2t_q;
   const uint8_t* w2t_s;
 } moe_mx_weights;
+
+/* ---- MXFP8 weight copies ---------------------------------------------------
+ * [kongchang] boundary-conditions section: MXFP8 operands with an authoritative FP32
+ * master weight.  Writes all eight buffers of *out (a HOST struct whose members are
+ * device pointers; the call writes through them) from the FP32 masters
+ * w1 [E, 2f, d] and w2 [E, d, f], each element quantised as mxfp8_quantize does
+ * (OCP floor rule), in one pass over each master.  d % 128 == 0, f % 128 == 0. */
+moe_status moe_mx_quantize_weights(moe_shape shape, const float* w1, const float* w2,
+                                   const moe_mx_weights* out, void* stream);
 
 /* ---- a4: grouped SwiGLU FFN, forward -------------------------------------
  * [kongchang] routing section: a device-scheduled grouped GEMM handles the

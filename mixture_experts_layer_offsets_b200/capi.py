@@ -57,6 +57,7 @@ _SIGS = {
                                  _I, _P, _SZ, _P]),
     "moe_route_bwd": (_I, [moe_shape, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "mxfp8_quantize": (_I, [_I64, _I64, _I, _P, _I, _P, _I, _P, _P, _P]),
+    "moe_mx_quantize_weights": (_I, [moe_shape, _P, _P, _P, _P]),
     "moe_padded_dispatch": (_I, [moe_shape, _I, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _P, _P]),
 }
 
@@ -189,6 +190,11 @@ def mxfp8_quantize(rows, K, src_dtype, src, axis, seg_offsets, nseg, q, scale,
     _check("mxfp8_quantize", lib().mxfp8_quantize(
         rows, K, src_dtype, _ptr(src), axis, _ptr(seg_offsets), nseg, _ptr(q), _ptr(scale),
         _stream(stream)))
+
+
+def moe_mx_quantize_weights(shape, w1, w2, out, stream=None) -> None:
+    _check("moe_mx_quantize_weights", lib().moe_mx_quantize_weights(
+        shape, _ptr(w1), _ptr(w2), _ptr(out), _stream(stream)))
 
 
 def moe_padded_dispatch(shape, dtype, capacity, x, topk_idx, slot_row, offsets, x_pad, pad_row,

@@ -244,6 +244,18 @@ moe_status moe_route_bwd(moe_shape s, int dtype, const void* x, const void* w_ro
                                       s.top_k, scratch(ws), status_word(ws), as_stream(stream)));
 }
 
+moe_status moe_mx_quantize_weights(moe_shape s, const float* w1, const float* w2,
+                                   const moe_mx_weights* out, void* stream) {
+  moe_status st = shape_ok(s);
+  if (st != MOE_OK) return st;
+  MxWeights w;
+  moe_status vs = mx_weights_ok(out, w);
+  if (vs != MOE_OK) return vs;
+  if (s.d_model % 128 || s.d_ff % 128) return MOE_ERR_UNSUPPORTED;
+  if (!ptrs_ok(w1, w2)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(mx_quantize_weights(s.E, s.d_model, s.d_ff, w1, w2, w, as_stream(stream)));
+}
+
 moe_status mxfp8_quantize(int64_t rows, int64_t K, int src_dtype, const void* src, int axis,
                           const int32_t* seg_offsets, int nseg, uint8_t* q, uint8_t* scale,
                           void* stream) {

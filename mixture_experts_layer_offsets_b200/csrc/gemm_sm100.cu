@@ -97,13 +97,10 @@ struct GemmParams {
   int split;
   // EPI_ROUTER_DX
   const int32_t* slot_row; // [rows_total][topk]
-  // MXFP8 operands: E8M0 scales, one byte per 32 K elements.
-  //   K-major operand (blocks along its rows):      s[row][K / 32]        (ld = K / 32)
-  //   MN-major operand (blocks of 32 K rows):       s[block row][MN]      (ld = MN extent)
-  //   GROUP_K operands: block rows restart at every group (segment) start.
+  // MXFP8 operands: E8M0 scales as 512-byte MMA atoms (128 rows x 4 blocks of 32
+  // along K), in the order the producer reads them (see the MXFP8 producer).
   const uint8_t* sfa;
   const uint8_t* sfb;
-  int64_t ld_sfa, ld_sfb;
 };
 
 template <int BN, bool PAIR = false, int EPI = 1, bool FP8 = false> struct Cfg {
@@ -477,10 +474,10 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
     }
   }
   if constexpr (GROUP_K && FP8) {
-    if (warp == 1) {  // first 32-row scale block of each group (blocks restart at group starts)
+    if (warp == 1) {  // first 128-row scale stage of each group (stages restart at group starts)
       const int lo = lane * 32, hi = min(lo + 32, E);
       int s = 0;
-      for (int g = lo; g < hi; ++g) s += (s_off[g + 1] - s_off[g] + 31) / 32;
+      for (int g = lo; g < hi; ++g) s += (s_off[g + 1] - s_off[g] + 127) / 128;
       int incl = s;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -490,7 +487,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
       int run = incl - s;
       for (int g = lo; g < hi; ++g) {
         s_pre[g] = run;
-        run += (s_off[g + 1] - s_off[g] + 31) / 32;
+        run += (s_off[g + 1] - s_off[g] + 127) / 128;
       }
     }
   }
@@ -515,85 +512,44 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
 
   if (warp == 0 && FP8) {
     // ---------------------------------------------------- producer (MXFP8)
-    // The warp writes the stage's scale atoms (scale of row mn, block kb at byte
-    // (mn % 32) * 16 + (mn / 32) * 4 + kb), then lane 0 issues the TMA loads.
+    // Per stage: the A and B tiles by TMA and their two 512-byte scale atoms by bulk
+    // copy, all completing on the stage's full barrier.  Atom order in global memory:
+    //   row-grouped A (K-major):   (M tile over all experts) * K/128 + k stage
+    //   K-major B (weights):       (expert * N tiles + n tile) * K/128 + k stage
+    //   MN-major B (weights):      (expert * K/128 + k stage) * N/128 + n tile
+    //   GROUP_K A and B:           (k stage over all groups) * (M or N)/128 + tile
     if (lane == 0) {
       tma_prefetch_desc(&p.tmA);
       tma_prefetch_desc(&p.tmB);
-    }
-    uint32_t it = 0;
-    bool ok = true;
-    for (int t = tile0; t < total && ok; t += tstride) {
-      const TileInfo ti = decode(t);
-      for (int kb = 0; kb < ti.nkb; ++kb, ++it) {
-        if (__any_sync(0xffffffffu, *s_abort)) { ok = false; break; }
-        const int s = it % S;
-        bool w = true;
-        if (lane == 0) w = mbar_wait(&empty[s], ((it / S) & 1) ^ 1);
-        if (!__shfl_sync(0xffffffffu, w, 0)) {
-          if (lane == 0) fail();
-          ok = false;
-          break;
-        }
-        uint8_t* sa = smem + s * C::kStage;
-        uint8_t* sb = sa + kABytes;
-        uint8_t* sf = sb + C::kBBytes;
-        const int kc = kb * C::kBKe;  // first K element of the stage
-        // blocks of this stage that lie inside the group's K range (GROUP_K tails)
-        const int nblk = GROUP_K ? min(4, (ti.klast + 31) / 32 + 4 * (ti.nkb - 1 - kb)) : 4;
-        const int nblk_ok = GROUP_K ? (kb == ti.nkb - 1 ? (ti.klast + 31) / 32 : 4) : nblk;
-        auto atom = [&](uint8_t* dst, const uint8_t* sfp, int64_t ld, bool mn_major, int mn0,
-                        int rows_limit, int64_t blk0) {
-          uint32_t wd[4];
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int mn = mn0 + lane + 32 * g;
-            uint32_t v = 0x7F7F7F7Fu;  // scale 1.0 where no data is multiplied
-            if (!mn_major) {
-              if (mn < rows_limit) v = __ldg(reinterpret_cast<const uint32_t*>(sfp + (int64_t)mn * ld + blk0));
-            } else {
-              v = 0;
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const uint32_t b = j < nblk_ok ? __ldg(sfp + (blk0 + j) * ld + mn) : 0x7Fu;
-                v |= b << (8 * j);
-              }
-            }
-            wd[g] = v;
-          }
-          *reinterpret_cast<uint4*>(dst + lane * 16) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-        };
-        (void)nblk;
+      uint32_t it = 0;
+      bool ok = true;
+      const int kq = GROUP_K ? 0 : p.K / C::kBKe;
+      for (int t = tile0; t < total && ok; t += tstride) {
+        const TileInfo ti = decode(t);
+        const uint8_t* atomA;
+        const uint8_t* atomB;
         if constexpr (GROUP_K) {
-          const int64_t blk = s_pre[ti.g] + kc / 32;  // both operands: segmented block rows
-          atom(sf, p.sfa, p.ld_sfa, true, ti.m0, 0, blk);
-          atom(sf + 512, p.sfb, p.ld_sfb, true, ti.n0, 0, blk);
+          atomA = p.sfa + ((int64_t)s_pre[ti.g] * (p.M / BM) + ti.m0 / BM) * 512;
+          atomB = p.sfb + ((int64_t)s_pre[ti.g] * (p.N / BN) + ti.n0 / BN) * 512;
         } else {
-          if constexpr (!A_MN) atom(sf, p.sfa, p.ld_sfa, false, ti.m0, p.rows_total, kc / 32);
-          else atom(sf, p.sfa, p.ld_sfa, true, ti.m0, 0, (ti.kbase + kc) / 32);
+          const int mt = s_pre[ti.g] / nN + (ti.m0 - s_off[ti.g]) / BM;
+          atomA = p.sfa + (int64_t)mt * kq * 512;
           if constexpr (!B_MN) {
-            // B rows: the expert's weight rows (SwiGLU: 64 gate rows, then 64 up rows)
-            if constexpr (EPI == EPI_SWIGLU_FWD) {
-              // rows n0 .. n0+63 and f + n0 .. f + n0 + 63: lane + 32 g covers them in order
-              uint32_t wd[4];
-#pragma unroll
-              for (int g = 0; g < 4; ++g) {
-                const int nn = lane + 32 * g;
-                const int row = ti.kbase + (nn < 64 ? ti.n0 + nn : p.f + ti.n0 + nn - 64);
-                wd[g] = __ldg(reinterpret_cast<const uint32_t*>(p.sfb + (int64_t)row * p.ld_sfb + kc / 32));
-              }
-              *reinterpret_cast<uint4*>(sf + 512 + lane * 16) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-            } else {
-              atom(sf + 512, p.sfb, p.ld_sfb, false, ti.kbase + ti.n0, 0x7FFFFFFF, kc / 32);
-            }
+            const int nt = ti.n0 / (EPI == EPI_SWIGLU_FWD ? BN / 2 : BN);
+            atomB = p.sfb + ((int64_t)ti.g * nN + nt) * kq * 512;
           } else {
-            atom(sf + 512, p.sfb, p.ld_sfb, true, ti.n0, 0, (ti.kbase + kc) / 32);
+            atomB = p.sfb + ((int64_t)ti.g * kq * (p.N / BN) + ti.n0 / BN) * 512;
           }
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&full[s], kABytes + C::kBBytes);
+        for (int kb = 0; kb < ti.nkb; ++kb, ++it) {
+          if (*s_abort) { ok = false; break; }
+          const int s = it % S;
+          if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1)) { fail(); ok = false; break; }
+          uint8_t* sa = smem + s * C::kStage;
+          uint8_t* sb = sa + kABytes;
+          uint8_t* sf = sb + C::kBBytes;
+          const int kc = kb * C::kBKe;  // first K element of the stage
+          mbar_arrive_expect_tx(&full[s], kABytes + C::kBBytes + 1024);
           if constexpr (!A_MN) tma_load_2d(sa, &p.tmA, kc, ti.m0, &full[s]);
           else tma_load_2d(sa, &p.tmA, ti.m0, ti.kbase + kc, &full[s]);
           if constexpr (!B_MN) {
@@ -606,12 +562,19 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
           } else {
             tma_load_2d(sb, &p.tmB, ti.n0, ti.kbase + kc, &full[s]);
           }
+          if constexpr (GROUP_K) {
+            bulk_load(sf, atomA + (int64_t)kb * (p.M / BM) * 512, 512, &full[s]);
+            bulk_load(sf + 512, atomB + (int64_t)kb * (p.N / BN) * 512, 512, &full[s]);
+          } else {
+            bulk_load(sf, atomA + kb * 512, 512, &full[s]);
+            bulk_load(sf + 512, atomB + (B_MN ? (int64_t)kb * (p.N / BN) * 512 : kb * 512), 512, &full[s]);
+          }
         }
       }
-    }
-    if (!ok && lane == 0) {
-      for (uint32_t j = it > (uint32_t)S ? it - S : 0; j < it; ++j)
-        (void)mbar_wait(&full[j % S], (j / S) & 1);
+      if (!ok) {  // let the copies already issued land before the CTA exits
+        for (uint32_t j = it > (uint32_t)S ? it - S : 0; j < it; ++j)
+          (void)mbar_wait(&full[j % S], (j / S) & 1);
+      }
     }
   } else if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -1407,10 +1370,12 @@ cudaError_t ffn_bwd_bf16(const FfnShape& s, const void* dy_perm, const void* x_p
 // GEMM's K right before it is used (forward: x and h along their rows; dgrad: dy and
 // [da|du] along their rows, the weights along their rows of K via the moe_mx_weights
 // copies; wgrad: dy, h, [da|du] and x in 32-row blocks that restart at every expert's
-// first row).  Accumulation is fp32; outputs are bf16 (dW fp32).
+// first row).  Accumulation is fp32; outputs are bf16 (dW fp32).  Scales are kept as
+// the MMA's 512-byte atoms in the order the GEMM reads them (see mxfp8.cu).
 namespace {
 
 struct MxLayout {
+  size_t rt;                                          // row -> tile map
   size_t qx0, sx0, qh0, sh0;                         // forward
   size_t dadu, qdy0, sdy0, qda0, sda0;               // backward, dgrad operands
   size_t qdy1, sdy1, qh1, sh1, qda1, sda1, qx1, sx1;  // backward, wgrad operands
@@ -1419,20 +1384,25 @@ struct MxLayout {
 
 MxLayout mx_layout(const FfnShape& s) {
   const size_t R = (size_t)s.rows, d = s.d, f = s.f;
-  const size_t sb = R / 32 + s.E + 1;  // 32-row blocks of a segmented (per expert) axis
+  // at most R/128 + E tiles (row-grouped) or stages (segmented) of 128 rows; an atom
+  // covers 128 rows x 128 K elements
+  const size_t tiles = R / 128 + s.E;
+  auto atoms = [&](size_t K) { return tiles * (K / 128) * 512; };
   MxLayout L;
   size_t o = 0;
   auto take = [&](size_t bytes) { const size_t at = o; o += align256(bytes); return at; };
-  L.qx0 = take(R * d); L.sx0 = take(R * d / 32); L.qh0 = take(R * f); L.sh0 = take(R * f / 32);
+  L.rt = take(R * 4);
+  const size_t base = o;
+  L.qx0 = take(R * d); L.sx0 = take(atoms(d)); L.qh0 = take(R * f); L.sh0 = take(atoms(f));
   L.fwd_bytes = o;
-  o = 0;
+  o = base;
   L.dadu = take(R * 2 * f * 2);
-  L.qdy0 = take(R * d); L.sdy0 = take(R * d / 32);
-  L.qda0 = take(R * 2 * f); L.sda0 = take(R * 2 * f / 32);
-  L.qdy1 = take(R * d); L.sdy1 = take(sb * d);
-  L.qh1 = take(R * f); L.sh1 = take(sb * f);
-  L.qda1 = take(R * 2 * f); L.sda1 = take(sb * 2 * f);
-  L.qx1 = take(R * d); L.sx1 = take(sb * d);
+  L.qdy0 = take(R * d); L.sdy0 = take(atoms(d));
+  L.qda0 = take(R * 2 * f); L.sda0 = take(atoms(2 * f));
+  L.qdy1 = take(R * d); L.sdy1 = take(atoms(d));
+  L.qh1 = take(R * f); L.sh1 = take(atoms(f));
+  L.qda1 = take(R * 2 * f); L.sda1 = take(atoms(2 * f));
+  L.qx1 = take(R * d); L.sx1 = take(atoms(d));
   L.bwd_bytes = o;
   return L;
 }
@@ -1455,6 +1425,15 @@ size_t ffn_mx_ws_bytes(const FfnShape& s) {
   return std::max(L.fwd_bytes, L.bwd_bytes);
 }
 
+cudaError_t mx_quantize_weights(int E, int d, int f, const float* w1, const float* w2,
+                                const MxWeights& w, cudaStream_t st) {
+  auto u8 = [](const uint8_t* p) { return const_cast<uint8_t*>(p); };
+  cudaError_t err = mxfp8_weights(w1, E, 2 * f, d, f, u8(w.w1_q), u8(w.w1_s), u8(w.w1t_q),
+                                  u8(w.w1t_s), st);
+  if (err != cudaSuccess) return err;
+  return mxfp8_weights(w2, E, d, f, 0, u8(w.w2_q), u8(w.w2_s), u8(w.w2t_q), u8(w.w2t_s), st);
+}
+
 cudaError_t ffn_fwd_mx(const FfnShape& s, const void* x_perm, const int32_t* offsets,
                        const MxWeights& w, void* act, void* y_perm, void* scratch, int* status,
                        cudaStream_t st) {
@@ -1466,30 +1445,32 @@ cudaError_t ffn_fwd_mx(const FfnShape& s, const void* x_perm, const int32_t* off
   uint8_t* ws = static_cast<uint8_t*>(scratch);
   const MxLayout L = mx_layout(s);
   const __nv_bfloat16* actb = static_cast<const __nv_bfloat16*>(act);
+  int32_t* rt = reinterpret_cast<int32_t*>(ws + L.rt);
+  if ((err = row_tile_launch(offsets, E, R, rt, st)) != cudaSuccess) return err;
   // x along d; gate/up GEMM with the SwiGLU epilogue
-  if ((err = mxfp8_launch_ld(R, d, d, true, x_perm, 0, nullptr, 0, ws + L.qx0, ws + L.sx0, st)) != cudaSuccess)
+  if ((err = mxfp8_rows_atoms(R, d, d, x_perm, rt, ws + L.qx0, ws + L.sx0, st)) != cudaSuccess)
     return err;
   GemmParams p1 = mx_params(s, offsets, status);
   if (!tmap(&p1.tmA, ws + L.qx0, d, R, d, 128, 128, false, true) ||
       !tmap(&p1.tmB, w.w1_q, d, (uint64_t)E * 2 * f, d, 128, 64, false, true) ||
       !tmap(&p1.tmOut, act, 3 * f, R, 3 * f, 64, 16))
     return cudaErrorInvalidValue;
-  p1.sfa = ws + L.sx0; p1.ld_sfa = d / 32;
-  p1.sfb = w.w1_s; p1.ld_sfb = d / 32;
+  p1.sfa = ws + L.sx0;
+  p1.sfb = w.w1_s;
   p1.N = f; p1.K = d; p1.b_rows = 2 * f;
   p1.out = static_cast<__nv_bfloat16*>(act); p1.ld_out = 3 * f;
   if ((err = launch_mx<false, false, EPI_SWIGLU_FWD, false>(p1, m_tile_bound(s) * (f / 64), st)) != cudaSuccess)
     return err;
   // h along f; down GEMM
-  if ((err = mxfp8_launch_ld(R, f, 3 * f, true, actb + 2 * f, 0, nullptr, 0, ws + L.qh0, ws + L.sh0, st)) != cudaSuccess)
+  if ((err = mxfp8_rows_atoms(R, f, 3 * f, actb + 2 * f, rt, ws + L.qh0, ws + L.sh0, st)) != cudaSuccess)
     return err;
   GemmParams p2 = mx_params(s, offsets, status);
   if (!tmap(&p2.tmA, ws + L.qh0, f, R, f, 128, 128, false, true) ||
       !tmap(&p2.tmB, w.w2_q, f, (uint64_t)E * d, f, 128, 128, false, true) ||
       !tmap(&p2.tmOut, y_perm, d, R, d, 64, 16))
     return cudaErrorInvalidValue;
-  p2.sfa = ws + L.sh0; p2.ld_sfa = f / 32;
-  p2.sfb = w.w2_s; p2.ld_sfb = f / 32;
+  p2.sfa = ws + L.sh0;
+  p2.sfb = w.w2_s;
   p2.N = d; p2.K = f; p2.b_rows = d;
   p2.out = static_cast<__nv_bfloat16*>(y_perm); p2.ld_out = d;
   return launch_mx<false, false, EPI_STORE, false>(p2, m_tile_bound(s) * (d / 128), st);
@@ -1507,41 +1488,43 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
   const MxLayout L = mx_layout(s);
   const __nv_bfloat16* actb = static_cast<const __nv_bfloat16*>(act);
   __nv_bfloat16* dadu = reinterpret_cast<__nv_bfloat16*>(ws + L.dadu);
+  int32_t* rt = reinterpret_cast<int32_t*>(ws + L.rt);
   if (R > 0) {
+    if ((err = row_tile_launch(offsets, E, R, rt, st)) != cudaSuccess) return err;
     // dgrad 1: dh = dy W2 (dy along d, W2 along its d rows), SwiGLU backward -> [da | du]
-    if ((err = mxfp8_launch_ld(R, d, d, true, dy_perm, 0, nullptr, 0, ws + L.qdy0, ws + L.sdy0, st)) != cudaSuccess)
+    if ((err = mxfp8_rows_atoms(R, d, d, dy_perm, rt, ws + L.qdy0, ws + L.sdy0, st)) != cudaSuccess)
       return err;
     GemmParams p3 = mx_params(s, offsets, status);
     if (!tmap(&p3.tmA, ws + L.qdy0, d, R, d, 128, 128, false, true) ||
         !tmap(&p3.tmB, w.w2t_q, f, (uint64_t)E * d, f, 128, 128, false, true) ||
         !tmap(&p3.tmOut, dadu, 2 * f, R, 2 * f, 64, 16))
       return cudaErrorInvalidValue;
-    p3.sfa = ws + L.sdy0; p3.ld_sfa = d / 32;
-    p3.sfb = w.w2t_s; p3.ld_sfb = f;
+    p3.sfa = ws + L.sdy0;
+    p3.sfb = w.w2t_s;
     p3.N = f; p3.K = d; p3.b_rows = d;
     p3.out = dadu; p3.ld_out = 2 * f;
     p3.act = actb; p3.ld_act = 3 * f;
     if ((err = launch_mx<false, true, EPI_SWIGLU_BWD, false>(p3, m_tile_bound(s) * (f / 128), st)) != cudaSuccess)
       return err;
     // dgrad 2: dx = [da | du] W1 ([da | du] along 2f, W1 along its 2f rows)
-    if ((err = mxfp8_launch_ld(R, 2 * f, 2 * f, true, dadu, 0, nullptr, 0, ws + L.qda0, ws + L.sda0, st)) != cudaSuccess)
+    if ((err = mxfp8_rows_atoms(R, 2 * f, 2 * f, dadu, rt, ws + L.qda0, ws + L.sda0, st)) != cudaSuccess)
       return err;
     GemmParams p4 = mx_params(s, offsets, status);
     if (!tmap(&p4.tmA, ws + L.qda0, 2 * f, R, 2 * f, 128, 128, false, true) ||
         !tmap(&p4.tmB, w.w1t_q, d, (uint64_t)E * 2 * f, d, 128, 128, false, true) ||
         !tmap(&p4.tmOut, dx_perm, d, R, d, 64, 16))
       return cudaErrorInvalidValue;
-    p4.sfa = ws + L.sda0; p4.ld_sfa = 2 * f / 32;
-    p4.sfb = w.w1t_s; p4.ld_sfb = d;
+    p4.sfa = ws + L.sda0;
+    p4.sfb = w.w1t_s;
     p4.N = d; p4.K = 2 * f; p4.b_rows = 2 * f;
     p4.out = static_cast<__nv_bfloat16*>(dx_perm); p4.ld_out = d;
     if ((err = launch_mx<false, true, EPI_STORE, false>(p4, m_tile_bound(s) * (d / 128), st)) != cudaSuccess)
       return err;
-    // wgrad operands along the token axis, blocks restarting at each expert
-    if ((err = mxfp8_launch_ld(R, d, d, true, dy_perm, 1, offsets, E, ws + L.qdy1, ws + L.sdy1, st)) != cudaSuccess ||
-        (err = mxfp8_launch_ld(R, f, 3 * f, true, actb + 2 * f, 1, offsets, E, ws + L.qh1, ws + L.sh1, st)) != cudaSuccess ||
-        (err = mxfp8_launch_ld(R, 2 * f, 2 * f, true, dadu, 1, offsets, E, ws + L.qda1, ws + L.sda1, st)) != cudaSuccess ||
-        (err = mxfp8_launch_ld(R, d, d, true, x_perm, 1, offsets, E, ws + L.qx1, ws + L.sx1, st)) != cudaSuccess)
+    // wgrad operands along the token axis, 32-row blocks restarting at each expert
+    if ((err = mxfp8_cols_atoms(R, d, d, dy_perm, offsets, E, ws + L.qdy1, ws + L.sdy1, st)) != cudaSuccess ||
+        (err = mxfp8_cols_atoms(R, f, 3 * f, actb + 2 * f, offsets, E, ws + L.qh1, ws + L.sh1, st)) != cudaSuccess ||
+        (err = mxfp8_cols_atoms(R, 2 * f, 2 * f, dadu, offsets, E, ws + L.qda1, ws + L.sda1, st)) != cudaSuccess ||
+        (err = mxfp8_cols_atoms(R, d, d, x_perm, offsets, E, ws + L.qx1, ws + L.sx1, st)) != cudaSuccess)
       return err;
   }
   // wgrad 2: dW2[e] = dy^T h  (M = d, N = f)
@@ -1550,8 +1533,8 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
       !tmap(&p5.tmB, ws + L.qh1, f, Rtm, f, 128, 128, false, true) ||
       !tmap(&p5.tmOut, dw2, f, (uint64_t)E * d, f, 32, 16, true))
     return cudaErrorInvalidValue;
-  p5.sfa = ws + L.sdy1; p5.ld_sfa = d;
-  p5.sfb = ws + L.sh1; p5.ld_sfb = f;
+  p5.sfa = ws + L.sdy1;
+  p5.sfb = ws + L.sh1;
   p5.M = d; p5.N = f;
   p5.out_f32 = dw2; p5.ld_out = f; p5.out_group = (int64_t)d * f;
   if ((err = launch_mx<true, true, EPI_WGRAD, true>(p5, (int64_t)E * (d / 128) * (f / 128), st)) != cudaSuccess)
@@ -1562,8 +1545,8 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
       !tmap(&p6.tmB, ws + L.qx1, d, Rtm, d, 128, 128, false, true) ||
       !tmap(&p6.tmOut, dw1, d, (uint64_t)E * 2 * f, d, 32, 16, true))
     return cudaErrorInvalidValue;
-  p6.sfa = ws + L.sda1; p6.ld_sfa = 2 * f;
-  p6.sfb = ws + L.sx1; p6.ld_sfb = d;
+  p6.sfa = ws + L.sda1;
+  p6.sfb = ws + L.sx1;
   p6.M = 2 * f; p6.N = d;
   p6.out_f32 = dw1; p6.ld_out = d; p6.out_group = (int64_t)2 * f * d;
   return launch_mx<true, true, EPI_WGRAD, true>(p6, (int64_t)E * (2 * f / 128) * (d / 128), st);

@@ -71,6 +71,21 @@ cudaError_t mxfp8_launch_ld(int64_t rows, int64_t K, int64_t ld, bool src_bf16, 
                             int axis, const int32_t* seg_offsets, int nseg, uint8_t* q,
                             uint8_t* scale, cudaStream_t st);
 
+// Scale atoms of the block-scaled MMA (512 bytes: 128 rows x 4 blocks of 32 along K,
+// byte (r % 32) * 16 + (r / 32) * 4 + kb), laid out in the order the grouped GEMM reads:
+//   row_tile_launch: row -> tile * 128 + row in tile of the row-grouped GEMMs (-1 outside)
+//   mxfp8_rows_atoms: blocks along rows (bf16 source, row stride ld), atom (tile * K/128 + kq)
+//   mxfp8_cols_atoms: 32-row blocks restarting at segments, atom (stage * K/128 + col / 128)
+//   mxfp8_weights: FP32 [E][Rw][Kw] -> row-block and column-block copies (see mxfp8.cu)
+cudaError_t row_tile_launch(const int32_t* offsets, int E, int64_t rows, int32_t* out, cudaStream_t st);
+cudaError_t mxfp8_rows_atoms(int64_t rows, int64_t K, int64_t ld, const void* src_bf16,
+                             const int32_t* row_tile, uint8_t* q, uint8_t* atoms, cudaStream_t st);
+cudaError_t mxfp8_cols_atoms(int64_t rows, int64_t K, int64_t ld, const void* src_bf16,
+                             const int32_t* seg, int nseg, uint8_t* q, uint8_t* atoms,
+                             cudaStream_t st);
+cudaError_t mxfp8_weights(const float* w, int E, int Rw, int Kw, int pair_f, uint8_t* q0,
+                          uint8_t* s0, uint8_t* q1, uint8_t* s1, cudaStream_t st);
+
 // ---------------------------------------------------------- grouped FFN
 struct FfnShape {
   int d, E, f;
@@ -99,6 +114,8 @@ struct MxWeights {
   const uint8_t *w1_q, *w1_s, *w1t_q, *w1t_s, *w2_q, *w2_s, *w2t_q, *w2t_s;
 };
 size_t ffn_mx_ws_bytes(const FfnShape& s);
+cudaError_t mx_quantize_weights(int E, int d, int f, const float* w1, const float* w2,
+                                const MxWeights& w, cudaStream_t st);
 cudaError_t ffn_fwd_mx(const FfnShape& s, const void* x_perm, const int32_t* offsets,
                        const MxWeights& w, void* act, void* y_perm, void* scratch, int* status,
                        cudaStream_t st);

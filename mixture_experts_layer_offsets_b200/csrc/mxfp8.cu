@@ -152,7 +152,307 @@ mx_cols_kernel(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
   }
 }
 
+// ---------------------------------------------------------------- scale atoms
+// The block-scaled MMA takes its E8M0 scales from TMEM, which each pipeline stage fills
+// from a 512-byte shared-memory atom: 128 rows (of M or N) x 4 blocks of 32 along K, the
+// scale of row r and block kb at byte (r % 32) * 16 + (r / 32) * 4 + kb.  Inside the FFN
+// every scale lives in global memory as such atoms, in the order in which the grouped
+// GEMM consumes them, so that one bulk copy per operand and stage fetches it.
+__device__ __forceinline__ int atom_byte(int r, int kb) {
+  return (r & 31) * 16 + ((r >> 5) & 3) * 4 + kb;
+}
+
+// Row -> (128-row tile, row in tile) of the row-grouped GEMMs: tile = number of 128-row
+// tiles of the experts before the row's expert + (row - expert start) / 128.  Encoded
+// as tile * 128 + row in tile; -1 for rows outside every expert segment.
+__global__ void __launch_bounds__(256)
+row_tile_kernel(const int32_t* __restrict__ offsets, int E, int64_t rows, int32_t* __restrict__ out) {
+  __shared__ int s_off[1025];
+  __shared__ int s_pre[1025];
+  for (int g = threadIdx.x; g <= E; g += blockDim.x) s_off[g] = offsets[g];
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x, lo = lane * 32, hi = min(lo + 32, E);
+    int sum = 0;
+    for (int g = lo; g < hi; ++g) sum += (s_off[g + 1] - s_off[g] + 127) / 128;
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    int run = incl - sum;
+    for (int g = lo; g < hi; ++g) {
+      s_pre[g] = run;
+      run += (s_off[g + 1] - s_off[g] + 127) / 128;
+    }
+  }
+  __syncthreads();
+  for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < rows;
+       r += (int64_t)gridDim.x * blockDim.x) {
+    int lo = 0, hi = E - 1;  // last expert whose start is <= r
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_off[mid] <= r) lo = mid; else hi = mid - 1;
+    }
+    const int lr = (int)(r - s_off[lo]);
+    out[r] = (r >= s_off[lo] && r < s_off[lo + 1]) ? (s_pre[lo] + lr / 128) * 128 + (lr & 127) : -1;
+  }
+}
+
+// axis 0 (blocks along rows) with scales written as row-tile atoms:
+// atom (tile * K/128 + k / 128), the tile and the row in it from row_tile.
+template <typename T>
+__global__ void __launch_bounds__(256)
+mx_rows_atoms_kernel(const T* __restrict__ src, int64_t nblocks, int64_t kblocks, int64_t ld,
+                     const int32_t* __restrict__ row_tile, uint8_t* __restrict__ q,
+                     uint8_t* __restrict__ atoms) {
+  const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t blk = g >> 2;
+  const int part = (int)(g & 3);
+  const bool live = blk < nblocks;
+  const int64_t row = live ? blk / kblocks : 0;
+  const int kb = live ? (int)(blk - row * kblocks) : 0;
+  float v[8];
+  if (live) {
+    const T* p = src + row * ld + (int64_t)kb * 32 + part * 8;
+    if constexpr (sizeof(T) == 2) {
+      Vec16<T> a;
+      a.raw = ldg16(p);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = a.get(i);
+    } else {
+      Vec16<T> a, b;
+      a.raw = ldg16(p);
+      b.raw = ldg16(p + 4);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) { v[i] = a.get(i); v[4 + i] = b.get(i); }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = 0.f;
+  }
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+  if (!live) return;
+  const int e = block_exponent(amax);
+  const float mul = pow2_neg(e);
+  uint2 out;
+  out.x = e4m3_pair(v[1] * mul, v[0] * mul) | (e4m3_pair(v[3] * mul, v[2] * mul) << 16);
+  out.y = e4m3_pair(v[5] * mul, v[4] * mul) | (e4m3_pair(v[7] * mul, v[6] * mul) << 16);
+  *reinterpret_cast<uint2*>(q + blk * 32 + part * 8) = out;
+  if (part == 0) {
+    const int rt = row_tile[row];
+    if (rt >= 0)
+      atoms[((int64_t)(rt >> 7) * (kblocks >> 2) + (kb >> 2)) * 512 + atom_byte(rt & 127, kb & 3)] =
+          (uint8_t)(e + 127);
+  }
+}
+
+// axis 1 (32-row blocks restarting at every segment) with scales written as stage
+// atoms: atom (stage * K/128 + column / 128), stage = 128-row stages of the segments
+// before + (row - segment start) / 128.  The blocks of a segment's last stage that lie
+// past its end get scale byte 127 (2^0), so that the zero rows there stay zero.
+template <typename T>
+__global__ void __launch_bounds__(128)
+mx_cols_atoms_kernel(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
+                     const int32_t* __restrict__ seg, int nseg, uint8_t* __restrict__ q,
+                     uint8_t* __restrict__ atoms) {
+  __shared__ int32_t s_pre[1026];   // 32-row block prefix per segment
+  __shared__ int32_t s_stg[1026];   // 128-row stage prefix per segment
+  __shared__ int32_t s_seg[1026];
+  const int tid = threadIdx.x;
+  for (int g = tid; g <= nseg; g += blockDim.x) s_seg[g] = seg ? seg[g] : (g == 0 ? 0 : (int)rows);
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0, st = 0;
+    for (int g = 0; g < nseg; ++g) {
+      s_pre[g] = acc;
+      s_stg[g] = st;
+      acc += (s_seg[g + 1] - s_seg[g] + 31) / 32;
+      st += (s_seg[g + 1] - s_seg[g] + 127) / 128;
+    }
+    s_pre[nseg] = acc;
+    s_stg[nseg] = st;
+  }
+  __syncthreads();
+  const int total = s_pre[nseg];
+  const int64_t col = ((int64_t)blockIdx.x * blockDim.x + tid) * 8;
+  if (col >= K) return;
+  const int64_t kq = K >> 7;
+  for (int rb = blockIdx.y; rb < total; rb += gridDim.y) {
+    int lo = 0, hi = nseg - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_pre[mid] <= rb) lo = mid; else hi = mid - 1;
+    }
+    const int g = lo;
+    const int lb = rb - s_pre[g];
+    const int64_t r0 = s_seg[g] + (int64_t)lb * 32;
+    const int64_t r1 = min((int64_t)s_seg[g + 1], r0 + 32);
+    float amax[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax[i] = 0.f;
+    for (int64_t r = r0; r < r1; ++r) {
+      const T* p = src + r * ld + col;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax[i] = fmaxf(amax[i], fabsf(to_f32(p[i])));
+    }
+    int ex[8];
+    float mul[8];
+    uint8_t* at = atoms + ((int64_t)(s_stg[g] + (lb >> 2)) * kq + (col >> 7)) * 512;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      ex[i] = block_exponent(amax[i]);
+      mul[i] = pow2_neg(ex[i]);
+      at[atom_byte((int)((col + i) & 127), lb & 3)] = (uint8_t)(ex[i] + 127);
+    }
+    if (rb == s_pre[g + 1] - 1) {  // the segment's last block: fill the rest of its stage
+      for (int kb = (lb & 3) + 1; kb < 4; ++kb)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) at[atom_byte((int)((col + i) & 127), kb)] = 0x7F;
+    }
+    for (int64_t r = r0; r < r1; ++r) {
+      const T* p = src + r * ld + col;
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = to_f32(p[i]) * mul[i];
+      uint2 out;
+      out.x = e4m3_pair(v[1], v[0]) | (e4m3_pair(v[3], v[2]) << 16);
+      out.y = e4m3_pair(v[5], v[4]) | (e4m3_pair(v[7], v[6]) << 16);
+      *reinterpret_cast<uint2*>(q + r * K + col) = out;
+    }
+  }
+}
+
+// FP32 master weights -> both MXFP8 copies in one pass over a 128 x 128 tile of one
+// expert's [Rw, Kw] matrix: q0 / s0 in blocks of 32 along a row (K-major GEMM operand),
+// q1 / s1 in blocks of 32 rows within a column (MN-major GEMM operand).
+//   s0 atom ((e * Rw/128 + tile) * Kw/128 + kq); with pair_f (W1 of the SwiGLU forward)
+//   a tile is 64 gate rows (64 j ..) followed by the 64 up rows (f + 64 j ..).
+//   s1 atom ((e * Rw/128 + kq) * Kw/128 + column tile), kq the 128-row stage.
+constexpr int kWPitch = 132;  // fp32 pitch of the staged tile (bank-conflict-free columns)
+__global__ void __launch_bounds__(256)
+mx_weights_kernel(const float* __restrict__ w, int Rw, int Kw, int pair_f, uint8_t* __restrict__ q0,
+                  uint8_t* __restrict__ s0, uint8_t* __restrict__ q1, uint8_t* __restrict__ s1) {
+  extern __shared__ float tile[];                       // [128][kWPitch]
+  uint8_t* qt = reinterpret_cast<uint8_t*>(tile + 128 * kWPitch);  // [128][128] q1 bytes
+  const int e = blockIdx.z, rt = blockIdx.y, ct = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int64_t row0 = (int64_t)e * Rw + rt * 128;
+  const int col0 = ct * 128;
+  // pass 1: blocks along rows; a quad of lanes covers one 32-wide block
+#pragma unroll 1
+  for (int it = 0; it < 8; ++it) {
+    const int task = it * 256 + tid;          // 2048 = 128 rows x 4 blocks x 4 parts
+    const int r = task >> 4, kb = (task >> 2) & 3, part = task & 3;
+    const float* p = w + (row0 + r) * Kw + col0 + kb * 32 + part * 8;
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p + 4));
+    float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    *reinterpret_cast<float4*>(tile + r * kWPitch + kb * 32 + part * 8) = a;
+    *reinterpret_cast<float4*>(tile + r * kWPitch + kb * 32 + part * 8 + 4) = b;
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    const int ex = block_exponent(amax);
+    const float mul = pow2_neg(ex);
+    uint2 out;
+    out.x = e4m3_pair(v[1] * mul, v[0] * mul) | (e4m3_pair(v[3] * mul, v[2] * mul) << 16);
+    out.y = e4m3_pair(v[5] * mul, v[4] * mul) | (e4m3_pair(v[7] * mul, v[6] * mul) << 16);
+    *reinterpret_cast<uint2*>(q0 + (row0 + r) * Kw + col0 + kb * 32 + part * 8) = out;
+    if (part == 0) {
+      const int rr = rt * 128 + r;               // row inside the expert
+      int atile, ai;
+      if (pair_f) {
+        const bool up = rr >= pair_f;
+        const int rl = up ? rr - pair_f : rr;
+        atile = rl >> 6;
+        ai = (up ? 64 : 0) + (rl & 63);
+      } else {
+        atile = rr >> 7;
+        ai = rr & 127;
+      }
+      s0[(((int64_t)e * (Rw >> 7) + atile) * (Kw >> 7) + ct) * 512 + atom_byte(ai, kb)] =
+          (uint8_t)(ex + 127);
+    }
+  }
+  (void)lane;
+  __syncthreads();
+  // pass 2: blocks of 32 rows within a column
+#pragma unroll 1
+  for (int it = 0; it < 2; ++it) {
+    const int c = tid & 127, rb = (tid >> 7) + 2 * it;
+    float amax = 0.f;
+#pragma unroll 8
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(tile[(rb * 32 + i) * kWPitch + c]));
+    const int ex = block_exponent(amax);
+    const float mul = pow2_neg(ex);
+#pragma unroll 8
+    for (int i = 0; i < 32; i += 2) {
+      const uint32_t pr = e4m3_pair(tile[(rb * 32 + i + 1) * kWPitch + c] * mul,
+                                    tile[(rb * 32 + i) * kWPitch + c] * mul);
+      qt[(rb * 32 + i) * 128 + c] = (uint8_t)(pr & 0xFF);
+      qt[(rb * 32 + i + 1) * 128 + c] = (uint8_t)(pr >> 8);
+    }
+    s1[(((int64_t)e * (Rw >> 7) + rt) * (Kw >> 7) + ct) * 512 + atom_byte(c, rb)] = (uint8_t)(ex + 127);
+  }
+  __syncthreads();
+  // write the q1 tile: 128 rows x 128 bytes, 16 bytes per thread and step
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int idx = it * 256 + tid;            // 1024 pieces of 16 bytes
+    const int r = idx >> 3, c16 = idx & 7;
+    *reinterpret_cast<uint4*>(q1 + (row0 + r) * Kw + col0 + c16 * 16) =
+        *reinterpret_cast<const uint4*>(qt + r * 128 + c16 * 16);
+  }
+}
+
 }  // namespace
+
+cudaError_t row_tile_launch(const int32_t* offsets, int E, int64_t rows, int32_t* out, cudaStream_t st) {
+  if (rows == 0) return cudaSuccess;
+  const int grid = (int)std::min<int64_t>((rows + 255) / 256, 1184);
+  row_tile_kernel<<<grid, 256, 0, st>>>(offsets, E, rows, out);
+  return cudaGetLastError();
+}
+
+cudaError_t mxfp8_rows_atoms(int64_t rows, int64_t K, int64_t ld, const void* src_bf16,
+                             const int32_t* row_tile, uint8_t* q, uint8_t* atoms, cudaStream_t st) {
+  if (rows == 0) return cudaSuccess;
+  const int64_t nblocks = rows * K / 32;
+  const int grid = (int)((nblocks * 4 + 255) / 256);
+  mx_rows_atoms_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(src_bf16), nblocks, K / 32, ld, row_tile, q, atoms);
+  return cudaGetLastError();
+}
+
+cudaError_t mxfp8_cols_atoms(int64_t rows, int64_t K, int64_t ld, const void* src_bf16,
+                             const int32_t* seg, int nseg, uint8_t* q, uint8_t* atoms,
+                             cudaStream_t st) {
+  if (rows == 0) return cudaSuccess;
+  dim3 grid((unsigned)((K / 8 + 127) / 128), (unsigned)std::min<int64_t>(rows / 32 + nseg + 1, 65535));
+  mx_cols_atoms_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(src_bf16), rows, K, ld, seg, nseg, q, atoms);
+  return cudaGetLastError();
+}
+
+cudaError_t mxfp8_weights(const float* w, int E, int Rw, int Kw, int pair_f, uint8_t* q0,
+                          uint8_t* s0, uint8_t* q1, uint8_t* s1, cudaStream_t st) {
+  if (E == 0) return cudaSuccess;
+  const size_t smem = 128 * kWPitch * sizeof(float) + 128 * 128;
+  cudaError_t err = cudaFuncSetAttribute(mx_weights_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+  if (err != cudaSuccess) return err;
+  dim3 grid((unsigned)(Kw / 128), (unsigned)(Rw / 128), (unsigned)E);
+  mx_weights_kernel<<<grid, 256, smem, st>>>(w, Rw, Kw, pair_f, q0, s0, q1, s1);
+  return cudaGetLastError();
+}
 
 cudaError_t mxfp8_launch_ld(int64_t rows, int64_t K, int64_t ld, bool src_bf16, const void* src,
                             int axis, const int32_t* seg_offsets, int nseg, uint8_t* q,

@@ -9,8 +9,8 @@ is used instead (moe_padded_dispatch after the route, uniform E x capacity
 rows in the grouped FFN, dropped pairs marked -1).
 
 dtype "mxfp8": bf16 activations and router, FP32 master expert weights whose
-MXFP8 copies (four orientations, see ``moe_mx_weights``) are made by
-mxfp8_quantize at the start of every forward, i.e. once per optimizer step
+MXFP8 copies (two orientations per weight, see ``moe_mx_weights``) are made
+by moe_mx_quantize_weights at the start of every forward, i.e. once per optimizer step
 when every step is one; the grouped FFN calls run with MOE_MXFP8 and write
 FP32 weight gradients.
 """
@@ -80,13 +80,13 @@ class MoELayer:
             u8 = dict(dtype=torch.uint8, device=dev)
             self.mxq = dict(
                 w1_q=torch.empty(E * 2 * d_ff, d_model, **u8),
-                w1_s=torch.empty(E * 2 * d_ff, d_model // 32, **u8),
+                w1_s=torch.empty(E * 2 * d_ff * d_model // 32, **u8),
                 w1t_q=torch.empty(E * 2 * d_ff, d_model, **u8),
-                w1t_s=torch.empty(E * 2 * d_ff // 32, d_model, **u8),
+                w1t_s=torch.empty(E * 2 * d_ff * d_model // 32, **u8),
                 w2_q=torch.empty(E * d_model, d_ff, **u8),
-                w2_s=torch.empty(E * d_model, d_ff // 32, **u8),
+                w2_s=torch.empty(E * d_model * d_ff // 32, **u8),
                 w2t_q=torch.empty(E * d_model, d_ff, **u8),
-                w2t_s=torch.empty(E * d_model // 32, d_ff, **u8),
+                w2t_s=torch.empty(E * d_model * d_ff // 32, **u8),
             )
             self.mx = capi.moe_mx_weights(**{k: v.data_ptr() for k, v in self.mxq.items()})
         else:
@@ -108,11 +108,7 @@ class MoELayer:
     def quantize_weights(self, w1, w2, stream=None):
         """MXFP8 copies of the FP32 master weights w1 [E, 2f, d], w2 [E, d, f]:
         blocks along each GEMM's contraction axis (d and 2f for W1, f and d for W2)."""
-        E, d, f, q = self.E, self.d, self.f, self.mxq
-        for src, rows, K, name, axis in ((w1, E * 2 * f, d, "w1", 0), (w1, E * 2 * f, d, "w1t", 1),
-                                         (w2, E * d, f, "w2", 0), (w2, E * d, f, "w2t", 1)):
-            capi.mxfp8_quantize(rows, K, capi.MOE_F32, src, axis, None, 0, q[name + "_q"],
-                                q[name + "_s"], stream)
+        capi.moe_mx_quantize_weights(self.shape, w1, w2, self.mx, stream)
 
     def forward(self, x, w_router, bias, w1, w2, stream=None):
         s, dt = self.shape, self.cdtype

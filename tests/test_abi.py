@@ -162,3 +162,12 @@ def test_mxfp8_ffn_validation(lib):
     assert fwd(ws_bytes=big // 2) == capi.MOE_ERR_INVALID_ARG
     assert bwd(dw_dtype=capi.MOE_BF16) == capi.MOE_ERR_INVALID_ARG       # dW is fp32
     assert bwd(ws_bytes=1024) == capi.MOE_ERR_INVALID_ARG
+
+
+def test_mx_quantize_weights_validation(lib):
+    g = lib.moe_mx_quantize_weights
+    mx = _mxw()
+    assert g(_shape(d_model=192), FAKE, FAKE, ctypes.addressof(mx), None) == capi.MOE_ERR_UNSUPPORTED
+    assert g(_shape(), None, FAKE, ctypes.addressof(mx), None) == capi.MOE_ERR_INVALID_ARG
+    assert g(_shape(), FAKE, FAKE, None, None) == capi.MOE_ERR_INVALID_ARG
+    assert g(_shape(), FAKE, FAKE, ctypes.addressof(_mxw(w1t_q=FAKE + 1)), None) == capi.MOE_ERR_INVALID_ARG

@@ -69,16 +69,54 @@ def test_mxfp8_layer_matches_oracle(name):
         assert not L.dw1[e].any() and not L.dw2[e].any()
 
 
+def _atom_rows_blocks():
+    """Row and 32-block index of each byte of a 512-byte scale atom (the layout
+    documented with moe_mx_weights: byte (r % 32) * 16 + (r / 32) * 4 + kb)."""
+    b = np.arange(512)
+    return (b // 16) + 32 * ((b % 16) // 4), b % 4
+
+
+def _k_major_plain(atoms, E, rows, K, pair_f=0):
+    """Atoms of a K-major weight copy -> plain scales [E * rows, K / 32]."""
+    r, kb = _atom_rows_blocks()
+    a = atoms.reshape(E, rows // 128, K // 128, 512)
+    e, t, j, b = np.indices(a.shape)
+    rr = t * 128 + r[b]
+    if pair_f:                      # atom t: 64 gate rows 64 t .., then 64 up rows f + 64 t ..
+        i = r[b]
+        rr = np.where(i < 64, 64 * t + i, pair_f + 64 * t + (i - 64))
+    out = np.full((E * rows, K // 32), -1, dtype=np.int64)
+    out[e * rows + rr, 4 * j + kb[b]] = a
+    return out
+
+
+def _mn_major_plain(atoms, E, rows, K):
+    """Atoms of a column-block weight copy -> plain scales [E * rows / 32, K]."""
+    r, kb = _atom_rows_blocks()
+    a = atoms.reshape(E, rows // 128, K // 128, 512)
+    e, j, nt, b = np.indices(a.shape)
+    out = np.full((E * rows // 32, K), -1, dtype=np.int64)
+    out[e * (rows // 32) + 4 * j + kb[b], nt * 128 + r[b]] = a
+    return out
+
+
 def test_mxfp8_weight_copies_are_byte_exact():
     cfg = CASES["mx_e16_odd"]
     cpu, L = run_layer(cfg)
     E, d, f = cfg.E, cfg.d_model, cfg.d_ff
     w1 = f64(cpu["w1"]).reshape(E * 2 * f, d)
     w2 = f64(cpu["w2"]).reshape(E * d, f)
+    got = {k: v.cpu().numpy() for k, v in L.mxq.items()}
+    plain = {
+        "w1": _k_major_plain(got["w1_s"], E, 2 * f, d, pair_f=f),
+        "w1t": _mn_major_plain(got["w1t_s"], E, 2 * f, d),
+        "w2": _k_major_plain(got["w2_s"], E, d, f),
+        "w2t": _mn_major_plain(got["w2t_s"], E, d, f),
+    }
     for name, src, axis in (("w1", w1, 0), ("w1t", w1, 1), ("w2", w2, 0), ("w2t", w2, 1)):
-        q, s = mx.mxfp8_quantize(src, axis=axis)
-        assert np.array_equal(L.mxq[name + "_q"].cpu().numpy(), q), name
-        assert np.array_equal(L.mxq[name + "_s"].cpu().numpy(), s), name
+        q, sc = mx.mxfp8_quantize(src, axis=axis)
+        assert np.array_equal(got[name + "_q"], q), name
+        assert np.array_equal(plain[name], sc), name
 
 
 def test_mxfp8_is_closer_to_its_oracle_than_to_the_unquantised_layer():
