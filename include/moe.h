@@ -165,8 +165,7 @@ moe_status moe_permute(moe_shape shape, int dtype, const void* x, const int32_t*
  * M or N) x 4 consecutive 32-blocks kb along its K, the scale of (r, kb) at byte
  *   (r % 32) * 16 + (r / 32) * 4 + kb.
  * Atom order, with j a 128-wide K stage:
- *   w1_s   atom (e * f/64 + t) * d/128 + j; atom rows 0..63 are the gate rows 64t..,
- *          rows 64..127 the up rows f + 64t.. of W1[e] (the forward's gate/up tile)
+ *   w1_s   atom (e * 2f/128 + r / 128) * d/128 + j, rows r = rows of W1[e]
  *   w1t_s  atom (e * 2f/128 + j) * d/128 + n / 128, rows n = columns of W1[e],
  *          K = its 2f rows
  *   w2_s   atom (e * d/128 + r / 128) * f/128 + j, rows r = rows of W2[e]

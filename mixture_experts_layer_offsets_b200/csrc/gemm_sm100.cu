@@ -107,14 +107,20 @@ template <int BN, bool PAIR = false, int EPI = 1, bool FP8 = false> struct Cfg {
   // PAIR: a CTA pair computes a 256-row tile; each CTA holds its 128 A rows and half
   // of the BN B rows (cta_group::2).
   // FP8 (MXFP8): 128 E4M3 elements (128 bytes) of K per stage, plus the stage's scale
-  // atoms for A (512 B) and B (BN / 128 x 512 B); TMEM columns 2 BN .. 2 BN + 7 hold the
-  // scales of the stage being multiplied.
+  // atoms for A (512 B) and B (BN / 128 x 512 B); each stage's scales go to one of 16
+  // slots of 8 TMEM columns after the accumulators.
   static constexpr int kBKe = FP8 ? 128 : BK;  // K elements per stage
   static constexpr uint32_t kBBytes = (PAIR ? BN / 2 : BN) * 128;
-  static constexpr uint32_t kSfBytes = FP8 ? 512 + (BN / 128) * 512 : 0;
+  // FP8: A atom (512 B) + BN/128 B atoms, padded to keep stages 1024-byte aligned
+  static constexpr uint32_t kSfBytes = FP8 ? ((512 + (BN / 128) * 512 + 1023) / 1024) * 1024 : 0;
   static constexpr uint32_t kStage = kABytes + kBBytes + kSfBytes;
   static_assert(kStage % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
-  static constexpr uint32_t kSfCol = 2 * BN;  // FP8: scale columns in TMEM
+  // accumulator buffers: two (the epilogue of one tile overlaps the main loop of the
+  // next), except for 256-wide MXFP8 tiles, whose scale columns leave room for one
+  static constexpr int kAccBufs = (FP8 && BN == 256) ? 1 : 2;
+  // FP8: 8 slots of 16 scale columns after the accumulators (A at +0, B atoms at +4, +8)
+  static constexpr uint32_t kSfCol = kAccBufs * BN;
+  static_assert(!FP8 || kSfCol + 8 * 16 <= 512, "scale slots fit in TMEM");
   static constexpr uint32_t kTmemCols = FP8 ? 512 : 2 * BN;
   static constexpr int kBoxRows = BN < 128 ? BN : 128;  // rows of one K-major B box
   static constexpr int kTileM = PAIR ? 2 * BM : BM;     // rows of one scheduled tile
@@ -398,13 +404,12 @@ template <int BN, bool A_MN, bool B_MN, int EPI, bool GROUP_K, bool PAIR = false
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
   using C = Cfg<BN, PAIR, EPI, FP8>;
-  static_assert(!FP8 || (BN == 128 && !PAIR), "MXFP8 tiles: 128 x 128, single CTA");
-  // epilogue warps 6..9 idle when a thread must hold a whole row (router) or the
-  // SwiGLU gate/up halves are 64 columns wide (BN = 128)
-  constexpr bool kHalfIdle = EPI == EPI_ROUTER || (EPI == EPI_SWIGLU_FWD && BN == 128);
+  static_assert(!FP8 || ((BN == 128 || BN == 256) && !PAIR), "MXFP8 tiles: 128 x 128 or 128 x 256, single CTA");
+  static_assert(!FP8 || EPI != EPI_SWIGLU_FWD || BN == 256, "MXFP8 SwiGLU tiles pair 128 gate with 128 up columns");
+  // epilogue warps 6..9 idle when a thread must hold a whole row (router)
+  constexpr bool kHalfIdle = EPI == EPI_ROUTER;
   constexpr int S = C::kStages;
-  static_assert(EPI != EPI_SWIGLU_FWD || BN == 256 || (FP8 && BN == 128),
-                "SwiGLU forward pairs BN/2 gate with BN/2 up columns (128 + 128, or 64 + 64 for MXFP8)");
+  static_assert(EPI != EPI_SWIGLU_FWD || BN == 256, "SwiGLU forward pairs 128 gate with 128 up columns");
   static_assert(!PAIR || (BN == 256 && !A_MN && !GROUP_K && EPI != EPI_ROUTER),
                 "CTA pairs serve the row-grouped GEMMs with N = 256");
   extern __shared__ uint8_t smem_raw[];
@@ -522,52 +527,73 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
       tma_prefetch_desc(&p.tmA);
       tma_prefetch_desc(&p.tmB);
       uint32_t it = 0;
+      int s = 0;
+      uint32_t ph = 1;  // the first pass over the ring finds every stage free
       bool ok = true;
       const int kq = GROUP_K ? 0 : p.K / C::kBKe;
       for (int t = tile0; t < total && ok; t += tstride) {
+        if (*s_abort) { ok = false; break; }
         const TileInfo ti = decode(t);
         const uint8_t* atomA;
         const uint8_t* atomB;
+        // atomB2: the second B atom of a 256-wide tile (K-major B only; MN-major atoms
+        // of one stage are adjacent and travel in one copy)
+        const uint8_t* atomB2 = nullptr;
         if constexpr (GROUP_K) {
           atomA = p.sfa + ((int64_t)s_pre[ti.g] * (p.M / BM) + ti.m0 / BM) * 512;
-          atomB = p.sfb + ((int64_t)s_pre[ti.g] * (p.N / BN) + ti.n0 / BN) * 512;
+          atomB = p.sfb + ((int64_t)s_pre[ti.g] * (p.N / 128) + ti.n0 / 128) * 512;
         } else {
           const int mt = s_pre[ti.g] / nN + (ti.m0 - s_off[ti.g]) / BM;
           atomA = p.sfa + (int64_t)mt * kq * 512;
           if constexpr (!B_MN) {
-            const int nt = ti.n0 / (EPI == EPI_SWIGLU_FWD ? BN / 2 : BN);
-            atomB = p.sfb + ((int64_t)ti.g * nN + nt) * kq * 512;
+            // K-major weights: atom (expert row tile) * K/128 + k stage, 128 rows per tile
+            const int ntiles = p.b_rows / 128;
+            if constexpr (EPI == EPI_SWIGLU_FWD && BN == 256) {
+              atomB = p.sfb + ((int64_t)ti.g * ntiles + ti.n0 / 128) * kq * 512;
+              atomB2 = p.sfb + ((int64_t)ti.g * ntiles + (p.f + ti.n0) / 128) * kq * 512;
+            } else {
+              atomB = p.sfb + ((int64_t)ti.g * ntiles + ti.n0 / 128) * kq * 512;
+              if constexpr (BN == 256) atomB2 = atomB + (int64_t)kq * 512;
+            }
           } else {
-            atomB = p.sfb + ((int64_t)ti.g * kq * (p.N / BN) + ti.n0 / BN) * 512;
+            atomB = p.sfb + ((int64_t)ti.g * kq * (p.N / 128) + ti.n0 / 128) * 512;
           }
         }
-        for (int kb = 0; kb < ti.nkb; ++kb, ++it) {
-          if (*s_abort) { ok = false; break; }
-          const int s = it % S;
-          if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1)) { fail(); ok = false; break; }
+        for (int kb = 0; kb < ti.nkb; ++kb, ++it, s = (s + 1 == S ? 0 : s + 1), ph ^= (s == 0)) {
+          if (!mbar_wait(&empty[s], ph)) { fail(); ok = false; break; }
           uint8_t* sa = smem + s * C::kStage;
           uint8_t* sb = sa + kABytes;
           uint8_t* sf = sb + C::kBBytes;
           const int kc = kb * C::kBKe;  // first K element of the stage
-          mbar_arrive_expect_tx(&full[s], kABytes + C::kBBytes + 1024);
+          constexpr uint32_t kSfB = (BN / 128) * 512;
+          mbar_arrive_expect_tx(&full[s], kABytes + C::kBBytes + 512 + kSfB);
           if constexpr (!A_MN) tma_load_2d(sa, &p.tmA, kc, ti.m0, &full[s]);
           else tma_load_2d(sa, &p.tmA, ti.m0, ti.kbase + kc, &full[s]);
           if constexpr (!B_MN) {
+            // boxes of BN/2 rows (SwiGLU: gate rows, then up rows) or of 128 rows
             if constexpr (EPI == EPI_SWIGLU_FWD) {
               tma_load_2d(sb, &p.tmB, kc, ti.kbase + ti.n0, &full[s]);
-              tma_load_2d(sb + 64 * 128, &p.tmB, kc, ti.kbase + p.f + ti.n0, &full[s]);
+              tma_load_2d(sb + (BN / 2) * 128, &p.tmB, kc, ti.kbase + p.f + ti.n0, &full[s]);
             } else {
-              tma_load_2d(sb, &p.tmB, kc, ti.kbase + ti.n0, &full[s]);
+#pragma unroll
+              for (int i = 0; i < BN / 128; ++i)
+                tma_load_2d(sb + i * 16384, &p.tmB, kc, ti.kbase + ti.n0 + 128 * i, &full[s]);
             }
           } else {
-            tma_load_2d(sb, &p.tmB, ti.n0, ti.kbase + kc, &full[s]);
+#pragma unroll
+            for (int i = 0; i < BN / 128; ++i)
+              tma_load_2d(sb + i * 16384, &p.tmB, ti.n0 + 128 * i, ti.kbase + kc, &full[s]);
           }
           if constexpr (GROUP_K) {
             bulk_load(sf, atomA + (int64_t)kb * (p.M / BM) * 512, 512, &full[s]);
-            bulk_load(sf + 512, atomB + (int64_t)kb * (p.N / BN) * 512, 512, &full[s]);
+            bulk_load(sf + 512, atomB + (int64_t)kb * (p.N / 128) * 512, kSfB, &full[s]);
+          } else if constexpr (B_MN) {
+            bulk_load(sf, atomA + kb * 512, 512, &full[s]);
+            bulk_load(sf + 512, atomB + (int64_t)kb * (p.N / 128) * 512, kSfB, &full[s]);
           } else {
             bulk_load(sf, atomA + kb * 512, 512, &full[s]);
-            bulk_load(sf + 512, atomB + (B_MN ? (int64_t)kb * (p.N / BN) * 512 : kb * 512), 512, &full[s]);
+            bulk_load(sf + 512, atomB + kb * 512, 512, &full[s]);
+            if constexpr (BN == 256) bulk_load(sf + 1024, atomB2 + kb * 512, 512, &full[s]);
           }
         }
       }
@@ -582,14 +608,15 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
       tma_prefetch_desc(&p.tmA);
       tma_prefetch_desc(&p.tmB);
       uint32_t it = 0;
+      int s = 0;
+      uint32_t ph = 1;  // the first pass over the ring finds every stage free
       bool ok = true;
       const uint32_t leader_full = PAIR ? map_to_rank(&full[0], 0) : 0;
       for (int t = tile0; t < total && ok; t += tstride) {
+        if (*s_abort) { ok = false; break; }
         const TileInfo ti = decode(t);
-        for (int kb = 0; kb < ti.nkb; ++kb, ++it) {
-          if (*s_abort) { ok = false; break; }
-          const int s = it % S;
-          if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1)) { fail(); ok = false; break; }
+        for (int kb = 0; kb < ti.nkb; ++kb, ++it, s = (s + 1 == S ? 0 : s + 1), ph ^= (s == 0)) {
+          if (!mbar_wait(&empty[s], ph)) { fail(); ok = false; break; }
           uint8_t* sa = smem + s * C::kStage;
           uint8_t* sb = sa + kABytes;
           const int kc = kb * BK;
@@ -638,15 +665,37 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
+    // One thread issues.  Its per-stage work is kept small, since at these tile sizes
+    // the issuing thread, not the tensor core, sets the pace: the ring position and the
+    // barrier parity advance incrementally, and a stage's shared-memory descriptors are
+    // the ring's base descriptors plus constants (the start-address field counts 16-byte
+    // units, and no start address of the ring reaches 2^18 bytes).
     constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)A_MN << 15) |
                                ((uint32_t)B_MN << 16) | ((uint32_t)(BN >> 3) << 17) |
                                ((uint32_t)(C::kTileM >> 4) << 24);
+    constexpr uint32_t idesc_mx = ((uint32_t)A_MN << 15) | ((uint32_t)B_MN << 16) |
+                                  ((uint32_t)(BN >> 3) << 17) | (1u << 23) | ((uint32_t)(BM >> 4) << 24);
+    // MN-major operands: LBO = distance between 64 (bf16) or 128 (fp8) element MN blocks
+    constexpr uint32_t kLboA = A_MN ? (FP8 ? 16384 : 8192) : 16;
+    constexpr uint32_t kLboB = B_MN ? (FP8 ? 16384 : 8192) : 16;
+    // advance of the start field per MMA along K (K = 16 bf16 or 32 fp8 per MMA)
+    constexpr uint32_t kStepA = (A_MN ? (FP8 ? 4096 : 2048) : 32) >> 4;
+    constexpr uint32_t kStepB = (B_MN ? (FP8 ? 4096 : 2048) : 32) >> 4;
+    constexpr uint32_t kStageU = C::kStage >> 4;
+    const uint32_t ring = smem_u32(smem);
+    const uint64_t desc_a0 = sdesc(ring, kLboA, 1024);
+    const uint64_t desc_b0 = sdesc(ring + kABytes, kLboB, 1024);
+    const uint64_t desc_f0 = sf_desc(ring + kABytes + C::kBBytes);
     uint32_t it = 0, acc_it = 0;
+    int stg = 0;
+    uint32_t ph = 0;
     bool ok = true;
     for (int t = tile0; t < total && ok && leader; t += tstride) {
+      if (__any_sync(0xffffffffu, *s_abort)) { ok = false; break; }
       const TileInfo ti = decode(t);
-      const int acc = acc_it & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&tempty[acc], ((acc_it >> 1) & 1) ^ 1))) {
+      const int acc = C::kAccBufs == 2 ? (int)(acc_it & 1) : 0;
+      const uint32_t acc_ph = C::kAccBufs == 2 ? (acc_it >> 1) & 1 : acc_it & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&tempty[acc], acc_ph ^ 1))) {
         if (lane == 0) fail();
         ok = false;
         break;
@@ -654,20 +703,20 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + acc * BN;
       for (int kb = 0; kb < ti.nkb; ++kb, ++it) {
-        if (__any_sync(0xffffffffu, *s_abort)) { ok = false; break; }
-        const int s = it % S;
-        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (it / S) & 1))) {
+        bool w = true;
+        if (lane == 0) w = mbar_wait(&full[stg], ph);
+        if (!__shfl_sync(0xffffffffu, (int)w, 0)) {
           if (lane == 0) fail();
           ok = false;
           break;
         }
         tc_fence_after();
-        uint8_t* sa = smem + s * C::kStage;
-        uint8_t* sb = sa + kABytes;
         if constexpr (GROUP_K) {
           if (kb == ti.nkb - 1 && ti.klast < C::kBKe) {
             // Rows [klast, K rows of a box) of every box hold the next expert's tokens:
             // zero them.  bf16 boxes are 64 M/N x 64 K rows (8 KB), fp8 boxes 128 x 128 (16 KB).
+            uint8_t* sa = smem + stg * C::kStage;
+            uint8_t* sb = sa + kABytes;
             constexpr int kBoxRowsK = C::kBKe;
             constexpr int kBoxBytes = kBoxRowsK * 128;
             constexpr int kABoxes = kABytes / kBoxBytes;
@@ -681,39 +730,38 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
             }
             fence_proxy_async_smem();
           }
+          __syncwarp();
         }
-        __syncwarp();
-        if (FP8 && lane == 0) {
-          // scales of this stage -> TMEM, then four K = 32 block-scaled MMAs
-          const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sb), f0 = smem_u32(sb + C::kBBytes);
-          const uint32_t tsf = tmem_base + C::kSfCol;
-          tmem_cp_sf(tsf, sf_desc(f0));
-          tmem_cp_sf(tsf + 4, sf_desc(f0 + 512));
-          constexpr uint32_t idesc_mx = ((uint32_t)A_MN << 15) | ((uint32_t)B_MN << 16) |
-                                        ((uint32_t)(BN >> 3) << 17) | (1u << 23) |
-                                        ((uint32_t)(BM >> 4) << 24);
+        if (lane == 0) {
+          const uint32_t so = (uint32_t)stg * kStageU;
+          const uint64_t ad = desc_a0 + so, bd = desc_b0 + so;
+          if constexpr (FP8) {
+            // scales of this stage -> TMEM, then four K = 32 block-scaled MMAs.  The
+            // scale slots rotate over 8 x 16 TMEM columns, so that the copy of the next
+            // stage's scales does not write columns that MMAs still in flight read; the
+            // scales of B atom i (rows 128 i ..) sit 4 i columns after the first.
+            const uint32_t tsf = tmem_base + C::kSfCol + 16 * (it & 7);
+            tmem_cp_sf(tsf, desc_f0 + so);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t ad = A_MN ? sdesc(a0 + k * 4096, 16384, 1024) : sdesc(a0 + k * 32, 16, 1024);
-            const uint64_t bd = B_MN ? sdesc(b0 + k * 4096, 16384, 1024) : sdesc(b0 + k * 32, 16, 1024);
-            const uint32_t id = idesc_mx | ((uint32_t)k << 4) | ((uint32_t)k << 29);
-            umma_mxf8(d_tmem, ad, bd, id, (kb | k) != 0, tsf | ((uint32_t)k << 30),
-                      (tsf + 4) | ((uint32_t)k << 30));
-          }
-          umma_commit(&empty[s]);
-        } else if (lane == 0) {
-          const uint32_t a0 = smem_u32(sa), b0 = smem_u32(sb);
+            for (int i = 0; i < BN / 128; ++i)
+              tmem_cp_sf(tsf + 4 + 4 * i, desc_f0 + so + ((512 + 512 * i) >> 4));
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            const uint64_t ad = A_MN ? sdesc(a0 + k * 2048, 8192, 1024) : sdesc(a0 + k * 32, 16, 1024);
-            const uint64_t bd = B_MN ? sdesc(b0 + k * 2048, 8192, 1024) : sdesc(b0 + k * 32, 16, 1024);
-            if constexpr (PAIR) umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0);
-            else umma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0);
+            for (int k = 0; k < 4; ++k)
+              umma_mxf8(d_tmem, ad + k * kStepA, bd + k * kStepB,
+                        idesc_mx | ((uint32_t)k << 4) | ((uint32_t)k << 29), (kb | k) != 0,
+                        tsf | ((uint32_t)k << 30), (tsf + 4) | ((uint32_t)k << 30));
+            umma_commit(&empty[stg]);
+          } else {
+#pragma unroll
+            for (int k = 0; k < BK / 16; ++k) {
+              if constexpr (PAIR) umma_bf16_pair(d_tmem, ad + k * kStepA, bd + k * kStepB, idesc, (kb | k) != 0);
+              else umma_bf16(d_tmem, ad + k * kStepA, bd + k * kStepB, idesc, (kb | k) != 0);
+            }
+            if constexpr (PAIR) umma_commit_pair(&empty[stg]);
+            else umma_commit(&empty[stg]);
           }
-          if constexpr (PAIR) umma_commit_pair(&empty[s]);
-          else umma_commit(&empty[s]);
         }
-        __syncwarp();
+        if (++stg == S) { stg = 0; ph ^= 1; }
       }
       if (!ok) break;
       if (lane == 0) {
@@ -752,7 +800,8 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
     for (int t = tile0; t < total && !idle; t += tstride) {
       if (__any_sync(0xffffffffu, *s_abort)) break;
       const TileInfo ti = decode(t);
-      const int acc = acc_it & 1;
+      const int acc = C::kAccBufs == 2 ? (int)(acc_it & 1) : 0;
+      const uint32_t acc_ph = C::kAccBufs == 2 ? (acc_it >> 1) & 1 : acc_it & 1;
       const bool valid = row < ti.rows;
       // SwiGLU backward: a and u of the first chunk do not depend on the
       // accumulator, so their loads are in flight while the main loop runs.
@@ -762,7 +811,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
         arow = p.act + (int64_t)(ti.m0 + row) * p.ld_act;
         if (valid) load_au(arow, ti.n0 + c0 * 32, p.f, av, uv);
       }
-      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], (acc_it >> 1) & 1))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_ph))) {
         fail();
         break;
       }
@@ -1135,11 +1184,11 @@ cudaError_t launch(const GemmParams& p, int64_t tile_bound, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-// MXFP8 variant: 128 x 128 tiles of E4M3 operands with E8M0 block scales.
-template <bool A_MN, bool B_MN, int EPI, bool GROUP_K>
+// MXFP8 variant: 128 x BN tiles of E4M3 operands with E8M0 block scales.
+template <int BN, bool A_MN, bool B_MN, int EPI, bool GROUP_K>
 cudaError_t launch_mx(const GemmParams& p, int64_t tile_bound, cudaStream_t st) {
-  auto kern = grouped_gemm_sm100<128, A_MN, B_MN, EPI, GROUP_K, false, true>;
-  constexpr size_t smem = Cfg<128, false, EPI, true>::kSmem;
+  auto kern = grouped_gemm_sm100<BN, A_MN, B_MN, EPI, GROUP_K, false, true>;
+  constexpr size_t smem = Cfg<BN, false, EPI, true>::kSmem;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tile_bound, num_sms()));
@@ -1177,6 +1226,14 @@ cudaError_t launch_pair(const GemmParams& p, int64_t pair_tile_bound, cudaStream
   const int clusters = (int)std::max<int64_t>(1, std::min<int64_t>(pair_tile_bound, dev < 64 ? max_clusters[dev] : num_sms() / 2));
   cfg.gridDim = dim3(2 * clusters);
   return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+// 256-wide MXFP8 tiles where N allows (twice the work per MMA instruction), else 128.
+// `units` is the tile count per 128 columns of N.
+template <bool A_MN, bool B_MN, int EPI, bool GROUP_K>
+cudaError_t launch_mx_n(const GemmParams& p, int N, int64_t units, cudaStream_t st) {
+  if (N % 256 == 0) return launch_mx<256, A_MN, B_MN, EPI, GROUP_K>(p, units * (N / 256), st);
+  return launch_mx<128, A_MN, B_MN, EPI, GROUP_K>(p, units * (N / 128), st);
 }
 
 GemmParams base_params(const FfnShape& s, const int32_t* offsets, int* status) {
@@ -1428,10 +1485,10 @@ size_t ffn_mx_ws_bytes(const FfnShape& s) {
 cudaError_t mx_quantize_weights(int E, int d, int f, const float* w1, const float* w2,
                                 const MxWeights& w, cudaStream_t st) {
   auto u8 = [](const uint8_t* p) { return const_cast<uint8_t*>(p); };
-  cudaError_t err = mxfp8_weights(w1, E, 2 * f, d, f, u8(w.w1_q), u8(w.w1_s), u8(w.w1t_q),
+  cudaError_t err = mxfp8_weights(w1, E, 2 * f, d, u8(w.w1_q), u8(w.w1_s), u8(w.w1t_q),
                                   u8(w.w1t_s), st);
   if (err != cudaSuccess) return err;
-  return mxfp8_weights(w2, E, d, f, 0, u8(w.w2_q), u8(w.w2_s), u8(w.w2t_q), u8(w.w2t_s), st);
+  return mxfp8_weights(w2, E, d, f, u8(w.w2_q), u8(w.w2_s), u8(w.w2t_q), u8(w.w2t_s), st);
 }
 
 cudaError_t ffn_fwd_mx(const FfnShape& s, const void* x_perm, const int32_t* offsets,
@@ -1452,14 +1509,15 @@ cudaError_t ffn_fwd_mx(const FfnShape& s, const void* x_perm, const int32_t* off
     return err;
   GemmParams p1 = mx_params(s, offsets, status);
   if (!tmap(&p1.tmA, ws + L.qx0, d, R, d, 128, 128, false, true) ||
-      !tmap(&p1.tmB, w.w1_q, d, (uint64_t)E * 2 * f, d, 128, 64, false, true) ||
+      !tmap(&p1.tmB, w.w1_q, d, (uint64_t)E * 2 * f, d, 128, 128, false, true) ||
       !tmap(&p1.tmOut, act, 3 * f, R, 3 * f, 64, 16))
     return cudaErrorInvalidValue;
   p1.sfa = ws + L.sx0;
   p1.sfb = w.w1_s;
   p1.N = f; p1.K = d; p1.b_rows = 2 * f;
   p1.out = static_cast<__nv_bfloat16*>(act); p1.ld_out = 3 * f;
-  if ((err = launch_mx<false, false, EPI_SWIGLU_FWD, false>(p1, m_tile_bound(s) * (f / 64), st)) != cudaSuccess)
+  // 128 gate + 128 up columns per tile
+  if ((err = launch_mx<256, false, false, EPI_SWIGLU_FWD, false>(p1, m_tile_bound(s) * (f / 128), st)) != cudaSuccess)
     return err;
   // h along f; down GEMM
   if ((err = mxfp8_rows_atoms(R, f, 3 * f, actb + 2 * f, rt, ws + L.qh0, ws + L.sh0, st)) != cudaSuccess)
@@ -1473,7 +1531,7 @@ cudaError_t ffn_fwd_mx(const FfnShape& s, const void* x_perm, const int32_t* off
   p2.sfb = w.w2_s;
   p2.N = d; p2.K = f; p2.b_rows = d;
   p2.out = static_cast<__nv_bfloat16*>(y_perm); p2.ld_out = d;
-  return launch_mx<false, false, EPI_STORE, false>(p2, m_tile_bound(s) * (d / 128), st);
+  return launch_mx_n<false, false, EPI_STORE, false>(p2, d, m_tile_bound(s), st);
 }
 
 cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_perm, const void* act,
@@ -1504,7 +1562,7 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
     p3.N = f; p3.K = d; p3.b_rows = d;
     p3.out = dadu; p3.ld_out = 2 * f;
     p3.act = actb; p3.ld_act = 3 * f;
-    if ((err = launch_mx<false, true, EPI_SWIGLU_BWD, false>(p3, m_tile_bound(s) * (f / 128), st)) != cudaSuccess)
+    if ((err = launch_mx_n<false, true, EPI_SWIGLU_BWD, false>(p3, f, m_tile_bound(s), st)) != cudaSuccess)
       return err;
     // dgrad 2: dx = [da | du] W1 ([da | du] along 2f, W1 along its 2f rows)
     if ((err = mxfp8_rows_atoms(R, 2 * f, 2 * f, dadu, rt, ws + L.qda0, ws + L.sda0, st)) != cudaSuccess)
@@ -1518,7 +1576,7 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
     p4.sfb = w.w1t_s;
     p4.N = d; p4.K = 2 * f; p4.b_rows = 2 * f;
     p4.out = static_cast<__nv_bfloat16*>(dx_perm); p4.ld_out = d;
-    if ((err = launch_mx<false, true, EPI_STORE, false>(p4, m_tile_bound(s) * (d / 128), st)) != cudaSuccess)
+    if ((err = launch_mx_n<false, true, EPI_STORE, false>(p4, d, m_tile_bound(s), st)) != cudaSuccess)
       return err;
     // wgrad operands along the token axis, 32-row blocks restarting at each expert
     if ((err = mxfp8_cols_atoms(R, d, d, dy_perm, offsets, E, ws + L.qdy1, ws + L.sdy1, st)) != cudaSuccess ||
@@ -1537,7 +1595,7 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
   p5.sfb = ws + L.sh1;
   p5.M = d; p5.N = f;
   p5.out_f32 = dw2; p5.ld_out = f; p5.out_group = (int64_t)d * f;
-  if ((err = launch_mx<true, true, EPI_WGRAD, true>(p5, (int64_t)E * (d / 128) * (f / 128), st)) != cudaSuccess)
+  if ((err = launch_mx_n<true, true, EPI_WGRAD, true>(p5, f, (int64_t)E * (d / 128), st)) != cudaSuccess)
     return err;
   // wgrad 1: dW1[e] = [da | du]^T x  (M = 2f, N = d)
   GemmParams p6 = mx_params(s, offsets, status);
@@ -1549,7 +1607,7 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
   p6.sfb = ws + L.sx1;
   p6.M = 2 * f; p6.N = d;
   p6.out_f32 = dw1; p6.ld_out = d; p6.out_group = (int64_t)2 * f * d;
-  return launch_mx<true, true, EPI_WGRAD, true>(p6, (int64_t)E * (2 * f / 128) * (d / 128), st);
+  return launch_mx_n<true, true, EPI_WGRAD, true>(p6, d, (int64_t)E * (2 * f / 128), st);
 }
 
 }  // namespace moe

@@ -83,8 +83,8 @@ cudaError_t mxfp8_rows_atoms(int64_t rows, int64_t K, int64_t ld, const void* sr
 cudaError_t mxfp8_cols_atoms(int64_t rows, int64_t K, int64_t ld, const void* src_bf16,
                              const int32_t* seg, int nseg, uint8_t* q, uint8_t* atoms,
                              cudaStream_t st);
-cudaError_t mxfp8_weights(const float* w, int E, int Rw, int Kw, int pair_f, uint8_t* q0,
-                          uint8_t* s0, uint8_t* q1, uint8_t* s1, cudaStream_t st);
+cudaError_t mxfp8_weights(const float* w, int E, int Rw, int Kw, uint8_t* q0, uint8_t* s0,
+                          uint8_t* q1, uint8_t* s1, cudaStream_t st);
 
 // ---------------------------------------------------------- grouped FFN
 struct FfnShape {

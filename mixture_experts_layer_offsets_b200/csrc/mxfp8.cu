@@ -152,6 +152,23 @@ mx_cols_kernel(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
   }
 }
 
+// eight consecutive elements (16-byte aligned for bf16, 32-byte for fp32) as floats
+template <typename T>
+__device__ __forceinline__ void load8(const T* p, float* v) {
+  if constexpr (sizeof(T) == 2) {
+    Vec16<T> a;
+    a.raw = ldg16(p);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = a.get(i);
+  } else {
+    Vec16<T> a, b;
+    a.raw = ldg16(p);
+    b.raw = ldg16(p + 4);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) { v[i] = a.get(i); v[4 + i] = b.get(i); }
+  }
+}
+
 // ---------------------------------------------------------------- scale atoms
 // The block-scaled MMA takes its E8M0 scales from TMEM, which each pipeline stage fills
 // from a 512-byte shared-memory atom: 128 rows (of M or N) x 4 blocks of 32 along K, the
@@ -297,9 +314,10 @@ mx_cols_atoms_kernel(const T* __restrict__ src, int64_t rows, int64_t K, int64_t
 #pragma unroll
     for (int i = 0; i < 8; ++i) amax[i] = 0.f;
     for (int64_t r = r0; r < r1; ++r) {
-      const T* p = src + r * ld + col;
+      float v[8];
+      load8(src + r * ld + col, v);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) amax[i] = fmaxf(amax[i], fabsf(to_f32(p[i])));
+      for (int i = 0; i < 8; ++i) amax[i] = fmaxf(amax[i], fabsf(v[i]));
     }
     int ex[8];
     float mul[8];
@@ -316,10 +334,10 @@ mx_cols_atoms_kernel(const T* __restrict__ src, int64_t rows, int64_t K, int64_t
         for (int i = 0; i < 8; ++i) at[atom_byte((int)((col + i) & 127), kb)] = 0x7F;
     }
     for (int64_t r = r0; r < r1; ++r) {
-      const T* p = src + r * ld + col;
       float v[8];
+      load8(src + r * ld + col, v);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = to_f32(p[i]) * mul[i];
+      for (int i = 0; i < 8; ++i) v[i] *= mul[i];
       uint2 out;
       out.x = e4m3_pair(v[1], v[0]) | (e4m3_pair(v[3], v[2]) << 16);
       out.y = e4m3_pair(v[5], v[4]) | (e4m3_pair(v[7], v[6]) << 16);
@@ -331,12 +349,11 @@ mx_cols_atoms_kernel(const T* __restrict__ src, int64_t rows, int64_t K, int64_t
 // FP32 master weights -> both MXFP8 copies in one pass over a 128 x 128 tile of one
 // expert's [Rw, Kw] matrix: q0 / s0 in blocks of 32 along a row (K-major GEMM operand),
 // q1 / s1 in blocks of 32 rows within a column (MN-major GEMM operand).
-//   s0 atom ((e * Rw/128 + tile) * Kw/128 + kq); with pair_f (W1 of the SwiGLU forward)
-//   a tile is 64 gate rows (64 j ..) followed by the 64 up rows (f + 64 j ..).
+//   s0 atom ((e * Rw/128 + row tile) * Kw/128 + kq), kq the 128-column stage.
 //   s1 atom ((e * Rw/128 + kq) * Kw/128 + column tile), kq the 128-row stage.
 constexpr int kWPitch = 132;  // fp32 pitch of the staged tile (bank-conflict-free columns)
 __global__ void __launch_bounds__(256)
-mx_weights_kernel(const float* __restrict__ w, int Rw, int Kw, int pair_f, uint8_t* __restrict__ q0,
+mx_weights_kernel(const float* __restrict__ w, int Rw, int Kw, uint8_t* __restrict__ q0,
                   uint8_t* __restrict__ s0, uint8_t* __restrict__ q1, uint8_t* __restrict__ s1) {
   extern __shared__ float tile[];                       // [128][kWPitch]
   uint8_t* qt = reinterpret_cast<uint8_t*>(tile + 128 * kWPitch);  // [128][128] q1 bytes
@@ -344,14 +361,22 @@ mx_weights_kernel(const float* __restrict__ w, int Rw, int Kw, int pair_f, uint8
   const int tid = threadIdx.x, lane = tid & 31;
   const int64_t row0 = (int64_t)e * Rw + rt * 128;
   const int col0 = ct * 128;
-  // pass 1: blocks along rows; a quad of lanes covers one 32-wide block
-#pragma unroll 1
+  // pass 1: blocks along rows; a quad of lanes covers one 32-wide block.  All sixteen
+  // 16-byte loads of a thread are issued before any is used.
+  float4 ld[16];
+#pragma unroll
   for (int it = 0; it < 8; ++it) {
     const int task = it * 256 + tid;          // 2048 = 128 rows x 4 blocks x 4 parts
     const int r = task >> 4, kb = (task >> 2) & 3, part = task & 3;
     const float* p = w + (row0 + r) * Kw + col0 + kb * 32 + part * 8;
-    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
-    const float4 b = __ldg(reinterpret_cast<const float4*>(p + 4));
+    ld[2 * it] = __ldg(reinterpret_cast<const float4*>(p));
+    ld[2 * it + 1] = __ldg(reinterpret_cast<const float4*>(p + 4));
+  }
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int task = it * 256 + tid;
+    const int r = task >> 4, kb = (task >> 2) & 3, part = task & 3;
+    const float4 a = ld[2 * it], b = ld[2 * it + 1];
     float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
     *reinterpret_cast<float4*>(tile + r * kWPitch + kb * 32 + part * 8) = a;
     *reinterpret_cast<float4*>(tile + r * kWPitch + kb * 32 + part * 8 + 4) = b;
@@ -366,21 +391,8 @@ mx_weights_kernel(const float* __restrict__ w, int Rw, int Kw, int pair_f, uint8
     out.x = e4m3_pair(v[1] * mul, v[0] * mul) | (e4m3_pair(v[3] * mul, v[2] * mul) << 16);
     out.y = e4m3_pair(v[5] * mul, v[4] * mul) | (e4m3_pair(v[7] * mul, v[6] * mul) << 16);
     *reinterpret_cast<uint2*>(q0 + (row0 + r) * Kw + col0 + kb * 32 + part * 8) = out;
-    if (part == 0) {
-      const int rr = rt * 128 + r;               // row inside the expert
-      int atile, ai;
-      if (pair_f) {
-        const bool up = rr >= pair_f;
-        const int rl = up ? rr - pair_f : rr;
-        atile = rl >> 6;
-        ai = (up ? 64 : 0) + (rl & 63);
-      } else {
-        atile = rr >> 7;
-        ai = rr & 127;
-      }
-      s0[(((int64_t)e * (Rw >> 7) + atile) * (Kw >> 7) + ct) * 512 + atom_byte(ai, kb)] =
-          (uint8_t)(ex + 127);
-    }
+    if (part == 0)
+      s0[(((int64_t)e * (Rw >> 7) + rt) * (Kw >> 7) + ct) * 512 + atom_byte(r, kb)] = (uint8_t)(ex + 127);
   }
   (void)lane;
   __syncthreads();
@@ -442,15 +454,15 @@ cudaError_t mxfp8_cols_atoms(int64_t rows, int64_t K, int64_t ld, const void* sr
   return cudaGetLastError();
 }
 
-cudaError_t mxfp8_weights(const float* w, int E, int Rw, int Kw, int pair_f, uint8_t* q0,
-                          uint8_t* s0, uint8_t* q1, uint8_t* s1, cudaStream_t st) {
+cudaError_t mxfp8_weights(const float* w, int E, int Rw, int Kw, uint8_t* q0, uint8_t* s0,
+                          uint8_t* q1, uint8_t* s1, cudaStream_t st) {
   if (E == 0) return cudaSuccess;
   const size_t smem = 128 * kWPitch * sizeof(float) + 128 * 128;
   cudaError_t err = cudaFuncSetAttribute(mx_weights_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
   if (err != cudaSuccess) return err;
   dim3 grid((unsigned)(Kw / 128), (unsigned)(Rw / 128), (unsigned)E);
-  mx_weights_kernel<<<grid, 256, smem, st>>>(w, Rw, Kw, pair_f, q0, s0, q1, s1);
+  mx_weights_kernel<<<grid, 256, smem, st>>>(w, Rw, Kw, q0, s0, q1, s1);
   return cudaGetLastError();
 }
 

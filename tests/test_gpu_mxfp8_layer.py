@@ -76,15 +76,12 @@ def _atom_rows_blocks():
     return (b // 16) + 32 * ((b % 16) // 4), b % 4
 
 
-def _k_major_plain(atoms, E, rows, K, pair_f=0):
+def _k_major_plain(atoms, E, rows, K):
     """Atoms of a K-major weight copy -> plain scales [E * rows, K / 32]."""
     r, kb = _atom_rows_blocks()
     a = atoms.reshape(E, rows // 128, K // 128, 512)
     e, t, j, b = np.indices(a.shape)
     rr = t * 128 + r[b]
-    if pair_f:                      # atom t: 64 gate rows 64 t .., then 64 up rows f + 64 t ..
-        i = r[b]
-        rr = np.where(i < 64, 64 * t + i, pair_f + 64 * t + (i - 64))
     out = np.full((E * rows, K // 32), -1, dtype=np.int64)
     out[e * rows + rr, 4 * j + kb[b]] = a
     return out
@@ -108,7 +105,7 @@ def test_mxfp8_weight_copies_are_byte_exact():
     w2 = f64(cpu["w2"]).reshape(E * d, f)
     got = {k: v.cpu().numpy() for k, v in L.mxq.items()}
     plain = {
-        "w1": _k_major_plain(got["w1_s"], E, 2 * f, d, pair_f=f),
+        "w1": _k_major_plain(got["w1_s"], E, 2 * f, d),
         "w1t": _mn_major_plain(got["w1t_s"], E, 2 * f, d),
         "w2": _k_major_plain(got["w2_s"], E, d, f),
         "w2t": _mn_major_plain(got["w2t_s"], E, d, f),
