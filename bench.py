@@ -49,6 +49,10 @@ LAUNCHES = {"route": 3, "permute": 1, "ffn_fwd": 2, "combine": 1, "combine_bwd":
             "ffn_bwd": 4, "route_bwd": 4, "padded_dispatch": 2}
 LAUNCHES_MX = {"quantize_w": 4, "ffn_fwd": 4, "ffn_bwd": 10}
 FP8_OVER_BF16 = 2.0   # nominal dense tensor-core ratio (4.5 / 2.25 PFLOP/s)
+# DRAM bytes (read + write) of the six grouped-GEMM launches of one step, from one ncu capture
+# of this build (profiles/launches_bf16_e8.md); None where no capture of the current kernels
+# exists.
+GEMM_TRAFFIC_BYTES = {"bf16_e8": 3.862e9}
 
 
 def _peaks():
@@ -273,7 +277,9 @@ def run_ours(args, rank, world):
             "bound": "tensor", "kernel": "grouped GEMM (tcgen05), all 6 launches of a step",
             "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4) if peak else None,
-            "peak_kind": peak_kind, "traffic": None,
+            "peak_kind": peak_kind,
+            "traffic": (GEMM_TRAFFIC_BYTES.get(cfg.name) if not capacity else None),
+            "traffic_unit": "DRAM bytes per step (6 launches), ncu dram__bytes_read.sum + dram__bytes_write.sum",
             "algorithmic_flop_per_step": gemm_flop, "gemm_ms_per_step": round(gemm_ms, 4),
             "rows_computed": rows,
         },
