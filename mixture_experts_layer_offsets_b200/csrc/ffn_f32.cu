@@ -202,7 +202,8 @@ cudaError_t ffn_bwd_f32(const FfnShape& s, const float* dy_perm, const float* x_
 }
 
 size_t ffn_bwd_ws_bytes(const FfnShape& s, bool bf16) {
-  return align256((size_t)s.rows * 2 * s.f * (bf16 ? 2 : 4));
+  // [da | du], then (tensor-core path) the split weight-gradient partial sums
+  return align256((size_t)s.rows * 2 * s.f * (bf16 ? 2 : 4)) + (bf16 ? wgrad_part_bytes(s, false) : 0);
 }
 
 }  // namespace moe

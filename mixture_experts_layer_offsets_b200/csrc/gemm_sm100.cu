@@ -95,6 +95,13 @@ struct GemmParams {
   int32_t* localrank;      // [rows_total][topk]
   // GROUP_K without offsets: groups are consecutive splits of `split` rows
   int split;
+  // GROUP_K with offsets: a group of c > kchunk rows is cut into ns K ranges of ck rows
+  // (wgrad_split); tile (g, range j) then writes an fp32 partial sum to slot
+  // (slot prefix of g) + j of `part` ([slots * M, N], tensor map tmPart), and
+  // wgrad_reduce adds the ranges in order.  kchunk = 0: no cut.
+  int kchunk;
+  float* part;
+  CUtensorMap tmPart;
   // EPI_ROUTER_DX
   const int32_t* slot_row; // [rows_total][topk]
   // MXFP8 operands: E8M0 scales as 512-byte MMA atoms (128 rows x 4 blocks of 32
@@ -131,12 +138,15 @@ template <int BN, bool PAIR = false, int EPI = 1, bool FP8 = false> struct Cfg {
   // shared memory after the stage ring: barriers (256 B), offsets and tile prefix
   // (2 x 1025 ints), router histogram (128 x kRouterKMax ints), then the 1024-aligned
   // staging area; as many stages as fit (up to 6)
-  static constexpr size_t kFixed = 1024 + 256 + 2 * 1025 * 4 + 128 * kRouterKMax * 4 + 1024 + kStoreBytes;
+  // weight-gradient kernels keep a third per-group array (split slot prefix)
+  static constexpr size_t kExtra = EPI == EPI_WGRAD ? 1025 * 4 : 0;
+  static constexpr size_t kFixed = 1024 + 256 + 2 * 1025 * 4 + 128 * kRouterKMax * 4 + kExtra + 1024 + kStoreBytes;
   static constexpr int kStages = (232448 - kFixed) / kStage > 6 ? 6 : (int)((232448 - kFixed) / kStage);
   static constexpr size_t kOffMisc = (size_t)kStages * kStage;
   static constexpr size_t kOffSoff = kOffMisc + 256;
   static constexpr size_t kOffSel = kOffSoff + 2 * 1025 * 4;
-  static constexpr size_t kOffStore = (kOffSel + 128 * kRouterKMax * 4 + 1023) & ~size_t(1023);
+  static constexpr size_t kOffExtra = kOffSel + 128 * kRouterKMax * 4;
+  static constexpr size_t kOffStore = (kOffExtra + kExtra + 1023) & ~size_t(1023);
   static constexpr size_t kSmem = 1024 + kOffStore + kStoreBytes;
   static_assert(kSmem <= 232448, "shared memory per CTA");
   static_assert(128 * kRouterKMax * 4 >= 4 * 256 * 4, "router histogram fits the selection area");
@@ -363,7 +373,17 @@ __device__ __forceinline__ void put_box_bf16(uint8_t* wbuf, uint32_t& slot, cons
 // ------------------------------------------------------------ tile decode
 struct TileInfo {
   int g, m0, n0, rows, nkb, kbase, klast;
+  int split, nsplit, kst;  // GROUP_K: K range j of nsplit, its first 128-row stage in the group
 };
+
+// K ranges of a weight-gradient group of c rows cut at threshold kc: ns ranges of ck rows
+// (ck a multiple of 128, the last range shorter); ns = 1 when c <= kc or kc == 0.
+__host__ __device__ __forceinline__ void wgrad_split(int c, int kc, int& ns, int& ck) {
+  if (kc <= 0 || c <= kc) { ns = 1; ck = c; return; }
+  const int n0 = (c + kc - 1) / kc;
+  ck = (((c + n0 - 1) / n0) + 127) & ~127;
+  ns = (c + ck - 1) / ck;
+}
 
 template <int BN, int EPI, bool GROUP_K, int TM = BM, int KE = BK>
 __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, const int* s_off,
@@ -371,15 +391,34 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, cons
   TileInfo ti;
   if constexpr (GROUP_K) {
     const int per = (p.M / BM) * nN;
-    ti.g = t / per;
-    const int local = t - ti.g * per;
-    ti.m0 = (local / nN) * BM;
-    ti.n0 = (local % nN) * BN;
+    int g, local;
+    if (p.kchunk) {  // tile prefix over groups (ranges x per)
+      int lo = 0, hi = p.E - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_pre[mid] <= t) lo = mid; else hi = mid - 1;
+      }
+      g = lo;
+      local = t - s_pre[g];
+    } else {
+      g = t / per;
+      local = t - g * per;
+    }
+    const int j = local / per, rem = local - j * per;
+    ti.g = g;
+    ti.m0 = (rem / nN) * BM;
+    ti.n0 = (rem % nN) * BN;
     ti.rows = BM;
-    const int k0 = s_off[ti.g], kg = s_off[ti.g + 1] - k0;
-    ti.kbase = k0;
-    ti.nkb = (kg + KE - 1) / KE;
-    ti.klast = kg - (ti.nkb - 1) * KE;
+    const int k0 = s_off[g], kg = s_off[g + 1] - k0;
+    int ns, ck;
+    wgrad_split(kg, p.kchunk, ns, ck);
+    const int kb0 = j * ck, kn = min(ck, kg - kb0);
+    ti.split = j;
+    ti.nsplit = ns;
+    ti.kst = kb0 / 128;
+    ti.kbase = k0 + kb0;
+    ti.nkb = (kn + KE - 1) / KE;
+    ti.klast = kn - (ti.nkb - 1) * KE;
   } else {
     int lo = 0, hi = p.E - 1;
     while (lo < hi) {  // last expert whose tile prefix is <= t (skips empty experts)
@@ -395,6 +434,9 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, cons
     ti.kbase = lo * p.b_rows;
     ti.nkb = p.K / KE;
     ti.klast = KE;
+    ti.split = 0;
+    ti.nsplit = 1;
+    ti.kst = 0;
   }
   return ti;
 }
@@ -425,6 +467,10 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
   int* s_off = reinterpret_cast<int*>(smem + C::kOffSoff);
   int* s_pre = s_off + 1025;
   int* s_sel = reinterpret_cast<int*>(smem + C::kOffSel);  // EPI_ROUTER: [4][256] histogram
+  // GROUP_K: s_pre = tile prefix (split groups), s_stg = MXFP8 128-row stage prefix (in the
+  // router histogram area), s_slot = partial-slot prefix
+  int* s_stg = s_sel;
+  int* s_slot = reinterpret_cast<int*>(smem + C::kOffExtra);
   uint8_t* s_store = smem + C::kOffStore;                   // TMA-store staging
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -478,28 +524,48 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
       if (lane == 31) s_pre[E] = incl;
     }
   }
-  if constexpr (GROUP_K && FP8) {
-    if (warp == 1) {  // first 128-row scale stage of each group (stages restart at group starts)
+  if constexpr (GROUP_K) {
+    // per-group prefixes, 32 groups per lane of warp 1 (E <= 1024): tiles (split groups),
+    // partial slots (groups cut into several K ranges) and MXFP8 128-row stages
+    if (warp == 1 && (p.kchunk || FP8)) {
+      const int per = (p.M / BM) * nN;
       const int lo = lane * 32, hi = min(lo + 32, E);
-      int s = 0;
-      for (int g = lo; g < hi; ++g) s += (s_off[g + 1] - s_off[g] + 127) / 128;
-      int incl = s;
+      int st = 0, sl = 0, sg = 0;
+      for (int g = lo; g < hi; ++g) {
+        const int c = s_off[g + 1] - s_off[g];
+        int ns, ck;
+        wgrad_split(c, p.kchunk, ns, ck);
+        st += ns * per;
+        sl += ns > 1 ? ns : 0;
+        sg += (c + 127) / 128;
+      }
+      int it_ = st, il = sl, ig = sg;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += n;
+        const int a = __shfl_up_sync(0xffffffffu, it_, o);
+        const int b = __shfl_up_sync(0xffffffffu, il, o);
+        const int c = __shfl_up_sync(0xffffffffu, ig, o);
+        if (lane >= o) { it_ += a; il += b; ig += c; }
       }
-      int run = incl - s;
+      int rt = it_ - st, rl = il - sl, rg = ig - sg;
       for (int g = lo; g < hi; ++g) {
-        s_pre[g] = run;
-        run += (s_off[g + 1] - s_off[g] + 127) / 128;
+        const int c = s_off[g + 1] - s_off[g];
+        int ns, ck;
+        wgrad_split(c, p.kchunk, ns, ck);
+        s_pre[g] = rt;
+        s_slot[g] = rl;
+        s_stg[g] = rg;
+        rt += ns * per;
+        rl += ns > 1 ? ns : 0;
+        rg += (c + 127) / 128;
       }
+      if (lane == 31) s_pre[E] = it_;
     }
   }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
-  const int total = GROUP_K ? E * (p.M / BM) * nN : s_pre[E];
+  const int total = GROUP_K ? (p.kchunk ? s_pre[E] : E * (p.M / BM) * nN) : s_pre[E];
 
   auto fail = [&]() {
     record_status(p.status, MOE_ERR_TIMEOUT);
@@ -540,8 +606,9 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
         // of one stage are adjacent and travel in one copy)
         const uint8_t* atomB2 = nullptr;
         if constexpr (GROUP_K) {
-          atomA = p.sfa + ((int64_t)s_pre[ti.g] * (p.M / BM) + ti.m0 / BM) * 512;
-          atomB = p.sfb + ((int64_t)s_pre[ti.g] * (p.N / 128) + ti.n0 / 128) * 512;
+          const int64_t stage0 = s_stg[ti.g] + ti.kst;
+          atomA = p.sfa + (stage0 * (p.M / BM) + ti.m0 / BM) * 512;
+          atomB = p.sfb + (stage0 * (p.N / 128) + ti.n0 / 128) * 512;
         } else {
           const int mt = s_pre[ti.g] / nN + (ti.m0 - s_off[ti.g]) / BM;
           atomA = p.sfa + (int64_t)mt * kq * 512;
@@ -1074,8 +1141,12 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
           }
         }
       } else {  // EPI_WGRAD
-        const int64_t orow0 = (int64_t)ti.g * p.M + ti.m0 + q * 32;  // first output row of this warp
-        if (p.out_f32) {
+        // a group cut into K ranges writes fp32 partial sums to its slot of `part`
+        const bool partial = ti.nsplit > 1;
+        const CUtensorMap* tmo = partial ? &p.tmPart : &p.tmOut;
+        const int64_t orow0 = (partial ? (int64_t)(s_slot[ti.g] + ti.split) : (int64_t)ti.g) * p.M +
+                              ti.m0 + q * 32;  // first output row of this warp
+        if (p.out_f32 || partial) {
           // fp32: stage 16 rows x 32 columns in shared memory (128-byte swizzle) and
           // write them with one TMA store per box: whole 128-byte lines to HBM.
           uint8_t* sbuf = wbuf;
@@ -1105,7 +1176,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
               fence_proxy_async_smem();
               __syncwarp();
               if (lane == 0)
-                tma_store_2d(&p.tmOut, ti.n0 + (c0 + ci) * 32, (int)(orow0 + 16 * hh), sbuf);
+                tma_store_2d(tmo, ti.n0 + (c0 + ci) * 32, (int)(orow0 + 16 * hh), sbuf);
             }
           }
         } else {
@@ -1141,6 +1212,48 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
     tc_fence_after();
     if constexpr (PAIR) tmem_dealloc_pair(tmem_base, C::kTmemCols);
     else tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// Weight gradients of groups cut into K ranges: dW[g] = sum over j (in order) of the fp32
+// partial sums in slots (slot prefix of g) + j; groups that were not cut are skipped.
+__global__ void __launch_bounds__(256)
+wgrad_reduce_kernel(const int32_t* __restrict__ offsets, int kc, int64_t mn4,
+                    const float4* __restrict__ part, float4* __restrict__ out32,
+                    __nv_bfloat16* __restrict__ out16) {
+  __shared__ int s_red[8];
+  const int g = blockIdx.y;
+  int ns, ck;
+  wgrad_split(offsets[g + 1] - offsets[g], kc, ns, ck);
+  if (ns <= 1) return;
+  int acc = 0;  // partial slots of the groups before g
+  for (int e = threadIdx.x; e < g; e += blockDim.x) {
+    int n2, c2;
+    wgrad_split(offsets[e + 1] - offsets[e], kc, n2, c2);
+    acc += n2 > 1 ? n2 : 0;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  int slot0 = 0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) slot0 += s_red[w];
+  const float4* src = part + (int64_t)slot0 * mn4;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < mn4; i += (int64_t)gridDim.x * blockDim.x) {
+    float4 a = src[i];
+    for (int j = 1; j < ns; ++j) {
+      const float4 b = src[(int64_t)j * mn4 + i];
+      a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+    }
+    if (out32) {
+      out32[(int64_t)g * mn4 + i] = a;
+    } else {
+      uint2 pk;
+      pk.x = pack_bf16(a.x, a.y);
+      pk.y = pack_bf16(a.z, a.w);
+      *reinterpret_cast<uint2*>(out16 + ((int64_t)g * mn4 + i) * 4) = pk;
+    }
   }
 }
 
@@ -1234,6 +1347,43 @@ template <bool A_MN, bool B_MN, int EPI, bool GROUP_K>
 cudaError_t launch_mx_n(const GemmParams& p, int N, int64_t units, cudaStream_t st) {
   if (N % 256 == 0) return launch_mx<256, A_MN, B_MN, EPI, GROUP_K>(p, units * (N / 256), st);
   return launch_mx<128, A_MN, B_MN, EPI, GROUP_K>(p, units * (N / 128), st);
+}
+
+// K threshold above which a weight-gradient group is cut into several K ranges: one tile
+// would carry more than an SM's fair share of the launch's K work (rows x tiles per group /
+// SMs), as when most tokens choose one expert; never less than 2048 rows.  (A lower
+// threshold was measured: at a quarter of the fair share the partial sums and their
+// reduction cost more than the better balance saved on the benchmark workloads.)
+int wgrad_kchunk(int64_t rows, int M, int N, int BN) {
+  const int64_t per = (int64_t)(M / BM) * (N / BN);
+  int64_t kc = (rows * per + num_sms() - 1) / num_sms();
+  kc = std::max<int64_t>(kc, 2048);
+  return (int)((kc + 127) & ~int64_t(127));
+}
+// partial slots: a group of c > kc rows takes ceil(c / kc) <= 2 c / kc of them
+int64_t wgrad_slots(int64_t rows, int kc) { return 2 * rows / kc + 1; }
+int wgrad_bn(int N, bool fp8) { return (!fp8 || N % 256 == 0) ? 256 : 128; }
+
+// Sets the split fields of a weight-gradient launch (M x N per group) and returns the
+// partial-buffer bytes it may use; `part` may be null when only the size is wanted.
+size_t wgrad_setup(GemmParams* p, int64_t rows, int M, int N, bool fp8, float* part) {
+  const int kc = wgrad_kchunk(rows, M, N, wgrad_bn(N, fp8));
+  const int64_t slots = wgrad_slots(rows, kc);
+  if (p) {
+    p->kchunk = kc;
+    p->part = part;
+    if (part && !tmap(&p->tmPart, part, N, (uint64_t)slots * M, N, 32, 16, true)) p->part = nullptr;
+  }
+  return (size_t)slots * M * N * sizeof(float);
+}
+
+cudaError_t wgrad_reduce_launch(const GemmParams& p, int64_t M, int64_t N, float* out32,
+                                __nv_bfloat16* out16, cudaStream_t st) {
+  const int64_t mn4 = M * N / 4;
+  dim3 grid((unsigned)std::min<int64_t>((mn4 + 255) / 256, 16), (unsigned)p.E);
+  wgrad_reduce_kernel<<<grid, 256, 0, st>>>(p.offsets, p.kchunk, mn4, reinterpret_cast<const float4*>(p.part),
+                                            reinterpret_cast<float4*>(out32), out16);
+  return cudaGetLastError();
 }
 
 GemmParams base_params(const FfnShape& s, const int32_t* offsets, int* status) {
@@ -1407,7 +1557,12 @@ cudaError_t ffn_bwd_bf16(const FfnShape& s, const void* dy_perm, const void* x_p
   p5.out = static_cast<__nv_bfloat16*>(dw2); p5.out_f32 = dw_f32 ? static_cast<float*>(dw2) : nullptr;
   p5.ld_out = f; p5.out_group = (int64_t)d * f;
   if (dw_f32 && !tmap(&p5.tmOut, dw2, f, (uint64_t)E * d, f, 32, 16, true)) return cudaErrorInvalidValue;
-  if ((err = launch<256, true, true, EPI_WGRAD, true>(p5, (int64_t)E * (d / 128) * (f / 256), st)) != cudaSuccess)
+  float* part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(scratch) +
+                                         align256((size_t)s.rows * 2 * f * 2));
+  wgrad_setup(&p5, s.rows, d, f, false, part);
+  if (!p5.part) return cudaErrorInvalidValue;
+  if ((err = launch<256, true, true, EPI_WGRAD, true>(p5, num_sms(), st)) != cudaSuccess ||
+      (err = wgrad_reduce_launch(p5, d, f, p5.out_f32, p5.out, st)) != cudaSuccess)
     return err;
   // wgrad 1: dW1[e] = [da | du]^T x   (M = 2f, N = d)
   GemmParams p6 = base_params(s, offsets, status);
@@ -1418,7 +1573,15 @@ cudaError_t ffn_bwd_bf16(const FfnShape& s, const void* dy_perm, const void* x_p
   p6.out = static_cast<__nv_bfloat16*>(dw1); p6.out_f32 = dw_f32 ? static_cast<float*>(dw1) : nullptr;
   p6.ld_out = d; p6.out_group = (int64_t)2 * f * d;
   if (dw_f32 && !tmap(&p6.tmOut, dw1, d, (uint64_t)E * 2 * f, d, 32, 16, true)) return cudaErrorInvalidValue;
-  return launch<256, true, true, EPI_WGRAD, true>(p6, (int64_t)E * (2 * f / 128) * (d / 256), st);
+  wgrad_setup(&p6, s.rows, 2 * f, d, false, part);
+  if (!p6.part) return cudaErrorInvalidValue;
+  if ((err = launch<256, true, true, EPI_WGRAD, true>(p6, num_sms(), st)) != cudaSuccess) return err;
+  return wgrad_reduce_launch(p6, 2 * f, d, p6.out_f32, p6.out, st);
+}
+
+size_t wgrad_part_bytes(const FfnShape& s, bool fp8) {
+  return std::max(wgrad_setup(nullptr, s.rows, s.d, s.f, fp8, nullptr),
+                  wgrad_setup(nullptr, s.rows, 2 * s.f, s.d, fp8, nullptr));
 }
 
 
@@ -1436,6 +1599,7 @@ struct MxLayout {
   size_t qx0, sx0, qh0, sh0;                         // forward
   size_t dadu, qdy0, sdy0, qda0, sda0;               // backward, dgrad operands
   size_t qdy1, sdy1, qh1, sh1, qda1, sda1, qx1, sx1;  // backward, wgrad operands
+  size_t part;                                        // split weight-gradient partial sums
   size_t fwd_bytes, bwd_bytes;
 };
 
@@ -1460,6 +1624,7 @@ MxLayout mx_layout(const FfnShape& s) {
   L.qh1 = take(R * f); L.sh1 = take(atoms(f));
   L.qda1 = take(R * 2 * f); L.sda1 = take(atoms(2 * f));
   L.qx1 = take(R * d); L.sx1 = take(atoms(d));
+  L.part = take(wgrad_part_bytes(s, true));
   L.bwd_bytes = o;
   return L;
 }
@@ -1595,7 +1760,10 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
   p5.sfb = ws + L.sh1;
   p5.M = d; p5.N = f;
   p5.out_f32 = dw2; p5.ld_out = f; p5.out_group = (int64_t)d * f;
-  if ((err = launch_mx_n<true, true, EPI_WGRAD, true>(p5, f, (int64_t)E * (d / 128), st)) != cudaSuccess)
+  wgrad_setup(&p5, R, d, f, true, reinterpret_cast<float*>(ws + L.part));
+  if (!p5.part) return cudaErrorInvalidValue;
+  if ((err = launch_mx_n<true, true, EPI_WGRAD, true>(p5, f, num_sms(), st)) != cudaSuccess ||
+      (err = wgrad_reduce_launch(p5, d, f, dw2, nullptr, st)) != cudaSuccess)
     return err;
   // wgrad 1: dW1[e] = [da | du]^T x  (M = 2f, N = d)
   GemmParams p6 = mx_params(s, offsets, status);
@@ -1607,7 +1775,10 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
   p6.sfb = ws + L.sx1;
   p6.M = 2 * f; p6.N = d;
   p6.out_f32 = dw1; p6.ld_out = d; p6.out_group = (int64_t)2 * f * d;
-  return launch_mx_n<true, true, EPI_WGRAD, true>(p6, d, (int64_t)E * (2 * f / 128), st);
+  wgrad_setup(&p6, R, 2 * f, d, true, reinterpret_cast<float*>(ws + L.part));
+  if (!p6.part) return cudaErrorInvalidValue;
+  if ((err = launch_mx_n<true, true, EPI_WGRAD, true>(p6, d, num_sms(), st)) != cudaSuccess) return err;
+  return wgrad_reduce_launch(p6, 2 * f, d, dw1, nullptr, st);
 }
 
 }  // namespace moe

@@ -92,6 +92,8 @@ struct FfnShape {
   int64_t rows;
 };
 size_t ffn_bwd_ws_bytes(const FfnShape& s, bool bf16);
+// fp32 partial sums of weight-gradient groups cut into K ranges (tensor-core paths)
+size_t wgrad_part_bytes(const FfnShape& s, bool fp8);
 // fp32 path: CUDA-core grouped GEMMs
 cudaError_t ffn_fwd_f32(const FfnShape& s, const float* x_perm, const int32_t* offsets,
                         const float* w1, const float* w2, float* act, float* y_perm,

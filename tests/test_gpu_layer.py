@@ -32,6 +32,11 @@ CASES = {
     # with ragged tails, ~80 rows per expert
     "bf16_e128_small": shrink(CONFIGS["bf16_e128"], name="bf16_e128_small", T=2600, d_model=256,
                               d_ff=256, router_std=1 / 16.0),
+    # skewed routing with experts of 2300 .. 5441 rows: their weight gradients are cut
+    # into 2 or 3 K ranges whose fp32 partial sums are added in order; 4 empty experts
+    "bf16_skew_split": shrink(CONFIGS["bf16_skew_e128"], name="bf16_skew_split", T=8000,
+                              d_model=256, E=16, top_k=2, d_ff=256, router_std=1 / 16.0,
+                              bias_std=3.0),
     # a single token; fp32
     "f32_one_token": shrink(CONFIGS["tiny_f32"], name="f32_one_token", T=1, d_model=16, E=4,
                             top_k=3, d_ff=8),
@@ -79,8 +84,9 @@ def test_layer_matches_oracle(name):
         assert not L.dw1[e].any() and not L.dw2[e].any()
 
 
-def test_bf16_weight_grads_in_bf16():
-    cfg = CASES["bf16_e8_small"]
+@pytest.mark.parametrize("name", ["bf16_e8_small", "bf16_skew_split"])
+def test_bf16_weight_grads_in_bf16(name):
+    cfg = CASES[name]
     cpu, L = run_layer(cfg, dw_dtype="bf16")
     o = oracle_for(cpu, L)
     assert L.dw1.dtype == torch.bfloat16
@@ -111,9 +117,11 @@ def test_padded_capacity_matches_oracle(name, cap):
         assert rel(f64(dev), o[key]) <= tol, key
 
 
-def test_routing_is_deterministic_across_runs():
-    cfg = CASES["bf16_skew_small"]
+@pytest.mark.parametrize("name", ["bf16_skew_small", "bf16_skew_split"])
+def test_routing_is_deterministic_across_runs(name):
+    cfg = CASES[name]
     _, a = run_layer(cfg)
     _, b = run_layer(cfg)
-    for name in ("logits", "topk_idx", "topk_gate", "slot_row", "out", "dx", "dw1", "dw_router"):
-        assert torch.equal(getattr(a, name), getattr(b, name)), name
+    for key in ("logits", "topk_idx", "topk_gate", "slot_row", "out", "dx", "dw1", "dw2",
+                "dw_router"):
+        assert torch.equal(getattr(a, key), getattr(b, key)), key

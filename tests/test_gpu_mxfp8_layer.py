@@ -30,6 +30,9 @@ CASES = {
     # skewed routing with a logit bias: heavy-tailed counts and empty experts
     "mx_skew": shrink(BASE, name="mx_skew", T=700, d_model=128, E=32, top_k=2, d_ff=128,
                       router_std=1 / 16.0, bias_std=2.0),
+    # experts of 3459 and 5998 rows: weight gradients cut into K ranges, partial sums added
+    "mx_skew_split": shrink(BASE, name="mx_skew_split", T=6000, d_model=128, E=16, top_k=2,
+                            d_ff=128, router_std=1 / 16.0, bias_std=3.0),
     # one token
     "mx_one_token": shrink(BASE, name="mx_one_token", T=1, d_model=128, E=4, top_k=2, d_ff=128),
 }
