@@ -52,7 +52,7 @@ FP8_OVER_BF16 = 2.0   # nominal dense tensor-core ratio (4.5 / 2.25 PFLOP/s)
 # DRAM bytes (read + write) of the six grouped-GEMM launches of one step, from one ncu capture
 # of this build (profiles/launches_bf16_e8.md); None where no capture of the current kernels
 # exists.
-GEMM_TRAFFIC_BYTES = {"bf16_e8": 3.862e9}
+GEMM_TRAFFIC_BYTES = {"bf16_e8": 3.857e+09}
 
 
 def _peaks():
@@ -301,45 +301,73 @@ def run_ours(args, rank, world):
 
 
 def run_e2e(args, L, inp, dev, flush, capacity, world):
-    """Same metric through the public API with pinned host buffers: per step the
-    inputs x and dout go host->device and the outputs out and dx come back."""
-    from mixture_experts_layer_offsets_b200 import capi  # noqa: F401
+    """Same metric through the public API with pinned host buffers: every step copies its
+    inputs x and dout host->device and its outputs out and dx device->host, inside the
+    timed region.  Steps are pipelined the way an input pipeline would run them: two layer
+    instances take turns, and while one step computes on the compute stream, the next
+    step's inputs come in on a copy stream and the previous step's outputs go out on
+    another; events order every copy against the compute that produces or reuses its
+    buffers.  Working set per step is several times L2, so no flush is needed."""
+    from mixture_experts_layer_offsets_b200.layer import MoELayer
+    L2 = MoELayer(L.T, L.d, L.E, L.k, L.f, L.dtype, dev, dw_dtype=L.dw_dtype, capacity=capacity)
+    layers = [L, L2]
     hx = inp["x"].cpu().pin_memory()
     hd = inp["dout"].cpu().pin_memory()
-    hout = torch.empty_like(hx).pin_memory()
-    hdx = torch.empty_like(hx).pin_memory()
-    dx_in = torch.empty_like(inp["x"])
-    ddout = torch.empty_like(inp["dout"])
+    hout = [torch.empty_like(hx).pin_memory() for _ in range(2)]
+    hdx = [torch.empty_like(hx).pin_memory() for _ in range(2)]
+    xin = [torch.empty_like(inp["x"]) for _ in range(2)]
+    din = [torch.empty_like(inp["dout"]) for _ in range(2)]
     wr, b, w1, w2 = inp["w_router"], inp["bias"], inp["w1"], inp["w2"]
+    cs = torch.cuda.current_stream()
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
-    def step():
-        dx_in.copy_(hx, non_blocking=True)
-        ddout.copy_(hd, non_blocking=True)
-        L.step(dx_in, wr, b, w1, w2, ddout)
-        hout.copy_(L.out, non_blocking=True)
-        hdx.copy_(L.dx, non_blocking=True)
+    def issue(i):
+        k = i % 2
+        h2d.wait_event(ev_comp[k])            # step i-2 has finished reading buffer k
+        with torch.cuda.stream(h2d):
+            xin[k].copy_(hx, non_blocking=True)
+            din[k].copy_(hd, non_blocking=True)
+            ev_in[k].record(h2d)
+        cs.wait_event(ev_in[k])
+        cs.wait_event(ev_out[k])              # step i-2's outputs have left layer k
+        layers[k].step(xin[k], wr, b, w1, w2, din[k])
+        ev_comp[k].record(cs)
+        d2h.wait_event(ev_comp[k])
+        with torch.cuda.stream(d2h):
+            hout[k].copy_(layers[k].out, non_blocking=True)
+            hdx[k].copy_(layers[k].dx, non_blocking=True)
+            ev_out[k].record(d2h)
 
-    for _ in range(max(1, args.warmup)):
-        step()
+    for i in range(max(2, args.warmup)):
+        issue(i)
     torch.cuda.synchronize()
-    n = max(1, args.steps // 2)
+    n = max(2, args.steps)
     st, en = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    times = []
     if world > 1:
         torch.distributed.barrier()
-    for _ in range(n):
-        flush.zero_()
-        st.record()
-        step()
-        en.record()
-        torch.cuda.synchronize()
-        times.append(st.elapsed_time(en))
-    ms = mdist.max_over_ranks(sum(times) / n, device=dev)
+    torch.cuda.synchronize()
+    st.record(cs)
+    h2d.wait_event(st)
+    d2h.wait_event(st)
+    for i in range(n):
+        issue(i)
+    cs.wait_event(ev_out[0])
+    cs.wait_event(ev_out[1])
+    en.record(cs)
+    torch.cuda.synchronize()
+    ms = mdist.max_over_ranks(st.elapsed_time(en) / n, device=dev)
+    status = max(layers[0].device_status(), layers[1].device_status())
     T = inp["x"].shape[0]
     nbytes = hx.numel() * hx.element_size()
+    del L2
     return {"value": round(T * world / (ms / 1e3), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": 2 * nbytes, "d2h_bytes_per_step": 2 * nbytes,
-            "ms_per_step": round(ms, 4), "api": "MoELayer.step (C ABI) with pinned host buffers"}
+            "ms_per_step": round(ms, 4), "steps": n, "device_status": status,
+            "api": "MoELayer.step (C ABI) with pinned host buffers; copies of step i+1 in and "
+                   "i-1 out overlap step i's compute (two layer instances, three streams)"}
 
 
 # ------------------------------------------------- CPU oracle (baseline)

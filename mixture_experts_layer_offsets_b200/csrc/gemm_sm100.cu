@@ -102,6 +102,11 @@ struct GemmParams {
   int kchunk;
   float* part;
   CUtensorMap tmPart;
+  // Failure-path test hooks (0 = off): the limit of every bounded wait, and a ring
+  // iteration at which CTA 0's producer skips its loads and its arrival, so that the MMA
+  // warp's wait runs out (see gemm_test_hooks).
+  uint64_t wait_ns;
+  int drop_it;
   // EPI_ROUTER_DX
   const int32_t* slot_row; // [rows_total][topk]
   // MXFP8 operands: E8M0 scales as 512-byte MMA atoms (128 rows x 4 blocks of 32
@@ -446,6 +451,7 @@ template <int BN, bool A_MN, bool B_MN, int EPI, bool GROUP_K, bool PAIR = false
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
   using C = Cfg<BN, PAIR, EPI, FP8>;
+  const uint64_t wl = p.wait_ns ? p.wait_ns : (uint64_t)MOE_WAIT_NS;  // bounded-wait limit
   static_assert(!FP8 || ((BN == 128 || BN == 256) && !PAIR), "MXFP8 tiles: 128 x 128 or 128 x 256, single CTA");
   static_assert(!FP8 || EPI != EPI_SWIGLU_FWD || BN == 256, "MXFP8 SwiGLU tiles pair 128 gate with 128 up columns");
   // epilogue warps 6..9 idle when a thread must hold a whole row (router)
@@ -627,7 +633,8 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
           }
         }
         for (int kb = 0; kb < ti.nkb; ++kb, ++it, s = (s + 1 == S ? 0 : s + 1), ph ^= (s == 0)) {
-          if (!mbar_wait(&empty[s], ph)) { fail(); ok = false; break; }
+          if (!mbar_wait(&empty[s], ph, wl)) { fail(); ok = false; break; }
+          if (p.drop_it && blockIdx.x == 0 && it + 1 == (uint32_t)p.drop_it) continue;  // test hook
           uint8_t* sa = smem + s * C::kStage;
           uint8_t* sb = sa + kABytes;
           uint8_t* sf = sb + C::kBBytes;
@@ -666,7 +673,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
       }
       if (!ok) {  // let the copies already issued land before the CTA exits
         for (uint32_t j = it > (uint32_t)S ? it - S : 0; j < it; ++j)
-          (void)mbar_wait(&full[j % S], (j / S) & 1);
+          (void)mbar_wait(&full[j % S], (j / S) & 1, wl);
       }
     }
   } else if (warp == 0) {
@@ -683,7 +690,8 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
         if (*s_abort) { ok = false; break; }
         const TileInfo ti = decode(t);
         for (int kb = 0; kb < ti.nkb; ++kb, ++it, s = (s + 1 == S ? 0 : s + 1), ph ^= (s == 0)) {
-          if (!mbar_wait(&empty[s], ph)) { fail(); ok = false; break; }
+          if (!mbar_wait(&empty[s], ph, wl)) { fail(); ok = false; break; }
+          if (!PAIR && p.drop_it && blockIdx.x == 0 && it + 1 == (uint32_t)p.drop_it) continue;  // test hook
           uint8_t* sa = smem + s * C::kStage;
           uint8_t* sb = sa + kABytes;
           const int kc = kb * BK;
@@ -727,7 +735,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
       }
       if (!ok && leader) {  // let the loads in flight land before shared memory is released
         for (uint32_t j = it > (uint32_t)S ? it - S : 0; j < it; ++j)
-          (void)mbar_wait(&full[j % S], (j / S) & 1);
+          (void)mbar_wait(&full[j % S], (j / S) & 1, wl);
       }
     }
   } else if (warp == 1) {
@@ -762,7 +770,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
       const TileInfo ti = decode(t);
       const int acc = C::kAccBufs == 2 ? (int)(acc_it & 1) : 0;
       const uint32_t acc_ph = C::kAccBufs == 2 ? (acc_it >> 1) & 1 : acc_it & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&tempty[acc], acc_ph ^ 1))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&tempty[acc], acc_ph ^ 1, wl))) {
         if (lane == 0) fail();
         ok = false;
         break;
@@ -771,7 +779,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
       const uint32_t d_tmem = tmem_base + acc * BN;
       for (int kb = 0; kb < ti.nkb; ++kb, ++it) {
         bool w = true;
-        if (lane == 0) w = mbar_wait(&full[stg], ph);
+        if (lane == 0) w = mbar_wait(&full[stg], ph, wl);
         if (!__shfl_sync(0xffffffffu, (int)w, 0)) {
           if (lane == 0) fail();
           ok = false;
@@ -841,7 +849,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
     if (!ok && lane == 0) {  // wait for this thread's MMAs before TMEM is freed
       if constexpr (PAIR) umma_commit_pair(drain);
       else umma_commit(drain);
-      (void)mbar_wait(drain, 0);
+      (void)mbar_wait(drain, 0, wl);
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -878,7 +886,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
         arow = p.act + (int64_t)(ti.m0 + row) * p.ld_act;
         if (valid) load_au(arow, ti.n0 + c0 * 32, p.f, av, uv);
       }
-      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_ph))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_ph, wl))) {
         fail();
         break;
       }
@@ -924,25 +932,30 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
           put_box_bf16(wbuf, slot, &p.tmOut, ph, hh, 2 * p.f + col, grow0 + 16 * hh, vr, arow + 2 * p.f + col);
         }
       } else if constexpr (EPI == EPI_STORE) {
+        // every chunk of this warp is read (and packed to bf16) before the accumulator is
+        // released, so that the next tile's MMAs overlap the stores
         __nv_bfloat16* orow = p.out + (int64_t)(ti.m0 + row) * p.ld_out;
+        uint32_t pk[kMine / 2][32];
 #pragma unroll
         for (int pc = 0; pc < kMine / 2; ++pc) {
-          uint32_t pk[32];
 #pragma unroll
           for (int ci = 0; ci < 2; ++ci) {
             uint32_t v[32];
             tmem_ld32(ta + (c0 + 2 * pc + ci) * 32, v);
             tmem_wait_ld();
             tmem_tie(v);
-            if (pc == kMine / 2 - 1 && ci == 1) release();
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-              pk[16 * ci + i] = pack_bf16(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+              pk[pc][16 * ci + i] = pack_bf16(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
           }
+        }
+        release();
+#pragma unroll
+        for (int pc = 0; pc < kMine / 2; ++pc) {
           const int col = ti.n0 + (c0 + 2 * pc) * 32;
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh)
-            put_box_bf16(wbuf, slot, &p.tmOut, pk, hh, col, grow0 + 16 * hh,
+            put_box_bf16(wbuf, slot, &p.tmOut, pk[pc], hh, col, grow0 + 16 * hh,
                          box_valid(q * 32 + 16 * hh), orow + col);
         }
       } else if constexpr (EPI == EPI_SWIGLU_BWD) {
@@ -1148,21 +1161,29 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
                               ti.m0 + q * 32;  // first output row of this warp
         if (p.out_f32 || partial) {
           // fp32: stage 16 rows x 32 columns in shared memory (128-byte swizzle) and
-          // write them with one TMA store per box: whole 128-byte lines to HBM.
+          // write them with one TMA store per box: whole 128-byte lines to HBM.  All of
+          // this warp's chunks are read before the accumulator is released.
           uint8_t* sbuf = wbuf;
-#pragma unroll 1
+          uint32_t va[kMine][32];
+#pragma unroll
           for (int ci = 0; ci < kMine; ++ci) {
-            uint32_t v[32];
             if (ti.nkb > 0) {
-              tmem_ld32(ta + (c0 + ci) * 32, v);
-              tmem_wait_ld();
-              tmem_tie(v);
+              tmem_ld32(ta + (c0 + ci) * 32, va[ci]);
             } else {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = 0;
+              for (int i = 0; i < 32; ++i) va[ci][i] = 0;
             }
-            if (ci == kMine - 1) release();
-#pragma unroll 1
+          }
+          if (ti.nkb > 0) {
+            tmem_wait_ld();
+#pragma unroll
+            for (int ci = 0; ci < kMine; ++ci) tmem_tie(va[ci]);
+          }
+          release();
+#pragma unroll
+          for (int ci = 0; ci < kMine; ++ci) {
+            const uint32_t* v = va[ci];
+#pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
               if (lane == 0) tma_store_wait_read();  // the previous box has left the buffer
               __syncwarp();
@@ -1181,23 +1202,24 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
           }
         } else {
           __nv_bfloat16* o = p.out + (orow0 + lane) * p.ld_out + ti.n0 + c0 * 32;
-#pragma unroll 1
+          uint32_t pk[kMine][16];
+#pragma unroll
           for (int ci = 0; ci < kMine; ++ci) {
-            uint32_t pk[16];
             if (ti.nkb > 0) {
               uint32_t v[32];
               tmem_ld32(ta + (c0 + ci) * 32, v);
               tmem_wait_ld();
               tmem_tie(v);
 #pragma unroll
-              for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+              for (int i = 0; i < 16; ++i) pk[ci][i] = pack_bf16(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
             } else {
 #pragma unroll
-              for (int i = 0; i < 16; ++i) pk[i] = 0;
+              for (int i = 0; i < 16; ++i) pk[ci][i] = 0;
             }
-            if (ci == kMine - 1) release();
-            store_64B(o + ci * 32, pk);
           }
+          release();
+#pragma unroll
+          for (int ci = 0; ci < kMine; ++ci) store_64B(o + ci * 32, pk[ci]);
         }
       }
       ++acc_it;
@@ -1286,6 +1308,31 @@ bool tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uin
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Failure-path test hooks, read once from the environment (unset in normal use):
+// MOE_B200_WAIT_NS sets the limit of every bounded wait of the GEMM kernels, and
+// MOE_B200_TEST_DROP_STAGE = n makes CTA 0's producer skip its n-th ring stage (no load,
+// no arrival), so that the MMA warp's wait for it runs out and the kernel takes its abort
+// path: MOE_ERR_TIMEOUT in the status word, then a clean exit.
+struct TestHooks {
+  uint64_t wait_ns = 0;
+  int drop_it = 0;
+};
+const TestHooks& gemm_test_hooks() {
+  static const TestHooks h = [] {
+    TestHooks t;
+    if (const char* w = getenv("MOE_B200_WAIT_NS")) t.wait_ns = strtoull(w, nullptr, 10);
+    if (const char* d = getenv("MOE_B200_TEST_DROP_STAGE")) t.drop_it = atoi(d);
+    return t;
+  }();
+  return h;
+}
+GemmParams with_hooks(const GemmParams& p) {
+  GemmParams q = p;
+  q.wait_ns = gemm_test_hooks().wait_ns;
+  q.drop_it = gemm_test_hooks().drop_it;
+  return q;
+}
+
 template <int BN, bool A_MN, bool B_MN, int EPI, bool GROUP_K>
 cudaError_t launch(const GemmParams& p, int64_t tile_bound, cudaStream_t st) {
   auto kern = grouped_gemm_sm100<BN, A_MN, B_MN, EPI, GROUP_K>;
@@ -1293,7 +1340,7 @@ cudaError_t launch(const GemmParams& p, int64_t tile_bound, cudaStream_t st) {
                                          (int)Cfg<BN, false, EPI>::kSmem);
   if (err != cudaSuccess) return err;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tile_bound, num_sms()));
-  kern<<<grid, kThreads, Cfg<BN, false, EPI>::kSmem, st>>>(p);
+  kern<<<grid, kThreads, Cfg<BN, false, EPI>::kSmem, st>>>(with_hooks(p));
   return cudaGetLastError();
 }
 
@@ -1305,7 +1352,7 @@ cudaError_t launch_mx(const GemmParams& p, int64_t tile_bound, cudaStream_t st) 
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tile_bound, num_sms()));
-  kern<<<grid, kThreads, smem, st>>>(p);
+  kern<<<grid, kThreads, smem, st>>>(with_hooks(p));
   return cudaGetLastError();
 }
 
@@ -1338,7 +1385,7 @@ cudaError_t launch_pair(const GemmParams& p, int64_t pair_tile_bound, cudaStream
   }
   const int clusters = (int)std::max<int64_t>(1, std::min<int64_t>(pair_tile_bound, dev < 64 ? max_clusters[dev] : num_sms() / 2));
   cfg.gridDim = dim3(2 * clusters);
-  return cudaLaunchKernelEx(&cfg, kern, p);
+  return cudaLaunchKernelEx(&cfg, kern, with_hooks(p));
 }
 
 // 256-wide MXFP8 tiles where N allows (twice the work per MMA instruction), else 128.

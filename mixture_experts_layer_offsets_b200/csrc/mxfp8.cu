@@ -357,6 +357,8 @@ mx_weights_kernel(const float* __restrict__ w, int Rw, int Kw, uint8_t* __restri
                   uint8_t* __restrict__ s0, uint8_t* __restrict__ q1, uint8_t* __restrict__ s1) {
   extern __shared__ float tile[];                       // [128][kWPitch]
   uint8_t* qt = reinterpret_cast<uint8_t*>(tile + 128 * kWPitch);  // [128][128] q1 bytes
+  uint8_t* sa0 = qt + 128 * 128;                        // this tile's s0 atom (512 B)
+  uint8_t* sa1 = sa0 + 512;                             // and its s1 atom
   const int e = blockIdx.z, rt = blockIdx.y, ct = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31;
   const int64_t row0 = (int64_t)e * Rw + rt * 128;
@@ -391,8 +393,7 @@ mx_weights_kernel(const float* __restrict__ w, int Rw, int Kw, uint8_t* __restri
     out.x = e4m3_pair(v[1] * mul, v[0] * mul) | (e4m3_pair(v[3] * mul, v[2] * mul) << 16);
     out.y = e4m3_pair(v[5] * mul, v[4] * mul) | (e4m3_pair(v[7] * mul, v[6] * mul) << 16);
     *reinterpret_cast<uint2*>(q0 + (row0 + r) * Kw + col0 + kb * 32 + part * 8) = out;
-    if (part == 0)
-      s0[(((int64_t)e * (Rw >> 7) + rt) * (Kw >> 7) + ct) * 512 + atom_byte(r, kb)] = (uint8_t)(ex + 127);
+    if (part == 0) sa0[atom_byte(r, kb)] = (uint8_t)(ex + 127);
   }
   (void)lane;
   __syncthreads();
@@ -412,10 +413,10 @@ mx_weights_kernel(const float* __restrict__ w, int Rw, int Kw, uint8_t* __restri
       qt[(rb * 32 + i) * 128 + c] = (uint8_t)(pr & 0xFF);
       qt[(rb * 32 + i + 1) * 128 + c] = (uint8_t)(pr >> 8);
     }
-    s1[(((int64_t)e * (Rw >> 7) + rt) * (Kw >> 7) + ct) * 512 + atom_byte(c, rb)] = (uint8_t)(ex + 127);
+    sa1[atom_byte(c, rb)] = (uint8_t)(ex + 127);
   }
   __syncthreads();
-  // write the q1 tile: 128 rows x 128 bytes, 16 bytes per thread and step
+  // write the q1 tile (128 rows x 128 bytes) and both scale atoms, 16 bytes per store
 #pragma unroll
   for (int it = 0; it < 4; ++it) {
     const int idx = it * 256 + tid;            // 1024 pieces of 16 bytes
@@ -423,6 +424,12 @@ mx_weights_kernel(const float* __restrict__ w, int Rw, int Kw, uint8_t* __restri
     *reinterpret_cast<uint4*>(q1 + (row0 + r) * Kw + col0 + c16 * 16) =
         *reinterpret_cast<const uint4*>(qt + r * 128 + c16 * 16);
   }
+  const int64_t atom = (((int64_t)e * (Rw >> 7) + rt) * (Kw >> 7) + ct) * 512;
+  if (tid < 32)
+    *reinterpret_cast<uint4*>(s0 + atom + tid * 16) = *reinterpret_cast<const uint4*>(sa0 + tid * 16);
+  else if (tid < 64)
+    *reinterpret_cast<uint4*>(s1 + atom + (tid - 32) * 16) =
+        *reinterpret_cast<const uint4*>(sa1 + (tid - 32) * 16);
 }
 
 }  // namespace
@@ -457,7 +464,7 @@ cudaError_t mxfp8_cols_atoms(int64_t rows, int64_t K, int64_t ld, const void* sr
 cudaError_t mxfp8_weights(const float* w, int E, int Rw, int Kw, uint8_t* q0, uint8_t* s0,
                           uint8_t* q1, uint8_t* s1, cudaStream_t st) {
   if (E == 0) return cudaSuccess;
-  const size_t smem = 128 * kWPitch * sizeof(float) + 128 * 128;
+  const size_t smem = 128 * kWPitch * sizeof(float) + 128 * 128 + 1024;
   cudaError_t err = cudaFuncSetAttribute(mx_weights_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
   if (err != cudaSuccess) return err;
