@@ -15,9 +15,9 @@ namespace moe {
 
 namespace {
 
-constexpr int kTT = 32;   // tokens per tile
 
-inline int route_bwd_splits(int T) { return std::max(1, std::min(128, T / 128)); }
+// token splits of the CUDA-core dW_r partial sums (about 1024 tokens each)
+inline int route_bwd_splits(int T) { return std::max(1, std::min(64, T / 1024)); }
 
 // dl, one warp per token, written to the workspace in fp32 (CUDA-core path) or
 // bf16 (tensor-core path, where dl is a GEMM operand).
@@ -118,54 +118,76 @@ dx_kernel(const float* __restrict__ dl, const T* __restrict__ w, const T* __rest
   }
 }
 
-// partial[s][e][c..c+V) = sum over the tokens of split s of dl[t,e] * x[t, c..c+V):
-// each thread owns one 16-byte column chunk and EB experts.
+// partial[s][e][cols] = sum over the tokens of split s of dl[t,e] * x[t, cols] for a
+// block of 8 column chunks (8 x V columns) and EB experts.  Thread (token lane tl,
+// chunk cc) walks the split's tokens tl, tl + 32, ... with several 16-byte loads in
+// flight; the 32 token lanes are then summed in a fixed order (warp shuffles, then
+// shared memory), so the result does not depend on timing.
 template <typename T, int EB>
 __global__ void __launch_bounds__(256)
 dwr_partial_kernel(const float* __restrict__ dl, const T* __restrict__ x,
                    float* __restrict__ partial, int ntok, int d, int E, int tok_per_split) {
   constexpr int V = Vec16<T>::N;
-  __shared__ float s_dl[kTT][EB];
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  const int e0 = blockIdx.y * EB;
-  const int s = blockIdx.z;
-  const int ta = s * tok_per_split, tb = min(ntok, ta + tok_per_split);
+  constexpr int U = 4;                       // tokens in flight per thread
+  __shared__ float s_red[8][8][EB * V];      // [warp][chunk][expert x element]
+  const int cc = threadIdx.x & 7, tl = threadIdx.x >> 3;   // tl: 0 .. 31
+  const int warp = threadIdx.x >> 5;
+  const int c = blockIdx.x * 8 + cc;         // 16-byte column chunk
+  const int e0 = blockIdx.z * EB;
+  const int ta = blockIdx.y * tok_per_split, tb = min(ntok, ta + tok_per_split);
   const bool live = c < d / V;
   float acc[EB][V];
 #pragma unroll
   for (int e = 0; e < EB; ++e)
 #pragma unroll
     for (int i = 0; i < V; ++i) acc[e][i] = 0.f;
-  for (int t0 = ta; t0 < tb; t0 += kTT) {
-    for (int i = threadIdx.x; i < kTT * EB; i += blockDim.x) {
-      const int r = i / EB, e = i % EB;
-      s_dl[r][e] = (t0 + r < tb && e0 + e < E) ? dl[(int64_t)(t0 + r) * E + e0 + e] : 0.f;
-    }
-    __syncthreads();
-    if (live) {
-      const int n = min(kTT, tb - t0);
-#pragma unroll 4
-      for (int r = 0; r < n; ++r) {
-        Vec16<T> xv;
-        xv.raw = ldg16(x + (int64_t)(t0 + r) * d + (int64_t)c * V);
+  if (live) {
+    for (int t0 = ta + tl; t0 < tb; t0 += 32 * U) {
+      Vec16<T> xv[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int t = t0 + 32 * u;
+        xv[u].raw = t < tb ? ldg16(x + (int64_t)t * d + (int64_t)c * V) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int t = t0 + 32 * u;
+        if (t >= tb) break;
 #pragma unroll
         for (int e = 0; e < EB; ++e) {
-          const float g = s_dl[r][e];
+          const float g = e0 + e < E ? __ldg(dl + (int64_t)t * E + e0 + e) : 0.f;
 #pragma unroll
-          for (int i = 0; i < V; ++i) acc[e][i] = fmaf(g, xv.get(i), acc[e][i]);
+          for (int i = 0; i < V; ++i) acc[e][i] = fmaf(g, xv[u].get(i), acc[e][i]);
         }
       }
     }
-    __syncthreads();
   }
-  if (!live) return;
+  // token lanes tl and tl ^ 1, tl ^ 2 of a warp differ in lane bits 3 and 4
 #pragma unroll
-  for (int e = 0; e < EB; ++e) {
-    if (e0 + e >= E) break;
-    float* dst = partial + ((int64_t)s * E + e0 + e) * d + (int64_t)c * V;
+  for (int e = 0; e < EB; ++e)
 #pragma unroll
-    for (int i = 0; i < V; i += 4)
-      *reinterpret_cast<float4*>(dst + i) = make_float4(acc[e][i], acc[e][i + 1], acc[e][i + 2], acc[e][i + 3]);
+    for (int i = 0; i < V; ++i) {
+      float v = acc[e][i];
+      v += __shfl_xor_sync(0xffffffffu, v, 8);
+      v += __shfl_xor_sync(0xffffffffu, v, 16);
+      acc[e][i] = v;
+    }
+  if ((threadIdx.x & 31) < 8) {
+#pragma unroll
+    for (int e = 0; e < EB; ++e)
+#pragma unroll
+      for (int i = 0; i < V; ++i) s_red[warp][cc][e * V + i] = acc[e][i];
+  }
+  __syncthreads();
+  // 8 chunks x EB x V sums over the 8 warps, in warp order
+  for (int o = threadIdx.x; o < 8 * EB * V; o += blockDim.x) {
+    const int ch = o / (EB * V), r = o % (EB * V), e = r / V, i = r % V;
+    const int cg = blockIdx.x * 8 + ch;
+    if (cg >= d / V || e0 + e >= E) continue;
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) v += s_red[w][ch][r];
+    partial[((int64_t)blockIdx.y * E + e0 + e) * d + (int64_t)cg * V + i] = v;
   }
 }
 
@@ -216,7 +238,7 @@ cudaError_t route_bwd_t(const void* x, const void* w_router, const float* logits
                                               static_cast<const T*>(dx_perm), slot_row,
                                               static_cast<T*>(dx), T_, d, E, k);
     const int tps = (T_ + splits - 1) / splits;
-    dim3 g2((d / V + 255) / 256, (E + EB - 1) / EB, splits);
+    dim3 g2((d / V + 7) / 8, splits, (E + EB - 1) / EB);
     dwr_partial_kernel<T, EB><<<g2, 256, 0, st>>>(dl, static_cast<const T*>(x), partial, T_, d,
                                                   E, tps);
     dwr_reduce_kernel<<<(int)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, st>>>(
