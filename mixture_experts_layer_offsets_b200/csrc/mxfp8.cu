@@ -346,29 +346,35 @@ mx_cols_atoms_kernel(const T* __restrict__ src, int64_t rows, int64_t K, int64_t
   }
 }
 
-// FP32 master weights -> both MXFP8 copies in one pass over a 128 x 128 tile of one
-// expert's [Rw, Kw] matrix: q0 / s0 in blocks of 32 along a row (K-major GEMM operand),
-// q1 / s1 in blocks of 32 rows within a column (MN-major GEMM operand).
+// FP32 master weights -> both MXFP8 copies in one pass over a 64 x 128 half tile (rows
+// 64 h .. of a 128 x 128 tile) of one expert's [Rw, Kw] matrix: q0 / s0 in blocks of 32
+// along a row (K-major GEMM operand), q1 / s1 in blocks of 32 rows within a column
+// (MN-major GEMM operand).
 //   s0 atom ((e * Rw/128 + row tile) * Kw/128 + kq), kq the 128-column stage.
 //   s1 atom ((e * Rw/128 + kq) * Kw/128 + column tile), kq the 128-row stage.
-constexpr int kWPitch = 132;  // fp32 pitch of the staged tile (bank-conflict-free columns)
-__global__ void __launch_bounds__(256)
+// The half tile is staged in shared memory with 36 floats per 32-column block (4 words of
+// padding, so that the row pass writes and the column pass reads without bank conflicts);
+// a half tile owns half of each of its two atoms' bytes.
+constexpr int kWBlk = 36;              // floats per staged 32-column block
+constexpr int kWPitch = 4 * kWBlk;     // floats per staged row
+constexpr int kWSmem = 64 * kWPitch * 4 + 64 * 128 + 256 + 256;
+__global__ void __launch_bounds__(128)
 mx_weights_kernel(const float* __restrict__ w, int Rw, int Kw, uint8_t* __restrict__ q0,
                   uint8_t* __restrict__ s0, uint8_t* __restrict__ q1, uint8_t* __restrict__ s1) {
-  extern __shared__ float tile[];                       // [128][kWPitch]
-  uint8_t* qt = reinterpret_cast<uint8_t*>(tile + 128 * kWPitch);  // [128][128] q1 bytes
-  uint8_t* sa0 = qt + 128 * 128;                        // this tile's s0 atom (512 B)
-  uint8_t* sa1 = sa0 + 512;                             // and its s1 atom
-  const int e = blockIdx.z, rt = blockIdx.y, ct = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid & 31;
-  const int64_t row0 = (int64_t)e * Rw + rt * 128;
+  extern __shared__ float tile[];                                  // [64][kWPitch]
+  uint8_t* qt = reinterpret_cast<uint8_t*>(tile + 64 * kWPitch);   // [64][128] q1 bytes
+  uint8_t* sa0 = qt + 64 * 128;          // s0 bytes of rows 64 h .. 64 h + 63: [32][8]
+  uint8_t* sa1 = sa0 + 256;              // s1 bytes of row blocks 2 h, 2 h + 1: [128][2]
+  const int e = blockIdx.z, rt = blockIdx.y >> 1, half = blockIdx.y & 1, ct = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int64_t row0 = (int64_t)e * Rw + rt * 128 + half * 64;
   const int col0 = ct * 128;
   // pass 1: blocks along rows; a quad of lanes covers one 32-wide block.  All sixteen
   // 16-byte loads of a thread are issued before any is used.
   float4 ld[16];
 #pragma unroll
   for (int it = 0; it < 8; ++it) {
-    const int task = it * 256 + tid;          // 2048 = 128 rows x 4 blocks x 4 parts
+    const int task = it * 128 + tid;          // 1024 = 64 rows x 4 blocks x 4 parts
     const int r = task >> 4, kb = (task >> 2) & 3, part = task & 3;
     const float* p = w + (row0 + r) * Kw + col0 + kb * 32 + part * 8;
     ld[2 * it] = __ldg(reinterpret_cast<const float4*>(p));
@@ -376,12 +382,13 @@ mx_weights_kernel(const float* __restrict__ w, int Rw, int Kw, uint8_t* __restri
   }
 #pragma unroll
   for (int it = 0; it < 8; ++it) {
-    const int task = it * 256 + tid;
+    const int task = it * 128 + tid;
     const int r = task >> 4, kb = (task >> 2) & 3, part = task & 3;
     const float4 a = ld[2 * it], b = ld[2 * it + 1];
     float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    *reinterpret_cast<float4*>(tile + r * kWPitch + kb * 32 + part * 8) = a;
-    *reinterpret_cast<float4*>(tile + r * kWPitch + kb * 32 + part * 8 + 4) = b;
+    float* t = tile + r * kWPitch + kb * kWBlk + part * 8;
+    *reinterpret_cast<float4*>(t) = a;
+    *reinterpret_cast<float4*>(t + 4) = b;
     float amax = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
@@ -393,43 +400,52 @@ mx_weights_kernel(const float* __restrict__ w, int Rw, int Kw, uint8_t* __restri
     out.x = e4m3_pair(v[1] * mul, v[0] * mul) | (e4m3_pair(v[3] * mul, v[2] * mul) << 16);
     out.y = e4m3_pair(v[5] * mul, v[4] * mul) | (e4m3_pair(v[7] * mul, v[6] * mul) << 16);
     *reinterpret_cast<uint2*>(q0 + (row0 + r) * Kw + col0 + kb * 32 + part * 8) = out;
-    if (part == 0) sa0[atom_byte(r, kb)] = (uint8_t)(ex + 127);
+    // atom row r % 32 holds groups (r / 32) of 4 bytes; this half owns groups 2 h, 2 h + 1
+    if (part == 0) sa0[(r & 31) * 8 + (r >> 5) * 4 + kb] = (uint8_t)(ex + 127);
   }
-  (void)lane;
   __syncthreads();
-  // pass 2: blocks of 32 rows within a column
-#pragma unroll 1
-  for (int it = 0; it < 2; ++it) {
-    const int c = tid & 127, rb = (tid >> 7) + 2 * it;
-    float amax = 0.f;
+  // pass 2: blocks of 32 rows within a column; a thread takes two adjacent columns of one
+  // row block (64 column pairs x 2 row blocks)
+  {
+    const int cp = tid & 63, rb = tid >> 6;
+    const int c = 2 * cp;
+    const float* col = tile + (c >> 5) * kWBlk + (c & 31);
+    float am0 = 0.f, am1 = 0.f;
 #pragma unroll 8
-    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(tile[(rb * 32 + i) * kWPitch + c]));
-    const int ex = block_exponent(amax);
-    const float mul = pow2_neg(ex);
-#pragma unroll 8
-    for (int i = 0; i < 32; i += 2) {
-      const uint32_t pr = e4m3_pair(tile[(rb * 32 + i + 1) * kWPitch + c] * mul,
-                                    tile[(rb * 32 + i) * kWPitch + c] * mul);
-      qt[(rb * 32 + i) * 128 + c] = (uint8_t)(pr & 0xFF);
-      qt[(rb * 32 + i + 1) * 128 + c] = (uint8_t)(pr >> 8);
+    for (int i = 0; i < 32; ++i) {
+      const float2 v = *reinterpret_cast<const float2*>(col + (rb * 32 + i) * kWPitch);
+      am0 = fmaxf(am0, fabsf(v.x));
+      am1 = fmaxf(am1, fabsf(v.y));
     }
-    sa1[atom_byte(c, rb)] = (uint8_t)(ex + 127);
+    const int ex0 = block_exponent(am0), ex1 = block_exponent(am1);
+    const float m0 = pow2_neg(ex0), m1 = pow2_neg(ex1);
+#pragma unroll 8
+    for (int i = 0; i < 32; ++i) {
+      const float2 v = *reinterpret_cast<const float2*>(col + (rb * 32 + i) * kWPitch);
+      *reinterpret_cast<uint16_t*>(qt + (rb * 32 + i) * 128 + c) = (uint16_t)e4m3_pair(v.y * m1, v.x * m0);
+    }
+    // atom bytes (c % 32) * 16 + (c / 32) * 4 + (2 h + rb): two bytes per column here
+    sa1[c * 2 + rb] = (uint8_t)(ex0 + 127);
+    sa1[(c + 1) * 2 + rb] = (uint8_t)(ex1 + 127);
   }
   __syncthreads();
-  // write the q1 tile (128 rows x 128 bytes) and both scale atoms, 16 bytes per store
+  // write the q1 half tile (64 rows x 128 bytes), 16 bytes per store
 #pragma unroll
   for (int it = 0; it < 4; ++it) {
-    const int idx = it * 256 + tid;            // 1024 pieces of 16 bytes
+    const int idx = it * 128 + tid;            // 512 pieces of 16 bytes
     const int r = idx >> 3, c16 = idx & 7;
     *reinterpret_cast<uint4*>(q1 + (row0 + r) * Kw + col0 + c16 * 16) =
         *reinterpret_cast<const uint4*>(qt + r * 128 + c16 * 16);
   }
-  const int64_t atom = (((int64_t)e * (Rw >> 7) + rt) * (Kw >> 7) + ct) * 512;
-  if (tid < 32)
-    *reinterpret_cast<uint4*>(s0 + atom + tid * 16) = *reinterpret_cast<const uint4*>(sa0 + tid * 16);
-  else if (tid < 64)
-    *reinterpret_cast<uint4*>(s1 + atom + (tid - 32) * 16) =
-        *reinterpret_cast<const uint4*>(sa1 + (tid - 32) * 16);
+  uint8_t* a0 = s0 + (((int64_t)e * (Rw >> 7) + rt) * (Kw >> 7) + ct) * 512;
+  uint8_t* a1 = s1 + (((int64_t)e * (Rw >> 7) + rt) * (Kw >> 7) + ct) * 512;
+  if (tid < 32) {   // s0: 8 bytes per atom row
+    *reinterpret_cast<uint2*>(a0 + tid * 16 + half * 8) = *reinterpret_cast<const uint2*>(sa0 + tid * 8);
+  } else {          // s1: 2 bytes per column, at offset (c % 32) * 16 + (c / 32) * 4 + 2 h
+    for (int c = tid - 32; c < 128; c += 96)
+      *reinterpret_cast<uint16_t*>(a1 + (c & 31) * 16 + (c >> 5) * 4 + half * 2) =
+          *reinterpret_cast<const uint16_t*>(sa1 + c * 2);
+  }
 }
 
 }  // namespace
@@ -464,12 +480,11 @@ cudaError_t mxfp8_cols_atoms(int64_t rows, int64_t K, int64_t ld, const void* sr
 cudaError_t mxfp8_weights(const float* w, int E, int Rw, int Kw, uint8_t* q0, uint8_t* s0,
                           uint8_t* q1, uint8_t* s1, cudaStream_t st) {
   if (E == 0) return cudaSuccess;
-  const size_t smem = 128 * kWPitch * sizeof(float) + 128 * 128 + 1024;
   cudaError_t err = cudaFuncSetAttribute(mx_weights_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+                                         kWSmem);
   if (err != cudaSuccess) return err;
-  dim3 grid((unsigned)(Kw / 128), (unsigned)(Rw / 128), (unsigned)E);
-  mx_weights_kernel<<<grid, 256, smem, st>>>(w, Rw, Kw, q0, s0, q1, s1);
+  dim3 grid((unsigned)(Kw / 128), (unsigned)(Rw / 64), (unsigned)E);
+  mx_weights_kernel<<<grid, 128, kWSmem, st>>>(w, Rw, Kw, q0, s0, q1, s1);
   return cudaGetLastError();
 }
 
