@@ -207,9 +207,10 @@ moe_status moe_mx_quantize_weights(moe_shape shape, const float* w1, const float
  * MOE_MXFP8 (kongchang, boundary-conditions section: MXFP8 cuts GEMM time and
  * saved-activation bytes): x_perm, act_saved and y_perm stay bf16; mx is a HOST
  * pointer to a moe_mx_weights whose members are device pointers (w1, w2 are not
- * read and may be NULL); x and h are quantised
- * along their rows in the workspace and the GEMMs run block-scaled E4M3 x E4M3
- * with fp32 accumulation.  Needs d % 128 == 0 and f % 128 == 0. */
+ * read and may be NULL); x and h are quantised, in one pass each, along their rows
+ * (for this call's GEMMs) and in 32-row token blocks (kept in `ws` for the backward), and
+ * the GEMMs run block-scaled E4M3 x E4M3 with fp32 accumulation.  Needs d % 128 == 0 and
+ * f % 128 == 0. */
 moe_status moe_grouped_ffn_fwd(moe_shape shape, int dtype, int64_t rows, const void* x_perm,
                                const int32_t* offsets, const void* w1, const void* w2,
                                const void* mx, void* act_saved, void* y_perm, void* ws,
@@ -244,7 +245,10 @@ moe_status moe_combine_bwd(moe_shape shape, int dtype, const void* dout, const v
  * Uses 2*f*rows elements of scratch in `ws` for [da | du].
  * MOE_MXFP8: dy_perm, x_perm, act_saved, dx_perm bf16; mx as for the forward;
  * dy and [da | du] are quantised along their rows for the dgrad GEMMs, and dy, h,
- * [da | du], x in 32-row blocks restarting at every expert for the wgrad GEMMs. */
+ * [da | du], x in 32-row blocks restarting at every expert for the wgrad GEMMs.  The
+ * token-block copies of x and h (and the row/block maps) are the ones the forward of the
+ * same step wrote into `ws`: pass the same workspace, with no call using it in between
+ * (moe_combine and moe_combine_bwd take none), and the same offsets. */
 moe_status moe_grouped_ffn_bwd(moe_shape shape, int dtype, int64_t rows, const void* dy_perm,
                                const void* x_perm, const void* act_saved,
                                const int32_t* offsets, const void* w1, const void* w2,

@@ -1644,10 +1644,12 @@ size_t wgrad_part_bytes(const FfnShape& s, bool fp8) {
 namespace {
 
 struct MxLayout {
-  size_t rt;                                          // row -> tile map
-  size_t qx0, sx0, qh0, sh0;                         // forward
-  size_t dadu, qdy0, sdy0, qda0, sda0;               // backward, dgrad operands
-  size_t qdy1, sdy1, qh1, sh1, qda1, sda1, qx1, sx1;  // backward, wgrad operands
+  // kept from the forward to the backward: the token-block copies of x and h
+  size_t qx1, sx1, qh1, sh1;
+  size_t rt, map, cnt;                                // row -> tile map, token-block map
+  size_t qx0, sx0, qh0, sh0;                          // forward row copies
+  size_t dadu, qdy0, sdy0, qda0, sda0;                // backward, dgrad operands
+  size_t qdy1, sdy1, qda1, sda1;                      // backward, wgrad operands
   size_t part;                                        // split weight-gradient partial sums
   size_t fwd_bytes, bwd_bytes;
 };
@@ -1661,7 +1663,11 @@ MxLayout mx_layout(const FfnShape& s) {
   MxLayout L;
   size_t o = 0;
   auto take = [&](size_t bytes) { const size_t at = o; o += align256(bytes); return at; };
+  L.qx1 = take(R * d); L.sx1 = take(atoms(d));
+  L.qh1 = take(R * f); L.sh1 = take(atoms(f));
   L.rt = take(R * 4);
+  L.map = take((R / 32 + s.E) * 16);
+  L.cnt = take(4);
   const size_t base = o;
   L.qx0 = take(R * d); L.sx0 = take(atoms(d)); L.qh0 = take(R * f); L.sh0 = take(atoms(f));
   L.fwd_bytes = o;
@@ -1670,9 +1676,7 @@ MxLayout mx_layout(const FfnShape& s) {
   L.qdy0 = take(R * d); L.sdy0 = take(atoms(d));
   L.qda0 = take(R * 2 * f); L.sda0 = take(atoms(2 * f));
   L.qdy1 = take(R * d); L.sdy1 = take(atoms(d));
-  L.qh1 = take(R * f); L.sh1 = take(atoms(f));
   L.qda1 = take(R * 2 * f); L.sda1 = take(atoms(2 * f));
-  L.qx1 = take(R * d); L.sx1 = take(atoms(d));
   L.part = take(wgrad_part_bytes(s, true));
   L.bwd_bytes = o;
   return L;
@@ -1717,9 +1721,14 @@ cudaError_t ffn_fwd_mx(const FfnShape& s, const void* x_perm, const int32_t* off
   const MxLayout L = mx_layout(s);
   const __nv_bfloat16* actb = static_cast<const __nv_bfloat16*>(act);
   int32_t* rt = reinterpret_cast<int32_t*>(ws + L.rt);
-  if ((err = row_tile_launch(offsets, E, R, rt, st)) != cudaSuccess) return err;
-  // x along d; gate/up GEMM with the SwiGLU epilogue
-  if ((err = mxfp8_rows_atoms(R, d, d, x_perm, rt, ws + L.qx0, ws + L.sx0, st)) != cudaSuccess)
+  int4* map = reinterpret_cast<int4*>(ws + L.map);
+  int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
+  if ((err = row_tile_launch(offsets, E, R, rt, st)) != cudaSuccess ||
+      (err = seg_blocks_launch(offsets, E, map, cnt, st)) != cudaSuccess)
+    return err;
+  // x along d (gate/up GEMM) and in token blocks (kept for the dW1 GEMM of the backward)
+  if ((err = mxfp8_act(R, E, d, d, x_perm, map, cnt, rt, ws + L.qx0, ws + L.sx0, ws + L.qx1,
+                       ws + L.sx1, st)) != cudaSuccess)
     return err;
   GemmParams p1 = mx_params(s, offsets, status);
   if (!tmap(&p1.tmA, ws + L.qx0, d, R, d, 128, 128, false, true) ||
@@ -1733,8 +1742,9 @@ cudaError_t ffn_fwd_mx(const FfnShape& s, const void* x_perm, const int32_t* off
   // 128 gate + 128 up columns per tile
   if ((err = launch_mx<256, false, false, EPI_SWIGLU_FWD, false>(p1, m_tile_bound(s) * (f / 128), st)) != cudaSuccess)
     return err;
-  // h along f; down GEMM
-  if ((err = mxfp8_rows_atoms(R, f, 3 * f, actb + 2 * f, rt, ws + L.qh0, ws + L.sh0, st)) != cudaSuccess)
+  // h along f (down GEMM) and in token blocks (kept for the dW2 GEMM of the backward)
+  if ((err = mxfp8_act(R, E, f, 3 * f, actb + 2 * f, map, cnt, rt, ws + L.qh0, ws + L.sh0,
+                       ws + L.qh1, ws + L.sh1, st)) != cudaSuccess)
     return err;
   GemmParams p2 = mx_params(s, offsets, status);
   if (!tmap(&p2.tmA, ws + L.qh0, f, R, f, 128, 128, false, true) ||
@@ -1761,10 +1771,15 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
   const __nv_bfloat16* actb = static_cast<const __nv_bfloat16*>(act);
   __nv_bfloat16* dadu = reinterpret_cast<__nv_bfloat16*>(ws + L.dadu);
   int32_t* rt = reinterpret_cast<int32_t*>(ws + L.rt);
+  int4* map = reinterpret_cast<int4*>(ws + L.map);
+  int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
+  (void)x_perm;  // its token-block copy comes from the forward
   if (R > 0) {
-    if ((err = row_tile_launch(offsets, E, R, rt, st)) != cudaSuccess) return err;
-    // dgrad 1: dh = dy W2 (dy along d, W2 along its d rows), SwiGLU backward -> [da | du]
-    if ((err = mxfp8_rows_atoms(R, d, d, dy_perm, rt, ws + L.qdy0, ws + L.sdy0, st)) != cudaSuccess)
+    // (the row-tile and token-block maps of the forward are still in the workspace)
+    // dgrad 1: dh = dy W2 (dy along d, W2 along its d rows), SwiGLU backward -> [da | du];
+    // dy also in token blocks for the dW2 GEMM
+    if ((err = mxfp8_act(R, E, d, d, dy_perm, map, cnt, rt, ws + L.qdy0, ws + L.sdy0, ws + L.qdy1,
+                         ws + L.sdy1, st)) != cudaSuccess)
       return err;
     GemmParams p3 = mx_params(s, offsets, status);
     if (!tmap(&p3.tmA, ws + L.qdy0, d, R, d, 128, 128, false, true) ||
@@ -1778,8 +1793,10 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
     p3.act = actb; p3.ld_act = 3 * f;
     if ((err = launch_mx_n<false, true, EPI_SWIGLU_BWD, false>(p3, f, m_tile_bound(s), st)) != cudaSuccess)
       return err;
-    // dgrad 2: dx = [da | du] W1 ([da | du] along 2f, W1 along its 2f rows)
-    if ((err = mxfp8_rows_atoms(R, 2 * f, 2 * f, dadu, rt, ws + L.qda0, ws + L.sda0, st)) != cudaSuccess)
+    // dgrad 2: dx = [da | du] W1 ([da | du] along 2f, W1 along its 2f rows); [da | du]
+    // also in token blocks for the dW1 GEMM
+    if ((err = mxfp8_act(R, E, 2 * f, 2 * f, dadu, map, cnt, rt, ws + L.qda0, ws + L.sda0,
+                         ws + L.qda1, ws + L.sda1, st)) != cudaSuccess)
       return err;
     GemmParams p4 = mx_params(s, offsets, status);
     if (!tmap(&p4.tmA, ws + L.qda0, 2 * f, R, 2 * f, 128, 128, false, true) ||
@@ -1791,12 +1808,6 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
     p4.N = d; p4.K = 2 * f; p4.b_rows = 2 * f;
     p4.out = static_cast<__nv_bfloat16*>(dx_perm); p4.ld_out = d;
     if ((err = launch_mx_n<false, true, EPI_STORE, false>(p4, d, m_tile_bound(s), st)) != cudaSuccess)
-      return err;
-    // wgrad operands along the token axis, 32-row blocks restarting at each expert
-    if ((err = mxfp8_cols_atoms(R, d, d, dy_perm, offsets, E, ws + L.qdy1, ws + L.sdy1, st)) != cudaSuccess ||
-        (err = mxfp8_cols_atoms(R, f, 3 * f, actb + 2 * f, offsets, E, ws + L.qh1, ws + L.sh1, st)) != cudaSuccess ||
-        (err = mxfp8_cols_atoms(R, 2 * f, 2 * f, dadu, offsets, E, ws + L.qda1, ws + L.sda1, st)) != cudaSuccess ||
-        (err = mxfp8_cols_atoms(R, d, d, x_perm, offsets, E, ws + L.qx1, ws + L.sx1, st)) != cudaSuccess)
       return err;
   }
   // wgrad 2: dW2[e] = dy^T h  (M = d, N = f)

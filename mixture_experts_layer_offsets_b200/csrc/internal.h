@@ -74,17 +74,18 @@ cudaError_t mxfp8_launch_ld(int64_t rows, int64_t K, int64_t ld, bool src_bf16, 
 // Scale atoms of the block-scaled MMA (512 bytes: 128 rows x 4 blocks of 32 along K,
 // byte (r % 32) * 16 + (r / 32) * 4 + kb), laid out in the order the grouped GEMM reads:
 //   row_tile_launch: row -> tile * 128 + row in tile of the row-grouped GEMMs (-1 outside)
-//   mxfp8_rows_atoms: blocks along rows (bf16 source, row stride ld), atom (tile * K/128 + kq)
-//   mxfp8_cols_atoms: 32-row blocks restarting at segments, atom (stage * K/128 + col / 128)
 //   mxfp8_weights: FP32 [E][Rw][Kw] -> row-block and column-block copies (see mxfp8.cu)
 cudaError_t row_tile_launch(const int32_t* offsets, int E, int64_t rows, int32_t* out, cudaStream_t st);
-cudaError_t mxfp8_rows_atoms(int64_t rows, int64_t K, int64_t ld, const void* src_bf16,
-                             const int32_t* row_tile, uint8_t* q, uint8_t* atoms, cudaStream_t st);
-cudaError_t mxfp8_cols_atoms(int64_t rows, int64_t K, int64_t ld, const void* src_bf16,
-                             const int32_t* seg, int nseg, uint8_t* q, uint8_t* atoms,
-                             cudaStream_t st);
 cudaError_t mxfp8_weights(const float* w, int E, int Rw, int Kw, uint8_t* q0, uint8_t* s0,
                           uint8_t* q1, uint8_t* s1, cudaStream_t st);
+//   seg_blocks_launch: the 32-row token blocks of all segments (at most rows/32 + E)
+//   mxfp8_act: one pass over a bf16 activation writing its row copy (row-tile atoms) and its
+//     token-block copy (stage atoms)
+cudaError_t seg_blocks_launch(const int32_t* offsets, int E, int4* map, int32_t* count,
+                              cudaStream_t st);
+cudaError_t mxfp8_act(int64_t rows, int E, int64_t K, int64_t ld, const void* src_bf16,
+                      const int4* map, const int32_t* count, const int32_t* row_tile, uint8_t* q_r,
+                      uint8_t* atoms_r, uint8_t* q_c, uint8_t* atoms_c, cudaStream_t st);
 
 // ---------------------------------------------------------- grouped FFN
 struct FfnShape {

@@ -217,135 +217,6 @@ row_tile_kernel(const int32_t* __restrict__ offsets, int E, int64_t rows, int32_
   }
 }
 
-// axis 0 (blocks along rows) with scales written as row-tile atoms:
-// atom (tile * K/128 + k / 128), the tile and the row in it from row_tile.
-template <typename T>
-__global__ void __launch_bounds__(256)
-mx_rows_atoms_kernel(const T* __restrict__ src, int64_t nblocks, int64_t kblocks, int64_t ld,
-                     const int32_t* __restrict__ row_tile, uint8_t* __restrict__ q,
-                     uint8_t* __restrict__ atoms) {
-  const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t blk = g >> 2;
-  const int part = (int)(g & 3);
-  const bool live = blk < nblocks;
-  const int64_t row = live ? blk / kblocks : 0;
-  const int kb = live ? (int)(blk - row * kblocks) : 0;
-  float v[8];
-  if (live) {
-    const T* p = src + row * ld + (int64_t)kb * 32 + part * 8;
-    if constexpr (sizeof(T) == 2) {
-      Vec16<T> a;
-      a.raw = ldg16(p);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = a.get(i);
-    } else {
-      Vec16<T> a, b;
-      a.raw = ldg16(p);
-      b.raw = ldg16(p + 4);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) { v[i] = a.get(i); v[4 + i] = b.get(i); }
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = 0.f;
-  }
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-  if (!live) return;
-  const int e = block_exponent(amax);
-  const float mul = pow2_neg(e);
-  uint2 out;
-  out.x = e4m3_pair(v[1] * mul, v[0] * mul) | (e4m3_pair(v[3] * mul, v[2] * mul) << 16);
-  out.y = e4m3_pair(v[5] * mul, v[4] * mul) | (e4m3_pair(v[7] * mul, v[6] * mul) << 16);
-  *reinterpret_cast<uint2*>(q + blk * 32 + part * 8) = out;
-  if (part == 0) {
-    const int rt = row_tile[row];
-    if (rt >= 0)
-      atoms[((int64_t)(rt >> 7) * (kblocks >> 2) + (kb >> 2)) * 512 + atom_byte(rt & 127, kb & 3)] =
-          (uint8_t)(e + 127);
-  }
-}
-
-// axis 1 (32-row blocks restarting at every segment) with scales written as stage
-// atoms: atom (stage * K/128 + column / 128), stage = 128-row stages of the segments
-// before + (row - segment start) / 128.  The blocks of a segment's last stage that lie
-// past its end get scale byte 127 (2^0), so that the zero rows there stay zero.
-template <typename T>
-__global__ void __launch_bounds__(128)
-mx_cols_atoms_kernel(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
-                     const int32_t* __restrict__ seg, int nseg, uint8_t* __restrict__ q,
-                     uint8_t* __restrict__ atoms) {
-  __shared__ int32_t s_pre[1026];   // 32-row block prefix per segment
-  __shared__ int32_t s_stg[1026];   // 128-row stage prefix per segment
-  __shared__ int32_t s_seg[1026];
-  const int tid = threadIdx.x;
-  for (int g = tid; g <= nseg; g += blockDim.x) s_seg[g] = seg ? seg[g] : (g == 0 ? 0 : (int)rows);
-  __syncthreads();
-  if (tid == 0) {
-    int acc = 0, st = 0;
-    for (int g = 0; g < nseg; ++g) {
-      s_pre[g] = acc;
-      s_stg[g] = st;
-      acc += (s_seg[g + 1] - s_seg[g] + 31) / 32;
-      st += (s_seg[g + 1] - s_seg[g] + 127) / 128;
-    }
-    s_pre[nseg] = acc;
-    s_stg[nseg] = st;
-  }
-  __syncthreads();
-  const int total = s_pre[nseg];
-  const int64_t col = ((int64_t)blockIdx.x * blockDim.x + tid) * 8;
-  if (col >= K) return;
-  const int64_t kq = K >> 7;
-  for (int rb = blockIdx.y; rb < total; rb += gridDim.y) {
-    int lo = 0, hi = nseg - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (s_pre[mid] <= rb) lo = mid; else hi = mid - 1;
-    }
-    const int g = lo;
-    const int lb = rb - s_pre[g];
-    const int64_t r0 = s_seg[g] + (int64_t)lb * 32;
-    const int64_t r1 = min((int64_t)s_seg[g + 1], r0 + 32);
-    float amax[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) amax[i] = 0.f;
-    for (int64_t r = r0; r < r1; ++r) {
-      float v[8];
-      load8(src + r * ld + col, v);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) amax[i] = fmaxf(amax[i], fabsf(v[i]));
-    }
-    int ex[8];
-    float mul[8];
-    uint8_t* at = atoms + ((int64_t)(s_stg[g] + (lb >> 2)) * kq + (col >> 7)) * 512;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      ex[i] = block_exponent(amax[i]);
-      mul[i] = pow2_neg(ex[i]);
-      at[atom_byte((int)((col + i) & 127), lb & 3)] = (uint8_t)(ex[i] + 127);
-    }
-    if (rb == s_pre[g + 1] - 1) {  // the segment's last block: fill the rest of its stage
-      for (int kb = (lb & 3) + 1; kb < 4; ++kb)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) at[atom_byte((int)((col + i) & 127), kb)] = 0x7F;
-    }
-    for (int64_t r = r0; r < r1; ++r) {
-      float v[8];
-      load8(src + r * ld + col, v);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] *= mul[i];
-      uint2 out;
-      out.x = e4m3_pair(v[1], v[0]) | (e4m3_pair(v[3], v[2]) << 16);
-      out.y = e4m3_pair(v[5], v[4]) | (e4m3_pair(v[7], v[6]) << 16);
-      *reinterpret_cast<uint2*>(q + r * K + col) = out;
-    }
-  }
-}
-
 // FP32 master weights -> both MXFP8 copies in one pass over a 64 x 128 half tile (rows
 // 64 h .. of a 128 x 128 tile) of one expert's [Rw, Kw] matrix: q0 / s0 in blocks of 32
 // along a row (K-major GEMM operand), q1 / s1 in blocks of 32 rows within a column
@@ -448,6 +319,138 @@ mx_weights_kernel(const float* __restrict__ w, int Rw, int Kw, uint8_t* __restri
   }
 }
 
+// 32-row blocks of the token axis, restarting at every segment (expert): block b (in
+// segment order) -> {first row, rows (1..32), 128-row stage over all segments, (position of
+// the block in its stage) | 4 if it is its segment's last block}.  count[0] = number of
+// blocks.  One CTA of 1024 threads (E <= 1024): a scan of the per-segment block counts,
+// then each thread writes its segment's entries.
+__global__ void __launch_bounds__(1024)
+seg_blocks_kernel(const int32_t* __restrict__ offsets, int E, int4* __restrict__ map,
+                  int32_t* __restrict__ count) {
+  const int g = threadIdx.x, lane = g & 31, w = g >> 5;
+  const int r0 = g < E ? offsets[g] : 0, c = g < E ? offsets[g + 1] - r0 : 0;
+  const int nb = (c + 31) / 32, ns = (c + 127) / 128;
+  // inclusive scans of nb and ns over the threads (warp shuffles, then warp totals)
+  int ib = nb, is = ns;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int a = __shfl_up_sync(0xffffffffu, ib, o), b = __shfl_up_sync(0xffffffffu, is, o);
+    if (lane >= o) { ib += a; is += b; }
+  }
+  __shared__ int s_wb[32], s_ws[32];
+  if (lane == 31) { s_wb[w] = ib; s_ws[w] = is; }
+  __syncthreads();
+  if (w == 0) {
+    int vb = s_wb[lane], vs = s_ws[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, vb, o), b = __shfl_up_sync(0xffffffffu, vs, o);
+      if (lane >= o) { vb += a; vs += b; }
+    }
+    s_wb[lane] = vb;
+    s_ws[lane] = vs;
+  }
+  __syncthreads();
+  const int b0 = ib - nb + (w > 0 ? s_wb[w - 1] : 0);
+  const int st0 = is - ns + (w > 0 ? s_ws[w - 1] : 0);
+  for (int lb = 0; lb < nb; ++lb)
+    map[b0 + lb] = make_int4(r0 + 32 * lb, min(32, c - 32 * lb), st0 + lb / 4,
+                             (lb & 3) | (lb == nb - 1 ? 4 : 0));
+  if (g == 1023) count[0] = b0 + nb;
+}
+
+// One pass over a bf16 activation tile of one 32-row token block (of one segment) x 128
+// columns, writing both MXFP8 copies: q_r / atoms_r in blocks of 32 along each row (row-tile
+// atoms, tile and row from row_tile), and q_c / atoms_c in the block's 32 rows within each
+// column (stage atoms; the blocks of a segment's last stage past its end get 2^0).
+constexpr int kActPitch = 136;  // bf16 per staged row (16 bytes of padding)
+__global__ void __launch_bounds__(128)
+mx_act_kernel(const __nv_bfloat16* __restrict__ src, int64_t K, int64_t ld,
+              const int4* __restrict__ map, const int32_t* __restrict__ count,
+              const int32_t* __restrict__ row_tile, uint8_t* __restrict__ q_r,
+              uint8_t* __restrict__ atoms_r, uint8_t* __restrict__ q_c,
+              uint8_t* __restrict__ atoms_c) {
+  __shared__ __align__(16) __nv_bfloat16 s_t[32 * kActPitch];
+  __shared__ __align__(16) uint8_t s_q[32 * 128];
+  const int tid = threadIdx.x, ct = blockIdx.x;
+  const int64_t c0 = (int64_t)ct * 128;
+  const int64_t kq = K >> 7;
+  const int nblocks = count[0];
+  for (int b = blockIdx.y; b < nblocks; b += gridDim.y) {
+    const int4 m = map[b];
+    const int r0 = m.x, n = m.y;
+    // load n rows x 128 columns (16 pieces of 16 bytes per row)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int i = tid + 128 * j, row = i >> 4, p8 = i & 15;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (row < n) v = ldg16(src + (int64_t)(r0 + row) * ld + c0 + p8 * 8);
+      *reinterpret_cast<uint4*>(s_t + row * kActPitch + p8 * 8) = v;
+    }
+    __syncthreads();
+    // rows: thread = (row, 32-column block)
+    {
+      const int row = tid >> 2, kb = tid & 3;
+      if (row < n) {
+        float v[32];
+        const __nv_bfloat16* t = s_t + row * kActPitch + kb * 32;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          Vec16<__nv_bfloat16> a;
+          a.raw = *reinterpret_cast<const uint4*>(t + 8 * i);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[8 * i + e] = a.get(e);
+        }
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+        const int ex = block_exponent(amax);
+        const float mul = pow2_neg(ex);
+        uint32_t w8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          w8[i] = e4m3_pair(v[4 * i + 1] * mul, v[4 * i] * mul) |
+                  (e4m3_pair(v[4 * i + 3] * mul, v[4 * i + 2] * mul) << 16);
+        uint8_t* dq = q_r + (int64_t)(r0 + row) * K + c0 + kb * 32;
+        *reinterpret_cast<uint4*>(dq) = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+        *reinterpret_cast<uint4*>(dq + 16) = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+        const int rt = row_tile[r0 + row];
+        if (rt >= 0) atoms_r[((int64_t)(rt >> 7) * kq + ct) * 512 + atom_byte(rt & 127, kb)] = (uint8_t)(ex + 127);
+      }
+    }
+    // columns: thread = column; the block's n rows
+    {
+      const __nv_bfloat16* t = s_t + tid;
+      float amax = 0.f;
+      for (int i = 0; i < n; ++i) amax = fmaxf(amax, fabsf(__bfloat162float(t[i * kActPitch])));
+      const int ex = block_exponent(amax);
+      const float mul = pow2_neg(ex);
+      for (int i = 0; i < n; i += 2) {
+        const float lo = __bfloat162float(t[i * kActPitch]) * mul;
+        const float hi = i + 1 < n ? __bfloat162float(t[(i + 1) * kActPitch]) * mul : 0.f;
+        const uint32_t pr = e4m3_pair(hi, lo);
+        s_q[i * 128 + tid] = (uint8_t)(pr & 0xFF);
+        if (i + 1 < n) s_q[(i + 1) * 128 + tid] = (uint8_t)(pr >> 8);
+      }
+      uint8_t* at = atoms_c + ((int64_t)m.z * kq + ct) * 512;
+      const int pos = m.w & 3;
+      at[atom_byte(tid, pos)] = (uint8_t)(ex + 127);
+      if (m.w & 4)
+        for (int kb = pos + 1; kb < 4; ++kb) at[atom_byte(tid, kb)] = 0x7F;
+    }
+    __syncthreads();
+    // the column copy's rows, 16 bytes per store
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int i = tid + 128 * j, row = i >> 3, p16 = i & 7;
+      if (row < n)
+        *reinterpret_cast<uint4*>(q_c + (int64_t)(r0 + row) * K + c0 + p16 * 16) =
+            *reinterpret_cast<const uint4*>(s_q + row * 128 + p16 * 16);
+    }
+    __syncthreads();
+  }
+}
+
 }  // namespace
 
 cudaError_t row_tile_launch(const int32_t* offsets, int E, int64_t rows, int32_t* out, cudaStream_t st) {
@@ -457,23 +460,19 @@ cudaError_t row_tile_launch(const int32_t* offsets, int E, int64_t rows, int32_t
   return cudaGetLastError();
 }
 
-cudaError_t mxfp8_rows_atoms(int64_t rows, int64_t K, int64_t ld, const void* src_bf16,
-                             const int32_t* row_tile, uint8_t* q, uint8_t* atoms, cudaStream_t st) {
-  if (rows == 0) return cudaSuccess;
-  const int64_t nblocks = rows * K / 32;
-  const int grid = (int)((nblocks * 4 + 255) / 256);
-  mx_rows_atoms_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(src_bf16), nblocks, K / 32, ld, row_tile, q, atoms);
+cudaError_t seg_blocks_launch(const int32_t* offsets, int E, int4* map, int32_t* count,
+                              cudaStream_t st) {
+  seg_blocks_kernel<<<1, 1024, 0, st>>>(offsets, E, map, count);
   return cudaGetLastError();
 }
 
-cudaError_t mxfp8_cols_atoms(int64_t rows, int64_t K, int64_t ld, const void* src_bf16,
-                             const int32_t* seg, int nseg, uint8_t* q, uint8_t* atoms,
-                             cudaStream_t st) {
+cudaError_t mxfp8_act(int64_t rows, int E, int64_t K, int64_t ld, const void* src_bf16,
+                      const int4* map, const int32_t* count, const int32_t* row_tile, uint8_t* q_r,
+                      uint8_t* atoms_r, uint8_t* q_c, uint8_t* atoms_c, cudaStream_t st) {
   if (rows == 0) return cudaSuccess;
-  dim3 grid((unsigned)((K / 8 + 127) / 128), (unsigned)std::min<int64_t>(rows / 32 + nseg + 1, 65535));
-  mx_cols_atoms_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(src_bf16), rows, K, ld, seg, nseg, q, atoms);
+  dim3 grid((unsigned)(K / 128), (unsigned)std::min<int64_t>(rows / 32 + E, 65535));
+  mx_act_kernel<<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(src_bf16), K, ld, map,
+                                       count, row_tile, q_r, atoms_r, q_c, atoms_c);
   return cudaGetLastError();
 }
 
