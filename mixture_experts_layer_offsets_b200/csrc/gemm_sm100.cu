@@ -138,8 +138,11 @@ template <int BN, bool PAIR = false, int EPI = 1, bool FP8 = false> struct Cfg {
   static constexpr int kTileM = PAIR ? 2 * BM : BM;     // rows of one scheduled tile
   // TMA-store staging per epilogue warp: bf16 outputs use two 2 KB slots, the fp32
   // weight gradient one; the router epilogues store directly.
+  // (MXFP8 weight gradients, whose short K makes the fp32 stores the longer part of a
+  // tile, keep two slots per warp as well)
   static constexpr size_t kStoreBytes =
-      EPI == EPI_WGRAD ? 8 * 2048 : ((EPI == EPI_ROUTER || EPI == EPI_ROUTER_DX) ? 0 : 8 * 4096);
+      EPI == EPI_WGRAD ? (FP8 ? 8 * 4096 : 8 * 2048)
+                       : ((EPI == EPI_ROUTER || EPI == EPI_ROUTER_DX) ? 0 : 8 * 4096);
   // shared memory after the stage ring: barriers (256 B), offsets and tile prefix
   // (2 x 1025 ints), router histogram (128 x kRouterKMax ints), then the 1024-aligned
   // staging area; as many stages as fit (up to 6)
@@ -1115,12 +1118,13 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
         asm volatile("bar.sync 1, 128;" ::: "memory");  // the histogram is reused by the next tile
       } else if constexpr (EPI == EPI_ROUTER_DX) {
         // router backward: dx = dl w_router (the accumulator) + the token's k expert rows
-        const int k = p.topk;
+        // (no slot_row: one row per token, the token's own row of p.act)
+        const int k = p.slot_row ? p.topk : 1;
         const int64_t tok = ti.m0 + row;
         int rj[kRouterKMax];
 #pragma unroll
         for (int j = 0; j < kRouterKMax; ++j)
-          rj[j] = (valid && j < k) ? __ldg(p.slot_row + tok * k + j) : -1;
+          rj[j] = (valid && j < k) ? (p.slot_row ? __ldg(p.slot_row + tok * k + j) : (int)tok) : -1;
         __nv_bfloat16* orow = p.out + tok * p.ld_out;
 #pragma unroll
         for (int ci = 0; ci < kMine; ++ci) {
@@ -1165,7 +1169,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
           // fp32: stage 16 rows x 32 columns in shared memory (128-byte swizzle) and
           // write them with one TMA store per box: whole 128-byte lines to HBM.  All of
           // this warp's chunks are read before the accumulator is released.
-          uint8_t* sbuf = wbuf;
+          constexpr bool kTwoSlots = kWarpStore >= 4096;
           uint32_t va[kMine][32];
 #pragma unroll
           for (int ci = 0; ci < kMine; ++ci) {
@@ -1187,7 +1191,12 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
             const uint32_t* v = va[ci];
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-              if (lane == 0) tma_store_wait_read();  // the previous box has left the buffer
+              uint8_t* sbuf = wbuf + (kTwoSlots ? (slot & 1) * 2048 : 0);
+              // the store that last used this slot has read it
+              if (lane == 0) {
+                if (kTwoSlots) tma_store_wait_read_le1();
+                else tma_store_wait_read();
+              }
               __syncwarp();
               if ((lane >> 4) == hh) {
                 const int r = lane & 15;
@@ -1200,6 +1209,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
               __syncwarp();
               if (lane == 0)
                 tma_store_2d(tmo, ti.n0 + (c0 + ci) * 32, (int)(orow0 + 16 * hh), sbuf);
+              ++slot;
             }
           }
         } else {

@@ -68,7 +68,7 @@ combine_kernel(const T* __restrict__ y_perm, const int32_t* __restrict__ slot_ro
   for (int t = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); t < ntok;
        t += gridDim.x * kWarpsPerBlock) {
     const int myrow = lane < k ? slot_row[(int64_t)t * k + lane] : -1;
-    const float mygate = lane < k ? gate[(int64_t)t * k + lane] : 0.f;
+    const float mygate = lane < k ? (gate ? gate[(int64_t)t * k + lane] : 1.f) : 0.f;  // no gate: sum
     for (int c0 = 0; c0 < chunks; c0 += 32 * kBatch) {
       float acc[kBatch][V];
 #pragma unroll

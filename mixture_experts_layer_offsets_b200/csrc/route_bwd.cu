@@ -219,8 +219,14 @@ cudaError_t route_bwd_t(const void* x, const void* w_router, const float* logits
     __nv_bfloat16* dl_bf = static_cast<__nv_bfloat16*>(scratch);
     const int tsplits = std::max(1, std::min(32, T_ / 1024));
     dlogit_kernel<<<lgrid, 256, 0, st>>>(logits, topk_idx, dgate, nullptr, dl_bf, T_, E, k);
-    cudaError_t err = route_bwd_tc_launch(x, w_router, dl_bf, dx_perm, slot_row, dx, partial,
-                                          tsplits, T_, d, E, k, status, st);
+    // the k expert rows of each token are summed first by the streaming row-sum (bf16
+    // [T, d] in the workspace); the dx GEMM's epilogue then adds one contiguous row
+    __nv_bfloat16* dxs = reinterpret_cast<__nv_bfloat16*>(
+        reinterpret_cast<uint8_t*>(partial) + align256((size_t)route_bwd_splits(T_) * E * d * 4));
+    cudaError_t err = combine_launch(true, dx_perm, slot_row, nullptr, dxs, T_, d, k, st);
+    if (err != cudaSuccess) return err;
+    err = route_bwd_tc_launch(x, w_router, dl_bf, dxs, nullptr, dx, partial, tsplits, T_, d, E,
+                              k, status, st);
     if (err != cudaSuccess) return err;
     dwr_reduce_kernel<<<(int)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, st>>>(
         partial, dw_router, n, tsplits);
@@ -252,7 +258,9 @@ cudaError_t route_bwd_t(const void* x, const void* w_router, const float* logits
 }  // namespace
 
 size_t route_bwd_ws_bytes(int T, int d, int E) {
-  return align256((size_t)T * E * 4) + align256((size_t)route_bwd_splits(T) * E * d * 4);
+  // dl, the dW_r partial sums, and (tensor-core path) the bf16 row sums of dx_perm
+  return align256((size_t)T * E * 4) + align256((size_t)route_bwd_splits(T) * E * d * 4) +
+         align256((size_t)T * d * 2);
 }
 
 cudaError_t route_bwd_launch(bool bf16, const void* x, const void* w_router, const float* logits,
