@@ -301,6 +301,23 @@ moe_status moe_padded_dispatch(moe_shape shape, int dtype, int32_t capacity, con
                                const int32_t* offsets, void* x_pad, int32_t* pad_row,
                                int32_t* offsets_pad, void* stream);
 
+/* ---- f4: load balance of a routing --------------------------------------
+ * [kongchang] routing section: how evenly the rows spread over the experts
+ * sets the grouped GEMM's speed, more than the auxiliary loss value does.
+ * From counts (device int32 [E], as moe_route writes them), with R = sum c,
+ * mean = R / E, writes device fp32 stats[8]:
+ *   [0] R   [1] mean   [2] max(c)/mean   [3] min(c)/mean
+ *   [4] coefficient of variation sqrt(sum (c - mean)^2 / E) / mean
+ *   [5] number of experts with c == 0
+ *   [6] dropped fraction sum max(0, c - C) / R  of a capacity-C layout
+ *   [7] used fraction (R - dropped) / (E*C)     of its E*C slots
+ * Ratios are 0 when R == 0; [6] and [7] are 0 when capacity == 0 (no padded
+ * layout).  Totals are exact integers, the deviations are summed in double in
+ * a fixed order, each entry rounded once to fp32.  One kernel; nothing goes
+ * to the host.  capacity < 0 or a bad pointer: MOE_ERR_INVALID_ARG. */
+moe_status moe_routing_stats(moe_shape shape, const int32_t* counts, int32_t capacity,
+                             float* stats, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

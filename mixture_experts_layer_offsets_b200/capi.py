@@ -59,6 +59,7 @@ _SIGS = {
     "mxfp8_quantize": (_I, [_I64, _I64, _I, _P, _I, _P, _I, _P, _P, _P]),
     "moe_mx_quantize_weights": (_I, [moe_shape, _P, _P, _P, _P]),
     "moe_padded_dispatch": (_I, [moe_shape, _I, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_routing_stats": (_I, [moe_shape, _P, ctypes.c_int32, _P, _P]),
 }
 
 _lib = None
@@ -202,3 +203,8 @@ def moe_padded_dispatch(shape, dtype, capacity, x, topk_idx, slot_row, offsets, 
     _check("moe_padded_dispatch", lib().moe_padded_dispatch(
         shape, dtype, capacity, _ptr(x), _ptr(topk_idx), _ptr(slot_row), _ptr(offsets),
         _ptr(x_pad), _ptr(pad_row), _ptr(offsets_pad), _stream(stream)))
+
+
+def moe_routing_stats(shape, counts, capacity, stats, stream=None) -> None:
+    _check("moe_routing_stats", lib().moe_routing_stats(
+        shape, _ptr(counts), capacity, _ptr(stats), _stream(stream)))

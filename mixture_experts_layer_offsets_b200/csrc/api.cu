@@ -289,4 +289,12 @@ moe_status moe_padded_dispatch(moe_shape s, int dtype, int32_t capacity, const v
                                             s.E, s.top_k, as_stream(stream)));
 }
 
+moe_status moe_routing_stats(moe_shape s, const int32_t* counts, int32_t capacity, float* stats,
+                             void* stream) {
+  moe_status st = shape_ok(s);
+  if (st != MOE_OK) return st;
+  if (capacity < 0 || !ptrs_ok(counts, stats)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(routing_stats_launch(counts, s.E, capacity, stats, as_stream(stream)));
+}
+
 }  // extern "C"

@@ -37,6 +37,9 @@ bool route_tc_supported(int E, int k, int d);
 cudaError_t route_tc_launch(const RouteArgs& a, int nb, cudaStream_t st);
 
 // ---------------------------------------------------------- row movement
+//   routing_stats_launch: the eight load statistics of moe_routing_stats (E <= 1024)
+cudaError_t routing_stats_launch(const int32_t* counts, int E, int capacity, float* stats,
+                                 cudaStream_t st);
 cudaError_t permute_launch(bool bf16, const void* x, const int32_t* slot_row, void* x_perm,
                            int32_t* perm_src, int T, int d, int k, cudaStream_t st);
 cudaError_t combine_launch(bool bf16, const void* y_perm, const int32_t* slot_row,

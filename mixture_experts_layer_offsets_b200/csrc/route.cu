@@ -338,6 +338,66 @@ cudaError_t route_launch(const RouteArgs& a0, bool bf16, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+
+// ---- load balance of a routing -------------------------------------------
+// [kongchang] routing section: the load spread over the experts is what sets
+// the grouped GEMM's throughput.  One block of 1024 threads, one expert per
+// thread (E <= 1024); integer totals, then the squared deviations in double,
+// both reduced in a fixed order so the result does not depend on timing.
+namespace {
+
+template <class T, class Op>
+__device__ T block_reduce(T v, Op op, T* red) {
+  for (int o = 16; o; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  v = red[l];
+  for (int o = 16; o; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__global__ void __launch_bounds__(1024) routing_stats_kernel(const int32_t* __restrict__ counts,
+                                                             int E, int capacity,
+                                                             float* __restrict__ stats) {
+  __shared__ long long red_i[32];
+  __shared__ double red_d[32];
+  const int e = threadIdx.x;
+  const long long c = e < E ? counts[e] : 0;
+  const long long big = 1ll << 62;
+  auto add = [](long long a, long long b) { return a + b; };
+  const long long R = block_reduce(c, add, red_i);
+  const long long mx = block_reduce(e < E ? c : -big, [](long long a, long long b) { return a > b ? a : b; }, red_i);
+  const long long mn = block_reduce(e < E ? c : big, [](long long a, long long b) { return a < b ? a : b; }, red_i);
+  const long long empty = block_reduce((long long)(e < E && c == 0), add, red_i);
+  const long long over = capacity > 0 ? (c > capacity ? c - capacity : 0) : 0;
+  const long long dropped = block_reduce(over, add, red_i);
+  const double mean = (double)R / E;
+  const double dev = e < E ? ((double)c - mean) * ((double)c - mean) : 0.0;
+  const double ss = block_reduce(dev, [](double a, double b) { return a + b; }, red_d);
+  if (e == 0) {
+    const bool any = R > 0;
+    stats[0] = (float)R;
+    stats[1] = (float)mean;
+    stats[2] = any ? (float)(mx / mean) : 0.f;
+    stats[3] = any ? (float)(mn / mean) : 0.f;
+    stats[4] = any ? (float)(sqrt(ss / E) / mean) : 0.f;
+    stats[5] = (float)empty;
+    const bool cap = capacity > 0 && any;
+    stats[6] = cap ? (float)((double)dropped / R) : 0.f;
+    stats[7] = cap ? (float)((double)(R - dropped) / ((double)E * capacity)) : 0.f;
+  }
+}
+
+}  // namespace
+
+cudaError_t routing_stats_launch(const int32_t* counts, int E, int capacity, float* stats,
+                                 cudaStream_t st) {
+  routing_stats_kernel<<<1, 1024, 0, st>>>(counts, E, capacity, stats);
+  return cudaGetLastError();
+}
+
 }  // namespace moe
 
 // ---------------------------------------------------------------------------

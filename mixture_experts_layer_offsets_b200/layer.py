@@ -73,6 +73,7 @@ class MoELayer:
         self.dw2 = torch.empty(E, d_model, d_ff, dtype=wdt, device=dev)
         self.dx = torch.empty(T, d_model, **act)
         self.dw_router = torch.empty(E, d_model, **f32)
+        self.stats = torch.zeros(8, **f32)
         if capacity:
             self.pad_row = torch.empty(T, top_k, **i32)
             self.offsets_pad = torch.empty(E + 1, **i32)
@@ -141,6 +142,14 @@ class MoELayer:
     def step(self, x, w_router, bias, w1, w2, dout, stream=None):
         self.forward(x, w_router, bias, w1, w2, stream)
         return self.backward(dout, x, w_router, w1, w2, stream)
+
+    def routing_stats(self, capacity: int | None = None, stream=None):
+        """Load statistics of the last forward's routing, on the device (fp32 [8]):
+        rows, mean, max/mean, min/mean, coefficient of variation, empty experts,
+        and for a capacity (the layer's own by default) the dropped and used fractions."""
+        cap = self.capacity if capacity is None else capacity
+        capi.moe_routing_stats(self.shape, self.counts, cap or 0, self.stats, stream)
+        return self.stats
 
     def device_status(self, stream=None) -> int:
         return capi.moe_get_device_status(self.ws, stream)

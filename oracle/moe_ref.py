@@ -23,7 +23,7 @@ __all__ = [
     "slot_rows", "perm_src_from_slots", "route", "route_from_logits",
     "permute", "sigmoid", "silu", "expert_ffn_fwd", "combine", "combine_bwd",
     "expert_ffn_bwd", "route_bwd", "layer_fwd_bwd", "capacity",
-    "padded_layout", "padded_layer_fwd_bwd",
+    "padded_layout", "padded_layer_fwd_bwd", "routing_stats",
 ]
 
 
@@ -397,3 +397,39 @@ def padded_layer_fwd_bwd(x, w_router, w1, w2, dout, k: int, C: int, bias=None,
              dgate=dgate, dy_pad=dy_pad, dx_pad=dx_pad, dw1=dw1, dw2=dw2, dx=dx,
              dw_router=dw_router, dl=dl)
     return r
+
+
+# --------------------------------------------------------------------------
+# Load balance of a routing (kongchang, routing section: balancing the load, not the loss
+# value, is what matters for throughput)
+# --------------------------------------------------------------------------
+
+ROUTING_STATS = ("rows", "mean", "max_over_mean", "min_over_mean", "cv", "empty",
+                 "dropped_frac", "capacity_use")
+
+
+def routing_stats(counts, C: int = 0) -> np.ndarray:
+    """Load statistics of the per-expert row counts ``c`` (R = sum c, E experts):
+
+    rows R; mean R / E; max(c) / mean; min(c) / mean; coefficient of variation
+    std(c) / mean (population std); number of empty experts; and for a capacity C > 0
+    the fraction of the R rows a capacity-C layout drops, sum max(0, c - C) / R, and the
+    fraction of its E * C slots that hold a row, (R - dropped) / (E C).  Ratios are 0
+    when R = 0; the capacity entries are 0 when C = 0.
+    """
+    c = np.asarray(counts, dtype=np.float64)
+    E = c.size
+    R = c.sum()
+    mean = R / E
+    out = np.zeros(8)
+    out[0], out[1] = R, mean
+    if R > 0:
+        out[2] = c.max() / mean
+        out[3] = c.min() / mean
+        out[4] = np.sqrt(np.mean((c - mean) ** 2)) / mean
+    out[5] = float(np.sum(c == 0))
+    if C > 0 and R > 0:
+        dropped = np.maximum(c - C, 0).sum()
+        out[6] = dropped / R
+        out[7] = (R - dropped) / (E * C)
+    return out

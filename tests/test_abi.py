@@ -116,6 +116,9 @@ def test_row_ops_validation(lib):
         == capi.MOE_ERR_INVALID_ARG
     assert lib.moe_padded_dispatch(s, capi.MOE_BF16, 0, *([FAKE] * 7), None) == capi.MOE_ERR_INVALID_ARG
     assert lib.moe_route_bwd(s, capi.MOE_BF16, *([FAKE] * 9), FAKE, 16, None) == capi.MOE_ERR_INVALID_ARG
+    assert lib.moe_routing_stats(s, FAKE, -1, FAKE, None) == capi.MOE_ERR_INVALID_ARG
+    assert lib.moe_routing_stats(s, None, 0, FAKE, None) == capi.MOE_ERR_INVALID_ARG
+    assert lib.moe_routing_stats(_shape(E=2048), FAKE, 0, FAKE, None) == capi.MOE_ERR_INVALID_ARG
     # T == 0 is a valid no-op for the row movers
     assert lib.moe_permute(_shape(T=0), capi.MOE_BF16, None, None, None, None, None) == capi.MOE_OK
 

@@ -14,6 +14,7 @@ import torch
 
 from gpu_helpers import TOL, f64, i64, oracle_for, rel, run_layer
 from mixture_experts_layer_offsets_b200.inputs import CONFIGS, shrink
+from oracle import moe_ref as ref
 
 pytestmark = pytest.mark.gpu
 
@@ -125,3 +126,40 @@ def test_routing_is_deterministic_across_runs(name):
     for key in ("logits", "topk_idx", "topk_gate", "slot_row", "out", "dx", "dw1", "dw2",
                 "dw_router"):
         assert torch.equal(getattr(a, key), getattr(b, key)), key
+
+
+def _stats_close(dev, want):
+    """fp32 entries rounded once from exact integers / double sums."""
+    want = np.asarray(want, dtype=np.float64)
+    got = dev.double().cpu().numpy()
+    assert np.allclose(got, want, rtol=2e-7, atol=0), (got, want)
+
+
+@pytest.mark.parametrize("name,cap", [("bf16_skew_small", 40), ("bf16_skew_small", None),
+                                      ("bf16_e128_small", 25), ("f32_e128", None),
+                                      ("f32_one_token", 1)])
+def test_routing_stats_of_the_layer(name, cap):
+    cfg = CASES[name]
+    cpu, L = run_layer(cfg)
+    o = oracle_for(cpu, L)
+    st = L.routing_stats(capacity=cap)
+    torch.cuda.synchronize()
+    _stats_close(st, ref.routing_stats(o["counts"], cap or 0))
+
+
+def test_routing_stats_edge_counts():
+    from mixture_experts_layer_offsets_b200 import capi
+    out = torch.full((8,), -1.0, device="cuda")
+    cases = [
+        (np.zeros(7, np.int64), 3),                             # no rows at all
+        (np.array([5]), 2),                                     # one expert
+        (np.r_[np.full(1023, 0), [1 << 30]], 1 << 20),          # E = 1024, one huge expert
+        (np.random.default_rng(1).integers(0, 5000, 1024), 0),  # no capacity
+        (np.arange(1, 301), 150),
+    ]
+    for c, cap in cases:
+        s = capi.shape_of(64, 64, len(c), 1, 64)
+        dev = torch.tensor(c, dtype=torch.int32, device="cuda")
+        capi.moe_routing_stats(s, dev, cap, out)
+        torch.cuda.synchronize()
+        _stats_close(out, ref.routing_stats(c, cap))

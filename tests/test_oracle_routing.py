@@ -121,3 +121,35 @@ def test_select_logits_drive_discrete_steps_only():
     r = ref.route_from_logits(l, 2, select_logits=sel)
     assert np.all(r["idx"][:, 0] == 0)
     np.testing.assert_allclose(r["gate"][:, 0], ref.softmax(l)[:, 0])
+
+
+# ---- routing_stats: closed forms of special cases ---------------------------
+
+def test_routing_stats_uniform_and_one_hot():
+    st = ref.routing_stats([5, 5, 5, 5], C=5)
+    assert list(st) == [20, 5, 1, 1, 0, 0, 0, 1]
+    st = ref.routing_stats([12, 0, 0, 0], C=4)          # everything on one expert
+    assert np.allclose(st, [12, 3, 4, 0, np.sqrt(3), 3, 8 / 12, 4 / 16], rtol=1e-15, atol=0)
+    assert list(ref.routing_stats([0, 0, 0])) == [0, 0, 0, 0, 0, 3, 0, 0]
+
+
+def test_routing_stats_two_values():
+    # half the experts hold a rows, half b rows: cv = |a - b| / (a + b)
+    a, b, E = 7, 1, 6
+    st = ref.routing_stats([a, b] * (E // 2), C=3)
+    mean = (a + b) / 2
+    assert np.isclose(st[4], abs(a - b) / (a + b))
+    assert np.isclose(st[2], a / mean) and np.isclose(st[3], b / mean)
+    assert np.isclose(st[6], (E // 2) * (a - 3) / ((a + b) * E // 2))
+
+
+def test_routing_stats_of_a_real_routing_matches_its_padded_layout():
+    rng = np.random.default_rng(3)
+    T, E, k = 200, 8, 2
+    l = rng.normal(size=(T, E)) + np.linspace(0, 3, E)      # skewed
+    r = ref.route_from_logits(l, k)
+    C = ref.capacity(T * k, E)
+    st = ref.routing_stats(r["counts"], C)
+    pad = ref.padded_layout(r["idx"], r["slot_row"], r["offsets"], C)
+    assert np.isclose(st[6], np.mean(pad < 0))                # dropped pairs
+    assert np.isclose(st[7], np.sum(pad >= 0) / (E * C))      # used slots
