@@ -318,6 +318,22 @@ moe_status moe_padded_dispatch(moe_shape shape, int dtype, int32_t capacity, con
 moe_status moe_routing_stats(moe_shape shape, const int32_t* counts, int32_t capacity,
                              float* stats, void* stream);
 
+/* ---- f4: renormalised gates (an optional gate rule) ----------------------
+ * The pages fix no gate rule; moe_route's gates are the softmax values of the
+ * selected experts as they are.  These two calls offer the other usual rule,
+ * the selected values rescaled to sum to one over each token's k experts:
+ *   S[t] = sum_j topk_gate[t,j] (in index order),  gate_out[t,j] = topk_gate[t,j] / S[t]
+ * Use gate_out in place of topk_gate in moe_combine and moe_combine_bwd; the
+ * gate gradient that moe_combine_bwd then writes (dgate_out) goes through
+ *   dgate[t,j] = (dgate_out[t,j] - sum_i gate_out[t,i] dgate_out[t,i]) / S[t]
+ * before moe_route_bwd, which takes dgate.  topk_gate is the un-renormalised
+ * output of moe_route (fp32 [T,k]); gate_out, dgate_out, dgate: fp32 [T,k].
+ * gate_out may be topk_gate itself (in place) only when no backward follows;
+ * dgate may be dgate_out.  T == 0 is a no-op. */
+moe_status moe_renorm_gates(moe_shape shape, const float* topk_gate, float* gate_out, void* stream);
+moe_status moe_renorm_gates_bwd(moe_shape shape, const float* topk_gate, const float* dgate_out,
+                                float* dgate, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

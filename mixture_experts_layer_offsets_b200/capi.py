@@ -60,6 +60,8 @@ _SIGS = {
     "moe_mx_quantize_weights": (_I, [moe_shape, _P, _P, _P, _P]),
     "moe_padded_dispatch": (_I, [moe_shape, _I, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_routing_stats": (_I, [moe_shape, _P, ctypes.c_int32, _P, _P]),
+    "moe_renorm_gates": (_I, [moe_shape, _P, _P, _P]),
+    "moe_renorm_gates_bwd": (_I, [moe_shape, _P, _P, _P, _P]),
 }
 
 _lib = None
@@ -208,3 +210,13 @@ def moe_padded_dispatch(shape, dtype, capacity, x, topk_idx, slot_row, offsets, 
 def moe_routing_stats(shape, counts, capacity, stats, stream=None) -> None:
     _check("moe_routing_stats", lib().moe_routing_stats(
         shape, _ptr(counts), capacity, _ptr(stats), _stream(stream)))
+
+
+def moe_renorm_gates(shape, topk_gate, gate_out, stream=None) -> None:
+    _check("moe_renorm_gates", lib().moe_renorm_gates(
+        shape, _ptr(topk_gate), _ptr(gate_out), _stream(stream)))
+
+
+def moe_renorm_gates_bwd(shape, topk_gate, dgate_out, dgate, stream=None) -> None:
+    _check("moe_renorm_gates_bwd", lib().moe_renorm_gates_bwd(
+        shape, _ptr(topk_gate), _ptr(dgate_out), _ptr(dgate), _stream(stream)))

@@ -297,4 +297,20 @@ moe_status moe_routing_stats(moe_shape s, const int32_t* counts, int32_t capacit
   return cuda_status(routing_stats_launch(counts, s.E, capacity, stats, as_stream(stream)));
 }
 
+moe_status moe_renorm_gates(moe_shape s, const float* topk_gate, float* gate_out, void* stream) {
+  moe_status st = shape_ok(s);
+  if (st != MOE_OK) return st;
+  if (s.T > 0 && !ptrs_ok(topk_gate, gate_out)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(renorm_gates_launch(topk_gate, gate_out, s.T, s.top_k, as_stream(stream)));
+}
+
+moe_status moe_renorm_gates_bwd(moe_shape s, const float* topk_gate, const float* dgate_out,
+                                float* dgate, void* stream) {
+  moe_status st = shape_ok(s);
+  if (st != MOE_OK) return st;
+  if (s.T > 0 && !ptrs_ok(topk_gate, dgate_out, dgate)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(renorm_gates_bwd_launch(topk_gate, dgate_out, dgate, s.T, s.top_k,
+                                             as_stream(stream)));
+}
+
 }  // extern "C"

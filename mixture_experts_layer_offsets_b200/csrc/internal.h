@@ -37,6 +37,10 @@ bool route_tc_supported(int E, int k, int d);
 cudaError_t route_tc_launch(const RouteArgs& a, int nb, cudaStream_t st);
 
 // ---------------------------------------------------------- row movement
+//   renorm_gates_launch / renorm_gates_bwd_launch: moe_renorm_gates and its backward (k <= 32)
+cudaError_t renorm_gates_launch(const float* gate, float* out, int T, int k, cudaStream_t st);
+cudaError_t renorm_gates_bwd_launch(const float* gate, const float* dgr, float* dgate, int T, int k,
+                                    cudaStream_t st);
 //   routing_stats_launch: the eight load statistics of moe_routing_stats (E <= 1024)
 cudaError_t routing_stats_launch(const int32_t* counts, int E, int capacity, float* stats,
                                  cudaStream_t st);

@@ -398,6 +398,59 @@ cudaError_t routing_stats_launch(const int32_t* counts, int E, int capacity, flo
   return cudaGetLastError();
 }
 
+
+// ---- renormalised gates (optional gate rule) -----------------------------
+// g'[t, j] = g[t, j] / S[t], S[t] = sum_j g[t, j]; backward
+// dg[t, j] = (dg'[t, j] - sum_i g'[t, i] dg'[t, i]) / S[t].  One thread per
+// token; the k gates of a token are summed in index order.
+namespace {
+
+__global__ void __launch_bounds__(256) renorm_gates_kernel(const float* __restrict__ gate,
+                                                           float* __restrict__ out, int T, int k) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  const float* g = gate + (int64_t)t * k;
+  float S = 0.f;
+  for (int j = 0; j < k; ++j) S += g[j];
+  float v[32];
+  for (int j = 0; j < k; ++j) v[j] = g[j] / S;
+  float* o = out + (int64_t)t * k;
+  for (int j = 0; j < k; ++j) o[j] = v[j];
+}
+
+__global__ void __launch_bounds__(256) renorm_gates_bwd_kernel(const float* __restrict__ gate,
+                                                               const float* __restrict__ dgr,
+                                                               float* __restrict__ dgate, int T,
+                                                               int k) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  const float* g = gate + (int64_t)t * k;
+  const float* dg = dgr + (int64_t)t * k;
+  float S = 0.f;
+  for (int j = 0; j < k; ++j) S += g[j];
+  float dot = 0.f;
+  for (int j = 0; j < k; ++j) dot += (g[j] / S) * dg[j];
+  float v[32];
+  for (int j = 0; j < k; ++j) v[j] = (dg[j] - dot) / S;
+  float* o = dgate + (int64_t)t * k;
+  for (int j = 0; j < k; ++j) o[j] = v[j];
+}
+
+}  // namespace
+
+cudaError_t renorm_gates_launch(const float* gate, float* out, int T, int k, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  renorm_gates_kernel<<<(T + 255) / 256, 256, 0, st>>>(gate, out, T, k);
+  return cudaGetLastError();
+}
+
+cudaError_t renorm_gates_bwd_launch(const float* gate, const float* dgr, float* dgate, int T, int k,
+                                    cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  renorm_gates_bwd_kernel<<<(T + 255) / 256, 256, 0, st>>>(gate, dgr, dgate, T, k);
+  return cudaGetLastError();
+}
+
 }  // namespace moe
 
 // ---------------------------------------------------------------------------

@@ -31,7 +31,8 @@ def capacity_for(rows: int, E: int, cf_num: int = 5, cf_den: int = 4) -> int:
 
 class MoELayer:
     def __init__(self, T: int, d_model: int, E: int, top_k: int, d_ff: int, dtype: str = "bf16",
-                 device="cuda", dw_dtype: str | None = None, capacity: int | None = None):
+                 device="cuda", dw_dtype: str | None = None, capacity: int | None = None,
+                 renorm: bool = False):
         if dtype not in _DT:
             raise ValueError(f"dtype {dtype!r} is not supported by the layer path")
         self.T, self.d, self.E, self.k, self.f = T, d_model, E, top_k, d_ff
@@ -45,6 +46,7 @@ class MoELayer:
         if dtype == "mxfp8" and capacity:
             raise ValueError("the padded layout is not offered with MXFP8")
         self.capacity = capacity
+        self.renorm = renorm
         self.shape = capi.shape_of(T, d_model, E, top_k, d_ff)
         self.R = T * top_k
         self.rows = E * capacity if capacity else self.R
@@ -74,6 +76,9 @@ class MoELayer:
         self.dx = torch.empty(T, d_model, **act)
         self.dw_router = torch.empty(E, d_model, **f32)
         self.stats = torch.zeros(8, **f32)
+        if renorm:  # the combine's gates and their gradient under the renormalised rule
+            self.gate_rn = torch.empty(T, top_k, **f32)
+            self.dgate_rn = torch.empty(T, top_k, **f32)
         if capacity:
             self.pad_row = torch.empty(T, top_k, **i32)
             self.offsets_pad = torch.empty(E + 1, **i32)
@@ -103,6 +108,10 @@ class MoELayer:
         return self.pad_row if self.capacity else self.slot_row
 
     @property
+    def combine_gate(self):
+        return self.gate_rn if self.renorm else self.topk_gate
+
+    @property
     def ffn_offsets(self):
         return self.offsets_pad if self.capacity else self.offsets
 
@@ -125,13 +134,17 @@ class MoELayer:
             capi.moe_permute(s, dt, x, self.slot_row, self.x_perm, self.perm_src, stream)
         capi.moe_grouped_ffn_fwd(s, self.ffn_dtype, self.rows, self.x_perm, self.ffn_offsets, w1,
                                  w2, self.act, self.y_perm, self.ws, mx=self.mx, stream=stream)
-        capi.moe_combine(s, dt, self.y_perm, self.row_map, self.topk_gate, self.out, stream)
+        if self.renorm:
+            capi.moe_renorm_gates(s, self.topk_gate, self.gate_rn, stream)
+        capi.moe_combine(s, dt, self.y_perm, self.row_map, self.combine_gate, self.out, stream)
         return self.out
 
     def backward(self, dout, x, w_router, w1, w2, stream=None):
         s, dt = self.shape, self.cdtype
-        capi.moe_combine_bwd(s, dt, dout, self.y_perm, self.row_map, self.topk_gate,
-                             self.dy_perm, self.dgate, stream)
+        capi.moe_combine_bwd(s, dt, dout, self.y_perm, self.row_map, self.combine_gate,
+                             self.dy_perm, self.dgate_rn if self.renorm else self.dgate, stream)
+        if self.renorm:
+            capi.moe_renorm_gates_bwd(s, self.topk_gate, self.dgate_rn, self.dgate, stream)
         capi.moe_grouped_ffn_bwd(s, self.ffn_dtype, self.rows, self.dy_perm, self.x_perm,
                                  self.act, self.ffn_offsets, w1, w2, self.dx_perm, self.dw1,
                                  self.dw2, _DT[self.dw_dtype], self.ws, mx=self.mx, stream=stream)

@@ -23,7 +23,8 @@ __all__ = [
     "slot_rows", "perm_src_from_slots", "route", "route_from_logits",
     "permute", "sigmoid", "silu", "expert_ffn_fwd", "combine", "combine_bwd",
     "expert_ffn_bwd", "route_bwd", "layer_fwd_bwd", "capacity",
-    "padded_layout", "padded_layer_fwd_bwd", "routing_stats",
+    "padded_layout", "padded_layer_fwd_bwd", "routing_stats", "renorm_gates",
+    "renorm_gates_bwd",
 ]
 
 
@@ -245,6 +246,29 @@ def combine_bwd(dout, y_perm, slot, gate):
     return dgate, dy_perm
 
 
+def renorm_gates(gate) -> np.ndarray:
+    """Optional gate rule: the k selected probabilities rescaled to sum to one,
+    ``g'[t, j] = g[t, j] / S[t]`` with ``S[t] = sum_j g[t, j]``.
+
+    Reading: the pages fix no gate rule (the default keeps the softmax values as
+    they are); renormalising over the selected experts is offered as an option
+    beside the routing-balance statistics (kongchang, routing section).
+    """
+    g = _f64(gate)
+    return g / g.sum(axis=1, keepdims=True)
+
+
+def renorm_gates_bwd(gate, dgate_rn) -> np.ndarray:
+    """Gradient of ``renorm_gates`` with respect to the selected probabilities:
+    ``dg[t, j] = (dg'[t, j] - sum_i g'[t, i] dg'[t, i]) / S[t]``, from
+    ``d g'_i / d g_j = (delta_ij - g'_i) / S``."""
+    g = _f64(gate)
+    S = g.sum(axis=1, keepdims=True)
+    gr = g / S
+    dgr = _f64(dgate_rn)
+    return (dgr - np.sum(gr * dgr, axis=1, keepdims=True)) / S
+
+
 def expert_ffn_bwd(dy_perm, x_perm, a, u, h, offsets, w1, w2):
     """Backward of ``expert_ffn_fwd``: grouped dgrad and wgrad.
 
@@ -306,22 +330,27 @@ def route_bwd(x, w_router, logits, idx, dgate, dx_perm, slot):
 
 
 def layer_fwd_bwd(x, w_router, w1, w2, dout, k: int, bias=None,
-                  select_logits=None) -> dict:
+                  select_logits=None, renorm: bool = False) -> dict:
     """One forward + backward pass of the whole layer, all intermediates.
 
     route -> permute -> grouped SwiGLU FFN -> combine; then combine-grad ->
     grouped dgrad/wgrad -> unpermute-grad + router grad.  ``select_logits``
-    is passed to ``route`` (see ``route_from_logits``).
+    is passed to ``route`` (see ``route_from_logits``).  With ``renorm`` the
+    combine takes ``renorm_gates`` of the gates; ``dgate_rn`` is then the
+    combine's gate gradient and ``dgate`` its image under ``renorm_gates_bwd``.
     """
     r = route(x, w_router, k, bias, select_logits)
     x_perm = permute(x, r["slot_row"])
     a, u, h, y_perm = expert_ffn_fwd(x_perm, r["offsets"], w1, w2)
-    out = combine(y_perm, r["slot_row"], r["gate"])
-    dgate, dy_perm = combine_bwd(dout, y_perm, r["slot_row"], r["gate"])
+    gate = renorm_gates(r["gate"]) if renorm else r["gate"]
+    out = combine(y_perm, r["slot_row"], gate)
+    dgate_c, dy_perm = combine_bwd(dout, y_perm, r["slot_row"], gate)
+    dgate = renorm_gates_bwd(r["gate"], dgate_c) if renorm else dgate_c
     dx_perm, dw1, dw2 = expert_ffn_bwd(dy_perm, x_perm, a, u, h, r["offsets"], w1, w2)
     dx, dw_router, dl = route_bwd(x, w_router, r["logits"], r["idx"], dgate, dx_perm,
                                   r["slot_row"])
     r.update(x_perm=x_perm, a=a, u=u, h=h, y_perm=y_perm, out=out, dgate=dgate,
+             gate_rn=gate, dgate_rn=dgate_c,
              dy_perm=dy_perm, dx_perm=dx_perm, dw1=dw1, dw2=dw2, dx=dx,
              dw_router=dw_router, dl=dl)
     return r
@@ -355,12 +384,13 @@ def padded_layout(idx, slot, offsets, C: int):
 
 
 def padded_layer_fwd_bwd(x, w_router, w1, w2, dout, k: int, C: int, bias=None,
-                         select_logits=None) -> dict:
+                         select_logits=None, renorm: bool = False) -> dict:
     """Forward + backward of the layer on the padded-capacity layout.
 
     Dropped pairs contribute nothing to ``out`` and get zero gradient; the gates
-    are not renormalised.  Unused padded rows are zero, so they produce zero
-    expert outputs and zero weight gradients.
+    are not renormalised after the drop (with ``renorm`` they are renormalised
+    over all k selected experts before it).  Unused padded rows are zero, so
+    they produce zero expert outputs and zero weight gradients.
     """
     x = _f64(x)
     r = route(x, w_router, k, bias, select_logits)
@@ -376,7 +406,7 @@ def padded_layer_fwd_bwd(x, w_router, w1, w2, dout, k: int, C: int, bias=None,
     out = np.zeros((T, d))
     dgate = np.zeros((T, k))
     dy_pad = np.zeros_like(y_pad)
-    gate = r["gate"]
+    gate = renorm_gates(r["gate"]) if renorm else r["gate"]
     dout = _f64(dout)
     for j in range(k):
         kj = keep[:, j]
@@ -391,10 +421,13 @@ def padded_layer_fwd_bwd(x, w_router, w1, w2, dout, k: int, C: int, bias=None,
     for j in range(k):
         kj = keep[:, j]
         dx_perm_like[r["slot_row"][kj, j]] = dx_pad[prow[kj, j]]
+    dgate_c = dgate
+    if renorm:
+        dgate = renorm_gates_bwd(r["gate"], dgate_c)
     dx, dw_router, dl = route_bwd(x, w_router, r["logits"], r["idx"], dgate,
                                   dx_perm_like, r["slot_row"])
     r.update(C=C, pad_row=prow, x_pad=x_pad, a=a, u=u, h=h, y_pad=y_pad, out=out,
-             dgate=dgate, dy_pad=dy_pad, dx_pad=dx_pad, dw1=dw1, dw2=dw2, dx=dx,
+             dgate=dgate, gate_rn=gate, dgate_rn=dgate_c, dy_pad=dy_pad, dx_pad=dx_pad, dw1=dw1, dw2=dw2, dx=dx,
              dw_router=dw_router, dl=dl)
     return r
 

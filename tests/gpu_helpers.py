@@ -30,12 +30,12 @@ def rel(a, b) -> float:
     return float(np.linalg.norm(a - b) / (nb if nb > 0 else 1.0))
 
 
-def run_layer(cfg, seed=0, capacity=None, dw_dtype="f32"):
+def run_layer(cfg, seed=0, capacity=None, dw_dtype="f32", renorm=False):
     """Seeded inputs drawn on the CPU, copied to the GPU, one fwd+bwd step."""
     cpu = inputs.make_inputs(cfg, device="cpu", seed=seed)
     dev = {k: (v.cuda() if v is not None else None) for k, v in cpu.items()}
     L = MoELayer(cfg.T, cfg.d_model, cfg.E, cfg.top_k, cfg.d_ff, cfg.dtype, "cuda",
-                 dw_dtype=dw_dtype, capacity=capacity)
+                 dw_dtype=dw_dtype, capacity=capacity, renorm=renorm)
     L.step(dev["x"], dev["w_router"], dev["bias"], dev["w1"], dev["w2"], dev["dout"])
     torch.cuda.synchronize()
     assert L.device_status() == 0
@@ -48,5 +48,6 @@ def oracle_for(cpu, L, capacity=None):
             L.k)
     bias = f64(cpu["bias"]) if cpu["bias"] is not None else None
     if capacity:
-        return ref.padded_layer_fwd_bwd(*args, capacity, bias, select_logits=f64(L.logits))
-    return ref.layer_fwd_bwd(*args, bias, select_logits=f64(L.logits))
+        return ref.padded_layer_fwd_bwd(*args, capacity, bias, select_logits=f64(L.logits),
+                                        renorm=L.renorm)
+    return ref.layer_fwd_bwd(*args, bias, select_logits=f64(L.logits), renorm=L.renorm)

@@ -119,6 +119,9 @@ def test_row_ops_validation(lib):
     assert lib.moe_routing_stats(s, FAKE, -1, FAKE, None) == capi.MOE_ERR_INVALID_ARG
     assert lib.moe_routing_stats(s, None, 0, FAKE, None) == capi.MOE_ERR_INVALID_ARG
     assert lib.moe_routing_stats(_shape(E=2048), FAKE, 0, FAKE, None) == capi.MOE_ERR_INVALID_ARG
+    assert lib.moe_renorm_gates(s, FAKE + 4, FAKE, None) == capi.MOE_ERR_INVALID_ARG
+    assert lib.moe_renorm_gates_bwd(s, FAKE, None, FAKE, None) == capi.MOE_ERR_INVALID_ARG
+    assert lib.moe_renorm_gates(_shape(T=0), None, None, None) == capi.MOE_OK
     # T == 0 is a valid no-op for the row movers
     assert lib.moe_permute(_shape(T=0), capi.MOE_BF16, None, None, None, None, None) == capi.MOE_OK
 

@@ -163,3 +163,43 @@ def test_routing_stats_edge_counts():
         capi.moe_routing_stats(s, dev, cap, out)
         torch.cuda.synchronize()
         _stats_close(out, ref.routing_stats(c, cap))
+
+
+@pytest.mark.parametrize("name,cap", [("bf16_skew_small", None), ("tiny_f32", None),
+                                      ("bf16_e128_small", None), ("bf16_skew_small", 40),
+                                      ("f32_one_token", None)])
+def test_renormalised_gates_match_oracle(name, cap):
+    cfg = CASES[name]
+    tol = TOL[cfg.dtype]
+    cpu, L = run_layer(cfg, capacity=cap, renorm=True)
+    o = oracle_for(cpu, L, capacity=cap)
+    _check_routing(L, o)
+    # the renormalisation itself runs in fp32 on fp32 gates
+    assert rel(f64(L.gate_rn), o["gate_rn"]) <= TOL["f32"]
+    assert np.allclose(f64(L.gate_rn).sum(axis=1), 1.0, rtol=1e-6)
+    checks = {"out": (L.out, o["out"]), "dgate_rn": (L.dgate_rn, o["dgate_rn"]),
+              "dgate": (L.dgate, o["dgate"]), "dx": (L.dx, o["dx"]),
+              "dw_router": (L.dw_router, o["dw_router"]), "dw1": (L.dw1, o["dw1"]),
+              "dw2": (L.dw2, o["dw2"])}
+    errs = {k: rel(f64(a), b) for k, (a, b) in checks.items()}
+    assert all(v <= tol for v in errs.values()), (name, errs)
+
+
+def test_renorm_kernels_match_oracle_directly():
+    from mixture_experts_layer_offsets_b200 import capi
+    rng = np.random.default_rng(7)
+    for T, k in [(1, 1), (333, 3), (1000, 8), (77, 32)]:
+        g = rng.uniform(1e-4, 1.0, size=(T, k)).astype(np.float32)
+        dg = rng.normal(size=(T, k)).astype(np.float32)
+        s = capi.shape_of(T, 64, max(k, 2), k, 64)
+        gd = torch.from_numpy(g).cuda()
+        dgd = torch.from_numpy(dg).cuda()
+        out = torch.empty_like(gd)
+        dout = torch.empty_like(gd)
+        capi.moe_renorm_gates(s, gd, out)
+        capi.moe_renorm_gates_bwd(s, gd, dgd, dout)
+        torch.cuda.synchronize()
+        want = ref.renorm_gates(g.astype(np.float64))
+        assert np.allclose(f64(out), want, rtol=1e-6, atol=0)
+        wb = ref.renorm_gates_bwd(g.astype(np.float64), dg.astype(np.float64))
+        assert rel(f64(dout), wb) <= 1e-6

@@ -191,3 +191,72 @@ def test_padded_gradients_match_finite_differences():
             arr[ix] = o
             fd[ix] = (lp - lm) / (2 * eps)
         assert np.linalg.norm(fd - g) / np.linalg.norm(g) < 1e-6
+
+
+# ---- renormalised gates (optional gate rule) --------------------------------
+
+def _softmax_of_selected(l, idx):
+    """Gates as a softmax over the k selected logits only, written out directly."""
+    sel = np.take_along_axis(l, idx, axis=1)
+    z = np.exp(sel - sel.max(axis=1, keepdims=True))
+    return z / z.sum(axis=1, keepdims=True)
+
+
+def test_renorm_gates_are_a_softmax_over_the_selected_logits():
+    x, wr, b, *_ = _tiny(seed=4, T=20, E=6, bias=True)
+    r = ref.route(x, wr, 3, b)
+    got = ref.renorm_gates(r["gate"])
+    assert np.allclose(got, _softmax_of_selected(r["logits"], r["idx"]), rtol=1e-14, atol=0)
+    assert np.allclose(got.sum(axis=1), 1.0, rtol=1e-15)
+
+
+def _loss_renorm(params, k, bias):
+    x, wr, w1, w2, dout = params
+    r = ref.route(x, wr, k, bias)
+    _, _, _, y = ref.expert_ffn_fwd(ref.permute(x, r["slot_row"]), r["offsets"], w1, w2)
+    g = _softmax_of_selected(r["logits"], r["idx"])
+    return float(np.sum(ref.combine(y, r["slot_row"], g) * dout))
+
+
+def test_renorm_gradients_match_finite_differences():
+    x, wr, b, w1, w2, dout = _tiny(seed=11, bias=True)
+    k = 2
+    assert _min_gap(x, wr, b, k) > 1e-3
+    res = ref.layer_fwd_bwd(x, wr, w1, w2, dout, k, b, renorm=True)
+    assert np.allclose(res["out"].sum(), _loss_renorm([x, wr, w1, w2, np.ones_like(dout)], k, b))
+    params = [x, wr, w1, w2, dout]
+    eps = 1e-6
+    for pi, g in {0: res["dx"], 1: res["dw_router"]}.items():
+        fd = np.zeros_like(params[pi])
+        it = np.nditer(params[pi], flags=["multi_index"])
+        for _ in it:
+            ix = it.multi_index
+            orig = params[pi][ix]
+            params[pi][ix] = orig + eps
+            lp = _loss_renorm(params, k, b)
+            params[pi][ix] = orig - eps
+            lm = _loss_renorm(params, k, b)
+            params[pi][ix] = orig
+            fd[ix] = (lp - lm) / (2 * eps)
+        err = np.linalg.norm(fd - g) / np.linalg.norm(g)
+        assert err < 1e-6, (pi, err)
+    # the renormalised gates change the router gradient (the option is not a no-op)
+    plain = ref.layer_fwd_bwd(x, wr, w1, w2, dout, k, b)
+    assert np.linalg.norm(plain["dw_router"] - res["dw_router"]) > 1e-3 * np.linalg.norm(plain["dw_router"])
+
+
+def test_renorm_changes_nothing_when_top_k_equals_E():
+    # all experts selected: the softmax values already sum to one
+    x, wr, b, w1, w2, dout = _tiny(seed=5, E=4)
+    a = ref.layer_fwd_bwd(x, wr, w1, w2, dout, 4, b)
+    r = ref.layer_fwd_bwd(x, wr, w1, w2, dout, 4, b, renorm=True)
+    for key in ("out", "dx", "dw_router", "dw1", "dw2"):
+        assert np.allclose(a[key], r[key], rtol=1e-12, atol=1e-13), key
+
+
+def test_padded_renorm_equals_dropless_renorm_when_nothing_drops():
+    x, wr, b, w1, w2, dout = _tiny(seed=6, T=10, E=4, bias=True)
+    full = ref.layer_fwd_bwd(x, wr, w1, w2, dout, 2, b, renorm=True)
+    pad = ref.padded_layer_fwd_bwd(x, wr, w1, w2, dout, 2, 20, b, renorm=True)
+    for key in ("out", "dgate", "dx", "dw_router", "dw1", "dw2"):
+        assert np.allclose(full[key], pad[key], rtol=1e-12, atol=1e-13), key
