@@ -43,11 +43,23 @@ from mixture_experts_layer_offsets_b200 import inputs  # noqa: E402
 
 METRIC = "MoE FFN fwd+bwd tokens/s on 1 B200; grouped-GEMM % of tensor-core peak"
 FLUSH_BYTES = 256 << 20
-# kernel launches of one step, per C-ABI call (bf16 path; MXFP8 adds the operand
-# quantisations: 4 for the weight copies, 2 in the forward FFN call, 6 in the backward)
-LAUNCHES = {"route": 3, "permute": 1, "ffn_fwd": 2, "combine": 1, "combine_bwd": 1,
-            "ffn_bwd": 4, "route_bwd": 4, "padded_dispatch": 2}
-LAUNCHES_MX = {"quantize_w": 4, "ffn_fwd": 4, "ffn_bwd": 10}
+def launches_per_step(cfg, capacity, recompute, fused_dispatch) -> int:
+    """Kernel launches of this library in one step, counted per C-ABI call from the
+    launch sequences in csrc (and checked against ncu launch lists)."""
+    mx, f32 = cfg.dtype == "mxfp8", cfg.dtype == "f32"
+    tc_router_bwd = not f32 and cfg.E % 128 == 0 and cfg.top_k <= 8 and cfg.d_model % 256 == 0
+    n = 2 if mx else 0                                   # the two weight quantisers
+    n += 3                                               # router, block scan, slot rows
+    n += 2 if capacity else (4 if fused_dispatch else 1)  # dispatch
+    n += (3 if fused_dispatch else 6) if mx else (3 if f32 else 2)   # forward FFN
+    n += 1 + 1                                           # combine, combine backward
+    n += 8 if mx else (5 if f32 else 6)                  # backward FFN
+    n += 5 if tc_router_bwd else 4                       # router backward
+    if recompute:                                        # the gate/up half again
+        n += 5 if mx else (2 if f32 else 1)
+    return n
+
+
 FP8_OVER_BF16 = 2.0   # nominal dense tensor-core ratio (4.5 / 2.25 PFLOP/s)
 # DRAM bytes (read + write) of the six grouped-GEMM launches of one step, from one ncu capture
 # of this build (profiles/launches_bf16_e8.md); None where no capture of the current kernels
@@ -64,7 +76,7 @@ def _peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def _workload_desc(cfg, capacity):
+def _workload_desc(cfg, capacity, recompute=False):
     d = {"workload": f"{cfg.name}: T={cfg.T} d_model={cfg.d_model} E={cfg.E} top_k={cfg.top_k} "
                      f"d_ff={cfg.d_ff} {cfg.dtype}",
          "T": cfg.T, "d_model": cfg.d_model, "E": cfg.E, "top_k": cfg.top_k, "d_ff": cfg.d_ff,
@@ -75,6 +87,8 @@ def _workload_desc(cfg, capacity):
         d["operands"] = ("MXFP8 (E4M3 + E8M0 per 32 along K) for all six expert GEMMs; bf16 "
                          "activations; FP32 master weights quantised to four MXFP8 copies "
                          "every step (inside the timed step)")
+    if recompute:
+        d["recompute"] = "gate/up GEMM re-run in the backward (a | u | h not kept from the forward)"
     if capacity:
         d["layout"] = f"padded capacity C={capacity} (overflow dropped)"
     else:
@@ -148,7 +162,7 @@ def run_ours(args, rank, world):
     capacity = capacity_for(cfg.R, cfg.E, *cfg.padded_cf) if args.capacity_factor and cfg.padded_cf else None
     inp = inputs.make_inputs(cfg, device=dev, seed=mdist.rank_seed(0, rank))
     L = MoELayer(cfg.T, cfg.d_model, cfg.E, cfg.top_k, cfg.d_ff, cfg.dtype, dev,
-                 dw_dtype="f32", capacity=capacity)
+                 dw_dtype="f32", capacity=capacity, recompute=args.recompute)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     x, wr, b, w1, w2, dout = (inp[k] for k in ("x", "w_router", "bias", "w1", "w2", "dout"))
@@ -173,7 +187,10 @@ def run_ours(args, rank, world):
             capi.moe_padded_dispatch(s, dt, capacity, x, L.topk_idx, L.slot_row, L.offsets,
                                      L.x_perm, L.pad_row, L.offsets_pad)
         else:
-            capi.moe_permute(s, dt, x, L.slot_row, L.x_perm, L.perm_src)
+            if L.fused_dispatch:
+                capi.moe_permute_mx(s, x, L.slot_row, L.offsets, L.perm_src, L.ws)
+            else:
+                capi.moe_permute(s, dt, x, L.slot_row, L.x_perm, L.perm_src)
         mark(3)
         capi.moe_grouped_ffn_fwd(s, fdt, L.rows, L.x_perm, L.ffn_offsets, w1, w2, L.act, L.y_perm,
                                  L.ws, mx=L.mx)
@@ -182,8 +199,9 @@ def run_ours(args, rank, world):
         mark(5)
         capi.moe_combine_bwd(s, dt, dout, L.y_perm, L.row_map, L.topk_gate, L.dy_perm, L.dgate)
         mark(6)
-        capi.moe_grouped_ffn_bwd(s, fdt, L.rows, L.dy_perm, L.x_perm, L.act, L.ffn_offsets, w1,
-                                 w2, L.dx_perm, L.dw1, L.dw2, capi.MOE_F32, L.ws, mx=L.mx)
+        bwd = capi.moe_grouped_ffn_bwd_recompute if args.recompute else capi.moe_grouped_ffn_bwd
+        bwd(s, fdt, L.rows, L.dy_perm, L.x_perm, L.act, L.ffn_offsets, w1, w2, L.dx_perm, L.dw1,
+            L.dw2, capi.MOE_F32, L.ws, mx=L.mx)
         mark(7)
         capi.moe_route_bwd(s, dt, x, wr, L.logits, L.topk_idx, L.dgate, L.dx_perm, L.row_map,
                            L.dx, L.dw_router, L.ws)
@@ -262,17 +280,13 @@ def run_ours(args, rank, world):
                      "the ffn phases include the activation quantisations")
     else:
         peak, peak_kind = None, "fp32 CUDA-core path: no tensor-core peak"
-    lt = dict(LAUNCHES, **(LAUNCHES_MX if mxfp8 else {"quantize_w": 0}))
-    launches_per_step = (lt["quantize_w"] + lt["route"]
-                         + (lt["padded_dispatch"] if capacity else lt["permute"])
-                         + lt["ffn_fwd"] + lt["combine"] + lt["combine_bwd"]
-                         + lt["ffn_bwd"] + lt["route_bwd"])
+    n_launch = launches_per_step(cfg, capacity, args.recompute, L.fused_dispatch)
     line = {
         "metric": METRIC, "value": round(tokens_per_s, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
         "data": "synthetic (seeded; random-init weights)",
-        "config": _workload_desc(cfg, capacity),
+        "config": _workload_desc(cfg, capacity, args.recompute),
         "roofline": {
             "bound": "tensor", "kernel": "grouped GEMM (tcgen05), all 6 launches of a step",
             "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
@@ -286,7 +300,7 @@ def run_ours(args, rank, world):
         "phases_ms": {k: round(v, 4) for k, v in ph.items()},
         "timing": "value: CUDA-graph replay of the step, CUDA events per step; phases_ms and "
                   "roofline: eager steps with events between calls (host kept ahead of the GPU)",
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": n_launch * args.steps,
         "device_status": status,
         "e2e": e2e,
         "clocks": clocks,
@@ -309,7 +323,8 @@ def run_e2e(args, L, inp, dev, flush, capacity, world):
     another; events order every copy against the compute that produces or reuses its
     buffers.  Working set per step is several times L2, so no flush is needed."""
     from mixture_experts_layer_offsets_b200.layer import MoELayer
-    L2 = MoELayer(L.T, L.d, L.E, L.k, L.f, L.dtype, dev, dw_dtype=L.dw_dtype, capacity=capacity)
+    L2 = MoELayer(L.T, L.d, L.E, L.k, L.f, L.dtype, dev, dw_dtype=L.dw_dtype, capacity=capacity,
+                  recompute=L.recompute)
     layers = [L, L2]
     hx = inp["x"].cpu().pin_memory()
     hd = inp["dout"].cpu().pin_memory()
@@ -438,6 +453,8 @@ def main():
     ap.add_argument("--workload", default="bf16_e8", choices=sorted(inputs.CONFIGS))
     ap.add_argument("--capacity-factor", action="store_true",
                     help="padded-capacity layout (workloads that define a capacity factor)")
+    ap.add_argument("--recompute", action="store_true",
+                    help="backward recomputes a | u | h (moe_grouped_ffn_bwd_recompute)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -192,6 +192,24 @@ typedef struct moe_mx_weights {
 moe_status moe_mx_quantize_weights(moe_shape shape, const float* w1, const float* w2,
                                    const moe_mx_weights* out, void* stream);
 
+/* ---- f1: MXFP8 dispatch (permute fused with the quantisation of x) --------
+ * [kongchang] boundary-conditions section: MXFP8 cuts the bytes the dispatch
+ * moves.  Instead of copying bf16 rows into x_perm for the MXFP8 grouped FFN to
+ * quantise, this call reads each routed row of x once where it lies and writes
+ * only the two MXFP8 copies the GEMMs use: along d (E4M3 rows, 1 byte per
+ * element + one E8M0 byte per 32) and in 32-row token blocks restarting at every
+ * expert (for the dW1 GEMM of the backward).  Both go to `ws`, with the row maps,
+ * where moe_grouped_ffn_fwd (dtype MOE_MXFP8, x_perm = NULL) reads them; no
+ * call may use `ws` in between.  The result is bit-identical to moe_permute
+ * followed by the forward's own quantisation.
+ * x: bf16 [T, d]; slot_row, offsets: from moe_route (dropless, rows = T*k);
+ * perm_src: int32 [T*k] written as in moe_permute (row r came from token
+ * perm_src[r]).  Needs d % 128 == 0 and f % 128 == 0 (else MOE_ERR_UNSUPPORTED);
+ * ws_bytes >= moe_workspace_size(shape, MOE_MXFP8, T*k). */
+moe_status moe_permute_mx(moe_shape shape, const void* x, const int32_t* slot_row,
+                          const int32_t* offsets, int32_t* perm_src, void* ws, size_t ws_bytes,
+                          void* stream);
+
 /* ---- a4: grouped SwiGLU FFN, forward -------------------------------------
  * [kongchang] routing section: a device-scheduled grouped GEMM handles the
  * uneven per-expert shapes; the tile scheduler reads `offsets` from device
@@ -210,7 +228,8 @@ moe_status moe_mx_quantize_weights(moe_shape shape, const float* w1, const float
  * read and may be NULL); x and h are quantised, in one pass each, along their rows
  * (for this call's GEMMs) and in 32-row token blocks (kept in `ws` for the backward), and
  * the GEMMs run block-scaled E4M3 x E4M3 with fp32 accumulation.  Needs d % 128 == 0 and
- * f % 128 == 0. */
+ * f % 128 == 0.  x_perm may be NULL when moe_permute_mx has just filled `ws` for the
+ * same offsets (the x quantisation is then skipped). */
 moe_status moe_grouped_ffn_fwd(moe_shape shape, int dtype, int64_t rows, const void* x_perm,
                                const int32_t* offsets, const void* w1, const void* w2,
                                const void* mx, void* act_saved, void* y_perm, void* ws,
@@ -248,12 +267,32 @@ moe_status moe_combine_bwd(moe_shape shape, int dtype, const void* dout, const v
  * [da | du], x in 32-row blocks restarting at every expert for the wgrad GEMMs.  The
  * token-block copies of x and h (and the row/block maps) are the ones the forward of the
  * same step wrote into `ws`: pass the same workspace, with no call using it in between
- * (moe_combine and moe_combine_bwd take none), and the same offsets. */
+ * (moe_combine and moe_combine_bwd take none), and the same offsets.  x_perm is not
+ * read and may be NULL. */
 moe_status moe_grouped_ffn_bwd(moe_shape shape, int dtype, int64_t rows, const void* dy_perm,
                                const void* x_perm, const void* act_saved,
                                const int32_t* offsets, const void* w1, const void* w2,
                                const void* mx, void* dx_perm, void* dw1, void* dw2,
                                int dw_dtype, void* ws, size_t ws_bytes, void* stream);
+
+/* ---- f3: grouped FFN backward with recompute ------------------------------
+ * [kongchang] boundary-conditions section: keeping only the layer input and
+ * recomputing the expert activations in the backward trades about a fifth of
+ * the throughput for two thirds of the activation memory.
+ * Same arguments and results as moe_grouped_ffn_bwd, except that act_scratch
+ * ([rows, 3f], same type as act_saved) need not hold anything: the call first
+ * recomputes a | u | h into it from x_perm with the gate/up GEMM of the
+ * forward (for MOE_MXFP8 also the token-block copies of x and h in `ws`, so the
+ * workspace may have served other calls since the forward), then runs the
+ * backward.  One act_scratch can serve every layer of a model.  act_scratch
+ * is overwritten; its contents afterwards are this layer's a | u | h.  x_perm
+ * is required here, for every dtype. */
+moe_status moe_grouped_ffn_bwd_recompute(moe_shape shape, int dtype, int64_t rows,
+                                         const void* dy_perm, const void* x_perm,
+                                         void* act_scratch, const int32_t* offsets,
+                                         const void* w1, const void* w2, const void* mx,
+                                         void* dx_perm, void* dw1, void* dw2, int dw_dtype,
+                                         void* ws, size_t ws_bytes, void* stream);
 
 /* ---- a9: unpermute-grad + router grad ------------------------------------
  *   dx[t,:]  = sum_{j, slot_row[t,j] >= 0} dx_perm[slot_row[t,j],:] + sum_e dl[t,e] w_router[e,:]

@@ -55,11 +55,14 @@ _SIGS = {
     "moe_combine_bwd": (_I, [moe_shape, _I, _P, _P, _P, _P, _P, _P, _P]),
     "moe_grouped_ffn_bwd": (_I, [moe_shape, _I, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                  _I, _P, _SZ, _P]),
+    "moe_grouped_ffn_bwd_recompute": (_I, [moe_shape, _I, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                 _I, _P, _SZ, _P]),
     "moe_route_bwd": (_I, [moe_shape, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "mxfp8_quantize": (_I, [_I64, _I64, _I, _P, _I, _P, _I, _P, _P, _P]),
     "moe_mx_quantize_weights": (_I, [moe_shape, _P, _P, _P, _P]),
     "moe_padded_dispatch": (_I, [moe_shape, _I, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_routing_stats": (_I, [moe_shape, _P, ctypes.c_int32, _P, _P]),
+    "moe_permute_mx": (_I, [moe_shape, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_renorm_gates": (_I, [moe_shape, _P, _P, _P]),
     "moe_renorm_gates_bwd": (_I, [moe_shape, _P, _P, _P, _P]),
 }
@@ -180,6 +183,15 @@ def moe_grouped_ffn_bwd(shape, dtype, rows, dy_perm, x_perm, act_saved, offsets,
         ws.numel() * ws.element_size(), _stream(stream)))
 
 
+def moe_grouped_ffn_bwd_recompute(shape, dtype, rows, dy_perm, x_perm, act_scratch, offsets, w1,
+                                  w2, dx_perm, dw1, dw2, dw_dtype, ws, mx=None,
+                                  stream=None) -> None:
+    _check("moe_grouped_ffn_bwd_recompute", lib().moe_grouped_ffn_bwd_recompute(
+        shape, dtype, rows, _ptr(dy_perm), _ptr(x_perm), _ptr(act_scratch), _ptr(offsets),
+        _ptr(w1), _ptr(w2), _ptr(mx), _ptr(dx_perm), _ptr(dw1), _ptr(dw2), dw_dtype, _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))
+
+
 def moe_route_bwd(shape, dtype, x, w_router, logits, topk_idx, dgate, dx_perm, slot_row, dx,
                   dw_router, ws, stream=None) -> None:
     _check("moe_route_bwd", lib().moe_route_bwd(
@@ -220,3 +232,9 @@ def moe_renorm_gates(shape, topk_gate, gate_out, stream=None) -> None:
 def moe_renorm_gates_bwd(shape, topk_gate, dgate_out, dgate, stream=None) -> None:
     _check("moe_renorm_gates_bwd", lib().moe_renorm_gates_bwd(
         shape, _ptr(topk_gate), _ptr(dgate_out), _ptr(dgate), _stream(stream)))
+
+
+def moe_permute_mx(shape, x, slot_row, offsets, perm_src, ws, stream=None) -> None:
+    _check("moe_permute_mx", lib().moe_permute_mx(
+        shape, _ptr(x), _ptr(slot_row), _ptr(offsets), _ptr(perm_src), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)))

@@ -127,6 +127,22 @@ moe_status moe_permute(moe_shape s, int dtype, const void* x, const int32_t* slo
                                     s.d_model, s.top_k, as_stream(stream)));
 }
 
+moe_status moe_permute_mx(moe_shape s, const void* x, const int32_t* slot_row,
+                          const int32_t* offsets, int32_t* perm_src, void* ws, size_t ws_bytes,
+                          void* stream) {
+  moe_status st = shape_ok(s);
+  if (st != MOE_OK) return st;
+  if (s.d_model % 128 || s.d_ff % 128) return MOE_ERR_UNSUPPORTED;
+  if (!ptrs_ok(offsets, ws)) return MOE_ERR_INVALID_ARG;
+  if (s.T > 0 && !ptrs_ok(x, slot_row, perm_src)) return MOE_ERR_INVALID_ARG;
+  FfnShape fs{s.d_model, s.E, s.d_ff, (int64_t)s.T * s.top_k};
+  if (ws_bytes < kStatusBytes + ffn_mx_ws_bytes(fs)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t cs = as_stream(stream);
+  cudaError_t e = perm_src_launch(slot_row, perm_src, s.T, s.top_k, cs);
+  if (e == cudaSuccess) e = mx_dispatch(fs, x, perm_src, offsets, scratch(ws), cs);
+  return cuda_status(e);
+}
+
 moe_status moe_grouped_ffn_fwd(moe_shape s, int dtype, int64_t rows, const void* x_perm,
                                const int32_t* offsets, const void* w1, const void* w2,
                                const void* mx, void* act_saved, void* y_perm, void* ws,
@@ -142,7 +158,9 @@ moe_status moe_grouped_ffn_fwd(moe_shape s, int dtype, int64_t rows, const void*
     if (vs != MOE_OK) return vs;
     if (s.d_model % 128 || s.d_ff % 128) return MOE_ERR_UNSUPPORTED;
     if (!ptrs_ok(offsets, ws)) return MOE_ERR_INVALID_ARG;
-    if (rows > 0 && !ptrs_ok(x_perm, act_saved, y_perm)) return MOE_ERR_INVALID_ARG;
+    // x_perm NULL: moe_permute_mx has put the quantised copies of x in ws
+    if (rows > 0 && (!ptrs_ok(act_saved, y_perm) || (x_perm && !aligned16(x_perm))))
+      return MOE_ERR_INVALID_ARG;
     if (ws_bytes < kStatusBytes + ffn_mx_ws_bytes(fs)) return MOE_ERR_INVALID_ARG;
     return cuda_status(ffn_fwd_mx(fs, x_perm, offsets, w, act_saved, y_perm, scratch(ws),
                                   status_word(ws), cs));
@@ -185,11 +203,17 @@ moe_status moe_combine_bwd(moe_shape s, int dtype, const void* dout, const void*
                                         as_stream(stream)));
 }
 
-moe_status moe_grouped_ffn_bwd(moe_shape s, int dtype, int64_t rows, const void* dy_perm,
-                               const void* x_perm, const void* act_saved,
-                               const int32_t* offsets, const void* w1, const void* w2,
-                               const void* mx, void* dx_perm, void* dw1, void* dw2,
-                               int dw_dtype, void* ws, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The grouped FFN backward; with `recompute` the call first refills act (a | u | h,
+// and for MXFP8 the token-block copies of x and h in ws) from x_perm.
+moe_status ffn_bwd_entry(moe_shape s, int dtype, int64_t rows, const void* dy_perm,
+                         const void* x_perm, void* act, const int32_t* offsets, const void* w1,
+                         const void* w2, const void* mx, void* dx_perm, void* dw1, void* dw2,
+                         int dw_dtype, void* ws, size_t ws_bytes, void* stream, bool recompute) {
+  const void* act_saved = act;
   moe_status st = shape_ok(s);
   if (st != MOE_OK) return st;
   if (rows < 0 || rows >= ((int64_t)1 << 31)) return MOE_ERR_INVALID_ARG;
@@ -200,9 +224,17 @@ moe_status moe_grouped_ffn_bwd(moe_shape s, int dtype, int64_t rows, const void*
     if (s.d_model % 128 || s.d_ff % 128) return MOE_ERR_UNSUPPORTED;
     if (dw_dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
     if (!ptrs_ok(offsets, dw1, dw2, ws)) return MOE_ERR_INVALID_ARG;
-    if (rows > 0 && !ptrs_ok(dy_perm, x_perm, act_saved, dx_perm)) return MOE_ERR_INVALID_ARG;
+    // x_perm is read only by the recompute (the backward uses the token-block copy)
+    if (rows > 0 && (!ptrs_ok(dy_perm, act_saved, dx_perm) || (recompute && !x_perm) ||
+                     (x_perm && !aligned16(x_perm))))
+      return MOE_ERR_INVALID_ARG;
     FfnShape fsm{s.d_model, s.E, s.d_ff, rows};
     if (ws_bytes < kStatusBytes + ffn_mx_ws_bytes(fsm)) return MOE_ERR_INVALID_ARG;
+    if (recompute) {
+      cudaError_t e = ffn_fwd_mx(fsm, x_perm, offsets, w, act, nullptr, scratch(ws),
+                                 status_word(ws), as_stream(stream));
+      if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
     return cuda_status(ffn_bwd_mx(fsm, dy_perm, x_perm, act_saved, offsets, w, dx_perm,
                                   static_cast<float*>(dw1), static_cast<float*>(dw2), scratch(ws),
                                   status_word(ws), as_stream(stream)));
@@ -216,6 +248,15 @@ moe_status moe_grouped_ffn_bwd(moe_shape s, int dtype, int64_t rows, const void*
   FfnShape fs{s.d_model, s.E, s.d_ff, rows};
   if (ws_bytes < kStatusBytes + ffn_bwd_ws_bytes(fs, dtype == MOE_BF16)) return MOE_ERR_INVALID_ARG;
   cudaStream_t cs = as_stream(stream);
+  if (dtype == MOE_BF16 && (s.d_model % 256 || s.d_ff % 256)) return MOE_ERR_UNSUPPORTED;
+  if (recompute) {
+    cudaError_t e = dtype == MOE_F32
+                        ? ffn_fwd_f32(fs, static_cast<const float*>(x_perm), offsets,
+                                      static_cast<const float*>(w1), static_cast<const float*>(w2),
+                                      static_cast<float*>(act), nullptr, cs)
+                        : ffn_fwd_bf16(fs, x_perm, offsets, w1, w2, act, nullptr, status_word(ws), cs);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+  }
   if (dtype == MOE_F32)
     return cuda_status(ffn_bwd_f32(fs, static_cast<const float*>(dy_perm),
                                    static_cast<const float*>(x_perm),
@@ -223,9 +264,31 @@ moe_status moe_grouped_ffn_bwd(moe_shape s, int dtype, int64_t rows, const void*
                                    static_cast<const float*>(w1), static_cast<const float*>(w2),
                                    static_cast<float*>(dx_perm), static_cast<float*>(dw1),
                                    static_cast<float*>(dw2), scratch(ws), cs));
-  if (s.d_model % 256 || s.d_ff % 256) return MOE_ERR_UNSUPPORTED;
   return cuda_status(ffn_bwd_bf16(fs, dy_perm, x_perm, act_saved, offsets, w1, w2, dx_perm, dw1,
                                   dw2, dw_dtype == MOE_F32, scratch(ws), status_word(ws), cs));
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_grouped_ffn_bwd(moe_shape s, int dtype, int64_t rows, const void* dy_perm,
+                               const void* x_perm, const void* act_saved,
+                               const int32_t* offsets, const void* w1, const void* w2,
+                               const void* mx, void* dx_perm, void* dw1, void* dw2,
+                               int dw_dtype, void* ws, size_t ws_bytes, void* stream) {
+  return ffn_bwd_entry(s, dtype, rows, dy_perm, x_perm, const_cast<void*>(act_saved), offsets, w1,
+                       w2, mx, dx_perm, dw1, dw2, dw_dtype, ws, ws_bytes, stream, false);
+}
+
+moe_status moe_grouped_ffn_bwd_recompute(moe_shape s, int dtype, int64_t rows,
+                                         const void* dy_perm, const void* x_perm,
+                                         void* act_scratch, const int32_t* offsets,
+                                         const void* w1, const void* w2, const void* mx,
+                                         void* dx_perm, void* dw1, void* dw2, int dw_dtype,
+                                         void* ws, size_t ws_bytes, void* stream) {
+  return ffn_bwd_entry(s, dtype, rows, dy_perm, x_perm, act_scratch, offsets, w1, w2, mx, dx_perm,
+                       dw1, dw2, dw_dtype, ws, ws_bytes, stream, true);
 }
 
 moe_status moe_route_bwd(moe_shape s, int dtype, const void* x, const void* w_router,

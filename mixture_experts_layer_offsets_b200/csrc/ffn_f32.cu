@@ -169,6 +169,7 @@ cudaError_t ffn_fwd_f32(const FfnShape& s, const float* x_perm, const int32_t* o
               0, 2 * f, d};
   if ((err = run(g1, bound_tiles_m(s.rows, s.E, 2 * f), st)) != cudaSuccess) return err;
   swiglu_fwd_kernel<<<elem_grid(s.rows * f), 256, 0, st>>>(act, offsets, s.E, s.rows, f);
+  if (!y_perm) return cudaGetLastError();  // recompute of a | u | h only
   SimtGemm g2{act + 2 * f, 3 * f, 1, w2, f, 1, (int64_t)d * f, y_perm, d, 0, offsets, s.E, 0,
               0, d, f};
   return run(g2, bound_tiles_m(s.rows, s.E, d), st);

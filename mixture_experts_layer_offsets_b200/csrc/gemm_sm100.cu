@@ -801,12 +801,15 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
             constexpr int kBoxBytes = kBoxRowsK * 128;
             constexpr int kABoxes = kABytes / kBoxBytes;
             constexpr int kBoxes = kABoxes + C::kBBytes / kBoxBytes;
-            const int nz = (kBoxRowsK - ti.klast) * 8;  // 16-byte pieces per box
-            for (int i = lane; i < nz * kBoxes; i += 32) {
-              const int box = i / nz, rem = i - box * nz;
-              uint8_t* base = box < kABoxes ? sa + box * kBoxBytes : sb + (box - kABoxes) * kBoxBytes;
-              *reinterpret_cast<uint4*>(base + (ti.klast + rem / 8) * 128 + (rem & 7) * 16) =
-                  make_uint4(0, 0, 0, 0);
+            // The rows are 128 bytes each, so the tail of a box is one contiguous range
+            // (the 128-byte swizzle only permutes 16-byte pieces within a row).
+            const int tail = (kBoxRowsK - ti.klast) * 128;
+#pragma unroll
+            for (int box = 0; box < kBoxes; ++box) {
+              uint8_t* z = (box < kABoxes ? sa + box * kBoxBytes : sb + (box - kABoxes) * kBoxBytes) +
+                           ti.klast * 128;
+              for (int o = lane * 16; o < tail; o += 512)
+                *reinterpret_cast<uint4*>(z + o) = make_uint4(0, 0, 0, 0);
             }
             fence_proxy_async_smem();
           }
@@ -1559,6 +1562,7 @@ cudaError_t ffn_fwd_bf16(const FfnShape& s, const void* x_perm, const int32_t* o
   err = pairs ? launch_pair<256, false, EPI_SWIGLU_FWD>(p1, pair_tile_bound(s) * (f / 128), st)
               : launch<256, false, false, EPI_SWIGLU_FWD, false>(p1, m_tile_bound(s) * (f / 128), st);
   if (err != cudaSuccess) return err;
+  if (!y_perm) return cudaSuccess;  // recompute of a | u | h only
   // down GEMM: y = h W2^T
   GemmParams p2 = base_params(s, offsets, status);
   if (!tmap(&p2.tmA, actb + 2 * f, f, s.rows, 3 * f, 64, 128) ||
@@ -1733,13 +1737,15 @@ cudaError_t ffn_fwd_mx(const FfnShape& s, const void* x_perm, const int32_t* off
   int32_t* rt = reinterpret_cast<int32_t*>(ws + L.rt);
   int4* map = reinterpret_cast<int4*>(ws + L.map);
   int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
-  if ((err = row_tile_launch(offsets, E, R, rt, st)) != cudaSuccess ||
-      (err = seg_blocks_launch(offsets, E, map, cnt, st)) != cudaSuccess)
-    return err;
-  // x along d (gate/up GEMM) and in token blocks (kept for the dW1 GEMM of the backward)
-  if ((err = mxfp8_act(R, E, d, d, x_perm, map, cnt, rt, ws + L.qx0, ws + L.sx0, ws + L.qx1,
-                       ws + L.sx1, st)) != cudaSuccess)
-    return err;
+  // x along d (gate/up GEMM) and in token blocks (kept for the dW1 GEMM of the backward);
+  // without x_perm, the fused dispatch has written both copies and the maps already
+  if (x_perm) {
+    if ((err = row_tile_launch(offsets, E, R, rt, st)) != cudaSuccess ||
+        (err = seg_blocks_launch(offsets, E, map, cnt, st)) != cudaSuccess ||
+        (err = mxfp8_act(R, E, d, d, x_perm, map, cnt, rt, ws + L.qx0, ws + L.sx0, ws + L.qx1,
+                         ws + L.sx1, st)) != cudaSuccess)
+      return err;
+  }
   GemmParams p1 = mx_params(s, offsets, status);
   if (!tmap(&p1.tmA, ws + L.qx0, d, R, d, 128, 128, false, true) ||
       !tmap(&p1.tmB, w.w1_q, d, (uint64_t)E * 2 * f, d, 128, 128, false, true) ||
@@ -1756,6 +1762,7 @@ cudaError_t ffn_fwd_mx(const FfnShape& s, const void* x_perm, const int32_t* off
   if ((err = mxfp8_act(R, E, f, 3 * f, actb + 2 * f, map, cnt, rt, ws + L.qh0, ws + L.sh0,
                        ws + L.qh1, ws + L.sh1, st)) != cudaSuccess)
     return err;
+  if (!y_perm) return cudaSuccess;  // recompute: a | u | h and the token-block copies only
   GemmParams p2 = mx_params(s, offsets, status);
   if (!tmap(&p2.tmA, ws + L.qh0, f, R, f, 128, 128, false, true) ||
       !tmap(&p2.tmB, w.w2_q, f, (uint64_t)E * d, f, 128, 128, false, true) ||
@@ -1766,6 +1773,22 @@ cudaError_t ffn_fwd_mx(const FfnShape& s, const void* x_perm, const int32_t* off
   p2.N = d; p2.K = f; p2.b_rows = d;
   p2.out = static_cast<__nv_bfloat16*>(y_perm); p2.ld_out = d;
   return launch_mx_n<false, false, EPI_STORE, false>(p2, d, m_tile_bound(s), st);
+}
+
+cudaError_t mx_dispatch(const FfnShape& s, const void* x, const int32_t* perm_src,
+                        const int32_t* offsets, void* scratch, cudaStream_t st) {
+  if (s.rows == 0) return cudaSuccess;
+  uint8_t* ws = static_cast<uint8_t*>(scratch);
+  const MxLayout L = mx_layout(s);
+  int32_t* rt = reinterpret_cast<int32_t*>(ws + L.rt);
+  int4* map = reinterpret_cast<int4*>(ws + L.map);
+  int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
+  cudaError_t err;
+  if ((err = row_tile_launch(offsets, s.E, s.rows, rt, st)) != cudaSuccess ||
+      (err = seg_blocks_launch(offsets, s.E, map, cnt, st)) != cudaSuccess)
+    return err;
+  return mxfp8_act(s.rows, s.E, s.d, s.d, x, map, cnt, rt, ws + L.qx0, ws + L.sx0, ws + L.qx1,
+                   ws + L.sx1, st, perm_src);
 }
 
 cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_perm, const void* act,

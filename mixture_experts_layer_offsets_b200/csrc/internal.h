@@ -87,22 +87,31 @@ cudaError_t mxfp8_weights(const float* w, int E, int Rw, int Kw, uint8_t* q0, ui
                           uint8_t* q1, uint8_t* s1, cudaStream_t st);
 //   seg_blocks_launch: the 32-row token blocks of all segments (at most rows/32 + E)
 //   mxfp8_act: one pass over a bf16 activation writing its row copy (row-tile atoms) and its
-//     token-block copy (stage atoms)
+//     token-block copy (stage atoms); with `gather`, operand row r is source row gather[r]
 cudaError_t seg_blocks_launch(const int32_t* offsets, int E, int4* map, int32_t* count,
                               cudaStream_t st);
 cudaError_t mxfp8_act(int64_t rows, int E, int64_t K, int64_t ld, const void* src_bf16,
                       const int4* map, const int32_t* count, const int32_t* row_tile, uint8_t* q_r,
-                      uint8_t* atoms_r, uint8_t* q_c, uint8_t* atoms_c, cudaStream_t st);
+                      uint8_t* atoms_r, uint8_t* q_c, uint8_t* atoms_c, cudaStream_t st,
+                      const int32_t* gather = nullptr);
+//   perm_src_launch: perm_src[slot_row[t, j]] = t (the permute's source map, no row copy)
+cudaError_t perm_src_launch(const int32_t* slot_row, int32_t* perm_src, int T, int k,
+                            cudaStream_t st);
 
 // ---------------------------------------------------------- grouped FFN
 struct FfnShape {
   int d, E, f;
   int64_t rows;
 };
+//   mx_dispatch: the fused MXFP8 dispatch: row maps and both quantised copies of x, gathered
+//     through perm_src, into the workspace regions that ffn_fwd_mx reads
+cudaError_t mx_dispatch(const FfnShape& s, const void* x, const int32_t* perm_src,
+                        const int32_t* offsets, void* scratch, cudaStream_t st);
 size_t ffn_bwd_ws_bytes(const FfnShape& s, bool bf16);
 // fp32 partial sums of weight-gradient groups cut into K ranges (tensor-core paths)
 size_t wgrad_part_bytes(const FfnShape& s, bool fp8);
 // fp32 path: CUDA-core grouped GEMMs
+//   ffn_fwd_*: y_perm == nullptr runs the gate/up half only (the recompute of a | u | h)
 cudaError_t ffn_fwd_f32(const FfnShape& s, const float* x_perm, const int32_t* offsets,
                         const float* w1, const float* w2, float* act, float* y_perm,
                         cudaStream_t st);

@@ -369,7 +369,7 @@ mx_act_kernel(const __nv_bfloat16* __restrict__ src, int64_t K, int64_t ld,
               const int4* __restrict__ map, const int32_t* __restrict__ count,
               const int32_t* __restrict__ row_tile, uint8_t* __restrict__ q_r,
               uint8_t* __restrict__ atoms_r, uint8_t* __restrict__ q_c,
-              uint8_t* __restrict__ atoms_c) {
+              uint8_t* __restrict__ atoms_c, const int32_t* __restrict__ gather) {
   __shared__ __align__(16) __nv_bfloat16 s_t[32 * kActPitch];
   __shared__ __align__(16) uint8_t s_q[32 * 128];
   const int tid = threadIdx.x, ct = blockIdx.x;
@@ -384,7 +384,11 @@ mx_act_kernel(const __nv_bfloat16* __restrict__ src, int64_t K, int64_t ld,
     for (int j = 0; j < 4; ++j) {
       const int i = tid + 128 * j, row = i >> 4, p8 = i & 15;
       uint4 v = make_uint4(0, 0, 0, 0);
-      if (row < n) v = ldg16(src + (int64_t)(r0 + row) * ld + c0 + p8 * 8);
+      if (row < n) {
+        // row r of the operand is source row gather[r] (the fused dispatch), else r
+        const int64_t sr = gather ? (int64_t)__ldg(gather + r0 + row) : (int64_t)(r0 + row);
+        v = ldg16(src + sr * ld + c0 + p8 * 8);
+      }
       *reinterpret_cast<uint4*>(s_t + row * kActPitch + p8 * 8) = v;
     }
     __syncthreads();
@@ -468,11 +472,12 @@ cudaError_t seg_blocks_launch(const int32_t* offsets, int E, int4* map, int32_t*
 
 cudaError_t mxfp8_act(int64_t rows, int E, int64_t K, int64_t ld, const void* src_bf16,
                       const int4* map, const int32_t* count, const int32_t* row_tile, uint8_t* q_r,
-                      uint8_t* atoms_r, uint8_t* q_c, uint8_t* atoms_c, cudaStream_t st) {
+                      uint8_t* atoms_r, uint8_t* q_c, uint8_t* atoms_c, cudaStream_t st,
+                      const int32_t* gather) {
   if (rows == 0) return cudaSuccess;
   dim3 grid((unsigned)(K / 128), (unsigned)std::min<int64_t>(rows / 32 + E, 65535));
   mx_act_kernel<<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(src_bf16), K, ld, map,
-                                       count, row_tile, q_r, atoms_r, q_c, atoms_c);
+                                       count, row_tile, q_r, atoms_r, q_c, atoms_c, gather);
   return cudaGetLastError();
 }
 

@@ -212,6 +212,23 @@ padded_dispatch_kernel(const T* __restrict__ x, const int32_t* __restrict__ topk
 
 }  // namespace
 
+namespace {
+__global__ void __launch_bounds__(256) perm_src_kernel(const int32_t* __restrict__ slot_row,
+                                                       int32_t* __restrict__ perm_src, int64_t n,
+                                                       int k) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) perm_src[slot_row[i]] = (int32_t)(i / k);
+}
+}  // namespace
+
+cudaError_t perm_src_launch(const int32_t* slot_row, int32_t* perm_src, int T, int k,
+                            cudaStream_t st) {
+  const int64_t n = (int64_t)T * k;
+  if (n == 0) return cudaSuccess;
+  perm_src_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(slot_row, perm_src, n, k);
+  return cudaGetLastError();
+}
+
 cudaError_t permute_launch(bool bf16, const void* x, const int32_t* slot_row, void* x_perm,
                            int32_t* perm_src, int T, int d, int k, cudaStream_t st) {
   if (T == 0) return cudaSuccess;

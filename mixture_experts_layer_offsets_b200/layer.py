@@ -32,7 +32,8 @@ def capacity_for(rows: int, E: int, cf_num: int = 5, cf_den: int = 4) -> int:
 class MoELayer:
     def __init__(self, T: int, d_model: int, E: int, top_k: int, d_ff: int, dtype: str = "bf16",
                  device="cuda", dw_dtype: str | None = None, capacity: int | None = None,
-                 renorm: bool = False):
+                 renorm: bool = False, recompute: bool = False, act_scratch=None, ws=None,
+                 fused_dispatch: bool | None = None):
         if dtype not in _DT:
             raise ValueError(f"dtype {dtype!r} is not supported by the layer path")
         self.T, self.d, self.E, self.k, self.f = T, d_model, E, top_k, d_ff
@@ -47,6 +48,16 @@ class MoELayer:
             raise ValueError("the padded layout is not offered with MXFP8")
         self.capacity = capacity
         self.renorm = renorm
+        # recompute: the backward refills a | u | h (and the MXFP8 token-block copies)
+        # from x_perm, so act_scratch and ws may be shared by several layers
+        self.recompute = recompute
+        # MXFP8: the dispatch writes the quantised copies of x directly (moe_permute_mx);
+        # the recompute needs the bf16 x_perm, so it keeps the plain permute
+        if fused_dispatch is None:
+            fused_dispatch = dtype == "mxfp8" and not recompute
+        if fused_dispatch and (dtype != "mxfp8" or recompute):
+            raise ValueError("the fused dispatch is the MXFP8 layer's, without recompute")
+        self.fused_dispatch = fused_dispatch
         self.shape = capi.shape_of(T, d_model, E, top_k, d_ff)
         self.R = T * top_k
         self.rows = E * capacity if capacity else self.R
@@ -64,8 +75,16 @@ class MoELayer:
         self.offsets = torch.empty(E + 1, **i32)
         self.slot_row = torch.empty(T, top_k, **i32)
         self.perm_src = torch.empty(max(self.R, 1), **i32)
-        self.x_perm = torch.empty(rows, d_model, **act)
-        self.act = torch.empty(rows, 3 * d_ff, **act)
+        # (the fused MXFP8 dispatch writes no bf16 copy of the routed rows)
+        self.x_perm = None if fused_dispatch else torch.empty(rows, d_model, **act)
+        if act_scratch is not None:
+            if not recompute:
+                raise ValueError("a shared activation buffer needs recompute=True")
+            if act_scratch.numel() < rows * 3 * d_ff or act_scratch.dtype != tdt:
+                raise ValueError("act_scratch is too small or of the wrong type")
+            self.act = act_scratch.view(-1)[:rows * 3 * d_ff].view(rows, 3 * d_ff)
+        else:
+            self.act = torch.empty(rows, 3 * d_ff, **act)
         self.y_perm = torch.empty(rows, d_model, **act)
         self.out = torch.empty(T, d_model, **act)
         self.dgate = torch.empty(T, top_k, **f32)
@@ -100,7 +119,12 @@ class MoELayer:
         nbytes = capi.moe_workspace_size(self.shape, self.ffn_dtype, self.rows)
         if nbytes == 0:
             raise ValueError("invalid MoE shape")
-        self.ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+        if ws is not None:
+            if ws.numel() * ws.element_size() < nbytes:
+                raise ValueError("the shared workspace is too small")
+            self.ws = ws
+        else:
+            self.ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
 
     # the row map and offsets that the grouped FFN and combine steps use
     @property
@@ -130,9 +154,12 @@ class MoELayer:
             capi.moe_padded_dispatch(s, dt, self.capacity, x, self.topk_idx, self.slot_row,
                                      self.offsets, self.x_perm, self.pad_row, self.offsets_pad,
                                      stream)
+        elif self.fused_dispatch:
+            capi.moe_permute_mx(s, x, self.slot_row, self.offsets, self.perm_src, self.ws, stream)
         else:
             capi.moe_permute(s, dt, x, self.slot_row, self.x_perm, self.perm_src, stream)
-        capi.moe_grouped_ffn_fwd(s, self.ffn_dtype, self.rows, self.x_perm, self.ffn_offsets, w1,
+        xp = None if self.fused_dispatch else self.x_perm
+        capi.moe_grouped_ffn_fwd(s, self.ffn_dtype, self.rows, xp, self.ffn_offsets, w1,
                                  w2, self.act, self.y_perm, self.ws, mx=self.mx, stream=stream)
         if self.renorm:
             capi.moe_renorm_gates(s, self.topk_gate, self.gate_rn, stream)
@@ -145,9 +172,11 @@ class MoELayer:
                              self.dy_perm, self.dgate_rn if self.renorm else self.dgate, stream)
         if self.renorm:
             capi.moe_renorm_gates_bwd(s, self.topk_gate, self.dgate_rn, self.dgate, stream)
-        capi.moe_grouped_ffn_bwd(s, self.ffn_dtype, self.rows, self.dy_perm, self.x_perm,
-                                 self.act, self.ffn_offsets, w1, w2, self.dx_perm, self.dw1,
-                                 self.dw2, _DT[self.dw_dtype], self.ws, mx=self.mx, stream=stream)
+        bwd = capi.moe_grouped_ffn_bwd_recompute if self.recompute else capi.moe_grouped_ffn_bwd
+        xp = None if self.fused_dispatch else self.x_perm
+        bwd(s, self.ffn_dtype, self.rows, self.dy_perm, xp, self.act, self.ffn_offsets,
+            w1, w2, self.dx_perm, self.dw1, self.dw2, _DT[self.dw_dtype], self.ws, mx=self.mx,
+            stream=stream)
         capi.moe_route_bwd(s, dt, x, w_router, self.logits, self.topk_idx, self.dgate,
                            self.dx_perm, self.row_map, self.dx, self.dw_router, self.ws, stream)
         return self.dx

@@ -30,12 +30,12 @@ def rel(a, b) -> float:
     return float(np.linalg.norm(a - b) / (nb if nb > 0 else 1.0))
 
 
-def run_layer(cfg, seed=0, capacity=None, dw_dtype="f32", renorm=False):
+def run_layer(cfg, seed=0, capacity=None, dw_dtype="f32", renorm=False, **kw):
     """Seeded inputs drawn on the CPU, copied to the GPU, one fwd+bwd step."""
     cpu = inputs.make_inputs(cfg, device="cpu", seed=seed)
     dev = {k: (v.cuda() if v is not None else None) for k, v in cpu.items()}
     L = MoELayer(cfg.T, cfg.d_model, cfg.E, cfg.top_k, cfg.d_ff, cfg.dtype, "cuda",
-                 dw_dtype=dw_dtype, capacity=capacity, renorm=renorm)
+                 dw_dtype=dw_dtype, capacity=capacity, renorm=renorm, **kw)
     L.step(dev["x"], dev["w_router"], dev["bias"], dev["w1"], dev["w2"], dev["dout"])
     torch.cuda.synchronize()
     assert L.device_status() == 0
@@ -51,3 +51,30 @@ def oracle_for(cpu, L, capacity=None):
         return ref.padded_layer_fwd_bwd(*args, capacity, bias, select_logits=f64(L.logits),
                                         renorm=L.renorm)
     return ref.layer_fwd_bwd(*args, bias, select_logits=f64(L.logits), renorm=L.renorm)
+
+
+def check_recompute_bit_exact(cfg):
+    """Two layers share one activation buffer and one workspace; layer A's backward
+    runs after layer B's forward has overwritten both, recomputing what it needs.  Its
+    results equal, bit for bit, those of a layer that kept its own activations."""
+    _, L0 = run_layer(cfg, seed=0)
+    dev = lambda d: {k: (v.cuda() if v is not None else None) for k, v in d.items()}
+    a_in = dev(inputs.make_inputs(cfg, device="cpu", seed=0))
+    b_in = dev(inputs.make_inputs(cfg, device="cpu", seed=1))
+    tdt = L0.act.dtype
+    act = torch.empty(L0.act.numel(), dtype=tdt, device="cuda")
+    ws = torch.zeros_like(L0.ws)
+    mk = lambda: MoELayer(cfg.T, cfg.d_model, cfg.E, cfg.top_k, cfg.d_ff, cfg.dtype, "cuda",
+                          recompute=True, act_scratch=act, ws=ws)
+    A, B = mk(), mk()
+    A.forward(a_in["x"], a_in["w_router"], a_in["bias"], a_in["w1"], a_in["w2"])
+    a_act = act.clone()
+    B.forward(b_in["x"], b_in["w_router"], b_in["bias"], b_in["w1"], b_in["w2"])
+    torch.cuda.synchronize()
+    assert cfg.T == 0 or not torch.equal(act, a_act), "layer B did not overwrite the shared buffer"
+    A.backward(a_in["dout"], a_in["x"], a_in["w_router"], a_in["w1"], a_in["w2"])
+    torch.cuda.synchronize()
+    assert A.device_status() == 0
+    assert torch.equal(act, a_act), "the recompute did not restore a | u | h"
+    for key in ("out", "dgate", "dx_perm", "dw1", "dw2", "dx", "dw_router"):
+        assert torch.equal(getattr(A, key), getattr(L0, key)), key

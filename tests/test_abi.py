@@ -122,6 +122,9 @@ def test_row_ops_validation(lib):
     assert lib.moe_renorm_gates(s, FAKE + 4, FAKE, None) == capi.MOE_ERR_INVALID_ARG
     assert lib.moe_renorm_gates_bwd(s, FAKE, None, FAKE, None) == capi.MOE_ERR_INVALID_ARG
     assert lib.moe_renorm_gates(_shape(T=0), None, None, None) == capi.MOE_OK
+    assert lib.moe_grouped_ffn_bwd_recompute(s, capi.MOE_BF16, 64, *([FAKE] * 3), None,
+                                             *([FAKE] * 6), capi.MOE_F32, FAKE, 1 << 30,
+                                             None) == capi.MOE_ERR_INVALID_ARG
     # T == 0 is a valid no-op for the row movers
     assert lib.moe_permute(_shape(T=0), capi.MOE_BF16, None, None, None, None, None) == capi.MOE_OK
 

@@ -12,7 +12,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import TOL, f64, i64, oracle_for, rel, run_layer
+from gpu_helpers import TOL, check_recompute_bit_exact, f64, i64, oracle_for, rel, run_layer
 from mixture_experts_layer_offsets_b200.inputs import CONFIGS, shrink
 from oracle import moe_ref as ref
 
@@ -203,3 +203,8 @@ def test_renorm_kernels_match_oracle_directly():
         assert np.allclose(f64(out), want, rtol=1e-6, atol=0)
         wb = ref.renorm_gates_bwd(g.astype(np.float64), dg.astype(np.float64))
         assert rel(f64(dout), wb) <= 1e-6
+
+
+@pytest.mark.parametrize("name", ["bf16_e8_small", "bf16_skew_split", "tiny_f32", "f32_one_token"])
+def test_recompute_with_shared_buffers_is_bit_exact(name):
+    check_recompute_bit_exact(CASES[name])

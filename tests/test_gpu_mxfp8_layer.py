@@ -14,7 +14,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import TOL, f64, i64, rel, run_layer
+from gpu_helpers import TOL, check_recompute_bit_exact, f64, i64, rel, run_layer
 from mixture_experts_layer_offsets_b200.inputs import CONFIGS, shrink
 from oracle import moe_mx_ref as mxr
 from oracle import mxfp8_ref as mx
@@ -132,3 +132,24 @@ def test_mxfp8_is_closer_to_its_oracle_than_to_the_unquantised_layer():
     for key, dev in (("out", L.out), ("dw1", L.dw1), ("dx", L.dx)):
         assert rel(f64(dev), o[key]) < 0.5 * rel(f64(dev), u[key]), key
 
+
+
+@pytest.mark.parametrize("name", ["mx_e8", "mx_skew_split", "mx_one_token"])
+def test_mxfp8_recompute_with_shared_buffers_is_bit_exact(name):
+    # the shared workspace loses the forward's token-block copies to layer B: the
+    # recompute rebuilds them along with a | u | h
+    check_recompute_bit_exact(CASES[name])
+
+
+@pytest.mark.parametrize("name", ["mx_e8", "mx_e16_odd", "mx_skew", "mx_one_token"])
+def test_fused_dispatch_is_bit_identical_to_permute_then_quantise(name):
+    cfg = CASES[name]
+    _, A = run_layer(cfg, fused_dispatch=True)
+    _, B = run_layer(cfg, fused_dispatch=False)
+    assert A.x_perm is None
+    for key in ("perm_src", "act", "y_perm", "out", "dgate", "dx_perm", "dw1", "dw2", "dx",
+                "dw_router"):
+        a, b = getattr(A, key), getattr(B, key)
+        if key in ("perm_src", "act", "y_perm", "dx_perm"):
+            a, b = a[:cfg.R], b[:cfg.R]
+        assert torch.equal(a, b), key
