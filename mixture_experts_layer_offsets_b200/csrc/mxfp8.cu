@@ -376,22 +376,34 @@ mx_act_kernel(const __nv_bfloat16* __restrict__ src, int64_t K, int64_t ld,
   const int64_t c0 = (int64_t)ct * 128;
   const int64_t kq = K >> 7;
   const int nblocks = count[0];
-  for (int b = blockIdx.y; b < nblocks; b += gridDim.y) {
-    const int4 m = map[b];
-    const int r0 = m.x, n = m.y;
-    // load n rows x 128 columns (16 pieces of 16 bytes per row)
+  // n rows x 128 columns of block b: 16 pieces of 16 bytes per row, 4 per thread.  The next
+  // block's pieces are loaded into registers while this block is quantised.
+  auto load = [&](int b, int4& m, uint4 (&v)[4]) {
+    m = map[b];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int i = tid + 128 * j, row = i >> 4, p8 = i & 15;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (row < n) {
+      v[j] = make_uint4(0, 0, 0, 0);
+      if (row < m.y) {
         // row r of the operand is source row gather[r] (the fused dispatch), else r
-        const int64_t sr = gather ? (int64_t)__ldg(gather + r0 + row) : (int64_t)(r0 + row);
-        v = ldg16(src + sr * ld + c0 + p8 * 8);
+        const int64_t sr = gather ? (int64_t)__ldg(gather + m.x + row) : (int64_t)(m.x + row);
+        v[j] = ldg16(src + sr * ld + c0 + p8 * 8);
       }
-      *reinterpret_cast<uint4*>(s_t + row * kActPitch + p8 * 8) = v;
+    }
+  };
+  int4 mnext;
+  uint4 vnext[4];
+  if (blockIdx.y < nblocks) load(blockIdx.y, mnext, vnext);
+  for (int b = blockIdx.y; b < nblocks; b += gridDim.y) {
+    const int4 m = mnext;
+    const int r0 = m.x, n = m.y;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int i = tid + 128 * j, row = i >> 4, p8 = i & 15;
+      *reinterpret_cast<uint4*>(s_t + row * kActPitch + p8 * 8) = vnext[j];
     }
     __syncthreads();
+    if (b + (int)gridDim.y < nblocks) load(b + gridDim.y, mnext, vnext);
     // rows: thread = (row, 32-column block)
     {
       const int row = tid >> 2, kb = tid & 3;
@@ -475,7 +487,9 @@ cudaError_t mxfp8_act(int64_t rows, int E, int64_t K, int64_t ld, const void* sr
                       uint8_t* atoms_r, uint8_t* q_c, uint8_t* atoms_c, cudaStream_t st,
                       const int32_t* gather) {
   if (rows == 0) return cudaSuccess;
-  dim3 grid((unsigned)(K / 128), (unsigned)std::min<int64_t>(rows / 32 + E, 65535));
+  // about 8 blocks of 128 threads per SM at a time, each looping over several token blocks
+  const int64_t want = std::max<int64_t>(1, (int64_t)num_sms() * 8 / (K / 128));
+  dim3 grid((unsigned)(K / 128), (unsigned)std::min<int64_t>({rows / 32 + E, want, 65535}));
   mx_act_kernel<<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(src_bf16), K, ld, map,
                                        count, row_tile, q_r, atoms_r, q_c, atoms_c, gather);
   return cudaGetLastError();
