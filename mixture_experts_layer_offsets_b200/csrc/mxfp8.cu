@@ -230,92 +230,109 @@ constexpr int kWBlk = 36;              // floats per staged 32-column block
 constexpr int kWPitch = 4 * kWBlk;     // floats per staged row
 constexpr int kWSmem = 64 * kWPitch * 4 + 64 * 128 + 256 + 256;
 __global__ void __launch_bounds__(128)
-mx_weights_kernel(const float* __restrict__ w, int Rw, int Kw, uint8_t* __restrict__ q0,
+mx_weights_kernel(const float* __restrict__ w, int E, int Rw, int Kw, uint8_t* __restrict__ q0,
                   uint8_t* __restrict__ s0, uint8_t* __restrict__ q1, uint8_t* __restrict__ s1) {
   extern __shared__ float tile[];                                  // [64][kWPitch]
   uint8_t* qt = reinterpret_cast<uint8_t*>(tile + 64 * kWPitch);   // [64][128] q1 bytes
   uint8_t* sa0 = qt + 64 * 128;          // s0 bytes of rows 64 h .. 64 h + 63: [32][8]
   uint8_t* sa1 = sa0 + 256;              // s1 bytes of row blocks 2 h, 2 h + 1: [128][2]
-  const int e = blockIdx.z, rt = blockIdx.y >> 1, half = blockIdx.y & 1, ct = blockIdx.x;
   const int tid = threadIdx.x;
-  const int64_t row0 = (int64_t)e * Rw + rt * 128 + half * 64;
-  const int col0 = ct * 128;
-  // pass 1: blocks along rows; a quad of lanes covers one 32-wide block.  All sixteen
-  // 16-byte loads of a thread are issued before any is used.
+  // half tiles in (expert, 64-row half, 128-column tile) order; the CTA loops over them
+  const int nct = Kw >> 7, nhalf = Rw >> 6;
+  const int64_t ntiles = (int64_t)E * nhalf * nct;
+  // pass 1 takes blocks along rows; a quad of lanes covers one 32-wide block.  The sixteen
+  // 16-byte loads of a thread for the next half tile are issued as soon as the current one
+  // sits in shared memory, so they are in flight during the column pass and the stores.
   float4 ld[16];
+  auto load = [&](int64_t t) {
+    const int ct = (int)(t % nct);
+    const int64_t rest = t / nct;
+    const int64_t row0 = (rest / nhalf) * Rw + (rest % nhalf) * 64;
 #pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    const int task = it * 128 + tid;          // 1024 = 64 rows x 4 blocks x 4 parts
-    const int r = task >> 4, kb = (task >> 2) & 3, part = task & 3;
-    const float* p = w + (row0 + r) * Kw + col0 + kb * 32 + part * 8;
-    ld[2 * it] = __ldg(reinterpret_cast<const float4*>(p));
-    ld[2 * it + 1] = __ldg(reinterpret_cast<const float4*>(p + 4));
-  }
-#pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    const int task = it * 128 + tid;
-    const int r = task >> 4, kb = (task >> 2) & 3, part = task & 3;
-    const float4 a = ld[2 * it], b = ld[2 * it + 1];
-    float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    float* t = tile + r * kWPitch + kb * kWBlk + part * 8;
-    *reinterpret_cast<float4*>(t) = a;
-    *reinterpret_cast<float4*>(t + 4) = b;
-    float amax = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    const int ex = block_exponent(amax);
-    const float mul = pow2_neg(ex);
-    uint2 out;
-    out.x = e4m3_pair(v[1] * mul, v[0] * mul) | (e4m3_pair(v[3] * mul, v[2] * mul) << 16);
-    out.y = e4m3_pair(v[5] * mul, v[4] * mul) | (e4m3_pair(v[7] * mul, v[6] * mul) << 16);
-    *reinterpret_cast<uint2*>(q0 + (row0 + r) * Kw + col0 + kb * 32 + part * 8) = out;
-    // atom row r % 32 holds groups (r / 32) of 4 bytes; this half owns groups 2 h, 2 h + 1
-    if (part == 0) sa0[(r & 31) * 8 + (r >> 5) * 4 + kb] = (uint8_t)(ex + 127);
-  }
-  __syncthreads();
-  // pass 2: blocks of 32 rows within a column; a thread takes two adjacent columns of one
-  // row block (64 column pairs x 2 row blocks)
-  {
-    const int cp = tid & 63, rb = tid >> 6;
-    const int c = 2 * cp;
-    const float* col = tile + (c >> 5) * kWBlk + (c & 31);
-    float am0 = 0.f, am1 = 0.f;
-#pragma unroll 8
-    for (int i = 0; i < 32; ++i) {
-      const float2 v = *reinterpret_cast<const float2*>(col + (rb * 32 + i) * kWPitch);
-      am0 = fmaxf(am0, fabsf(v.x));
-      am1 = fmaxf(am1, fabsf(v.y));
+    for (int it = 0; it < 8; ++it) {
+      const int task = it * 128 + tid;          // 1024 = 64 rows x 4 blocks x 4 parts
+      const int r = task >> 4, kb = (task >> 2) & 3, part = task & 3;
+      const float* p = w + (row0 + r) * Kw + ct * 128 + kb * 32 + part * 8;
+      ld[2 * it] = __ldg(reinterpret_cast<const float4*>(p));
+      ld[2 * it + 1] = __ldg(reinterpret_cast<const float4*>(p + 4));
     }
-    const int ex0 = block_exponent(am0), ex1 = block_exponent(am1);
-    const float m0 = pow2_neg(ex0), m1 = pow2_neg(ex1);
-#pragma unroll 8
-    for (int i = 0; i < 32; ++i) {
-      const float2 v = *reinterpret_cast<const float2*>(col + (rb * 32 + i) * kWPitch);
-      *reinterpret_cast<uint16_t*>(qt + (rb * 32 + i) * 128 + c) = (uint16_t)e4m3_pair(v.y * m1, v.x * m0);
-    }
-    // atom bytes (c % 32) * 16 + (c / 32) * 4 + (2 h + rb): two bytes per column here
-    sa1[c * 2 + rb] = (uint8_t)(ex0 + 127);
-    sa1[(c + 1) * 2 + rb] = (uint8_t)(ex1 + 127);
-  }
-  __syncthreads();
-  // write the q1 half tile (64 rows x 128 bytes), 16 bytes per store
+  };
+  if ((int64_t)blockIdx.x < ntiles) load(blockIdx.x);
+  for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    const int ct = (int)(t % nct);
+    const int64_t rest = t / nct;
+    const int e = (int)(rest / nhalf), hrow = (int)(rest % nhalf);
+    const int rt = hrow >> 1, half = hrow & 1;
+    const int64_t row0 = (int64_t)e * Rw + hrow * 64;
+    const int col0 = ct * 128;
 #pragma unroll
-  for (int it = 0; it < 4; ++it) {
-    const int idx = it * 128 + tid;            // 512 pieces of 16 bytes
-    const int r = idx >> 3, c16 = idx & 7;
-    *reinterpret_cast<uint4*>(q1 + (row0 + r) * Kw + col0 + c16 * 16) =
-        *reinterpret_cast<const uint4*>(qt + r * 128 + c16 * 16);
-  }
-  uint8_t* a0 = s0 + (((int64_t)e * (Rw >> 7) + rt) * (Kw >> 7) + ct) * 512;
-  uint8_t* a1 = s1 + (((int64_t)e * (Rw >> 7) + rt) * (Kw >> 7) + ct) * 512;
-  if (tid < 32) {   // s0: 8 bytes per atom row
-    *reinterpret_cast<uint2*>(a0 + tid * 16 + half * 8) = *reinterpret_cast<const uint2*>(sa0 + tid * 8);
-  } else {          // s1: 2 bytes per column, at offset (c % 32) * 16 + (c / 32) * 4 + 2 h
-    for (int c = tid - 32; c < 128; c += 96)
-      *reinterpret_cast<uint16_t*>(a1 + (c & 31) * 16 + (c >> 5) * 4 + half * 2) =
-          *reinterpret_cast<const uint16_t*>(sa1 + c * 2);
+    for (int it = 0; it < 8; ++it) {
+      const int task = it * 128 + tid;
+      const int r = task >> 4, kb = (task >> 2) & 3, part = task & 3;
+      const float4 a = ld[2 * it], b = ld[2 * it + 1];
+      float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      float* tp = tile + r * kWPitch + kb * kWBlk + part * 8;
+      *reinterpret_cast<float4*>(tp) = a;
+      *reinterpret_cast<float4*>(tp + 4) = b;
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      const int ex = block_exponent(amax);
+      const float mul = pow2_neg(ex);
+      uint2 out;
+      out.x = e4m3_pair(v[1] * mul, v[0] * mul) | (e4m3_pair(v[3] * mul, v[2] * mul) << 16);
+      out.y = e4m3_pair(v[5] * mul, v[4] * mul) | (e4m3_pair(v[7] * mul, v[6] * mul) << 16);
+      *reinterpret_cast<uint2*>(q0 + (row0 + r) * Kw + col0 + kb * 32 + part * 8) = out;
+      // atom row r % 32 holds groups (r / 32) of 4 bytes; this half owns groups 2 h, 2 h + 1
+      if (part == 0) sa0[(r & 31) * 8 + (r >> 5) * 4 + kb] = (uint8_t)(ex + 127);
+    }
+    if (t + (int64_t)gridDim.x < ntiles) load(t + gridDim.x);
+    __syncthreads();
+    // pass 2: blocks of 32 rows within a column; a thread takes two adjacent columns of one
+    // row block (64 column pairs x 2 row blocks)
+    {
+      const int cp = tid & 63, rb = tid >> 6;
+      const int c = 2 * cp;
+      const float* col = tile + (c >> 5) * kWBlk + (c & 31);
+      float am0 = 0.f, am1 = 0.f;
+#pragma unroll 8
+      for (int i = 0; i < 32; ++i) {
+        const float2 v = *reinterpret_cast<const float2*>(col + (rb * 32 + i) * kWPitch);
+        am0 = fmaxf(am0, fabsf(v.x));
+        am1 = fmaxf(am1, fabsf(v.y));
+      }
+      const int ex0 = block_exponent(am0), ex1 = block_exponent(am1);
+      const float m0 = pow2_neg(ex0), m1 = pow2_neg(ex1);
+#pragma unroll 8
+      for (int i = 0; i < 32; ++i) {
+        const float2 v = *reinterpret_cast<const float2*>(col + (rb * 32 + i) * kWPitch);
+        *reinterpret_cast<uint16_t*>(qt + (rb * 32 + i) * 128 + c) = (uint16_t)e4m3_pair(v.y * m1, v.x * m0);
+      }
+      // atom bytes (c % 32) * 16 + (c / 32) * 4 + (2 h + rb): two bytes per column here
+      sa1[c * 2 + rb] = (uint8_t)(ex0 + 127);
+      sa1[(c + 1) * 2 + rb] = (uint8_t)(ex1 + 127);
+    }
+    __syncthreads();
+    // write the q1 half tile (64 rows x 128 bytes), 16 bytes per store
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int idx = it * 128 + tid;            // 512 pieces of 16 bytes
+      const int r = idx >> 3, c16 = idx & 7;
+      *reinterpret_cast<uint4*>(q1 + (row0 + r) * Kw + col0 + c16 * 16) =
+          *reinterpret_cast<const uint4*>(qt + r * 128 + c16 * 16);
+    }
+    uint8_t* a0 = s0 + (((int64_t)e * (Rw >> 7) + rt) * (Kw >> 7) + ct) * 512;
+    uint8_t* a1 = s1 + (((int64_t)e * (Rw >> 7) + rt) * (Kw >> 7) + ct) * 512;
+    if (tid < 32) {   // s0: 8 bytes per atom row
+      *reinterpret_cast<uint2*>(a0 + tid * 16 + half * 8) = *reinterpret_cast<const uint2*>(sa0 + tid * 8);
+    } else {          // s1: 2 bytes per column, at offset (c % 32) * 16 + (c / 32) * 4 + 2 h
+      for (int c = tid - 32; c < 128; c += 96)
+        *reinterpret_cast<uint16_t*>(a1 + (c & 31) * 16 + (c >> 5) * 4 + half * 2) =
+            *reinterpret_cast<const uint16_t*>(sa1 + c * 2);
+    }
+    __syncthreads();  // the staging areas are rewritten by the next half tile
   }
 }
 
@@ -501,8 +518,14 @@ cudaError_t mxfp8_weights(const float* w, int E, int Rw, int Kw, uint8_t* q0, ui
   cudaError_t err = cudaFuncSetAttribute(mx_weights_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kWSmem);
   if (err != cudaSuccess) return err;
-  dim3 grid((unsigned)(Kw / 128), (unsigned)(Rw / 64), (unsigned)E);
-  mx_weights_kernel<<<grid, 128, kWSmem, st>>>(w, Rw, Kw, q0, s0, q1, s1);
+  // persistent: exactly as many CTAs as are resident at once (registers allow three per SM),
+  // so that every CTA runs from the start and they all finish together
+  int per_sm = 0;
+  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, mx_weights_kernel, 128, kWSmem);
+  if (err != cudaSuccess) return err;
+  const int64_t ntiles = (int64_t)E * (Rw / 64) * (Kw / 128);
+  const int grid = (int)std::min<int64_t>(ntiles, (int64_t)num_sms() * std::max(per_sm, 1));
+  mx_weights_kernel<<<grid, 128, kWSmem, st>>>(w, E, Rw, Kw, q0, s0, q1, s1);
   return cudaGetLastError();
 }
 
