@@ -67,6 +67,16 @@ typedef enum moe_status {
 
 typedef enum moe_dtype { MOE_F32 = 0, MOE_BF16 = 1, MOE_MXFP8 = 2 } moe_dtype;
 
+/* Flag OR-ed into the dw_dtype of moe_grouped_ffn_bwd / _recompute and into the dtype of
+ * moe_route_bwd: the weight gradients (dW1, dW2; dW_router) are ADDED to what the output
+ * buffers hold instead of overwriting them, for gradient accumulation over micro-batches
+ * before the one all-reduce of an optimizer step (kongchang, capacity-tax section: one
+ * gradient synchronisation per optimizer step).  fp32 outputs: each element gets exactly
+ * one fp32 addition, old + new, where new is the value the overwriting call would write
+ * (bit-identical to adding the two results afterwards); bf16 dW: old + new in fp32,
+ * rounded once to bf16. */
+#define MOE_DW_ACCUMULATE 0x100
+
 /* The problem as the pages state it: T tokens of width d_model, E experts,
  * each token routed to top_k of them, expert hidden width d_ff.
  * Limits: 1 <= top_k <= min(E, 32), E <= 1024, d_model % 8 == 0,
@@ -257,7 +267,8 @@ moe_status moe_combine_bwd(moe_shape shape, int dtype, const void* dout, const v
  *   da = dh*u*s*(1 + a*(1-s)); du = dh*silu(a);
  *   dx_perm = da W1[e,0:f] + du W1[e,f:2f];
  *   dW2[e] = dy^T h; dW1[e,0:f] = da^T x; dW1[e,f:2f] = du^T x.
- * An expert with no rows gets dW1[e] = dW2[e] = 0 (dW is overwritten).
+ * An expert with no rows gets dW1[e] = dW2[e] = 0 (dW is overwritten; with
+ * MOE_DW_ACCUMULATE in dw_dtype it is added to, and such an expert's dW is unchanged).
  * dy_perm, x_perm: [rows, d]; act_saved: [rows, 3f] from the forward;
  * dx_perm: [rows, d]; dw1: [E, 2f, d]; dw2: [E, d, f] of type dw_dtype
  * (MOE_F32 or MOE_BF16; MOE_F32 only when dtype is MOE_F32 or MOE_MXFP8).
@@ -298,7 +309,8 @@ moe_status moe_grouped_ffn_bwd_recompute(moe_shape shape, int dtype, int64_t row
  *   dx[t,:]  = sum_{j, slot_row[t,j] >= 0} dx_perm[slot_row[t,j],:] + sum_e dl[t,e] w_router[e,:]
  *   dl[t,:]  = p * (dp - <p, dp>),  p = softmax(logits[t,:]),
  *              dp[e] = dgate[t,j] where e = topk_idx[t,j], else 0
- *   dw_router = dl^T x                                   (fp32 [E, d], overwritten)
+ *   dw_router = dl^T x                                   (fp32 [E, d], overwritten;
+ *               added to instead with MOE_DW_ACCUMULATE OR-ed into dtype)
  * x, dx: [T, d]; w_router: [E, d]; logits fp32 [T,E]; dgate fp32 [T,k].
  * Deterministic: fixed summation order, no floating-point atomics. */
 moe_status moe_route_bwd(moe_shape shape, int dtype, const void* x, const void* w_router,

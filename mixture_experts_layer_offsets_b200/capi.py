@@ -18,6 +18,7 @@ HEADER = os.path.join(os.path.dirname(HERE), "include", "moe.h")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = range(5)
 MOE_F32, MOE_BF16, MOE_MXFP8 = 0, 1, 2
+MOE_DW_ACCUMULATE = 0x100   # OR into dw_dtype / the router backward's dtype: dW += ...
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
                 3: "MOE_ERR_CUDA", 4: "MOE_ERR_TIMEOUT"}
 

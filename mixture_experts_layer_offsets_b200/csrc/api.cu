@@ -214,6 +214,8 @@ moe_status ffn_bwd_entry(moe_shape s, int dtype, int64_t rows, const void* dy_pe
                          const void* w2, const void* mx, void* dx_perm, void* dw1, void* dw2,
                          int dw_dtype, void* ws, size_t ws_bytes, void* stream, bool recompute) {
   const void* act_saved = act;
+  const bool accumulate = (dw_dtype & MOE_DW_ACCUMULATE) != 0;
+  dw_dtype &= ~MOE_DW_ACCUMULATE;
   moe_status st = shape_ok(s);
   if (st != MOE_OK) return st;
   if (rows < 0 || rows >= ((int64_t)1 << 31)) return MOE_ERR_INVALID_ARG;
@@ -237,7 +239,7 @@ moe_status ffn_bwd_entry(moe_shape s, int dtype, int64_t rows, const void* dy_pe
     }
     return cuda_status(ffn_bwd_mx(fsm, dy_perm, x_perm, act_saved, offsets, w, dx_perm,
                                   static_cast<float*>(dw1), static_cast<float*>(dw2), scratch(ws),
-                                  status_word(ws), as_stream(stream)));
+                                  status_word(ws), as_stream(stream), accumulate));
   }
   if (mx) return MOE_ERR_INVALID_ARG;
   if (!dtype_act_ok(dtype)) return MOE_ERR_INVALID_ARG;
@@ -263,9 +265,10 @@ moe_status ffn_bwd_entry(moe_shape s, int dtype, int64_t rows, const void* dy_pe
                                    static_cast<const float*>(act_saved), offsets,
                                    static_cast<const float*>(w1), static_cast<const float*>(w2),
                                    static_cast<float*>(dx_perm), static_cast<float*>(dw1),
-                                   static_cast<float*>(dw2), scratch(ws), cs));
+                                   static_cast<float*>(dw2), scratch(ws), cs, accumulate));
   return cuda_status(ffn_bwd_bf16(fs, dy_perm, x_perm, act_saved, offsets, w1, w2, dx_perm, dw1,
-                                  dw2, dw_dtype == MOE_F32, scratch(ws), status_word(ws), cs));
+                                  dw2, dw_dtype == MOE_F32, scratch(ws), status_word(ws), cs,
+                                  accumulate));
 }
 
 }  // namespace
@@ -295,6 +298,8 @@ moe_status moe_route_bwd(moe_shape s, int dtype, const void* x, const void* w_ro
                          const float* logits, const int32_t* topk_idx, const float* dgate,
                          const void* dx_perm, const int32_t* slot_row, void* dx,
                          float* dw_router, void* ws, size_t ws_bytes, void* stream) {
+  const bool accumulate = (dtype & MOE_DW_ACCUMULATE) != 0;
+  dtype &= ~MOE_DW_ACCUMULATE;
   moe_status st = shape_ok(s);
   if (st != MOE_OK) return st;
   if (!dtype_act_ok(dtype)) return dtype == MOE_MXFP8 ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
@@ -304,7 +309,8 @@ moe_status moe_route_bwd(moe_shape s, int dtype, const void* x, const void* w_ro
   if (ws_bytes < kStatusBytes + route_bwd_ws_bytes(s.T, s.d_model, s.E)) return MOE_ERR_INVALID_ARG;
   return cuda_status(route_bwd_launch(dtype == MOE_BF16, x, w_router, logits, topk_idx, dgate,
                                       dx_perm, slot_row, dx, dw_router, s.T, s.d_model, s.E,
-                                      s.top_k, scratch(ws), status_word(ws), as_stream(stream)));
+                                      s.top_k, scratch(ws), status_word(ws), as_stream(stream),
+                                      accumulate));
 }
 
 moe_status moe_mx_quantize_weights(moe_shape s, const float* w1, const float* w2,

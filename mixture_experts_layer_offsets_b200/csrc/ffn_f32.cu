@@ -30,6 +30,7 @@ struct SimtGemm {
   int E;
   int group_k;
   int M, N, K;             // M fixed for GROUP_K, K fixed for GROUP_M
+  int accumulate = 0;      // C += A B^T instead of C = A B^T
 };
 
 __global__ void __launch_bounds__(256) simt_grouped_gemm(const SimtGemm p) {
@@ -103,7 +104,10 @@ __global__ void __launch_bounds__(256) simt_grouped_gemm(const SimtGemm p) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int n = n0 + tx + 16 * j;
-        if (n < p.N) C[(row_base + m) * p.c_sm + n] = acc[i][j];
+        if (n < p.N) {
+          float* c = C + (row_base + m) * p.c_sm + n;
+          *c = p.accumulate ? *c + acc[i][j] : acc[i][j];
+        }
       }
     }
   }
@@ -178,7 +182,7 @@ cudaError_t ffn_fwd_f32(const FfnShape& s, const float* x_perm, const int32_t* o
 cudaError_t ffn_bwd_f32(const FfnShape& s, const float* dy_perm, const float* x_perm,
                         const float* act, const int32_t* offsets, const float* w1,
                         const float* w2, float* dx_perm, float* dw1, float* dw2, void* scratch,
-                        cudaStream_t st) {
+                        cudaStream_t st, bool accumulate) {
   const int d = s.d, f = s.f, E = s.E;
   float* dadu = static_cast<float*>(scratch);
   cudaError_t err;
@@ -194,11 +198,11 @@ cudaError_t ffn_bwd_f32(const FfnShape& s, const float* dy_perm, const float* x_
   }
   // dW2[e] = dy^T h:  A(m=c of d, k=row) = dy[k][m];  B(n=c of f, k=row) = h[k][n]
   SimtGemm g3{dy_perm, 1, d, act + 2 * f, 1, 3 * f, 0, dw2, f, (int64_t)d * f, offsets, E, 1,
-              d, f, 0};
+              d, f, 0, accumulate};
   if ((err = run(g3, (int64_t)E * ((d + 63) / 64) * ((f + 63) / 64), st)) != cudaSuccess) return err;
   // dW1[e] = [da|du]^T x:  A(m=c of 2f, k=row) = dadu[k][m];  B(n=c of d, k=row) = x[k][n]
   SimtGemm g4{dadu, 1, 2 * f, x_perm, 1, d, 0, dw1, d, (int64_t)2 * f * d, offsets, E, 1,
-              2 * f, d, 0};
+              2 * f, d, 0, accumulate};
   return run(g4, (int64_t)E * ((2 * f + 63) / 64) * ((d + 63) / 64), st);
 }
 

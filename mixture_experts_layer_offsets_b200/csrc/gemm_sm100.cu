@@ -82,6 +82,7 @@ struct GemmParams {
   const __nv_bfloat16* act;
   int64_t ld_act;
   int64_t out_group;       // EPI_WGRAD: elements per expert
+  int accumulate;          // EPI_WGRAD: add into the output instead of overwriting it
   int* status;
   // EPI_ROUTER (one group of rows_total tokens; N = number of experts)
   int rows_total;
@@ -300,6 +301,16 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* tm, int x, int y
                    reinterpret_cast<uint64_t>(tm)),
                "r"(x), "r"(y), "r"(smem_u32(smem_src))
                : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// The same box added element-wise into global memory (fp32 adds in L2, one per element)
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* tm, int x, int y,
+                                                  const void* smem_src) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+          reinterpret_cast<uint64_t>(tm)),
+      "r"(x), "r"(y), "r"(smem_u32(smem_src))
+      : "memory");
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
 __device__ __forceinline__ void tma_store_wait_read() {
@@ -1210,11 +1221,47 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
               }
               fence_proxy_async_smem();
               __syncwarp();
-              if (lane == 0)
-                tma_store_2d(tmo, ti.n0 + (c0 + ci) * 32, (int)(orow0 + 16 * hh), sbuf);
+              if (lane == 0) {
+                // a partial sum always overwrites its slot; the result is added into the
+                // output when the call accumulates
+                if (p.accumulate && !partial)
+                  tma_reduce_add_2d(tmo, ti.n0 + (c0 + ci) * 32, (int)(orow0 + 16 * hh), sbuf);
+                else
+                  tma_store_2d(tmo, ti.n0 + (c0 + ci) * 32, (int)(orow0 + 16 * hh), sbuf);
+              }
               ++slot;
             }
           }
+        } else if (p.accumulate) {
+          // bf16 output added to: existing + new in fp32, rounded once, chunk by chunk
+          __nv_bfloat16* o = p.out + (orow0 + lane) * p.ld_out + ti.n0 + c0 * 32;
+#pragma unroll 1
+          for (int ci = 0; ci < kMine; ++ci) {
+            uint32_t v[32];
+            if (ti.nkb > 0) {
+              tmem_ld32(ta + (c0 + ci) * 32, v);
+              tmem_wait_ld();
+              tmem_tie(v);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] = 0;
+            }
+            const uint4* src = reinterpret_cast<const uint4*>(o + ci * 32);
+            uint32_t pk[16];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const uint4 w = src[q4];
+              const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                const int i = 4 * q4 + h;
+                pk[i] = pack_bf16(bf_lo(ww[h]) + __uint_as_float(v[2 * i]),
+                                  bf_hi(ww[h]) + __uint_as_float(v[2 * i + 1]));
+              }
+            }
+            store_64B(o + ci * 32, pk);
+          }
+          release();
         } else {
           __nv_bfloat16* o = p.out + (orow0 + lane) * p.ld_out + ti.n0 + c0 * 32;
           uint32_t pk[kMine][16];
@@ -1257,7 +1304,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
 __global__ void __launch_bounds__(256)
 wgrad_reduce_kernel(const int32_t* __restrict__ offsets, int kc, int64_t mn4,
                     const float4* __restrict__ part, float4* __restrict__ out32,
-                    __nv_bfloat16* __restrict__ out16) {
+                    __nv_bfloat16* __restrict__ out16, int accumulate) {
   __shared__ int s_red[8];
   const int g = blockIdx.y;
   int ns, ck;
@@ -1283,13 +1330,24 @@ wgrad_reduce_kernel(const int32_t* __restrict__ offsets, int kc, int64_t mn4,
       const float4 b = src[(int64_t)j * mn4 + i];
       a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
     }
+    // the K ranges are summed first; an accumulating call then adds that sum to the output
     if (out32) {
-      out32[(int64_t)g * mn4 + i] = a;
+      float4* o = out32 + (int64_t)g * mn4 + i;
+      if (accumulate) {
+        const float4 b = *o;
+        a = make_float4(b.x + a.x, b.y + a.y, b.z + a.z, b.w + a.w);
+      }
+      *o = a;
     } else {
+      uint2* o = reinterpret_cast<uint2*>(out16 + ((int64_t)g * mn4 + i) * 4);
+      if (accumulate) {
+        const uint2 b = *o;
+        a = make_float4(bf_lo(b.x) + a.x, bf_hi(b.x) + a.y, bf_lo(b.y) + a.z, bf_hi(b.y) + a.w);
+      }
       uint2 pk;
       pk.x = pack_bf16(a.x, a.y);
       pk.y = pack_bf16(a.z, a.w);
-      *reinterpret_cast<uint2*>(out16 + ((int64_t)g * mn4 + i) * 4) = pk;
+      *o = pk;
     }
   }
 }
@@ -1444,7 +1502,7 @@ cudaError_t wgrad_reduce_launch(const GemmParams& p, int64_t M, int64_t N, float
   const int64_t mn4 = M * N / 4;
   dim3 grid((unsigned)std::min<int64_t>((mn4 + 255) / 256, 16), (unsigned)p.E);
   wgrad_reduce_kernel<<<grid, 256, 0, st>>>(p.offsets, p.kchunk, mn4, reinterpret_cast<const float4*>(p.part),
-                                            reinterpret_cast<float4*>(out32), out16);
+                                            reinterpret_cast<float4*>(out32), out16, p.accumulate);
   return cudaGetLastError();
 }
 
@@ -1578,7 +1636,8 @@ cudaError_t ffn_fwd_bf16(const FfnShape& s, const void* x_perm, const int32_t* o
 cudaError_t ffn_bwd_bf16(const FfnShape& s, const void* dy_perm, const void* x_perm,
                          const void* act, const int32_t* offsets, const void* w1, const void* w2,
                          void* dx_perm, void* dw1, void* dw2, bool dw_f32, void* scratch,
-                         int* status, cudaStream_t st) {
+                         int* status, cudaStream_t st,
+                         bool accumulate) {
   cudaError_t err = get_encode();
   if (err != cudaSuccess) return err;
   const int d = s.d, f = s.f, E = s.E;
@@ -1618,7 +1677,7 @@ cudaError_t ffn_bwd_bf16(const FfnShape& s, const void* dy_perm, const void* x_p
     return cudaErrorInvalidValue;
   p5.M = d; p5.N = f;
   p5.out = static_cast<__nv_bfloat16*>(dw2); p5.out_f32 = dw_f32 ? static_cast<float*>(dw2) : nullptr;
-  p5.ld_out = f; p5.out_group = (int64_t)d * f;
+  p5.ld_out = f; p5.out_group = (int64_t)d * f; p5.accumulate = accumulate;
   if (dw_f32 && !tmap(&p5.tmOut, dw2, f, (uint64_t)E * d, f, 32, 16, true)) return cudaErrorInvalidValue;
   float* part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(scratch) +
                                          align256((size_t)s.rows * 2 * f * 2));
@@ -1634,7 +1693,7 @@ cudaError_t ffn_bwd_bf16(const FfnShape& s, const void* dy_perm, const void* x_p
     return cudaErrorInvalidValue;
   p6.M = 2 * f; p6.N = d;
   p6.out = static_cast<__nv_bfloat16*>(dw1); p6.out_f32 = dw_f32 ? static_cast<float*>(dw1) : nullptr;
-  p6.ld_out = d; p6.out_group = (int64_t)2 * f * d;
+  p6.ld_out = d; p6.out_group = (int64_t)2 * f * d; p6.accumulate = accumulate;
   if (dw_f32 && !tmap(&p6.tmOut, dw1, d, (uint64_t)E * 2 * f, d, 32, 16, true)) return cudaErrorInvalidValue;
   wgrad_setup(&p6, s.rows, 2 * f, d, false, part);
   if (!p6.part) return cudaErrorInvalidValue;
@@ -1793,7 +1852,8 @@ cudaError_t mx_dispatch(const FfnShape& s, const void* x, const int32_t* perm_sr
 
 cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_perm, const void* act,
                        const int32_t* offsets, const MxWeights& w, void* dx_perm, float* dw1,
-                       float* dw2, void* scratch, int* status, cudaStream_t st) {
+                       float* dw2, void* scratch, int* status, cudaStream_t st,
+                       bool accumulate) {
   cudaError_t err = get_encode();
   if (err != cudaSuccess) return err;
   const int d = s.d, f = s.f, E = s.E;
@@ -1852,7 +1912,7 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
   p5.sfa = ws + L.sdy1;
   p5.sfb = ws + L.sh1;
   p5.M = d; p5.N = f;
-  p5.out_f32 = dw2; p5.ld_out = f; p5.out_group = (int64_t)d * f;
+  p5.out_f32 = dw2; p5.ld_out = f; p5.out_group = (int64_t)d * f; p5.accumulate = accumulate;
   wgrad_setup(&p5, R, d, f, true, reinterpret_cast<float*>(ws + L.part));
   if (!p5.part) return cudaErrorInvalidValue;
   if ((err = launch_mx_n<true, true, EPI_WGRAD, true>(p5, f, num_sms(), st)) != cudaSuccess ||
@@ -1867,7 +1927,7 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
   p6.sfa = ws + L.sda1;
   p6.sfb = ws + L.sx1;
   p6.M = 2 * f; p6.N = d;
-  p6.out_f32 = dw1; p6.ld_out = d; p6.out_group = (int64_t)2 * f * d;
+  p6.out_f32 = dw1; p6.ld_out = d; p6.out_group = (int64_t)2 * f * d; p6.accumulate = accumulate;
   wgrad_setup(&p6, R, 2 * f, d, true, reinterpret_cast<float*>(ws + L.part));
   if (!p6.part) return cudaErrorInvalidValue;
   if ((err = launch_mx_n<true, true, EPI_WGRAD, true>(p6, d, num_sms(), st)) != cudaSuccess) return err;

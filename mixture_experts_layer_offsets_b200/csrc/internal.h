@@ -67,7 +67,8 @@ cudaError_t route_bwd_tc_launch(const void* x, const void* w_router, const void*
 cudaError_t route_bwd_launch(bool bf16, const void* x, const void* w_router, const float* logits,
                              const int32_t* topk_idx, const float* dgate, const void* dx_perm,
                              const int32_t* slot_row, void* dx, float* dw_router, int T, int d,
-                             int E, int k, void* scratch, int* status, cudaStream_t st);
+                             int E, int k, void* scratch, int* status, cudaStream_t st,
+                             bool accumulate = false);
 
 // ----------------------------------------------------------------- MXFP8
 cudaError_t mxfp8_launch(int64_t rows, int64_t K, bool src_bf16, const void* src, int axis,
@@ -118,7 +119,7 @@ cudaError_t ffn_fwd_f32(const FfnShape& s, const float* x_perm, const int32_t* o
 cudaError_t ffn_bwd_f32(const FfnShape& s, const float* dy_perm, const float* x_perm,
                         const float* act, const int32_t* offsets, const float* w1,
                         const float* w2, float* dx_perm, float* dw1, float* dw2, void* scratch,
-                        cudaStream_t st);
+                        cudaStream_t st, bool accumulate = false);
 // bf16 path: tcgen05 tensor-core grouped GEMMs
 cudaError_t ffn_fwd_bf16(const FfnShape& s, const void* x_perm, const int32_t* offsets,
                          const void* w1, const void* w2, void* act, void* y_perm, int* status,
@@ -126,7 +127,7 @@ cudaError_t ffn_fwd_bf16(const FfnShape& s, const void* x_perm, const int32_t* o
 cudaError_t ffn_bwd_bf16(const FfnShape& s, const void* dy_perm, const void* x_perm,
                          const void* act, const int32_t* offsets, const void* w1, const void* w2,
                          void* dx_perm, void* dw1, void* dw2, bool dw_f32, void* scratch,
-                         int* status, cudaStream_t st);
+                         int* status, cudaStream_t st, bool accumulate = false);
 
 // MXFP8 path: E4M3 operands with E8M0 scales (see include/moe.h, moe_mx_weights)
 struct MxWeights {
@@ -140,7 +141,9 @@ cudaError_t ffn_fwd_mx(const FfnShape& s, const void* x_perm, const int32_t* off
                        cudaStream_t st);
 cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_perm, const void* act,
                        const int32_t* offsets, const MxWeights& w, void* dx_perm, float* dw1,
-                       float* dw2, void* scratch, int* status, cudaStream_t st);
+                       float* dw2, void* scratch, int* status, cudaStream_t st,
+                       bool accumulate = false);
+// (accumulate: the weight gradients are added into dw1, dw2 instead of overwriting them)
 
 int num_sms();
 

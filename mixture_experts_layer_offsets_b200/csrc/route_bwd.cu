@@ -192,12 +192,12 @@ dwr_partial_kernel(const float* __restrict__ dl, const T* __restrict__ x,
 }
 
 __global__ void dwr_reduce_kernel(const float* __restrict__ partial, float* __restrict__ dw,
-                                  int64_t n, int splits) {
+                                  int64_t n, int splits, int accumulate) {
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
     float v = 0.f;
     for (int s = 0; s < splits; ++s) v += partial[(int64_t)s * n + i];
-    dw[i] = v;
+    dw[i] = accumulate ? dw[i] + v : v;  // the splits are summed first, then added
   }
 }
 
@@ -205,7 +205,7 @@ template <typename T>
 cudaError_t route_bwd_t(const void* x, const void* w_router, const float* logits,
                         const int32_t* topk_idx, const float* dgate, const void* dx_perm,
                         const int32_t* slot_row, void* dx, float* dw_router, int T_, int d, int E,
-                        int k, void* scratch, int* status, cudaStream_t st) {
+                        int k, void* scratch, int* status, cudaStream_t st, bool accumulate) {
   constexpr int V = Vec16<T>::N;
   constexpr int EB = 8;
   const int splits = route_bwd_splits(T_);
@@ -229,7 +229,7 @@ cudaError_t route_bwd_t(const void* x, const void* w_router, const float* logits
                               k, status, st);
     if (err != cudaSuccess) return err;
     dwr_reduce_kernel<<<(int)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, st>>>(
-        partial, dw_router, n, tsplits);
+        partial, dw_router, n, tsplits, accumulate);
     return cudaGetLastError();
   }
   if (T_ > 0) {
@@ -248,8 +248,8 @@ cudaError_t route_bwd_t(const void* x, const void* w_router, const float* logits
     dwr_partial_kernel<T, EB><<<g2, 256, 0, st>>>(dl, static_cast<const T*>(x), partial, T_, d,
                                                   E, tps);
     dwr_reduce_kernel<<<(int)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, st>>>(
-        partial, dw_router, n, splits);
-  } else {
+        partial, dw_router, n, splits, accumulate);
+  } else if (!accumulate) {
     cudaMemsetAsync(dw_router, 0, n * sizeof(float), st);
   }
   return cudaGetLastError();
@@ -266,12 +266,13 @@ size_t route_bwd_ws_bytes(int T, int d, int E) {
 cudaError_t route_bwd_launch(bool bf16, const void* x, const void* w_router, const float* logits,
                              const int32_t* topk_idx, const float* dgate, const void* dx_perm,
                              const int32_t* slot_row, void* dx, float* dw_router, int T, int d,
-                             int E, int k, void* scratch, int* status, cudaStream_t st) {
+                             int E, int k, void* scratch, int* status, cudaStream_t st,
+                             bool accumulate) {
   if (bf16)
     return route_bwd_t<__nv_bfloat16>(x, w_router, logits, topk_idx, dgate, dx_perm, slot_row, dx,
-                                      dw_router, T, d, E, k, scratch, status, st);
+                                      dw_router, T, d, E, k, scratch, status, st, accumulate);
   return route_bwd_t<float>(x, w_router, logits, topk_idx, dgate, dx_perm, slot_row, dx,
-                            dw_router, T, d, E, k, scratch, status, st);
+                            dw_router, T, d, E, k, scratch, status, st, accumulate);
 }
 
 }  // namespace moe

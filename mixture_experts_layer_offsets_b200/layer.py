@@ -166,8 +166,11 @@ class MoELayer:
         capi.moe_combine(s, dt, self.y_perm, self.row_map, self.combine_gate, self.out, stream)
         return self.out
 
-    def backward(self, dout, x, w_router, w1, w2, stream=None):
+    def backward(self, dout, x, w_router, w1, w2, stream=None, accumulate: bool = False):
+        """With ``accumulate`` the weight gradients are added to dw1, dw2 and dw_router
+        (gradient accumulation over micro-batches) instead of overwriting them."""
         s, dt = self.shape, self.cdtype
+        acc = capi.MOE_DW_ACCUMULATE if accumulate else 0
         capi.moe_combine_bwd(s, dt, dout, self.y_perm, self.row_map, self.combine_gate,
                              self.dy_perm, self.dgate_rn if self.renorm else self.dgate, stream)
         if self.renorm:
@@ -175,15 +178,15 @@ class MoELayer:
         bwd = capi.moe_grouped_ffn_bwd_recompute if self.recompute else capi.moe_grouped_ffn_bwd
         xp = None if self.fused_dispatch else self.x_perm
         bwd(s, self.ffn_dtype, self.rows, self.dy_perm, xp, self.act, self.ffn_offsets,
-            w1, w2, self.dx_perm, self.dw1, self.dw2, _DT[self.dw_dtype], self.ws, mx=self.mx,
+            w1, w2, self.dx_perm, self.dw1, self.dw2, _DT[self.dw_dtype] | acc, self.ws, mx=self.mx,
             stream=stream)
-        capi.moe_route_bwd(s, dt, x, w_router, self.logits, self.topk_idx, self.dgate,
+        capi.moe_route_bwd(s, dt | acc, x, w_router, self.logits, self.topk_idx, self.dgate,
                            self.dx_perm, self.row_map, self.dx, self.dw_router, self.ws, stream)
         return self.dx
 
-    def step(self, x, w_router, bias, w1, w2, dout, stream=None):
+    def step(self, x, w_router, bias, w1, w2, dout, stream=None, accumulate: bool = False):
         self.forward(x, w_router, bias, w1, w2, stream)
-        return self.backward(dout, x, w_router, w1, w2, stream)
+        return self.backward(dout, x, w_router, w1, w2, stream, accumulate)
 
     def routing_stats(self, capacity: int | None = None, stream=None):
         """Load statistics of the last forward's routing, on the device (fp32 [8]):

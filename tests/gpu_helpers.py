@@ -78,3 +78,34 @@ def check_recompute_bit_exact(cfg):
     assert torch.equal(act, a_act), "the recompute did not restore a | u | h"
     for key in ("out", "dgate", "dx_perm", "dw1", "dw2", "dx", "dw_router"):
         assert torch.equal(getattr(A, key), getattr(L0, key)), key
+
+
+def check_accumulate(cfg, dw_dtype="f32"):
+    """A layer that steps on batch A, then on batch B with MOE_DW_ACCUMULATE, holds the sum of
+    the weight gradients of two layers that each stepped on one batch.  fp32 weight gradients
+    get one fp32 addition per element, so the sum is exact against torch's fp32 addition
+    (subnormal results aside); bf16 ones are rounded once, within the bf16 tolerance."""
+    _, A = run_layer(cfg, seed=0, dw_dtype=dw_dtype)
+    _, B = run_layer(cfg, seed=1, dw_dtype=dw_dtype)
+    dev = lambda d: {k: (v.cuda() if v is not None else None) for k, v in d.items()}
+    a_in = dev(inputs.make_inputs(cfg, device="cpu", seed=0))
+    b_in = dev(inputs.make_inputs(cfg, device="cpu", seed=1))
+    C = MoELayer(cfg.T, cfg.d_model, cfg.E, cfg.top_k, cfg.d_ff, cfg.dtype, "cuda", dw_dtype=dw_dtype)
+    args = lambda i: (i["x"], i["w_router"], i["bias"], i["w1"], i["w2"], i["dout"])
+    C.step(*args(a_in))
+    C.step(*args(b_in), accumulate=True)
+    torch.cuda.synchronize()
+    assert C.device_status() == 0
+    keys = ("dw1", "dw2", "dw_router")
+    for key in keys:
+        got, a, b = getattr(C, key), getattr(A, key), getattr(B, key)
+        if got.dtype == torch.float32:
+            want = a + b
+            diff = got != want
+            # only a subnormal sum may differ (flushed to zero by the reducing store)
+            assert not diff.any() or bool((want[diff].abs() < 1.2e-38).all()), key
+        else:
+            want = a.double() + b.double()
+            assert rel(f64(got), want.cpu().numpy()) <= TOL["bf16"], key
+    # the step that accumulated still computed its own non-gradient outputs normally
+    assert torch.equal(C.out, B.out) and torch.equal(C.dx, B.dx)

@@ -12,7 +12,8 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import TOL, check_recompute_bit_exact, f64, i64, oracle_for, rel, run_layer
+from gpu_helpers import (TOL, check_accumulate, check_recompute_bit_exact, f64, i64, oracle_for,
+                         rel, run_layer)
 from mixture_experts_layer_offsets_b200.inputs import CONFIGS, shrink
 from oracle import moe_ref as ref
 
@@ -208,3 +209,10 @@ def test_renorm_kernels_match_oracle_directly():
 @pytest.mark.parametrize("name", ["bf16_e8_small", "bf16_skew_split", "tiny_f32", "f32_one_token"])
 def test_recompute_with_shared_buffers_is_bit_exact(name):
     check_recompute_bit_exact(CASES[name])
+
+
+@pytest.mark.parametrize("name,dw", [("bf16_e8_small", "f32"), ("bf16_skew_split", "f32"),
+                                     ("bf16_e128_small", "f32"), ("tiny_f32", "f32"),
+                                     ("bf16_e8_small", "bf16"), ("bf16_skew_split", "bf16")])
+def test_accumulated_weight_grads_are_the_sum_of_two_steps(name, dw):
+    check_accumulate(CASES[name], dw_dtype=dw)

@@ -14,7 +14,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import TOL, check_recompute_bit_exact, f64, i64, rel, run_layer
+from gpu_helpers import TOL, check_accumulate, check_recompute_bit_exact, f64, i64, rel, run_layer
 from mixture_experts_layer_offsets_b200.inputs import CONFIGS, shrink
 from oracle import moe_mx_ref as mxr
 from oracle import mxfp8_ref as mx
@@ -153,3 +153,8 @@ def test_fused_dispatch_is_bit_identical_to_permute_then_quantise(name):
         if key in ("perm_src", "act", "y_perm", "dx_perm"):
             a, b = a[:cfg.R], b[:cfg.R]
         assert torch.equal(a, b), key
+
+
+@pytest.mark.parametrize("name", ["mx_e8", "mx_skew_split"])
+def test_mxfp8_accumulated_weight_grads_are_the_sum_of_two_steps(name):
+    check_accumulate(CASES[name])
