@@ -1519,13 +1519,15 @@ GemmParams base_params(const FfnShape& s, const int32_t* offsets, int* status) {
 int64_t m_tile_bound(const FfnShape& s) { return s.rows / BM + s.E; }
 int64_t pair_tile_bound(const FfnShape& s) { return s.rows / (2 * BM) + s.E; }
 
-// CTA pairs (256-row tiles) pay off when experts hold many rows; with few rows
-// per expert the ragged last tile wastes more.  MOE_B200_PAIR=0/1 forces a mode.
+// CTA pairs (256-row tiles, each weight tile read once per pair) pay off when experts hold
+// a few hundred rows or more; with fewer the ragged last tile of every expert wastes more
+// (at 512 rows per expert pairs still took 2 % off the step).  MOE_B200_PAIR=0/1 forces
+// a mode.
 bool use_pairs(const FfnShape& s) {
-  const char* env = getenv("MOE_B200_PAIR");
+  const char* env = getenv("MOE_B200_PAIR");  // read per call: tests switch it
   if (env && env[0] == '0') return false;
   if (env && env[0] == '1') return true;
-  return s.E > 0 && s.rows / s.E >= 1024;
+  return s.E > 0 && s.rows / s.E >= 512;
 }
 
 template <int BN>
