@@ -64,6 +64,14 @@ enum : int {
 };
 
 constexpr int kRouterKMax = 8;  // top-k kept in registers by the router epilogue
+// MXFP8 CTA pairs: where the B scales of a 256-column tile sit.  0 (used): each CTA's
+// TMEM holds the scales of all 256 columns, as the pair's block-scaled MMA reads them;
+// 1: each CTA holds those of its own B half only.  On a B200 the second gives results
+// far from the single-CTA tiles, the first gives the same bits.
+#ifndef MOE_PAIR_SFB_SPLIT
+#define MOE_PAIR_SFB_SPLIT 0
+#endif
+constexpr bool kPairSfbSplit = MOE_PAIR_SFB_SPLIT != 0;
 
 struct GemmParams {
   CUtensorMap tmA;
@@ -103,6 +111,9 @@ struct GemmParams {
   int kchunk;
   float* part;
   CUtensorMap tmPart;
+  // MXFP8 CTA pairs: the scale atoms as [2 x atoms, 256] byte tensors (box 256 x 2 = one
+  // atom), so that they load with the pair's TMA form onto the leader's barrier
+  CUtensorMap tmSfa, tmSfb;
   // Failure-path test hooks (0 = off): the limit of every bounded wait, and a ring
   // iteration at which CTA 0's producer skips its loads and its arrival, so that the MMA
   // warp's wait runs out (see gemm_test_hooks).
@@ -124,8 +135,11 @@ template <int BN, bool PAIR = false, int EPI = 1, bool FP8 = false> struct Cfg {
   // slots of 8 TMEM columns after the accumulators.
   static constexpr int kBKe = FP8 ? 128 : BK;  // K elements per stage
   static constexpr uint32_t kBBytes = (PAIR ? BN / 2 : BN) * 128;
-  // FP8: A atom (512 B) + BN/128 B atoms, padded to keep stages 1024-byte aligned
-  static constexpr uint32_t kSfBytes = FP8 ? ((512 + (BN / 128) * 512 + 1023) / 1024) * 1024 : 0;
+  // FP8: A atom (512 B) + the B atoms (BN/128 of them; a CTA of a pair holding the scales
+  // of its own B half takes one), padded to keep stages 1024-byte aligned
+  static constexpr uint32_t kSfB = (PAIR && kPairSfbSplit) ? 512 : (BN / 128) * 512;
+  static constexpr uint32_t kSfLoad = FP8 ? 512 + kSfB : 0;   // bytes loaded per stage
+  static constexpr uint32_t kSfBytes = FP8 ? ((kSfLoad + 1023) / 1024) * 1024 : 0;
   static constexpr uint32_t kStage = kABytes + kBBytes + kSfBytes;
   static_assert(kStage % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
   // accumulator buffers: two (the epilogue of one tile overlaps the main loop of the
@@ -230,6 +244,18 @@ __device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a, uint
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a), "l"(b), "r"(idesc), "r"(accum));
+}
+__device__ __forceinline__ void umma_mxf8_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                               uint32_t accum, uint32_t tsfa, uint32_t tsfb) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accum), "r"(tsfa), "r"(tsfb));
+}
+// each CTA of the pair copies the atom at this shared-memory offset into its own TMEM
+__device__ __forceinline__ void tmem_cp_sf_pair(uint32_t taddr, uint64_t sdesc_src) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc_src)
+               : "memory");
 }
 // Arrive on the barrier at this offset in both CTAs of the pair once the MMAs are done.
 __device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
@@ -468,7 +494,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
   using C = Cfg<BN, PAIR, EPI, FP8>;
   const uint64_t wl = p.wait_ns ? p.wait_ns : (uint64_t)MOE_WAIT_NS;  // bounded-wait limit
-  static_assert(!FP8 || ((BN == 128 || BN == 256) && !PAIR), "MXFP8 tiles: 128 x 128 or 128 x 256, single CTA");
+  static_assert(!FP8 || ((BN == 128 || BN == 256) && (!PAIR || BN == 256)),
+                "MXFP8 tiles: 128 x 128 or 128 x 256, or 256 x 256 on a CTA pair");
   static_assert(!FP8 || EPI != EPI_SWIGLU_FWD || BN == 256, "MXFP8 SwiGLU tiles pair 128 gate with 128 up columns");
   // epilogue warps 6..9 idle when a thread must hold a whole row (router)
   constexpr bool kHalfIdle = EPI == EPI_ROUTER;
@@ -544,6 +571,22 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
         run += ((s_off[g + 1] - s_off[g] + C::kTileM - 1) / C::kTileM) * nN;
       }
       if (lane == 31) s_pre[E] = incl;
+      if constexpr (FP8 && PAIR) {
+        // the A scale atoms are numbered per 128-row tile of each expert
+        int s1 = 0;
+        for (int g = lo; g < hi; ++g) s1 += (s_off[g + 1] - s_off[g] + BM - 1) / BM;
+        int incl1 = s1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int n = __shfl_up_sync(0xffffffffu, incl1, o);
+          if (lane >= o) incl1 += n;
+        }
+        int run1 = incl1 - s1;
+        for (int g = lo; g < hi; ++g) {
+          s_sel[g] = run1;
+          run1 += (s_off[g + 1] - s_off[g] + BM - 1) / BM;
+        }
+      }
     }
   }
   if constexpr (GROUP_K) {
@@ -619,6 +662,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
       uint32_t ph = 1;  // the first pass over the ring finds every stage free
       bool ok = true;
       const int kq = GROUP_K ? 0 : p.K / C::kBKe;
+      const uint32_t leader_full = PAIR ? map_to_rank(&full[0], 0) : 0;
       for (int t = tile0; t < total && ok; t += tstride) {
         if (*s_abort) { ok = false; break; }
         const TileInfo ti = decode(t);
@@ -648,13 +692,52 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
             atomB = p.sfb + ((int64_t)ti.g * kq * (p.N / 128) + ti.n0 / 128) * 512;
           }
         }
+        // CTA pairs: atom indices (the atom tensors' row is twice the index).  A: this CTA's
+        // 128-row tile of its expert; B: the CTA's own half of the 256 columns, or both.
+        int64_t pa0 = 0, pb0 = 0, pb1 = 0;
+        if constexpr (PAIR) {
+          pa0 = ((int64_t)s_sel[ti.g] + (ti.m0 - s_off[ti.g]) / BM) * kq;
+          if constexpr (!B_MN) {
+            const int ntiles = p.b_rows / 128;
+            const int t0 = EPI == EPI_SWIGLU_FWD ? ti.n0 / 128 : ti.n0 / 128;
+            const int t1 = EPI == EPI_SWIGLU_FWD ? (p.f + ti.n0) / 128 : ti.n0 / 128 + 1;
+            pb0 = ((int64_t)ti.g * ntiles + t0) * kq;
+            pb1 = ((int64_t)ti.g * ntiles + t1) * kq;
+          } else {
+            pb0 = (int64_t)ti.g * kq * (p.N / 128) + ti.n0 / 128;
+            pb1 = pb0 + 1;
+          }
+          if constexpr (kPairSfbSplit) {
+            if (rank == 1) pb0 = pb1;
+          }
+        }
         for (int kb = 0; kb < ti.nkb; ++kb, ++it, s = (s + 1 == S ? 0 : s + 1), ph ^= (s == 0)) {
           if (!mbar_wait(&empty[s], ph, wl)) { fail(); ok = false; break; }
-          if (p.drop_it && blockIdx.x == 0 && it + 1 == (uint32_t)p.drop_it) continue;  // test hook
+          if (!PAIR && p.drop_it && blockIdx.x == 0 && it + 1 == (uint32_t)p.drop_it) continue;  // test hook
           uint8_t* sa = smem + s * C::kStage;
           uint8_t* sb = sa + kABytes;
           uint8_t* sf = sb + C::kBBytes;
           const int kc = kb * C::kBKe;  // first K element of the stage
+          if constexpr (PAIR) {
+            // every load of both CTAs completes on the leader's barrier; only the leader arrives
+            if (leader) mbar_arrive_expect_tx(&full[s], 2 * (kABytes + C::kBBytes + C::kSfLoad));
+            const uint32_t bar = leader_full + 8 * s;
+            tma_load_2d_pair(sa, &p.tmA, kc, ti.m0, bar);
+            if constexpr (!B_MN) {
+              const int row = ti.kbase + (EPI == EPI_SWIGLU_FWD ? (rank == 0 ? ti.n0 : p.f + ti.n0)
+                                                               : ti.n0 + 128 * (int)rank);
+              tma_load_2d_pair(sb, &p.tmB, kc, row, bar);
+            } else {
+              tma_load_2d_pair(sb, &p.tmB, ti.n0 + 128 * (int)rank, ti.kbase + kc, bar);
+            }
+            // MN-major B atoms of one stage are N/128 apart in k; K-major ones 1 apart
+            const int64_t bstep = B_MN ? (int64_t)kb * (p.N / 128) : (int64_t)kb;
+            tma_load_2d_pair(sf, &p.tmSfa, 0, (int)(2 * (pa0 + kb)), bar);
+            tma_load_2d_pair(sf + 512, &p.tmSfb, 0, (int)(2 * (pb0 + bstep)), bar);
+            if constexpr (!kPairSfbSplit)
+              tma_load_2d_pair(sf + 1024, &p.tmSfb, 0, (int)(2 * (pb1 + bstep)), bar);
+            continue;
+          }
           constexpr uint32_t kSfB = (BN / 128) * 512;
           mbar_arrive_expect_tx(&full[s], kABytes + C::kBBytes + 512 + kSfB);
           if constexpr (!A_MN) tma_load_2d(sa, &p.tmA, kc, ti.m0, &full[s]);
@@ -765,7 +848,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
                                ((uint32_t)B_MN << 16) | ((uint32_t)(BN >> 3) << 17) |
                                ((uint32_t)(C::kTileM >> 4) << 24);
     constexpr uint32_t idesc_mx = ((uint32_t)A_MN << 15) | ((uint32_t)B_MN << 16) |
-                                  ((uint32_t)(BN >> 3) << 17) | (1u << 23) | ((uint32_t)(BM >> 4) << 24);
+                                  ((uint32_t)(BN >> 3) << 17) | (1u << 23) | ((uint32_t)(C::kTileM >> 4) << 24);
     // MN-major operands: LBO = distance between 64 (bf16) or 128 (fp8) element MN blocks
     constexpr uint32_t kLboA = A_MN ? (FP8 ? 16384 : 8192) : 16;
     constexpr uint32_t kLboB = B_MN ? (FP8 ? 16384 : 8192) : 16;
@@ -835,16 +918,31 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
             // stage's scales does not write columns that MMAs still in flight read; the
             // scales of B atom i (rows 128 i ..) sit 4 i columns after the first.
             const uint32_t tsf = tmem_base + C::kSfCol + 16 * (it & 7);
-            tmem_cp_sf(tsf, desc_f0 + so);
+            if constexpr (PAIR) {
+              // each CTA copies its own atoms into its own TMEM; the leader's MMAs then
+              // read both CTAs' A rows, B halves and scales
+              tmem_cp_sf_pair(tsf, desc_f0 + so);
 #pragma unroll
-            for (int i = 0; i < BN / 128; ++i)
-              tmem_cp_sf(tsf + 4 + 4 * i, desc_f0 + so + ((512 + 512 * i) >> 4));
+              for (int i = 0; i < (kPairSfbSplit ? 1 : 2); ++i)
+                tmem_cp_sf_pair(tsf + 4 + 4 * i, desc_f0 + so + ((512 + 512 * i) >> 4));
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              umma_mxf8(d_tmem, ad + k * kStepA, bd + k * kStepB,
-                        idesc_mx | ((uint32_t)k << 4) | ((uint32_t)k << 29), (kb | k) != 0,
-                        tsf | ((uint32_t)k << 30), (tsf + 4) | ((uint32_t)k << 30));
-            umma_commit(&empty[stg]);
+              for (int k = 0; k < 4; ++k)
+                umma_mxf8_pair(d_tmem, ad + k * kStepA, bd + k * kStepB,
+                               idesc_mx | ((uint32_t)k << 4) | ((uint32_t)k << 29), (kb | k) != 0,
+                               tsf | ((uint32_t)k << 30), (tsf + 4) | ((uint32_t)k << 30));
+              umma_commit_pair(&empty[stg]);
+            } else {
+              tmem_cp_sf(tsf, desc_f0 + so);
+#pragma unroll
+              for (int i = 0; i < BN / 128; ++i)
+                tmem_cp_sf(tsf + 4 + 4 * i, desc_f0 + so + ((512 + 512 * i) >> 4));
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                umma_mxf8(d_tmem, ad + k * kStepA, bd + k * kStepB,
+                          idesc_mx | ((uint32_t)k << 4) | ((uint32_t)k << 29), (kb | k) != 0,
+                          tsf | ((uint32_t)k << 30), (tsf + 4) | ((uint32_t)k << 30));
+              umma_commit(&empty[stg]);
+            }
           } else {
 #pragma unroll
             for (int k = 0; k < BK / 16; ++k) {
@@ -1381,6 +1479,18 @@ bool tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uin
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// An array of 512-byte scale atoms as a [2 x natoms, 256] byte tensor whose 256 x 2 box is
+// one atom (the CTA-pair form of the TMA load then brings it in on the leader's barrier).
+bool tmap_atoms(CUtensorMap* tm, const void* base, uint64_t natoms) {
+  const cuuint64_t dims[2] = {256, 2 * natoms};
+  const cuuint64_t strides[1] = {256};
+  const cuuint32_t box[2] = {256, 2};
+  const cuuint32_t es[2] = {1, 1};
+  return g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+                  es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Failure-path test hooks, read once from the environment (unset in normal use):
 // MOE_B200_WAIT_NS sets the limit of every bounded wait of the GEMM kernels, and
 // MOE_B200_TEST_DROP_STAGE = n makes CTA 0's producer skip its n-th ring stage (no load,
@@ -1430,10 +1540,10 @@ cudaError_t launch_mx(const GemmParams& p, int64_t tile_bound, cudaStream_t st) 
 }
 
 // CTA-pair variant: clusters of 2 CTAs, as many as can be resident at once.
-template <int BN, bool B_MN, int EPI>
+template <int BN, bool B_MN, int EPI, bool FP8 = false>
 cudaError_t launch_pair(const GemmParams& p, int64_t pair_tile_bound, cudaStream_t st) {
-  auto kern = grouped_gemm_sm100<BN, false, B_MN, EPI, false, true>;
-  constexpr size_t smem = Cfg<BN, true, EPI>::kSmem;
+  auto kern = grouped_gemm_sm100<BN, false, B_MN, EPI, false, true, FP8>;
+  constexpr size_t smem = Cfg<BN, true, EPI, FP8>::kSmem;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
@@ -1816,9 +1926,18 @@ cudaError_t ffn_fwd_mx(const FfnShape& s, const void* x_perm, const int32_t* off
   p1.sfb = w.w1_s;
   p1.N = f; p1.K = d; p1.b_rows = 2 * f;
   p1.out = static_cast<__nv_bfloat16*>(act); p1.ld_out = 3 * f;
-  // 128 gate + 128 up columns per tile
-  if ((err = launch_mx<256, false, false, EPI_SWIGLU_FWD, false>(p1, m_tile_bound(s) * (f / 128), st)) != cudaSuccess)
-    return err;
+  // 128 gate + 128 up columns per tile; CTA pairs where experts are large enough
+  const bool pairs = use_pairs(s);
+  const uint64_t tiles = (uint64_t)R / 128 + E;  // row-tile atoms per 128 columns of K
+  if (pairs) {
+    if (!tmap_atoms(&p1.tmSfa, ws + L.sx0, tiles * (d / 128)) ||
+        !tmap_atoms(&p1.tmSfb, w.w1_s, (uint64_t)E * 2 * f * d / (32 * 512)))
+      return cudaErrorInvalidValue;
+    err = launch_pair<256, false, EPI_SWIGLU_FWD, true>(p1, pair_tile_bound(s) * (f / 128), st);
+  } else {
+    err = launch_mx<256, false, false, EPI_SWIGLU_FWD, false>(p1, m_tile_bound(s) * (f / 128), st);
+  }
+  if (err != cudaSuccess) return err;
   // h along f (down GEMM) and in token blocks (kept for the dW2 GEMM of the backward)
   if ((err = mxfp8_act(R, E, f, 3 * f, actb + 2 * f, map, cnt, rt, ws + L.qh0, ws + L.sh0,
                        ws + L.qh1, ws + L.sh1, st)) != cudaSuccess)
@@ -1833,6 +1952,12 @@ cudaError_t ffn_fwd_mx(const FfnShape& s, const void* x_perm, const int32_t* off
   p2.sfb = w.w2_s;
   p2.N = d; p2.K = f; p2.b_rows = d;
   p2.out = static_cast<__nv_bfloat16*>(y_perm); p2.ld_out = d;
+  if (pairs && d % 256 == 0) {
+    if (!tmap_atoms(&p2.tmSfa, ws + L.sh0, tiles * (f / 128)) ||
+        !tmap_atoms(&p2.tmSfb, w.w2_s, (uint64_t)E * d * f / (32 * 512)))
+      return cudaErrorInvalidValue;
+    return launch_pair<256, false, EPI_STORE, true>(p2, pair_tile_bound(s) * (d / 256), st);
+  }
   return launch_mx_n<false, false, EPI_STORE, false>(p2, d, m_tile_bound(s), st);
 }
 
@@ -1886,8 +2011,17 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
     p3.N = f; p3.K = d; p3.b_rows = d;
     p3.out = dadu; p3.ld_out = 2 * f;
     p3.act = actb; p3.ld_act = 3 * f;
-    if ((err = launch_mx_n<false, true, EPI_SWIGLU_BWD, false>(p3, f, m_tile_bound(s), st)) != cudaSuccess)
-      return err;
+    const bool pairs = use_pairs(s);
+    const uint64_t tiles = (uint64_t)R / 128 + E;
+    if (pairs && f % 256 == 0) {
+      if (!tmap_atoms(&p3.tmSfa, ws + L.sdy0, tiles * (d / 128)) ||
+          !tmap_atoms(&p3.tmSfb, w.w2t_s, (uint64_t)E * d * f / (32 * 512)))
+        return cudaErrorInvalidValue;
+      err = launch_pair<256, true, EPI_SWIGLU_BWD, true>(p3, pair_tile_bound(s) * (f / 256), st);
+    } else {
+      err = launch_mx_n<false, true, EPI_SWIGLU_BWD, false>(p3, f, m_tile_bound(s), st);
+    }
+    if (err != cudaSuccess) return err;
     // dgrad 2: dx = [da | du] W1 ([da | du] along 2f, W1 along its 2f rows); [da | du]
     // also in token blocks for the dW1 GEMM
     if ((err = mxfp8_act(R, E, 2 * f, 2 * f, dadu, map, cnt, rt, ws + L.qda0, ws + L.sda0,
@@ -1902,8 +2036,15 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
     p4.sfb = w.w1t_s;
     p4.N = d; p4.K = 2 * f; p4.b_rows = 2 * f;
     p4.out = static_cast<__nv_bfloat16*>(dx_perm); p4.ld_out = d;
-    if ((err = launch_mx_n<false, true, EPI_STORE, false>(p4, d, m_tile_bound(s), st)) != cudaSuccess)
-      return err;
+    if (pairs && d % 256 == 0) {
+      if (!tmap_atoms(&p4.tmSfa, ws + L.sda0, tiles * (2 * f / 128)) ||
+          !tmap_atoms(&p4.tmSfb, w.w1t_s, (uint64_t)E * 2 * f * d / (32 * 512)))
+        return cudaErrorInvalidValue;
+      err = launch_pair<256, true, EPI_STORE, true>(p4, pair_tile_bound(s) * (d / 256), st);
+    } else {
+      err = launch_mx_n<false, true, EPI_STORE, false>(p4, d, m_tile_bound(s), st);
+    }
+    if (err != cudaSuccess) return err;
   }
   // wgrad 2: dW2[e] = dy^T h  (M = d, N = f)
   GemmParams p5 = mx_params(s, offsets, status);

@@ -33,6 +33,8 @@ CASES = {
     # experts of 3459 and 5998 rows: weight gradients cut into K ranges, partial sums added
     "mx_skew_split": shrink(BASE, name="mx_skew_split", T=6000, d_model=128, E=16, top_k=2,
                             d_ff=128, router_std=1 / 16.0, bias_std=3.0),
+    # d and f multiples of 256, ~512 rows per expert: the row-grouped GEMMs run on CTA pairs
+    "mx_pairs": shrink(BASE, name="mx_pairs", T=2048, d_model=512, E=8, top_k=2, d_ff=256),
     # one token
     "mx_one_token": shrink(BASE, name="mx_one_token", T=1, d_model=128, E=4, top_k=2, d_ff=128),
 }
@@ -158,3 +160,20 @@ def test_fused_dispatch_is_bit_identical_to_permute_then_quantise(name):
 @pytest.mark.parametrize("name", ["mx_e8", "mx_skew_split"])
 def test_mxfp8_accumulated_weight_grads_are_the_sum_of_two_steps(name):
     check_accumulate(CASES[name])
+
+
+
+@pytest.mark.parametrize("name", ["mx_pairs", "mx_skew_split"])
+def test_mxfp8_cta_pairs_give_the_bits_of_single_ctas(name, monkeypatch):
+    # the same dot products in the same K order: 256-row tiles on CTA pairs must reproduce
+    # the 128-row single-CTA results exactly
+    cfg = CASES[name]
+    monkeypatch.setenv("MOE_B200_PAIR", "0")
+    _, A = run_layer(cfg)
+    monkeypatch.setenv("MOE_B200_PAIR", "1")
+    _, B = run_layer(cfg)
+    for key in ("act", "y_perm", "out", "dx_perm", "dx", "dw1", "dw2", "dw_router"):
+        a, b = getattr(A, key), getattr(B, key)
+        if key in ("act", "y_perm", "dx_perm"):
+            a, b = a[:cfg.R], b[:cfg.R]
+        assert torch.equal(a, b), key
