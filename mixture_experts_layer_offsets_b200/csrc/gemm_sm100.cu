@@ -64,14 +64,7 @@ enum : int {
 };
 
 constexpr int kRouterKMax = 8;  // top-k kept in registers by the router epilogue
-// MXFP8 CTA pairs: where the B scales of a 256-column tile sit.  0 (used): each CTA's
-// TMEM holds the scales of all 256 columns, as the pair's block-scaled MMA reads them;
-// 1: each CTA holds those of its own B half only.  On a B200 the second gives results
-// far from the single-CTA tiles, the first gives the same bits.
-#ifndef MOE_PAIR_SFB_SPLIT
-#define MOE_PAIR_SFB_SPLIT 0
-#endif
-constexpr bool kPairSfbSplit = MOE_PAIR_SFB_SPLIT != 0;
+
 
 struct GemmParams {
   CUtensorMap tmA;
@@ -135,9 +128,10 @@ template <int BN, bool PAIR = false, int EPI = 1, bool FP8 = false> struct Cfg {
   // slots of 8 TMEM columns after the accumulators.
   static constexpr int kBKe = FP8 ? 128 : BK;  // K elements per stage
   static constexpr uint32_t kBBytes = (PAIR ? BN / 2 : BN) * 128;
-  // FP8: A atom (512 B) + the B atoms (BN/128 of them; a CTA of a pair holding the scales
-  // of its own B half takes one), padded to keep stages 1024-byte aligned
-  static constexpr uint32_t kSfB = (PAIR && kPairSfbSplit) ? 512 : (BN / 128) * 512;
+  // FP8: A atom (512 B) + the B atoms (BN/128 of them; in a CTA pair each CTA holds the
+  // scales of all BN columns, as the pair's block-scaled MMA reads them from each CTA's
+  // TMEM), padded to keep stages 1024-byte aligned
+  static constexpr uint32_t kSfB = (BN / 128) * 512;
   static constexpr uint32_t kSfLoad = FP8 ? 512 + kSfB : 0;   // bytes loaded per stage
   static constexpr uint32_t kSfBytes = FP8 ? ((kSfLoad + 1023) / 1024) * 1024 : 0;
   static constexpr uint32_t kStage = kABytes + kBBytes + kSfBytes;
@@ -693,22 +687,20 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
           }
         }
         // CTA pairs: atom indices (the atom tensors' row is twice the index).  A: this CTA's
-        // 128-row tile of its expert; B: the CTA's own half of the 256 columns, or both.
+        // 128-row tile of its expert; B: both 128-column halves of the tile.
         int64_t pa0 = 0, pb0 = 0, pb1 = 0;
         if constexpr (PAIR) {
           pa0 = ((int64_t)s_sel[ti.g] + (ti.m0 - s_off[ti.g]) / BM) * kq;
           if constexpr (!B_MN) {
             const int ntiles = p.b_rows / 128;
-            const int t0 = EPI == EPI_SWIGLU_FWD ? ti.n0 / 128 : ti.n0 / 128;
+            // SwiGLU: the gate and the up row tiles; otherwise two adjacent row tiles
+            const int t0 = ti.n0 / 128;
             const int t1 = EPI == EPI_SWIGLU_FWD ? (p.f + ti.n0) / 128 : ti.n0 / 128 + 1;
             pb0 = ((int64_t)ti.g * ntiles + t0) * kq;
             pb1 = ((int64_t)ti.g * ntiles + t1) * kq;
           } else {
             pb0 = (int64_t)ti.g * kq * (p.N / 128) + ti.n0 / 128;
             pb1 = pb0 + 1;
-          }
-          if constexpr (kPairSfbSplit) {
-            if (rank == 1) pb0 = pb1;
           }
         }
         for (int kb = 0; kb < ti.nkb; ++kb, ++it, s = (s + 1 == S ? 0 : s + 1), ph ^= (s == 0)) {
@@ -734,8 +726,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
             const int64_t bstep = B_MN ? (int64_t)kb * (p.N / 128) : (int64_t)kb;
             tma_load_2d_pair(sf, &p.tmSfa, 0, (int)(2 * (pa0 + kb)), bar);
             tma_load_2d_pair(sf + 512, &p.tmSfb, 0, (int)(2 * (pb0 + bstep)), bar);
-            if constexpr (!kPairSfbSplit)
-              tma_load_2d_pair(sf + 1024, &p.tmSfb, 0, (int)(2 * (pb1 + bstep)), bar);
+            tma_load_2d_pair(sf + 1024, &p.tmSfb, 0, (int)(2 * (pb1 + bstep)), bar);
             continue;
           }
           constexpr uint32_t kSfB = (BN / 128) * 512;
@@ -923,7 +914,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
               // read both CTAs' A rows, B halves and scales
               tmem_cp_sf_pair(tsf, desc_f0 + so);
 #pragma unroll
-              for (int i = 0; i < (kPairSfbSplit ? 1 : 2); ++i)
+              for (int i = 0; i < 2; ++i)
                 tmem_cp_sf_pair(tsf + 4 + 4 * i, desc_f0 + so + ((512 + 512 * i) >> 4));
 #pragma unroll
               for (int k = 0; k < 4; ++k)
