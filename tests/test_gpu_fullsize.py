@@ -147,3 +147,36 @@ def test_fullsize_skewed_padded():
             _, _, _, y = ref.expert_ffn_fwd(x, [0, 1], f64(inp["w1"][e:e + 1]), f64(inp["w2"][e:e + 1]))
             want += p[e] * y[0]
         assert rel(f64(L.out[t]), want) <= TOL[cfg.dtype]
+
+
+def test_fullsize_mxfp8_sampled_expert():
+    """mxfp8_e128 at full size (fused dispatch, CTA pairs): every discrete output for all
+    tokens, then one sampled expert end to end from its own rows (its row-wise operand
+    blocks and its token blocks depend on nothing else): a, u, h, y_perm, dx_perm and its
+    weight gradients against the MXFP8 oracle."""
+    from oracle import moe_mx_ref as mxr
+    cfg = inputs.CONFIGS["mxfp8_e128"]
+    inp, L = _run(cfg)
+    o = _check_discrete(L)
+    rng = np.random.default_rng(3)
+    e = int(rng.choice(np.nonzero(o["counts"] > 0)[0]))
+    r0, r1 = int(o["offsets"][e]), int(o["offsets"][e + 1])
+    toks = torch.from_numpy(o["perm_src"][r0:r1]).cuda()
+    wr = f64(inp["w_router"])
+    bias = f64(inp["bias"]) if inp["bias"] is not None else None
+    x = f64(inp["x"][toks])
+    p = ref.softmax(ref.router_logits(x, wr, bias))
+    dy = p[:, e:e + 1] * f64(inp["dout"][toks])
+    w1 = f64(inp["w1"][e:e + 1])
+    w2 = f64(inp["w2"][e:e + 1])
+    off = [0, r1 - r0]
+    a, u, h, y = mxr.expert_ffn_fwd_mx(x, off, w1, w2, act_round=mxr.round_bf16)
+    dxp, dw1, dw2 = mxr.expert_ffn_bwd_mx(dy, x, a, u, h, off, w1, w2, act_round=mxr.round_bf16)
+    f = cfg.d_ff
+    act = f64(L.act[r0:r1])
+    tol = TOL["mxfp8"]
+    checks = {"a": (act[:, :f], a), "u": (act[:, f:2 * f], u), "h": (act[:, 2 * f:], h),
+              "y_perm": (f64(L.y_perm[r0:r1]), y), "dx_perm": (f64(L.dx_perm[r0:r1]), dxp),
+              "dw1": (f64(L.dw1[e]), dw1[0]), "dw2": (f64(L.dw2[e]), dw2[0])}
+    errs = {k: rel(g, w) for k, (g, w) in checks.items()}
+    assert all(v <= tol for v in errs.values()), (e, r1 - r0, errs)
