@@ -62,8 +62,8 @@ def launches_per_step(cfg, capacity, recompute, fused_dispatch) -> int:
 
 FP8_OVER_BF16 = 2.0   # nominal dense tensor-core ratio (4.5 / 2.25 PFLOP/s)
 # DRAM bytes (read + write) of the six grouped-GEMM launches of one step, from one ncu capture
-# of this build (profiles/launches_bf16_e8.md); None where no capture of the current kernels
-# exists.
+# of the current kernels per workload (profiles/launches_bf16_e8.md,
+# profiles/launches_mxfp8_e128.md); None for workloads without such a capture.
 GEMM_TRAFFIC_BYTES = {"bf16_e8": 3.820e+09, "mxfp8_e128": 2.4088e+10}
 
 
