@@ -381,14 +381,15 @@ seg_blocks_kernel(const int32_t* __restrict__ offsets, int E, int4* __restrict__
 // atoms, tile and row from row_tile), and q_c / atoms_c in the block's 32 rows within each
 // column (stage atoms; the blocks of a segment's last stage past its end get 2^0).
 constexpr int kActPitch = 136;  // bf16 per staged row (16 bytes of padding)
-__global__ void __launch_bounds__(128)
+constexpr int kSqPitch = 144;   // bytes per staged row of the column copy (16 bytes of padding)
+__global__ void __launch_bounds__(128, 8)
 mx_act_kernel(const __nv_bfloat16* __restrict__ src, int64_t K, int64_t ld,
               const int4* __restrict__ map, const int32_t* __restrict__ count,
               const int32_t* __restrict__ row_tile, uint8_t* __restrict__ q_r,
               uint8_t* __restrict__ atoms_r, uint8_t* __restrict__ q_c,
               uint8_t* __restrict__ atoms_c, const int32_t* __restrict__ gather) {
   __shared__ __align__(16) __nv_bfloat16 s_t[32 * kActPitch];
-  __shared__ __align__(16) uint8_t s_q[32 * 128];
+  __shared__ __align__(16) uint8_t s_q[32 * kSqPitch];
   const int tid = threadIdx.x, ct = blockIdx.x;
   const int64_t c0 = (int64_t)ct * 128;
   const int64_t kq = K >> 7;
@@ -451,25 +452,41 @@ mx_act_kernel(const __nv_bfloat16* __restrict__ src, int64_t K, int64_t ld,
         if (rt >= 0) atoms_r[((int64_t)(rt >> 7) * kq + ct) * 512 + atom_byte(rt & 127, kb)] = (uint8_t)(ex + 127);
       }
     }
-    // columns: thread = column; the block's n rows
+    // columns: thread = (pair of adjacent columns, half of the 32 rows); the two halves of
+    // a pair are neighbouring lanes.  The rows a lane pair reads in one step are 4 apart
+    // (rows 0-3, 8-11, .. for one half, 4-7, 12-15, .. for the other), which puts the two
+    // halves 16 banks apart.  Rows past n are zero in s_t, so they do not change the
+    // maximum, and their codes are never written out.
     {
-      const __nv_bfloat16* t = s_t + tid;
-      float amax = 0.f;
-      for (int i = 0; i < n; ++i) amax = fmaxf(amax, fabsf(__bfloat162float(t[i * kActPitch])));
-      const int ex = block_exponent(amax);
-      const float mul = pow2_neg(ex);
-      for (int i = 0; i < n; i += 2) {
-        const float lo = __bfloat162float(t[i * kActPitch]) * mul;
-        const float hi = i + 1 < n ? __bfloat162float(t[(i + 1) * kActPitch]) * mul : 0.f;
-        const uint32_t pr = e4m3_pair(hi, lo);
-        s_q[i * 128 + tid] = (uint8_t)(pr & 0xFF);
-        if (i + 1 < n) s_q[(i + 1) * 128 + tid] = (uint8_t)(pr >> 8);
+      const int cp = tid >> 1, rh = tid & 1;
+      uint32_t w[16];
+      __nv_bfloat162 am = __float2bfloat162_rn(0.f);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int r = (i & 3) + ((i >> 2) << 3) + 4 * rh;
+        w[i] = *reinterpret_cast<const uint32_t*>(s_t + r * kActPitch + 2 * cp);
+        am = __hmax2(am, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w[i])));
       }
+      uint32_t amw = *reinterpret_cast<uint32_t*>(&am);
+      const uint32_t oth = __shfl_xor_sync(0xffffffffu, amw, 1);
+      am = __hmax2(am, *reinterpret_cast<const __nv_bfloat162*>(&oth));
+      const int ex0 = block_exponent(__low2float(am)), ex1 = block_exponent(__high2float(am));
+      const float m0 = pow2_neg(ex0), m1 = pow2_neg(ex1);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int r = (i & 3) + ((i >> 2) << 3) + 4 * rh;
+        const float lo = __uint_as_float(w[i] << 16) * m0;          // column 2 cp
+        const float hi = __uint_as_float(w[i] & 0xFFFF0000u) * m1;  // column 2 cp + 1
+        *reinterpret_cast<uint16_t*>(s_q + r * kSqPitch + 2 * cp) = (uint16_t)e4m3_pair(hi, lo);
+      }
+      // each of the pair's two threads writes the scale byte of one of its columns
+      const int col = 2 * cp + rh;
+      const int ex = rh ? ex1 : ex0;
       uint8_t* at = atoms_c + ((int64_t)m.z * kq + ct) * 512;
       const int pos = m.w & 3;
-      at[atom_byte(tid, pos)] = (uint8_t)(ex + 127);
+      at[atom_byte(col, pos)] = (uint8_t)(ex + 127);
       if (m.w & 4)
-        for (int kb = pos + 1; kb < 4; ++kb) at[atom_byte(tid, kb)] = 0x7F;
+        for (int kb = pos + 1; kb < 4; ++kb) at[atom_byte(col, kb)] = 0x7F;
     }
     __syncthreads();
     // the column copy's rows, 16 bytes per store
@@ -478,7 +495,7 @@ mx_act_kernel(const __nv_bfloat16* __restrict__ src, int64_t K, int64_t ld,
       const int i = tid + 128 * j, row = i >> 3, p16 = i & 7;
       if (row < n)
         *reinterpret_cast<uint4*>(q_c + (int64_t)(r0 + row) * K + c0 + p16 * 16) =
-            *reinterpret_cast<const uint4*>(s_q + row * 128 + p16 * 16);
+            *reinterpret_cast<const uint4*>(s_q + row * kSqPitch + p16 * 16);
     }
     __syncthreads();
   }
