@@ -216,3 +216,16 @@ def test_recompute_with_shared_buffers_is_bit_exact(name):
                                      ("bf16_e8_small", "bf16"), ("bf16_skew_split", "bf16")])
 def test_accumulated_weight_grads_are_the_sum_of_two_steps(name, dw):
     check_accumulate(CASES[name], dw_dtype=dw)
+
+
+@pytest.mark.parametrize("dtype,d,f", [("f32", 64, 32), ("bf16", 256, 256), ("mxfp8", 256, 256)])
+def test_empty_batch_is_a_clean_no_op(dtype, d, f):
+    # T = 0: nothing is routed; every count and offset is 0 and every weight gradient,
+    # written or accumulated, is exactly 0 (each expert's tile sums over no rows)
+    base = CONFIGS["tiny_f32"] if dtype == "f32" else CONFIGS["bf16_e8"]
+    cfg = shrink(base, name=f"empty_{dtype}", T=0, d_model=d, d_ff=f, E=8, top_k=2, dtype=dtype)
+    cpu, L = run_layer(cfg)
+    assert not L.counts.any() and not L.offsets.any()
+    for key in ("dw1", "dw2", "dw_router"):
+        assert not getattr(L, key).any(), key
+    assert L.out.numel() == 0 and L.dx.numel() == 0
