@@ -5,7 +5,12 @@
  * softmax/top-k, on-device expert counts and offsets, a rowwise permute into
  * contiguous per-expert buffers, a device-scheduled grouped SwiGLU GEMM,
  * a gate-weighted combine, and the backward of each step; plus MXFP8 block
- * quantisation.
+ * quantisation.  Besides the steps themselves: a dispatch that writes the MXFP8
+ * operands directly (moe_permute_mx), a backward that recomputes the expert
+ * activations (moe_grouped_ffn_bwd_recompute), weight-gradient accumulation
+ * (MOE_DW_ACCUMULATE), routing-balance statistics (moe_routing_stats), an
+ * optional renormalised gate rule (moe_renorm_gates, moe_renorm_gates_bwd),
+ * and the padded-capacity comparison layout (moe_padded_dispatch).
  *
  * Sources (news pages about the Olmo-core 3 release; they describe the method
  * in prose only):
