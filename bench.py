@@ -1,31 +1,49 @@
 """Benchmark: MoE FFN layer forward + backward on B200, tokens/s.
 
 One step = the whole hot path over one batch: route (logits, softmax/top-k,
-counts, offsets, slot rows) -> permute -> grouped SwiGLU FFN forward ->
+counts, offsets, slot rows) -> dispatch -> grouped SwiGLU FFN forward ->
 combine -> combine backward -> grouped FFN backward (dgrad + wgrad) ->
-unpermute-grad + router grad.  Inputs are seeded synthetic tensors already
-resident in HBM; L2 is flushed (256 MiB write) between timed steps, outside
-the timed events.  The timed step is a CUDA-graph replay of the C-ABI calls;
-the per-phase breakdown comes from eager steps with events between calls.
+unpermute-grad + router grad (the MXFP8 workload also quantises its FP32
+master weights inside every step).  Inputs are seeded synthetic tensors
+already resident in HBM; L2 is flushed (256 MiB write) between timed steps,
+outside the timed events.  The timed step is a CUDA-graph replay of the C-ABI
+calls.  A profiled pass of eager steps then times every kernel launch of the
+library with CUDA events (moe_profile_begin / moe_profile_end): the roofline
+of the grouped GEMM is taken from the GEMM launches alone.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--capacity-factor] [--impl {ours,reference}]
+                    [--capacity-factor] [--recompute] [--accum G] [--no-sweep]
+                    [--impl {ours,reference}]
 
-Multi-GPU (torchrun, one process per GPU): data parallel with weak scaling,
-each rank runs its own token batch (seed = rank) through its own copy of the
-layer; there is no collective inside a step.  The timed region is bracketed
-by a barrier and a device synchronisation; the time is the max over ranks.
+Default workload: mxfp8_e128 (T=32768, d_model=4096, E=128, top_k=4,
+d_ff=1536, MXFP8), the largest configuration that fits one GPU.  With the
+default workload on one GPU the line also carries a ``sweep`` measured in the
+same process: bf16_e8 and bf16_e128 (the expert-pool sweep at fixed
+activation), bf16_skew_e128 dropless and padded (device-scheduled against
+uniform capacity), and the MXFP8 workload's shapes in bf16 (MXFP8 vs bf16).
+
+Multi-GPU: ``--gpus N`` starts N ranks itself (torch.distributed.run, one
+process per GPU, NCCL) unless it already runs under a launcher.  Data
+parallel with weak scaling: each rank runs its own token batch (seed = rank)
+through its own replica of the layer.  One step is then one optimizer step of
+the pages' DDP (kongchang, 容量税: gradients synchronised once per optimizer
+step): G micro-batches (``--accum``, default 8 when N > 1) whose weight
+gradients accumulate in place, then one all-reduce of dW1, dW2 and dW_router
+over NCCL.  The timed region is bracketed by a barrier and a device
+synchronisation; the time is the max over ranks.
 
 ``--impl reference`` times the float64 CPU oracle on the host cores on a
-bounded token sample of the same workload (rank 0 only).
+bounded sample of the same workload (rank 0 only).
 """
 
 from __future__ import annotations
 
 import argparse
+import datetime
+import hashlib
 import json
-import math
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -42,29 +60,28 @@ from mixture_experts_layer_offsets_b200 import dist as mdist  # noqa: E402
 from mixture_experts_layer_offsets_b200 import inputs  # noqa: E402
 
 METRIC = "MoE FFN fwd+bwd tokens/s on 1 B200; grouped-GEMM % of tensor-core peak"
+DEFAULT_WORKLOAD = "mxfp8_e128"
 FLUSH_BYTES = 256 << 20
-def launches_per_step(cfg, capacity, recompute, fused_dispatch) -> int:
-    """Kernel launches of this library in one step, counted per C-ABI call from the
-    launch sequences in csrc (and checked against ncu launch lists)."""
-    mx, f32 = cfg.dtype == "mxfp8", cfg.dtype == "f32"
-    tc_router_bwd = not f32 and cfg.E % 128 == 0 and cfg.top_k <= 8 and cfg.d_model % 256 == 0
-    n = 2 if mx else 0                                   # the two weight quantisers
-    n += 3                                               # router, block scan, slot rows
-    n += 2 if capacity else (4 if fused_dispatch else 1)  # dispatch
-    n += (3 if fused_dispatch else 6) if mx else (3 if f32 else 2)   # forward FFN
-    n += 1 + 1                                           # combine, combine backward
-    n += 8 if mx else (5 if f32 else 6)                  # backward FFN
-    n += 5 if tc_router_bwd else 4                       # router backward
-    if recompute:                                        # the gate/up half again
-        n += 5 if mx else (2 if f32 else 1)
-    return n
-
-
 FP8_OVER_BF16 = 2.0   # nominal dense tensor-core ratio (4.5 / 2.25 PFLOP/s)
-# DRAM bytes (read + write) of the six grouped-GEMM launches of one step, from one ncu capture
-# of the current kernels per workload (profiles/launches_bf16_e8.md,
-# profiles/launches_mxfp8_e128.md); None for workloads without such a capture.
-GEMM_TRAFFIC_BYTES = {"bf16_e8": 3.820e+09, "mxfp8_e128": 2.4088e+10}
+PHASES = ["quantize_w", "route", "dispatch", "ffn_fwd", "combine", "combine_bwd", "ffn_bwd",
+          "route_bwd"]
+SWEEP = [("bf16_e8", False, None), ("bf16_e128", False, None), ("bf16_skew_e128", False, None),
+         ("bf16_skew_e128", True, None), ("mxfp8_e128", False, "bf16")]
+
+# DRAM bytes (read + write) of the grouped-GEMM launches of one step, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum) per workload, with the SHA-256 of the
+# GEMM source it was taken on: reported only while that source is unchanged.
+GEMM_TRAFFIC = {}
+GEMM_SOURCES = ("mixture_experts_layer_offsets_b200/csrc/gemm_sm100.cu",
+                "mixture_experts_layer_offsets_b200/csrc/common.cuh")
+
+
+def gemm_source_sha() -> str:
+    h = hashlib.sha256()
+    for rel in GEMM_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
 
 
 def _peaks():
@@ -76,7 +93,18 @@ def _peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def _workload_desc(cfg, capacity, recompute=False):
+def resolve(args) -> inputs.MoEConfig:
+    cfg = inputs.CONFIGS[args.workload]
+    if args.tokens:
+        cfg = inputs.shrink(cfg, name=f"{cfg.name}@T{args.tokens}", T=args.tokens)
+    if args.experts:
+        cfg = inputs.shrink(cfg, name=f"{cfg.name}@E{args.experts}", E=args.experts)
+    if args.dtype and args.dtype != cfg.dtype:
+        cfg = inputs.shrink(cfg, name=f"{cfg.name}@{args.dtype}", dtype=args.dtype)
+    return cfg
+
+
+def _workload_desc(cfg, capacity, recompute=False, accum=1, world=1):
     d = {"workload": f"{cfg.name}: T={cfg.T} d_model={cfg.d_model} E={cfg.E} top_k={cfg.top_k} "
                      f"d_ff={cfg.d_ff} {cfg.dtype}",
          "T": cfg.T, "d_model": cfg.d_model, "E": cfg.E, "top_k": cfg.top_k, "d_ff": cfg.d_ff,
@@ -89,10 +117,13 @@ def _workload_desc(cfg, capacity, recompute=False):
                          "every step (inside the timed step)")
     if recompute:
         d["recompute"] = "gate/up GEMM re-run in the backward (a | u | h not kept from the forward)"
-    if capacity:
-        d["layout"] = f"padded capacity C={capacity} (overflow dropped)"
-    else:
-        d["layout"] = "dropless, device-scheduled grouped GEMM"
+    d["layout"] = (f"padded capacity C={capacity} (overflow dropped)" if capacity else
+                   "dropless, device-scheduled grouped GEMM")
+    d["parallelism"] = f"dp{world}"
+    if world > 1:
+        d["step"] = (f"one optimizer step: {accum} micro-batches of T tokens per rank, weight "
+                     "gradients accumulated in place, then one NCCL all-reduce of dW1, dW2, "
+                     "dW_router")
     return d
 
 
@@ -146,51 +177,72 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
-# ------------------------------------------------------------- our arm
-def run_ours(args, rank, world):
-    from mixture_experts_layer_offsets_b200.layer import MoELayer, capacity_for
+# ------------------------------------------------------- algorithmic work
+def gemm_flop(cfg) -> float:
+    """Algorithmic FLOPs of the six expert GEMMs of one step: 18 R d f (dropless rows)."""
+    return 18.0 * cfg.R * cfg.d_model * cfg.d_ff
 
-    cfg = inputs.CONFIGS[args.workload]
-    if args.tokens:
-        cfg = inputs.shrink(cfg, name=f"{cfg.name}@T{args.tokens}", T=args.tokens)
-    if args.experts:
-        cfg = inputs.shrink(cfg, name=f"{cfg.name}@E{args.experts}", E=args.experts)
-    if args.dtype and args.dtype != cfg.dtype:
-        cfg = inputs.shrink(cfg, name=f"{cfg.name}@{args.dtype}", dtype=args.dtype)
-    mxfp8 = cfg.dtype == "mxfp8"
-    dev = torch.device("cuda", torch.cuda.current_device())
-    capacity = capacity_for(cfg.R, cfg.E, *cfg.padded_cf) if args.capacity_factor and cfg.padded_cf else None
-    inp = inputs.make_inputs(cfg, device=dev, seed=mdist.rank_seed(0, rank))
-    L = MoELayer(cfg.T, cfg.d_model, cfg.E, cfg.top_k, cfg.d_ff, cfg.dtype, dev,
-                 dw_dtype="f32", capacity=capacity, recompute=args.recompute)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream()
-    x, wr, b, w1, w2, dout = (inp[k] for k in ("x", "w_router", "bias", "w1", "w2", "dout"))
-    phases = ["quantize_w", "route", "dispatch", "ffn_fwd", "combine", "combine_bwd", "ffn_bwd",
-              "route_bwd"]
-    fdt = L.ffn_dtype
 
-    def step(ev=None):
+def kernel_bytes(cfg, capacity=None) -> dict:
+    """Algorithmic HBM bytes per step of the row-moving and quantising kernels (each
+    operand read once, each result written once), by launch name."""
+    T, d, E, k, f = cfg.T, cfg.d_model, cfg.E, cfg.top_k, cfg.d_ff
+    R = E * capacity if capacity else cfg.R
+    s = 4 if cfg.dtype == "f32" else 2
+    out = {
+        "router_gemm": T * d * s + E * d * s + T * E * 4 + T * k * 12,
+        "permute": T * d * s + R * d * s + T * k * 8,
+        "combine": R * d * s + T * d * s + T * k * 8,
+        "combine_bwd": T * d * s + 2 * R * d * s + T * k * 12,
+    }
+    if cfg.dtype == "mxfp8":
+        mx = 2 * (1 + 1 / 32)  # two E4M3 copies with their E8M0 scales, per element
+        out["mx_weights"] = 4 * E * 3 * f * d + mx * E * 3 * f * d
+        # x (gathered rows), h, dy, [da | du]: bf16 in, both MXFP8 copies out
+        out["mx_act"] = R * (d + f + d + 2 * f) * (2 + mx)
+    return out
+
+
+# ------------------------------------------------------------ one layer
+class LayerStep:
+    """Device buffers, inputs and the call sequence of one layer step through the C ABI."""
+
+    def __init__(self, cfg, dev, seed, capacity=None, recompute=False):
+        from mixture_experts_layer_offsets_b200.layer import MoELayer
+        self.cfg, self.dev, self.capacity, self.recompute = cfg, dev, capacity, recompute
+        self.inp = inputs.make_inputs(cfg, device=dev, seed=seed)
+        self.L = MoELayer(cfg.T, cfg.d_model, cfg.E, cfg.top_k, cfg.d_ff, cfg.dtype, dev,
+                          dw_dtype="f32", capacity=capacity, recompute=recompute)
+
+    def grads(self):
+        return [self.L.dw1, self.L.dw2, self.L.dw_router]
+
+    def run(self, ev=None, accumulate=False, stream=None):
+        from mixture_experts_layer_offsets_b200 import capi
+        L, cfg = self.L, self.cfg
+        st = stream or torch.cuda.current_stream()
+        x, wr, b, w1, w2, dout = (self.inp[k] for k in ("x", "w_router", "bias", "w1", "w2",
+                                                         "dout"))
+
         def mark(i):
             if ev is not None:
-                ev[i].record(stream)
-        s, dt = L.shape, L.cdtype
-        from mixture_experts_layer_offsets_b200 import capi
+                ev[i].record(st)
+        s, dt, fdt = L.shape, L.cdtype, L.ffn_dtype
+        acc = capi.MOE_DW_ACCUMULATE if accumulate else 0
         mark(0)
-        if mxfp8:
+        if cfg.dtype == "mxfp8":
             L.quantize_weights(w1, w2)
         mark(1)
         capi.moe_route(s, dt, x, wr, b, L.logits, L.topk_idx, L.topk_gate, L.counts, L.offsets,
                        L.slot_row, L.ws)
         mark(2)
-        if capacity:
-            capi.moe_padded_dispatch(s, dt, capacity, x, L.topk_idx, L.slot_row, L.offsets,
+        if self.capacity:
+            capi.moe_padded_dispatch(s, dt, self.capacity, x, L.topk_idx, L.slot_row, L.offsets,
                                      L.x_perm, L.pad_row, L.offsets_pad)
+        elif L.fused_dispatch:
+            capi.moe_permute_mx(s, x, L.slot_row, L.offsets, L.perm_src, L.ws)
         else:
-            if L.fused_dispatch:
-                capi.moe_permute_mx(s, x, L.slot_row, L.offsets, L.perm_src, L.ws)
-            else:
-                capi.moe_permute(s, dt, x, L.slot_row, L.x_perm, L.perm_src)
+            capi.moe_permute(s, dt, x, L.slot_row, L.x_perm, L.perm_src)
         mark(3)
         capi.moe_grouped_ffn_fwd(s, fdt, L.rows, L.x_perm, L.ffn_offsets, w1, w2, L.act, L.y_perm,
                                  L.ws, mx=L.mx)
@@ -199,133 +251,270 @@ def run_ours(args, rank, world):
         mark(5)
         capi.moe_combine_bwd(s, dt, dout, L.y_perm, L.row_map, L.topk_gate, L.dy_perm, L.dgate)
         mark(6)
-        bwd = capi.moe_grouped_ffn_bwd_recompute if args.recompute else capi.moe_grouped_ffn_bwd
+        bwd = capi.moe_grouped_ffn_bwd_recompute if self.recompute else capi.moe_grouped_ffn_bwd
         bwd(s, fdt, L.rows, L.dy_perm, L.x_perm, L.act, L.ffn_offsets, w1, w2, L.dx_perm, L.dw1,
-            L.dw2, capi.MOE_F32, L.ws, mx=L.mx)
+            L.dw2, capi.MOE_F32 | acc, L.ws, mx=L.mx)
         mark(7)
-        capi.moe_route_bwd(s, dt, x, wr, L.logits, L.topk_idx, L.dgate, L.dx_perm, L.row_map,
-                           L.dx, L.dw_router, L.ws)
+        capi.moe_route_bwd(s, dt | acc, x, wr, L.logits, L.topk_idx, L.dgate, L.dx_perm,
+                           L.row_map, L.dx, L.dw_router, L.ws)
         mark(8)
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    if L.device_status() != 0:
-        raise SystemExit("device status reported a timeout during warm-up")
 
-    # The timed step is one CUDA-graph replay of the whole path (the library makes
-    # no host synchronisation and no allocation, so the step captures as is).
-    graph = torch.cuda.CUDAGraph()
+def capture(fn):
+    """A CUDA graph of fn() (warmed once on a side stream, as graph capture requires)."""
+    g = torch.cuda.CUDAGraph()
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):
-        step()
+        fn()
     torch.cuda.current_stream().wait_stream(side)
-    with torch.cuda.graph(graph):
-        step()
+    with torch.cuda.graph(g):
+        fn()
     torch.cuda.synchronize()
+    return g
 
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+
+def dp_timed(step_fn, steps, warmup, world, device, flush=None, sampler=None, timer="cuda"):
+    """Time `steps` calls of step_fn after `warmup` untimed ones: barrier and device
+    synchronisation on both sides, one event pair (or host clock on CPU) per step, L2
+    flushed between steps outside the events; returns (max over ranks of the total ms,
+    per-step ms of this rank)."""
+    cuda = timer == "cuda"
+    for _ in range(warmup):
+        step_fn()
+    if cuda:
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
     if world > 1:
         torch.distributed.barrier()
-    torch.cuda.synchronize()
+    if cuda:
+        torch.cuda.synchronize()
     if sampler:
         sampler.start()
         time.sleep(0.3)
-    for i in range(args.steps):
-        flush.zero_()
-        evs[i][0].record(stream)
-        graph.replay()
-        evs[i][1].record(stream)
-    torch.cuda.synchronize()
+    per = []
+    for i in range(steps):
+        if flush is not None:
+            flush.zero_()
+        if cuda:
+            evs[i][0].record()
+            step_fn()
+            evs[i][1].record()
+        else:
+            t0 = time.perf_counter()
+            step_fn()
+            per.append((time.perf_counter() - t0) * 1e3)
+    if cuda:
+        torch.cuda.synchronize()
+        per = [a.elapsed_time(b) for a, b in evs]
     if world > 1:
         torch.distributed.barrier()
     clocks = sampler.stop() if sampler else None
-    per_step = [a.elapsed_time(b) for a, b in evs]
-    total_ms = mdist.max_over_ranks(sum(per_step), device=dev)
-    ms_per_step = total_ms / args.steps
+    total = mdist.max_over_ranks(sum(per), device=device)
+    return total, per, clocks
 
-    # Phase breakdown: eager steps with CUDA events between the calls; a GPU-side
-    # delay before each step lets the host enqueue the whole step first, so the
-    # events see device time only.
-    nph = min(args.steps, 10)
-    pevs = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in range(nph)]
+
+def measure(cfg, dev, rank, world, steps, warmup, capacity=None, recompute=False, accum=1,
+            clocks=True, profile_steps=5):
+    """Timed CUDA-graph steps of one workload, then a profiled pass of eager steps.
+    Returns (LayerStep, result dict)."""
+    from mixture_experts_layer_offsets_b200 import capi
+    ls = LayerStep(cfg, dev, mdist.rank_seed(0, rank), capacity, recompute)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        ls.run()
+    torch.cuda.synchronize()
+    if ls.L.device_status() != 0:
+        raise SystemExit("device status reported a timeout during warm-up")
+    # The timed step replays CUDA graphs of the whole path (the library makes no host
+    # synchronisation and no allocation, so the calls capture as they are).
+    g_over = capture(lambda: ls.run())
+    g_acc = capture(lambda: ls.run(accumulate=True)) if accum > 1 else None
+
+    def step():
+        for m in range(accum):
+            (g_acc if m else g_over).replay()
+        if world > 1:
+            mdist.allreduce_grads(ls.grads())
+
+    sampler = ClockSampler(torch.cuda.current_device()) if (clocks and rank == 0) else None
+    total_ms, per, clk = dp_timed(step, steps, warmup, world, dev, flush, sampler)
+    ms_per_step = total_ms / steps
+    del g_over, g_acc
+
+    # Profiled pass: eager steps, a GPU-side delay first so that the host enqueues the
+    # whole step before the GPU reaches it (the events then see device time only).
+    nph = max(1, profile_steps)
+    pev = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in range(nph)]
+    kernels = {}
+    n_launch = 0
     for i in range(nph):
         flush.zero_()
         torch.cuda._sleep(3_000_000)
-        step(pevs[i])
+        with capi.Profile(256) as prof:
+            ls.run(pev[i])
+        for name, ms in prof.launches():
+            e = kernels.setdefault(name, [0, 0.0])
+            e[0] += 1
+            e[1] += ms
+        n_launch = prof.count
     torch.cuda.synchronize()
-    ph = {p: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in pevs) for i, p in enumerate(phases)}
-    status = L.device_status()
-    del graph
+    ph = {p: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in pev)
+          for i, p in enumerate(PHASES)}
+    kern = {k: {"launches_per_step": v[0] // nph, "ms_per_step": round(v[1] / nph, 4)}
+            for k, v in sorted(kernels.items(), key=lambda kv: -kv[1][1])}
+    gemm_ms = sum(v[1] for k, v in kernels.items() if k.startswith("gemm_")) / nph
+    gemm_launches = sum(v[0] for k, v in kernels.items() if k.startswith("gemm_")) // nph
+    status = ls.L.device_status()
+    res = {"ms_per_step": ms_per_step, "per_step_ms": per, "clocks": clk, "phases_ms": ph,
+           "kernels": kern, "gemm_ms": gemm_ms, "gemm_launches": gemm_launches,
+           "launches_per_micro_batch": n_launch, "device_status": status}
+    return ls, res
 
-    # e2e: through the public API with host buffers, copies inside the timed region
-    e2e = None if args.no_e2e else run_e2e(args, L, inp, dev, flush, capacity, world)
+
+def dp_line(cfg, total_ms, steps, warmup, accum, world) -> dict:
+    """The head of the JSON line: whole-job tokens/s over all ranks from the max-over-ranks
+    time of `steps` timed steps of `accum` micro-batches of T tokens per rank."""
+    ms = total_ms / steps
+    return {"metric": METRIC, "value": round(cfg.T * accum * world / (ms / 1e3), 1),
+            "unit": "tokens/s", "n_gpus": world, "steps": steps, "warmup": warmup,
+            "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": cfg.dtype,
+            "data": "synthetic (seeded; random-init weights)"}
+
+
+def roofline(cfg, res, capacity=None):
+    pk, pk_kind = _peaks()
+    flop = gemm_flop(cfg)
+    gemm_ms = res["gemm_ms"]
+    achieved = flop / (gemm_ms / 1e3) / 1e12
+    if cfg.dtype == "bf16":
+        peak, kind = pk["bf16_tflops"], f"bf16_tflops burst, {pk_kind}"
+    elif cfg.dtype == "mxfp8":
+        peak = pk["bf16_tflops"] * FP8_OVER_BF16
+        kind = f"bf16_tflops burst ({pk_kind}) x {FP8_OVER_BF16} nominal fp8/bf16 ratio"
+    else:
+        peak, kind = None, "fp32 CUDA-core path: no tensor-core peak"
+    tr = GEMM_TRAFFIC.get(cfg.name) if not capacity else None
+    traffic = tr[0] if tr and tr[1] == gemm_source_sha() else None
+    out = {"bound": "tensor",
+           "kernel": f"grouped GEMM (tcgen05): the {res['gemm_launches']} expert-FFN GEMM "
+                     "launches of a step (gemm_* in kernels_ms)",
+           "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+           "frac": round(achieved / peak, 4) if peak else None, "peak_kind": kind,
+           "traffic": traffic,
+           "traffic_unit": "DRAM bytes per step over those launches (ncu dram__bytes_read.sum "
+                           "+ dram__bytes_write.sum); null unless captured on this GEMM source",
+           "algorithmic_flop_per_step": flop, "gemm_ms_per_step": round(gemm_ms, 4),
+           "timing": "CUDA events around each GEMM launch (moe_profile_begin), eager steps"}
+    return out
+
+
+def hbm_kernels(cfg, res, capacity=None):
+    """Achieved bandwidth of the memory-bound kernels from their algorithmic bytes."""
+    pk, pk_kind = _peaks()
+    out = {}
+    for name, nbytes in kernel_bytes(cfg, capacity).items():
+        k = res["kernels"].get(name)
+        if not k or k["ms_per_step"] <= 0:
+            continue
+        gbs = nbytes / (k["ms_per_step"] / 1e3) / 1e9
+        out[name] = {"bytes_per_step": int(nbytes), "ms_per_step": k["ms_per_step"],
+                     "gb_s": round(gbs, 1), "frac_of_hbm": round(gbs / pk["hbm_gbs"], 4)}
+    return out
+
+
+def run_ours(args, rank, world):
+    cfg = resolve(args)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    from mixture_experts_layer_offsets_b200 import capi
+    shape = capi.shape_of(cfg.T, cfg.d_model, cfg.E, cfg.top_k, cfg.d_ff)
+    capacity = (capi.moe_capacity(shape, *cfg.padded_cf)
+                if args.capacity_factor and cfg.padded_cf else None)
+    accum = args.accum if args.accum else (8 if world > 1 else 1)
+    ls, res = measure(cfg, dev, rank, world, args.steps, args.warmup, capacity, args.recompute,
+                      accum)
+    e2e = None if args.no_e2e else run_e2e(args, ls, dev, capacity, world, accum)
+    del ls
+    torch.cuda.empty_cache()
+
+    sweep = None
+    if (not args.no_sweep and world == 1 and args.workload == DEFAULT_WORKLOAD and
+            not (args.tokens or args.experts or args.dtype or args.capacity_factor or
+                 args.recompute)):
+        sweep = run_sweep(args, dev)
 
     if rank != 0:
         return None
-    tokens_per_s = cfg.T * world / (ms_per_step / 1e3)
-    pk, pk_kind = _peaks()
-    gemm_ms = ph["ffn_fwd"] + ph["ffn_bwd"]
-    rows = L.rows
-    gemm_flop = 18.0 * cfg.R * cfg.d_model * cfg.d_ff   # algorithmic (dropless) FLOPs per step
-    achieved = gemm_flop / (gemm_ms / 1e3) / 1e12
-    if cfg.dtype == "bf16":
-        peak, peak_kind = pk["bf16_tflops"], f"bf16_tflops burst, {pk_kind}"
-    elif mxfp8:
-        peak = pk["bf16_tflops"] * FP8_OVER_BF16
-        peak_kind = (f"bf16_tflops burst ({pk_kind}) x {FP8_OVER_BF16} nominal fp8/bf16 ratio; "
-                     "the ffn phases include the activation quantisations")
-    else:
-        peak, peak_kind = None, "fp32 CUDA-core path: no tensor-core peak"
-    n_launch = launches_per_step(cfg, capacity, args.recompute, L.fused_dispatch)
-    line = {
-        "metric": METRIC, "value": round(tokens_per_s, 1), "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
-        "data": "synthetic (seeded; random-init weights)",
-        "config": _workload_desc(cfg, capacity, args.recompute),
-        "roofline": {
-            "bound": "tensor", "kernel": "grouped GEMM (tcgen05), all 6 launches of a step",
-            "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-            "frac": round(achieved / peak, 4) if peak else None,
-            "peak_kind": peak_kind,
-            "traffic": (GEMM_TRAFFIC_BYTES.get(cfg.name) if not capacity else None),
-            "traffic_unit": "DRAM bytes per step (6 launches), ncu dram__bytes_read.sum + dram__bytes_write.sum",
-            "algorithmic_flop_per_step": gemm_flop, "gemm_ms_per_step": round(gemm_ms, 4),
-            "rows_computed": rows,
-        },
-        "phases_ms": {k: round(v, 4) for k, v in ph.items()},
-        "timing": "value: CUDA-graph replay of the step, CUDA events per step; phases_ms and "
-                  "roofline: eager steps with events between calls (host kept ahead of the GPU)",
-        "gpu_launches": n_launch * args.steps,
-        "device_status": status,
+    line = dp_line(cfg, res["ms_per_step"] * args.steps, args.steps, args.warmup, accum, world)
+    line.update({
+        "config": _workload_desc(cfg, capacity, args.recompute, accum, world),
+        "roofline": roofline(cfg, res, capacity),
+        "hbm_kernels": hbm_kernels(cfg, res, capacity),
+        "phases_ms": {k: round(v, 4) for k, v in res["phases_ms"].items()},
+        "kernels_ms": res["kernels"],
+        "timing": "value: CUDA-graph replay of the step, CUDA events per step, max over ranks; "
+                  "phases_ms, kernels_ms and roofline: eager steps with CUDA events between "
+                  "calls and around every launch (host kept ahead of the GPU)",
+        "gpu_launches": res["launches_per_micro_batch"] * accum * args.steps,
+        "device_status": res["device_status"],
         "e2e": e2e,
-        "clocks": clocks,
-    }
+        "clocks": res["clocks"],
+    })
+    if sweep:
+        line["sweep"] = sweep
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = (cpu_baseline(cfg, budget_s=args.cpu_seconds) if not mxfp8 else
-                                {"value": None, "unit": "tokens/s", "kind": "oracle", "cores": None,
-                                 "sample": "not run: the MXFP8 oracle quantises the full FP32 "
-                                           "expert weights (2.4e9 values) on every call, which "
-                                           "alone exceeds the CPU time budget"})
+        line["cpu_baseline"] = cpu_baseline(cfg, budget_s=args.cpu_seconds)
     return line
 
 
-def run_e2e(args, L, inp, dev, flush, capacity, world):
-    """Same metric through the public API with pinned host buffers: every step copies its
-    inputs x and dout host->device and its outputs out and dx device->host, inside the
-    timed region.  Steps are pipelined the way an input pipeline would run them: two layer
-    instances take turns, and while one step computes on the compute stream, the next
-    step's inputs come in on a copy stream and the previous step's outputs go out on
-    another; events order every copy against the compute that produces or reuses its
-    buffers.  Working set per step is several times L2, so no flush is needed."""
+def run_sweep(args, dev):
+    """The comparison workloads, measured in this process with the same timing."""
+    out = {}
+    steps = min(args.steps, 10)
+    from mixture_experts_layer_offsets_b200 import capi
+    for name, padded, dtype in SWEEP:
+        cfg = inputs.CONFIGS[name]
+        if dtype:
+            cfg = inputs.shrink(cfg, name=f"{name}@{dtype}", dtype=dtype)
+        shape = capi.shape_of(cfg.T, cfg.d_model, cfg.E, cfg.top_k, cfg.d_ff)
+        capacity = capi.moe_capacity(shape, *cfg.padded_cf) if padded else None
+        ls, res = measure(cfg, dev, 0, 1, steps, 3, capacity, profile_steps=3)
+        del ls
+        torch.cuda.empty_cache()
+        rf = roofline(cfg, res, capacity)
+        key = cfg.name + ("_padded" if padded else "")
+        out[key] = {"value": round(cfg.T / (res["ms_per_step"] / 1e3), 1), "unit": "tokens/s",
+                    "ms_per_step": round(res["ms_per_step"], 4), "steps": steps,
+                    "gemm_tflops": rf["achieved"], "gemm_frac": rf["frac"],
+                    "gemm_ms_per_step": rf["gemm_ms_per_step"],
+                    "layout": "padded capacity C=%d" % capacity if capacity else "dropless",
+                    "clocks": res["clocks"], "device_status": res["device_status"]}
+    if "bf16_e8" in out and "bf16_e128" in out:
+        out["e_sweep_drop"] = round(1 - out["bf16_e128"]["value"] / out["bf16_e8"]["value"], 4)
+    if "bf16_skew_e128" in out and "bf16_skew_e128_padded" in out:
+        out["padded_over_dropless"] = round(out["bf16_skew_e128_padded"]["value"] /
+                                            out["bf16_skew_e128"]["value"], 4)
+    return out
+
+
+def run_e2e(args, ls, dev, capacity, world, accum):
+    """Same metric through the public API with pinned host buffers: every micro-batch copies
+    its inputs x and dout host->device and its outputs out and dx device->host, inside the
+    timed region.  Micro-batches are pipelined the way an input pipeline would run them: two
+    layer instances take turns (sharing one set of weight-gradient buffers), and while one
+    computes on the compute stream, the next one's inputs come in on a copy stream and the
+    previous one's outputs go out on another; events order every copy against the compute
+    that produces or reuses its buffers.  With N > 1 every `accum` micro-batches end with
+    the all-reduce of the gradients.  The working set is several times L2, so no flush."""
     from mixture_experts_layer_offsets_b200.layer import MoELayer
+    L = ls.L
     L2 = MoELayer(L.T, L.d, L.E, L.k, L.f, L.dtype, dev, dw_dtype=L.dw_dtype, capacity=capacity,
                   recompute=L.recompute)
+    L2.dw1, L2.dw2, L2.dw_router = L.dw1, L.dw2, L.dw_router
     layers = [L, L2]
+    inp = ls.inp
     hx = inp["x"].cpu().pin_memory()
     hd = inp["dout"].cpu().pin_memory()
     hout = [torch.empty_like(hx).pin_memory() for _ in range(2)]
@@ -341,14 +530,16 @@ def run_e2e(args, L, inp, dev, flush, capacity, world):
 
     def issue(i):
         k = i % 2
-        h2d.wait_event(ev_comp[k])            # step i-2 has finished reading buffer k
+        h2d.wait_event(ev_comp[k])            # micro-batch i-2 has finished reading buffer k
         with torch.cuda.stream(h2d):
             xin[k].copy_(hx, non_blocking=True)
             din[k].copy_(hd, non_blocking=True)
             ev_in[k].record(h2d)
         cs.wait_event(ev_in[k])
-        cs.wait_event(ev_out[k])              # step i-2's outputs have left layer k
-        layers[k].step(xin[k], wr, b, w1, w2, din[k])
+        cs.wait_event(ev_out[k])              # micro-batch i-2's outputs have left layer k
+        layers[k].step(xin[k], wr, b, w1, w2, din[k], accumulate=(i % accum) != 0)
+        if world > 1 and (i % accum) == accum - 1:
+            mdist.allreduce_grads([L.dw1, L.dw2, L.dw_router])
         ev_comp[k].record(cs)
         d2h.wait_event(ev_comp[k])
         with torch.cuda.stream(d2h):
@@ -356,10 +547,11 @@ def run_e2e(args, L, inp, dev, flush, capacity, world):
             hdx[k].copy_(layers[k].dx, non_blocking=True)
             ev_out[k].record(d2h)
 
-    for i in range(max(2, args.warmup)):
+    n_warm = max(2, args.warmup) * accum
+    for i in range(n_warm):
         issue(i)
     torch.cuda.synchronize()
-    n = max(2, args.steps)
+    n = max(2, args.steps) * accum
     st, en = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
@@ -379,10 +571,11 @@ def run_e2e(args, L, inp, dev, flush, capacity, world):
     nbytes = hx.numel() * hx.element_size()
     del L2
     return {"value": round(T * world / (ms / 1e3), 1), "unit": "tokens/s",
-            "h2d_bytes_per_step": 2 * nbytes, "d2h_bytes_per_step": 2 * nbytes,
-            "ms_per_step": round(ms, 4), "steps": n, "device_status": status,
-            "api": "MoELayer.step (C ABI) with pinned host buffers; copies of step i+1 in and "
-                   "i-1 out overlap step i's compute (two layer instances, three streams)"}
+            "h2d_bytes_per_step": 2 * nbytes * accum, "d2h_bytes_per_step": 2 * nbytes * accum,
+            "ms_per_micro_batch": round(ms, 4), "micro_batches": n, "device_status": status,
+            "api": "MoELayer.step (C ABI) with pinned host buffers; copies of micro-batch i+1 in "
+                   "and i-1 out overlap micro-batch i's compute (two layer instances, three "
+                   "streams)"}
 
 
 # ------------------------------------------------- CPU oracle (baseline)
@@ -397,16 +590,33 @@ def _blas_threads():
     return os.cpu_count()
 
 
-def cpu_baseline(cfg, budget_s=12.0, chunk=64):
-    """Float64 oracle fwd+bwd on micro-batches of `chunk` tokens of the workload's
-    shapes until `budget_s` seconds of CPU work have run; tokens/s."""
-    from oracle import moe_ref as ref
-    g = torch.Generator().manual_seed(0)
-    T, d, E, k, f = cfg.T, cfg.d_model, cfg.E, cfg.top_k, cfg.d_ff
+def _draw_weights(cfg, g, E):
+    T, d, f = cfg.T, cfg.d_model, cfg.d_ff
     wr = (torch.randn(E, d, generator=g) * cfg.router_std).to(cfg.act_dtype).double().numpy()
     w1 = (torch.randn(E, 2 * f, d, generator=g) * cfg.w_std).to(cfg.weight_dtype).double().numpy()
     w2 = (torch.randn(E, d, f, generator=g) * cfg.w_std).to(cfg.weight_dtype).double().numpy()
     bias = (torch.randn(E, generator=g) * cfg.bias_std).double().numpy() if cfg.bias_std else None
+    return wr, w1, w2, bias
+
+
+def cpu_baseline(cfg, budget_s=12.0, chunk=64):
+    """The float64 oracle on a bounded sample of the workload, tokens/s.
+
+    bf16 / fp32 workloads: whole oracle fwd+bwd calls on micro-batches of `chunk` tokens
+    (the full expert weights) until `budget_s` seconds have run.
+
+    MXFP8: the oracle quantises every expert weight on each call (four MXFP8 copies of the
+    FP32 masters), which at E = 128 alone is minutes of float64 work.  The step is
+    therefore extrapolated from a sample with the workload's d_model, d_ff and top_k but
+    E_s = max(top_k, 4) experts: (a) the oracle's four weight quantisations of the E_s
+    experts, timed alone, scaled by E / E_s (once per step, as the layer does); (b) one
+    oracle call on 256 tokens, minus (a), per token, scaled by T."""
+    if cfg.dtype == "mxfp8":
+        return _cpu_baseline_mx(cfg)
+    from oracle import moe_ref as ref
+    g = torch.Generator().manual_seed(0)
+    T, d, k = cfg.T, cfg.d_model, cfg.top_k
+    wr, w1, w2, bias = _draw_weights(cfg, g, cfg.E)
     done = 0
     t0 = time.perf_counter()
     while True:
@@ -418,56 +628,114 @@ def cpu_baseline(cfg, budget_s=12.0, chunk=64):
         if el >= budget_s or done >= T:
             break
     return {"value": round(done / el, 2), "unit": "tokens/s", "cores": _blas_threads(),
-            "kind": "oracle",
+            "kind": "oracle", "extrapolated": False, "sample_s": round(el, 2),
             "sample": f"{done} of {T} tokens of {cfg.name} in micro-batches of {chunk} "
                       f"(full expert weights; float64 NumPy), {el:.1f} s"}
 
 
+def _cpu_baseline_mx(cfg, tokens=256):
+    from oracle import moe_mx_ref as mxr
+    g = torch.Generator().manual_seed(0)
+    Es = max(cfg.top_k, 4)
+    d, f, k = cfg.d_model, cfg.d_ff, cfg.top_k
+    wr, w1, w2, bias = _draw_weights(cfg, g, Es)
+    t0 = time.perf_counter()
+    mxr.mx_qdq(w1.reshape(Es * 2 * f, d), 0)
+    mxr.mx_qdq(w2.reshape(Es * d, f), 0)
+    mxr.mx_qdq(w2.reshape(Es * d, f), 1)
+    mxr.mx_qdq(w1.reshape(Es * 2 * f, d), 1)
+    t_w = time.perf_counter() - t0
+    x = torch.randn(tokens, d, generator=g).to(cfg.act_dtype).double().numpy()
+    dout = torch.randn(tokens, d, generator=g).to(cfg.act_dtype).double().numpy()
+    t0 = time.perf_counter()
+    mxr.layer_fwd_bwd_mx(x, wr, w1, w2, dout, k, bias, act_round=mxr.round_bf16)
+    t_call = time.perf_counter() - t0
+    per_token = max(t_call - t_w, 1e-9) / tokens
+    step_s = t_w * cfg.E / Es + per_token * cfg.T
+    return {"value": round(cfg.T / step_s, 3), "unit": "tokens/s", "cores": _blas_threads(),
+            "kind": "oracle", "extrapolated": True, "sample_s": round(t_w + t_call, 2),
+            "extrapolated_step_s": round(step_s, 1),
+            "sample": (f"{cfg.name} extrapolated: oracle weight quantisation of {Es} of "
+                       f"{cfg.E} experts {t_w:.1f} s (x {cfg.E / Es:g}, once per step) + one "
+                       f"oracle MXFP8 layer call on {tokens} tokens with {Es} experts, "
+                       f"d_model={d}, d_ff={f}, top_k={k}: {t_call:.1f} s including its own "
+                       f"weight quantisation ({per_token * 1e3:.2f} ms per token, x {cfg.T})")}
+
+
 def run_reference(args, rank, world):
+    """The float64 oracle as the reference arm: each step is one bounded sample of the
+    workload (see cpu_baseline); ms_per_step is the time that sample took, value the rate
+    it gives for the workload (extrapolated for MXFP8)."""
     if rank != 0:
         return None
-    cfg = inputs.CONFIGS[args.workload]
-    steps = []
+    cfg = resolve(args)
     budget = max(2.0, args.cpu_seconds / max(1, args.steps))
-    for _ in range(args.warmup):
+    for _ in range(min(args.warmup, 1)):
         cpu_baseline(cfg, budget_s=min(1.0, budget))
-    for _ in range(args.steps):
-        steps.append(cpu_baseline(cfg, budget_s=budget))
+    steps = [cpu_baseline(cfg, budget_s=budget) for _ in range(args.steps)]
     v = statistics.mean(s["value"] for s in steps)
     cb = dict(steps[-1])
-    cb["value"] = round(v, 2)
-    return {"impl": "reference", "metric": METRIC, "value": round(v, 2), "unit": "tokens/s",
+    cb["value"] = round(v, 3)
+    ms = statistics.mean(s["sample_s"] for s in steps) * 1e3
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(cfg.T / v * 1e3, 3), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": _workload_desc(cfg, None), "cpu_baseline": cb,
-            "e2e": {"value": round(v, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+            "ms_per_step": round(ms, 1),
+            "ms_per_step_kind": "measured time of one sampled step (see cpu_baseline.sample)",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": _workload_desc(cfg, None), "cpu_baseline": cb,
+            "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
 
-def main():
+# ----------------------------------------------------------- launching
+def _free_port() -> int:
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def launcher_argv(n: int, argv: list[str], port: int) -> list[str]:
+    """The command that runs this script as n ranks of one node."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={n}", "--master-addr=127.0.0.1", f"--master-port={port}",
+            os.path.abspath(__file__), *argv]
+
+
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="bf16_e8", choices=sorted(inputs.CONFIGS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(inputs.CONFIGS))
     ap.add_argument("--capacity-factor", action="store_true",
                     help="padded-capacity layout (workloads that define a capacity factor)")
     ap.add_argument("--recompute", action="store_true",
                     help="backward recomputes a | u | h (moe_grouped_ffn_bwd_recompute)")
+    ap.add_argument("--accum", type=int, default=0,
+                    help="micro-batches per optimizer step (default 1 on one GPU, 8 on more)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--dtype", default=None, choices=["f32", "bf16", "mxfp8"],
                     help="run the workload's shapes at another compute dtype")
     ap.add_argument("--experts", type=int, default=0,
                     help="override E (smaller cases for profiling); not a bench line")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override T (smaller cases for profiling); not a bench line")
-    args = ap.parse_args()
-    if args.warmup < 3:
-        args.warmup = 3
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)
+    return args
+
+
+def main(argv=None):
+    argv = sys.argv[1:] if argv is None else argv
+    args = parse_args(argv)
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        if args.impl == "ours" and torch.cuda.device_count() < args.gpus:
+            raise SystemExit(f"--gpus {args.gpus}: only {torch.cuda.device_count()} GPUs visible")
+        return subprocess.call(launcher_argv(args.gpus, argv, _free_port()))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -475,10 +743,9 @@ def main():
         line = run_reference(args, rank, world)
         if line:
             print(json.dumps(line), flush=True)
-        return
+        return 0
     torch.cuda.set_device(local)
     if world > 1:
-        import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local))
     try:
@@ -488,7 +755,8 @@ def main():
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()
+    return 0
 
 
 if __name__ == "__main__":
-    main()
+    sys.exit(main())

@@ -109,6 +109,21 @@ size_t moe_workspace_size(moe_shape shape, int dtype, int64_t rows);
  * the host, unlike every other call. */
 moe_status moe_get_device_status(void* ws, void* stream, int32_t* status_out);
 
+/* ---- per-launch device timing (diagnostic) --------------------------------
+ * Between moe_profile_begin and moe_profile_end, on the calling host thread, every
+ * kernel launch made by this library's entry points is bracketed by two CUDA
+ * events recorded on the launch's stream: launch i records events[2i] right before
+ * and events[2i+1] right after it, and names[i] receives a static string naming the
+ * kernel (the expert-FFN GEMMs start with "gemm_", the router's with "router_").
+ * events: host array of 2*capacity cudaEvent_t created by the caller (timing
+ * enabled, on the device of the launches); names: host array of capacity entries.
+ * Launches beyond capacity run unrecorded; moe_profile_end writes the number of
+ * launches made (recorded or not).  Not for use while a stream is being captured
+ * (the event records would be captured too).  begin while a profile is open, or
+ * null arguments: MOE_ERR_INVALID_ARG; end without begin: MOE_ERR_INVALID_ARG. */
+moe_status moe_profile_begin(void* const* events, const char** names, int capacity);
+moe_status moe_profile_end(int32_t* count);
+
 /* ---- a1 + a2: route ------------------------------------------------------
  * [kongchang] capacity tax: each token is routed to a few of the experts;
  * routing section: routing metadata (split sizes and expert GEMM group sizes)
@@ -143,23 +158,36 @@ moe_status moe_route(moe_shape shape, int dtype, const void* x, const void* w_ro
  *   bytes of device memory that every GPU loading the library holds until the
  *   process exits.  The call allocates nothing (no cudaMalloc, no cudaFree, no
  *   allocating library routine).
- *   Limit: the shape needs 2*r(4*E*nb) + r(4*T*top_k) bytes of scratch, where
- *   r() rounds up to a multiple of 256, nb = ceil(T / tb) and tb = 32 for
- *   E <= 256, 16 for E <= 512, else 8; above MOE_ROUTE_NOALLOC_MAX_SCRATCH the
- *   call returns MOE_ERR_UNSUPPORTED and runs nothing (use moe_route then).
- *   First call on a device: it looks up the array's device address with that
- *   device current (a one-time set-up per device); make that first call
- *   before any stream capture.
+ *   Limit: the array's first 256 bytes hold a status word (below); the shape
+ *   needs 2*r(4*E*nb) + r(4*T*top_k) bytes of scratch besides, where r() rounds
+ *   up to a multiple of 256, nb = ceil(T / tb) and tb = 32 for E <= 256, 16 for
+ *   E <= 512, else 8; above MOE_ROUTE_NOALLOC_MAX_SCRATCH - 256 bytes the call
+ *   returns MOE_ERR_UNSUPPORTED and runs nothing (use moe_route then).
+ *   Device address: every call looks up the array's device address with the
+ *   caller's device current (no allocation); the first call on a device also
+ *   loads the array, so make that first call before any stream capture.
  *   Sharing: all calls on a device use the same array, which keeps whatever
- *   the last call left in it; nothing in it has to start at zero because each
- *   call writes every scratch byte before reading it.  Calls whose kernels can
- *   overlap on the GPU (different streams without ordering between them) race
- *   on the array and produce wrong results: order them on one stream. */
+ *   the last call left in it; nothing in the scratch part has to start at zero
+ *   because each call writes every scratch byte before reading it.  Calls whose
+ *   kernels can overlap on the GPU (different streams without ordering between
+ *   them) race on the array and produce wrong results: order them on one stream.
+ *   Errors on the device: the array's status word works like the workspace
+ *   status word of moe_route.  It is zero when the library is loaded; a kernel
+ *   that gives up a bounded wait sets it to MOE_ERR_TIMEOUT (its outputs are then
+ *   incomplete) and it keeps that value until moe_route_noalloc_status reads and
+ *   clears it. */
 #define MOE_ROUTE_NOALLOC_MAX_SCRATCH (4u << 20)
 moe_status moe_route_noalloc(moe_shape shape, int dtype, const void* x, const void* w_router,
                              const float* bias, float* logits, int32_t* topk_idx,
                              float* topk_gate, int32_t* counts, int32_t* offsets,
                              int32_t* slot_row, void* stream);
+
+/* Read and clear the status word of moe_route_noalloc's array on the current
+ * device: *status_out = MOE_OK or MOE_ERR_TIMEOUT (a bounded wait of a call since
+ * the last read gave up).  Diagnostic only: like moe_get_device_status it
+ * SYNCHRONISES `stream` and copies 4 bytes to the host; it allocates nothing.
+ * Order it after the calls it reports on (same stream). */
+moe_status moe_route_noalloc_status(void* stream, int32_t* status_out);
 
 /* ---- a3: rowwise permute -------------------------------------------------
  * [bytechap] how it works: rowwise dispatch places routed rows directly in
@@ -224,6 +252,37 @@ moe_status moe_mx_quantize_weights(moe_shape shape, const float* w1, const float
 moe_status moe_permute_mx(moe_shape shape, const void* x, const int32_t* slot_row,
                           const int32_t* offsets, int32_t* perm_src, void* ws, size_t ws_bytes,
                           void* stream);
+
+/* ---- MXFP8 operand copies in the workspace (diagnostic) ------------------
+ * The MXFP8 grouped FFN calls keep each quantised activation in `ws`: a row copy
+ * (E4M3 codes [rows, K] row-major, blocks of 32 along each row; E8M0 scales as
+ * 512-byte MMA atoms per 128-row tile of the row-grouped GEMMs) and a token-block
+ * copy (codes [rows, K], blocks of 32 rows within each column restarting at every
+ * expert offset; scales as atoms per 128-row stage of the token axis).  This call
+ * writes the byte offsets, from the start of `ws`, of the 20 regions below into
+ * offsets_out[0..19] (n >= 20), for a workspace sized by moe_workspace_size(shape,
+ * MOE_MXFP8, rows) (rows <= 0 means T*top_k), so that tests and debuggers can read
+ * the bytes the layer produced.  No launch and no device access.
+ *   0 x token-block codes [rows, d]      1 x token-block scale atoms
+ *   2 h token-block codes [rows, f]      3 h token-block scale atoms
+ *   4 row_tile int32 [rows]: row r -> 128 * tile + row within the tile (-1 outside)
+ *   5 token blocks int4 [rows/32 + E]: {first row, rows (1..32), stage,
+ *     block in stage | 4 if last of its expert}     6 number of token blocks (int32)
+ *   7 x row codes [rows, d]   8 x row-tile scale atoms
+ *   9 h row codes [rows, f]  10 h row-tile scale atoms
+ *  11 [da | du] bf16 [rows, 2f]
+ *  12 dy row codes [rows, d]  13 dy row-tile atoms  14 [da|du] row codes [rows, 2f]
+ *  15 [da|du] row-tile atoms  16 dy token-block codes  17 dy token-block atoms
+ *  18 [da|du] token-block codes  19 [da|du] token-block atoms
+ * Regions 0-6 hold from the forward (moe_permute_mx writes 0, 1 and 4-8) to the
+ * backward; 7-10 from the forward until the backward starts (they share memory
+ * with 11-19); 11-19 after the backward.  Atom byte of (row r, block kb) within a
+ * 128 x 4-block atom: (r % 32) * 16 + (r / 32) * 4 + kb; row-tile atom index
+ * tile * (K/128) + K/128-column block; token-block atom index stage * (K/128) +
+ * column block, with the blocks of a stage as kb (blocks past an expert's last one
+ * hold 0x7F, the scale 2^0).  d % 128 == 0 and f % 128 == 0 (else
+ * MOE_ERR_UNSUPPORTED); a bad shape or pointer: MOE_ERR_INVALID_ARG. */
+moe_status moe_mx_workspace_layout(moe_shape shape, int64_t rows, int64_t* offsets_out, int n);
 
 /* ---- a4: grouped SwiGLU FFN, forward -------------------------------------
  * [kongchang] routing section: a device-scheduled grouped GEMM handles the
@@ -352,6 +411,13 @@ moe_status mxfp8_quantize(int64_t rows, int64_t K, int src_dtype, const void* sr
  * The grouped FFN, combine, combine-bwd and route-bwd calls then take
  * rows = E*C, offsets_pad and pad_row in place of offsets and slot_row.
  * x_pad: [E*C, d]; pad_row: int32 [T,k]. */
+/* Capacity of the padded layout for capacity factor cf = cf_num / cf_den:
+ *   C = ceil(cf * T*top_k / E), computed in exact integer arithmetic
+ * ([kongchang] routing section: every expert batch padded to one uniform capacity;
+ * the comparison uses cf = 5/4).  Returns -1 for a bad shape, cf_num <= 0,
+ * cf_den <= 0, or a C above INT32_MAX.  Host only: no launch. */
+int32_t moe_capacity(moe_shape shape, int32_t cf_num, int32_t cf_den);
+
 moe_status moe_padded_dispatch(moe_shape shape, int dtype, int32_t capacity, const void* x,
                                const int32_t* topk_idx, const int32_t* slot_row,
                                const int32_t* offsets, void* x_pad, int32_t* pad_row,

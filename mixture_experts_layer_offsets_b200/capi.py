@@ -50,6 +50,11 @@ _SIGS = {
     "moe_get_device_status": (_I, [_P, _P, _P]),
     "moe_route": (_I, [moe_shape, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "moe_route_noalloc": (_I, [moe_shape, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_route_noalloc_status": (_I, [_P, _P]),
+    "moe_mx_workspace_layout": (_I, [moe_shape, _I64, _P, _I]),
+    "moe_profile_begin": (_I, [_P, _P, _I]),
+    "moe_capacity": (ctypes.c_int32, [moe_shape, ctypes.c_int32, ctypes.c_int32]),
+    "moe_profile_end": (_I, [_P]),
     "moe_permute": (_I, [moe_shape, _I, _P, _P, _P, _P, _P]),
     "moe_grouped_ffn_fwd": (_I, [moe_shape, _I, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "moe_combine": (_I, [moe_shape, _I, _P, _P, _P, _P, _P]),
@@ -90,7 +95,8 @@ def lib() -> ctypes.CDLL:
 def header_symbols() -> list[str]:
     """Entry points declared in include/moe.h."""
     txt = open(HEADER).read()
-    return sorted(set(re.findall(r"^\s*(?:moe_status|size_t|const char\*)\s+(\w+)\s*\(", txt, re.M)))
+    return sorted(set(re.findall(r"^\s*(?:moe_status|size_t|int32_t|const char\*)\s+(\w+)\s*\(",
+                                 txt, re.M)))
 
 
 def _ptr(t) -> int | None:
@@ -134,6 +140,39 @@ def moe_get_device_status(ws, stream=None) -> int:
     return out.value
 
 
+class Profile:
+    """Per-launch device times of the library's kernels (moe_profile_begin /
+    moe_profile_end): ``with Profile() as p: <calls>`` then ``p.launches()`` gives
+    (kernel name, milliseconds) per launch, in launch order."""
+
+    def __init__(self, capacity: int = 256):
+        import torch
+        self.cap = capacity
+        self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * capacity)]
+        for e in self.ev:          # CUDA events are created on their first record
+            e.record()
+        self._events = (ctypes.c_void_p * (2 * capacity))(*[e.cuda_event for e in self.ev])
+        self._names = (ctypes.c_char_p * capacity)()
+        self.count = 0
+
+    def __enter__(self):
+        _check("moe_profile_begin", lib().moe_profile_begin(self._events, self._names, self.cap))
+        return self
+
+    def __exit__(self, *exc):
+        n = ctypes.c_int32(0)
+        _check("moe_profile_end", lib().moe_profile_end(ctypes.byref(n)))
+        self.count = n.value
+        return False
+
+    def launches(self) -> list[tuple[str, float]]:
+        import torch
+        torch.cuda.synchronize()
+        n = min(self.count, self.cap)
+        return [(self._names[i].decode(), self.ev[2 * i].elapsed_time(self.ev[2 * i + 1]))
+                for i in range(n)]
+
+
 def moe_route(shape, dtype, x, w_router, bias, logits, topk_idx, topk_gate, counts, offsets,
               slot_row, ws, stream=None) -> None:
     _check("moe_route", lib().moe_route(
@@ -149,6 +188,14 @@ def moe_route_noalloc(shape, dtype, x, w_router, bias, logits, topk_idx, topk_ga
     _check("moe_route_noalloc", lib().moe_route_noalloc(
         shape, dtype, _ptr(x), _ptr(w_router), _ptr(bias), _ptr(logits), _ptr(topk_idx),
         _ptr(topk_gate), _ptr(counts), _ptr(offsets), _ptr(slot_row), _stream(stream)))
+
+
+def moe_route_noalloc_status(stream=None) -> int:
+    """Read and clear the status word of moe_route_noalloc's fixed array (synchronises)."""
+    out = ctypes.c_int32(0)
+    _check("moe_route_noalloc_status",
+           lib().moe_route_noalloc_status(_stream(stream), ctypes.byref(out)))
+    return out.value
 
 
 def moe_permute(shape, dtype, x, slot_row, x_perm, perm_src, stream=None) -> None:
@@ -213,6 +260,14 @@ def moe_mx_quantize_weights(shape, w1, w2, out, stream=None) -> None:
         shape, _ptr(w1), _ptr(w2), _ptr(out), _stream(stream)))
 
 
+def moe_capacity(shape, cf_num: int = 5, cf_den: int = 4) -> int:
+    """Uniform per-expert capacity of the padded layout (computed by the library)."""
+    c = lib().moe_capacity(shape, cf_num, cf_den)
+    if c < 0:
+        raise MoEError("moe_capacity", MOE_ERR_INVALID_ARG)
+    return c
+
+
 def moe_padded_dispatch(shape, dtype, capacity, x, topk_idx, slot_row, offsets, x_pad, pad_row,
                         offsets_pad, stream=None) -> None:
     _check("moe_padded_dispatch", lib().moe_padded_dispatch(
@@ -233,6 +288,19 @@ def moe_renorm_gates(shape, topk_gate, gate_out, stream=None) -> None:
 def moe_renorm_gates_bwd(shape, topk_gate, dgate_out, dgate, stream=None) -> None:
     _check("moe_renorm_gates_bwd", lib().moe_renorm_gates_bwd(
         shape, _ptr(topk_gate), _ptr(dgate_out), _ptr(dgate), _stream(stream)))
+
+
+MX_WS_REGIONS = ("qx1", "sx1", "qh1", "sh1", "row_tile", "blocks", "nblocks", "qx0", "sx0",
+                 "qh0", "sh0", "dadu", "qdy0", "sdy0", "qda0", "sda0", "qdy1", "sdy1", "qda1",
+                 "sda1")
+
+
+def moe_mx_workspace_layout(shape, rows: int = 0) -> dict:
+    """Byte offsets in the workspace of the MXFP8 operand copies (diagnostic)."""
+    n = len(MX_WS_REGIONS)
+    out = (ctypes.c_int64 * n)()
+    _check("moe_mx_workspace_layout", lib().moe_mx_workspace_layout(shape, rows, out, n))
+    return dict(zip(MX_WS_REGIONS, list(out)))
 
 
 def moe_permute_mx(shape, x, slot_row, offsets, perm_src, ws, stream=None) -> None:

@@ -22,6 +22,30 @@ int num_sms() {
   return cached[dev];
 }
 
+namespace {
+struct ProfState {
+  void* const* events = nullptr;  // 2 * cap cudaEvent_t of the caller
+  const char** names = nullptr;   // cap entries
+  int cap = 0;
+  int n = 0;
+  bool on = false;
+};
+thread_local ProfState g_prof;
+}  // namespace
+
+ProfScope::ProfScope(const char* name, cudaStream_t st) : st_(st), slot_(-1) {
+  if (!g_prof.on) return;
+  const int i = g_prof.n++;
+  if (i >= g_prof.cap) return;
+  slot_ = i;
+  g_prof.names[i] = name;
+  cudaEventRecord(static_cast<cudaEvent_t>(g_prof.events[2 * i]), st);
+}
+
+ProfScope::~ProfScope() {
+  if (slot_ >= 0) cudaEventRecord(static_cast<cudaEvent_t>(g_prof.events[2 * slot_ + 1]), st_);
+}
+
 }  // namespace moe
 
 using namespace moe;
@@ -87,6 +111,38 @@ const char* moe_version(void) { return "moe-b200 0.1 (sm_100a)"; }
 size_t moe_workspace_size(moe_shape shape, int dtype, int64_t rows) {
   if (shape_ok(shape) != MOE_OK) return 0;
   return ws_need(shape, dtype, rows);
+}
+
+moe_status moe_mx_workspace_layout(moe_shape s, int64_t rows, int64_t* offsets_out, int n) {
+  if (shape_ok(s) != MOE_OK || !offsets_out || n < kMxRegions) return MOE_ERR_INVALID_ARG;
+  if (s.d_model % 128 || s.d_ff % 128) return MOE_ERR_UNSUPPORTED;
+  if (rows <= 0) rows = (int64_t)s.T * s.top_k;
+  size_t r[kMxRegions];
+  ffn_mx_ws_regions(FfnShape{s.d_model, s.E, s.d_ff, rows}, r);
+  for (int i = 0; i < kMxRegions; ++i) offsets_out[i] = (int64_t)(kStatusBytes + r[i]);
+  return MOE_OK;
+}
+
+int32_t moe_capacity(moe_shape s, int32_t cf_num, int32_t cf_den) {
+  if (shape_ok(s) != MOE_OK || cf_num <= 0 || cf_den <= 0) return -1;
+  // ceil(cf_num * T * k / (cf_den * E)) in exact integer arithmetic
+  const __int128 num = (__int128)cf_num * s.T * s.top_k;
+  const __int128 den = (__int128)cf_den * s.E;
+  const __int128 c = (num + den - 1) / den;
+  return c > INT32_MAX ? -1 : (int32_t)c;
+}
+
+moe_status moe_profile_begin(void* const* events, const char** names, int capacity) {
+  if (!events || !names || capacity <= 0 || g_prof.on) return MOE_ERR_INVALID_ARG;
+  g_prof = ProfState{events, names, capacity, 0, true};
+  return MOE_OK;
+}
+
+moe_status moe_profile_end(int32_t* count) {
+  if (!count || !g_prof.on) return MOE_ERR_INVALID_ARG;
+  *count = g_prof.n;
+  g_prof = ProfState{};
+  return MOE_OK;
 }
 
 moe_status moe_get_device_status(void* ws, void* stream, int32_t* status_out) {

@@ -115,7 +115,10 @@ __global__ void __launch_bounds__(256) simt_grouped_gemm(const SimtGemm p) {
 
 cudaError_t run(const SimtGemm& p, int64_t max_tiles, cudaStream_t st) {
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(max_tiles, (int64_t)num_sms() * 8));
-  simt_grouped_gemm<<<grid, 256, 0, st>>>(p);
+  {
+    ProfScope prof("gemm_simt_f32", st);
+    simt_grouped_gemm<<<grid, 256, 0, st>>>(p);
+  }
   return cudaGetLastError();
 }
 
@@ -172,7 +175,10 @@ cudaError_t ffn_fwd_f32(const FfnShape& s, const float* x_perm, const int32_t* o
   SimtGemm g1{x_perm, d, 1, w1, d, 1, (int64_t)2 * f * d, act, 3 * f, 0, offsets, s.E, 0,
               0, 2 * f, d};
   if ((err = run(g1, bound_tiles_m(s.rows, s.E, 2 * f), st)) != cudaSuccess) return err;
-  swiglu_fwd_kernel<<<elem_grid(s.rows * f), 256, 0, st>>>(act, offsets, s.E, s.rows, f);
+  {
+    ProfScope prof("swiglu_fwd_f32", st);
+    swiglu_fwd_kernel<<<elem_grid(s.rows * f), 256, 0, st>>>(act, offsets, s.E, s.rows, f);
+  }
   if (!y_perm) return cudaGetLastError();  // recompute of a | u | h only
   SimtGemm g2{act + 2 * f, 3 * f, 1, w2, f, 1, (int64_t)d * f, y_perm, d, 0, offsets, s.E, 0,
               0, d, f};
@@ -190,7 +196,10 @@ cudaError_t ffn_bwd_f32(const FfnShape& s, const float* dy_perm, const float* x_
     // dh = dy W2[e]  (B(n=c of f, k=row of d) = W2[k][n])
     SimtGemm g1{dy_perm, d, 1, w2, 1, f, (int64_t)d * f, dadu, 2 * f, 0, offsets, E, 0, 0, f, d};
     if ((err = run(g1, bound_tiles_m(s.rows, E, f), st)) != cudaSuccess) return err;
-    swiglu_bwd_kernel<<<elem_grid(s.rows * f), 256, 0, st>>>(dadu, act, offsets, E, s.rows, f);
+    {
+      ProfScope prof("swiglu_bwd_f32", st);
+      swiglu_bwd_kernel<<<elem_grid(s.rows * f), 256, 0, st>>>(dadu, act, offsets, E, s.rows, f);
+    }
     // dx = [da|du] W1[e]  (B(n=c of d, k=row of 2f) = W1[k][n])
     SimtGemm g2{dadu, 2 * f, 1, w1, 1, d, (int64_t)2 * f * d, dx_perm, d, 0, offsets, E, 0,
                 0, d, 2 * f};

@@ -1507,6 +1507,18 @@ GemmParams with_hooks(const GemmParams& p) {
   return q;
 }
 
+// Name of a launch in per-launch timing: the expert-FFN GEMMs start with "gemm_", the
+// router's tensor-core GEMMs with "router_".
+template <int EPI, bool FP8>
+constexpr const char* gemm_name() {
+  return EPI == EPI_SWIGLU_FWD   ? (FP8 ? "gemm_swiglu_fwd_mx" : "gemm_swiglu_fwd")
+         : EPI == EPI_STORE      ? (FP8 ? "gemm_store_mx" : "gemm_store")
+         : EPI == EPI_SWIGLU_BWD ? (FP8 ? "gemm_swiglu_bwd_mx" : "gemm_swiglu_bwd")
+         : EPI == EPI_WGRAD      ? (FP8 ? "gemm_wgrad_mx" : "gemm_wgrad")
+         : EPI == EPI_ROUTER     ? "router_gemm"
+                                 : "router_dx_gemm";
+}
+
 template <int BN, bool A_MN, bool B_MN, int EPI, bool GROUP_K>
 cudaError_t launch(const GemmParams& p, int64_t tile_bound, cudaStream_t st) {
   auto kern = grouped_gemm_sm100<BN, A_MN, B_MN, EPI, GROUP_K>;
@@ -1514,6 +1526,7 @@ cudaError_t launch(const GemmParams& p, int64_t tile_bound, cudaStream_t st) {
                                          (int)Cfg<BN, false, EPI>::kSmem);
   if (err != cudaSuccess) return err;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tile_bound, num_sms()));
+  ProfScope prof(EPI == EPI_WGRAD && !p.offsets ? "router_dw_gemm" : gemm_name<EPI, false>(), st);
   kern<<<grid, kThreads, Cfg<BN, false, EPI>::kSmem, st>>>(with_hooks(p));
   return cudaGetLastError();
 }
@@ -1526,6 +1539,7 @@ cudaError_t launch_mx(const GemmParams& p, int64_t tile_bound, cudaStream_t st) 
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tile_bound, num_sms()));
+  ProfScope prof(gemm_name<EPI, true>(), st);
   kern<<<grid, kThreads, smem, st>>>(with_hooks(p));
   return cudaGetLastError();
 }
@@ -1559,6 +1573,7 @@ cudaError_t launch_pair(const GemmParams& p, int64_t pair_tile_bound, cudaStream
   }
   const int clusters = (int)std::max<int64_t>(1, std::min<int64_t>(pair_tile_bound, dev < 64 ? max_clusters[dev] : num_sms() / 2));
   cfg.gridDim = dim3(2 * clusters);
+  ProfScope prof(gemm_name<EPI, FP8>(), st);
   return cudaLaunchKernelEx(&cfg, kern, with_hooks(p));
 }
 
@@ -1602,6 +1617,7 @@ cudaError_t wgrad_reduce_launch(const GemmParams& p, int64_t M, int64_t N, float
                                 __nv_bfloat16* out16, cudaStream_t st) {
   const int64_t mn4 = M * N / 4;
   dim3 grid((unsigned)std::min<int64_t>((mn4 + 255) / 256, 16), (unsigned)p.E);
+  ProfScope prof("gemm_wgrad_reduce", st);
   wgrad_reduce_kernel<<<grid, 256, 0, st>>>(p.offsets, p.kchunk, mn4, reinterpret_cast<const float4*>(p.part),
                                             reinterpret_cast<float4*>(out32), out16, p.accumulate);
   return cudaGetLastError();
@@ -1874,6 +1890,14 @@ GemmParams mx_params(const FfnShape& s, const int32_t* offsets, int* status) {
 size_t ffn_mx_ws_bytes(const FfnShape& s) {
   const MxLayout L = mx_layout(s);
   return std::max(L.fwd_bytes, L.bwd_bytes);
+}
+
+void ffn_mx_ws_regions(const FfnShape& s, size_t out[kMxRegions]) {
+  const MxLayout L = mx_layout(s);
+  const size_t r[kMxRegions] = {L.qx1, L.sx1, L.qh1, L.sh1, L.rt, L.map, L.cnt,
+                                L.qx0, L.sx0, L.qh0, L.sh0, L.dadu, L.qdy0, L.sdy0,
+                                L.qda0, L.sda0, L.qdy1, L.sdy1, L.qda1, L.sda1};
+  for (int i = 0; i < kMxRegions; ++i) out[i] = r[i];
 }
 
 cudaError_t mx_quantize_weights(int E, int d, int f, const float* w1, const float* w2,

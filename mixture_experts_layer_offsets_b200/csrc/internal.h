@@ -47,7 +47,8 @@ cudaError_t routing_stats_launch(const int32_t* counts, int E, int capacity, flo
 cudaError_t permute_launch(bool bf16, const void* x, const int32_t* slot_row, void* x_perm,
                            int32_t* perm_src, int T, int d, int k, cudaStream_t st);
 cudaError_t combine_launch(bool bf16, const void* y_perm, const int32_t* slot_row,
-                           const float* gate, void* out, int T, int d, int k, cudaStream_t st);
+                           const float* gate, void* out, int T, int d, int k, cudaStream_t st,
+                           const char* prof_name = "combine");
 cudaError_t combine_bwd_launch(bool bf16, const void* dout, const void* y_perm,
                                const int32_t* slot_row, const float* gate, void* dy_perm,
                                float* dgate, int T, int d, int k, cudaStream_t st);
@@ -134,6 +135,10 @@ struct MxWeights {
   const uint8_t *w1_q, *w1_s, *w1t_q, *w1t_s, *w2_q, *w2_s, *w2t_q, *w2t_s;
 };
 size_t ffn_mx_ws_bytes(const FfnShape& s);
+// byte offsets (within the scratch part of the workspace) of the MXFP8 operand copies,
+// in the order documented with moe_mx_workspace_layout
+constexpr int kMxRegions = 20;
+void ffn_mx_ws_regions(const FfnShape& s, size_t out[kMxRegions]);
 cudaError_t mx_quantize_weights(int E, int d, int f, const float* w1, const float* w2,
                                 const MxWeights& w, cudaStream_t st);
 cudaError_t ffn_fwd_mx(const FfnShape& s, const void* x_perm, const int32_t* offsets,
@@ -146,5 +151,21 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
 // (accumulate: the weight gradients are added into dw1, dw2 instead of overwriting them)
 
 int num_sms();
+
+// Per-launch device timing for diagnostics (moe_profile_begin / moe_profile_end):
+// a ProfScope built right before a kernel launch records the caller's start event
+// on the launch stream, and its destructor, right after the launch, the end event.
+// Inactive (no CUDA call at all) unless a profile is open on this host thread.
+class ProfScope {
+ public:
+  ProfScope(const char* name, cudaStream_t st);
+  ~ProfScope();
+  ProfScope(const ProfScope&) = delete;
+  ProfScope& operator=(const ProfScope&) = delete;
+
+ private:
+  cudaStream_t st_;
+  int slot_;
+};
 
 }  // namespace moe

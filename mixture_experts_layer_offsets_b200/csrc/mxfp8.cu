@@ -506,13 +506,19 @@ mx_act_kernel(const __nv_bfloat16* __restrict__ src, int64_t K, int64_t ld,
 cudaError_t row_tile_launch(const int32_t* offsets, int E, int64_t rows, int32_t* out, cudaStream_t st) {
   if (rows == 0) return cudaSuccess;
   const int grid = (int)std::min<int64_t>((rows + 255) / 256, 1184);
-  row_tile_kernel<<<grid, 256, 0, st>>>(offsets, E, rows, out);
+  {
+    ProfScope prof("mx_row_tile", st);
+    row_tile_kernel<<<grid, 256, 0, st>>>(offsets, E, rows, out);
+  }
   return cudaGetLastError();
 }
 
 cudaError_t seg_blocks_launch(const int32_t* offsets, int E, int4* map, int32_t* count,
                               cudaStream_t st) {
-  seg_blocks_kernel<<<1, 1024, 0, st>>>(offsets, E, map, count);
+  {
+    ProfScope prof("mx_seg_blocks", st);
+    seg_blocks_kernel<<<1, 1024, 0, st>>>(offsets, E, map, count);
+  }
   return cudaGetLastError();
 }
 
@@ -524,8 +530,11 @@ cudaError_t mxfp8_act(int64_t rows, int E, int64_t K, int64_t ld, const void* sr
   // about 8 blocks of 128 threads per SM at a time, each looping over several token blocks
   const int64_t want = std::max<int64_t>(1, (int64_t)num_sms() * 8 / (K / 128));
   dim3 grid((unsigned)(K / 128), (unsigned)std::min<int64_t>({rows / 32 + E, want, 65535}));
-  mx_act_kernel<<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(src_bf16), K, ld, map,
-                                       count, row_tile, q_r, atoms_r, q_c, atoms_c, gather);
+  {
+    ProfScope prof("mx_act", st);
+    mx_act_kernel<<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(src_bf16), K, ld, map,
+                                         count, row_tile, q_r, atoms_r, q_c, atoms_c, gather);
+  }
   return cudaGetLastError();
 }
 
@@ -542,7 +551,10 @@ cudaError_t mxfp8_weights(const float* w, int E, int Rw, int Kw, uint8_t* q0, ui
   if (err != cudaSuccess) return err;
   const int64_t ntiles = (int64_t)E * (Rw / 64) * (Kw / 128);
   const int grid = (int)std::min<int64_t>(ntiles, (int64_t)num_sms() * std::max(per_sm, 1));
-  mx_weights_kernel<<<grid, 128, kWSmem, st>>>(w, E, Rw, Kw, q0, s0, q1, s1);
+  {
+    ProfScope prof("mx_weights", st);
+    mx_weights_kernel<<<grid, 128, kWSmem, st>>>(w, E, Rw, Kw, q0, s0, q1, s1);
+  }
   return cudaGetLastError();
 }
 
@@ -554,23 +566,29 @@ cudaError_t mxfp8_launch_ld(int64_t rows, int64_t K, int64_t ld, bool src_bf16, 
     const int64_t nblocks = rows * K / 32;
     const int64_t threads = nblocks * 4;
     const int grid = (int)((threads + 255) / 256);
-    if (src_bf16)
+    if (src_bf16) {
+      ProfScope prof("mx_rows", st);
       mx_rows_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(src),
                                                           nblocks, K / 32, ld, q, scale);
-    else
+    } else {
+      ProfScope prof("mx_rows", st);
       mx_rows_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(src), nblocks, K / 32,
                                                   ld, q, scale);
+    }
     return cudaGetLastError();
   }
   const int nsegs = seg_offsets ? nseg : 1;
   dim3 grid((unsigned)((K / 8 + 127) / 128),
             (unsigned)std::min<int64_t>(rows / 32 + nsegs + 1, 65535));
-  if (src_bf16)
+  if (src_bf16) {
+    ProfScope prof("mx_cols", st);
     mx_cols_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(src),
                                                         rows, K, ld, seg_offsets, nsegs, q, scale);
-  else
+  } else {
+    ProfScope prof("mx_cols", st);
     mx_cols_kernel<float><<<grid, 128, 0, st>>>(static_cast<const float*>(src), rows, K, ld,
                                                 seg_offsets, nsegs, q, scale);
+  }
   return cudaGetLastError();
 }
 

@@ -225,7 +225,10 @@ cudaError_t perm_src_launch(const int32_t* slot_row, int32_t* perm_src, int T, i
                             cudaStream_t st) {
   const int64_t n = (int64_t)T * k;
   if (n == 0) return cudaSuccess;
-  perm_src_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(slot_row, perm_src, n, k);
+  {
+    ProfScope prof("perm_src", st);
+    perm_src_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(slot_row, perm_src, n, k);
+  }
   return cudaGetLastError();
 }
 
@@ -233,27 +236,34 @@ cudaError_t permute_launch(bool bf16, const void* x, const int32_t* slot_row, vo
                            int32_t* perm_src, int T, int d, int k, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
   const int grid = row_grid(T);
-  if (bf16)
+  if (bf16) {
+    ProfScope prof("permute", st);
     permute_kernel<__nv_bfloat16><<<grid, kWarpsPerBlock * 32, 0, st>>>(
         static_cast<const __nv_bfloat16*>(x), slot_row, static_cast<__nv_bfloat16*>(x_perm),
         perm_src, T, d, k);
-  else
+  } else {
+    ProfScope prof("permute", st);
     permute_kernel<float><<<grid, kWarpsPerBlock * 32, 0, st>>>(
         static_cast<const float*>(x), slot_row, static_cast<float*>(x_perm), perm_src, T, d, k);
+  }
   return cudaGetLastError();
 }
 
 cudaError_t combine_launch(bool bf16, const void* y_perm, const int32_t* slot_row,
-                           const float* gate, void* out, int T, int d, int k, cudaStream_t st) {
+                           const float* gate, void* out, int T, int d, int k, cudaStream_t st,
+                           const char* prof_name) {
   if (T == 0) return cudaSuccess;
   const int grid = row_grid(T);
-  if (bf16)
+  if (bf16) {
+    ProfScope prof(prof_name, st);
     combine_kernel<__nv_bfloat16><<<grid, kWarpsPerBlock * 32, 0, st>>>(
         static_cast<const __nv_bfloat16*>(y_perm), slot_row, gate,
         static_cast<__nv_bfloat16*>(out), T, d, k);
-  else
+  } else {
+    ProfScope prof(prof_name, st);
     combine_kernel<float><<<grid, kWarpsPerBlock * 32, 0, st>>>(
         static_cast<const float*>(y_perm), slot_row, gate, static_cast<float*>(out), T, d, k);
+  }
   return cudaGetLastError();
 }
 
@@ -262,14 +272,17 @@ static void combine_bwd_t(const void* dout, const void* y_perm, const int32_t* s
                           const float* gate, void* dy_perm, float* dgate, int ntok, int d, int k,
                           cudaStream_t st) {
   const int grid = row_grid(ntok);
-  if (k <= 8)
+  if (k <= 8) {
+    ProfScope prof("combine_bwd", st);
     combine_bwd_kernel<T, 8><<<grid, kWarpsPerBlock * 32, 0, st>>>(
         static_cast<const T*>(dout), static_cast<const T*>(y_perm), slot_row, gate,
         static_cast<T*>(dy_perm), dgate, ntok, d, k);
-  else
+  } else {
+    ProfScope prof("combine_bwd", st);
     combine_bwd_kernel<T, 32><<<grid, kWarpsPerBlock * 32, 0, st>>>(
         static_cast<const T*>(dout), static_cast<const T*>(y_perm), slot_row, gate,
         static_cast<T*>(dy_perm), dgate, ntok, d, k);
+  }
 }
 
 cudaError_t combine_bwd_launch(bool bf16, const void* dout, const void* y_perm,
@@ -290,12 +303,17 @@ static void padded_t(int C, const void* x, const int32_t* topk_idx, const int32_
   const int64_t nrows = (int64_t)E * C;
   int grid = row_grid(nrows);
   grid = std::max(grid, (E + 1 + kWarpsPerBlock * 32 - 1) / (kWarpsPerBlock * 32));
-  padded_zero_kernel<T><<<grid, kWarpsPerBlock * 32, 0, st>>>(offsets, static_cast<T*>(x_pad),
-                                                             offsets_pad, E, C, d);
-  if (ntok > 0)
+  {
+    ProfScope prof("padded_zero", st);
+    padded_zero_kernel<T><<<grid, kWarpsPerBlock * 32, 0, st>>>(offsets, static_cast<T*>(x_pad),
+                                                               offsets_pad, E, C, d);
+  }
+  if (ntok > 0) {
+    ProfScope prof("padded_dispatch", st);
     padded_dispatch_kernel<T><<<row_grid(ntok), kWarpsPerBlock * 32, 0, st>>>(
         static_cast<const T*>(x), topk_idx, slot_row, offsets, static_cast<T*>(x_pad), pad_row,
         ntok, d, k, C);
+  }
 }
 
 cudaError_t padded_dispatch_launch(bool bf16, int capacity, const void* x, const int32_t* topk_idx,

@@ -273,7 +273,15 @@ slot_rows_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict
        i += (int64_t)gridDim.x * blockDim.x) {
     const int t = (int)(i / k);
     const int e = topk_idx[i];
-    slot_row[i] = s_off[e] + blockoffs[(int64_t)e * nb + t / tb] + localrank[i];
+    // A routing pass that gave up a bounded wait leaves some indices and ranks
+    // unwritten: a pair whose expert or row falls outside its segment gets row -1
+    // (which every later step skips), so no later launch indexes out of bounds.
+    int r = -1;
+    if ((unsigned)e < (unsigned)E) {
+      r = s_off[e] + blockoffs[(int64_t)e * nb + t / tb] + localrank[i];
+      if (r < s_off[e] || r >= s_off[e + 1]) r = -1;
+    }
+    slot_row[i] = r;
   }
 }
 
@@ -284,9 +292,12 @@ cudaError_t launch_topk(const RouteArgs& a, int nb, cudaStream_t st) {
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)lg_bytes);
   if (err != cudaSuccess) return err;
-  kern<<<nb, kRouteThreads, lg_bytes, st>>>(
-      static_cast<const T*>(a.x), static_cast<const T*>(a.w_router), a.bias, a.T, a.d, a.E, a.k,
-      a.logits, a.topk_idx, a.topk_gate, a.blockcounts, a.localrank, nb);
+  {
+    ProfScope prof("router_simt", st);
+    kern<<<nb, kRouteThreads, lg_bytes, st>>>(
+        static_cast<const T*>(a.x), static_cast<const T*>(a.w_router), a.bias, a.T, a.d, a.E, a.k,
+        a.logits, a.topk_idx, a.topk_gate, a.blockcounts, a.localrank, nb);
+  }
   return cudaGetLastError();
 }
 
@@ -329,12 +340,18 @@ cudaError_t route_launch(const RouteArgs& a0, bool bf16, cudaStream_t st) {
     if (err != cudaSuccess) return err;
   }
   // With T == 0 the scan still writes zero counts and offsets.
-  block_scan_kernel<<<a.E, 256, 0, st>>>(a.blockcounts, blockoffs, nb, a.counts);
+  {
+    ProfScope prof("route_block_scan", st);
+    block_scan_kernel<<<a.E, 256, 0, st>>>(a.blockcounts, blockoffs, nb, a.counts);
+  }
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   const int64_t n = (int64_t)a.T * a.k;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 1184));
-  slot_rows_kernel<<<grid, 256, 0, st>>>(a.topk_idx, a.localrank, blockoffs, a.counts, a.T, a.E,
-                                          a.k, tb, nb, a.offsets, a.slot_row);
+  {
+    ProfScope prof("route_slot_rows", st);
+    slot_rows_kernel<<<grid, 256, 0, st>>>(a.topk_idx, a.localrank, blockoffs, a.counts, a.T, a.E,
+                                            a.k, tb, nb, a.offsets, a.slot_row);
+  }
   return cudaGetLastError();
 }
 
@@ -394,7 +411,10 @@ __global__ void __launch_bounds__(1024) routing_stats_kernel(const int32_t* __re
 
 cudaError_t routing_stats_launch(const int32_t* counts, int E, int capacity, float* stats,
                                  cudaStream_t st) {
-  routing_stats_kernel<<<1, 1024, 0, st>>>(counts, E, capacity, stats);
+  {
+    ProfScope prof("routing_stats", st);
+    routing_stats_kernel<<<1, 1024, 0, st>>>(counts, E, capacity, stats);
+  }
   return cudaGetLastError();
 }
 
@@ -440,14 +460,20 @@ __global__ void __launch_bounds__(256) renorm_gates_bwd_kernel(const float* __re
 
 cudaError_t renorm_gates_launch(const float* gate, float* out, int T, int k, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  renorm_gates_kernel<<<(T + 255) / 256, 256, 0, st>>>(gate, out, T, k);
+  {
+    ProfScope prof("renorm_gates", st);
+    renorm_gates_kernel<<<(T + 255) / 256, 256, 0, st>>>(gate, out, T, k);
+  }
   return cudaGetLastError();
 }
 
 cudaError_t renorm_gates_bwd_launch(const float* gate, const float* dgr, float* dgate, int T, int k,
                                     cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  renorm_gates_bwd_kernel<<<(T + 255) / 256, 256, 0, st>>>(gate, dgr, dgate, T, k);
+  {
+    ProfScope prof("renorm_gates_bwd", st);
+    renorm_gates_bwd_kernel<<<(T + 255) / 256, 256, 0, st>>>(gate, dgr, dgate, T, k);
+  }
   return cudaGetLastError();
 }
 
@@ -459,35 +485,25 @@ cudaError_t renorm_gates_bwd_launch(const float* gate, const float* dgr, float* 
 // latency-critical path where cudaMalloc could synchronise the device, a
 // deployment with a footprint fixed at start-up).  Its scratch is one fixed
 // array of this library instead of a caller workspace.
-#include <mutex>
-
 namespace moe {
 
-// Device scratch of moe_route_noalloc, shared by every call on a device.
+// Device scratch of moe_route_noalloc, shared by every call on a device: the first
+// kNoallocStatusBytes hold the status word of the bounded waits, the rest the route
+// scratch.  Zero at load; moe_route_noalloc_status reads and clears the status word.
+constexpr size_t kNoallocStatusBytes = 256;
 static __device__ __align__(256) uint8_t g_route_scratch[MOE_ROUTE_NOALLOC_MAX_SCRATCH];
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
-
-// In host code g_route_scratch names a host-side stand-in, not device memory:
-// the kernels get the array's device address, looked up once per device with
-// that device current.
+// In host code g_route_scratch names a host-side stand-in, not device memory: the
+// kernels get the array's device address, looked up with the caller's device current.
+// The lookup is repeated on every call (it allocates nothing and is cheap), so an
+// address never outlives the context it was taken in.
 cudaError_t noalloc_scratch(void** out) {
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
+  void* p = nullptr;
+  const cudaError_t err = cudaGetSymbolAddress(&p, g_route_scratch);
   if (err != cudaSuccess) return err;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    err = cudaGetSymbolAddress(&p, g_route_scratch);
-    if (err != cudaSuccess) return err;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return cudaSuccess;
 }
 
@@ -517,13 +533,30 @@ extern "C" moe_status moe_route_noalloc(moe_shape s, int dtype, const void* x,
       if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
   }
   if (bias && !aligned16(bias)) return MOE_ERR_INVALID_ARG;
-  // the fixed scratch bounds the shapes this variant can take
-  if (route_ws_bytes(s.T, s.E, s.top_k) > MOE_ROUTE_NOALLOC_MAX_SCRATCH) return MOE_ERR_UNSUPPORTED;
-  void* scratch = nullptr;
-  if (noalloc_scratch(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
+  // the fixed scratch (after its status word) bounds the shapes this variant can take
+  if (route_ws_bytes(s.T, s.E, s.top_k) > MOE_ROUTE_NOALLOC_MAX_SCRATCH - kNoallocStatusBytes)
+    return MOE_ERR_UNSUPPORTED;
+  void* base = nullptr;
+  if (noalloc_scratch(&base) != cudaSuccess) return MOE_ERR_CUDA;
+  uint8_t* b = static_cast<uint8_t*>(base);
   RouteArgs a{x, w_router, bias, s.T, s.d_model, s.E, s.top_k, logits, topk_idx, topk_gate,
-              counts, offsets, slot_row, scratch};
+              counts, offsets, slot_row, b + kNoallocStatusBytes, reinterpret_cast<int*>(b)};
   return route_launch(a, dtype == MOE_BF16, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
+}
+
+extern "C" moe_status moe_route_noalloc_status(void* stream, int32_t* status_out) {
+  using namespace moe;
+  if (!status_out) return MOE_ERR_INVALID_ARG;
+  void* base = nullptr;
+  if (noalloc_scratch(&base) != cudaSuccess) return MOE_ERR_CUDA;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, base, sizeof(v), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(base, 0, sizeof(v), st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  *status_out = v;
+  return MOE_OK;
 }

@@ -218,37 +218,56 @@ cudaError_t route_bwd_t(const void* x, const void* w_router, const float* logits
     // tensor cores: dl (bf16) is the A operand of both the dx and the dW_r GEMM
     __nv_bfloat16* dl_bf = static_cast<__nv_bfloat16*>(scratch);
     const int tsplits = std::max(1, std::min(32, T_ / 1024));
-    dlogit_kernel<<<lgrid, 256, 0, st>>>(logits, topk_idx, dgate, nullptr, dl_bf, T_, E, k);
+    {
+      ProfScope prof("router_dlogit", st);
+      dlogit_kernel<<<lgrid, 256, 0, st>>>(logits, topk_idx, dgate, nullptr, dl_bf, T_, E, k);
+    }
     // the k expert rows of each token are summed first by the streaming row-sum (bf16
     // [T, d] in the workspace); the dx GEMM's epilogue then adds one contiguous row
     __nv_bfloat16* dxs = reinterpret_cast<__nv_bfloat16*>(
         reinterpret_cast<uint8_t*>(partial) + align256((size_t)route_bwd_splits(T_) * E * d * 4));
-    cudaError_t err = combine_launch(true, dx_perm, slot_row, nullptr, dxs, T_, d, k, st);
+    cudaError_t err = combine_launch(true, dx_perm, slot_row, nullptr, dxs, T_, d, k, st,
+                                     "router_rowsum");
     if (err != cudaSuccess) return err;
     err = route_bwd_tc_launch(x, w_router, dl_bf, dxs, nullptr, dx, partial, tsplits, T_, d, E,
                               k, status, st);
     if (err != cudaSuccess) return err;
-    dwr_reduce_kernel<<<(int)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, st>>>(
-        partial, dw_router, n, tsplits, accumulate);
+    {
+      ProfScope prof("router_dw_reduce", st);
+      dwr_reduce_kernel<<<(int)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, st>>>(
+          partial, dw_router, n, tsplits, accumulate);
+    }
     return cudaGetLastError();
   }
   if (T_ > 0) {
-    dlogit_kernel<<<lgrid, 256, 0, st>>>(logits, topk_idx, dgate, dl, nullptr, T_, E, k);
+    {
+      ProfScope prof("router_dlogit", st);
+      dlogit_kernel<<<lgrid, 256, 0, st>>>(logits, topk_idx, dgate, dl, nullptr, T_, E, k);
+    }
     const int tpw = k <= 8 ? 4 : 1;
     const size_t dl_smem = (size_t)8 * tpw * E * sizeof(float);
     auto dxk = k <= 4 ? dx_kernel<T, 4, 4> : (k <= 8 ? dx_kernel<T, 4, 8> : dx_kernel<T, 1, 8>);
     cudaError_t err = cudaFuncSetAttribute(dxk, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)dl_smem);
     if (err != cudaSuccess) return err;
-    dxk<<<(T_ + 8 * tpw - 1) / (8 * tpw), 256, dl_smem, st>>>(dl, static_cast<const T*>(w_router),
-                                              static_cast<const T*>(dx_perm), slot_row,
-                                              static_cast<T*>(dx), T_, d, E, k);
+    {
+      ProfScope prof("router_dx_simt", st);
+      dxk<<<(T_ + 8 * tpw - 1) / (8 * tpw), 256, dl_smem, st>>>(dl, static_cast<const T*>(w_router),
+                                                static_cast<const T*>(dx_perm), slot_row,
+                                                static_cast<T*>(dx), T_, d, E, k);
+    }
     const int tps = (T_ + splits - 1) / splits;
     dim3 g2((d / V + 7) / 8, splits, (E + EB - 1) / EB);
-    dwr_partial_kernel<T, EB><<<g2, 256, 0, st>>>(dl, static_cast<const T*>(x), partial, T_, d,
-                                                  E, tps);
-    dwr_reduce_kernel<<<(int)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, st>>>(
-        partial, dw_router, n, splits, accumulate);
+    {
+      ProfScope prof("router_dw_simt", st);
+      dwr_partial_kernel<T, EB><<<g2, 256, 0, st>>>(dl, static_cast<const T*>(x), partial, T_, d,
+                                                    E, tps);
+    }
+    {
+      ProfScope prof("router_dw_reduce", st);
+      dwr_reduce_kernel<<<(int)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, st>>>(
+          partial, dw_router, n, splits, accumulate);
+    }
   } else if (!accumulate) {
     cudaMemsetAsync(dw_router, 0, n * sizeof(float), st);
   }

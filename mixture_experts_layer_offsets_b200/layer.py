@@ -24,11 +24,6 @@ from . import capi
 _DT = {"f32": capi.MOE_F32, "bf16": capi.MOE_BF16, "mxfp8": capi.MOE_MXFP8}
 
 
-def capacity_for(rows: int, E: int, cf_num: int = 5, cf_den: int = 4) -> int:
-    """Uniform per-expert capacity ceil(cf * rows / E) for cf = cf_num / cf_den."""
-    return -((-cf_num * rows) // (cf_den * E))
-
-
 class MoELayer:
     def __init__(self, T: int, d_model: int, E: int, top_k: int, d_ff: int, dtype: str = "bf16",
                  device="cuda", dw_dtype: str | None = None, capacity: int | None = None,

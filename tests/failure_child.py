@@ -1,6 +1,8 @@
-"""Child process of test_gpu_failure.py (run with the GEMM test hooks set in its
-environment): one grouped-FFN forward in which CTA 0 of every GEMM launch loses a pipeline
-stage, so that its bounded wait runs out.  Prints one line of JSON."""
+"""Child process of the failure tests (run with the GEMM test hooks set in its
+environment): one call in which CTA 0 of every tensor-core launch loses a pipeline stage,
+so that its bounded wait runs out.  Modes: "bf16" / "mxfp8" (a grouped-FFN forward with a
+workspace status word) and "route_noalloc" (the tensor-core router of moe_route_noalloc,
+whose status word sits in the library's fixed array).  Prints one line of JSON."""
 
 import json
 import os
@@ -13,7 +15,51 @@ sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
 from mixture_experts_layer_offsets_b200 import capi  # noqa: E402
 
 
+def _usable_after(dev) -> bool:
+    """The context still works: a row permute with a valid map, checked by torch."""
+    T, d, k = 600, 256, 2
+    R = T * k
+    shape = capi.shape_of(T, d, 8, k, 256)
+    slot = torch.randperm(R, device=dev).to(torch.int32).view(T, k)
+    x = torch.randn(T, d, device=dev).to(torch.bfloat16)
+    xp = torch.empty(R, d, dtype=torch.bfloat16, device=dev)
+    src = torch.empty(R, dtype=torch.int32, device=dev)
+    capi.moe_permute(shape, capi.MOE_BF16, x, slot, xp, src)
+    torch.cuda.synchronize()
+    return bool(torch.equal(xp[slot.view(-1).long()], x.repeat_interleave(k, 0)))
+
+
+def route_noalloc() -> None:
+    torch.manual_seed(0)
+    T, d, E, k = 600, 256, 8, 2
+    dev = torch.device("cuda")
+    shape = capi.shape_of(T, d, E, k, 256)
+    x = torch.randn(T, d, device=dev).to(torch.bfloat16)
+    w = (torch.randn(E, d, device=dev) * 0.05).to(torch.bfloat16)
+    logits = torch.empty(T, E, dtype=torch.float32, device=dev)
+    # indices start as a valid expert: the tile whose kernel gives up leaves them unwritten,
+    # and the slot-row pass that follows reads them
+    idx = torch.zeros(T, k, dtype=torch.int32, device=dev)
+    gate = torch.empty(T, k, dtype=torch.float32, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    slot = torch.empty(T, k, dtype=torch.int32, device=dev)
+    before = capi.moe_route_noalloc_status()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    capi.moe_route_noalloc(shape, capi.MOE_BF16, x, w, None, logits, idx, gate, counts, offsets,
+                           slot)
+    torch.cuda.synchronize()
+    elapsed = time.perf_counter() - t0
+    status = capi.moe_route_noalloc_status()
+    cleared = capi.moe_route_noalloc_status()
+    print(json.dumps({"before": before, "status": status, "cleared": cleared,
+                      "elapsed_s": elapsed, "usable_after": _usable_after(dev)}))
+
+
 def main(dtype: str) -> None:
+    if dtype == "route_noalloc":
+        return route_noalloc()
     torch.manual_seed(0)
     T, d, E, k, f = 600, 256, 8, 2, 256
     R = T * k
@@ -45,14 +91,7 @@ def main(dtype: str) -> None:
     torch.cuda.synchronize()
     elapsed = time.perf_counter() - t0
     status = capi.moe_get_device_status(ws)
-    # the context is still usable: a row permute with a valid map, then a torch op
-    slot = torch.randperm(R, device=dev).to(torch.int32).view(T, k)
-    x = torch.randn(T, d, device=dev).to(torch.bfloat16)
-    xp = torch.empty(R, d, dtype=torch.bfloat16, device=dev)
-    src = torch.empty(R, dtype=torch.int32, device=dev)
-    capi.moe_permute(shape, capi.MOE_BF16, x, slot, xp, src)
-    torch.cuda.synchronize()
-    ok_after = bool(torch.equal(xp[slot.view(-1).long()], x.repeat_interleave(k, 0)))
+    ok_after = _usable_after(dev)
     print(json.dumps({"status": status, "elapsed_s": elapsed, "usable_after": ok_after}))
 
 

@@ -109,3 +109,106 @@ def check_accumulate(cfg, dw_dtype="f32"):
             assert rel(f64(got), want.cpu().numpy()) <= TOL["bf16"], key
     # the step that accumulated still computed its own non-gradient outputs normally
     assert torch.equal(C.out, B.out) and torch.equal(C.dx, B.dx)
+
+
+# ---------------------------------------------------------------- MXFP8 operand bytes
+def _atom_byte(r, kb):
+    """Byte of (row r, 32-block kb) in a 512-byte scale atom of 128 rows x 4 blocks."""
+    return (r % 32) * 16 + (r // 32) * 4 + kb
+
+
+def expected_row_tiles(offsets) -> np.ndarray:
+    """Row -> 128 * tile + row within the tile, tiles numbered expert by expert
+    (each expert's rows start a new 128-row tile)."""
+    offsets = np.asarray(offsets, dtype=np.int64)
+    c = np.diff(offsets)
+    pre = np.concatenate([[0], np.cumsum(-(-c // 128))])
+    out = np.full(int(offsets[-1]), -1, dtype=np.int64)
+    for e in range(len(c)):
+        out[offsets[e]:offsets[e + 1]] = pre[e] * 128 + np.arange(c[e])
+    return out
+
+
+def expected_token_blocks(offsets) -> np.ndarray:
+    """The 32-row token blocks of every expert, in order: {first row, rows, 128-row
+    stage (stages numbered expert by expert), block in stage | 4 if last}."""
+    offsets = np.asarray(offsets, dtype=np.int64)
+    c = np.diff(offsets)
+    st = np.concatenate([[0], np.cumsum(-(-c // 128))])
+    rows = []
+    for e in range(len(c)):
+        nb = -(-int(c[e]) // 32)
+        for lb in range(nb):
+            rows.append((offsets[e] + 32 * lb, min(32, c[e] - 32 * lb), st[e] + lb // 4,
+                         (lb & 3) | (4 if lb == nb - 1 else 0)))
+    return np.array(rows, dtype=np.int64).reshape(-1, 4)
+
+
+def check_mx_operand(values, K, offsets, e0, e1, q_row, atoms_row, q_blk, atoms_blk, row_tile,
+                     blocks):
+    """Byte-exact check of one MXFP8 activation as the layer stores it, on the rows of
+    experts e0..e1-1 against oracle mxfp8_quantize of the same bf16 values.
+
+    values: float64 [r1 - r0, K] (the bf16 operand rows r0..r1); q_row / q_blk: u8 codes of
+    those rows (row copy, token-block copy); atoms_row / atoms_blk: the whole atom regions
+    (u8); row_tile: int [rows] (the layer's map); blocks: int [nblocks, 4] (the layer's)."""
+    from oracle import mxfp8_ref as mx
+    offsets = np.asarray(offsets, dtype=np.int64)
+    r0, r1 = int(offsets[e0]), int(offsets[e1])
+    n = r1 - r0
+    assert values.shape == (n, K)
+    kq = K // 128
+    # the maps themselves
+    assert np.array_equal(row_tile[r0:r1], expected_row_tiles(offsets)[r0:r1]), "row_tile"
+    want_blocks = expected_token_blocks(offsets)
+    sel = (want_blocks[:, 0] >= r0) & (want_blocks[:, 0] < r1)
+    assert np.array_equal(blocks[sel], want_blocks[sel]), "token blocks"
+    # row copy: codes and row-tile scale atoms
+    q0, s0 = mx.mxfp8_quantize(values, axis=0)
+    assert np.array_equal(q_row, q0), "row codes"
+    rt = row_tile[r0:r1]
+    kbg = np.arange(K // 32)
+    idx = ((rt[:, None] >> 7) * kq + kbg[None, :] // 4) * 512 + \
+        _atom_byte(rt[:, None] & 127, kbg[None, :] % 4)
+    assert np.array_equal(atoms_row[idx], s0), "row scales"
+    # token-block copy: codes (blocks restart at every expert), stage scale atoms, 2^0 pads
+    q1, s1 = mx.mxfp8_quantize(values, axis=1, seg_offsets=offsets[e0:e1 + 1] - r0)
+    assert np.array_equal(q_blk, q1), "token-block codes"
+    bl = want_blocks[sel]
+    cols = np.arange(K)
+    base = (bl[:, 2:3] * kq + cols[None, :] // 128) * 512
+    cc = cols[None, :] % 128
+    idx = base + _atom_byte(cc, bl[:, 3:4] & 3)
+    assert np.array_equal(atoms_blk[idx], s1), "token-block scales"
+    last = bl[bl[:, 3] & 4 > 0]
+    for kb in range(1, 4):
+        pad = last[(last[:, 3] & 3) < kb]
+        if len(pad):
+            pidx = (pad[:, 2:3] * kq + cols[None, :] // 128) * 512 + _atom_byte(cc, kb)
+            assert np.all(atoms_blk[pidx] == 0x7F), "pad scales"
+
+
+def routing_divergence(L, inp, gap_frac=1e-3):
+    """Tokens whose routing on the oracle's own float64 logits differs from the device's
+    (the device routes on its fp32 logits; both use the same tie rule).  Such a token is
+    allowed only where its k-th and (k+1)-th largest oracle logits lie within
+    gap_frac * max|l| of each other (a near tie that the fp32 sum may order either way).
+    Returns (number of such tokens, their largest gap as a fraction of max|l|)."""
+    x = f64(inp["x"])
+    bias = f64(inp["bias"]) if inp["bias"] is not None else None
+    lg = ref.router_logits(x, f64(inp["w_router"]), bias)
+    own = ref.route_from_logits(lg, L.k)["idx"]
+    dev = i64(L.topk_idx)
+    diff = np.nonzero((own != dev).any(axis=1))[0]
+    if len(diff) == 0:
+        return 0, 0.0
+    scale = np.abs(lg).max()
+    srt = -np.sort(-lg[diff], axis=1)
+    k = L.k
+    gap = (srt[:, k - 1] - srt[:, k]) if k < lg.shape[1] else np.zeros(len(diff))
+    # a reordering inside the selected set needs a near tie among the selected values
+    inside = np.array([np.min(np.diff(-srt[i, :k])) if k > 1 else 0.0 for i in range(len(diff))])
+    same_set = np.array([set(own[t]) == set(dev[t]) for t in diff])
+    g = np.where(same_set, inside, gap)
+    assert np.all(g <= gap_frac * scale), (diff[g > gap_frac * scale][:5], g.max() / scale)
+    return len(diff), float(g.max() / scale)

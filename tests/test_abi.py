@@ -180,3 +180,54 @@ def test_mx_quantize_weights_validation(lib):
     assert g(_shape(), None, FAKE, ctypes.addressof(mx), None) == capi.MOE_ERR_INVALID_ARG
     assert g(_shape(), FAKE, FAKE, None, None) == capi.MOE_ERR_INVALID_ARG
     assert g(_shape(), FAKE, FAKE, ctypes.addressof(_mxw(w1t_q=FAKE + 1)), None) == capi.MOE_ERR_INVALID_ARG
+
+
+def test_capacity_is_the_exact_integer_ceiling(lib):
+    # ceil(cf * T*k / E); the skewed workload: ceil(1.25 * 131072 / 128) = 1280
+    assert capi.moe_capacity(capi.shape_of(32768, 2048, 128, 4, 1024), 5, 4) == 1280
+    for T, E, k, num, den in [(3, 4, 2, 5, 4), (1, 7, 1, 5, 4), (1000, 3, 3, 1, 1), (0, 8, 2, 5, 4),
+                              (999, 64, 4, 3, 2)]:
+        want = -(-num * T * k // (den * E))
+        assert capi.moe_capacity(capi.shape_of(T, 256, E, k, 256), num, den) == want
+    assert lib.moe_capacity(_shape(), 0, 4) == -1
+    assert lib.moe_capacity(_shape(), 5, 0) == -1
+    assert lib.moe_capacity(_shape(top_k=9), 5, 4) == -1
+    assert lib.moe_capacity(capi.shape_of(1 << 28, 256, 1, 1, 256), 1 << 30, 1) == -1  # > INT32_MAX
+
+
+def test_mx_workspace_layout(lib):
+    s = capi.shape_of(500, 384, 16, 4, 384)
+    lay = capi.moe_mx_workspace_layout(s)
+    assert list(lay) == list(capi.MX_WS_REGIONS)
+    size = capi.moe_workspace_size(s, capi.MOE_MXFP8, 0)
+    R, d, f = 2000, 384, 384
+    # regions are 256-byte aligned, past the status word, and inside the workspace
+    for name, off in lay.items():
+        assert off % 256 == 0 and 256 <= off < size, name
+    assert lay["qx0"] == lay["dadu"]                    # forward row copies share with backward
+    assert lay["sx1"] - lay["qx1"] >= R * d and lay["sh1"] - lay["qh1"] >= R * f
+    assert lay["qdy0"] - lay["dadu"] >= R * 2 * f * 2
+    out = (ctypes.c_int64 * 20)()
+    assert lib.moe_mx_workspace_layout(s, 0, out, 19) == capi.MOE_ERR_INVALID_ARG
+    assert lib.moe_mx_workspace_layout(_shape(d_model=192), 0, out, 20) == capi.MOE_ERR_UNSUPPORTED
+    assert lib.moe_mx_workspace_layout(_shape(top_k=9), 0, out, 20) == capi.MOE_ERR_INVALID_ARG
+
+
+def test_profile_begin_end_bookkeeping(lib):
+    # no launch happens between begin and end here, so no event is touched
+    ev = (ctypes.c_void_p * 4)()
+    names = (ctypes.c_char_p * 2)()
+    n = ctypes.c_int32(-1)
+    assert lib.moe_profile_end(ctypes.byref(n)) == capi.MOE_ERR_INVALID_ARG      # not open
+    assert lib.moe_profile_begin(None, names, 2) == capi.MOE_ERR_INVALID_ARG
+    assert lib.moe_profile_begin(ev, names, 0) == capi.MOE_ERR_INVALID_ARG
+    assert lib.moe_profile_begin(ev, names, 2) == capi.MOE_OK
+    assert lib.moe_profile_begin(ev, names, 2) == capi.MOE_ERR_INVALID_ARG      # already open
+    # a call rejected on the host launches nothing and records nothing
+    assert lib.moe_permute(_shape(), capi.MOE_BF16, FAKE, None, FAKE, FAKE, None) == \
+        capi.MOE_ERR_INVALID_ARG
+    assert lib.moe_profile_end(ctypes.byref(n)) == capi.MOE_OK and n.value == 0
+
+
+def test_noalloc_status_validation(lib):
+    assert lib.moe_route_noalloc_status(None, None) == capi.MOE_ERR_INVALID_ARG
