@@ -37,4 +37,4 @@ check it against brute force, closed forms, library routines, hand-derived
 fixtures or finite differences (see ``tests/test_oracle_*.py``).
 """
 
-from . import moe_ref, mxfp8_ref  # noqa: F401
+from . import moe_ep_ref, moe_ref, mxfp8_ref  # noqa: F401
