@@ -189,8 +189,10 @@ def kernel_bytes(cfg, capacity=None) -> dict:
     T, d, E, k, f = cfg.T, cfg.d_model, cfg.E, cfg.top_k, cfg.d_ff
     R = E * capacity if capacity else cfg.R
     s = 4 if cfg.dtype == "f32" else 2
+    router = T * d * s + E * d * s + T * E * 4 + T * k * 12
     out = {
-        "router_gemm": T * d * s + E * d * s + T * E * 4 + T * k * 12,
+        "router_gemm": router,   # tensor-core tile router (up to 256 experts)
+        "router_mma": router,    # warp-level router (up to 32 experts)
         "permute": T * d * s + R * d * s + T * k * 8,
         "combine": R * d * s + T * d * s + T * k * 8,
         "combine_bwd": T * d * s + 2 * R * d * s + T * k * 12,

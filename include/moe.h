@@ -376,11 +376,74 @@ moe_status moe_grouped_ffn_bwd_recompute(moe_shape shape, int dtype, int64_t row
  *   dw_router = dl^T x                                   (fp32 [E, d], overwritten;
  *               added to instead with MOE_DW_ACCUMULATE OR-ed into dtype)
  * x, dx: [T, d]; w_router: [E, d]; logits fp32 [T,E]; dgate fp32 [T,k].
+ * slot_row may be NULL: dx_perm is then [T, d] and its row t, the sum of token t's
+ * expert-row gradients (as moe_ep_combine gathers them under expert parallelism), is
+ * what is added to dx[t].
  * Deterministic: fixed summation order, no floating-point atomics. */
 moe_status moe_route_bwd(moe_shape shape, int dtype, const void* x, const void* w_router,
                          const float* logits, const int32_t* topk_idx, const float* dgate,
                          const void* dx_perm, const int32_t* slot_row, void* dx,
                          float* dw_router, void* ws, size_t ws_bytes, void* stream);
+
+/* ---- f2: expert parallelism across ranks -----------------------------------
+ * [kongchang] capacity-tax section: expert parallelism spreads the routed experts over
+ * the ranks and writes only the selected token rows directly into the target rank's
+ * buffer; routing section: the exchange's split sizes never go to the host.
+ * [bytechap] how it works: each device holds a fraction of the experts, and routed rows
+ * are placed directly in the experts' input buffers.
+ * Setting: n_ranks ranks (one GPU each; n_ranks <= 64), each with its own T tokens
+ * routed over all E experts (shape.E = the total; E % n_ranks == 0).  Rank o owns the
+ * E_loc = E / n_ranks experts [o E_loc, (o + 1) E_loc).  An owner's receive buffer
+ * holds its experts' rows expert by expert, within an expert by source rank, within a
+ * source in token order: the rows one device would permute from the ranks' batches
+ * concatenated (rank 0's tokens first), in the same order.
+ * Peer buffers (peer_x, peer_y, peer_dy): a HOST array of n_ranks device pointers, entry
+ * o = rank o's buffer as mapped on the calling device (a peer mapping over NVLink, e.g.
+ * a symmetric-memory allocation, or this rank's own memory for o == rank), each with room
+ * for every row the owner can receive (n_ranks * T * top_k rows of d_model at most).  The
+ * kernels use plain loads and stores on them.  Ordering between ranks is the caller's:
+ * the rows a call writes into other ranks' memory are visible to work the owner starts
+ * after a collective (e.g. an NCCL all-reduce of one word) that follows the call on the
+ * writer's stream; a reader must likewise wait until the owner's writes are done. */
+
+/* Layout of the exchange.  counts_all: device int32 [n_ranks, E], row s = moe_route's
+ * counts on rank s (gathered by the caller, e.g. an all-gather on the device).
+ *   recv_offsets: int32 [E_loc + 1], this rank's receive-buffer segments (the last entry
+ *                 = rows received), ready for moe_grouped_ffn_fwd / _bwd with E_loc experts;
+ *   send_base:    int32 [E], for every expert e, the row of e's owner's buffer where this
+ *                 rank's rows of e begin.
+ * One launch of one block.  Bad sizes or pointers: MOE_ERR_INVALID_ARG. */
+moe_status moe_ep_layout(moe_shape shape, int n_ranks, int rank, const int32_t* counts_all,
+                         int32_t* recv_offsets, int32_t* send_base, void* stream);
+
+/* Dispatch: for every pair (t, j), x[t] is written to row
+ *   ep_row[t, j] = send_base[e] + slot_row[t, j] - offsets[e],   e = topk_idx[t, j]
+ * of peer_x[e / E_loc] (each row of x read once, 16-byte stores through the peer
+ * pointers); ep_row (int32 [T, k]) is written here for the combine steps.  x: [T, d] of
+ * dtype (MOE_F32 or MOE_BF16); topk_idx, slot_row, offsets: this rank's moe_route results;
+ * send_base: from moe_ep_layout.  A pair left unrouted by a routing pass that gave up a
+ * wait (slot_row -1) gets ep_row -1 and moves nothing. */
+moe_status moe_ep_dispatch(moe_shape shape, int dtype, int n_ranks, const void* x,
+                           const int32_t* topk_idx, const int32_t* slot_row,
+                           const int32_t* offsets, const int32_t* send_base, void* const* peer_x,
+                           int32_t* ep_row, void* stream);
+
+/* Combine from the owners' rows:
+ *   out[t] = sum_{j ascending} gate[t, j] * peer_y[e / E_loc][ep_row[t, j]]
+ * in fp32, rounded once to dtype; gate == NULL gives the plain sum (the gather of the
+ * input-gradient rows after the owners' backward, then moe_route_bwd with slot_row NULL).
+ * Rows with ep_row -1 contribute nothing.  out: [T, d]. */
+moe_status moe_ep_combine(moe_shape shape, int dtype, int n_ranks, const void* const* peer_y,
+                          const int32_t* topk_idx, const int32_t* ep_row, const float* gate,
+                          void* out, void* stream);
+
+/* Combine backward across ranks:
+ *   dgate[t, j] = <dout[t], peer_y[o][ep_row[t, j]]>,  peer_dy[o][ep_row[t, j]] = gate[t, j] dout[t]
+ * with o = topk_idx[t, j] / E_loc (fp32 dot products; dy rows written to the owners). */
+moe_status moe_ep_combine_bwd(moe_shape shape, int dtype, int n_ranks, const void* dout,
+                              const void* const* peer_y, const int32_t* topk_idx,
+                              const int32_t* ep_row, const float* gate, void* const* peer_dy,
+                              float* dgate, void* stream);
 
 /* ---- a10: MXFP8 quantisation ---------------------------------------------
  * [kongchang] boundary-conditions section: MXFP8 shares one scale among every

@@ -54,6 +54,10 @@ _SIGS = {
     "moe_mx_workspace_layout": (_I, [moe_shape, _I64, _P, _I]),
     "moe_profile_begin": (_I, [_P, _P, _I]),
     "moe_capacity": (ctypes.c_int32, [moe_shape, ctypes.c_int32, ctypes.c_int32]),
+    "moe_ep_layout": (_I, [moe_shape, _I, _I, _P, _P, _P, _P]),
+    "moe_ep_dispatch": (_I, [moe_shape, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_ep_combine": (_I, [moe_shape, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "moe_ep_combine_bwd": (_I, [moe_shape, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_profile_end": (_I, [_P]),
     "moe_permute": (_I, [moe_shape, _I, _P, _P, _P, _P, _P]),
     "moe_grouped_ffn_fwd": (_I, [moe_shape, _I, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
@@ -307,3 +311,36 @@ def moe_permute_mx(shape, x, slot_row, offsets, perm_src, ws, stream=None) -> No
     _check("moe_permute_mx", lib().moe_permute_mx(
         shape, _ptr(x), _ptr(slot_row), _ptr(offsets), _ptr(perm_src), _ptr(ws),
         ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def _ptr_array(ptrs) -> ctypes.Array:
+    """Host array of device pointers (tensors or integer addresses)."""
+    return (ctypes.c_void_p * len(ptrs))(*[_ptr(p) for p in ptrs])
+
+
+def moe_ep_layout(shape, n_ranks, rank, counts_all, recv_offsets, send_base, stream=None) -> None:
+    _check("moe_ep_layout", lib().moe_ep_layout(shape, n_ranks, rank, _ptr(counts_all),
+                                                _ptr(recv_offsets), _ptr(send_base),
+                                                _stream(stream)))
+
+
+def moe_ep_dispatch(shape, dtype, n_ranks, x, topk_idx, slot_row, offsets, send_base, peer_x,
+                    ep_row, stream=None) -> None:
+    """peer_x: the n_ranks receive buffers (tensors or device addresses)."""
+    _check("moe_ep_dispatch", lib().moe_ep_dispatch(
+        shape, dtype, n_ranks, _ptr(x), _ptr(topk_idx), _ptr(slot_row), _ptr(offsets),
+        _ptr(send_base), _ptr_array(peer_x), _ptr(ep_row), _stream(stream)))
+
+
+def moe_ep_combine(shape, dtype, n_ranks, peer_y, topk_idx, ep_row, gate, out,
+                   stream=None) -> None:
+    _check("moe_ep_combine", lib().moe_ep_combine(
+        shape, dtype, n_ranks, _ptr_array(peer_y), _ptr(topk_idx), _ptr(ep_row), _ptr(gate),
+        _ptr(out), _stream(stream)))
+
+
+def moe_ep_combine_bwd(shape, dtype, n_ranks, dout, peer_y, topk_idx, ep_row, gate, peer_dy,
+                       dgate, stream=None) -> None:
+    _check("moe_ep_combine_bwd", lib().moe_ep_combine_bwd(
+        shape, dtype, n_ranks, _ptr(dout), _ptr_array(peer_y), _ptr(topk_idx), _ptr(ep_row),
+        _ptr(gate), _ptr_array(peer_dy), _ptr(dgate), _stream(stream)))

@@ -360,13 +360,91 @@ moe_status moe_route_bwd(moe_shape s, int dtype, const void* x, const void* w_ro
   if (st != MOE_OK) return st;
   if (!dtype_act_ok(dtype)) return dtype == MOE_MXFP8 ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
   if (!ptrs_ok(w_router, dw_router, ws)) return MOE_ERR_INVALID_ARG;
-  if (s.T > 0 && !ptrs_ok(x, logits, topk_idx, dgate, dx_perm, slot_row, dx))
-    return MOE_ERR_INVALID_ARG;
+  if (s.T > 0 && !ptrs_ok(x, logits, topk_idx, dgate, dx_perm, dx)) return MOE_ERR_INVALID_ARG;
+  if (slot_row && !aligned16(slot_row)) return MOE_ERR_INVALID_ARG;
   if (ws_bytes < kStatusBytes + route_bwd_ws_bytes(s.T, s.d_model, s.E)) return MOE_ERR_INVALID_ARG;
   return cuda_status(route_bwd_launch(dtype == MOE_BF16, x, w_router, logits, topk_idx, dgate,
                                       dx_perm, slot_row, dx, dw_router, s.T, s.d_model, s.E,
                                       s.top_k, scratch(ws), status_word(ws), as_stream(stream),
                                       accumulate));
+}
+
+// ---- f2: expert parallelism across ranks
+namespace {
+// host array of n device pointers, all present and 16-byte aligned
+bool peers_ok(const void* const* peers, int n, EpPeers& out) {
+  if (!peers || n < 1 || n > kMaxRanks) return false;
+  memset(&out, 0, sizeof(out));
+  for (int i = 0; i < n; ++i) {
+    if (!peers[i] || !aligned16(peers[i])) return false;
+    out.p[i] = const_cast<void*>(peers[i]);
+  }
+  return true;
+}
+moe_status ep_args_ok(const moe_shape& s, int n_ranks) {
+  moe_status st = shape_ok(s);
+  if (st != MOE_OK) return st;
+  if (n_ranks < 1 || n_ranks > kMaxRanks || s.E % n_ranks) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+}  // namespace
+
+moe_status moe_ep_layout(moe_shape s, int n_ranks, int rank, const int32_t* counts_all,
+                         int32_t* recv_offsets, int32_t* send_base, void* stream) {
+  moe_status st = ep_args_ok(s, n_ranks);
+  if (st != MOE_OK) return st;
+  if (rank < 0 || rank >= n_ranks) return MOE_ERR_INVALID_ARG;
+  if (!ptrs_ok(counts_all, recv_offsets, send_base)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(ep_layout_launch(counts_all, n_ranks, s.E, rank, recv_offsets, send_base,
+                                      as_stream(stream)));
+}
+
+moe_status moe_ep_dispatch(moe_shape s, int dtype, int n_ranks, const void* x,
+                           const int32_t* topk_idx, const int32_t* slot_row,
+                           const int32_t* offsets, const int32_t* send_base,
+                           void* const* peer_x, int32_t* ep_row, void* stream) {
+  moe_status st = ep_args_ok(s, n_ranks);
+  if (st != MOE_OK) return st;
+  if (!dtype_act_ok(dtype)) return dtype == MOE_MXFP8 ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
+  if (s.T == 0) return MOE_OK;
+  EpPeers peers;
+  if (!peers_ok(peer_x, n_ranks, peers)) return MOE_ERR_INVALID_ARG;
+  if (!ptrs_ok(x, topk_idx, slot_row, offsets, send_base, ep_row)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(ep_dispatch_launch(dtype == MOE_BF16, x, topk_idx, slot_row, offsets,
+                                        send_base, peers, ep_row, s.T, s.d_model, s.top_k,
+                                        s.E / n_ranks, n_ranks, as_stream(stream)));
+}
+
+moe_status moe_ep_combine(moe_shape s, int dtype, int n_ranks, const void* const* peer_y,
+                          const int32_t* topk_idx, const int32_t* ep_row, const float* gate,
+                          void* out, void* stream) {
+  moe_status st = ep_args_ok(s, n_ranks);
+  if (st != MOE_OK) return st;
+  if (!dtype_act_ok(dtype)) return dtype == MOE_MXFP8 ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
+  if (s.T == 0) return MOE_OK;
+  EpPeers peers;
+  if (!peers_ok(peer_y, n_ranks, peers)) return MOE_ERR_INVALID_ARG;
+  if (!ptrs_ok(topk_idx, ep_row, out)) return MOE_ERR_INVALID_ARG;
+  if (gate && !aligned16(gate)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(ep_combine_launch(dtype == MOE_BF16, peers, topk_idx, ep_row, gate, out,
+                                       s.T, s.d_model, s.top_k, s.E / n_ranks,
+                                       as_stream(stream)));
+}
+
+moe_status moe_ep_combine_bwd(moe_shape s, int dtype, int n_ranks, const void* dout,
+                              const void* const* peer_y, const int32_t* topk_idx,
+                              const int32_t* ep_row, const float* gate, void* const* peer_dy,
+                              float* dgate, void* stream) {
+  moe_status st = ep_args_ok(s, n_ranks);
+  if (st != MOE_OK) return st;
+  if (!dtype_act_ok(dtype)) return dtype == MOE_MXFP8 ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
+  if (s.T == 0) return MOE_OK;
+  EpPeers py, pdy;
+  if (!peers_ok(peer_y, n_ranks, py) || !peers_ok(peer_dy, n_ranks, pdy)) return MOE_ERR_INVALID_ARG;
+  if (!ptrs_ok(dout, topk_idx, ep_row, gate, dgate)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(ep_combine_bwd_launch(dtype == MOE_BF16, dout, py, pdy, topk_idx, ep_row,
+                                           gate, dgate, s.T, s.d_model, s.top_k, s.E / n_ranks,
+                                           as_stream(stream)));
 }
 
 moe_status moe_mx_quantize_weights(moe_shape s, const float* w1, const float* w2,

@@ -139,9 +139,15 @@ template <int BN, bool PAIR = false, int EPI = 1, bool FP8 = false> struct Cfg {
   // accumulator buffers: two (the epilogue of one tile overlaps the main loop of the
   // next), except for 256-wide MXFP8 tiles, whose scale columns leave room for one
   static constexpr int kAccBufs = (FP8 && BN == 256) ? 1 : 2;
-  // FP8: 8 slots of 16 scale columns after the accumulators (A at +0, B atoms at +4, +8)
+  // FP8: 4 slots of 16 scale columns after the accumulators (A at +0, B atoms at +4, +8),
+  // used in rotation.  The tensor pipe runs one thread's scale copies and MMAs in issue
+  // order, so a slot is rewritten only after the MMAs of the stage that used it.
   static constexpr uint32_t kSfCol = kAccBufs * BN;
-  static_assert(!FP8 || kSfCol + 8 * 16 <= 512, "scale slots fit in TMEM");
+  static constexpr uint32_t kSfSlots = 4;
+  static_assert(!FP8 || kSfCol + kSfSlots * 16 <= 512, "scale slots fit in TMEM");
+  // columns after the scale slots, free for the epilogue (a single 256-wide accumulator
+  // leaves 192: three 32-column chunks for each of the two warps of a lane quarter)
+  static constexpr uint32_t kSpareCol = kSfCol + kSfSlots * 16;
   static constexpr uint32_t kTmemCols = FP8 ? 512 : 2 * BN;
   static constexpr int kBoxRows = BN < 128 ? BN : 128;  // rows of one K-major B box
   static constexpr int kTileM = PAIR ? 2 * BM : BM;     // rows of one scheduled tile
@@ -312,6 +318,20 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
       : MOE_R8(0), MOE_R8(8)
       : "r"(taddr));
+}
+#define MOE_S8(i) "r"(r[i + 0]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), \
+                  "r"(r[i + 4]), "r"(r[i + 5]), "r"(r[i + 6]), "r"(r[i + 7])
+// 32 consecutive fp32 columns of this thread's TMEM lane, written from registers.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      MOE_S8(0), MOE_S8(8), MOE_S8(16), MOE_S8(24)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void tmem_tie16(uint32_t (&r)[16]) {
   asm volatile("" : MOE_T8(0), MOE_T8(8));
@@ -905,10 +925,9 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
           const uint64_t ad = desc_a0 + so, bd = desc_b0 + so;
           if constexpr (FP8) {
             // scales of this stage -> TMEM, then four K = 32 block-scaled MMAs.  The
-            // scale slots rotate over 8 x 16 TMEM columns, so that the copy of the next
-            // stage's scales does not write columns that MMAs still in flight read; the
-            // scales of B atom i (rows 128 i ..) sit 4 i columns after the first.
-            const uint32_t tsf = tmem_base + C::kSfCol + 16 * (it & 7);
+            // scale slots rotate over 4 x 16 TMEM columns; the scales of B atom i (rows
+            // 128 i ..) sit 4 i columns after the first.
+            const uint32_t tsf = tmem_base + C::kSfCol + 16 * (it & (C::kSfSlots - 1));
             if constexpr (PAIR) {
               // each CTA copies its own atoms into its own TMEM; the leader's MMAs then
               // read both CTAs' A rows, B halves and scales
@@ -1068,6 +1087,30 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
         }
       } else if constexpr (EPI == EPI_SWIGLU_BWD) {
         __nv_bfloat16* drow = p.out + (int64_t)(ti.m0 + row) * p.ld_out;
+        // A single accumulator (256-wide MXFP8 tiles) would stay busy through this warp's
+        // loads of a and u and its stores, holding back the next tile's MMAs.  Instead its
+        // chunks 1..3 are parked in the spare TMEM columns and chunk 0 is kept in registers,
+        // so the accumulator is released at once.
+        constexpr bool kPark = C::kAccBufs == 1;
+        static_assert(!kPark || (kMine == 4 && C::kSpareCol + 2 * 96 <= 512),
+                      "three parked chunks per warp fit after the scale slots");
+        uint32_t v0[32];
+        const uint32_t tsp = tmem_base + ((uint32_t)(q * 32) << 16) + C::kSpareCol + half * 96;
+        if constexpr (kPark) {
+#pragma unroll
+          for (int i = 1; i < kMine; ++i) {
+            uint32_t t[32];
+            tmem_ld32(ta + (c0 + i) * 32, t);
+            tmem_wait_ld();
+            tmem_tie(t);
+            tmem_st32(tsp + (i - 1) * 32, t);
+          }
+          tmem_ld32(ta + c0 * 32, v0);
+          tmem_wait_ld();
+          tmem_tie(v0);
+          tmem_wait_st();
+          release();
+        }
 #pragma unroll
         for (int pc = 0; pc < kMine / 2; ++pc) {
           uint32_t pda[32], pdu[32];
@@ -1078,10 +1121,21 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
             uint32_t an[16], un[16];
             if (cidx + 1 < kMine && valid) load_au(arow, col + 32, p.f, an, un);  // one chunk ahead
             uint32_t v[32];
-            tmem_ld32(ta + (c0 + cidx) * 32, v);
-            tmem_wait_ld();
-            tmem_tie(v);
-            if (cidx == kMine - 1) release();
+            if constexpr (kPark) {
+              if (cidx == 0) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = v0[i];
+              } else {
+                tmem_ld32(tsp + (cidx - 1) * 32, v);
+                tmem_wait_ld();
+                tmem_tie(v);
+              }
+            } else {
+              tmem_ld32(ta + (c0 + cidx) * 32, v);
+              tmem_wait_ld();
+              tmem_tie(v);
+              if (cidx == kMine - 1) release();
+            }
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               float da[2], du[2];

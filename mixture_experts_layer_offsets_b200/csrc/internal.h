@@ -100,6 +100,27 @@ cudaError_t mxfp8_act(int64_t rows, int E, int64_t K, int64_t ld, const void* sr
 cudaError_t perm_src_launch(const int32_t* slot_row, int32_t* perm_src, int T, int k,
                             cudaStream_t st);
 
+// ------------------------------------------------------ expert parallelism
+// Peer buffers of the ranks (device pointers valid on this device: peer mappings over
+// NVLink, or this device's own memory), passed to the kernels by value.
+constexpr int kMaxRanks = 64;
+struct EpPeers {
+  void* p[kMaxRanks];
+};
+cudaError_t ep_layout_launch(const int32_t* counts_all, int N, int E, int rank,
+                             int32_t* recv_offsets, int32_t* send_base, cudaStream_t st);
+cudaError_t ep_dispatch_launch(bool bf16, const void* x, const int32_t* topk_idx,
+                               const int32_t* slot_row, const int32_t* offsets,
+                               const int32_t* send_base, const EpPeers& peers, int32_t* ep_row,
+                               int T, int d, int k, int El, int nranks, cudaStream_t st);
+cudaError_t ep_combine_launch(bool bf16, const EpPeers& peers, const int32_t* topk_idx,
+                              const int32_t* ep_row, const float* gate, void* out, int T, int d,
+                              int k, int El, cudaStream_t st);
+cudaError_t ep_combine_bwd_launch(bool bf16, const void* dout, const EpPeers& peers_y,
+                                  const EpPeers& peers_dy, const int32_t* topk_idx,
+                                  const int32_t* ep_row, const float* gate, float* dgate, int T,
+                                  int d, int k, int El, cudaStream_t st);
+
 // ---------------------------------------------------------- grouped FFN
 struct FfnShape {
   int d, E, f;

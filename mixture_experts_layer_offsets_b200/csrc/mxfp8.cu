@@ -11,8 +11,8 @@
 // floor(log2(amax)) comes straight from the fp32 exponent bits (exact, also for
 // subnormal inputs); v * 2^-e is exact in fp32 (a power-of-two scaling whose
 // result lies below 512); the element rounding is the hardware conversion
-// cvt.rn.satfinite.e4m3x2.f32 applied to |v * 2^-e|, with the sign bit set
-// from v afterwards.
+// cvt.rn.satfinite.e4m3x2.f32 applied to v * 2^-e (it carries the sign of v,
+// signed zeros included).
 #include "common.cuh"
 #include "internal.h"
 
@@ -37,13 +37,13 @@ __device__ __forceinline__ int block_exponent(float amax) {
 // 2^-e as an fp32 (e <= 119 for any finite fp32 amax, so 2^-e is normal).
 __device__ __forceinline__ float pow2_neg(int e) { return __uint_as_float((uint32_t)(127 - e) << 23); }
 
+// Two E4M3 codes (hi in the upper byte): the hardware conversion rounds to nearest even,
+// saturates at +-448 and keeps the sign, a negative value that rounds to zero included
+// (code 0x80).
 __device__ __forceinline__ uint32_t e4m3_pair(float hi, float lo) {
   uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(fabsf(hi)), "f"(fabsf(lo)));
-  uint32_t v = r;
-  if (signbit(lo)) v |= 0x80u;
-  if (signbit(hi)) v |= 0x8000u;
-  return v;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 // axis 0: a quad of lanes covers one 32-element block, 8 elements per lane.

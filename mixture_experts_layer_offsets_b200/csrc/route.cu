@@ -79,6 +79,82 @@ __device__ __forceinline__ void logits_narrow(const T* __restrict__ x, const T* 
     }
 }
 
+// Softmax and top-k of a block's TB x E logit tile in shared memory (lg, with the bias
+// already added), one warp per token: writes logits, topk_idx, topk_gate and the block's
+// selection table sel (-1 for tokens past ntok).  The lowest index wins ties.
+template <int TB>
+__device__ void topk_tile(const float* lg, int t0, int ntok, int E, int k,
+                          float* __restrict__ logits, int32_t* __restrict__ topk_idx,
+                          float* __restrict__ topk_gate, int32_t (*sel)[32]) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int r = warp; r < TB; r += kRouteThreads / 32) {
+    const int t = t0 + r;
+    if (t >= ntok) {
+      if (lane < k) sel[r][lane] = -1;
+      continue;
+    }
+    const float* row = lg + r * E;
+    float m = -INFINITY;
+    for (int e = lane; e < E; e += 32) m = fmaxf(m, row[e]);
+    m = warp_max(m);
+    float s = 0.f;
+    for (int e = lane; e < E; e += 32) {
+      s += expf(row[e] - m);
+      logits[(int64_t)t * E + e] = row[e];
+    }
+    s = warp_sum(s);
+    uint32_t taken = 0;  // bit i <-> expert lane + 32 i
+    for (int j = 0; j < k; ++j) {
+      float bv = 0.f;
+      int be = -1;
+      for (int i = 0, e = lane; e < E; ++i, e += 32) {
+        if (taken & (1u << i)) continue;
+        const float v = row[e];
+        if (be < 0 || v > bv) { bv = v; be = e; }  // ascending e: ties keep the lower index
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        if (oe >= 0 && (be < 0 || ov > bv || (ov == bv && oe < be))) { bv = ov; be = oe; }
+      }
+      if ((be & 31) == lane) taken |= 1u << (be >> 5);
+      if (lane == 0) {
+        topk_idx[(int64_t)t * k + j] = be;
+        topk_gate[(int64_t)t * k + j] = expf(bv - m) / s;
+        sel[r][j] = be;
+      }
+    }
+  }
+  __syncthreads();
+}
+
+// The block's per-expert counts (blockcounts[e * nb + block]) and each pair's rank among
+// the block's earlier pairs of the same expert (token order).
+template <int TB>
+__device__ void counts_ranks(const int32_t (*sel)[32], int t0, int ntok, int E, int k,
+                             int32_t* __restrict__ blockcounts, int32_t* __restrict__ localrank,
+                             int nb) {
+  const int tid = threadIdx.x;
+  for (int i = tid; i < TB * k; i += kRouteThreads) {
+    const int r = i / k, j = i % k;
+    const int t = t0 + r;
+    if (t >= ntok) continue;
+    const int e = sel[r][j];
+    int rank = 0;
+    for (int rr = 0; rr < r; ++rr)
+      for (int jj = 0; jj < k; ++jj) rank += (sel[rr][jj] == e);
+    localrank[(int64_t)t * k + j] = rank;
+  }
+  const int nvalid = min(TB, ntok - t0);
+  for (int e = tid; e < E; e += kRouteThreads) {
+    int c = 0;
+    for (int r = 0; r < nvalid; ++r)
+      for (int j = 0; j < k; ++j) c += (sel[r][j] == e);
+    blockcounts[(int64_t)e * nb + blockIdx.x] = c;
+  }
+}
+
 // EC experts per pass of the dot-product phase; EMAX > 0 selects the narrow
 // (E <= EMAX, TB = 32) logit phase instead of the shared-memory tiles.
 template <typename T, int TB, int EC, int EMAX>
@@ -135,67 +211,8 @@ route_topk_kernel(const T* __restrict__ x, const T* __restrict__ w, const float*
   }
   __syncthreads();
 
-  // ---- softmax + top-k: one warp per token
-  const int warp = tid >> 5, lane = tid & 31;
-  for (int r = warp; r < TB; r += kRouteThreads / 32) {
-    const int t = t0 + r;
-    if (t >= ntok) {
-      if (lane < k) sel[r][lane] = -1;
-      continue;
-    }
-    const float* row = lg + r * E;
-    float m = -INFINITY;
-    for (int e = lane; e < E; e += 32) m = fmaxf(m, row[e]);
-    m = warp_max(m);
-    float s = 0.f;
-    for (int e = lane; e < E; e += 32) {
-      s += expf(row[e] - m);
-      logits[(int64_t)t * E + e] = row[e];
-    }
-    s = warp_sum(s);
-    uint32_t taken = 0;  // bit i <-> expert lane + 32 i
-    for (int j = 0; j < k; ++j) {
-      float bv = 0.f;
-      int be = -1;
-      for (int i = 0, e = lane; e < E; ++i, e += 32) {
-        if (taken & (1u << i)) continue;
-        const float v = row[e];
-        if (be < 0 || v > bv) { bv = v; be = e; }  // ascending e: ties keep the lower index
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-        if (oe >= 0 && (be < 0 || ov > bv || (ov == bv && oe < be))) { bv = ov; be = oe; }
-      }
-      if ((be & 31) == lane) taken |= 1u << (be >> 5);
-      if (lane == 0) {
-        topk_idx[(int64_t)t * k + j] = be;
-        topk_gate[(int64_t)t * k + j] = expf(bv - m) / s;
-        sel[r][j] = be;
-      }
-    }
-  }
-  __syncthreads();
-
-  // ---- per-block counts and ranks (token order inside the block)
-  for (int i = tid; i < TB * k; i += kRouteThreads) {
-    const int r = i / k, j = i % k;
-    const int t = t0 + r;
-    if (t >= ntok) continue;
-    const int e = sel[r][j];
-    int rank = 0;
-    for (int rr = 0; rr < r; ++rr)
-      for (int jj = 0; jj < k; ++jj) rank += (sel[rr][jj] == e);
-    localrank[(int64_t)t * k + j] = rank;
-  }
-  const int nvalid = min(TB, ntok - t0);
-  for (int e = tid; e < E; e += kRouteThreads) {
-    int c = 0;
-    for (int r = 0; r < nvalid; ++r)
-      for (int j = 0; j < k; ++j) c += (sel[r][j] == e);
-    blockcounts[(int64_t)e * nb + blockIdx.x] = c;
-  }
+  topk_tile<TB>(lg, t0, ntok, E, k, logits, topk_idx, topk_gate, sel);
+  counts_ranks<TB>(sel, t0, ntok, E, k, blockcounts, localrank, nb);
 }
 
 // Exclusive scan of blockcounts[e][0..nb) for expert e = blockIdx.x.
@@ -263,8 +280,10 @@ __global__ void __launch_bounds__(256)
 slot_rows_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ localrank,
                  const int32_t* __restrict__ blockoffs, const int32_t* __restrict__ counts,
                  int ntok, int E, int k, int tb, int nb, int32_t* __restrict__ offsets,
-                 int32_t* __restrict__ slot_row) {
+                 int32_t* __restrict__ slot_row, int* __restrict__ done_reset) {
   __shared__ int32_t s_off[1025];
+  // every block of the routing pass has counted itself (stream order): ready for the next call
+  if (done_reset && blockIdx.x == 0 && threadIdx.x == 0) *done_reset = 0;
   block_offsets(counts, E, s_off);
   if (blockIdx.x == 0)
     for (int e = threadIdx.x; e <= E; e += blockDim.x) offsets[e] = s_off[e];
@@ -314,7 +333,220 @@ cudaError_t dispatch_topk(const RouteArgs& a, int nb, cudaStream_t st) {
   return launch_topk<T, 8, 64>(a, nb, st);
 }
 
+// ---- router for a few experts (bf16, E <= 32): warp-level tensor-core MMA
+// The logits are a skinny product (N = E), so the step is bound by reading x once.  Each
+// block takes 32 tokens; its 8 warps split them into two 16-token groups and d into four
+// quarters, so that the whole token range is spread evenly over every SM in one wave.  A
+// warp accumulates its 16 x 8 x NT logit fragment with mma.sync m16n8k16 (bf16 in, fp32
+// accumulate) while streaming its rows with 16-byte loads: inside each 32-column chunk,
+// lane (g, q) loads columns 8q .. 8q+7 of rows g and g+8 and of expert row g, and the two
+// K = 16 steps take elements 0-3 and 4-7 of those loads, so every column of the chunk is
+// summed exactly once (the order of the K terms inside a chunk is a fixed permutation,
+// the same for x and w_router).  The four quarters' sums are then added in quarter
+// order in shared memory, with the bias, which keeps the logits deterministic.
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <int NT>  // E <= 8 * NT
+__global__ void __launch_bounds__(kRouteThreads, NT == 1 ? 4 : 2)
+route_mma_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w,
+                 const float* __restrict__ bias, int ntok, int d, int E, int k,
+                 float* __restrict__ logits, int32_t* __restrict__ topk_idx,
+                 float* __restrict__ topk_gate, int32_t* __restrict__ blockcounts,
+                 int32_t* __restrict__ blockoffs, int32_t* __restrict__ localrank,
+                 int32_t* __restrict__ counts, int nb, int* __restrict__ done) {
+  constexpr int TB = 32;
+  constexpr int EP = 8 * NT + 1;  // padded row of the partial-sum tile
+  __shared__ float part[4][TB][EP];
+  __shared__ int32_t sel[TB][32];
+  __shared__ int s_last;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int t0 = blockIdx.x * TB;
+  const int grp = warp & 1, quarter = warp >> 1;
+  const int g = lane >> 2, q = lane & 3;
+  const int ra = t0 + 16 * grp + g, rb = ra + 8;
+  const __nv_bfloat16* xa = x + (int64_t)min(ra, ntok - 1) * d + 8 * q;
+  const __nv_bfloat16* xb = x + (int64_t)min(rb, ntok - 1) * d + 8 * q;
+  const bool va = ra < ntok, vb = rb < ntok;
+  const __nv_bfloat16* wr[NT];
+  bool we[NT];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int e = 8 * nt + g;
+    we[nt] = e < E;
+    wr[nt] = w + (int64_t)min(e, E - 1) * d + 8 * q;
+  }
+  float acc[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
+  const uint4 zero = make_uint4(0, 0, 0, 0);
+  // 64-column chunks, dealt round robin to the four warps of a token group, so that at any
+  // time the group's warps read neighbouring 128-byte pieces of the same rows; the next
+  // chunk's loads are issued before this chunk's MMAs.
+  struct Chunk { uint4 a[2], b[2], w[2][NT]; };
+  auto load = [&](int c, Chunk& k_) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      k_.a[h] = va ? ldg16(xa + c + 32 * h) : zero;
+      k_.b[h] = vb ? ldg16(xb + c + 32 * h) : zero;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) k_.w[h][nt] = we[nt] ? ldg16(wr[nt] + c + 32 * h) : zero;
+    }
+  };
+  const int nchunk = d >> 6;  // d % 128 == 0
+  Chunk cur, nxt;
+  int ch = quarter;
+  if (ch < nchunk) load(ch << 6, cur);
+  for (; ch < nchunk; ch += 4) {
+    if (ch + 4 < nchunk) load((ch + 4) << 6, nxt);
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        mma_bf16_16816(acc[nt], cur.a[h].x, cur.b[h].x, cur.a[h].y, cur.b[h].y, cur.w[h][nt].x,
+                       cur.w[h][nt].y);
+        mma_bf16_16816(acc[nt], cur.a[h].z, cur.b[h].z, cur.a[h].w, cur.b[h].w, cur.w[h][nt].z,
+                       cur.w[h][nt].w);
+      }
+    cur = nxt;
+  }
+  // fragment: acc[nt][0..1] = (row g, experts 8nt + 2q, +1), acc[nt][2..3] = row g + 8
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int e = 8 * nt + 2 * q;
+    float* p0 = &part[quarter][16 * grp + g][e];
+    float* p1 = &part[quarter][16 * grp + g + 8][e];
+    p0[0] = acc[nt][0];
+    p0[1] = acc[nt][1];
+    p1[0] = acc[nt][2];
+    p1[1] = acc[nt][3];
+  }
+  __syncthreads();
+  // Epilogue, warp 0, one lane per token with its E <= 32 logits in registers: the four
+  // quarters' partial sums added in order (+ bias), softmax, top-k (experts in ascending
+  // index, so equal logits keep the lower index), then the block's counts and each pair's
+  // rank among the earlier tokens of the block, both from one ballot per expert.
+  if (warp == 0) {
+    const int t = t0 + lane;
+    const bool valid = t < ntok;
+    float l[8 * NT];
+    float m = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < 8 * NT; ++e) {
+      l[e] = -INFINITY;
+      if (e < E) {
+        l[e] = ((part[0][lane][e] + part[1][lane][e]) + part[2][lane][e]) + part[3][lane][e] +
+               (bias ? bias[e] : 0.f);
+        m = fmaxf(m, l[e]);
+      }
+    }
+    float sum = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8 * NT; ++e)
+      if (e < E) sum += expf(l[e] - m);
+    uint32_t taken = 0;  // bit e: expert e is one of this token's selection
+    for (int j = 0; j < k; ++j) {
+      int be = -1;
+      float bv = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < 8 * NT; ++e)
+        if (e < E && !(taken >> e & 1u) && (be < 0 || l[e] > bv)) { bv = l[e]; be = e; }
+      taken |= 1u << be;
+      if (valid) {
+        topk_idx[(int64_t)t * k + j] = be;
+        topk_gate[(int64_t)t * k + j] = expf(bv - m) / sum;
+      }
+      sel[lane][j] = be;
+    }
+    if (valid) {
+#pragma unroll
+      for (int e4 = 0; e4 < 8 * NT; e4 += 4)
+        if (e4 < E) {
+          float* o = logits + (int64_t)t * E + e4;
+          if ((E & 3) == 0) {
+            *reinterpret_cast<float4*>(o) = make_float4(l[e4], l[e4 + 1], l[e4 + 2], l[e4 + 3]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              if (e4 + i < E) o[i] = l[e4 + i];
+          }
+        }
+    }
+    if (!valid) taken = 0;
+    const uint32_t below = (1u << lane) - 1u;
+    for (int e = 0; e < E; ++e) {
+      const uint32_t has = __ballot_sync(0xffffffffu, taken >> e & 1u);
+      if (lane == 0) blockcounts[(int64_t)e * nb + blockIdx.x] = __popc(has);
+      if (taken >> e & 1u) {
+        const int rank = __popc(has & below);
+        for (int j = 0; j < k; ++j)
+          if (sel[lane][j] == e) localrank[(int64_t)t * k + j] = rank;
+      }
+    }
+  }
+
+  // The last block to finish scans every block's counts (no launch of its own): each
+  // expert's exclusive prefix over the blocks, and its total.  `done` counts finished
+  // blocks; the slot-row pass that follows resets it to zero.
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(done, 1) == nb - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // one warp per expert: the counts come in rounds of 32 blocks, up to 32 rounds loaded
+  // at once (independent loads, one L2 latency), then scanned round by round
+  for (int e = warp; e < E; e += kRouteThreads / 32) {
+    const int32_t* src = blockcounts + (int64_t)e * nb;
+    int32_t* dst = blockoffs + (int64_t)e * nb;
+    int carry = 0;
+    for (int base = 0; base < nb; base += 1024) {
+      int v[32];
+#pragma unroll
+      for (int r = 0; r < 32; ++r) {
+        const int b = base + 32 * r + lane;
+        v[r] = b < nb ? __ldcg(src + b) : 0;
+      }
+#pragma unroll
+      for (int r = 0; r < 32; ++r) {
+        if (base + 32 * r >= nb) break;
+        int incl = v[r];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int n = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += n;
+        }
+        const int b = base + 32 * r + lane;
+        if (b < nb) dst[b] = carry + incl - v[r];
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+      }
+    }
+    if (lane == 0) counts[e] = carry;
+  }
+}
+
+template <int NT>
+cudaError_t launch_route_mma(const RouteArgs& a, int32_t* blockoffs, int nb, cudaStream_t st) {
+  ProfScope prof("router_mma", st);
+  route_mma_kernel<NT><<<nb, kRouteThreads, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(a.x), static_cast<const __nv_bfloat16*>(a.w_router),
+      a.bias, a.T, a.d, a.E, a.k, a.logits, a.topk_idx, a.topk_gate, a.blockcounts, blockoffs,
+      a.localrank, a.counts, nb, a.status + 1);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+bool route_mma_supported(int E, int k, int d) { return E <= 32 && k <= E && d % 128 == 0; }
 
 size_t route_ws_bytes(int T, int E, int k) {
   const int tb = route_tb(E);
@@ -324,7 +556,10 @@ size_t route_ws_bytes(int T, int E, int k) {
 
 cudaError_t route_launch(const RouteArgs& a0, bool bf16, cudaStream_t st) {
   RouteArgs a = a0;
-  const bool tc = bf16 && a.T > 0 && route_tc_supported(a.E, a.k, a.d);
+  // a few experts (bf16): the warp-level MMA router, which needs the workspace's block
+  // counter next to its status word; up to 256 experts the tensor-core tile router
+  const bool mma = bf16 && a.T > 0 && a.status && route_mma_supported(a.E, a.k, a.d);
+  const bool tc = !mma && bf16 && a.T > 0 && route_tc_supported(a.E, a.k, a.d);
   const int tb = tc ? 128 : route_tb(a.E);  // tokens per block of the count/rank pass
   const int nb = (a.T + tb - 1) / tb;
   uint8_t* ws = static_cast<uint8_t*>(a.scratch);
@@ -332,25 +567,34 @@ cudaError_t route_launch(const RouteArgs& a0, bool bf16, cudaStream_t st) {
   int32_t* blockoffs = reinterpret_cast<int32_t*>(ws + align256((size_t)nb * a.E * 4));
   a.localrank = reinterpret_cast<int32_t*>(ws + 2 * align256((size_t)nb * a.E * 4));
   cudaError_t err;
-  if (nb > 0) {
-    if (tc)
-      err = route_tc_launch(a, nb, st);
-    else
-      err = bf16 ? dispatch_topk<__nv_bfloat16>(a, nb, st) : dispatch_topk<float>(a, nb, st);
+  if (mma) {
+    // logits, top-k, block counts and (in its last block) the scan of the counts
+    err = a.E <= 8 ? launch_route_mma<1>(a, blockoffs, nb, st)
+                   : (a.E <= 16 ? launch_route_mma<2>(a, blockoffs, nb, st)
+                                : launch_route_mma<4>(a, blockoffs, nb, st));
     if (err != cudaSuccess) return err;
+  } else {
+    if (nb > 0) {
+      if (tc)
+        err = route_tc_launch(a, nb, st);
+      else
+        err = bf16 ? dispatch_topk<__nv_bfloat16>(a, nb, st) : dispatch_topk<float>(a, nb, st);
+      if (err != cudaSuccess) return err;
+    }
+    // With T == 0 the scan still writes zero counts and offsets.
+    {
+      ProfScope prof("route_block_scan", st);
+      block_scan_kernel<<<a.E, 256, 0, st>>>(a.blockcounts, blockoffs, nb, a.counts);
+    }
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
-  // With T == 0 the scan still writes zero counts and offsets.
-  {
-    ProfScope prof("route_block_scan", st);
-    block_scan_kernel<<<a.E, 256, 0, st>>>(a.blockcounts, blockoffs, nb, a.counts);
-  }
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
   const int64_t n = (int64_t)a.T * a.k;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 1184));
   {
     ProfScope prof("route_slot_rows", st);
     slot_rows_kernel<<<grid, 256, 0, st>>>(a.topk_idx, a.localrank, blockoffs, a.counts, a.T, a.E,
-                                            a.k, tb, nb, a.offsets, a.slot_row);
+                                            a.k, tb, nb, a.offsets, a.slot_row,
+                                            mma ? a.status + 1 : nullptr);
   }
   return cudaGetLastError();
 }

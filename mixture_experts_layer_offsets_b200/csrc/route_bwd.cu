@@ -72,7 +72,8 @@ dx_kernel(const float* __restrict__ dl, const T* __restrict__ w, const T* __rest
   int myrow = -1;
   if (lane < TPW * k) {
     const int t = t0 + lane / k;
-    if (t < ntok) myrow = slot_row[(int64_t)t * k + lane % k];
+    // without slot_row, dx_perm holds one row per token: the sum of its expert rows
+    if (t < ntok) myrow = slot_row ? slot_row[(int64_t)t * k + lane % k] : (lane % k ? -1 : t);
   }
   __syncwarp();
   const int chunks = d / V;
@@ -226,11 +227,13 @@ cudaError_t route_bwd_t(const void* x, const void* w_router, const float* logits
     // [T, d] in the workspace); the dx GEMM's epilogue then adds one contiguous row
     __nv_bfloat16* dxs = reinterpret_cast<__nv_bfloat16*>(
         reinterpret_cast<uint8_t*>(partial) + align256((size_t)route_bwd_splits(T_) * E * d * 4));
-    cudaError_t err = combine_launch(true, dx_perm, slot_row, nullptr, dxs, T_, d, k, st,
-                                     "router_rowsum");
+    // (without slot_row, dx_perm already holds each token's summed row)
+    cudaError_t err = slot_row ? combine_launch(true, dx_perm, slot_row, nullptr, dxs, T_, d, k,
+                                                st, "router_rowsum")
+                               : cudaSuccess;
     if (err != cudaSuccess) return err;
-    err = route_bwd_tc_launch(x, w_router, dl_bf, dxs, nullptr, dx, partial, tsplits, T_, d, E,
-                              k, status, st);
+    err = route_bwd_tc_launch(x, w_router, dl_bf, slot_row ? dxs : dx_perm, nullptr, dx, partial,
+                              tsplits, T_, d, E, k, status, st);
     if (err != cudaSuccess) return err;
     {
       ProfScope prof("router_dw_reduce", st);

@@ -31,7 +31,9 @@ def _usable_after(dev) -> bool:
 
 def route_noalloc() -> None:
     torch.manual_seed(0)
-    T, d, E, k = 600, 256, 8, 2
+    # 64 experts: the tensor-core tile router, whose pipeline waits are bounded (the
+    # warp-level router of up to 32 experts has no waits)
+    T, d, E, k = 600, 256, 64, 2
     dev = torch.device("cuda")
     shape = capi.shape_of(T, d, E, k, 256)
     x = torch.randn(T, d, device=dev).to(torch.bfloat16)
@@ -47,14 +49,17 @@ def route_noalloc() -> None:
     before = capi.moe_route_noalloc_status()
     torch.cuda.synchronize()
     t0 = time.perf_counter()
-    capi.moe_route_noalloc(shape, capi.MOE_BF16, x, w, None, logits, idx, gate, counts, offsets,
-                           slot)
+    with capi.Profile(16) as prof:
+        capi.moe_route_noalloc(shape, capi.MOE_BF16, x, w, None, logits, idx, gate, counts,
+                               offsets, slot)
     torch.cuda.synchronize()
+    names = [n for n, _ in prof.launches()]
     elapsed = time.perf_counter() - t0
     status = capi.moe_route_noalloc_status()
     cleared = capi.moe_route_noalloc_status()
     print(json.dumps({"before": before, "status": status, "cleared": cleared,
-                      "elapsed_s": elapsed, "usable_after": _usable_after(dev)}))
+                      "elapsed_s": elapsed, "usable_after": _usable_after(dev),
+                      "launches": names}))
 
 
 def main(dtype: str) -> None:

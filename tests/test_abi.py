@@ -231,3 +231,34 @@ def test_profile_begin_end_bookkeeping(lib):
 
 def test_noalloc_status_validation(lib):
     assert lib.moe_route_noalloc_status(None, None) == capi.MOE_ERR_INVALID_ARG
+
+
+def test_expert_parallel_validation(lib):
+    s = _shape()   # E = 8
+    peers2 = (ctypes.c_void_p * 2)(FAKE, FAKE)
+    bad_peers = (ctypes.c_void_p * 2)(FAKE, FAKE + 8)
+    lay = lib.moe_ep_layout
+    assert lay(s, 3, 0, FAKE, FAKE, FAKE, None) == capi.MOE_ERR_INVALID_ARG     # E % N
+    assert lay(s, 2, 2, FAKE, FAKE, FAKE, None) == capi.MOE_ERR_INVALID_ARG     # rank >= N
+    assert lay(s, 0, 0, FAKE, FAKE, FAKE, None) == capi.MOE_ERR_INVALID_ARG
+    assert lay(s, 2, 0, None, FAKE, FAKE, None) == capi.MOE_ERR_INVALID_ARG
+    assert lay(_shape(E=128, top_k=2), 65, 0, FAKE, FAKE, FAKE, None) == capi.MOE_ERR_INVALID_ARG
+    dis = lib.moe_ep_dispatch
+    args = [FAKE] * 5
+    assert dis(s, capi.MOE_BF16, 2, *args, bad_peers, FAKE, None) == capi.MOE_ERR_INVALID_ARG
+    assert dis(s, capi.MOE_BF16, 2, *args, None, FAKE, None) == capi.MOE_ERR_INVALID_ARG
+    assert dis(s, capi.MOE_MXFP8, 2, *args, peers2, FAKE, None) == capi.MOE_ERR_UNSUPPORTED
+    assert dis(s, capi.MOE_BF16, 2, FAKE, None, FAKE, FAKE, FAKE, peers2, FAKE, None) == \
+        capi.MOE_ERR_INVALID_ARG
+    assert dis(_shape(T=0), capi.MOE_BF16, 2, None, None, None, None, None, None, None,
+               None) == capi.MOE_OK
+    com = lib.moe_ep_combine
+    assert com(s, capi.MOE_BF16, 2, bad_peers, FAKE, FAKE, None, FAKE, None) == \
+        capi.MOE_ERR_INVALID_ARG
+    assert com(s, capi.MOE_BF16, 2, peers2, FAKE, FAKE, FAKE + 4, FAKE, None) == \
+        capi.MOE_ERR_INVALID_ARG
+    cb = lib.moe_ep_combine_bwd
+    assert cb(s, capi.MOE_BF16, 2, FAKE, peers2, FAKE, FAKE, FAKE, bad_peers, FAKE, None) == \
+        capi.MOE_ERR_INVALID_ARG
+    assert cb(s, capi.MOE_BF16, 2, FAKE, peers2, FAKE, FAKE, None, peers2, FAKE, None) == \
+        capi.MOE_ERR_INVALID_ARG   # gates required

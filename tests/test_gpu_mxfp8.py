@@ -75,3 +75,23 @@ def test_golden_blocks_on_device(golden_dir):
     for i, b in enumerate(fx["blocks"]):
         assert s[i, 0] == b["scale_byte"], b["note"]
         assert q[i, : len(b["codes"])].tolist() == b["codes"], b["note"]
+
+
+def test_every_finite_bf16_pattern_bytes_exact():
+    """All 65024 finite bf16 bit patterns (signed zeros and subnormals included), in a
+    fixed shuffled order, blocked along rows and along columns: the device's element codes
+    (sign of every value, ties, saturation) and scales equal the oracle's rule."""
+    bits = np.arange(1 << 16, dtype=np.uint32)
+    finite = bits[((bits >> 7) & 0xFF) != 0xFF]
+    rng = np.random.default_rng(7)
+    pat = rng.permutation(finite)
+    n = -(-len(pat) // 1024) * 1024
+    pat = np.concatenate([pat, np.zeros(n - len(pat), dtype=np.uint32)])
+    vals = (pat << 16).view(np.float32).reshape(-1, 64)
+    src = torch.from_numpy(vals.copy()).to(torch.bfloat16)   # exact: every value is a bf16
+    for axis in (0, 1):
+        q, s = _dev_quant(src, axis, [0, 333, vals.shape[0]] if axis else None)
+        segs = [0, 333, vals.shape[0]] if axis else None
+        rq, rs = mx.mxfp8_quantize(vals.astype(np.float64), axis=axis, seg_offsets=segs)
+        assert np.array_equal(q, rq), axis
+        assert np.array_equal(s[: rs.shape[0]], rs), axis

@@ -152,7 +152,8 @@ def test_no_alloc_route_matches_the_oracle(dtype):
 @pytest.mark.timeout(120)
 def test_no_alloc_route_reports_a_timeout_in_its_status_word():
     """A child process sets the library's test hooks (20 ms wait limit, CTA 0 of the
-    tensor-core router skips its second pipeline stage): the router gives up its wait,
+    tensor-core tile router, used for 64 experts, skips its second pipeline stage): the
+    router gives up its wait,
     the status word of the fixed array reads MOE_ERR_TIMEOUT, a second read finds it
     cleared, and the context still works.  Nothing traps, faults or hangs."""
     env = dict(os.environ, MOE_B200_WAIT_NS="20000000", MOE_B200_TEST_DROP_STAGE="2")
@@ -161,6 +162,7 @@ def test_no_alloc_route_reports_a_timeout_in_its_status_word():
     assert out.returncode == 0, out.stderr[-2000:]
     res = json.loads(out.stdout.strip().splitlines()[-1])
     assert res["before"] == capi.MOE_OK
+    assert res["launches"][0] == "router_gemm", res["launches"]
     assert res["status"] == capi.MOE_ERR_TIMEOUT
     assert res["cleared"] == capi.MOE_OK
     assert res["usable_after"]
