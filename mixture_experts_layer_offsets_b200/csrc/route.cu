@@ -22,6 +22,8 @@
 #include "common.cuh"
 #include "internal.h"
 
+#include <stdlib.h>
+
 namespace moe {
 
 namespace {
@@ -557,8 +559,11 @@ size_t route_ws_bytes(int T, int E, int k) {
 cudaError_t route_launch(const RouteArgs& a0, bool bf16, cudaStream_t st) {
   RouteArgs a = a0;
   // a few experts (bf16): the warp-level MMA router, which needs the workspace's block
-  // counter next to its status word; up to 256 experts the tensor-core tile router
-  const bool mma = bf16 && a.T > 0 && a.status && route_mma_supported(a.E, a.k, a.d);
+  // counter next to its status word; up to 256 experts the tensor-core tile router.
+  // MOE_B200_ROUTER=tile / warp selects one of the two where both apply (read per call).
+  const char* force = getenv("MOE_B200_ROUTER");
+  const bool no_warp = force && force[0] == 't';
+  const bool mma = !no_warp && bf16 && a.T > 0 && a.status && route_mma_supported(a.E, a.k, a.d);
   const bool tc = !mma && bf16 && a.T > 0 && route_tc_supported(a.E, a.k, a.d);
   const int tb = tc ? 128 : route_tb(a.E);  // tokens per block of the count/rank pass
   const int nb = (a.T + tb - 1) / tb;

@@ -91,3 +91,15 @@ def test_router_paths_agree_on_their_own_logits():
         b, _, names = _route(cfg, dev)
         assert names[0] == ("router_mma" if E <= 32 else "router_gemm")
         _check(cfg, cpu, b)
+
+
+def test_tile_router_on_the_same_shapes(monkeypatch):
+    """The tensor-core tile router (forced) on shapes the warp router takes by default:
+    its own logits routed by the same rule."""
+    monkeypatch.setenv("MOE_B200_ROUTER", "tile")
+    cfg = inputs.shrink(BASE, name="tile_e8", T=1000, d_model=256, E=8, top_k=4, d_ff=128)
+    cpu = inputs.make_inputs(cfg, device="cpu", seed=4)
+    dev = {k: (v.cuda() if v is not None else None) for k, v in cpu.items()}
+    b, _, names = _route(cfg, dev)
+    assert names[0] == "router_gemm", names
+    _check(cfg, cpu, b)
