@@ -257,23 +257,30 @@ moe_status moe_permute_mx(moe_shape shape, const void* x, const int32_t* slot_ro
  * The MXFP8 grouped FFN calls keep each quantised activation in `ws`: a row copy
  * (E4M3 codes [rows, K] row-major, blocks of 32 along each row; E8M0 scales as
  * 512-byte MMA atoms per 128-row tile of the row-grouped GEMMs) and a token-block
- * copy (codes [rows, K], blocks of 32 rows within each column restarting at every
- * expert offset; scales as atoms per 128-row stage of the token axis).  This call
+ * copy (codes [K][Rp], blocks of 32 rows within each column restarting at every
+ * expert offset, stored column by column; scales as atoms per 128-row stage of the
+ * token axis).  This call
  * writes the byte offsets, from the start of `ws`, of the 20 regions below into
  * offsets_out[0..19] (n >= 20), for a workspace sized by moe_workspace_size(shape,
  * MOE_MXFP8, rows) (rows <= 0 means T*top_k), so that tests and debuggers can read
- * the bytes the layer produced.  No launch and no device access.
- *   0 x token-block codes [rows, d]      1 x token-block scale atoms
- *   2 h token-block codes [rows, f]      3 h token-block scale atoms
+ * the bytes the layer produced.  No launch and no device access.  Token-block codes are
+ * column-major over a stage-padded token axis of Rp = (rows/128 + E) * 128 positions:
+ * every expert's tokens start a 128-row stage (stage numbering as for the atoms), column
+ * c's code of the token at position p is at byte c * Rp + p, and the positions past an
+ * expert's last token up to the end of its last stage hold code 0.
+ *   0 x token-block codes [d][Rp]        1 x token-block scale atoms
+ *   2 h token-block codes [f][Rp]        3 h token-block scale atoms
  *   4 row_tile int32 [rows]: row r -> 128 * tile + row within the tile (-1 outside)
  *   5 token blocks int4 [rows/32 + E]: {first row, rows (1..32), stage,
- *     block in stage | 4 if last of its expert}     6 number of token blocks (int32)
+ *     block in stage | 4 if last of its expert}, then the stage table int32
+ *     [rows/128 + E + 1]: first token block of each stage (entry nstages = nblocks)
+ *   6 int32 [2]: number of token blocks, number of stages
  *   7 x row codes [rows, d]   8 x row-tile scale atoms
  *   9 h row codes [rows, f]  10 h row-tile scale atoms
  *  11 [da | du] bf16 [rows, 2f]
  *  12 dy row codes [rows, d]  13 dy row-tile atoms  14 [da|du] row codes [rows, 2f]
- *  15 [da|du] row-tile atoms  16 dy token-block codes  17 dy token-block atoms
- *  18 [da|du] token-block codes  19 [da|du] token-block atoms
+ *  15 [da|du] row-tile atoms  16 dy token-block codes [d][Rp]  17 dy token-block atoms
+ *  18 [da|du] token-block codes [2f][Rp]  19 [da|du] token-block atoms
  * Regions 0-6 hold from the forward (moe_permute_mx writes 0, 1 and 4-8) to the
  * backward; 7-10 from the forward until the backward starts (they share memory
  * with 11-19); 11-19 after the backward.  Atom byte of (row r, block kb) within a

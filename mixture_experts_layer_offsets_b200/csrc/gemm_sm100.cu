@@ -446,9 +446,13 @@ __host__ __device__ __forceinline__ void wgrad_split(int c, int kc, int& ns, int
   ns = (c + ck - 1) / ck;
 }
 
+// GROUP_K with s_stg (MXFP8 weight gradients): the operands' token axis is stage-padded,
+// every expert's tokens starting a 128-row stage (stage prefix s_stg) and the rows past
+// its last token holding zero codes, so K runs over whole stages and nothing is zeroed.
 template <int BN, int EPI, bool GROUP_K, int TM = BM, int KE = BK>
 __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, const int* s_off,
-                                                const int* s_pre, int nN) {
+                                                const int* s_pre, int nN,
+                                                const int* s_stg = nullptr) {
   TileInfo ti;
   if constexpr (GROUP_K) {
     const int per = (p.M / BM) * nN;
@@ -477,9 +481,9 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, cons
     ti.split = j;
     ti.nsplit = ns;
     ti.kst = kb0 / 128;
-    ti.kbase = k0 + kb0;
+    ti.kbase = (s_stg ? s_stg[g] * 128 : k0) + kb0;
     ti.nkb = (kn + KE - 1) / KE;
-    ti.klast = kn - (ti.nkb - 1) * KE;
+    ti.klast = s_stg ? KE : kn - (ti.nkb - 1) * KE;
   } else {
     int lo = 0, hi = p.E - 1;
     while (lo < hi) {  // last expert whose tile prefix is <= t (skips empty experts)
@@ -652,7 +656,8 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
   };
   // this CTA's share of tile t (a pair splits the 256 rows 128 / 128)
   auto decode = [&](int t) {
-    TileInfo ti = decode_tile<BN, EPI, GROUP_K, C::kTileM, C::kBKe>(t, p, s_off, s_pre, nN);
+    TileInfo ti = decode_tile<BN, EPI, GROUP_K, C::kTileM, C::kBKe>(t, p, s_off, s_pre, nN,
+                                                                     GROUP_K && FP8 ? s_stg : nullptr);
     if constexpr (PAIR) {
       ti.m0 += BM * (int)rank;
       ti.rows = max(0, min(BM, ti.rows - BM * (int)rank));
@@ -751,9 +756,19 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
           }
           constexpr uint32_t kSfB = (BN / 128) * 512;
           mbar_arrive_expect_tx(&full[s], kABytes + C::kBBytes + 512 + kSfB);
-          if constexpr (!A_MN) tma_load_2d(sa, &p.tmA, kc, ti.m0, &full[s]);
-          else tma_load_2d(sa, &p.tmA, ti.m0, ti.kbase + kc, &full[s]);
-          if constexpr (!B_MN) {
+          if constexpr (GROUP_K) {
+            // weight gradients: A and B K-major over the stage-padded token axis
+            static_assert(!FP8 || (!A_MN && !B_MN), "MXFP8 weight-gradient operands are K-major");
+            tma_load_2d(sa, &p.tmA, ti.kbase + kc, ti.m0, &full[s]);
+#pragma unroll
+            for (int i = 0; i < BN / 128; ++i)
+              tma_load_2d(sb + i * 16384, &p.tmB, ti.kbase + kc, ti.n0 + 128 * i, &full[s]);
+          } else if constexpr (!A_MN) {
+            tma_load_2d(sa, &p.tmA, kc, ti.m0, &full[s]);
+          } else {
+            tma_load_2d(sa, &p.tmA, ti.m0, ti.kbase + kc, &full[s]);
+          }
+          if constexpr (!GROUP_K && !B_MN) {
             // boxes of BN/2 rows (SwiGLU: gate rows, then up rows) or of 128 rows
             if constexpr (EPI == EPI_SWIGLU_FWD) {
               tma_load_2d(sb, &p.tmB, kc, ti.kbase + ti.n0, &full[s]);
@@ -763,7 +778,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
               for (int i = 0; i < BN / 128; ++i)
                 tma_load_2d(sb + i * 16384, &p.tmB, kc, ti.kbase + ti.n0 + 128 * i, &full[s]);
             }
-          } else {
+          } else if constexpr (!GROUP_K) {
 #pragma unroll
             for (int i = 0; i < BN / 128; ++i)
               tma_load_2d(sb + i * 16384, &p.tmB, ti.n0 + 128 * i, ti.kbase + kc, &full[s]);
@@ -1906,14 +1921,16 @@ MxLayout mx_layout(const FfnShape& s) {
   // covers 128 rows x 128 K elements
   const size_t tiles = R / 128 + s.E;
   auto atoms = [&](size_t K) { return tiles * (K / 128) * 512; };
+  // token-block copies: [K][Rp], the token axis padded to whole 128-row stages per expert
+  const size_t Rp = tiles * 128;
   MxLayout L;
   size_t o = 0;
   auto take = [&](size_t bytes) { const size_t at = o; o += align256(bytes); return at; };
-  L.qx1 = take(R * d); L.sx1 = take(atoms(d));
-  L.qh1 = take(R * f); L.sh1 = take(atoms(f));
+  L.qx1 = take(Rp * d); L.sx1 = take(atoms(d));
+  L.qh1 = take(Rp * f); L.sh1 = take(atoms(f));
   L.rt = take(R * 4);
-  L.map = take((R / 32 + s.E) * 16);
-  L.cnt = take(4);
+  L.map = take((R / 32 + s.E) * 16 + (R / 128 + s.E + 1) * 4);  // block map, stage table
+  L.cnt = take(8);
   const size_t base = o;
   L.qx0 = take(R * d); L.sx0 = take(atoms(d)); L.qh0 = take(R * f); L.sh0 = take(atoms(f));
   L.fwd_bytes = o;
@@ -1921,8 +1938,8 @@ MxLayout mx_layout(const FfnShape& s) {
   L.dadu = take(R * 2 * f * 2);
   L.qdy0 = take(R * d); L.sdy0 = take(atoms(d));
   L.qda0 = take(R * 2 * f); L.sda0 = take(atoms(2 * f));
-  L.qdy1 = take(R * d); L.sdy1 = take(atoms(d));
-  L.qda1 = take(R * 2 * f); L.sda1 = take(atoms(2 * f));
+  L.qdy1 = take(Rp * d); L.sdy1 = take(atoms(d));
+  L.qda1 = take(Rp * 2 * f); L.sda1 = take(atoms(2 * f));
   L.part = take(wgrad_part_bytes(s, true));
   L.bwd_bytes = o;
   return L;
@@ -1976,13 +1993,14 @@ cudaError_t ffn_fwd_mx(const FfnShape& s, const void* x_perm, const int32_t* off
   const __nv_bfloat16* actb = static_cast<const __nv_bfloat16*>(act);
   int32_t* rt = reinterpret_cast<int32_t*>(ws + L.rt);
   int4* map = reinterpret_cast<int4*>(ws + L.map);
+  int32_t* smap = reinterpret_cast<int32_t*>(ws + L.map + (s.rows / 32 + s.E) * 16);
   int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
   // x along d (gate/up GEMM) and in token blocks (kept for the dW1 GEMM of the backward);
   // without x_perm, the fused dispatch has written both copies and the maps already
   if (x_perm) {
     if ((err = row_tile_launch(offsets, E, R, rt, st)) != cudaSuccess ||
-        (err = seg_blocks_launch(offsets, E, map, cnt, st)) != cudaSuccess ||
-        (err = mxfp8_act(R, E, d, d, x_perm, map, cnt, rt, ws + L.qx0, ws + L.sx0, ws + L.qx1,
+        (err = seg_blocks_launch(offsets, E, map, cnt, smap, st)) != cudaSuccess ||
+        (err = mxfp8_act(R, E, d, d, x_perm, map, cnt, smap, rt, ws + L.qx0, ws + L.sx0, ws + L.qx1,
                          ws + L.sx1, st)) != cudaSuccess)
       return err;
   }
@@ -2008,7 +2026,7 @@ cudaError_t ffn_fwd_mx(const FfnShape& s, const void* x_perm, const int32_t* off
   }
   if (err != cudaSuccess) return err;
   // h along f (down GEMM) and in token blocks (kept for the dW2 GEMM of the backward)
-  if ((err = mxfp8_act(R, E, f, 3 * f, actb + 2 * f, map, cnt, rt, ws + L.qh0, ws + L.sh0,
+  if ((err = mxfp8_act(R, E, f, 3 * f, actb + 2 * f, map, cnt, smap, rt, ws + L.qh0, ws + L.sh0,
                        ws + L.qh1, ws + L.sh1, st)) != cudaSuccess)
     return err;
   if (!y_perm) return cudaSuccess;  // recompute: a | u | h and the token-block copies only
@@ -2037,12 +2055,13 @@ cudaError_t mx_dispatch(const FfnShape& s, const void* x, const int32_t* perm_sr
   const MxLayout L = mx_layout(s);
   int32_t* rt = reinterpret_cast<int32_t*>(ws + L.rt);
   int4* map = reinterpret_cast<int4*>(ws + L.map);
+  int32_t* smap = reinterpret_cast<int32_t*>(ws + L.map + (s.rows / 32 + s.E) * 16);
   int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
   cudaError_t err;
   if ((err = row_tile_launch(offsets, s.E, s.rows, rt, st)) != cudaSuccess ||
-      (err = seg_blocks_launch(offsets, s.E, map, cnt, st)) != cudaSuccess)
+      (err = seg_blocks_launch(offsets, s.E, map, cnt, smap, st)) != cudaSuccess)
     return err;
-  return mxfp8_act(s.rows, s.E, s.d, s.d, x, map, cnt, rt, ws + L.qx0, ws + L.sx0, ws + L.qx1,
+  return mxfp8_act(s.rows, s.E, s.d, s.d, x, map, cnt, smap, rt, ws + L.qx0, ws + L.sx0, ws + L.qx1,
                    ws + L.sx1, st, perm_src);
 }
 
@@ -2054,20 +2073,20 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
   if (err != cudaSuccess) return err;
   const int d = s.d, f = s.f, E = s.E;
   const int64_t R = s.rows;
-  const uint64_t Rtm = std::max<int64_t>(R, 1);
   uint8_t* ws = static_cast<uint8_t*>(scratch);
   const MxLayout L = mx_layout(s);
   const __nv_bfloat16* actb = static_cast<const __nv_bfloat16*>(act);
   __nv_bfloat16* dadu = reinterpret_cast<__nv_bfloat16*>(ws + L.dadu);
   int32_t* rt = reinterpret_cast<int32_t*>(ws + L.rt);
   int4* map = reinterpret_cast<int4*>(ws + L.map);
+  int32_t* smap = reinterpret_cast<int32_t*>(ws + L.map + (s.rows / 32 + s.E) * 16);
   int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
   (void)x_perm;  // its token-block copy comes from the forward
   if (R > 0) {
     // (the row-tile and token-block maps of the forward are still in the workspace)
     // dgrad 1: dh = dy W2 (dy along d, W2 along its d rows), SwiGLU backward -> [da | du];
     // dy also in token blocks for the dW2 GEMM
-    if ((err = mxfp8_act(R, E, d, d, dy_perm, map, cnt, rt, ws + L.qdy0, ws + L.sdy0, ws + L.qdy1,
+    if ((err = mxfp8_act(R, E, d, d, dy_perm, map, cnt, smap, rt, ws + L.qdy0, ws + L.sdy0, ws + L.qdy1,
                          ws + L.sdy1, st)) != cudaSuccess)
       return err;
     GemmParams p3 = mx_params(s, offsets, status);
@@ -2093,7 +2112,7 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
     if (err != cudaSuccess) return err;
     // dgrad 2: dx = [da | du] W1 ([da | du] along 2f, W1 along its 2f rows); [da | du]
     // also in token blocks for the dW1 GEMM
-    if ((err = mxfp8_act(R, E, 2 * f, 2 * f, dadu, map, cnt, rt, ws + L.qda0, ws + L.sda0,
+    if ((err = mxfp8_act(R, E, 2 * f, 2 * f, dadu, map, cnt, smap, rt, ws + L.qda0, ws + L.sda0,
                          ws + L.qda1, ws + L.sda1, st)) != cudaSuccess)
       return err;
     GemmParams p4 = mx_params(s, offsets, status);
@@ -2115,10 +2134,12 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
     }
     if (err != cudaSuccess) return err;
   }
-  // wgrad 2: dW2[e] = dy^T h  (M = d, N = f)
+  // wgrad 2: dW2[e] = dy^T h  (M = d, N = f); both operands K-major over the padded
+  // token axis ([columns][Rp] token-block copies)
+  const uint64_t Rp = ((uint64_t)R / 128 + E) * 128;
   GemmParams p5 = mx_params(s, offsets, status);
-  if (!tmap(&p5.tmA, ws + L.qdy1, d, Rtm, d, 128, 128, false, true) ||
-      !tmap(&p5.tmB, ws + L.qh1, f, Rtm, f, 128, 128, false, true) ||
+  if (!tmap(&p5.tmA, ws + L.qdy1, Rp, d, Rp, 128, 128, false, true) ||
+      !tmap(&p5.tmB, ws + L.qh1, Rp, f, Rp, 128, 128, false, true) ||
       !tmap(&p5.tmOut, dw2, f, (uint64_t)E * d, f, 32, 16, true))
     return cudaErrorInvalidValue;
   p5.sfa = ws + L.sdy1;
@@ -2127,13 +2148,13 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
   p5.out_f32 = dw2; p5.ld_out = f; p5.out_group = (int64_t)d * f; p5.accumulate = accumulate;
   wgrad_setup(&p5, R, d, f, true, reinterpret_cast<float*>(ws + L.part));
   if (!p5.part) return cudaErrorInvalidValue;
-  if ((err = launch_mx_n<true, true, EPI_WGRAD, true>(p5, f, num_sms(), st)) != cudaSuccess ||
+  if ((err = launch_mx_n<false, false, EPI_WGRAD, true>(p5, f, num_sms(), st)) != cudaSuccess ||
       (err = wgrad_reduce_launch(p5, d, f, dw2, nullptr, st)) != cudaSuccess)
     return err;
   // wgrad 1: dW1[e] = [da | du]^T x  (M = 2f, N = d)
   GemmParams p6 = mx_params(s, offsets, status);
-  if (!tmap(&p6.tmA, ws + L.qda1, 2 * f, Rtm, 2 * f, 128, 128, false, true) ||
-      !tmap(&p6.tmB, ws + L.qx1, d, Rtm, d, 128, 128, false, true) ||
+  if (!tmap(&p6.tmA, ws + L.qda1, Rp, 2 * f, Rp, 128, 128, false, true) ||
+      !tmap(&p6.tmB, ws + L.qx1, Rp, d, Rp, 128, 128, false, true) ||
       !tmap(&p6.tmOut, dw1, d, (uint64_t)E * 2 * f, d, 32, 16, true))
     return cudaErrorInvalidValue;
   p6.sfa = ws + L.sda1;
@@ -2142,7 +2163,7 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
   p6.out_f32 = dw1; p6.ld_out = d; p6.out_group = (int64_t)2 * f * d; p6.accumulate = accumulate;
   wgrad_setup(&p6, R, 2 * f, d, true, reinterpret_cast<float*>(ws + L.part));
   if (!p6.part) return cudaErrorInvalidValue;
-  if ((err = launch_mx_n<true, true, EPI_WGRAD, true>(p6, d, num_sms(), st)) != cudaSuccess) return err;
+  if ((err = launch_mx_n<false, false, EPI_WGRAD, true>(p6, d, num_sms(), st)) != cudaSuccess) return err;
   return wgrad_reduce_launch(p6, 2 * f, d, dw1, nullptr, st);
 }
 

@@ -87,15 +87,16 @@ cudaError_t mxfp8_launch_ld(int64_t rows, int64_t K, int64_t ld, bool src_bf16, 
 cudaError_t row_tile_launch(const int32_t* offsets, int E, int64_t rows, int32_t* out, cudaStream_t st);
 cudaError_t mxfp8_weights(const float* w, int E, int Rw, int Kw, uint8_t* q0, uint8_t* s0,
                           uint8_t* q1, uint8_t* s1, cudaStream_t st);
-//   seg_blocks_launch: the 32-row token blocks of all segments (at most rows/32 + E)
+//   seg_blocks_launch: the 32-row token blocks of all segments (at most rows/32 + E) and
+//     the first block of every 128-row stage (smap, at most rows/128 + E + 1 entries)
 //   mxfp8_act: one pass over a bf16 activation writing its row copy (row-tile atoms) and its
 //     token-block copy (stage atoms); with `gather`, operand row r is source row gather[r]
 cudaError_t seg_blocks_launch(const int32_t* offsets, int E, int4* map, int32_t* count,
-                              cudaStream_t st);
+                              int32_t* smap, cudaStream_t st);
 cudaError_t mxfp8_act(int64_t rows, int E, int64_t K, int64_t ld, const void* src_bf16,
-                      const int4* map, const int32_t* count, const int32_t* row_tile, uint8_t* q_r,
-                      uint8_t* atoms_r, uint8_t* q_c, uint8_t* atoms_c, cudaStream_t st,
-                      const int32_t* gather = nullptr);
+                      const int4* map, const int32_t* count, const int32_t* smap,
+                      const int32_t* row_tile, uint8_t* q_r, uint8_t* atoms_r, uint8_t* q_c,
+                      uint8_t* atoms_c, cudaStream_t st, const int32_t* gather = nullptr);
 //   perm_src_launch: perm_src[slot_row[t, j]] = t (the permute's source map, no row copy)
 cudaError_t perm_src_launch(const int32_t* slot_row, int32_t* perm_src, int T, int k,
                             cudaStream_t st);

@@ -339,11 +339,12 @@ mx_weights_kernel(const float* __restrict__ w, int E, int Rw, int Kw, uint8_t* _
 // 32-row blocks of the token axis, restarting at every segment (expert): block b (in
 // segment order) -> {first row, rows (1..32), 128-row stage over all segments, (position of
 // the block in its stage) | 4 if it is its segment's last block}.  count[0] = number of
-// blocks.  One CTA of 1024 threads (E <= 1024): a scan of the per-segment block counts,
+// blocks, count[1] = number of stages, smap[z] = first block of stage z (smap[count[1]] =
+// count[0]).  One CTA of 1024 threads (E <= 1024): a scan of the per-segment block counts,
 // then each thread writes its segment's entries.
 __global__ void __launch_bounds__(1024)
 seg_blocks_kernel(const int32_t* __restrict__ offsets, int E, int4* __restrict__ map,
-                  int32_t* __restrict__ count) {
+                  int32_t* __restrict__ count, int32_t* __restrict__ smap) {
   const int g = threadIdx.x, lane = g & 31, w = g >> 5;
   const int r0 = g < E ? offsets[g] : 0, c = g < E ? offsets[g + 1] - r0 : 0;
   const int nb = (c + 31) / 32, ns = (c + 127) / 128;
@@ -373,27 +374,36 @@ seg_blocks_kernel(const int32_t* __restrict__ offsets, int E, int4* __restrict__
   for (int lb = 0; lb < nb; ++lb)
     map[b0 + lb] = make_int4(r0 + 32 * lb, min(32, c - 32 * lb), st0 + lb / 4,
                              (lb & 3) | (lb == nb - 1 ? 4 : 0));
-  if (g == 1023) count[0] = b0 + nb;
+  for (int s2 = 0; s2 < ns; ++s2) smap[st0 + s2] = b0 + 4 * s2;  // first block of each stage
+  if (g == 1023) {
+    count[0] = b0 + nb;
+    count[1] = st0 + ns;
+    smap[st0 + ns] = b0 + nb;
+  }
 }
 
 // One pass over a bf16 activation tile of one 32-row token block (of one segment) x 128
 // columns, writing both MXFP8 copies: q_r / atoms_r in blocks of 32 along each row (row-tile
 // atoms, tile and row from row_tile), and q_c / atoms_c in the block's 32 rows within each
-// column (stage atoms; the blocks of a segment's last stage past its end get 2^0).
+// column (stage atoms; the blocks of a segment's last stage past its end get 2^0).  q_c is
+// column-major over the stage-padded token axis: column c's code of the block's row i sits
+// at q_c[c * Rp + 128 * stage + 32 * (block in stage) + i]; the rows past a segment's last
+// token, up to the end of its last stage, get code 0.  A CTA takes whole stages (their
+// blocks one after another) and writes each column's 128 codes of a stage as one line.
 constexpr int kActPitch = 136;  // bf16 per staged row (16 bytes of padding)
-constexpr int kSqPitch = 144;   // bytes per staged row of the column copy (16 bytes of padding)
+constexpr int kQtPitch = 132;   // bytes per staged column of a stage's column copy
 __global__ void __launch_bounds__(128, 8)
 mx_act_kernel(const __nv_bfloat16* __restrict__ src, int64_t K, int64_t ld,
               const int4* __restrict__ map, const int32_t* __restrict__ count,
-              const int32_t* __restrict__ row_tile, uint8_t* __restrict__ q_r,
-              uint8_t* __restrict__ atoms_r, uint8_t* __restrict__ q_c,
-              uint8_t* __restrict__ atoms_c, const int32_t* __restrict__ gather) {
+              const int32_t* __restrict__ smap, const int32_t* __restrict__ row_tile,
+              uint8_t* __restrict__ q_r, uint8_t* __restrict__ atoms_r, uint8_t* __restrict__ q_c,
+              uint8_t* __restrict__ atoms_c, const int32_t* __restrict__ gather, int64_t Rp) {
   __shared__ __align__(16) __nv_bfloat16 s_t[32 * kActPitch];
-  __shared__ __align__(16) uint8_t s_q[32 * kSqPitch];
+  __shared__ __align__(16) uint8_t s_q[128 * kQtPitch];
   const int tid = threadIdx.x, ct = blockIdx.x;
   const int64_t c0 = (int64_t)ct * 128;
   const int64_t kq = K >> 7;
-  const int nblocks = count[0];
+  const int nstages = count[1];
   // n rows x 128 columns of block b: 16 pieces of 16 bytes per row, 4 per thread.  The next
   // block's pieces are loaded into registers while this block is quantised.
   auto load = [&](int b, int4& m, uint4 (&v)[4]) {
@@ -409,19 +419,29 @@ mx_act_kernel(const __nv_bfloat16* __restrict__ src, int64_t K, int64_t ld,
       }
     }
   };
+  // this CTA's blocks: stages blockIdx.y, + gridDim.y, ..., each stage's blocks in order
+  int z = blockIdx.y;
+  int b = z < nstages ? smap[z] : 0;
   int4 mnext;
   uint4 vnext[4];
-  if (blockIdx.y < nblocks) load(blockIdx.y, mnext, vnext);
-  for (int b = blockIdx.y; b < nblocks; b += gridDim.y) {
+  if (z < nstages) load(b, mnext, vnext);
+  while (z < nstages) {
     const int4 m = mnext;
     const int r0 = m.x, n = m.y;
+    const int pos = m.w & 3;
+    const bool stage_end = b + 1 == smap[z + 1];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int i = tid + 128 * j, row = i >> 4, p8 = i & 15;
       *reinterpret_cast<uint4*>(s_t + row * kActPitch + p8 * 8) = vnext[j];
     }
     __syncthreads();
-    if (b + (int)gridDim.y < nblocks) load(b + gridDim.y, mnext, vnext);
+    int zn = z, bn = b + 1;
+    if (stage_end) {
+      zn = z + gridDim.y;
+      bn = zn < nstages ? smap[zn] : 0;
+    }
+    if (zn < nstages) load(bn, mnext, vnext);
     // rows: thread = (row, 32-column block)
     {
       const int row = tid >> 2, kb = tid & 3;
@@ -456,7 +476,7 @@ mx_act_kernel(const __nv_bfloat16* __restrict__ src, int64_t K, int64_t ld,
     // a pair are neighbouring lanes.  The rows a lane pair reads in one step are 4 apart
     // (rows 0-3, 8-11, .. for one half, 4-7, 12-15, .. for the other), which puts the two
     // halves 16 banks apart.  Rows past n are zero in s_t, so they do not change the
-    // maximum, and their codes are never written out.
+    // maximum and their codes are 0.
     {
       const int cp = tid >> 1, rh = tid & 1;
       uint32_t w[16];
@@ -472,32 +492,50 @@ mx_act_kernel(const __nv_bfloat16* __restrict__ src, int64_t K, int64_t ld,
       am = __hmax2(am, *reinterpret_cast<const __nv_bfloat162*>(&oth));
       const int ex0 = block_exponent(__low2float(am)), ex1 = block_exponent(__high2float(am));
       const float m0 = pow2_neg(ex0), m1 = pow2_neg(ex1);
+      // rows 8 g + 4 rh .. + 3 of the two columns, four codes per 32-bit store into the
+      // stage's column-major staging (132-byte pitch: no bank conflicts)
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int r = (i & 3) + ((i >> 2) << 3) + 4 * rh;
-        const float lo = __uint_as_float(w[i] << 16) * m0;          // column 2 cp
-        const float hi = __uint_as_float(w[i] & 0xFFFF0000u) * m1;  // column 2 cp + 1
-        *reinterpret_cast<uint16_t*>(s_q + r * kSqPitch + 2 * cp) = (uint16_t)e4m3_pair(hi, lo);
+      for (int g = 0; g < 4; ++g) {
+        uint32_t wl = 0, wh = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t v = w[4 * g + i];
+          const uint32_t pr = e4m3_pair(__uint_as_float(v & 0xFFFF0000u) * m1,
+                                        __uint_as_float(v << 16) * m0);
+          wl |= (pr & 0xFFu) << (8 * i);
+          wh |= (pr >> 8) << (8 * i);
+        }
+        *reinterpret_cast<uint32_t*>(s_q + (2 * cp) * kQtPitch + 32 * pos + 8 * g + 4 * rh) = wl;
+        *reinterpret_cast<uint32_t*>(s_q + (2 * cp + 1) * kQtPitch + 32 * pos + 8 * g + 4 * rh) = wh;
       }
       // each of the pair's two threads writes the scale byte of one of its columns
       const int col = 2 * cp + rh;
       const int ex = rh ? ex1 : ex0;
       uint8_t* at = atoms_c + ((int64_t)m.z * kq + ct) * 512;
-      const int pos = m.w & 3;
       at[atom_byte(col, pos)] = (uint8_t)(ex + 127);
       if (m.w & 4)
         for (int kb = pos + 1; kb < 4; ++kb) at[atom_byte(col, kb)] = 0x7F;
     }
-    __syncthreads();
-    // the column copy's rows, 16 bytes per store
+    if (stage_end) {
+      // the stage's column copy: each column's 128 codes as one 128-byte line, eight
+      // lanes per line (16 bytes each), so that one warp store writes four whole lines;
+      // the blocks the stage does not have (past its segment's end) are zero.  The
+      // lanes of one load touch 32 distinct banks (pitch 33 words).
+      __syncthreads();
+      const int p16 = tid & 7;
+      const bool have = p16 < 2 * (pos + 1);  // 32 bytes per block present
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int i = tid + 128 * j, row = i >> 3, p16 = i & 7;
-      if (row < n)
-        *reinterpret_cast<uint4*>(q_c + (int64_t)(r0 + row) * K + c0 + p16 * 16) =
-            *reinterpret_cast<const uint4*>(s_q + row * kSqPitch + p16 * 16);
+      for (int j = 0; j < 8; ++j) {
+        const int col = 16 * j + (tid >> 3);
+        const uint32_t* sc = reinterpret_cast<const uint32_t*>(s_q + col * kQtPitch + 16 * p16);
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (have) v = make_uint4(sc[0], sc[1], sc[2], sc[3]);
+        *reinterpret_cast<uint4*>(q_c + (c0 + col) * Rp + 128 * (int64_t)m.z + 16 * p16) = v;
+      }
     }
     __syncthreads();
+    z = zn;
+    b = bn;
   }
 }
 
@@ -514,26 +552,28 @@ cudaError_t row_tile_launch(const int32_t* offsets, int E, int64_t rows, int32_t
 }
 
 cudaError_t seg_blocks_launch(const int32_t* offsets, int E, int4* map, int32_t* count,
-                              cudaStream_t st) {
+                              int32_t* smap, cudaStream_t st) {
   {
     ProfScope prof("mx_seg_blocks", st);
-    seg_blocks_kernel<<<1, 1024, 0, st>>>(offsets, E, map, count);
+    seg_blocks_kernel<<<1, 1024, 0, st>>>(offsets, E, map, count, smap);
   }
   return cudaGetLastError();
 }
 
 cudaError_t mxfp8_act(int64_t rows, int E, int64_t K, int64_t ld, const void* src_bf16,
-                      const int4* map, const int32_t* count, const int32_t* row_tile, uint8_t* q_r,
-                      uint8_t* atoms_r, uint8_t* q_c, uint8_t* atoms_c, cudaStream_t st,
-                      const int32_t* gather) {
+                      const int4* map, const int32_t* count, const int32_t* smap,
+                      const int32_t* row_tile, uint8_t* q_r, uint8_t* atoms_r, uint8_t* q_c,
+                      uint8_t* atoms_c, cudaStream_t st, const int32_t* gather) {
   if (rows == 0) return cudaSuccess;
-  // about 8 blocks of 128 threads per SM at a time, each looping over several token blocks
+  const int64_t Rp = (rows / 128 + E) * 128;  // padded token axis of the column copy
+  // about 8 blocks of 128 threads per SM at a time, each looping over several stages
   const int64_t want = std::max<int64_t>(1, (int64_t)num_sms() * 8 / (K / 128));
-  dim3 grid((unsigned)(K / 128), (unsigned)std::min<int64_t>({rows / 32 + E, want, 65535}));
+  dim3 grid((unsigned)(K / 128), (unsigned)std::min<int64_t>({rows / 128 + E, want, 65535}));
   {
     ProfScope prof("mx_act", st);
     mx_act_kernel<<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(src_bf16), K, ld, map,
-                                         count, row_tile, q_r, atoms_r, q_c, atoms_c, gather);
+                                         count, smap, row_tile, q_r, atoms_r, q_c, atoms_c, gather,
+                                         Rp);
   }
   return cudaGetLastError();
 }

@@ -8,7 +8,8 @@ of 32 along each row) feeds the row-grouped GEMMs, the token-block copy (blocks 
 rows within each column, restarting at every expert) the weight-gradient GEMMs.  Here
 the codes and scales the layer left in its workspace (located with
 moe_mx_workspace_layout) are decoded and compared byte for byte with the oracle's
-mxfp8_quantize on the same bf16 values (the layer stores its activations in bf16, so
+mxfp8_quantize on the same bf16 values (the token-block copy is column-major over a token
+axis padded to whole 128-row stages per expert; its pad codes must be zero) (the layer stores its activations in bf16, so
 both sides take their codes on those values), including the 2^0 scales that pad an
 expert's last stage and the maps that place every block.
 """
@@ -65,9 +66,34 @@ class _Ws:
     def maps(self):
         R = self.L.rows
         rt = self._bytes("row_tile", 0, 4 * R).view(torch.int32).cpu().numpy().astype(np.int64)
-        nb = int(self._bytes("nblocks", 0, 4).view(torch.int32).item())
+        nb, ns = self._bytes("nblocks", 0, 8).view(torch.int32).tolist()
         bl = self._bytes("blocks", 0, 16 * nb).view(torch.int32).view(nb, 4).cpu().numpy()
-        return rt, bl.astype(np.int64)
+        # the stage table after the block map: first block of every stage, then nb
+        sm = self._bytes("blocks", 16 * (R // 32 + self.L.E), 4 * (ns + 1))
+        sm = sm.view(torch.int32).cpu().numpy().astype(np.int64)
+        bl = bl.astype(np.int64)
+        assert sm[-1] == nb and np.all(np.diff(sm) >= 1) and np.all(np.diff(sm) <= 4)
+        assert np.array_equal(bl[sm[:-1], 2], np.arange(ns)), "stage table"
+        assert np.all(bl[sm[:-1], 3] & 3 == 0), "a stage starts at its first block"
+        return rt, bl
+
+    def blk_codes(self, name, K, blocks, r0, r1):
+        """Token-block codes of operand rows r0..r1 as [r1 - r0, K], read from the copy's
+        column-major layout over the stage-padded token axis ([K][Rp]), and the padded
+        positions of those rows' stages that hold no row (they must be zero)."""
+        Rp = (self.L.rows // 128 + self.L.E) * 128
+        qT = self._bytes(name, 0, K * Rp).view(K, Rp)
+        sel = blocks[(blocks[:, 0] >= r0) & (blocks[:, 0] < r1)]
+        pos = np.zeros(r1 - r0, dtype=np.int64)
+        for rb, n, z, w in sel:
+            pos[rb - r0:rb - r0 + n] = 128 * z + 32 * (w & 3) + np.arange(n)
+        codes = qT[:, torch.from_numpy(pos).cuda()].t().cpu().numpy() if r1 > r0 else \
+            np.zeros((0, K), dtype=np.uint8)
+        stages = np.unique(sel[:, 2]) if len(sel) else np.zeros(0, dtype=np.int64)
+        allpos = (128 * stages[:, None] + np.arange(128)[None, :]).ravel()
+        pads = np.setdiff1d(allpos, pos)
+        padv = qT[:, torch.from_numpy(pads).cuda()].cpu().numpy() if len(pads) else np.zeros(0)
+        return codes, padv
 
     def dadu(self, r0, r1):
         f2 = 2 * self.L.f
@@ -78,10 +104,11 @@ class _Ws:
 def _check(ws, name, values, K, offsets, e0, e1, q_row, s_row, q_blk, s_blk):
     r0, r1 = int(offsets[e0]), int(offsets[e1])
     rt, bl = ws.maps()
+    blk, pads = ws.blk_codes(q_blk, K, bl, r0, r1)
     try:
         check_mx_operand(values, K, offsets, e0, e1, ws.codes(q_row, r0, r1, K),
-                         ws.atoms(s_row, K), ws.codes(q_blk, r0, r1, K), ws.atoms(s_blk, K),
-                         rt, bl)
+                         ws.atoms(s_row, K), blk, ws.atoms(s_blk, K), rt, bl)
+        assert not np.any(pads), "token-block pad codes"
     except AssertionError as err:
         raise AssertionError(f"{name}: {err}") from None
 
