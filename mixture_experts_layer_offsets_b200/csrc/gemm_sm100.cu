@@ -455,7 +455,7 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, cons
                                                 const int* s_stg = nullptr) {
   TileInfo ti;
   if constexpr (GROUP_K) {
-    const int per = (p.M / BM) * nN;
+    const int per = (p.M / TM) * nN;
     int g, local;
     if (p.kchunk) {  // tile prefix over groups (ranges x per)
       int lo = 0, hi = p.E - 1;
@@ -471,9 +471,9 @@ __device__ __forceinline__ TileInfo decode_tile(int t, const GemmParams& p, cons
     }
     const int j = local / per, rem = local - j * per;
     ti.g = g;
-    ti.m0 = (rem / nN) * BM;
+    ti.m0 = (rem / nN) * TM;
     ti.n0 = (rem % nN) * BN;
-    ti.rows = BM;
+    ti.rows = TM;
     const int k0 = s_off[g], kg = s_off[g + 1] - k0;
     int ns, ck;
     wgrad_split(kg, p.kchunk, ns, ck);
@@ -519,8 +519,8 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
   constexpr bool kHalfIdle = EPI == EPI_ROUTER;
   constexpr int S = C::kStages;
   static_assert(EPI != EPI_SWIGLU_FWD || BN == 256, "SwiGLU forward pairs 128 gate with 128 up columns");
-  static_assert(!PAIR || (BN == 256 && !A_MN && !GROUP_K && EPI != EPI_ROUTER),
-                "CTA pairs serve the row-grouped GEMMs with N = 256");
+  static_assert(!PAIR || (BN == 256 && !A_MN && EPI != EPI_ROUTER && (!GROUP_K || FP8)),
+                "CTA pairs serve the row-grouped GEMMs with N = 256 and the MXFP8 weight gradients");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -611,7 +611,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
     // per-group prefixes, 32 groups per lane of warp 1 (E <= 1024): tiles (split groups),
     // partial slots (groups cut into several K ranges) and MXFP8 128-row stages
     if (warp == 1 && (p.kchunk || FP8)) {
-      const int per = (p.M / BM) * nN;
+      const int per = (p.M / C::kTileM) * nN;
       const int lo = lane * 32, hi = min(lo + 32, E);
       int st = 0, sl = 0, sg = 0;
       for (int g = lo; g < hi; ++g) {
@@ -648,7 +648,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
-  const int total = GROUP_K ? (p.kchunk ? s_pre[E] : E * (p.M / BM) * nN) : s_pre[E];
+  const int total = GROUP_K ? (p.kchunk ? s_pre[E] : E * (p.M / C::kTileM) * nN) : s_pre[E];
 
   auto fail = [&]() {
     record_status(p.status, MOE_ERR_TIMEOUT);
@@ -714,7 +714,7 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
         // CTA pairs: atom indices (the atom tensors' row is twice the index).  A: this CTA's
         // 128-row tile of its expert; B: both 128-column halves of the tile.
         int64_t pa0 = 0, pb0 = 0, pb1 = 0;
-        if constexpr (PAIR) {
+        if constexpr (PAIR && !GROUP_K) {
           pa0 = ((int64_t)s_sel[ti.g] + (ti.m0 - s_off[ti.g]) / BM) * kq;
           if constexpr (!B_MN) {
             const int ntiles = p.b_rows / 128;
@@ -739,6 +739,20 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
             // every load of both CTAs completes on the leader's barrier; only the leader arrives
             if (leader) mbar_arrive_expect_tx(&full[s], 2 * (kABytes + C::kBBytes + C::kSfLoad));
             const uint32_t bar = leader_full + 8 * s;
+            if constexpr (GROUP_K) {
+              // weight gradients (256 x 256 tiles): this CTA's 128 A rows and 128 of the
+              // 256 B rows, K-major over the stage-padded token axis; the A atom of its
+              // rows and both B atoms of the stage
+              const int64_t zk = (int64_t)s_stg[ti.g] + ti.kst + kb;
+              const int64_t ia = zk * (p.M / BM) + ti.m0 / BM;
+              const int64_t ib = zk * (p.N / 128) + ti.n0 / 128;
+              tma_load_2d_pair(sa, &p.tmA, ti.kbase + kc, ti.m0, bar);
+              tma_load_2d_pair(sb, &p.tmB, ti.kbase + kc, ti.n0 + 128 * (int)rank, bar);
+              tma_load_2d_pair(sf, &p.tmSfa, 0, (int)(2 * ia), bar);
+              tma_load_2d_pair(sf + 512, &p.tmSfb, 0, (int)(2 * ib), bar);
+              tma_load_2d_pair(sf + 1024, &p.tmSfb, 0, (int)(2 * ib + 2), bar);
+              continue;
+            }
             tma_load_2d_pair(sa, &p.tmA, kc, ti.m0, bar);
             if constexpr (!B_MN) {
               const int row = ti.kbase + (EPI == EPI_SWIGLU_FWD ? (rank == 0 ? ti.n0 : p.f + ti.n0)
@@ -1614,9 +1628,9 @@ cudaError_t launch_mx(const GemmParams& p, int64_t tile_bound, cudaStream_t st) 
 }
 
 // CTA-pair variant: clusters of 2 CTAs, as many as can be resident at once.
-template <int BN, bool B_MN, int EPI, bool FP8 = false>
+template <int BN, bool B_MN, int EPI, bool FP8 = false, bool GROUP_K = false>
 cudaError_t launch_pair(const GemmParams& p, int64_t pair_tile_bound, cudaStream_t st) {
-  auto kern = grouped_gemm_sm100<BN, false, B_MN, EPI, false, true, FP8>;
+  auto kern = grouped_gemm_sm100<BN, false, B_MN, EPI, GROUP_K, true, FP8>;
   constexpr size_t smem = Cfg<BN, true, EPI, FP8>::kSmem;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
@@ -1668,6 +1682,13 @@ int wgrad_kchunk(int64_t rows, int M, int N, int BN) {
 // partial slots: a group of c > kc rows takes ceil(c / kc) <= 2 c / kc of them
 int64_t wgrad_slots(int64_t rows, int kc) { return 2 * rows / kc + 1; }
 int wgrad_bn(int N, bool fp8) { return (!fp8 || N % 256 == 0) ? 256 : 128; }
+// MXFP8 weight gradients on CTA pairs (256 x 256 tiles) when M and N are multiples of 256;
+// MOE_B200_PAIR=0 turns pairs off here too (read per call: tests switch it)
+bool wgrad_pairs(int M, int N) {
+  const char* env = getenv("MOE_B200_PAIR");
+  if (env && env[0] == '0') return false;
+  return M % 256 == 0 && N % 256 == 0;
+}
 
 // Sets the split fields of a weight-gradient launch (M x N per group) and returns the
 // partial-buffer bytes it may use; `part` may be null when only the size is wanted.
@@ -2135,8 +2156,20 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
     if (err != cudaSuccess) return err;
   }
   // wgrad 2: dW2[e] = dy^T h  (M = d, N = f); both operands K-major over the padded
-  // token axis ([columns][Rp] token-block copies)
+  // token axis ([columns][Rp] token-block copies).  256 x 256 tiles on CTA pairs where
+  // M and N allow: each CTA reads half of the B rows, so a tile's operand bytes per MMA
+  // fall by a third and the smaller stages leave room for a deeper ring.
   const uint64_t Rp = ((uint64_t)R / 128 + E) * 128;
+  const uint64_t stages = (uint64_t)R / 128 + E;  // atoms per 128 columns of a token-block copy
+  auto wgrad_mx = [&](GemmParams& pw, const uint8_t* sfa, const uint8_t* sfb, int M, int N) {
+    if (wgrad_pairs(M, N)) {
+      if (!tmap_atoms(&pw.tmSfa, sfa, stages * (M / 128)) ||
+          !tmap_atoms(&pw.tmSfb, sfb, stages * (N / 128)))
+        return cudaErrorInvalidValue;
+      return launch_pair<256, false, EPI_WGRAD, true, true>(pw, num_sms() / 2, st);
+    }
+    return launch_mx_n<false, false, EPI_WGRAD, true>(pw, N, num_sms(), st);
+  };
   GemmParams p5 = mx_params(s, offsets, status);
   if (!tmap(&p5.tmA, ws + L.qdy1, Rp, d, Rp, 128, 128, false, true) ||
       !tmap(&p5.tmB, ws + L.qh1, Rp, f, Rp, 128, 128, false, true) ||
@@ -2148,7 +2181,7 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
   p5.out_f32 = dw2; p5.ld_out = f; p5.out_group = (int64_t)d * f; p5.accumulate = accumulate;
   wgrad_setup(&p5, R, d, f, true, reinterpret_cast<float*>(ws + L.part));
   if (!p5.part) return cudaErrorInvalidValue;
-  if ((err = launch_mx_n<false, false, EPI_WGRAD, true>(p5, f, num_sms(), st)) != cudaSuccess ||
+  if ((err = wgrad_mx(p5, ws + L.sdy1, ws + L.sh1, d, f)) != cudaSuccess ||
       (err = wgrad_reduce_launch(p5, d, f, dw2, nullptr, st)) != cudaSuccess)
     return err;
   // wgrad 1: dW1[e] = [da | du]^T x  (M = 2f, N = d)
@@ -2163,7 +2196,7 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
   p6.out_f32 = dw1; p6.ld_out = d; p6.out_group = (int64_t)2 * f * d; p6.accumulate = accumulate;
   wgrad_setup(&p6, R, 2 * f, d, true, reinterpret_cast<float*>(ws + L.part));
   if (!p6.part) return cudaErrorInvalidValue;
-  if ((err = launch_mx_n<false, false, EPI_WGRAD, true>(p6, d, num_sms(), st)) != cudaSuccess) return err;
+  if ((err = wgrad_mx(p6, ws + L.sda1, ws + L.sx1, 2 * f, d)) != cudaSuccess) return err;
   return wgrad_reduce_launch(p6, 2 * f, d, dw1, nullptr, st);
 }
 

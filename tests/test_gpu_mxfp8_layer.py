@@ -35,6 +35,10 @@ CASES = {
                             d_ff=128, router_std=1 / 16.0, bias_std=3.0),
     # d and f multiples of 256, ~512 rows per expert: the row-grouped GEMMs run on CTA pairs
     "mx_pairs": shrink(BASE, name="mx_pairs", T=2048, d_model=512, E=8, top_k=2, d_ff=256),
+    # skewed, d and f multiples of 256: weight gradients on CTA pairs (256 x 256 tiles)
+    # with their K cut into ranges and partial sums added
+    "mx_skew_split_pairs": shrink(BASE, name="mx_skew_split_pairs", T=6000, d_model=256, E=16,
+                                  top_k=2, d_ff=256, router_std=1 / 16.0, bias_std=3.0),
     # one token
     "mx_one_token": shrink(BASE, name="mx_one_token", T=1, d_model=128, E=4, top_k=2, d_ff=128),
 }
@@ -157,16 +161,16 @@ def test_fused_dispatch_is_bit_identical_to_permute_then_quantise(name):
         assert torch.equal(a, b), key
 
 
-@pytest.mark.parametrize("name", ["mx_e8", "mx_skew_split"])
+@pytest.mark.parametrize("name", ["mx_e8", "mx_skew_split", "mx_skew_split_pairs"])
 def test_mxfp8_accumulated_weight_grads_are_the_sum_of_two_steps(name):
     check_accumulate(CASES[name])
 
 
 
-@pytest.mark.parametrize("name", ["mx_pairs", "mx_skew_split"])
+@pytest.mark.parametrize("name", ["mx_pairs", "mx_skew_split", "mx_skew_split_pairs"])
 def test_mxfp8_cta_pairs_give_the_bits_of_single_ctas(name, monkeypatch):
-    # the same dot products in the same K order: 256-row tiles on CTA pairs must reproduce
-    # the 128-row single-CTA results exactly
+    # the same dot products in the same K order: 256-row tiles on CTA pairs (row-grouped
+    # GEMMs and weight gradients) must reproduce the single-CTA results exactly
     cfg = CASES[name]
     monkeypatch.setenv("MOE_B200_PAIR", "0")
     _, A = run_layer(cfg)
