@@ -28,6 +28,8 @@ CASES = {
     "e16": dict(T=64, d_model=2048, E=16, top_k=4),
     "e32_k8": dict(T=2049, d_model=512, E=32, top_k=8, router_std=512 ** -0.5),
     "one_token": dict(T=1, d_model=128, E=8, top_k=2),
+    # more 16-token groups than 8 per SM: CTAs loop over several token tiles
+    "e8_many_tiles": dict(T=20000, d_model=256, E=8, top_k=2),
 }
 
 
@@ -103,3 +105,4 @@ def test_tile_router_on_the_same_shapes(monkeypatch):
     b, _, names = _route(cfg, dev)
     assert names[0] == "router_gemm", names
     _check(cfg, cpu, b)
+
