@@ -183,9 +183,11 @@ def gemm_flop(cfg) -> float:
     return 18.0 * cfg.R * cfg.d_model * cfg.d_ff
 
 
-def kernel_bytes(cfg, capacity=None) -> dict:
+def kernel_bytes(cfg, capacity=None, recompute=False) -> dict:
     """Algorithmic HBM bytes per step of the row-moving and quantising kernels (each
-    operand read once, each result written once), by launch name."""
+    operand read once, each result written once), by launch name.  The MXFP8 layer
+    (without recompute) runs the combine backward fused with dy's quantisation: that
+    launch writes no dy_perm rows, and the quantiser reads dout's rows instead."""
     T, d, E, k, f = cfg.T, cfg.d_model, cfg.E, cfg.top_k, cfg.d_ff
     R = E * capacity if capacity else cfg.R
     s = 4 if cfg.dtype == "f32" else 2
@@ -195,7 +197,8 @@ def kernel_bytes(cfg, capacity=None) -> dict:
         "router_mma": router,    # warp-level router (up to 32 experts)
         "permute": T * d * s + R * d * s + T * k * 8,
         "combine": R * d * s + T * d * s + T * k * 8,
-        "combine_bwd": T * d * s + 2 * R * d * s + T * k * 12,
+        "combine_bwd": T * d * s + (1 if cfg.dtype == "mxfp8" and not recompute else 2) * R * d * s
+        + T * k * 12,
     }
     if cfg.dtype == "mxfp8":
         mx = 2 * (1 + 1 / 32)  # two E4M3 copies with their E8M0 scales, per element
@@ -251,7 +254,12 @@ class LayerStep:
         mark(4)
         capi.moe_combine(s, dt, L.y_perm, L.row_map, L.topk_gate, L.out)
         mark(5)
-        capi.moe_combine_bwd(s, dt, dout, L.y_perm, L.row_map, L.topk_gate, L.dy_perm, L.dgate)
+        if L.fused_dispatch:
+            capi.moe_combine_bwd_mx(s, dout, L.y_perm, L.row_map, L.topk_gate, L.perm_src,
+                                    L.dgate, L.ws)
+        else:
+            capi.moe_combine_bwd(s, dt, dout, L.y_perm, L.row_map, L.topk_gate, L.dy_perm,
+                                 L.dgate)
         mark(6)
         bwd = capi.moe_grouped_ffn_bwd_recompute if self.recompute else capi.moe_grouped_ffn_bwd
         bwd(s, fdt, L.rows, L.dy_perm, L.x_perm, L.act, L.ffn_offsets, w1, w2, L.dx_perm, L.dw1,
@@ -413,11 +421,11 @@ def roofline(cfg, res, capacity=None):
     return out
 
 
-def hbm_kernels(cfg, res, capacity=None):
+def hbm_kernels(cfg, res, capacity=None, recompute=False):
     """Achieved bandwidth of the memory-bound kernels from their algorithmic bytes."""
     pk, pk_kind = _peaks()
     out = {}
-    for name, nbytes in kernel_bytes(cfg, capacity).items():
+    for name, nbytes in kernel_bytes(cfg, capacity, recompute).items():
         k = res["kernels"].get(name)
         if not k or k["ms_per_step"] <= 0:
             continue
@@ -453,7 +461,7 @@ def run_ours(args, rank, world):
     line.update({
         "config": _workload_desc(cfg, capacity, args.recompute, accum, world),
         "roofline": roofline(cfg, res, capacity),
-        "hbm_kernels": hbm_kernels(cfg, res, capacity),
+        "hbm_kernels": hbm_kernels(cfg, res, capacity, args.recompute),
         "phases_ms": {k: round(v, 4) for k, v in res["phases_ms"].items()},
         "kernels_ms": res["kernels"],
         "timing": "value: CUDA-graph replay of the step, CUDA events per step, max over ranks; "

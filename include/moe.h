@@ -333,6 +333,26 @@ moe_status moe_combine_bwd(moe_shape shape, int dtype, const void* dout, const v
                            const int32_t* slot_row, const float* topk_gate, void* dy_perm,
                            float* dgate, void* stream);
 
+/* ---- f1 (backward): MXFP8 combine backward --------------------------------
+ * [kongchang] boundary-conditions section: MXFP8 cuts the bytes the rows move.  In the
+ * MXFP8 layer the rows dy_perm[slot_row[t,j]] = topk_gate[t,j] * dout[t,:] are read only
+ * as their two MXFP8 copies (along d for the dh GEMM, in 32-row token blocks for the dW2
+ * GEMM).  This call writes dgate exactly as moe_combine_bwd does (fp32 [T, k]) and those
+ * two copies into `ws`, each operand row r taken from dout[perm_src[r],:] times its gate,
+ * rounded to bf16 first as moe_combine_bwd rounds dy_perm, without writing dy_perm; then
+ * moe_grouped_ffn_bwd (MOE_MXFP8, dy_perm = NULL) reads them.  The result is bit-identical
+ * to moe_combine_bwd followed by that backward's own quantisation of dy_perm.
+ * dout, y_perm: bf16 [T, d] / [T*k, d]; slot_row, perm_src: from the dropless route and
+ * dispatch (perm_src[r] = the token of row r); topk_gate: the gates the combine used.
+ * `ws` must be the workspace of this step's MXFP8 forward (moe_grouped_ffn_fwd, which
+ * leaves the row and block maps there), sized for rows = T*top_k, with no call using it
+ * in between.  Not with moe_grouped_ffn_bwd_recompute, whose forward half reuses that
+ * memory.  d % 128 == 0 and f % 128 == 0 (else MOE_ERR_UNSUPPORTED). */
+moe_status moe_combine_bwd_mx(moe_shape shape, const void* dout, const void* y_perm,
+                              const int32_t* slot_row, const float* topk_gate,
+                              const int32_t* perm_src, float* dgate, void* ws, size_t ws_bytes,
+                              void* stream);
+
 /* ---- a7 + a8: grouped SwiGLU FFN, backward -------------------------------
  * Per expert e on its rows: dh = dy W2[e]; s = sigmoid(a);
  *   da = dh*u*s*(1 + a*(1-s)); du = dh*silu(a);
@@ -350,7 +370,8 @@ moe_status moe_combine_bwd(moe_shape shape, int dtype, const void* dout, const v
  * token-block copies of x and h (and the row/block maps) are the ones the forward of the
  * same step wrote into `ws`: pass the same workspace, with no call using it in between
  * (moe_combine and moe_combine_bwd take none), and the same offsets.  x_perm is not
- * read and may be NULL. */
+ * read and may be NULL.  dy_perm may be NULL when moe_combine_bwd_mx has just written
+ * dy's copies into `ws` (its quantisation is then skipped). */
 moe_status moe_grouped_ffn_bwd(moe_shape shape, int dtype, int64_t rows, const void* dy_perm,
                                const void* x_perm, const void* act_saved,
                                const int32_t* offsets, const void* w1, const void* w2,
@@ -368,7 +389,7 @@ moe_status moe_grouped_ffn_bwd(moe_shape shape, int dtype, int64_t rows, const v
  * workspace may have served other calls since the forward), then runs the
  * backward.  One act_scratch can serve every layer of a model.  act_scratch
  * is overwritten; its contents afterwards are this layer's a | u | h.  x_perm
- * is required here, for every dtype. */
+ * and dy_perm are required here, for every dtype. */
 moe_status moe_grouped_ffn_bwd_recompute(moe_shape shape, int dtype, int64_t rows,
                                          const void* dy_perm, const void* x_perm,
                                          void* act_scratch, const int32_t* offsets,

@@ -73,6 +73,7 @@ _SIGS = {
     "moe_padded_dispatch": (_I, [moe_shape, _I, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_routing_stats": (_I, [moe_shape, _P, ctypes.c_int32, _P, _P]),
     "moe_permute_mx": (_I, [moe_shape, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_combine_bwd_mx": (_I, [moe_shape, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_renorm_gates": (_I, [moe_shape, _P, _P, _P]),
     "moe_renorm_gates_bwd": (_I, [moe_shape, _P, _P, _P, _P]),
 }
@@ -225,6 +226,13 @@ def moe_combine_bwd(shape, dtype, dout, y_perm, slot_row, topk_gate, dy_perm, dg
     _check("moe_combine_bwd", lib().moe_combine_bwd(
         shape, dtype, _ptr(dout), _ptr(y_perm), _ptr(slot_row), _ptr(topk_gate), _ptr(dy_perm),
         _ptr(dgate), _stream(stream)))
+
+
+def moe_combine_bwd_mx(shape, dout, y_perm, slot_row, topk_gate, perm_src, dgate, ws,
+                       stream=None) -> None:
+    _check("moe_combine_bwd_mx", lib().moe_combine_bwd_mx(
+        shape, _ptr(dout), _ptr(y_perm), _ptr(slot_row), _ptr(topk_gate), _ptr(perm_src),
+        _ptr(dgate), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def moe_grouped_ffn_bwd(shape, dtype, rows, dy_perm, x_perm, act_saved, offsets, w1, w2,

@@ -259,6 +259,23 @@ moe_status moe_combine_bwd(moe_shape s, int dtype, const void* dout, const void*
                                         as_stream(stream)));
 }
 
+moe_status moe_combine_bwd_mx(moe_shape s, const void* dout, const void* y_perm,
+                              const int32_t* slot_row, const float* topk_gate,
+                              const int32_t* perm_src, float* dgate, void* ws, size_t ws_bytes,
+                              void* stream) {
+  moe_status st = shape_ok(s);
+  if (st != MOE_OK) return st;
+  if (s.d_model % 128 || s.d_ff % 128) return MOE_ERR_UNSUPPORTED;
+  if (!ptrs_ok(ws)) return MOE_ERR_INVALID_ARG;
+  if (s.T > 0 && !ptrs_ok(dout, y_perm, slot_row, topk_gate, perm_src, dgate))
+    return MOE_ERR_INVALID_ARG;
+  FfnShape fs{s.d_model, s.E, s.d_ff, (int64_t)s.T * s.top_k};
+  if (ws_bytes < kStatusBytes + ffn_mx_ws_bytes(fs)) return MOE_ERR_INVALID_ARG;
+  if (s.T == 0) return MOE_OK;
+  return cuda_status(mx_combine_bwd(fs, dout, y_perm, slot_row, topk_gate, perm_src, dgate, s.T,
+                                    s.top_k, scratch(ws), as_stream(stream)));
+}
+
 }  // extern "C"
 
 namespace {
@@ -282,9 +299,12 @@ moe_status ffn_bwd_entry(moe_shape s, int dtype, int64_t rows, const void* dy_pe
     if (s.d_model % 128 || s.d_ff % 128) return MOE_ERR_UNSUPPORTED;
     if (dw_dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
     if (!ptrs_ok(offsets, dw1, dw2, ws)) return MOE_ERR_INVALID_ARG;
-    // x_perm is read only by the recompute (the backward uses the token-block copy)
-    if (rows > 0 && (!ptrs_ok(dy_perm, act_saved, dx_perm) || (recompute && !x_perm) ||
-                     (x_perm && !aligned16(x_perm))))
+    // x_perm is read only by the recompute (the backward uses the token-block copy);
+    // dy_perm NULL: moe_combine_bwd_mx has put dy's copies in ws (not with the recompute,
+    // whose forward half reuses that memory)
+    if (rows > 0 && (!ptrs_ok(act_saved, dx_perm) || (recompute && !x_perm) ||
+                     (x_perm && !aligned16(x_perm)) || (recompute && !dy_perm) ||
+                     (dy_perm && !aligned16(dy_perm))))
       return MOE_ERR_INVALID_ARG;
     FfnShape fsm{s.d_model, s.E, s.d_ff, rows};
     if (ws_bytes < kStatusBytes + ffn_mx_ws_bytes(fsm)) return MOE_ERR_INVALID_ARG;

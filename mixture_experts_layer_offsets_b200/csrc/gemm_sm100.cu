@@ -2086,6 +2086,25 @@ cudaError_t mx_dispatch(const FfnShape& s, const void* x, const int32_t* perm_sr
                    ws + L.sx1, st, perm_src);
 }
 
+cudaError_t mx_combine_bwd(const FfnShape& s, const void* dout, const void* y_perm,
+                           const int32_t* slot_row, const float* gate, const int32_t* perm_src,
+                           float* dgate, int T, int k, void* scratch, cudaStream_t st) {
+  cudaError_t err = combine_bwd_launch(true, dout, y_perm, slot_row, gate, nullptr, dgate, T, s.d,
+                                       k, st);
+  if (err != cudaSuccess || s.rows == 0) return err;
+  uint8_t* ws = static_cast<uint8_t*>(scratch);
+  const MxLayout L = mx_layout(s);
+  int32_t* rt = reinterpret_cast<int32_t*>(ws + L.rt);
+  int4* map = reinterpret_cast<int4*>(ws + L.map);
+  int32_t* smap = reinterpret_cast<int32_t*>(ws + L.map + (s.rows / 32 + s.E) * 16);
+  int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
+  // each routed row's gate, in the permuted order, where [da | du] goes later
+  float* gate_perm = reinterpret_cast<float*>(ws + L.dadu);
+  if ((err = perm_gate_launch(slot_row, gate, gate_perm, T, k, st)) != cudaSuccess) return err;
+  return mxfp8_act(s.rows, s.E, s.d, s.d, dout, map, cnt, smap, rt, ws + L.qdy0, ws + L.sdy0,
+                   ws + L.qdy1, ws + L.sdy1, st, perm_src, gate_perm);
+}
+
 cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_perm, const void* act,
                        const int32_t* offsets, const MxWeights& w, void* dx_perm, float* dw1,
                        float* dw2, void* scratch, int* status, cudaStream_t st,
@@ -2107,7 +2126,9 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
     // (the row-tile and token-block maps of the forward are still in the workspace)
     // dgrad 1: dh = dy W2 (dy along d, W2 along its d rows), SwiGLU backward -> [da | du];
     // dy also in token blocks for the dW2 GEMM
-    if ((err = mxfp8_act(R, E, d, d, dy_perm, map, cnt, smap, rt, ws + L.qdy0, ws + L.sdy0, ws + L.qdy1,
+    // (without dy_perm, the fused combine backward has written both copies already)
+    if (dy_perm &&
+        (err = mxfp8_act(R, E, d, d, dy_perm, map, cnt, smap, rt, ws + L.qdy0, ws + L.sdy0, ws + L.qdy1,
                          ws + L.sdy1, st)) != cudaSuccess)
       return err;
     GemmParams p3 = mx_params(s, offsets, status);

@@ -90,14 +90,19 @@ cudaError_t mxfp8_weights(const float* w, int E, int Rw, int Kw, uint8_t* q0, ui
 //   seg_blocks_launch: the 32-row token blocks of all segments (at most rows/32 + E) and
 //     the first block of every 128-row stage (smap, at most rows/128 + E + 1 entries)
 //   mxfp8_act: one pass over a bf16 activation writing its row copy (row-tile atoms) and its
-//     token-block copy (stage atoms); with `gather`, operand row r is source row gather[r]
+//     token-block copy (stage atoms); with `gather`, operand row r is source row gather[r];
+//     with `row_mul`, row r is first scaled by row_mul[r] and rounded to bf16
 cudaError_t seg_blocks_launch(const int32_t* offsets, int E, int4* map, int32_t* count,
                               int32_t* smap, cudaStream_t st);
 cudaError_t mxfp8_act(int64_t rows, int E, int64_t K, int64_t ld, const void* src_bf16,
                       const int4* map, const int32_t* count, const int32_t* smap,
                       const int32_t* row_tile, uint8_t* q_r, uint8_t* atoms_r, uint8_t* q_c,
-                      uint8_t* atoms_c, cudaStream_t st, const int32_t* gather = nullptr);
+                      uint8_t* atoms_c, cudaStream_t st, const int32_t* gather = nullptr,
+                      const float* row_mul = nullptr);
 //   perm_src_launch: perm_src[slot_row[t, j]] = t (the permute's source map, no row copy)
+//   perm_gate_launch: gate_perm[slot_row[t, j]] = gate[t, j]
+cudaError_t perm_gate_launch(const int32_t* slot_row, const float* gate, float* gate_perm, int T,
+                             int k, cudaStream_t st);
 cudaError_t perm_src_launch(const int32_t* slot_row, int32_t* perm_src, int T, int k,
                             cudaStream_t st);
 
@@ -131,6 +136,12 @@ struct FfnShape {
 //     through perm_src, into the workspace regions that ffn_fwd_mx reads
 cudaError_t mx_dispatch(const FfnShape& s, const void* x, const int32_t* perm_src,
                         const int32_t* offsets, void* scratch, cudaStream_t st);
+//   mx_combine_bwd: dgate as the combine backward computes it, and the two MXFP8 copies of
+//     dy_perm (gate x dout rows, rounded to bf16) into the workspace regions that ffn_bwd_mx
+//     reads when given no dy_perm; the block maps come from the forward
+cudaError_t mx_combine_bwd(const FfnShape& s, const void* dout, const void* y_perm,
+                           const int32_t* slot_row, const float* gate, const int32_t* perm_src,
+                           float* dgate, int T, int k, void* scratch, cudaStream_t st);
 size_t ffn_bwd_ws_bytes(const FfnShape& s, bool bf16);
 // fp32 partial sums of weight-gradient groups cut into K ranges (tensor-core paths)
 size_t wgrad_part_bytes(const FfnShape& s, bool fp8);

@@ -397,7 +397,8 @@ mx_act_kernel(const __nv_bfloat16* __restrict__ src, int64_t K, int64_t ld,
               const int4* __restrict__ map, const int32_t* __restrict__ count,
               const int32_t* __restrict__ smap, const int32_t* __restrict__ row_tile,
               uint8_t* __restrict__ q_r, uint8_t* __restrict__ atoms_r, uint8_t* __restrict__ q_c,
-              uint8_t* __restrict__ atoms_c, const int32_t* __restrict__ gather, int64_t Rp) {
+              uint8_t* __restrict__ atoms_c, const int32_t* __restrict__ gather, int64_t Rp,
+              const float* __restrict__ row_mul) {
   __shared__ __align__(16) __nv_bfloat16 s_t[32 * kActPitch];
   __shared__ __align__(16) uint8_t s_q[128 * kQtPitch];
   const int tid = threadIdx.x, ct = blockIdx.x;
@@ -413,9 +414,19 @@ mx_act_kernel(const __nv_bfloat16* __restrict__ src, int64_t K, int64_t ld,
       const int i = tid + 128 * j, row = i >> 4, p8 = i & 15;
       v[j] = make_uint4(0, 0, 0, 0);
       if (row < m.y) {
-        // row r of the operand is source row gather[r] (the fused dispatch), else r
+        // row r of the operand is source row gather[r] (the fused dispatch), else r; with
+        // row_mul, the bf16 of row_mul[r] times the source values (the fused combine
+        // backward: gate times output gradient, rounded as the combine backward rounds)
         const int64_t sr = gather ? (int64_t)__ldg(gather + m.x + row) : (int64_t)(m.x + row);
         v[j] = ldg16(src + sr * ld + c0 + p8 * 8);
+        if (row_mul) {
+          const float g = __ldg(row_mul + m.x + row);
+          Vec16<__nv_bfloat16> a, o;
+          a.raw = v[j];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o.set(e, g * a.get(e));
+          v[j] = o.raw;
+        }
       }
     }
   };
@@ -563,7 +574,8 @@ cudaError_t seg_blocks_launch(const int32_t* offsets, int E, int4* map, int32_t*
 cudaError_t mxfp8_act(int64_t rows, int E, int64_t K, int64_t ld, const void* src_bf16,
                       const int4* map, const int32_t* count, const int32_t* smap,
                       const int32_t* row_tile, uint8_t* q_r, uint8_t* atoms_r, uint8_t* q_c,
-                      uint8_t* atoms_c, cudaStream_t st, const int32_t* gather) {
+                      uint8_t* atoms_c, cudaStream_t st, const int32_t* gather,
+                      const float* row_mul) {
   if (rows == 0) return cudaSuccess;
   const int64_t Rp = (rows / 128 + E) * 128;  // padded token axis of the column copy
   // about 8 blocks of 128 threads per SM at a time, each looping over several stages
@@ -573,7 +585,7 @@ cudaError_t mxfp8_act(int64_t rows, int E, int64_t K, int64_t ld, const void* sr
     ProfScope prof("mx_act", st);
     mx_act_kernel<<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(src_bf16), K, ld, map,
                                          count, smap, row_tile, q_r, atoms_r, q_c, atoms_c, gather,
-                                         Rp);
+                                         Rp, row_mul);
   }
   return cudaGetLastError();
 }

@@ -134,7 +134,7 @@ combine_bwd_kernel(const T* __restrict__ dout, const T* __restrict__ y_perm,
         const float gt = __shfl_sync(0xffffffffu, mygate, j);
         if (r < 0) continue;
         const T* ysrc = y_perm + (int64_t)r * d;
-        T* dst = dy_perm + (int64_t)r * d;
+        T* dst = dy_perm ? dy_perm + (int64_t)r * d : nullptr;
 #pragma unroll
         for (int b = 0; b < kBatch; ++b) {
           const int c = c0 + b * 32 + lane;
@@ -147,7 +147,7 @@ combine_bwd_kernel(const T* __restrict__ dout, const T* __restrict__ y_perm,
               dot[j] = fmaf(g[b].get(i), yv.get(i), dot[j]);
               o.set(i, gt * g[b].get(i));
             }
-            stg16(dst + c * V, o.raw);
+            if (dy_perm) stg16(dst + c * V, o.raw);  // null: dgate only
           }
         }
       }
@@ -213,6 +213,14 @@ padded_dispatch_kernel(const T* __restrict__ x, const int32_t* __restrict__ topk
 }  // namespace
 
 namespace {
+// gate_perm[slot_row[i]] = gate[i]: each routed row's gate, in the permuted row order
+__global__ void __launch_bounds__(256) perm_gate_kernel(const int32_t* __restrict__ slot_row,
+                                                        const float* __restrict__ gate,
+                                                        float* __restrict__ gate_perm, int64_t n) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) gate_perm[slot_row[i]] = gate[i];
+}
+
 __global__ void __launch_bounds__(256) perm_src_kernel(const int32_t* __restrict__ slot_row,
                                                        int32_t* __restrict__ perm_src, int64_t n,
                                                        int k) {
@@ -228,6 +236,17 @@ cudaError_t perm_src_launch(const int32_t* slot_row, int32_t* perm_src, int T, i
   {
     ProfScope prof("perm_src", st);
     perm_src_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(slot_row, perm_src, n, k);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t perm_gate_launch(const int32_t* slot_row, const float* gate, float* gate_perm, int T,
+                             int k, cudaStream_t st) {
+  const int64_t n = (int64_t)T * k;
+  if (n == 0) return cudaSuccess;
+  {
+    ProfScope prof("perm_gate", st);
+    perm_gate_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(slot_row, gate, gate_perm, n);
   }
   return cudaGetLastError();
 }

@@ -12,7 +12,10 @@ dtype "mxfp8": bf16 activations and router, FP32 master expert weights whose
 MXFP8 copies (two orientations per weight, see ``moe_mx_weights``) are made
 by moe_mx_quantize_weights at the start of every forward, i.e. once per optimizer step
 when every step is one; the grouped FFN calls run with MOE_MXFP8 and write
-FP32 weight gradients.
+FP32 weight gradients.  Unless it recomputes, the MXFP8 layer dispatches with
+moe_permute_mx and runs the combine backward as moe_combine_bwd_mx: both write the
+MXFP8 operand copies of x and dy straight into the workspace, and no bf16 x_perm or
+dy_perm exists (those attributes are None).
 """
 
 from __future__ import annotations
@@ -53,6 +56,8 @@ class MoELayer:
         if fused_dispatch and (dtype != "mxfp8" or recompute):
             raise ValueError("the fused dispatch is the MXFP8 layer's, without recompute")
         self.fused_dispatch = fused_dispatch
+        # with it, the combine backward writes dy's MXFP8 copies directly
+        # (moe_combine_bwd_mx) and no bf16 dy_perm
         self.shape = capi.shape_of(T, d_model, E, top_k, d_ff)
         self.R = T * top_k
         self.rows = E * capacity if capacity else self.R
@@ -83,7 +88,7 @@ class MoELayer:
         self.y_perm = torch.empty(rows, d_model, **act)
         self.out = torch.empty(T, d_model, **act)
         self.dgate = torch.empty(T, top_k, **f32)
-        self.dy_perm = torch.zeros(rows, d_model, **act)
+        self.dy_perm = None if fused_dispatch else torch.zeros(rows, d_model, **act)
         self.dx_perm = torch.empty(rows, d_model, **act)
         self.dw1 = torch.empty(E, 2 * d_ff, d_model, dtype=wdt, device=dev)
         self.dw2 = torch.empty(E, d_model, d_ff, dtype=wdt, device=dev)
@@ -166,8 +171,13 @@ class MoELayer:
         (gradient accumulation over micro-batches) instead of overwriting them."""
         s, dt = self.shape, self.cdtype
         acc = capi.MOE_DW_ACCUMULATE if accumulate else 0
-        capi.moe_combine_bwd(s, dt, dout, self.y_perm, self.row_map, self.combine_gate,
-                             self.dy_perm, self.dgate_rn if self.renorm else self.dgate, stream)
+        dg = self.dgate_rn if self.renorm else self.dgate
+        if self.fused_dispatch:
+            capi.moe_combine_bwd_mx(s, dout, self.y_perm, self.row_map, self.combine_gate,
+                                    self.perm_src, dg, self.ws, stream)
+        else:
+            capi.moe_combine_bwd(s, dt, dout, self.y_perm, self.row_map, self.combine_gate,
+                                 self.dy_perm, dg, stream)
         if self.renorm:
             capi.moe_renorm_gates_bwd(s, self.topk_gate, self.dgate_rn, self.dgate, stream)
         bwd = capi.moe_grouped_ffn_bwd_recompute if self.recompute else capi.moe_grouped_ffn_bwd

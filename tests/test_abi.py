@@ -173,6 +173,32 @@ def test_mxfp8_ffn_validation(lib):
     assert bwd(ws_bytes=1024) == capi.MOE_ERR_INVALID_ARG
 
 
+def test_mxfp8_combine_bwd_validation(lib):
+    """moe_combine_bwd_mx (dgate plus dy's MXFP8 copies into the workspace) and the
+    backward's dy_perm = NULL form, which the recompute backward refuses."""
+    s = _shape()
+    big = capi.moe_workspace_size(s, capi.MOE_MXFP8, 0)
+
+    def cb(shape=s, dout=FAKE, perm_src=FAKE, ws=FAKE, ws_bytes=big):
+        return lib.moe_combine_bwd_mx(shape, dout, FAKE, FAKE, FAKE, perm_src, FAKE, ws, ws_bytes,
+                                      None)
+
+    assert cb(shape=_shape(d_model=192)) == capi.MOE_ERR_UNSUPPORTED      # d % 128
+    assert cb(dout=None) == capi.MOE_ERR_INVALID_ARG
+    assert cb(perm_src=None) == capi.MOE_ERR_INVALID_ARG
+    assert cb(perm_src=FAKE + 4) == capi.MOE_ERR_INVALID_ARG               # misaligned
+    assert cb(ws=None) == capi.MOE_ERR_INVALID_ARG
+    assert cb(ws_bytes=big // 2) == capi.MOE_ERR_INVALID_ARG
+    assert cb(shape=_shape(top_k=9)) == capi.MOE_ERR_INVALID_ARG
+    mx = _mxw()
+    rows = s.T * s.top_k
+    wsb = capi.moe_workspace_size(s, capi.MOE_MXFP8, rows)
+    rc = lib.moe_grouped_ffn_bwd_recompute(s, capi.MOE_MXFP8, rows, None, FAKE, FAKE, FAKE, None,
+                                           None, ctypes.addressof(mx), FAKE, FAKE, FAKE,
+                                           capi.MOE_F32, FAKE, wsb, None)
+    assert rc == capi.MOE_ERR_INVALID_ARG   # the recompute needs dy_perm
+
+
 def test_mx_quantize_weights_validation(lib):
     g = lib.moe_mx_quantize_weights
     mx = _mxw()

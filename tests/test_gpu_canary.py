@@ -48,8 +48,10 @@ CASES = {
 }
 
 
-@pytest.mark.parametrize("name", list(CASES))
-def test_no_write_outside_outputs(name):
+@pytest.mark.parametrize("name,fused", [("bf16", False), ("mxfp8", False), ("mxfp8", True)])
+def test_no_write_outside_outputs(name, fused):
+    """fused: the MXFP8 layer's own path (moe_permute_mx and moe_combine_bwd_mx write the
+    quantised copies of x and dy into the workspace; no x_perm, no dy_perm)."""
     cfg = CASES[name]
     T, d, E, k, f = cfg.T, cfg.d_model, cfg.E, cfg.top_k, cfg.d_ff
     R = T * k
@@ -81,14 +83,23 @@ def test_no_write_outside_outputs(name):
     w2 = inp["w2"] if mx is None else None
     capi.moe_route(shape, capi.MOE_BF16, x, wr, b, o["logits"], o["idx"], o["gate"], o["counts"],
                    o["offsets"], o["slot"], ws)
-    capi.moe_permute(shape, capi.MOE_BF16, x, o["slot"], o["x_perm"], o["perm_src"])
-    capi.moe_grouped_ffn_fwd(shape, fdt, R, o["x_perm"], o["offsets"], w1, w2, o["act"], o["y"],
-                             ws, mx=mx)
+    if fused:
+        capi.moe_permute_mx(shape, x, o["slot"], o["offsets"], o["perm_src"], ws)
+    else:
+        capi.moe_permute(shape, capi.MOE_BF16, x, o["slot"], o["x_perm"], o["perm_src"])
+    xp = None if fused else o["x_perm"]
+    capi.moe_grouped_ffn_fwd(shape, fdt, R, xp, o["offsets"], w1, w2, o["act"], o["y"], ws,
+                             mx=mx)
     capi.moe_combine(shape, capi.MOE_BF16, o["y"], o["slot"], o["gate"], o["out"])
-    capi.moe_combine_bwd(shape, capi.MOE_BF16, inp["dout"], o["y"], o["slot"], o["gate"], o["dy"],
-                         o["dgate"])
-    capi.moe_grouped_ffn_bwd(shape, fdt, R, o["dy"], o["x_perm"], o["act"], o["offsets"], w1, w2,
-                             o["dx_perm"], o["dw1"], o["dw2"], capi.MOE_F32, ws, mx=mx)
+    if fused:
+        capi.moe_combine_bwd_mx(shape, inp["dout"], o["y"], o["slot"], o["gate"], o["perm_src"],
+                                o["dgate"], ws)
+    else:
+        capi.moe_combine_bwd(shape, capi.MOE_BF16, inp["dout"], o["y"], o["slot"], o["gate"],
+                             o["dy"], o["dgate"])
+    capi.moe_grouped_ffn_bwd(shape, fdt, R, None if fused else o["dy"], xp, o["act"],
+                             o["offsets"], w1, w2, o["dx_perm"], o["dw1"], o["dw2"], capi.MOE_F32,
+                             ws, mx=mx)
     capi.moe_route_bwd(shape, capi.MOE_BF16, x, wr, o["logits"], o["idx"], o["dgate"],
                        o["dx_perm"], o["slot"], o["dx"], o["dwr"], ws)
     torch.cuda.synchronize()

@@ -137,7 +137,16 @@ def run_and_check_bytes(cfg, fused, expert=None):
     L.backward(dev["dout"], dev["x"], dev["w_router"], dev["w1"], dev["w2"])
     torch.cuda.synchronize()
     assert L.device_status() == 0
-    _check(ws, "dy", f64(L.dy_perm[r0:r1]), d, offsets, e0, e1, "qdy0", "sdy0", "qdy1", "sdy1")
+    if L.dy_perm is not None:
+        dy_rows = f64(L.dy_perm[r0:r1])
+    else:
+        # the fused combine backward quantises gate x dout rows, rounded to bf16 first, as
+        # the combine backward rounds dy_perm
+        gp = torch.zeros(max(L.R, 1), dtype=torch.float32, device="cuda")
+        gp[L.slot_row.reshape(-1).long()] = L.topk_gate.reshape(-1)
+        dy = dev["dout"][src].float() * gp[r0:r1, None]
+        dy_rows = f64(dy.to(torch.bfloat16))
+    _check(ws, "dy", dy_rows, d, offsets, e0, e1, "qdy0", "sdy0", "qdy1", "sdy1")
     _check(ws, "[da|du]", ws.dadu(r0, r1), 2 * f, offsets, e0, e1, "qda0", "sda0", "qda1",
            "sda1")
     return L, offsets
