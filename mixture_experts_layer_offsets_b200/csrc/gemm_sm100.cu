@@ -40,6 +40,7 @@
 // MOE_ERR_TIMEOUT, raises a CTA-wide abort flag, waits (bounded) for its own
 // TMA loads and MMAs in flight, frees TMEM and returns.
 #include "common.cuh"
+#include "mx_common.cuh"
 #include "internal.h"
 
 #include <cudaTypedefs.h>
@@ -114,6 +115,15 @@ struct GemmParams {
   int drop_it;
   // EPI_ROUTER_DX
   const int32_t* slot_row; // [rows_total][topk]
+  // EPI_SWIGLU_BWD (MXFP8): [da | du] leaves as its two MXFP8 operand copies instead of
+  // bf16 (mx_q_r non-null): the row copy [rows][2f] with row-tile atoms, and the
+  // token-block copy [2f][mx_rp] (column-major, stage-padded) with stage atoms; `out`,
+  // when also set, receives the bf16 rows as well (a diagnostic form)
+  uint8_t* mx_q_r;
+  uint8_t* mx_s_r;
+  uint8_t* mx_q_c;
+  uint8_t* mx_s_c;
+  int64_t mx_rp;
   // MXFP8 operands: E8M0 scales as 512-byte MMA atoms (128 rows x 4 blocks of 32
   // along K), in the order the producer reads them (see the MXFP8 producer).
   const uint8_t* sfa;
@@ -429,6 +439,76 @@ __device__ __forceinline__ void put_box_bf16(uint8_t* wbuf, uint32_t& slot, cons
   __syncwarp();
   if (lane == 0) tma_store_2d(tm, x, y, buf);
   ++slot;
+}
+
+// MXFP8 copies of one 32 x 32 block of an activation that a warp holds: lane = row of a
+// 32-token block (rows past the segment's end held as zero), pk = the row's 32 bf16 values
+// of this block's columns.  Writes the row copy (32 codes + one scale per valid row) and
+// the token-block copy (per column, the 32 codes down the block's rows as one 32-byte run
+// of the column-major copy, + one scale), exactly as the activation quantiser does.  A
+// block with no row in the segment (`live` false; its stage still exists) gets zero codes
+// and 2^0 scales.  s_tr: 32 x 17 words of this warp's shared memory.
+//   q_r_row:  row copy at this row and the block's first column (unused if !row_valid)
+//   at_r:     this row's scale byte in its row-tile atom (unused if !row_valid)
+//   q_c_blk:  token-block copy at the block's first column and first row
+//   at_c:     the stage atom of the block's 128-column slab; c0: the block's first column
+//             within that slab (0, 32, 64, 96); tb: the token block within the stage
+__device__ __forceinline__ void mx_emit_block(const uint32_t* pk, bool row_valid, bool live,
+                                              uint8_t* q_r_row, uint8_t* at_r, uint8_t* q_c_blk,
+                                              int64_t rp, uint8_t* at_c, int c0, int tb,
+                                              uint32_t* s_tr) {
+  const int lane = threadIdx.x & 31;
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    v[2 * i] = row_valid ? bf_lo(pk[i]) : 0.f;
+    v[2 * i + 1] = row_valid ? bf_hi(pk[i]) : 0.f;
+  }
+  if (row_valid) {
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    const int ex = block_exponent(amax);
+    const float mul = pow2_neg(ex);
+    uint32_t w8[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      w8[i] = e4m3_pair(v[4 * i + 1] * mul, v[4 * i] * mul) |
+              (e4m3_pair(v[4 * i + 3] * mul, v[4 * i + 2] * mul) << 16);
+    *reinterpret_cast<uint4*>(q_r_row) = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+    *reinterpret_cast<uint4*>(q_r_row + 16) = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+    *at_r = (uint8_t)(ex + 127);
+  }
+  // columns: the block passes through shared memory (row `lane` at a pitch of 17 words,
+  // so neither the writes nor the column reads conflict), and lane c takes column c: its
+  // 32 values down the rows give its scale and its 32 codes, which are the column's run
+  // of the token-block copy as they stand
+  __syncwarp();
+#pragma unroll
+  for (int w = 0; w < 16; ++w) s_tr[lane * 17 + w] = row_valid ? pk[w] : 0u;
+  __syncwarp();
+  float cv[32];
+#pragma unroll
+  for (int r = 0; r < 32; ++r) {
+    const uint32_t x = s_tr[r * 17 + (lane >> 1)];
+    cv[r] = (lane & 1) ? bf_hi(x) : bf_lo(x);
+  }
+  float cmax = 0.f;
+#pragma unroll
+  for (int r = 0; r < 32; ++r) cmax = fmaxf(cmax, fabsf(cv[r]));
+  const int cex = block_exponent(cmax);
+  const float cmul = pow2_neg(cex);
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    o[i] = live ? (e4m3_pair(cv[4 * i + 1] * cmul, cv[4 * i] * cmul) |
+                   (e4m3_pair(cv[4 * i + 3] * cmul, cv[4 * i + 2] * cmul) << 16))
+                : 0u;
+  uint8_t* dst = q_c_blk + (int64_t)lane * rp;
+  *reinterpret_cast<uint4*>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+  *reinterpret_cast<uint4*>(dst + 16) = make_uint4(o[4], o[5], o[6], o[7]);
+  at_c[atom_byte(c0 + lane, tb)] = live ? (uint8_t)(cex + 127) : (uint8_t)0x7F;
+  __syncwarp();  // s_tr is read before the next block writes it
 }
 
 // ------------------------------------------------------------ tile decode
@@ -1186,6 +1266,44 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
             }
           }
           const int col = ti.n0 + (c0 + 2 * pc) * 32;
+          if constexpr (FP8) {
+            if (p.mx_q_r) {
+              // [da | du] as its MXFP8 operand copies: this warp's 32 rows are one 32-token
+              // block (tiles and stages both start at every expert), and its tile is a stage
+              if (ti.rows > 0) {
+                const int stage = (PAIR ? s_sel[ti.g] : s_pre[ti.g] / nN) + (ti.m0 - s_off[ti.g]) / BM;
+                const int kq = 2 * p.f / 128;
+                uint32_t* s_tr = reinterpret_cast<uint32_t*>(wbuf);
+                const int64_t grow = ti.m0 + row;
+#pragma unroll
+                for (int ci = 0; ci < 2; ++ci) {
+#pragma unroll
+                  for (int du_part = 0; du_part < 2; ++du_part) {
+                    const int gc = (du_part ? p.f : 0) + col + 32 * ci;  // column of [da | du]
+                    const uint32_t* pk = (du_part ? pdu : pda) + 16 * ci;
+                    mx_emit_block(pk, valid, q * 32 < ti.rows, p.mx_q_r + grow * (2 * p.f) + gc,
+                                  p.mx_s_r + ((int64_t)stage * kq + gc / 128) * 512 +
+                                      atom_byte(row, (gc & 127) >> 5),
+                                  p.mx_q_c + (int64_t)gc * p.mx_rp + 128 * (int64_t)stage + 32 * q,
+                                  p.mx_rp, p.mx_s_c + ((int64_t)stage * kq + gc / 128) * 512,
+                                  gc & 96, q, s_tr);
+                  }
+                }
+              }
+              if (p.out && valid) {
+                uint32_t lo[16], hi[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) { lo[i] = pda[i]; hi[i] = pda[16 + i]; }
+                store_64B(drow + col, lo);
+                store_64B(drow + col + 32, hi);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) { lo[i] = pdu[i]; hi[i] = pdu[16 + i]; }
+                store_64B(drow + p.f + col, lo);
+                store_64B(drow + p.f + col + 32, hi);
+              }
+              continue;
+            }
+          }
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             const int vr = box_valid(q * 32 + 16 * hh);
@@ -2141,6 +2259,19 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
     p3.N = f; p3.K = d; p3.b_rows = d;
     p3.out = dadu; p3.ld_out = 2 * f;
     p3.act = actb; p3.ld_act = 3 * f;
+    // [da | du] leaves the SwiGLU-backward epilogue as its two MXFP8 copies (no bf16 round
+    // trip); MOE_B200_DADU=0 writes bf16 [da | du] and quantises it in a pass of its own,
+    // =keep writes both (read per call: tests compare the forms)
+    const char* dadu_env = getenv("MOE_B200_DADU");
+    const bool dadu_mx = !(dadu_env && dadu_env[0] == '0');
+    if (dadu_mx) {
+      p3.mx_q_r = ws + L.qda0;
+      p3.mx_s_r = ws + L.sda0;
+      p3.mx_q_c = ws + L.qda1;
+      p3.mx_s_c = ws + L.sda1;
+      p3.mx_rp = ((int64_t)R / 128 + E) * 128;
+      if (!(dadu_env && dadu_env[0] == 'k')) p3.out = nullptr;
+    }
     const bool pairs = use_pairs(s);
     const uint64_t tiles = (uint64_t)R / 128 + E;
     if (pairs && f % 256 == 0) {
@@ -2154,7 +2285,8 @@ cudaError_t ffn_bwd_mx(const FfnShape& s, const void* dy_perm, const void* x_per
     if (err != cudaSuccess) return err;
     // dgrad 2: dx = [da | du] W1 ([da | du] along 2f, W1 along its 2f rows); [da | du]
     // also in token blocks for the dW1 GEMM
-    if ((err = mxfp8_act(R, E, 2 * f, 2 * f, dadu, map, cnt, smap, rt, ws + L.qda0, ws + L.sda0,
+    if (!dadu_mx &&
+        (err = mxfp8_act(R, E, 2 * f, 2 * f, dadu, map, cnt, smap, rt, ws + L.qda0, ws + L.sda0,
                          ws + L.qda1, ws + L.sda1, st)) != cudaSuccess)
       return err;
     GemmParams p4 = mx_params(s, offsets, status);

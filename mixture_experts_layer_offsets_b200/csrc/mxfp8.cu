@@ -15,36 +15,11 @@
 // signed zeros included).
 #include "common.cuh"
 #include "internal.h"
+#include "mx_common.cuh"
 
 namespace moe {
 
 namespace {
-
-__device__ __forceinline__ int block_exponent(float amax) {
-  const uint32_t bits = __float_as_uint(amax);
-  const int ex = (int)((bits >> 23) & 0xFF);
-  int fl;
-  if (ex == 0) {
-    const uint32_t man = bits & 0x7FFFFF;
-    if (man == 0) return -127;
-    fl = -149 + (31 - __clz(man));
-  } else {
-    fl = ex - 127;
-  }
-  return min(max(fl - 8, -127), 127);
-}
-
-// 2^-e as an fp32 (e <= 119 for any finite fp32 amax, so 2^-e is normal).
-__device__ __forceinline__ float pow2_neg(int e) { return __uint_as_float((uint32_t)(127 - e) << 23); }
-
-// Two E4M3 codes (hi in the upper byte): the hardware conversion rounds to nearest even,
-// saturates at +-448 and keeps the sign, a negative value that rounds to zero included
-// (code 0x80).
-__device__ __forceinline__ uint32_t e4m3_pair(float hi, float lo) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-  return r;
-}
 
 // axis 0: a quad of lanes covers one 32-element block, 8 elements per lane.
 template <typename T>
@@ -167,16 +142,6 @@ __device__ __forceinline__ void load8(const T* p, float* v) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) { v[i] = a.get(i); v[4 + i] = b.get(i); }
   }
-}
-
-// ---------------------------------------------------------------- scale atoms
-// The block-scaled MMA takes its E8M0 scales from TMEM, which each pipeline stage fills
-// from a 512-byte shared-memory atom: 128 rows (of M or N) x 4 blocks of 32 along K, the
-// scale of row r and block kb at byte (r % 32) * 16 + (r / 32) * 4 + kb.  Inside the FFN
-// every scale lives in global memory as such atoms, in the order in which the grouped
-// GEMM consumes them, so that one bulk copy per operand and stage fetches it.
-__device__ __forceinline__ int atom_byte(int r, int kb) {
-  return (r & 31) * 16 + ((r >> 5) & 3) * 4 + kb;
 }
 
 // Row -> (128-row tile, row in tile) of the row-grouped GEMMs: tile = number of 128-row

@@ -155,17 +155,21 @@ def run_and_check_bytes(cfg, fused, expert=None):
 @pytest.mark.parametrize("name,fused", [("mx_e16_odd", True), ("mx_e16_odd", False),
                                         ("mx_skew", True), ("mx_skew_split", True),
                                         ("mx_pairs", False), ("mx_one_token", True)])
-def test_mxfp8_activation_bytes_are_exact(name, fused):
+def test_mxfp8_activation_bytes_are_exact(name, fused, monkeypatch):
+    # [da | du] leaves the SwiGLU-backward epilogue as its MXFP8 copies; "keep" also writes
+    # its bf16 rows, against which those copies are checked
+    monkeypatch.setenv("MOE_B200_DADU", "keep")
     cfg = CASES[name]
     L, offsets = run_and_check_bytes(cfg, fused)
     if name == "mx_skew":
         assert (np.diff(offsets) == 0).any(), "the skewed case must leave experts empty"
 
 
-def test_fullsize_mxfp8_activation_bytes_of_a_sampled_expert():
+def test_fullsize_mxfp8_activation_bytes_of_a_sampled_expert(monkeypatch):
     """mxfp8_e128 at full size (T = 32768, d = 4096, E = 128, f = 1536), fused dispatch as
     the benchmark runs it: the four activations' codes and scales on one sampled expert's
     rows (a row's codes and an expert's token blocks depend on nothing else)."""
+    monkeypatch.setenv("MOE_B200_DADU", "keep")
     cfg = BASE
     rng = np.random.default_rng(5)
     expert = int(rng.integers(0, cfg.E))

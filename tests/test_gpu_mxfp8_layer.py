@@ -150,6 +150,22 @@ def test_mxfp8_recompute_with_shared_buffers_is_bit_exact(name):
 
 
 @pytest.mark.parametrize("name", ["mx_e8", "mx_e16_odd", "mx_skew", "mx_one_token",
+                                  "mx_skew_split_pairs", "mx_pairs"])
+def test_fused_dadu_epilogue_is_bit_identical_to_bf16_then_quantise(name, monkeypatch):
+    # [da | du] quantised in the SwiGLU-backward epilogue against bf16 [da | du] followed by
+    # the activation quantiser: every result of the step bit for bit
+    cfg = CASES[name]
+    _, A = run_layer(cfg)
+    monkeypatch.setenv("MOE_B200_DADU", "0")
+    _, B = run_layer(cfg)
+    for key in ("act", "y_perm", "out", "dgate", "dx_perm", "dw1", "dw2", "dx", "dw_router"):
+        a, b = getattr(A, key), getattr(B, key)
+        if key in ("act", "y_perm", "dx_perm"):
+            a, b = a[:cfg.R], b[:cfg.R]
+        assert torch.equal(a, b), key
+
+
+@pytest.mark.parametrize("name", ["mx_e8", "mx_e16_odd", "mx_skew", "mx_one_token",
                                   "mx_skew_split_pairs"])
 def test_fused_dispatch_is_bit_identical_to_permute_then_quantise(name):
     # the fused dispatch (x's copies from x through perm_src) and the fused combine
