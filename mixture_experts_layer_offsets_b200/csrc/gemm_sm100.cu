@@ -115,10 +115,11 @@ struct GemmParams {
   int drop_it;
   // EPI_ROUTER_DX
   const int32_t* slot_row; // [rows_total][topk]
-  // EPI_SWIGLU_BWD (MXFP8): [da | du] leaves as its two MXFP8 operand copies instead of
-  // bf16 (mx_q_r non-null): the row copy [rows][2f] with row-tile atoms, and the
-  // token-block copy [2f][mx_rp] (column-major, stage-padded) with stage atoms; `out`,
-  // when also set, receives the bf16 rows as well (a diagnostic form)
+  // MXFP8 operand copies written by the epilogue (mx_q_r non-null): the row copy
+  // [rows][K] with row-tile atoms, and the token-block copy [K][mx_rp] (column-major,
+  // stage-padded) with stage atoms.  EPI_SWIGLU_BWD: [da | du] (K = 2f) instead of bf16
+  // (`out`, when also set, receives the bf16 rows as well: a diagnostic form);
+  // EPI_SWIGLU_FWD: h (K = f), besides a | u | h in bf16
   uint8_t* mx_q_r;
   uint8_t* mx_s_r;
   uint8_t* mx_q_c;
@@ -1160,6 +1161,29 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
         }
         const int col = ti.n0 + c0 * 32;
         __nv_bfloat16* arow = p.out + (int64_t)(ti.m0 + row) * p.ld_out;
+        if constexpr (FP8) {
+          if (p.mx_q_r && ti.rows > 0) {
+            // h (the down GEMM's operand) also leaves as its two MXFP8 copies: this warp's 32
+            // rows are one 32-token block and its tile a stage, as for [da | du].  Its
+            // shared-memory scratch is the warp's store staging: the stores that read it
+            // finish first.
+            if (lane == 0) tma_store_wait_read();
+            __syncwarp();
+            const int stage = (PAIR ? s_sel[ti.g] : s_pre[ti.g] / nN) + (ti.m0 - s_off[ti.g]) / BM;
+            const int kq = p.f / 128;
+            const int64_t grow = ti.m0 + row;
+#pragma unroll
+            for (int ci = 0; ci < 2; ++ci) {
+              const int gc = col + 32 * ci;  // column of h
+              mx_emit_block(ph + 16 * ci, valid, q * 32 < ti.rows, p.mx_q_r + grow * p.f + gc,
+                            p.mx_s_r + ((int64_t)stage * kq + gc / 128) * 512 +
+                                atom_byte(row, (gc & 127) >> 5),
+                            p.mx_q_c + (int64_t)gc * p.mx_rp + 128 * (int64_t)stage + 32 * q,
+                            p.mx_rp, p.mx_s_c + ((int64_t)stage * kq + gc / 128) * 512, gc & 96,
+                            q, reinterpret_cast<uint32_t*>(wbuf));
+            }
+          }
+        }
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const int vr = box_valid(q * 32 + 16 * hh);
@@ -2152,6 +2176,17 @@ cudaError_t ffn_fwd_mx(const FfnShape& s, const void* x_perm, const int32_t* off
   p1.sfb = w.w1_s;
   p1.N = f; p1.K = d; p1.b_rows = 2 * f;
   p1.out = static_cast<__nv_bfloat16*>(act); p1.ld_out = 3 * f;
+  // h's two MXFP8 copies come from the gate/up epilogue (MOE_B200_HMX=0: from a pass of
+  // the activation quantiser over the bf16 h instead; read per call, tests compare them)
+  const char* hmx_env = getenv("MOE_B200_HMX");
+  const bool h_mx = !(hmx_env && hmx_env[0] == '0');
+  if (h_mx) {
+    p1.mx_q_r = ws + L.qh0;
+    p1.mx_s_r = ws + L.sh0;
+    p1.mx_q_c = ws + L.qh1;
+    p1.mx_s_c = ws + L.sh1;
+    p1.mx_rp = ((int64_t)R / 128 + E) * 128;
+  }
   // 128 gate + 128 up columns per tile; CTA pairs where experts are large enough
   const bool pairs = use_pairs(s);
   const uint64_t tiles = (uint64_t)R / 128 + E;  // row-tile atoms per 128 columns of K
@@ -2165,7 +2200,8 @@ cudaError_t ffn_fwd_mx(const FfnShape& s, const void* x_perm, const int32_t* off
   }
   if (err != cudaSuccess) return err;
   // h along f (down GEMM) and in token blocks (kept for the dW2 GEMM of the backward)
-  if ((err = mxfp8_act(R, E, f, 3 * f, actb + 2 * f, map, cnt, smap, rt, ws + L.qh0, ws + L.sh0,
+  if (!h_mx &&
+      (err = mxfp8_act(R, E, f, 3 * f, actb + 2 * f, map, cnt, smap, rt, ws + L.qh0, ws + L.sh0,
                        ws + L.qh1, ws + L.sh1, st)) != cudaSuccess)
     return err;
   if (!y_perm) return cudaSuccess;  // recompute: a | u | h and the token-block copies only

@@ -149,14 +149,17 @@ def test_mxfp8_recompute_with_shared_buffers_is_bit_exact(name):
     check_recompute_bit_exact(CASES[name])
 
 
+@pytest.mark.parametrize("flag", ["MOE_B200_DADU", "MOE_B200_HMX"])
 @pytest.mark.parametrize("name", ["mx_e8", "mx_e16_odd", "mx_skew", "mx_one_token",
                                   "mx_skew_split_pairs", "mx_pairs"])
-def test_fused_dadu_epilogue_is_bit_identical_to_bf16_then_quantise(name, monkeypatch):
-    # [da | du] quantised in the SwiGLU-backward epilogue against bf16 [da | du] followed by
-    # the activation quantiser: every result of the step bit for bit
+def test_fused_epilogue_quantisation_is_bit_identical_to_a_separate_pass(name, flag,
+                                                                          monkeypatch):
+    # [da | du] quantised in the SwiGLU-backward epilogue (MOE_B200_DADU), h in the gate/up
+    # epilogue (MOE_B200_HMX), against the bf16 values followed by the activation
+    # quantiser: every result of the step bit for bit
     cfg = CASES[name]
     _, A = run_layer(cfg)
-    monkeypatch.setenv("MOE_B200_DADU", "0")
+    monkeypatch.setenv(flag, "0")
     _, B = run_layer(cfg)
     for key in ("act", "y_perm", "out", "dgate", "dx_perm", "dw1", "dw2", "dx", "dw_router"):
         a, b = getattr(A, key), getattr(B, key)
