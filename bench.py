@@ -203,8 +203,17 @@ def kernel_bytes(cfg, capacity=None, recompute=False) -> dict:
     if cfg.dtype == "mxfp8":
         mx = 2 * (1 + 1 / 32)  # two E4M3 copies with their E8M0 scales, per element
         out["mx_weights"] = 4 * E * 3 * f * d + mx * E * 3 * f * d
-        # x (gathered rows), h, dy, [da | du]: bf16 in, both MXFP8 copies out
-        out["mx_act"] = R * (d + f + d + 2 * f) * (2 + mx)
+        # x (gathered rows) and dy (gate x dout rows, without recompute): bf16 in, both
+        # MXFP8 copies out; h and [da | du] leave the GEMM epilogues already quantised
+        # unless MOE_B200_HMX / MOE_B200_DADU = 0 route them through this kernel too
+        # (the recompute quantises x, and h if it goes through here, a second time)
+        passes = 2 if recompute else 1
+        widths = [d] * passes + [d]
+        if os.environ.get("MOE_B200_HMX", "") == "0":
+            widths += [f] * passes
+        if os.environ.get("MOE_B200_DADU", "") == "0":
+            widths.append(2 * f)
+        out["mx_act"] = R * sum(widths) * (2 + mx)
     return out
 
 
