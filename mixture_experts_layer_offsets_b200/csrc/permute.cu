@@ -162,6 +162,60 @@ combine_bwd_kernel(const T* __restrict__ dout, const T* __restrict__ y_perm,
   }
 }
 
+// dgate alone (the combine backward of a layer that needs no dy_perm rows): every load of
+// a chunk round, the output gradient's and all k expert rows', is issued before the first
+// product, so the k rows' latencies overlap.  Each lane visits its chunks lane, lane + 32,
+// ... in the same order as combine_bwd_kernel, whatever KB is, so the dot products, and
+// dgate, are bit-identical to it.
+template <typename T, int KMAX, int KB>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+dgate_kernel(const T* __restrict__ dout, const T* __restrict__ y_perm,
+             const int32_t* __restrict__ slot_row, float* __restrict__ dgate, int ntok, int d,
+             int k) {
+  constexpr int V = Vec16<T>::N;
+  const int lane = threadIdx.x & 31;
+  const int chunks = d / V;
+  for (int t = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); t < ntok;
+       t += gridDim.x * kWarpsPerBlock) {
+    const int myrow = lane < k ? slot_row[(int64_t)t * k + lane] : -1;
+    int rows[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) rows[j] = __shfl_sync(0xffffffffu, myrow, j);
+    float dot[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) dot[j] = 0.f;
+    for (int c0 = 0; c0 < chunks; c0 += 32 * KB) {
+      Vec16<T> g[KB], y[KMAX][KB];
+#pragma unroll
+      for (int b = 0; b < KB; ++b) {
+        const int c = c0 + b * 32 + lane;
+        g[b].raw = c < chunks ? ldg16(dout + (int64_t)t * d + c * V) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j)
+          y[j][b].raw = (j < k && rows[j] >= 0 && c < chunks)
+                            ? ldg16(y_perm + (int64_t)rows[j] * d + c * V)
+                            : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        if (j >= k || rows[j] < 0) continue;
+#pragma unroll
+        for (int b = 0; b < KB; ++b) {
+          if (c0 + b * 32 + lane >= chunks) continue;
+#pragma unroll
+          for (int i = 0; i < V; ++i) dot[j] = fmaf(g[b].get(i), y[j][b].get(i), dot[j]);
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      if (j >= k) break;
+      const float s = warp_sum(dot[j]);
+      if (lane == 0) dgate[(int64_t)t * k + j] = rows[j] >= 0 ? s : 0.f;
+    }
+  }
+}
+
 // Zero the unused rows of x_pad (rank >= count) and write offsets_pad[e] = e * C.
 template <typename T>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
@@ -291,6 +345,16 @@ static void combine_bwd_t(const void* dout, const void* y_perm, const int32_t* s
                           const float* gate, void* dy_perm, float* dgate, int ntok, int d, int k,
                           cudaStream_t st) {
   const int grid = row_grid(ntok);
+  if (!dy_perm && k <= 8) {  // dgate only
+    ProfScope prof("combine_bwd", st);
+    if (k <= 4)
+      dgate_kernel<T, 4, 4><<<grid, kWarpsPerBlock * 32, 0, st>>>(
+          static_cast<const T*>(dout), static_cast<const T*>(y_perm), slot_row, dgate, ntok, d, k);
+    else
+      dgate_kernel<T, 8, 2><<<grid, kWarpsPerBlock * 32, 0, st>>>(
+          static_cast<const T*>(dout), static_cast<const T*>(y_perm), slot_row, dgate, ntok, d, k);
+    return;
+  }
   if (k <= 8) {
     ProfScope prof("combine_bwd", st);
     combine_bwd_kernel<T, 8><<<grid, kWarpsPerBlock * 32, 0, st>>>(
