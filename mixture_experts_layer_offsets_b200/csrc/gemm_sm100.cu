@@ -459,56 +459,60 @@ __device__ __forceinline__ void mx_emit_block(const uint32_t* pk, bool row_valid
                                               int64_t rp, uint8_t* at_c, int c0, int tb,
                                               uint32_t* s_tr) {
   const int lane = threadIdx.x & 31;
-  float v[32];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    v[2 * i] = row_valid ? bf_lo(pk[i]) : 0.f;
-    v[2 * i + 1] = row_valid ? bf_hi(pk[i]) : 0.f;
-  }
   if (row_valid) {
-    float amax = 0.f;
+    // the row: maximum on packed bf16 pairs (exact), then 32 codes and the scale
+    __nv_bfloat162 am = __float2bfloat162_rn(0.f);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
-    const int ex = block_exponent(amax);
+    for (int i = 0; i < 16; ++i) am = __hmax2(am, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&pk[i])));
+    const int ex = block_exponent(fmaxf(__low2float(am), __high2float(am)));
     const float mul = pow2_neg(ex);
     uint32_t w8[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
-      w8[i] = e4m3_pair(v[4 * i + 1] * mul, v[4 * i] * mul) |
-              (e4m3_pair(v[4 * i + 3] * mul, v[4 * i + 2] * mul) << 16);
+      w8[i] = e4m3_pair(bf_hi(pk[2 * i]) * mul, bf_lo(pk[2 * i]) * mul) |
+              (e4m3_pair(bf_hi(pk[2 * i + 1]) * mul, bf_lo(pk[2 * i + 1]) * mul) << 16);
     *reinterpret_cast<uint4*>(q_r_row) = make_uint4(w8[0], w8[1], w8[2], w8[3]);
     *reinterpret_cast<uint4*>(q_r_row + 16) = make_uint4(w8[4], w8[5], w8[6], w8[7]);
     *at_r = (uint8_t)(ex + 127);
   }
-  // columns: the block passes through shared memory (row `lane` at a pitch of 17 words,
-  // so neither the writes nor the column reads conflict), and lane c takes column c: its
-  // 32 values down the rows give its scale and its 32 codes, which are the column's run
-  // of the token-block copy as they stand
+  // columns: the block passes through shared memory (row `lane` at a pitch of 17 words), and
+  // lane (cp, rh) takes the column pair 2 cp, 2 cp + 1 over rows 16 rh .. 16 rh + 15 (the
+  // reads of one step hit 32 distinct banks); the pair's two lanes combine their maxima
   __syncwarp();
 #pragma unroll
   for (int w = 0; w < 16; ++w) s_tr[lane * 17 + w] = row_valid ? pk[w] : 0u;
   __syncwarp();
-  float cv[32];
+  const int cp = lane >> 1, rh = lane & 1;
+  uint32_t cw[16];
+  __nv_bfloat162 cm = __float2bfloat162_rn(0.f);
 #pragma unroll
-  for (int r = 0; r < 32; ++r) {
-    const uint32_t x = s_tr[r * 17 + (lane >> 1)];
-    cv[r] = (lane & 1) ? bf_hi(x) : bf_lo(x);
+  for (int i = 0; i < 16; ++i) {
+    cw[i] = s_tr[(16 * rh + i) * 17 + cp];
+    cm = __hmax2(cm, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&cw[i])));
   }
-  float cmax = 0.f;
+  const uint32_t cmu = *reinterpret_cast<uint32_t*>(&cm);
+  const uint32_t oth = __shfl_xor_sync(0xffffffffu, cmu, 1);
+  cm = __hmax2(cm, *reinterpret_cast<const __nv_bfloat162*>(&oth));
+  const int ex0 = block_exponent(__low2float(cm)), ex1 = block_exponent(__high2float(cm));
+  const float m0 = pow2_neg(ex0), m1 = pow2_neg(ex1);
+  // codes of rows 16 rh + 4 j .. + 3: column 2 cp's bytes in o0, column 2 cp + 1's in o1
+  uint32_t o0[4], o1[4];
 #pragma unroll
-  for (int r = 0; r < 32; ++r) cmax = fmaxf(cmax, fabsf(cv[r]));
-  const int cex = block_exponent(cmax);
-  const float cmul = pow2_neg(cex);
-  uint32_t o[8];
+  for (int j = 0; j < 4; ++j) {
+    uint32_t pr[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
-    o[i] = live ? (e4m3_pair(cv[4 * i + 1] * cmul, cv[4 * i] * cmul) |
-                   (e4m3_pair(cv[4 * i + 3] * cmul, cv[4 * i + 2] * cmul) << 16))
-                : 0u;
-  uint8_t* dst = q_c_blk + (int64_t)lane * rp;
-  *reinterpret_cast<uint4*>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
-  *reinterpret_cast<uint4*>(dst + 16) = make_uint4(o[4], o[5], o[6], o[7]);
-  at_c[atom_byte(c0 + lane, tb)] = live ? (uint8_t)(cex + 127) : (uint8_t)0x7F;
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t w = cw[4 * j + i];
+      pr[i] = e4m3_pair(bf_hi(w) * m1, bf_lo(w) * m0);
+    }
+    const uint32_t x = pr[0] | (pr[1] << 16), y = pr[2] | (pr[3] << 16);
+    o0[j] = live ? __byte_perm(x, y, 0x6420) : 0u;
+    o1[j] = live ? __byte_perm(x, y, 0x7531) : 0u;
+  }
+  uint8_t* dst = q_c_blk + (int64_t)(2 * cp) * rp + 16 * rh;
+  *reinterpret_cast<uint4*>(dst) = make_uint4(o0[0], o0[1], o0[2], o0[3]);
+  *reinterpret_cast<uint4*>(dst + rp) = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+  at_c[atom_byte(c0 + 2 * cp + rh, tb)] = live ? (uint8_t)((rh ? ex1 : ex0) + 127) : (uint8_t)0x7F;
   __syncwarp();  // s_tr is read before the next block writes it
 }
 
