@@ -277,13 +277,17 @@ moe_status moe_permute_mx(moe_shape shape, const void* x, const int32_t* slot_ro
  *   6 int32 [2]: number of token blocks, number of stages
  *   7 x row codes [rows, d]   8 x row-tile scale atoms
  *   9 h row codes [rows, f]  10 h row-tile scale atoms
- *  11 [da | du] bf16 [rows, 2f]
+ *  11 [da | du] bf16 [rows, 2f] (the SwiGLU-backward epilogue writes [da | du] straight
+ *     into 14-15 and 18-19; this region holds bf16 [da | du] only in the library's
+ *     diagnostic forms, and each routed row's gate (fp32 [rows]) during
+ *     moe_combine_bwd_mx)
  *  12 dy row codes [rows, d]  13 dy row-tile atoms  14 [da|du] row codes [rows, 2f]
  *  15 [da|du] row-tile atoms  16 dy token-block codes [d][Rp]  17 dy token-block atoms
  *  18 [da|du] token-block codes [2f][Rp]  19 [da|du] token-block atoms
  * Regions 0-6 hold from the forward (moe_permute_mx writes 0, 1 and 4-8) to the
  * backward; 7-10 from the forward until the backward starts (they share memory
- * with 11-19); 11-19 after the backward.  Atom byte of (row r, block kb) within a
+ * with 11-19); 11-19 after the backward (moe_combine_bwd_mx writes 12, 13, 16 and 17,
+ * which the backward then reads).  Atom byte of (row r, block kb) within a
  * 128 x 4-block atom: (r % 32) * 16 + (r / 32) * 4 + kb; row-tile atom index
  * tile * (K/128) + K/128-column block; token-block atom index stage * (K/128) +
  * column block, with the blocks of a stage as kb (blocks past an expert's last one
