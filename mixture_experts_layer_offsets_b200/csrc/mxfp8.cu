@@ -371,27 +371,21 @@ mx_act_kernel(const __nv_bfloat16* __restrict__ src, int64_t K, int64_t ld,
   const int64_t kq = K >> 7;
   const int nstages = count[1];
   // n rows x 128 columns of block b: 16 pieces of 16 bytes per row, 4 per thread.  The next
-  // block's pieces are loaded into registers while this block is quantised.
-  auto load = [&](int b, int4& m, uint4 (&v)[4]) {
+  // block's pieces are loaded into registers while this block is quantised (nothing
+  // consumes them before they are staged, so the loads stay in flight meanwhile).
+  auto load = [&](int b, int4& m, uint4 (&v)[4], float (&g)[4]) {
     m = map[b];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int i = tid + 128 * j, row = i >> 4, p8 = i & 15;
       v[j] = make_uint4(0, 0, 0, 0);
+      g[j] = 1.f;
       if (row < m.y) {
         // row r of the operand is source row gather[r] (the fused dispatch), else r; with
-        // row_mul, the bf16 of row_mul[r] times the source values (the fused combine
-        // backward: gate times output gradient, rounded as the combine backward rounds)
+        // row_mul, its factor row_mul[r], applied when the row is staged
         const int64_t sr = gather ? (int64_t)__ldg(gather + m.x + row) : (int64_t)(m.x + row);
         v[j] = ldg16(src + sr * ld + c0 + p8 * 8);
-        if (row_mul) {
-          const float g = __ldg(row_mul + m.x + row);
-          Vec16<__nv_bfloat16> a, o;
-          a.raw = v[j];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) o.set(e, g * a.get(e));
-          v[j] = o.raw;
-        }
+        if (row_mul) g[j] = __ldg(row_mul + m.x + row);
       }
     }
   };
@@ -400,7 +394,8 @@ mx_act_kernel(const __nv_bfloat16* __restrict__ src, int64_t K, int64_t ld,
   int b = z < nstages ? smap[z] : 0;
   int4 mnext;
   uint4 vnext[4];
-  if (z < nstages) load(b, mnext, vnext);
+  float gnext[4];
+  if (z < nstages) load(b, mnext, vnext, gnext);
   while (z < nstages) {
     const int4 m = mnext;
     const int r0 = m.x, n = m.y;
@@ -409,7 +404,17 @@ mx_act_kernel(const __nv_bfloat16* __restrict__ src, int64_t K, int64_t ld,
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int i = tid + 128 * j, row = i >> 4, p8 = i & 15;
-      *reinterpret_cast<uint4*>(s_t + row * kActPitch + p8 * 8) = vnext[j];
+      uint4 v = vnext[j];
+      if (row_mul) {
+        // the fused combine backward's rows: the bf16 of gate times output gradient,
+        // rounded as the combine backward rounds dy_perm
+        Vec16<__nv_bfloat16> a, o;
+        a.raw = v;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o.set(e, gnext[j] * a.get(e));
+        v = o.raw;
+      }
+      *reinterpret_cast<uint4*>(s_t + row * kActPitch + p8 * 8) = v;
     }
     __syncthreads();
     int zn = z, bn = b + 1;
@@ -417,7 +422,7 @@ mx_act_kernel(const __nv_bfloat16* __restrict__ src, int64_t K, int64_t ld,
       zn = z + gridDim.y;
       bn = zn < nstages ? smap[zn] : 0;
     }
-    if (zn < nstages) load(bn, mnext, vnext);
+    if (zn < nstages) load(bn, mnext, vnext, gnext);
     // rows: thread = (row, 32-column block)
     {
       const int row = tid >> 2, kb = tid & 3;

@@ -168,6 +168,20 @@ def test_fused_epilogue_quantisation_is_bit_identical_to_a_separate_pass(name, f
         assert torch.equal(a, b), key
 
 
+@pytest.mark.parametrize("name", ["mx_e8", "mx_skew"])
+def test_fused_paths_with_renormalised_gates_are_bit_identical(name):
+    # the fused combine backward takes the renormalised gates the combine used and writes
+    # their gradient, which the renormalisation backward then maps back
+    cfg = CASES[name]
+    _, A = run_layer(cfg, renorm=True, fused_dispatch=True)
+    _, B = run_layer(cfg, renorm=True, fused_dispatch=False)
+    for key in ("out", "dgate", "dx_perm", "dw1", "dw2", "dx", "dw_router"):
+        a, b = getattr(A, key), getattr(B, key)
+        if key == "dx_perm":
+            a, b = a[:cfg.R], b[:cfg.R]
+        assert torch.equal(a, b), key
+
+
 @pytest.mark.parametrize("name", ["mx_e8", "mx_e16_odd", "mx_skew", "mx_one_token",
                                   "mx_skew_split_pairs"])
 def test_fused_dispatch_is_bit_identical_to_permute_then_quantise(name):
