@@ -114,16 +114,17 @@ def _workload_desc(cfg, capacity, recompute=False, accum=1, world=1):
     if cfg.dtype == "mxfp8":
         d["operands"] = ("MXFP8 (E4M3 + E8M0 per 32 along K) for all six expert GEMMs; bf16 "
                          "activations; FP32 master weights quantised to four MXFP8 copies "
-                         "every step (inside the timed step)")
+                         "once per optimizer step, by its first micro-batch (inside the timed "
+                         "step)")
     if recompute:
         d["recompute"] = "gate/up GEMM re-run in the backward (a | u | h not kept from the forward)"
     d["layout"] = (f"padded capacity C={capacity} (overflow dropped)" if capacity else
                    "dropless, device-scheduled grouped GEMM")
     d["parallelism"] = f"dp{world}"
-    if world > 1:
+    if world > 1 or accum > 1:
         d["step"] = (f"one optimizer step: {accum} micro-batches of T tokens per rank, weight "
-                     "gradients accumulated in place, then one NCCL all-reduce of dW1, dW2, "
-                     "dW_router")
+                     "gradients accumulated in place" +
+                     (", then one NCCL all-reduce of dW1, dW2, dW_router" if world > 1 else ""))
     return d
 
 
@@ -244,7 +245,9 @@ class LayerStep:
         s, dt, fdt = L.shape, L.cdtype, L.ffn_dtype
         acc = capi.MOE_DW_ACCUMULATE if accumulate else 0
         mark(0)
-        if cfg.dtype == "mxfp8":
+        # the MXFP8 weight copies are made once per optimizer step, by its first
+        # micro-batch (the later ones, which accumulate, run on the same weights)
+        if cfg.dtype == "mxfp8" and not accumulate:
             L.quantize_weights(w1, w2)
         mark(1)
         capi.moe_route(s, dt, x, wr, b, L.logits, L.topk_idx, L.topk_gate, L.counts, L.offsets,
@@ -532,6 +535,8 @@ def run_e2e(args, ls, dev, capacity, world, accum):
     L2 = MoELayer(L.T, L.d, L.E, L.k, L.f, L.dtype, dev, dw_dtype=L.dw_dtype, capacity=capacity,
                   recompute=L.recompute)
     L2.dw1, L2.dw2, L2.dw_router = L.dw1, L.dw2, L.dw_router
+    if L.mx is not None:
+        L2.share_weight_copies(L)
     layers = [L, L2]
     inp = ls.inp
     hx = inp["x"].cpu().pin_memory()
@@ -556,7 +561,8 @@ def run_e2e(args, ls, dev, capacity, world, accum):
             ev_in[k].record(h2d)
         cs.wait_event(ev_in[k])
         cs.wait_event(ev_out[k])              # micro-batch i-2's outputs have left layer k
-        layers[k].step(xin[k], wr, b, w1, w2, din[k], accumulate=(i % accum) != 0)
+        first = i % accum == 0  # first micro-batch of an optimizer step
+        layers[k].step(xin[k], wr, b, w1, w2, din[k], accumulate=not first, requantize=first)
         if world > 1 and (i % accum) == accum - 1:
             mdist.allreduce_grads([L.dw1, L.dw2, L.dw_router])
         ev_comp[k].record(cs)

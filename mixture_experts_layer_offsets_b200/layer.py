@@ -144,9 +144,21 @@ class MoELayer:
         blocks along each GEMM's contraction axis (d and 2f for W1, f and d for W2)."""
         capi.moe_mx_quantize_weights(self.shape, w1, w2, self.mx, stream)
 
-    def forward(self, x, w_router, bias, w1, w2, stream=None):
+    def share_weight_copies(self, other: "MoELayer") -> None:
+        """Use ``other``'s MXFP8 weight copies (layers of one shape that run the same
+        weights, e.g. instances that take turns over micro-batches): a quantisation by
+        either serves both.  Both must run on one stream, or be ordered by the caller."""
+        dims = lambda L: (L.T, L.d, L.E, L.k, L.f)
+        if self.mx is None or other.mx is None or dims(self) != dims(other):
+            raise ValueError("weight copies are shared between MXFP8 layers of one shape")
+        self.mxq, self.mx = other.mxq, other.mx
+
+    def forward(self, x, w_router, bias, w1, w2, stream=None, requantize: bool = True):
+        """With ``requantize=False`` an MXFP8 layer reuses the weight copies of an earlier
+        forward instead of quantising w1 and w2 again: valid while the master weights have
+        not changed since, as within the micro-batches of one optimizer step."""
         s, dt = self.shape, self.cdtype
-        if self.mx is not None:
+        if self.mx is not None and requantize:
             self.quantize_weights(w1, w2, stream)
         capi.moe_route(s, dt, x, w_router, bias, self.logits, self.topk_idx, self.topk_gate,
                        self.counts, self.offsets, self.slot_row, self.ws, stream)
@@ -189,8 +201,9 @@ class MoELayer:
                            self.dx_perm, self.row_map, self.dx, self.dw_router, self.ws, stream)
         return self.dx
 
-    def step(self, x, w_router, bias, w1, w2, dout, stream=None, accumulate: bool = False):
-        self.forward(x, w_router, bias, w1, w2, stream)
+    def step(self, x, w_router, bias, w1, w2, dout, stream=None, accumulate: bool = False,
+             requantize: bool = True):
+        self.forward(x, w_router, bias, w1, w2, stream, requantize)
         return self.backward(dout, x, w_router, w1, w2, stream, accumulate)
 
     def routing_stats(self, capacity: int | None = None, stream=None):

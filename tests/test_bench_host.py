@@ -29,6 +29,26 @@ def test_defaults_measure_the_largest_workload():
     assert bench.parse_args(["--warmup", "1"]).warmup == 3
 
 
+def test_weight_copies_are_made_once_per_optimizer_step():
+    # the config names when the MXFP8 weight copies are made, and an accumulation window
+    # is described at one rank too; two layer instances of one shape share their copies
+    from mixture_experts_layer_offsets_b200.layer import MoELayer
+    cfg = inputs.CONFIGS["mxfp8_e128"]
+    d = bench._workload_desc(cfg, None, accum=4, world=1)
+    assert "once per optimizer step" in d["operands"] and "4 micro-batches" in d["step"]
+    assert "all-reduce" not in d["step"]
+    assert "all-reduce" in bench._workload_desc(cfg, None, accum=8, world=2)["step"]
+    assert "step" not in bench._workload_desc(cfg, None)
+    a = MoELayer(64, 128, 8, 2, 128, "mxfp8", "cpu")
+    b = MoELayer(64, 128, 8, 2, 128, "mxfp8", "cpu")
+    b.share_weight_copies(a)
+    assert b.mx is a.mx and b.mxq["w1_q"] is a.mxq["w1_q"]
+    with pytest.raises(ValueError):
+        MoELayer(64, 128, 8, 2, 256, "mxfp8", "cpu").share_weight_copies(a)
+    with pytest.raises(ValueError):
+        MoELayer(64, 128, 8, 2, 128, "bf16", "cpu").share_weight_copies(a)
+
+
 def test_launcher_starts_n_ranks_of_this_script_on_one_node():
     cmd = bench.launcher_argv(8, ["--gpus", "8", "--steps", "4"], 29555)
     assert cmd[1:3] == ["-m", "torch.distributed.run"]

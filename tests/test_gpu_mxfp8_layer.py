@@ -205,6 +205,37 @@ def test_mxfp8_accumulated_weight_grads_are_the_sum_of_two_steps(name):
     check_accumulate(CASES[name])
 
 
+@pytest.mark.parametrize("name", ["mx_e8", "mx_pairs"])
+def test_reused_weight_copies_give_the_bits_of_a_fresh_quantisation(name):
+    # the micro-batches of one optimizer step after the first run on the weight copies the
+    # first one made (requantize=False), also when two layer instances share them: the
+    # second micro-batch (other tokens, same weights) must match a layer that quantised
+    from mixture_experts_layer_offsets_b200.inputs import make_inputs
+    from mixture_experts_layer_offsets_b200.layer import MoELayer
+    cfg = CASES[name]
+    dev = lambda d: {k: (v.cuda() if v is not None else None) for k, v in d.items()}
+    a_in = dev(make_inputs(cfg, device="cpu", seed=0))
+    b_in = dev(make_inputs(cfg, device="cpu", seed=1))
+    for k in ("w_router", "bias", "w1", "w2"):  # batch B: new tokens, A's weights
+        b_in[k] = a_in[k]
+    args = lambda i: (i["x"], i["w_router"], i["bias"], i["w1"], i["w2"], i["dout"])
+    new = lambda: MoELayer(cfg.T, cfg.d_model, cfg.E, cfg.top_k, cfg.d_ff, cfg.dtype, "cuda")
+    ref = new()
+    ref.step(*args(b_in))
+    first, second = new(), new()
+    second.share_weight_copies(first)
+    first.step(*args(a_in))
+    first.step(*args(b_in), accumulate=False, requantize=False)
+    second.step(*args(b_in), requantize=False)
+    torch.cuda.synchronize()
+    for L in (first, second):
+        assert L.device_status() == 0
+        for key in ("out", "dgate", "dx_perm", "dw1", "dw2", "dx", "dw_router"):
+            assert torch.equal(getattr(L, key), getattr(ref, key)), key
+    with pytest.raises(ValueError):
+        MoELayer(cfg.T, cfg.d_model, cfg.E, cfg.top_k, cfg.d_ff, "bf16", "cuda").share_weight_copies(first)
+
+
 
 @pytest.mark.parametrize("name", ["mx_pairs", "mx_skew_split", "mx_skew_split_pairs"])
 def test_mxfp8_cta_pairs_give_the_bits_of_single_ctas(name, monkeypatch):
