@@ -73,7 +73,8 @@ SWEEP = [("bf16_e8", False, None), ("bf16_e128", False, None), ("bf16_skew_e128"
 # GEMM source it was taken on: reported only while that source is unchanged.
 GEMM_TRAFFIC = {}
 GEMM_SOURCES = ("mixture_experts_layer_offsets_b200/csrc/gemm_sm100.cu",
-                "mixture_experts_layer_offsets_b200/csrc/common.cuh")
+                "mixture_experts_layer_offsets_b200/csrc/common.cuh",
+                "mixture_experts_layer_offsets_b200/csrc/mx_common.cuh")
 
 
 def gemm_source_sha() -> str:
