@@ -71,7 +71,16 @@ SWEEP = [("bf16_e8", False, None), ("bf16_e128", False, None), ("bf16_skew_e128"
 # DRAM bytes (read + write) of the grouped-GEMM launches of one step, from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum) per workload, with the SHA-256 of the
 # GEMM source it was taken on: reported only while that source is unchanged.
-GEMM_TRAFFIC = {}
+GEMM_TRAFFIC = {
+    # the six grouped-GEMM launches of a step of mxfp8_e128 at E=16, T=4096 (the same 1024
+    # tokens per expert, so every operand and result is 1/8 of the full step's), mean of
+    # two steps (2.7177e9 and 2.7139e9 bytes), times 8
+    "mxfp8_e128": (21726412800,
+                   "4a187244306d58435e65d13790c698ee2139a25fe545e4384a2de886e5041ccb",
+                   "scaled x8 from a capture at E=16, T=4096 (1024 tokens per expert as here); "
+                   "ncu flushes L2 before each launch and counts the writes that reach DRAM "
+                   "while it runs"),
+}
 GEMM_SOURCES = ("mixture_experts_layer_offsets_b200/csrc/gemm_sm100.cu",
                 "mixture_experts_layer_offsets_b200/csrc/common.cuh",
                 "mixture_experts_layer_offsets_b200/csrc/mx_common.cuh")
@@ -183,6 +192,31 @@ class ClockSampler:
 def gemm_flop(cfg) -> float:
     """Algorithmic FLOPs of the six expert GEMMs of one step: 18 R d f (dropless rows)."""
     return 18.0 * cfg.R * cfg.d_model * cfg.d_ff
+
+
+def gemm_bytes(cfg) -> float:
+    """Algorithmic DRAM bytes of the six expert GEMMs of one dropless step without recompute:
+    each operand read once (a weight once per GEMM), each result written once.  MXFP8
+    operands are 1 byte per element plus one scale byte per 32; the MXFP8 epilogues write
+    h and [da | du] as their two MXFP8 copies, the bf16 ones write them in bf16."""
+    R, d, f, E = cfg.R, cfg.d_model, cfg.d_ff, cfg.E
+    if cfg.dtype == "mxfp8":
+        s = 1 + 1 / 32
+        fwd = (R * d * s + E * 2 * f * d * s + R * 3 * f * 2 + 2 * R * f * s +   # gate/up
+               R * f * s + E * d * f * s + R * d * 2)                            # down
+        bwd = (R * d * s + E * d * f * s + R * 2 * f * 2 + 2 * R * 2 * f * s +   # dh, da|du
+               R * 2 * f * s + E * 2 * f * d * s + R * d * 2 +                   # dx_perm
+               R * d * s + R * f * s + E * d * f * 4 +                           # dW2
+               R * 2 * f * s + R * d * s + E * 2 * f * d * 4)                    # dW1
+        return fwd + bwd
+    b = 4 if cfg.dtype == "f32" else 2
+    fwd = (R * d * b + E * 2 * f * d * b + R * 3 * f * b +
+           R * f * b + E * d * f * b + R * d * b)
+    bwd = (R * d * b + E * d * f * b + R * 2 * f * b + R * 2 * f * b +
+           R * 2 * f * b + E * 2 * f * d * b + R * d * b +
+           R * d * b + R * f * b + E * d * f * 4 +
+           R * 2 * f * b + R * d * b + E * 2 * f * d * 4)
+    return fwd + bwd
 
 
 def kernel_bytes(cfg, capacity=None, recompute=False) -> dict:
@@ -407,7 +441,7 @@ def dp_line(cfg, total_ms, steps, warmup, accum, world) -> dict:
             "data": "synthetic (seeded; random-init weights)"}
 
 
-def roofline(cfg, res, capacity=None):
+def roofline(cfg, res, capacity=None, recompute=False):
     pk, pk_kind = _peaks()
     flop = gemm_flop(cfg)
     gemm_ms = res["gemm_ms"]
@@ -421,14 +455,18 @@ def roofline(cfg, res, capacity=None):
         peak, kind = None, "fp32 CUDA-core path: no tensor-core peak"
     tr = GEMM_TRAFFIC.get(cfg.name) if not capacity else None
     traffic = tr[0] if tr and tr[1] == gemm_source_sha() else None
+    alg = None if capacity or recompute else round(gemm_bytes(cfg))
     out = {"bound": "tensor",
            "kernel": f"grouped GEMM (tcgen05): the {res['gemm_launches']} expert-FFN GEMM "
                      "launches of a step (gemm_* in kernels_ms)",
            "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
            "frac": round(achieved / peak, 4) if peak else None, "peak_kind": kind,
            "traffic": traffic,
-           "traffic_unit": "DRAM bytes per step over those launches (ncu dram__bytes_read.sum "
-                           "+ dram__bytes_write.sum); null unless captured on this GEMM source",
+           "traffic_unit": "DRAM bytes per step over the six grouped-GEMM launches (ncu "
+                           "dram__bytes_read.sum + dram__bytes_write.sum); null unless "
+                           "captured on this GEMM source",
+           "traffic_note": tr[2] if traffic else None,
+           "algorithmic_bytes_per_step": alg,
            "algorithmic_flop_per_step": flop, "gemm_ms_per_step": round(gemm_ms, 4),
            "timing": "CUDA events around each GEMM launch (moe_profile_begin), eager steps"}
     return out
@@ -473,7 +511,7 @@ def run_ours(args, rank, world):
     line = dp_line(cfg, res["ms_per_step"] * args.steps, args.steps, args.warmup, accum, world)
     line.update({
         "config": _workload_desc(cfg, capacity, args.recompute, accum, world),
-        "roofline": roofline(cfg, res, capacity),
+        "roofline": roofline(cfg, res, capacity, args.recompute),
         "hbm_kernels": hbm_kernels(cfg, res, capacity, args.recompute),
         "phases_ms": {k: round(v, 4) for k, v in res["phases_ms"].items()},
         "kernels_ms": res["kernels"],

@@ -69,6 +69,17 @@ def test_algorithmic_work():
     # padded layout: the row count is E * C
     assert bench.kernel_bytes(c["bf16_skew_e128"], 1280)["combine"] > \
         bench.kernel_bytes(c["bf16_skew_e128"])["combine"]
+    # the six expert GEMMs at bf16_e8, summed by hand from the operand and result sizes
+    # (R = 65536, d = 2048, f = 1024, E = 8; fp32 weight gradients): 1174405120 forward
+    # + 2583691264 backward
+    assert bench.gemm_bytes(c["bf16_e8"]) == 3758096384
+    # MXFP8 moves fewer operand bytes than the same shapes in bf16, and the captured
+    # traffic of the default workload is reported with its algorithmic bytes
+    big = c["mxfp8_e128"]
+    assert bench.gemm_bytes(big) < bench.gemm_bytes(inputs.shrink(big, name="x", dtype="bf16"))
+    rf = bench.roofline(big, {"gemm_ms": 9.0, "gemm_launches": 8})
+    assert rf["algorithmic_bytes_per_step"] == round(bench.gemm_bytes(big))
+    assert rf["traffic"] is None or 0.8 < rf["traffic"] / rf["algorithmic_bytes_per_step"] < 1.2
 
 
 CFG = inputs.shrink(inputs.CONFIGS["tiny_f32"], name="gloo_bench", T=24, d_model=16, E=4,
