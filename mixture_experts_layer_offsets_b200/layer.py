@@ -10,8 +10,9 @@ rows in the grouped FFN, dropped pairs marked -1).
 
 dtype "mxfp8": bf16 activations and router, FP32 master expert weights whose
 MXFP8 copies (two orientations per weight, see ``moe_mx_weights``) are made
-by moe_mx_quantize_weights at the start of every forward, i.e. once per optimizer step
-when every step is one; the grouped FFN calls run with MOE_MXFP8 and write
+by moe_mx_quantize_weights at the start of a forward; the later micro-batches of an
+optimizer step pass ``requantize=False`` and reuse them, so they are made once per
+optimizer step.  The grouped FFN calls run with MOE_MXFP8 and write
 FP32 weight gradients.  Unless it recomputes, the MXFP8 layer dispatches with
 moe_permute_mx and runs the combine backward as moe_combine_bwd_mx: both write the
 MXFP8 operand copies of x and dy straight into the workspace, and no bf16 x_perm or
