@@ -364,7 +364,9 @@ moe_status moe_combine_bwd_mx(moe_shape shape, const void* dout, const void* y_p
  *   dW2[e] = dy^T h; dW1[e,0:f] = da^T x; dW1[e,f:2f] = du^T x.
  * An expert with no rows gets dW1[e] = dW2[e] = 0 (dW is overwritten; with
  * MOE_DW_ACCUMULATE in dw_dtype it is added to, and such an expert's dW is unchanged).
- * dy_perm, x_perm: [rows, d]; act_saved: [rows, 3f] from the forward;
+ * dy_perm, x_perm: [rows, d]; act_saved: [rows, 3f] from the forward, 32-byte
+ * aligned for MOE_BF16 and MOE_MXFP8 (a and u are read in 32-byte pieces; a
+ * buffer aligned only to 16 bytes gets MOE_ERR_INVALID_ARG);
  * dx_perm: [rows, d]; dw1: [E, 2f, d]; dw2: [E, d, f] of type dw_dtype
  * (MOE_F32 or MOE_BF16; MOE_F32 only when dtype is MOE_F32 or MOE_MXFP8).
  * Uses 2*f*rows elements of scratch in `ws` for [da | du].

@@ -53,6 +53,7 @@ using namespace moe;
 namespace {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+inline bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31) == 0; }
 
 // All pointers non-null and 16-byte aligned.
 template <typename... P>
@@ -302,7 +303,8 @@ moe_status ffn_bwd_entry(moe_shape s, int dtype, int64_t rows, const void* dy_pe
     // x_perm is read only by the recompute (the backward uses the token-block copy);
     // dy_perm NULL: moe_combine_bwd_mx has put dy's copies in ws (not with the recompute,
     // whose forward half reuses that memory)
-    if (rows > 0 && (!ptrs_ok(act_saved, dx_perm) || (recompute && !x_perm) ||
+    if (rows > 0 && (!ptrs_ok(act_saved, dx_perm) || !aligned32(act_saved) ||
+                     (recompute && !x_perm) ||
                      (x_perm && !aligned16(x_perm)) || (recompute && !dy_perm) ||
                      (dy_perm && !aligned16(dy_perm))))
       return MOE_ERR_INVALID_ARG;
@@ -323,6 +325,8 @@ moe_status ffn_bwd_entry(moe_shape s, int dtype, int64_t rows, const void* dy_pe
   if (dtype == MOE_F32 && dw_dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
   if (!ptrs_ok(offsets, w1, w2, dw1, dw2, ws)) return MOE_ERR_INVALID_ARG;
   if (rows > 0 && !ptrs_ok(dy_perm, x_perm, act_saved, dx_perm)) return MOE_ERR_INVALID_ARG;
+  // the bf16 SwiGLU backward reads a and u in 32-byte pieces
+  if (rows > 0 && dtype == MOE_BF16 && !aligned32(act_saved)) return MOE_ERR_INVALID_ARG;
   FfnShape fs{s.d_model, s.E, s.d_ff, rows};
   if (ws_bytes < kStatusBytes + ffn_bwd_ws_bytes(fs, dtype == MOE_BF16)) return MOE_ERR_INVALID_ARG;
   cudaStream_t cs = as_stream(stream);

@@ -106,6 +106,9 @@ def test_ffn_validation(lib):
              None) == capi.MOE_ERR_INVALID_ARG
     assert b(s, capi.MOE_BF16, 128, *args, None, FAKE, FAKE, FAKE, capi.MOE_F32, FAKE, 300, None) \
         == capi.MOE_ERR_INVALID_ARG  # workspace too small
+    # the SwiGLU backward reads a and u in 32-byte pieces: act_saved aligned to 16 only
+    assert b(s, capi.MOE_BF16, 128, FAKE, FAKE, FAKE + 16, FAKE, FAKE, FAKE, None, FAKE, FAKE,
+             FAKE, capi.MOE_F32, FAKE, 1 << 30, None) == capi.MOE_ERR_INVALID_ARG
 
 
 def test_row_ops_validation(lib):
@@ -160,8 +163,8 @@ def test_mxfp8_ffn_validation(lib):
         return f(shape, capi.MOE_MXFP8, 128, FAKE, FAKE, None, None, ctypes.addressof(mxw), FAKE,
                  FAKE, FAKE, ws_bytes, None)
 
-    def bwd(dw_dtype=capi.MOE_F32, mxw=mx, ws_bytes=big):
-        return b(s, capi.MOE_MXFP8, 128, FAKE, FAKE, FAKE, FAKE, None, None, ctypes.addressof(mxw),
+    def bwd(dw_dtype=capi.MOE_F32, mxw=mx, ws_bytes=big, act=FAKE):
+        return b(s, capi.MOE_MXFP8, 128, FAKE, FAKE, act, FAKE, None, None, ctypes.addressof(mxw),
                  FAKE, FAKE, FAKE, dw_dtype, FAKE, ws_bytes, None)
 
     assert fwd(shape=_shape(d_model=192)) == capi.MOE_ERR_UNSUPPORTED     # d % 128
@@ -171,6 +174,7 @@ def test_mxfp8_ffn_validation(lib):
     assert fwd(ws_bytes=big // 2) == capi.MOE_ERR_INVALID_ARG
     assert bwd(dw_dtype=capi.MOE_BF16) == capi.MOE_ERR_INVALID_ARG       # dW is fp32
     assert bwd(ws_bytes=1024) == capi.MOE_ERR_INVALID_ARG
+    assert bwd(act=FAKE + 16) == capi.MOE_ERR_INVALID_ARG               # act_saved 32-byte aligned
 
 
 def test_mxfp8_combine_bwd_validation(lib):
