@@ -462,6 +462,12 @@ __device__ __forceinline__ void put_box_bf16(uint8_t* wbuf, uint32_t& slot, cons
 //   q_c_blk:  token-block copy at the block's first column and first row
 //   at_c:     the stage atom of the block's 128-column slab; c0: the block's first column
 //             within that slab (0, 32, 64, 96); tb: the token block within the stage
+// 32 bytes (one sector) in one store; p is 32-byte aligned
+__device__ __forceinline__ void stg32(void* p, const uint32_t* r) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
 __device__ __forceinline__ void mx_emit_block(const uint32_t* pk, bool row_valid, bool live,
                                               uint8_t* q_r_row, uint8_t* at_r, uint8_t* q_c_blk,
                                               int64_t rp, uint8_t* at_c, int c0, int tb,
@@ -479,8 +485,7 @@ __device__ __forceinline__ void mx_emit_block(const uint32_t* pk, bool row_valid
     for (int i = 0; i < 8; ++i)
       w8[i] = e4m3_pair(bf_hi(pk[2 * i]) * mul, bf_lo(pk[2 * i]) * mul) |
               (e4m3_pair(bf_hi(pk[2 * i + 1]) * mul, bf_lo(pk[2 * i + 1]) * mul) << 16);
-    *reinterpret_cast<uint4*>(q_r_row) = make_uint4(w8[0], w8[1], w8[2], w8[3]);
-    *reinterpret_cast<uint4*>(q_r_row + 16) = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+    stg32(q_r_row, w8);
     *at_r = (uint8_t)(ex + 127);
   }
   // columns: the block passes through shared memory (row `lane` at a pitch of 17 words), and
@@ -517,9 +522,16 @@ __device__ __forceinline__ void mx_emit_block(const uint32_t* pk, bool row_valid
     o0[j] = live ? __byte_perm(x, y, 0x6420) : 0u;
     o1[j] = live ? __byte_perm(x, y, 0x7531) : 0u;
   }
-  uint8_t* dst = q_c_blk + (int64_t)(2 * cp) * rp + 16 * rh;
-  *reinterpret_cast<uint4*>(dst) = make_uint4(o0[0], o0[1], o0[2], o0[3]);
-  *reinterpret_cast<uint4*>(dst + rp) = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+  // the pair swaps halves so that lane rh holds all 32 rows of column 2 cp + rh, written
+  // as one 32-byte store
+  uint32_t c8[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t got = __shfl_xor_sync(0xffffffffu, rh ? o0[j] : o1[j], 1);
+    c8[j] = rh ? got : o0[j];          // rows 4 j .. 4 j + 3
+    c8[4 + j] = rh ? o1[j] : got;      // rows 16 + 4 j .. 16 + 4 j + 3
+  }
+  stg32(q_c_blk + (int64_t)(2 * cp + rh) * rp, c8);
   at_c[atom_byte(c0 + 2 * cp + rh, tb)] = live ? (uint8_t)((rh ? ex1 : ex0) + 127) : (uint8_t)0x7F;
   __syncwarp();  // s_tr is read before the next block writes it
 }
