@@ -35,8 +35,10 @@
  *     ([kongchang] routing section: metadata stays on the GPU; [bytechap] how
  *     it works: the CPU queues work without waiting).  Calls can be captured
  *     in a CUDA graph.
- *   - Device pointers must be 16-byte aligned.  Row counts and offsets are
- *     int32.
+ *   - Device pointers must be 16-byte aligned; the workspace of the MXFP8
+ *     grouped FFN calls and act_saved of the bf16 and MXFP8 backward 32-byte
+ *     aligned (cudaMalloc and PyTorch allocations are 256-byte aligned).  Row
+ *     counts and offsets are int32.
  *   - Errors: a call validates its arguments on the host before it launches
  *     anything and returns MOE_ERR_INVALID_ARG (bad sizes, null or misaligned
  *     pointers, too small workspace) or MOE_ERR_UNSUPPORTED (valid but not

@@ -214,7 +214,8 @@ moe_status moe_grouped_ffn_fwd(moe_shape s, int dtype, int64_t rows, const void*
     moe_status vs = mx_weights_ok(mx, w);
     if (vs != MOE_OK) return vs;
     if (s.d_model % 128 || s.d_ff % 128) return MOE_ERR_UNSUPPORTED;
-    if (!ptrs_ok(offsets, ws)) return MOE_ERR_INVALID_ARG;
+    // the epilogues write h's MXFP8 copies into ws with 32-byte stores
+    if (!ptrs_ok(offsets, ws) || !aligned32(ws)) return MOE_ERR_INVALID_ARG;
     // x_perm NULL: moe_permute_mx has put the quantised copies of x in ws
     if (rows > 0 && (!ptrs_ok(act_saved, y_perm) || (x_perm && !aligned16(x_perm))))
       return MOE_ERR_INVALID_ARG;
@@ -299,7 +300,8 @@ moe_status ffn_bwd_entry(moe_shape s, int dtype, int64_t rows, const void* dy_pe
     if (vs != MOE_OK) return vs;
     if (s.d_model % 128 || s.d_ff % 128) return MOE_ERR_UNSUPPORTED;
     if (dw_dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
-    if (!ptrs_ok(offsets, dw1, dw2, ws)) return MOE_ERR_INVALID_ARG;
+    // the epilogues write [da | du]'s MXFP8 copies into ws with 32-byte stores
+    if (!ptrs_ok(offsets, dw1, dw2, ws) || !aligned32(ws)) return MOE_ERR_INVALID_ARG;
     // x_perm is read only by the recompute (the backward uses the token-block copy);
     // dy_perm NULL: moe_combine_bwd_mx has put dy's copies in ws (not with the recompute,
     // whose forward half reuses that memory)

@@ -175,6 +175,11 @@ def test_mxfp8_ffn_validation(lib):
     assert bwd(dw_dtype=capi.MOE_BF16) == capi.MOE_ERR_INVALID_ARG       # dW is fp32
     assert bwd(ws_bytes=1024) == capi.MOE_ERR_INVALID_ARG
     assert bwd(act=FAKE + 16) == capi.MOE_ERR_INVALID_ARG               # act_saved 32-byte aligned
+    # the MXFP8 epilogues write their operand copies into ws with 32-byte stores
+    assert f(s, capi.MOE_MXFP8, 128, FAKE, FAKE, None, None, ctypes.addressof(mx), FAKE, FAKE,
+             FAKE + 16, big, None) == capi.MOE_ERR_INVALID_ARG
+    assert b(s, capi.MOE_MXFP8, 128, FAKE, FAKE, FAKE, FAKE, None, None, ctypes.addressof(mx),
+             FAKE, FAKE, FAKE, capi.MOE_F32, FAKE + 16, big, None) == capi.MOE_ERR_INVALID_ARG
 
 
 def test_mxfp8_combine_bwd_validation(lib):
