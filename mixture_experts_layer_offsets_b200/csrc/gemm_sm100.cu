@@ -1538,20 +1538,27 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
             for (int ci = 0; ci < kMine; ++ci) tmem_tie(va[ci]);
           }
           release();
+          // a partial sum always overwrites its slot; the result is added into the output
+          // when the call accumulates
+          auto put = [&](int ci, int hh, uint8_t* sbuf) {
+            if (p.accumulate && !partial)
+              tma_reduce_add_2d(tmo, ti.n0 + (c0 + ci) * 32, (int)(orow0 + 16 * hh), sbuf);
+            else
+              tma_store_2d(tmo, ti.n0 + (c0 + ci) * 32, (int)(orow0 + 16 * hh), sbuf);
+          };
+          if constexpr (kTwoSlots) {
+            // all 32 lanes stage both 16-row boxes of a chunk at once (lane l: row l % 16 of
+            // box l / 16, one slot per box), once the previous chunk's stores have read the
+            // slots; with half the lanes per box the MMAs beside this epilogue ran ~6 %
+            // slower per stage
 #pragma unroll
-          for (int ci = 0; ci < kMine; ++ci) {
-            const uint32_t* v = va[ci];
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              uint8_t* sbuf = wbuf + (kTwoSlots ? (slot & 1) * 2048 : 0);
-              // the store that last used this slot has read it
-              if (lane == 0) {
-                if (kTwoSlots) tma_store_wait_read_le1();
-                else tma_store_wait_read();
-              }
+            for (int ci = 0; ci < kMine; ++ci) {
+              const uint32_t* v = va[ci];
+              if (lane == 0) tma_store_wait_read();
               __syncwarp();
-              if ((lane >> 4) == hh) {
+              {
                 const int r = lane & 15;
+                uint8_t* sbuf = wbuf + (lane >> 4) * 2048;
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
                   *reinterpret_cast<uint4*>(sbuf + r * 128 + ((j ^ (r & 7)) * 16)) =
@@ -1560,14 +1567,31 @@ grouped_gemm_sm100(const __grid_constant__ GemmParams p) {
               fence_proxy_async_smem();
               __syncwarp();
               if (lane == 0) {
-                // a partial sum always overwrites its slot; the result is added into the
-                // output when the call accumulates
-                if (p.accumulate && !partial)
-                  tma_reduce_add_2d(tmo, ti.n0 + (c0 + ci) * 32, (int)(orow0 + 16 * hh), sbuf);
-                else
-                  tma_store_2d(tmo, ti.n0 + (c0 + ci) * 32, (int)(orow0 + 16 * hh), sbuf);
+                put(ci, 0, wbuf);
+                put(ci, 1, wbuf + 2048);
               }
-              ++slot;
+            }
+          } else {
+            // one 2 KB slot: each box is staged by its 16 lanes after the previous store
+            // has read the slot
+#pragma unroll
+            for (int ci = 0; ci < kMine; ++ci) {
+              const uint32_t* v = va[ci];
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                if (lane == 0) tma_store_wait_read();
+                __syncwarp();
+                if ((lane >> 4) == hh) {
+                  const int r = lane & 15;
+#pragma unroll
+                  for (int j = 0; j < 8; ++j)
+                    *reinterpret_cast<uint4*>(wbuf + r * 128 + ((j ^ (r & 7)) * 16)) =
+                        make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) put(ci, hh, wbuf);
+              }
             }
           }
         } else if (p.accumulate) {
