@@ -74,9 +74,9 @@ SWEEP = [("bf16_e8", False, None), ("bf16_e128", False, None), ("bf16_skew_e128"
 GEMM_TRAFFIC = {
     # the six grouped-GEMM launches of a step of mxfp8_e128 at E=16, T=4096 (the same 1024
     # tokens per expert, so every operand and result is 1/8 of the full step's), mean of
-    # two steps (2.7185e9 and 2.7166e9 bytes), times 8
-    "mxfp8_e128": (21740364800,
-                   "ff14e41c58c01b1de0485c8c82742386d7c7208023e5a6d60fee06326afcd442",
+    # two steps (2.7199e9 and 2.7174e9 bytes), times 8
+    "mxfp8_e128": (21749104640,
+                   "378c5362fcf5a9c14aff1d513afeccb423d593e6630c61d4407135140546b152",
                    "scaled x8 from a capture at E=16, T=4096 (1024 tokens per expert as here); "
                    "ncu flushes L2 before each launch and counts the writes that reach DRAM "
                    "while it runs"),
