@@ -676,8 +676,8 @@ def cpu_baseline(cfg, budget_s=12.0, chunk=64, single_core=False):
     experts, timed alone, scaled by E / E_s (once per step, as the layer does); (b) one
     oracle call on 256 tokens, minus (a), per token, scaled by T.
 
-    With ``single_core`` the line also carries the rate with one BLAS thread (the survey
-    asks for both figures)."""
+    With ``single_core`` the line also carries the rate with one BLAS thread, so that the
+    all-core and the one-core figure are both reported."""
     if cfg.dtype == "mxfp8":
         cb = _cpu_baseline_mx(cfg)
         if single_core:
