@@ -49,6 +49,27 @@ def test_weight_copies_are_made_once_per_optimizer_step():
         MoELayer(64, 128, 8, 2, 128, "bf16", "cpu").share_weight_copies(a)
 
 
+def test_cpu_baseline_samples_are_bounded_and_labelled():
+    # the oracle's rate on a bounded sample: bf16 whole calls within the budget; MXFP8 per
+    # sample the weight quantisation of whole experts (at least one), with the cost per
+    # token measured once per process and reused
+    small = inputs.shrink(inputs.CONFIGS["bf16_e8"], name="cb_bf16", T=64, d_model=128, E=4,
+                          top_k=2, d_ff=128)
+    cb = bench.cpu_baseline(small, budget_s=0.2)
+    assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["cores"] >= 1
+    mx = inputs.shrink(inputs.CONFIGS["mxfp8_e128"], name="cb_mx", T=64, d_model=128, E=8,
+                       top_k=2, d_ff=128)
+    bench._MX_TOKEN_COST.clear()
+    a = bench.cpu_baseline(mx, budget_s=0.0)
+    assert len(bench._MX_TOKEN_COST) == 1
+    cost = dict(bench._MX_TOKEN_COST)
+    b = bench.cpu_baseline(mx, budget_s=0.0)
+    assert bench._MX_TOKEN_COST == cost          # measured once, reused
+    for r in (a, b):
+        assert r["extrapolated"] and r["value"] > 0 and "of 8 experts" in r["sample"]
+        assert "1 of 8 experts" in r["sample"]    # a zero budget still times one expert
+
+
 def test_launcher_starts_n_ranks_of_this_script_on_one_node():
     cmd = bench.launcher_argv(8, ["--gpus", "8", "--steps", "4"], 29555)
     assert cmd[1:3] == ["-m", "torch.distributed.run"]
