@@ -312,11 +312,12 @@ moe_status moe_mx_workspace_layout(moe_shape shape, int64_t rows, int64_t* offse
  * MOE_MXFP8 (kongchang, boundary-conditions section: MXFP8 cuts GEMM time and
  * saved-activation bytes): x_perm, act_saved and y_perm stay bf16; mx is a HOST
  * pointer to a moe_mx_weights whose members are device pointers (w1, w2 are not
- * read and may be NULL); x and h are quantised, in one pass each, along their rows
- * (for this call's GEMMs) and in 32-row token blocks (kept in `ws` for the backward), and
- * the GEMMs run block-scaled E4M3 x E4M3 with fp32 accumulation.  Needs d % 128 == 0 and
- * f % 128 == 0.  x_perm may be NULL when moe_permute_mx has just filled `ws` for the
- * same offsets (the x quantisation is then skipped). */
+ * read and may be NULL); x (in one pass) and h (in the gate/up GEMM's epilogue) are
+ * quantised along their rows (for this call's GEMMs) and in 32-row token blocks (kept in
+ * `ws` for the backward), and the GEMMs run block-scaled E4M3 x E4M3 with fp32
+ * accumulation.  Needs d % 128 == 0 and f % 128 == 0, and `ws` 32-byte aligned.  x_perm
+ * may be NULL when moe_permute_mx has just filled `ws` for the same offsets (the x
+ * quantisation is then skipped). */
 moe_status moe_grouped_ffn_fwd(moe_shape shape, int dtype, int64_t rows, const void* x_perm,
                                const int32_t* offsets, const void* w1, const void* w2,
                                const void* mx, void* act_saved, void* y_perm, void* ws,
@@ -372,9 +373,10 @@ moe_status moe_combine_bwd_mx(moe_shape shape, const void* dout, const void* y_p
  * dx_perm: [rows, d]; dw1: [E, 2f, d]; dw2: [E, d, f] of type dw_dtype
  * (MOE_F32 or MOE_BF16; MOE_F32 only when dtype is MOE_F32 or MOE_MXFP8).
  * Uses 2*f*rows elements of scratch in `ws` for [da | du].
- * MOE_MXFP8: dy_perm, x_perm, act_saved, dx_perm bf16; mx as for the forward;
- * dy and [da | du] are quantised along their rows for the dgrad GEMMs, and dy, h,
- * [da | du], x in 32-row blocks restarting at every expert for the wgrad GEMMs.  The
+ * MOE_MXFP8: dy_perm, x_perm, act_saved, dx_perm bf16; mx as for the forward; `ws`
+ * 32-byte aligned; dy (in one pass) and [da | du] (in the SwiGLU-backward GEMM's
+ * epilogue) are quantised along their rows for the dgrad GEMMs, and dy, h, [da | du], x
+ * in 32-row blocks restarting at every expert for the wgrad GEMMs.  The
  * token-block copies of x and h (and the row/block maps) are the ones the forward of the
  * same step wrote into `ws`: pass the same workspace, with no call using it in between
  * (moe_combine and moe_combine_bwd take none), and the same offsets.  x_perm is not
